@@ -1,0 +1,205 @@
+"""fp64 CPU oracle for the attention forward pass -- TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  The product path (the CUDA library in
+``tiled_attention_18_b200`` and its binding) never imports, links or calls it.
+It shares no code with the CUDA path; the two meet only in the seeded input
+generators of ``tiled_attention_18_b200.workloads``, which hold none of the
+method's arithmetic.
+
+The arithmetic lives in ``attn_oracle.c`` (plain C, fp64, OpenMP over rows);
+this module builds it with gcc when needed and marshals numpy arrays through
+ctypes.  Function-level citations are in the C file's header:
+- ``attn_fwd``   : the definition softmax(scale * Q K^T [+ causal]) V and the
+  per-row log-sum-exp ("FlashAttention-2 在昇腾 NPU 上如何做到 3 倍加速？" section 1;
+  "ops-transformer FlashAttention 算子实战" section 4.2).
+- ``attn_rows``  : the same definition for sampled rows.
+- ``attn_tiled`` : the tiled online-softmax recurrence of the FlashAttention-2
+  page, sections 2.1-2.2, with causal key-tile skipping (gsyq.cn catlass
+  page, "Causal Mask的实现差异", mode 2).
+- ``attn_probs`` : the softmax matrix P of one head (tiny sizes).
+- ``causal_tile_count`` : element-wise enumeration of computed/skipped tile pairs.
+
+Parity pins: every function above is pinned by tests in tests/test_oracle.py.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "attn_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+F16 = 0
+BF16 = 1
+
+
+def build(force: bool = False) -> str:
+    """Compile attn_oracle.c into liboracle.so next to it (gcc, OpenMP)."""
+    if (not force and os.path.exists(_LIB_PATH)
+            and os.path.getmtime(_LIB_PATH) >= os.path.getmtime(_SRC)):
+        return _LIB_PATH
+    tmp = _LIB_PATH + f".tmp{os.getpid()}"
+    cmd = ["gcc", "-O2", "-std=c99", "-fopenmp", "-shared", "-fPIC", "-o", tmp, _SRC, "-lm"]
+    subprocess.run(cmd, check=True)
+    os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        lib = ctypes.CDLL(build())
+        u16p = ctypes.POINTER(ctypes.c_uint16)
+        f64p = ctypes.POINTER(ctypes.c_double)
+        i64p = ctypes.POINTER(ctypes.c_int64)
+        i64 = ctypes.c_int64
+        lib.oracle_f16_to_f64.argtypes = [ctypes.c_uint16]
+        lib.oracle_f16_to_f64.restype = ctypes.c_double
+        lib.oracle_bf16_to_f64.argtypes = [ctypes.c_uint16]
+        lib.oracle_bf16_to_f64.restype = ctypes.c_double
+        lib.oracle_decode.argtypes = [u16p, f64p, i64, ctypes.c_int]
+        lib.oracle_decode.restype = None
+        lib.oracle_attn_fwd.argtypes = [u16p, u16p, u16p, i64, i64, i64, i64, ctypes.c_float,
+                                        ctypes.c_int, ctypes.c_int, f64p, f64p]
+        lib.oracle_attn_fwd.restype = ctypes.c_int
+        lib.oracle_attn_rows.argtypes = [u16p, u16p, u16p, i64, i64, i64, i64, ctypes.c_float,
+                                         ctypes.c_int, ctypes.c_int, i64p, i64p, i64, f64p, f64p]
+        lib.oracle_attn_rows.restype = ctypes.c_int
+        lib.oracle_attn_probs.argtypes = [u16p, u16p, i64, i64, i64, i64, ctypes.c_float,
+                                          ctypes.c_int, ctypes.c_int, i64, f64p]
+        lib.oracle_attn_probs.restype = ctypes.c_int
+        lib.oracle_attn_tiled.argtypes = [u16p, u16p, u16p, i64, i64, i64, i64, ctypes.c_float,
+                                          ctypes.c_int, ctypes.c_int, i64, i64, ctypes.c_int,
+                                          f64p, f64p]
+        lib.oracle_attn_tiled.restype = ctypes.c_int
+        lib.oracle_causal_tile_count.argtypes = [i64, i64, i64, i64p, i64p, i64p]
+        lib.oracle_causal_tile_count.restype = None
+        lib.oracle_num_threads.argtypes = []
+        lib.oracle_num_threads.restype = ctypes.c_int
+        _lib = lib
+        return lib
+
+
+def _dtype_code(dtype) -> int:
+    name = str(dtype).replace("torch.", "")
+    if name in ("fp16", "float16", "half"):
+        return F16
+    if name in ("bf16", "bfloat16"):
+        return BF16
+    raise ValueError(f"oracle: unsupported dtype {dtype!r}")
+
+
+def _bits(x) -> np.ndarray:
+    """16-bit bit patterns of a torch fp16/bf16 tensor or a uint16 numpy array."""
+    if isinstance(x, np.ndarray):
+        if x.dtype == np.uint16:
+            return np.ascontiguousarray(x)
+        if x.dtype == np.float16:
+            return np.ascontiguousarray(x).view(np.uint16)
+        raise TypeError("oracle: numpy input must be uint16 bit patterns or float16")
+    import torch  # local: only tensors need it
+    t = x.detach().to("cpu").contiguous()
+    if t.dtype not in (torch.float16, torch.bfloat16):
+        raise TypeError("oracle: tensor input must be float16 or bfloat16")
+    return t.view(torch.int16).numpy().view(np.uint16)
+
+
+def _ptr(a: np.ndarray, ctype):
+    return a.ctypes.data_as(ctypes.POINTER(ctype))
+
+
+def decode(bits: np.ndarray, dtype) -> np.ndarray:
+    lib = _load()
+    b = np.ascontiguousarray(bits, dtype=np.uint16)
+    out = np.empty(b.shape, dtype=np.float64)
+    lib.oracle_decode(_ptr(b, ctypes.c_uint16), _ptr(out, ctypes.c_double), b.size, _dtype_code(dtype))
+    return out
+
+
+def attn_fwd(q, k, v, scale: float, causal: bool, dtype):
+    """Naive fp64 attention on BHSD inputs. Returns (O [B,H,S,D], LSE [B,H,S]) float64."""
+    lib = _load()
+    qb, kb, vb = _bits(q), _bits(k), _bits(v)
+    B, H, S, D = qb.shape
+    o = np.empty((B, H, S, D), dtype=np.float64)
+    lse = np.empty((B, H, S), dtype=np.float64)
+    rc = lib.oracle_attn_fwd(_ptr(qb, ctypes.c_uint16), _ptr(kb, ctypes.c_uint16),
+                             _ptr(vb, ctypes.c_uint16), B, H, S, D, float(np.float32(scale)),
+                             int(bool(causal)), _dtype_code(dtype),
+                             _ptr(o, ctypes.c_double), _ptr(lse, ctypes.c_double))
+    if rc != 0:
+        raise RuntimeError(f"oracle_attn_fwd failed with {rc}")
+    return o, lse
+
+
+def attn_rows(q, k, v, scale: float, causal: bool, dtype, bh_idx, row_idx):
+    """The definition for selected rows only. Returns (O [n,D], LSE [n]) float64."""
+    lib = _load()
+    qb, kb, vb = _bits(q), _bits(k), _bits(v)
+    B, H, S, D = qb.shape
+    bh = np.ascontiguousarray(bh_idx, dtype=np.int64)
+    ri = np.ascontiguousarray(row_idx, dtype=np.int64)
+    n = bh.size
+    o = np.empty((n, D), dtype=np.float64)
+    lse = np.empty((n,), dtype=np.float64)
+    rc = lib.oracle_attn_rows(_ptr(qb, ctypes.c_uint16), _ptr(kb, ctypes.c_uint16),
+                              _ptr(vb, ctypes.c_uint16), B, H, S, D, float(np.float32(scale)),
+                              int(bool(causal)), _dtype_code(dtype),
+                              _ptr(bh, ctypes.c_int64), _ptr(ri, ctypes.c_int64), n,
+                              _ptr(o, ctypes.c_double), _ptr(lse, ctypes.c_double))
+    if rc != 0:
+        raise RuntimeError(f"oracle_attn_rows failed with {rc}")
+    return o, lse
+
+
+def attn_tiled(q, k, v, scale: float, causal: bool, dtype, Br: int, Bc: int, form: int = 0):
+    """Tiled online-softmax reference (form 0 deferred /l, form 1 per-step normalised)."""
+    lib = _load()
+    qb, kb, vb = _bits(q), _bits(k), _bits(v)
+    B, H, S, D = qb.shape
+    o = np.empty((B, H, S, D), dtype=np.float64)
+    lse = np.empty((B, H, S), dtype=np.float64)
+    rc = lib.oracle_attn_tiled(_ptr(qb, ctypes.c_uint16), _ptr(kb, ctypes.c_uint16),
+                               _ptr(vb, ctypes.c_uint16), B, H, S, D, float(np.float32(scale)),
+                               int(bool(causal)), _dtype_code(dtype), int(Br), int(Bc), int(form),
+                               _ptr(o, ctypes.c_double), _ptr(lse, ctypes.c_double))
+    if rc != 0:
+        raise RuntimeError(f"oracle_attn_tiled failed with {rc}")
+    return o, lse
+
+
+def attn_probs(q, k, scale: float, causal: bool, dtype, bh: int = 0) -> np.ndarray:
+    """Softmax matrix P [S,S] of head ``bh`` (flattened b*H+h)."""
+    lib = _load()
+    qb, kb = _bits(q), _bits(k)
+    B, H, S, D = qb.shape
+    p = np.empty((S, S), dtype=np.float64)
+    rc = lib.oracle_attn_probs(_ptr(qb, ctypes.c_uint16), _ptr(kb, ctypes.c_uint16), B, H, S, D,
+                               float(np.float32(scale)), int(bool(causal)), _dtype_code(dtype),
+                               int(bh), _ptr(p, ctypes.c_double))
+    if rc != 0:
+        raise RuntimeError(f"oracle_attn_probs failed with {rc}")
+    return p
+
+
+def causal_tile_count(S: int, BM: int, BN: int):
+    """(total, computed, skipped) tile pairs of a causal S x S problem, by enumeration."""
+    lib = _load()
+    t, c, s = ctypes.c_int64(), ctypes.c_int64(), ctypes.c_int64()
+    lib.oracle_causal_tile_count(int(S), int(BM), int(BN), ctypes.byref(t), ctypes.byref(c),
+                                 ctypes.byref(s))
+    return t.value, c.value, s.value
+
+
+def num_threads() -> int:
+    return int(_load().oracle_num_threads())

@@ -1,0 +1,405 @@
+/*
+ * attn_oracle.c -- plain, slow, fp64 CPU oracle for the attention forward pass.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path (the CUDA library
+ * and its Python binding) may link, load or call this file.  It is used by
+ * tests/, by the smoke check, and by the CPU-baseline leg of the benchmark.
+ * It shares no code, header, table or constant with the CUDA path.
+ *
+ * What it computes (the definition, not an algorithm):
+ *
+ *   For every (b, h) and query row i in [0, S):
+ *     s_ij  = scale * sum_d q_id * k_jd            for j in J_i
+ *     m_i   = max_j s_ij
+ *     p_ij  = exp(s_ij - m_i)
+ *     l_i   = sum_j p_ij
+ *     O_id  = (sum_j p_ij * v_jd) / l_i
+ *     LSE_i = m_i + log(l_i)                      (natural log)
+ *   where J_i = [0, S) without the causal mask and J_i = [0, i] with it.
+ *
+ *   Sources:
+ *   - Scaled dot-product attention softmax(QK^T / sqrt(d_k)) V:
+ *     "FlashAttention-2 在昇腾 NPU 上如何做到 3 倍加速？深度拆解 ops-transformer 的实现",
+ *     section 1 (the Attention(Q,K,V) equation); and
+ *     "ops-transformer FlashAttention 算子实战：让昇腾NPU算力彻底释放",
+ *     section 4.2 (the naive_attention comparison function).
+ *   - Causal attention (each position sees only itself and earlier tokens):
+ *     the gsyq.cn catlass page (13B service moved to Ascend), section
+ *     "Causal Mask的实现差异"; and the ops-transformer page, section 4.1
+ *     (causal=True for autoregressive models).
+ *   - The log-sum-exp per row is not defined on the pages; it is read as the
+ *     natural log of sum_j exp(s_ij) with s already scaled.
+ *
+ * The naive path materialises each query's full score row and runs a
+ * two-pass softmax (max, then exp/sum).  The tiled path is a separately
+ * written online-softmax recurrence that follows the page's section 2.1
+ * (tiling) and 2.2 (online softmax) of the FlashAttention-2 page, in two forms:
+ *   form 0: deferred normalisation (O and l rescaled by e^{m_old-m_new},
+ *           one division by l at the end);
+ *   form 1: the page's printed recurrence, which normalises at every step
+ *           (p_j divided by l_new, O rescaled by (l_old/l_new) e^{m_old-m_new}).
+ * With the causal mask the tiled path skips key tiles whose first key lies
+ * after the last query of the query tile (mode 2 "对角线跳过" of the gsyq.cn
+ * catlass page; the comparison operator is lost in the page's text and is
+ * read as ">=").
+ *
+ * Inputs are the exact 16-bit values the GPU receives (IEEE binary16 or
+ * bfloat16 bit patterns), decoded here to double by this file's own decoders.
+ * All arithmetic is double precision; scale is the caller's float promoted
+ * to double.
+ *
+ * Build: gcc -O2 -fopenmp -shared -fPIC -o liboracle.so attn_oracle.c -lm
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+#define ORACLE_F16 0
+#define ORACLE_BF16 1
+
+/* ---------------------------------------------------------------- decoders */
+
+/* IEEE 754 binary16: 1 sign bit, 5 exponent bits (bias 15), 10 fraction bits. */
+double oracle_f16_to_f64(uint16_t h)
+{
+    int sign = (h >> 15) & 1;
+    int e = (h >> 10) & 0x1f;
+    int f = h & 0x3ff;
+    double mag;
+    if (e == 0) {
+        mag = ldexp((double)f, -24);            /* subnormal: f * 2^-14 * 2^-10 */
+    } else if (e == 31) {
+        mag = (f == 0) ? INFINITY : NAN;
+    } else {
+        mag = ldexp((double)(1024 + f), e - 25); /* (1 + f/2^10) * 2^(e-15) */
+    }
+    return sign ? -mag : mag;
+}
+
+/* bfloat16: 1 sign bit, 8 exponent bits (bias 127), 7 fraction bits. */
+double oracle_bf16_to_f64(uint16_t b)
+{
+    int sign = (b >> 15) & 1;
+    int e = (b >> 7) & 0xff;
+    int f = b & 0x7f;
+    double mag;
+    if (e == 0) {
+        mag = ldexp((double)f, -133);           /* f * 2^-126 * 2^-7 */
+    } else if (e == 255) {
+        mag = (f == 0) ? INFINITY : NAN;
+    } else {
+        mag = ldexp((double)(128 + f), e - 134); /* (1 + f/2^7) * 2^(e-127) */
+    }
+    return sign ? -mag : mag;
+}
+
+void oracle_decode(const uint16_t *src, double *dst, int64_t n, int dtype)
+{
+    for (int64_t i = 0; i < n; ++i)
+        dst[i] = (dtype == ORACLE_BF16) ? oracle_bf16_to_f64(src[i]) : oracle_f16_to_f64(src[i]);
+}
+
+static int check_args(int64_t B, int64_t H, int64_t S, int64_t D, int dtype)
+{
+    if (B < 0 || H < 0 || S < 0 || D <= 0) return -2;
+    if (dtype != ORACLE_F16 && dtype != ORACLE_BF16) return -4;
+    return 0;
+}
+
+/* Decode one (b,h) slice [S, D] of a BHSD tensor. */
+static double *decode_head(const uint16_t *x, int64_t bh, int64_t S, int64_t D, int dtype)
+{
+    double *out = (double *)malloc(sizeof(double) * (size_t)(S * D > 0 ? S * D : 1));
+    if (!out) return NULL;
+    oracle_decode(x + bh * S * D, out, S * D, dtype);
+    return out;
+}
+
+/* ------------------------------------------------------- naive definition */
+
+/*
+ * One query row of the definition above.  qi: [D]; kh, vh: [S, D] decoded.
+ * srow: scratch of length S (the materialised score row).
+ */
+static void naive_row(const double *qi, const double *kh, const double *vh, int64_t i, int64_t S,
+                      int64_t D, double scale, int causal, double *srow, double *o, double *lse)
+{
+    int64_t nj = causal ? (i + 1 < S ? i + 1 : S) : S; /* J_i = [0, nj) */
+    /* scores */
+    for (int64_t j = 0; j < nj; ++j) {
+        double dot = 0.0;
+        for (int64_t d = 0; d < D; ++d) dot += qi[d] * kh[j * D + d];
+        srow[j] = scale * dot;
+    }
+    /* pass 1: max */
+    double m = -INFINITY;
+    for (int64_t j = 0; j < nj; ++j)
+        if (srow[j] > m) m = srow[j];
+    /* pass 2: exponentials and their sum */
+    double l = 0.0;
+    for (int64_t j = 0; j < nj; ++j) {
+        srow[j] = exp(srow[j] - m);
+        l += srow[j];
+    }
+    /* P V, then normalise */
+    for (int64_t d = 0; d < D; ++d) o[d] = 0.0;
+    for (int64_t j = 0; j < nj; ++j) {
+        double p = srow[j];
+        for (int64_t d = 0; d < D; ++d) o[d] += p * vh[j * D + d];
+    }
+    for (int64_t d = 0; d < D; ++d) o[d] /= l;
+    *lse = m + log(l);
+}
+
+/*
+ * Full naive attention.  q, k, v: BHSD 16-bit bit patterns.
+ * o: [B,H,S,D] double, lse: [B,H,S] double.  Returns 0 or a negative code.
+ */
+int oracle_attn_fwd(const uint16_t *q, const uint16_t *k, const uint16_t *v, int64_t B, int64_t H,
+                    int64_t S, int64_t D, float scale, int causal, int dtype, double *o, double *lse)
+{
+    int rc = check_args(B, H, S, D, dtype);
+    if (rc) return rc;
+    const double sc = (double)scale;
+    for (int64_t bh = 0; bh < B * H; ++bh) {
+        double *qh = decode_head(q, bh, S, D, dtype);
+        double *kh = decode_head(k, bh, S, D, dtype);
+        double *vh = decode_head(v, bh, S, D, dtype);
+        if (!qh || !kh || !vh) {
+            free(qh); free(kh); free(vh);
+            return -10;
+        }
+#pragma omp parallel
+        {
+            double *srow = (double *)malloc(sizeof(double) * (size_t)(S > 0 ? S : 1));
+#pragma omp for schedule(dynamic, 16)
+            for (int64_t i = 0; i < S; ++i)
+                naive_row(qh + i * D, kh, vh, i, S, D, sc, causal, srow, o + (bh * S + i) * D,
+                          lse + bh * S + i);
+            free(srow);
+        }
+        free(qh); free(kh); free(vh);
+    }
+    return 0;
+}
+
+/*
+ * The same definition for a list of (bh, i) rows only: used to check sampled
+ * rows of full-size runs.  o: [nrows, D], lse: [nrows].
+ */
+int oracle_attn_rows(const uint16_t *q, const uint16_t *k, const uint16_t *v, int64_t B, int64_t H,
+                     int64_t S, int64_t D, float scale, int causal, int dtype, const int64_t *bh_idx,
+                     const int64_t *row_idx, int64_t nrows, double *o, double *lse)
+{
+    int rc = check_args(B, H, S, D, dtype);
+    if (rc) return rc;
+    for (int64_t r = 0; r < nrows; ++r)
+        if (bh_idx[r] < 0 || bh_idx[r] >= B * H || row_idx[r] < 0 || row_idx[r] >= S) return -2;
+    const double sc = (double)scale;
+    int bad = 0;
+#pragma omp parallel
+    {
+        double *srow = (double *)malloc(sizeof(double) * (size_t)(S > 0 ? S : 1));
+        double *qi = (double *)malloc(sizeof(double) * (size_t)D);
+        double *kh = (double *)malloc(sizeof(double) * (size_t)(S * D > 0 ? S * D : 1));
+        double *vh = (double *)malloc(sizeof(double) * (size_t)(S * D > 0 ? S * D : 1));
+        int64_t cur_bh = -1;
+        if (!srow || !qi || !kh || !vh) {
+#pragma omp atomic write
+            bad = 1;
+        }
+        /* rows are expected grouped by bh; each thread decodes a head once per run of rows */
+#pragma omp for schedule(static)
+        for (int64_t r = 0; r < nrows; ++r) {
+            if (!srow || !qi || !kh || !vh) continue;
+            int64_t bh = bh_idx[r], i = row_idx[r];
+            if (bh != cur_bh) {
+                oracle_decode(k + bh * S * D, kh, S * D, dtype);
+                oracle_decode(v + bh * S * D, vh, S * D, dtype);
+                cur_bh = bh;
+            }
+            oracle_decode(q + (bh * S + i) * D, qi, D, dtype);
+            naive_row(qi, kh, vh, i, S, D, sc, causal, srow, o + r * D, lse + r);
+        }
+        free(srow); free(qi); free(kh); free(vh);
+    }
+    return bad ? -10 : 0;
+}
+
+/*
+ * Softmax probabilities P [S, S] of one (b,h) slice (tiny sizes only), by the
+ * definition above; masked entries are 0.
+ */
+int oracle_attn_probs(const uint16_t *q, const uint16_t *k, int64_t B, int64_t H, int64_t S,
+                      int64_t D, float scale, int causal, int dtype, int64_t bh, double *p)
+{
+    int rc = check_args(B, H, S, D, dtype);
+    if (rc) return rc;
+    if (bh < 0 || bh >= B * H) return -2;
+    double *qh = decode_head(q, bh, S, D, dtype);
+    double *kh = decode_head(k, bh, S, D, dtype);
+    if (!qh || !kh) { free(qh); free(kh); return -10; }
+    const double sc = (double)scale;
+    for (int64_t i = 0; i < S; ++i) {
+        double *row = p + i * S;
+        int64_t nj = causal ? i + 1 : S;
+        double m = -INFINITY;
+        for (int64_t j = 0; j < S; ++j) {
+            if (j >= nj) { row[j] = -INFINITY; continue; }
+            double dot = 0.0;
+            for (int64_t d = 0; d < D; ++d) dot += qh[i * D + d] * kh[j * D + d];
+            row[j] = sc * dot;
+            if (row[j] > m) m = row[j];
+        }
+        double l = 0.0;
+        for (int64_t j = 0; j < S; ++j) {
+            row[j] = (j < nj) ? exp(row[j] - m) : 0.0;
+            l += row[j];
+        }
+        for (int64_t j = 0; j < S; ++j) row[j] /= l;
+    }
+    free(qh); free(kh);
+    return 0;
+}
+
+/* ------------------------------------------- tiled online-softmax reference */
+
+/*
+ * Causal mode 2 of the gsyq.cn catlass page: key tile tn is skipped for query
+ * tile tm when its first key comes after the last query of the query tile.
+ */
+static int tile_skipped(int64_t tm, int64_t tn, int64_t Br, int64_t Bc)
+{
+    return tn * Bc >= (tm + 1) * Br;
+}
+
+/*
+ * Tiled reference: Q in tiles of Br rows, K/V in tiles of Bc rows, an outer
+ * loop over Q tiles and an inner loop over K/V tiles, with the running max m
+ * and running sum l of the FlashAttention-2 page, section 2.2.
+ * form 0: deferred normalisation.  form 1: the page's per-step normalised
+ * recurrence.  Keys beyond S in a ragged last tile are not visited.
+ */
+int oracle_attn_tiled(const uint16_t *q, const uint16_t *k, const uint16_t *v, int64_t B, int64_t H,
+                      int64_t S, int64_t D, float scale, int causal, int dtype, int64_t Br,
+                      int64_t Bc, int form, double *o, double *lse)
+{
+    int rc = check_args(B, H, S, D, dtype);
+    if (rc) return rc;
+    if (Br <= 0 || Bc <= 0 || (form != 0 && form != 1)) return -2;
+    const double sc = (double)scale;
+    const int64_t nq = (S + Br - 1) / Br, nk = (S + Bc - 1) / Bc;
+    for (int64_t bh = 0; bh < B * H; ++bh) {
+        double *qh = decode_head(q, bh, S, D, dtype);
+        double *kh = decode_head(k, bh, S, D, dtype);
+        double *vh = decode_head(v, bh, S, D, dtype);
+        if (!qh || !kh || !vh) { free(qh); free(kh); free(vh); return -10; }
+#pragma omp parallel for schedule(dynamic, 1)
+        for (int64_t tm = 0; tm < nq; ++tm) {
+            int64_t r0 = tm * Br, r1 = (r0 + Br < S) ? r0 + Br : S;
+            int64_t nr = r1 - r0;
+            double *m = (double *)malloc(sizeof(double) * (size_t)nr);
+            double *l = (double *)malloc(sizeof(double) * (size_t)nr);
+            double *acc = (double *)calloc((size_t)(nr * D), sizeof(double));
+            double *s = (double *)malloc(sizeof(double) * (size_t)Bc);
+            for (int64_t r = 0; r < nr; ++r) { m[r] = -INFINITY; l[r] = 0.0; }
+            for (int64_t tn = 0; tn < nk; ++tn) {
+                if (causal && tile_skipped(tm, tn, Br, Bc)) continue;
+                int64_t c0 = tn * Bc, c1 = (c0 + Bc < S) ? c0 + Bc : S;
+                for (int64_t r = 0; r < nr; ++r) {
+                    int64_t i = r0 + r;
+                    /* score block row, masked entries -inf */
+                    double bmax = -INFINITY;
+                    for (int64_t j = c0; j < c1; ++j) {
+                        double x = -INFINITY;
+                        if (!causal || j <= i) {
+                            double dot = 0.0;
+                            for (int64_t d = 0; d < D; ++d) dot += qh[i * D + d] * kh[j * D + d];
+                            x = sc * dot;
+                        }
+                        s[j - c0] = x;
+                        if (x > bmax) bmax = x;
+                    }
+                    if (bmax == -INFINITY) continue; /* whole block masked for this row */
+                    double m_old = m[r];
+                    double m_new = (bmax > m_old) ? bmax : m_old;
+                    double alpha = (m_old == -INFINITY) ? 0.0 : exp(m_old - m_new);
+                    double psum = 0.0;
+                    for (int64_t j = c0; j < c1; ++j) {
+                        double e = (s[j - c0] == -INFINITY) ? 0.0 : exp(s[j - c0] - m_new);
+                        s[j - c0] = e;
+                        psum += e;
+                    }
+                    double l_new = alpha * l[r] + psum;
+                    double *a = acc + r * D;
+                    if (form == 0) {
+                        for (int64_t d = 0; d < D; ++d) {
+                            double pv = 0.0;
+                            for (int64_t j = c0; j < c1; ++j) pv += s[j - c0] * vh[j * D + d];
+                            a[d] = alpha * a[d] + pv;
+                        }
+                    } else {
+                        /* o <- p_j v_j + (l_old / l_new) e^{m_old - m_new} o, p_j = e^{s-m_new}/l_new */
+                        double keep = (l[r] == 0.0) ? 0.0 : (l[r] / l_new) * alpha;
+                        for (int64_t d = 0; d < D; ++d) {
+                            double pv = 0.0;
+                            for (int64_t j = c0; j < c1; ++j) pv += (s[j - c0] / l_new) * vh[j * D + d];
+                            a[d] = pv + keep * a[d];
+                        }
+                    }
+                    m[r] = m_new;
+                    l[r] = l_new;
+                }
+            }
+            for (int64_t r = 0; r < nr; ++r) {
+                int64_t i = r0 + r;
+                for (int64_t d = 0; d < D; ++d)
+                    o[(bh * S + i) * D + d] = (form == 0) ? acc[r * D + d] / l[r] : acc[r * D + d];
+                lse[bh * S + i] = m[r] + log(l[r]);
+            }
+            free(m); free(l); free(acc); free(s);
+        }
+        free(qh); free(kh); free(vh);
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------ causal tile counts */
+
+/*
+ * Brute-force count of (query tile, key tile) pairs for an S x S causal
+ * problem with BM x BN tiles: a pair is "computed" when at least one of its
+ * (i, j) elements has j <= i, else "skipped".  total = computed + skipped.
+ * This is an element-by-element enumeration, independent of any loop bound.
+ */
+void oracle_causal_tile_count(int64_t S, int64_t BM, int64_t BN, int64_t *total, int64_t *computed,
+                              int64_t *skipped)
+{
+    int64_t nq = (S + BM - 1) / BM, nk = (S + BN - 1) / BN;
+    int64_t c = 0, s = 0;
+    for (int64_t tm = 0; tm < nq; ++tm)
+        for (int64_t tn = 0; tn < nk; ++tn) {
+            int any = 0;
+            for (int64_t i = tm * BM; i < (tm + 1) * BM && i < S && !any; ++i)
+                for (int64_t j = tn * BN; j < (tn + 1) * BN && j < S; ++j)
+                    if (j <= i) { any = 1; break; }
+            if (any) ++c; else ++s;
+        }
+    *total = nq * nk;
+    *computed = c;
+    *skipped = s;
+}
+
+int oracle_num_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
