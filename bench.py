@@ -1,0 +1,386 @@
+"""Benchmark of the fused attention forward pass on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl fa|reference]
+                    [--workload c5|c1|c2|c3|c4|c5a|c5b] [--no-e2e] [--no-cpu-baseline]
+
+A step is one pass of the whole forward path over one batch of synthetic
+input.  The default workload is the long-context configuration
+B=1, H=32, S=16384, D=128, bf16, run both without and with the causal mask
+(two fa_fwd launches per step).  Inputs (512 MiB) are larger than the 126 MB
+L2, so no L2 flush is needed between steps.
+
+Throughput is attention TFLOP/s with the causal case counted at half
+(4*B*H*S^2*D per non-causal run), over the whole job: with N GPUs (one
+process per GPU, torchrun) every rank runs its own independent batch of the
+same shape (weak scaling, no data-path collective) and the value is the
+total work of all ranks over the slowest rank's device time.
+
+``--impl reference`` times the fp64 CPU oracle on bounded row samples of the
+same workload (rank 0 only) and prints the same JSON line with
+"impl": "reference".
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from tiled_attention_18_b200.workloads import WORKLOADS, attention_flops, make_inputs, sample_rows  # noqa: E402
+
+METRIC = "attention fwd TFLOPS (causal-adjusted) and % of B200 dense fp16/bf16 peak"
+UNIT = "TFLOP/s"
+FALLBACK_BF16_TFLOPS = 1590.0
+PEAKS_PATH = os.path.join(ROOT, "MEASURED_PEAKS.json")
+TRAFFIC_PATH = os.path.join(ROOT, "profiles", "fa_fwd_traffic.json")
+KERNEL_SRC = os.path.join(ROOT, "tiled_attention_18_b200", "csrc", "fa_fwd_sm100.cu")
+
+
+def workload_runs(name: str):
+    """The fa_fwd runs of one step: (Workload, ...)."""
+    if name == "c5":
+        return [WORKLOADS["c5a"], WORKLOADS["c5b"]]
+    return [WORKLOADS[name]]
+
+
+def workload_label(name: str) -> str:
+    runs = workload_runs(name)
+    w = runs[0]
+    causal = "non-causal + causal" if len(runs) == 2 else ("causal" if w.causal else "non-causal")
+    extra = f", Q,K x{w.qk_mult:g}" if w.qk_mult != 1.0 else ""
+    return f"attention fwd {w.dtype} B={w.B} H={w.H} S={w.S} D={w.D}, {causal}{extra}"
+
+
+def peak_tflops():
+    try:
+        with open(PEAKS_PATH) as f:
+            p = json.load(f)
+        return float(p["bf16_tflops"]), "measured (MEASURED_PEAKS.json bf16_tflops, burst)"
+    except Exception:
+        return FALLBACK_BF16_TFLOPS, "fallback (1.59 PFLOP/s pool measurement)"
+
+
+def kernel_source_hash() -> str:
+    import hashlib
+    with open(KERNEL_SRC, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def traffic_per_launch():
+    """DRAM bytes per launch from the committed ncu summary, if taken on this kernel source."""
+    try:
+        with open(TRAFFIC_PATH) as f:
+            t = json.load(f)
+        if t.get("kernel_source_sha256_16") != kernel_source_hash():
+            return None
+        return float(t["dram_bytes_per_step"])
+    except Exception:
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi clocks/throttle sampling during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.samples = []
+        self._stop = threading.Event()
+        self._proc = None
+        self._thread = None
+
+    def start(self):
+        try:
+            self._proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self._proc = None
+            return
+        self._thread = threading.Thread(target=self._read, daemon=True)
+        self._thread.start()
+
+    def _read(self):
+        for line in self._proc.stdout:
+            if self._stop.is_set():
+                break
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 9:
+                self.samples.append(parts)
+
+    def stop(self):
+        self._stop.set()
+        if self._proc is not None:
+            self._proc.terminate()
+            try:
+                self._proc.wait(timeout=5)
+            except Exception:
+                self._proc.kill()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        sm = [float(s[1]) for s in self.samples if s[1].replace(".", "").isdigit()]
+        smax = [float(s[2]) for s in self.samples if s[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = set()
+        for s in self.samples:
+            for n, val in zip(names, s[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(self.samples)}
+
+
+def cpu_baseline(name: str, target_s: float = 12.0):
+    """Time the oracle on a bounded row sample of the workload; TFLOP/s of the sample."""
+    import oracle
+    runs = workload_runs(name)
+    per_run_s = target_s / len(runs)
+    flops_total, t_total, rows_total = 0.0, 0.0, 0
+    desc = []
+    for w in runs:
+        q, k, v = make_inputs(w.B, w.H, w.S, w.D, w.dtype, w.qk_mult, w.seed)
+        # rows of the sample: random rows over all heads; cost per row = 4*D*(keys seen)
+        n = 64
+        while True:
+            bh, rows = sample_rows(w.B, w.H, w.S, n_random=n, edge=0, seed=99)
+            t0 = time.perf_counter()
+            oracle.attn_rows(q, k, v, w.scale, w.causal, w.dtype, bh, rows)
+            dt = time.perf_counter() - t0
+            if dt >= per_run_s * 0.5 or n >= (1 << 20):
+                break
+            n = int(n * min(16.0, max(2.0, per_run_s / max(dt, 1e-3))))
+        keys = (rows + 1) if w.causal else np.full_like(rows, w.S)
+        flops = float(4.0 * w.D * keys.sum())
+        flops_total += flops
+        t_total += dt
+        rows_total += len(rows)
+        desc.append(f"{len(rows)} random query rows of {w.describe()}")
+    return {"value": flops_total / t_total / 1e12, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": "; ".join(desc) + f" ({t_total:.1f} s fp64 on the host cores; TFLOP/s of the sample's"
+                      " algorithmic flops)"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    runs = workload_runs(args.workload)
+    for _ in range(args.warmup):
+        pass  # the oracle has no warm-up state; warm-up steps are not needed
+    cb = None
+    times = []
+    flops_total = 0.0
+    for _ in range(args.steps):
+        cb = cpu_baseline(args.workload, target_s=max(2.0, 60.0 / max(args.steps, 1)))
+        times.append(cb)
+    value = float(np.median([c["value"] for c in times]))
+    cb = dict(times[-1])
+    cb["value"] = value
+    step_flops = sum(w.flops for w in runs)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_flops / (value * 1e12) * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": workload_label(args.workload), "note": "fp64 CPU oracle on bounded row samples"},
+        "cpu_baseline": cb,
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    del flops_total
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main(argv=None) -> int:
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["fa", "reference"], default="fa")
+    ap.add_argument("--workload", default="c5", choices=["c5"] + list(WORKLOADS))
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+    import torch.distributed as dist
+
+    import tiled_attention_18_b200 as fa
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        print(f"warning: --gpus {args.gpus} but WORLD_SIZE={world}; using WORLD_SIZE", file=sys.stderr)
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    fa.load()
+    runs = workload_runs(args.workload)
+    stream = torch.cuda.current_stream(dev)
+    sid = stream.cuda_stream
+
+    # inputs: each rank draws its own independent batch (seed = workload seed + rank)
+    host_in, dev_in, dev_out = [], [], []
+    for i, w in enumerate(runs):
+        if i > 0 and (w.B, w.H, w.S, w.D, w.dtype, w.qk_mult) == (runs[0].B, runs[0].H, runs[0].S, runs[0].D,
+                                                                   runs[0].dtype, runs[0].qk_mult):
+            host_in.append(host_in[0])
+            dev_in.append(dev_in[0])
+        else:
+            q, k, v = make_inputs(w.B, w.H, w.S, w.D, w.dtype, w.qk_mult, w.seed + rank)
+            host_in.append(tuple(t.pin_memory() for t in (q, k, v)))
+            dev_in.append(tuple(t.to(dev) for t in (q, k, v)))
+        o = torch.empty((w.B, w.H, w.S, w.D), dtype=w.torch_dtype, device=dev)
+        lse = torch.empty((w.B, w.H, w.S), dtype=torch.float32, device=dev)
+        dev_out.append((o, lse))
+
+    def launch(i):
+        w = runs[i]
+        q, k, v = dev_in[i]
+        o, lse = dev_out[i]
+        st = fa.fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), w.B, w.H, w.S, w.D,
+                       w.scale, int(w.causal), fa.FA_BF16 if w.dtype == "bf16" else fa.FA_FP16, sid)
+        if st != 0:
+            raise fa.FaError(st)
+
+    # warm-up
+    for _ in range(args.warmup):
+        for i in range(len(runs)):
+            launch(i)
+    torch.cuda.synchronize(dev)
+    st = fa.fa_check_status(sid)
+    if st != 0:
+        raise fa.FaError(st, "warm-up")
+
+    # timed region: per-launch events on the launching stream
+    ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in runs]
+          for _ in range(args.steps)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.3)
+    barrier()
+    torch.cuda.synchronize(dev)
+    start.record(stream)
+    for s in range(args.steps):
+        for i in range(len(runs)):
+            ev[s][i][0].record(stream)
+            launch(i)
+            ev[s][i][1].record(stream)
+    stop.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    sampler.stop()
+    st = fa.fa_check_status(sid)
+    if st != 0:
+        raise fa.FaError(st, "timed region")
+    elapsed_ms = start.elapsed_time(stop)
+    kern_ms = np.array([[a.elapsed_time(b) for (a, b) in row] for row in ev])  # [steps, runs]
+    t = torch.tensor([elapsed_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    max_ms = float(t.item())
+    step_flops = sum(w.flops for w in runs)
+    value = step_flops * world * args.steps / (max_ms * 1e-3) / 1e12
+    peak, peak_src = peak_tflops()
+
+    # roofline of the kernel: algorithmic flops per launch / mean launch duration
+    per_run = []
+    for i, w in enumerate(runs):
+        mean_ms = float(kern_ms[:, i].mean())
+        per_run.append({"run": w.describe(), "mean_ms": mean_ms, "tflops": w.flops / (mean_ms * 1e-3) / 1e12})
+    achieved = step_flops / (float(kern_ms.sum(axis=1).mean()) * 1e-3) / 1e12
+    traffic = traffic_per_launch()
+
+    # end to end through the public call with host buffers
+    e2e = None
+    if not args.no_e2e:
+        host_out = [(torch.empty(o.shape, dtype=o.dtype).pin_memory(), torch.empty(l.shape, dtype=l.dtype).pin_memory())
+                    for (o, l) in dev_out]
+        h2d = sum(sum(t.numel() * t.element_size() for t in host_in[i]) for i in range(len(runs))
+                  if i == 0 or host_in[i] is not host_in[0])
+        d2h = sum(o.numel() * o.element_size() + l.numel() * l.element_size() for (o, l) in host_out)
+
+        def e2e_step():
+            for i, w in enumerate(runs):
+                if i == 0 or host_in[i] is not host_in[0]:
+                    for hsrc, dsrc in zip(host_in[i], dev_in[i]):
+                        dsrc.copy_(hsrc, non_blocking=True)
+                launch(i)
+                dev_out_o, dev_out_l = dev_out[i]
+                host_out[i][0].copy_(dev_out_o, non_blocking=True)
+                host_out[i][1].copy_(dev_out_l, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize(dev)
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier()
+        te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
+        if world > 1:
+            dist.all_reduce(te, op=dist.ReduceOp.MAX)
+        e2e_val = step_flops * world * args.e2e_steps / (float(te.item()) * 1e-3) / 1e12
+        e2e = {"value": e2e_val, "unit": UNIT, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+
+    cb = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cb = cpu_baseline(args.workload)
+
+    if rank == 0:
+        w0 = runs[0]
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": max_ms / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": w0.dtype, "data": "synthetic",
+            "config": {"workload": workload_label(args.workload), "B": w0.B, "H": w0.H, "S": w0.S, "D": w0.D,
+                       "runs_per_step": len(runs), "l2": "inputs larger than L2 (no flush)",
+                       "parallelism": f"independent batch per GPU x{world}"},
+            "pct_of_peak": 100.0 * value / (peak * world),
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": UNIT,
+                         "frac": achieved / peak, "traffic": traffic, "peak_source": peak_src,
+                         "per_run": per_run},
+            "clocks": sampler.summary(),
+            "e2e": e2e,
+            "gpu_launches": len(runs) * args.steps,
+            "cpu_baseline": cb,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

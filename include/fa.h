@@ -1,0 +1,128 @@
+/*
+ * fa.h -- C ABI of libfa.so: fused attention forward (FlashAttention-2 style)
+ * for NVIDIA B200 (sm_100a).
+ *
+ * The operation, per batch b, head h and query row i of contiguous BHSD
+ * tensors:
+ *
+ *   O[b,h,i,:]  = sum_j softmax_j( scale * Q[b,h,i,:] . K[b,h,j,:] ) * V[b,h,j,:]
+ *   LSE[b,h,i]  = log( sum_j exp( scale * Q[b,h,i,:] . K[b,h,j,:] ) )   (natural log)
+ *
+ * with j over [0, S), or over [0, i] when causal (each position sees only
+ * itself and earlier tokens; top-left aligned, Sq = Sk = S).
+ *
+ * Sources (page title, section):
+ *  - the attention equation softmax(QK^T / sqrt(d_k)) V and the tiled,
+ *    online-softmax evaluation that never stores the S x S score matrix:
+ *    "FlashAttention-2 在昇腾 NPU 上如何做到 3 倍加速？深度拆解 ops-transformer 的实现",
+ *    sections 1, 2.1 and 2.2;
+ *  - the operator call flash_attention(Q, K, V, causal=True) on [B, H, S, D]
+ *    tensors: "ops-transformer FlashAttention 算子实战：让昇腾NPU算力彻底释放",
+ *    section 4.1;
+ *  - the [batch, heads, seq_len, head_dim] row-major layout, FP16/BF16 inputs
+ *    and in-kernel causal tile skipping: the gsyq.cn catlass FlashAttention
+ *    page, sections on precision choice, data layout and "Causal Mask的实现差异";
+ *  - the explicit softmax scale (the caller passes it; there is no default):
+ *    the omica.com.cn cann-learning-hub FlashAttention tutorial, the step that
+ *    compares against SDPA.
+ * The per-row LSE is not defined on the pages; it is the natural log of the
+ * softmax denominator of the scaled scores.
+ *
+ * All calls are thread-safe and return an fa_status code; none aborts.
+ */
+#ifndef FA_H_
+#define FA_H_
+
+#include <cuda_runtime_api.h>
+
+#if defined(__GNUC__)
+#define FA_API __attribute__((visibility("default")))
+#else
+#define FA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum { FA_FP16 = 0, FA_BF16 = 1 } fa_dtype;
+
+typedef enum {
+    FA_OK = 0,
+    FA_ERR_NULL = -1,     /* a required pointer is NULL */
+    FA_ERR_SHAPE = -2,    /* B, H or S negative, or too large for 32-bit indexing */
+    FA_ERR_HEADDIM = -3,  /* D is not 64 or 128 */
+    FA_ERR_DTYPE = -4,    /* dtype is not FA_FP16 or FA_BF16 */
+    FA_ERR_ALIGN = -5,    /* q, k, v, o not 16-byte aligned, or lse not 4-byte aligned */
+    FA_ERR_ARCH = -6,     /* the current device is not compute capability 10.0 (sm_100) */
+    FA_ERR_LAUNCH = -7,   /* a CUDA runtime error (launch, tensor-map encoding, sync) */
+    FA_ERR_TIMEOUT = -8,  /* a device-side wait exceeded its bound (reported by fa_check_status) */
+    FA_ERR_SCALE = -9,    /* scale is not finite and > 0 */
+    FA_ERR_ARG = -10,     /* causal is not 0 or 1 */
+    FA_ERR_PTR = -11      /* a pointer is not device memory of the current device */
+} fa_status;
+
+/*
+ * fa_fwd -- attention forward pass with per-row log-sum-exp.
+ *
+ * q, k, v : device pointers, [B, H, S, D] contiguous (BHSD, row-major), dtype
+ *           elements; 16-byte aligned.  Read only.
+ * o       : device pointer, [B, H, S, D] contiguous, dtype; 16-byte aligned.
+ *           Written.  Must not overlap q, k, v or lse.
+ * lse     : device pointer, [B, H, S] contiguous fp32, 4-byte aligned.
+ *           Written (natural log).  Required.
+ * B, H, S : batch, heads, sequence length (queries = keys = S).  Any of them
+ *           0 is an empty problem: FA_OK, nothing is launched and the pointers
+ *           are not inspected.  B*H*S must fit in 31 bits.
+ * D       : head dimension, 64 or 128.
+ * scale   : softmax scale (commonly 1/sqrt(D)); finite and > 0.
+ * causal  : 0 = attend to all keys; 1 = key j attends to query i iff j <= i.
+ * dtype   : FA_FP16 or FA_BF16 (inputs and output).  Scores, the softmax
+ *           statistics and the accumulation are fp32; the softmax weights
+ *           are rounded to dtype before the P.V product; O is rounded to
+ *           nearest even.
+ * stream  : the CUDA stream to launch on (0 = legacy default stream).
+ *
+ * Ownership: the caller owns every buffer and the stream; fa_fwd allocates
+ * no device memory.  Synchronicity: asynchronous on `stream`; fa_fwd never
+ * synchronises.  Errors: argument checks run before any launch and return a
+ * negative fa_status with nothing launched; a launch failure returns
+ * FA_ERR_LAUNCH.  A device-side wait that exceeds its bound (about two
+ * seconds) makes the kernel stop early and is reported by fa_check_status.
+ */
+FA_API int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int S,
+           int D, float scale, int causal, int dtype, cudaStream_t stream);
+
+/*
+ * fa_check_status -- synchronise `stream`, then report and clear the device
+ * status word of the current device: FA_OK, FA_ERR_TIMEOUT if a kernel
+ * stopped on a bounded wait since the last call, or FA_ERR_LAUNCH on a CUDA
+ * error.  Meant for tests and diagnostics; it blocks the host.
+ */
+FA_API int fa_check_status(cudaStream_t stream);
+
+/*
+ * fa_last_timeout_site -- diagnostic word of the first failed wait recorded
+ * by the last fa_check_status that returned FA_ERR_TIMEOUT:
+ * (wait site) | (CTA index << 8).  0 if none.
+ */
+FA_API int fa_last_timeout_site(void);
+
+/* fa_status_string -- static, NUL-terminated description of a status code. */
+FA_API const char* fa_status_string(int status);
+
+/* fa_version -- library version as major*10000 + minor*100 + patch. */
+FA_API int fa_version(void);
+
+/*
+ * fa_num_units -- number of work units (b, h, 256-row query block) that
+ * fa_fwd distributes over persistent CTAs for the given shape; 0 for an empty
+ * problem, negative fa_status on invalid sizes.  Host only, no CUDA call.
+ */
+FA_API long long fa_num_units(int B, int H, int S);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_H_ */

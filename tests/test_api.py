@@ -1,0 +1,104 @@
+"""C-ABI checks that need no GPU: the library loads, exports every symbol
+include/fa.h declares, and rejects invalid arguments before any CUDA call."""
+import ctypes
+import math
+import os
+import re
+
+import pytest
+
+import tiled_attention_18_b200 as fa
+from tiled_attention_18_b200 import _lib
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_symbols():
+    with open(os.path.join(ROOT, "include", "fa.h")) as f:
+        text = f.read()
+    return re.findall(r"FA_API\s+[\w\s\*]+?\b(fa_\w+)\s*\(", text)
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from tiled_attention_18_b200 import build
+    build.build()
+    return fa.load()
+
+
+def test_header_declares_the_entry_points():
+    syms = _declared_symbols()
+    assert set(syms) == {name for name, _, _ in _lib.SIGNATURES}
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in _declared_symbols():
+        assert isinstance(getattr(lib, name), ctypes._CFuncPtr), name
+
+
+def test_status_enum_matches_header(lib):
+    with open(os.path.join(ROOT, "include", "fa.h")) as f:
+        text = f.read()
+    codes = dict((k, int(v)) for k, v in re.findall(r"(FA_(?:OK|ERR_\w+))\s*=\s*(-?\d+)", text))
+    for name, value in codes.items():
+        assert getattr(_lib, name) == value, name
+        assert fa.fa_status_string(value) not in ("", "unknown status")
+    assert fa.fa_status_string(12345) == "unknown status"
+
+
+def test_version_and_units(lib):
+    assert fa.fa_version() == 100
+    assert fa.fa_num_units(1, 32, 16384) == 32 * 64
+    assert fa.fa_num_units(2, 12, 2048) == 24 * 8
+    assert fa.fa_num_units(1, 1, 257) == 2
+    assert fa.fa_num_units(1, 1, 256) == 1
+    assert fa.fa_num_units(0, 4, 100) == 0
+    assert fa.fa_num_units(1, 1, -1) == _lib.FA_ERR_SHAPE
+
+
+A = 0x10000  # an aligned, non-null address (never dereferenced: checks fail first)
+
+
+@pytest.mark.parametrize("args,code", [
+    (dict(B=-1), _lib.FA_ERR_SHAPE),
+    (dict(S=-5), _lib.FA_ERR_SHAPE),
+    (dict(D=96), _lib.FA_ERR_HEADDIM),
+    (dict(D=256), _lib.FA_ERR_HEADDIM),
+    (dict(dtype=2), _lib.FA_ERR_DTYPE),
+    (dict(scale=0.0), _lib.FA_ERR_SCALE),
+    (dict(scale=-1.0), _lib.FA_ERR_SCALE),
+    (dict(scale=math.nan), _lib.FA_ERR_SCALE),
+    (dict(scale=math.inf), _lib.FA_ERR_SCALE),
+    (dict(causal=2), _lib.FA_ERR_ARG),
+    (dict(q=0), _lib.FA_ERR_NULL),
+    (dict(lse=0), _lib.FA_ERR_NULL),
+    (dict(o=A + 8), _lib.FA_ERR_ALIGN),
+    (dict(lse=A + 2), _lib.FA_ERR_ALIGN),
+    (dict(B=1 << 16, H=1 << 16), _lib.FA_ERR_SHAPE),
+])
+def test_invalid_arguments_rejected_before_launch(lib, args, code):
+    a = dict(q=A, k=A, v=A, o=A, lse=A, B=1, H=2, S=128, D=64, scale=0.125, causal=0, dtype=0, stream=0)
+    a.update(args)
+    st = fa.fa_fwd(a["q"], a["k"], a["v"], a["o"], a["lse"], a["B"], a["H"], a["S"], a["D"], a["scale"],
+                   a["causal"], a["dtype"], a["stream"])
+    assert st == code
+
+
+def test_empty_problem_is_a_noop(lib):
+    for B, H, S in ((0, 2, 128), (1, 0, 128), (1, 2, 0)):
+        assert fa.fa_fwd(0, 0, 0, 0, 0, B, H, S, 64, 0.125, 0, 0, 0) == _lib.FA_OK
+
+
+def test_no_device_is_reported_not_faulted(lib):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a device is present")
+    st = fa.fa_fwd(A, A, A, A, A, 1, 2, 128, 64, 0.125, 0, 0, 0)
+    assert st == _lib.FA_ERR_LAUNCH
+
+
+def test_missing_library_fails_loudly(tmp_path, monkeypatch):
+    monkeypatch.setattr(_lib, "LIB_PATH", str(tmp_path / "missing.so"))
+    monkeypatch.setattr(_lib, "_lib", None)
+    with pytest.raises(OSError):
+        _lib.load()

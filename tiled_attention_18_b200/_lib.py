@@ -1,0 +1,104 @@
+"""ctypes binding of libfa.so (include/fa.h): argument marshalling only.
+
+Every step of the attention computation runs in the CUDA kernels of
+libfa.so.  If the library is missing or cannot be loaded, every call raises:
+there is no fallback of any kind.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libfa.so")
+
+FA_FP16 = 0
+FA_BF16 = 1
+
+FA_OK = 0
+FA_ERR_NULL = -1
+FA_ERR_SHAPE = -2
+FA_ERR_HEADDIM = -3
+FA_ERR_DTYPE = -4
+FA_ERR_ALIGN = -5
+FA_ERR_ARCH = -6
+FA_ERR_LAUNCH = -7
+FA_ERR_TIMEOUT = -8
+FA_ERR_SCALE = -9
+FA_ERR_ARG = -10
+FA_ERR_PTR = -11
+
+# (name, restype, argtypes) of every symbol include/fa.h declares
+SIGNATURES = [
+    ("fa_fwd", ctypes.c_int,
+     [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+      ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_float, ctypes.c_int,
+      ctypes.c_int, ctypes.c_void_p]),
+    ("fa_check_status", ctypes.c_int, [ctypes.c_void_p]),
+    ("fa_last_timeout_site", ctypes.c_int, []),
+    ("fa_status_string", ctypes.c_char_p, [ctypes.c_int]),
+    ("fa_version", ctypes.c_int, []),
+    ("fa_num_units", ctypes.c_longlong, [ctypes.c_int, ctypes.c_int, ctypes.c_int]),
+]
+
+_lock = threading.Lock()
+_lib = None
+
+
+class FaError(RuntimeError):
+    def __init__(self, status: int, what: str = "fa_fwd"):
+        self.status = status
+        super().__init__(f"{what} failed: {status} ({status_string(status)})")
+
+
+def load() -> ctypes.CDLL:
+    """Load libfa.so (raises OSError if it is missing: build it with
+    ``python -m tiled_attention_18_b200.build``)."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        if not os.path.exists(LIB_PATH):
+            raise OSError(f"{LIB_PATH} not found; build it with `python -m tiled_attention_18_b200.build`")
+        lib = ctypes.CDLL(LIB_PATH)
+        for name, res, args in SIGNATURES:
+            fn = getattr(lib, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = lib
+        return lib
+
+
+def fa_fwd(q_ptr: int, k_ptr: int, v_ptr: int, o_ptr: int, lse_ptr: int, B: int, H: int, S: int, D: int,
+           scale: float, causal: int, dtype: int, stream: int) -> int:
+    """Raw C call: device pointers as integers, returns the fa_status code."""
+    return int(load().fa_fwd(q_ptr, k_ptr, v_ptr, o_ptr, lse_ptr, B, H, S, D, float(scale), int(causal),
+                             int(dtype), stream))
+
+
+def fa_check_status(stream: int = 0) -> int:
+    return int(load().fa_check_status(stream))
+
+
+def fa_last_timeout_site() -> int:
+    return int(load().fa_last_timeout_site())
+
+
+def fa_status_string(status: int) -> str:
+    return load().fa_status_string(int(status)).decode()
+
+
+def status_string(status: int) -> str:
+    try:
+        return fa_status_string(status)
+    except OSError:
+        return "libfa.so not loaded"
+
+
+def fa_version() -> int:
+    return int(load().fa_version())
+
+
+def fa_num_units(B: int, H: int, S: int) -> int:
+    return int(load().fa_num_units(B, H, S))

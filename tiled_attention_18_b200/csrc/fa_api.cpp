@@ -1,0 +1,200 @@
+// fa_api.cpp -- host side of libfa.so: argument validation, TMA tensor-map
+// encoding, persistent-grid sizing and the launch (declared in include/fa.h).
+//
+// The host layer plays the part of the pages' host tiling step (block sizes,
+// block counts: "FlashAttention-2 在昇腾 NPU 上如何做到 3 倍加速？" section 3.2)
+// and of the host operator entry that returns a status code (the lanjinlin.com.cn
+// page "解析CANN ops-transformer的FlashAttention算子", host Compute function),
+// except that it never synchronises the stream.
+#include "fa.h"
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <climits>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "fa_internal.h"
+
+namespace {
+
+constexpr int FA_VERSION = 100;  // 0.1.0
+
+// Per-device facts read once: compute capability and SM count.
+struct DeviceInfo {
+    bool known = false;
+    int major = 0;
+    int minor = 0;
+    int sms = 0;
+};
+
+constexpr int MAX_DEVICES = 64;
+DeviceInfo g_dev[MAX_DEVICES];
+std::mutex g_dev_mu;
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn g_encode = nullptr;
+std::once_flag g_encode_once;
+
+thread_local int t_last_site = 0;
+
+int device_info(DeviceInfo* out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= MAX_DEVICES) return FA_ERR_LAUNCH;
+    std::lock_guard<std::mutex> lock(g_dev_mu);
+    DeviceInfo& d = g_dev[dev];
+    if (!d.known) {
+        if (cudaDeviceGetAttribute(&d.major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&d.minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return FA_ERR_LAUNCH;
+        d.known = true;
+    }
+    *out = d;
+    return FA_OK;
+}
+
+EncodeTiledFn encoder() {
+    std::call_once(g_encode_once, [] {
+        void* fn = nullptr;
+        cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+    });
+    return g_encode;
+}
+
+// 3-D map over a BHSD tensor viewed as [B*H][S][D] (innermost first: D, S, B*H),
+// box {64, 128, 1}: one 128-byte-wide column chunk of 128 rows, 128-byte swizzle
+// (the swizzle atom the tcgen05 operand descriptors expect).  Rows past S read
+// as zeros and never bleed into the next head.
+bool encode_bhsd(CUtensorMap* map, const void* ptr, int BH, int S, int D, int dtype) {
+    EncodeTiledFn enc = encoder();
+    if (!enc) return false;
+    const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)S, (cuuint64_t)BH};
+    const cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)S * (cuuint64_t)D * 2};
+    const cuuint32_t box[3] = {64, (cuuint32_t)fa::BLOCK_M, 1};
+    const cuuint32_t elem[3] = {1, 1, 1};
+    const CUtensorMapDataType dt =
+        dtype == FA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    CUresult r = enc(map, dt, 3, const_cast<void*>(ptr), dims, strides, box, elem, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+int check_device_pointer(const void* p, int dev) {
+    cudaPointerAttributes attr;
+    if (cudaPointerGetAttributes(&attr, p) != cudaSuccess) {
+        cudaGetLastError();  // clear the sticky-free error of a failed query
+        return FA_ERR_PTR;
+    }
+    if (attr.type != cudaMemoryTypeDevice && attr.type != cudaMemoryTypeManaged) return FA_ERR_PTR;
+    if (attr.type == cudaMemoryTypeDevice && attr.device != dev) return FA_ERR_PTR;
+    return FA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+long long fa_num_units(int B, int H, int S) {
+    if (B < 0 || H < 0 || S < 0) return FA_ERR_SHAPE;
+    if (B == 0 || H == 0 || S == 0) return 0;
+    return (long long)fa::num_units((int64_t)B * H, S);
+}
+
+int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int S, int D,
+           float scale, int causal, int dtype, cudaStream_t stream) {
+    if (B < 0 || H < 0 || S < 0) return FA_ERR_SHAPE;
+    if (D != 64 && D != 128) return FA_ERR_HEADDIM;
+    if (dtype != FA_FP16 && dtype != FA_BF16) return FA_ERR_DTYPE;
+    if (!(std::isfinite(scale) && scale > 0.f)) return FA_ERR_SCALE;
+    if (causal != 0 && causal != 1) return FA_ERR_ARG;
+    if (B == 0 || H == 0 || S == 0) return FA_OK;  // empty problem
+    const int64_t BH = (int64_t)B * H;
+    if (BH > INT_MAX || BH * (int64_t)S > INT_MAX) return FA_ERR_SHAPE;
+    if (!q || !k || !v || !o || !lse) return FA_ERR_NULL;
+    const uintptr_t a16 = (uintptr_t)q | (uintptr_t)k | (uintptr_t)v | (uintptr_t)o;
+    if ((a16 & 15u) != 0 || ((uintptr_t)lse & 3u) != 0) return FA_ERR_ALIGN;
+
+    DeviceInfo dev;
+    int rc = device_info(&dev);
+    if (rc != FA_OK) return rc;
+    if (dev.major != 10 || dev.minor != 0) return FA_ERR_ARCH;
+    int cur = 0;
+    cudaGetDevice(&cur);
+    const void* ptrs[5] = {q, k, v, o, lse};
+    for (const void* p : ptrs) {
+        rc = check_device_pointer(p, cur);
+        if (rc != FA_OK) return rc;
+    }
+
+    fa::LaunchArgs a;
+    std::memset(&a, 0, sizeof(a));
+    if (!encode_bhsd(&a.tmap_q, q, (int)BH, S, D, dtype) || !encode_bhsd(&a.tmap_k, k, (int)BH, S, D, dtype) ||
+        !encode_bhsd(&a.tmap_v, v, (int)BH, S, D, dtype))
+        return FA_ERR_LAUNCH;
+    a.o = o;
+    a.lse = lse;
+    a.BH = (int)BH;
+    a.S = S;
+    a.D = D;
+    a.dtype = dtype;
+    a.causal = causal;
+    a.scale_log2 = (float)((double)scale * 1.4426950408889634074);  // scale * log2(e)
+    const int64_t units = fa::num_units(BH, S);
+    a.grid = (int)(units < dev.sms ? units : dev.sms);
+    if (fa::launch_fwd_sm100(a, stream) != cudaSuccess) {
+        cudaGetLastError();
+        return FA_ERR_LAUNCH;
+    }
+    if (cudaPeekAtLastError() != cudaSuccess) {
+        cudaGetLastError();
+        return FA_ERR_LAUNCH;
+    }
+    return FA_OK;
+}
+
+int fa_check_status(cudaStream_t stream) {
+    int st = 0, site = 0;
+    if (fa::read_and_clear_status(stream, &st, &site) != cudaSuccess) {
+        cudaGetLastError();
+        return FA_ERR_LAUNCH;
+    }
+    if (st != fa::DEV_OK) {
+        t_last_site = site;
+        return FA_ERR_TIMEOUT;
+    }
+    return FA_OK;
+}
+
+int fa_last_timeout_site(void) { return t_last_site; }
+
+const char* fa_status_string(int status) {
+    switch (status) {
+        case FA_OK: return "ok";
+        case FA_ERR_NULL: return "a required pointer is NULL";
+        case FA_ERR_SHAPE: return "invalid B, H or S";
+        case FA_ERR_HEADDIM: return "head dimension must be 64 or 128";
+        case FA_ERR_DTYPE: return "dtype must be FA_FP16 or FA_BF16";
+        case FA_ERR_ALIGN: return "q, k, v, o must be 16-byte aligned and lse 4-byte aligned";
+        case FA_ERR_ARCH: return "the current device is not sm_100 (B200)";
+        case FA_ERR_LAUNCH: return "CUDA runtime error";
+        case FA_ERR_TIMEOUT: return "a device-side wait exceeded its bound";
+        case FA_ERR_SCALE: return "scale must be finite and > 0";
+        case FA_ERR_ARG: return "causal must be 0 or 1";
+        case FA_ERR_PTR: return "pointer is not device memory of the current device";
+        default: return "unknown status";
+    }
+}
+
+int fa_version(void) { return FA_VERSION; }
+
+}  // extern "C"

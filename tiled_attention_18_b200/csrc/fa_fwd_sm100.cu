@@ -1,0 +1,733 @@
+// fa_fwd_sm100.cu -- fused attention forward for sm_100a (B200).
+//
+// Computes, per (b, h) and query row i,
+//   O_i   = sum_j softmax_j(scale * q_i . k_j) v_j      (j <= i when causal)
+//   LSE_i = log sum_j exp(scale * q_i . k_j)
+// tile by tile with the online-softmax recurrence (running max m, running
+// sum l), so the score matrix never reaches HBM.
+//
+// Method sources (page title, section):
+//  - tiling of Q into row blocks and K/V into column blocks, outer loop over
+//    Q tiles and inner loop over K/V tiles: "FlashAttention-2 在昇腾 NPU 上如何
+//    做到 3 倍加速？深度拆解 ops-transformer 的实现", section 2.1;
+//  - online softmax with running max and running exponential sum, and the
+//    e^{m_old - m_new} rescale of the output: same page, section 2.2;
+//  - fusion of QK^T, softmax and PV in one kernel with only O written back:
+//    same page, sections 2.3 and 3.4;
+//  - causal masking by skipping key tiles above the diagonal inside the
+//    kernel (mode 2): the gsyq.cn catlass page, "Causal Mask的实现差异";
+//  - double-buffered loads overlapping compute: "ops-transformer
+//    FlashAttention 算子实战：让昇腾NPU算力彻底释放", section 5.
+// The pages target Ascend Cube/Vector units; this kernel is a B200 design:
+//
+//  * persistent CTAs (one per SM), each owning work units of two 128-row
+//    query tiles of one (b, h); units are ordered longest-first when causal;
+//  * warp 8 is the TMA producer: Q tiles once per unit, then K_j and V_j into
+//    a ring of shared-memory slots guarded by full/empty mbarriers;
+//  * warp 9 issues tcgen05.mma (one thread): S_t = Q_t K_j^T into TMEM, and
+//    O_t += P_t V_j with P_t read from TMEM; the two query tiles ping-pong so
+//    the tensor pipe works on one tile while the other's softmax runs;
+//  * warps 0-3 and 4-7 are the softmax warpgroups of tiles 0 and 1: each
+//    thread owns one query row (one TMEM lane), reads its 128 scores, applies
+//    the diagonal/tail mask, updates m and l in the log2 domain with the
+//    scale folded into one FMA before ex2, writes P as packed 16-bit values
+//    back over the scores in TMEM, and rescales its O row only when the
+//    running max grew by more than TAU (lazy rescale); at the end of a unit it
+//    normalises O by 1/l, stores O and the LSE.
+//
+// Every mbarrier wait is bounded: after WAIT_TIMEOUT_NS the waiting thread
+// raises the CTA's abort flag and the device status word, every role leaves
+// its loop, outstanding TMA copies and MMAs are waited for (bounded), TMEM
+// is freed and the kernel returns.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "fa_internal.h"
+
+namespace fa {
+
+__device__ int g_status = 0;       // first error code, 0 if none
+__device__ int g_status_site = 0;  // (site) | (block << 8) of the first failing wait
+
+namespace {
+
+constexpr int NUM_THREADS = 320;   // 10 warps
+constexpr int WARP_TMA = 8;
+constexpr int WARP_MMA = 9;
+constexpr uint32_t TMEM_COLS = 512;
+constexpr float TAU = 8.0f;        // lazy-rescale threshold, log2 units
+constexpr uint64_t WAIT_TIMEOUT_NS = 2000000000ull;
+constexpr uint64_t DRAIN_TIMEOUT_NS = 100000000ull;
+
+// TMEM column map: S/P of tile 0 and 1, then O of tile 0 and 1.
+constexpr uint32_t COL_S0 = 0;
+constexpr uint32_t COL_S1 = 128;
+constexpr uint32_t COL_O0 = 256;
+constexpr uint32_t COL_O1 = 384;
+
+template <int D>
+struct Smem {
+    static constexpr int CHUNKS = D / 64;                  // 128-byte swizzle atoms along D
+    static constexpr int CHUNK_BYTES = 128 * 128;          // 128 rows x 128 bytes
+    static constexpr int TILE_BYTES = BLOCK_M * D * 2;     // one Q, K or V tile
+    static constexpr int NSLOT = (D == 128) ? 4 : 8;       // K/V ring depth
+    static constexpr int Q_OFF = 0;
+    static constexpr int KV_OFF = Q_OFF + Q_TILES_PER_CTA * TILE_BYTES;
+    static constexpr int BAR_OFF = KV_OFF + NSLOT * TILE_BYTES;
+    // barrier indices
+    static constexpr int B_QFULL = 0;
+    static constexpr int B_QEMPTY = 1;
+    static constexpr int B_KVFULL = 2;
+    static constexpr int B_KVEMPTY = B_KVFULL + NSLOT;
+    static constexpr int B_SFULL = B_KVEMPTY + NSLOT;      // [2]
+    static constexpr int B_PFULL = B_SFULL + 2;            // [2]
+    static constexpr int B_OFULL = B_PFULL + 2;            // [2]
+    static constexpr int B_FIN = B_OFULL + 2;
+    static constexpr int NBAR = B_FIN + 1;
+    static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;    // tmem base (u32), abort flag (u32)
+    static constexpr int BYTES = MISC_OFF + 16;
+    static constexpr int ALLOC = BYTES + 1024;             // slack for 1 KiB alignment
+};
+
+struct KParams {
+    CUtensorMap tmap_q;
+    CUtensorMap tmap_k;
+    CUtensorMap tmap_v;
+    uint8_t* o;
+    float* lse;
+    int BH;
+    int S;
+    int n_mblk;    // 256-row query blocks per head
+    int n_units;
+    int nkv;       // key tiles per head
+    int causal;
+    float scale_log2;
+};
+
+// ------------------------------------------------------------------ PTX helpers
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ uint64_t globaltimer() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+__device__ __noinline__ void record_failure(int site) {
+    if (atomicCAS(&g_status, 0, DEV_TIMEOUT) == 0) {
+        atomicExch(&g_status_site, site | (int)(blockIdx.x << 8));
+    }
+}
+
+// Wait for the phase of `bar` with the given parity.  Returns false when the
+// wait timed out (the abort flag and the status word are then set) or when
+// another role has already aborted.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile uint32_t* abort_flag,
+                                          int site) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer();
+    for (uint32_t it = 1; it < (1u << 30); ++it) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((it & 31u) == 0) {
+            if (*abort_flag) return false;
+            if (globaltimer() - t0 > WAIT_TIMEOUT_NS) break;
+        }
+    }
+    *abort_flag = 1u;
+    record_failure(site);
+    return false;
+}
+
+// Bounded wait that ignores the abort flag: used to drain in-flight copies.
+__device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity) {
+    const uint64_t t0 = globaltimer();
+    for (uint32_t it = 0; it < (1u << 24); ++it) {
+        if (mbar_try_wait(bar, parity)) return;
+        if (globaltimer() - t0 > DRAIN_TIMEOUT_NS) return;
+    }
+}
+
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, uint32_t bar, int c0,
+                                            int c1, int c2) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cta.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
+        : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+                 : "memory");
+}
+// D(tmem) (+)= A(smem desc) * B(smem desc)
+__device__ __forceinline__ void tc_mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+// D(tmem) (+)= A(tmem) * B(smem desc)
+__device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// 32 lanes x 32 consecutive 32-bit columns; thread i gets lane (base + i).
+// The wait is inside the same statement so the results are valid on return.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+          "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]),
+          "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]),
+          "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr)
+        : "memory");
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]),
+        "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]),
+        "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]),
+        "r"(r[30]), "r"(r[31])
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_wait_st() {
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+template <bool BF16>
+__device__ __forceinline__ uint32_t pack2(float lo, float hi) {
+    uint32_t r;
+    if constexpr (BF16) {
+        asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    } else {
+        asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    }
+    return r;
+}
+
+// Shared-memory matrix descriptor for a 128-byte-swizzled operand (sm_100 format:
+// start>>4 in [0,14), leading byte offset>>4 in [16,30), stride byte offset>>4
+// in [32,46), version 1 at bit 46, layout type 2 (128-byte swizzle) in [61,64)).
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+    d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+    d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+    d |= (uint64_t)1 << 46;
+    d |= (uint64_t)2 << 61;
+    return d;
+}
+
+// Instruction descriptor for kind::f16 with fp32 accumulate, M = 128.
+__host__ __device__ constexpr uint32_t make_idesc(bool bf16, int N, bool b_mn_major) {
+    return (1u << 4)                                   // D format: f32
+           | ((bf16 ? 1u : 0u) << 7)                   // A format
+           | ((bf16 ? 1u : 0u) << 10)                  // B format
+           | (0u << 15)                                // A K-major
+           | ((b_mn_major ? 1u : 0u) << 16)            // B major
+           | ((uint32_t)(N >> 3) << 17)                // N / 8
+           | ((uint32_t)(BLOCK_M >> 4) << 24);         // M / 16
+}
+
+struct Unit {
+    int bh;
+    int q0[2];   // first query row of each tile
+    int n[2];    // key tiles visited by each tile (0 = tile beyond S)
+    int N;       // key tiles streamed for the unit
+};
+
+// Work-unit order: with the causal mask, longest units first (query block
+// descending), heads innermost; without it, heads outermost so that CTAs
+// running together share one head's K/V in L2.
+__device__ __forceinline__ Unit decode_unit(const KParams& p, int u) {
+    Unit U;
+    int mb;
+    if (p.causal) {
+        mb = p.n_mblk - 1 - u / p.BH;
+        U.bh = u % p.BH;
+    } else {
+        U.bh = u / p.n_mblk;
+        mb = u % p.n_mblk;
+    }
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+        const int q0 = mb * ROWS_PER_UNIT + t * BLOCK_M;
+        U.q0[t] = q0;
+        int n = 0;
+        if (q0 < p.S) {
+            // diagonal bound: key tile j is visited iff its first key j*BLOCK_N is
+            // not after the tile's last query row q0 + BLOCK_M - 1
+            n = p.causal ? min((q0 + BLOCK_M - 1) / BLOCK_N + 1, p.nkv) : p.nkv;
+        }
+        U.n[t] = n;
+    }
+    U.N = max(U.n[0], U.n[1]);
+    return U;
+}
+
+// ------------------------------------------------------------------ roles
+
+template <int D>
+__device__ void producer_role(const KParams& p, uint8_t* smem, volatile uint32_t* abort_flag) {
+    using L = Smem<D>;
+    const uint32_t base = smem_u32(smem);
+    const uint32_t bar0 = base + L::BAR_OFF;
+    auto bar = [&](int i) { return bar0 + 8u * (uint32_t)i; };
+    int slot = 0;
+    uint32_t phase = 0;
+    uint32_t qe_phase = 0;
+    int last_fill[L::NSLOT];
+#pragma unroll
+    for (int i = 0; i < L::NSLOT; ++i) last_fill[i] = -1;
+    int last_q_fill = -1;
+    bool ok = true;
+
+    for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
+        const Unit U = decode_unit(p, u);
+        if (!mbar_wait(bar(L::B_QEMPTY), qe_phase ^ 1u, abort_flag, 1)) { ok = false; break; }
+        qe_phase ^= 1u;
+        const uint32_t qbytes = (U.n[0] > 0 ? L::TILE_BYTES : 0) + (U.n[1] > 0 ? L::TILE_BYTES : 0);
+        mbar_expect_tx(bar(L::B_QFULL), qbytes);
+        last_q_fill = (int)(qe_phase ^ 1u);  // parity of the q_full phase this fill completes
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+            if (U.n[t] == 0) continue;
+            const uint32_t dst = base + L::Q_OFF + t * L::TILE_BYTES;
+#pragma unroll
+            for (int c = 0; c < L::CHUNKS; ++c)
+                tma_load_3d(dst + c * L::CHUNK_BYTES, &p.tmap_q, bar(L::B_QFULL), c * 64, U.q0[t], U.bh);
+        }
+        for (int j = 0; j < U.N; ++j) {
+#pragma unroll
+            for (int kv = 0; kv < 2; ++kv) {
+                if (!mbar_wait(bar(L::B_KVEMPTY + slot), phase ^ 1u, abort_flag, 2)) { ok = false; break; }
+                mbar_expect_tx(bar(L::B_KVFULL + slot), L::TILE_BYTES);
+                last_fill[slot] = (int)phase;
+                const uint32_t dst = base + L::KV_OFF + slot * L::TILE_BYTES;
+                const CUtensorMap* map = kv ? &p.tmap_v : &p.tmap_k;
+#pragma unroll
+                for (int c = 0; c < L::CHUNKS; ++c)
+                    tma_load_3d(dst + c * L::CHUNK_BYTES, map, bar(L::B_KVFULL + slot), c * 64, j * BLOCK_N,
+                                U.bh);
+                if (++slot == L::NSLOT) { slot = 0; phase ^= 1u; }
+            }
+            if (!ok) break;
+        }
+    }
+    if (!ok) {
+        // drain the copies this thread issued before leaving
+        for (int i = 0; i < L::NSLOT; ++i)
+            if (last_fill[i] >= 0) mbar_drain(bar(L::B_KVFULL + i), (uint32_t)last_fill[i]);
+        if (last_q_fill >= 0) mbar_drain(bar(L::B_QFULL), (uint32_t)last_q_fill);
+    }
+}
+
+template <int D, bool BF16>
+__device__ void mma_role(const KParams& p, uint8_t* smem, uint32_t tmem, volatile uint32_t* abort_flag) {
+    using L = Smem<D>;
+    const uint32_t base = smem_u32(smem);
+    const uint32_t bar0 = base + L::BAR_OFF;
+    auto bar = [&](int i) { return bar0 + 8u * (uint32_t)i; };
+    constexpr uint32_t IDESC_S = make_idesc(BF16, BLOCK_N, false);
+    constexpr uint32_t IDESC_PV = make_idesc(BF16, D, true);
+    constexpr int KSTEPS_S = D / 16;        // QK^T: K = D
+    constexpr int KSTEPS_PV = BLOCK_N / 16; // PV: K = BLOCK_N keys
+
+    const uint32_t tm_s[2] = {tmem + COL_S0, tmem + COL_S1};
+    const uint32_t tm_o[2] = {tmem + COL_O0, tmem + COL_O1};
+    const uint32_t q_addr[2] = {base + L::Q_OFF, base + L::Q_OFF + L::TILE_BYTES};
+
+    // S_t = Q_t K^T : A = Q tile (K-major), B = K tile (K-major), 128-byte swizzle,
+    // 8-row groups 1024 bytes apart; K steps of 16 elements advance 32 bytes
+    // inside a swizzle atom and 16 KiB across the 64-column chunks.
+    auto issue_s = [&](int t, int kslot) {
+        const uint32_t k_addr = base + L::KV_OFF + kslot * L::TILE_BYTES;
+#pragma unroll
+        for (int ks = 0; ks < KSTEPS_S; ++ks) {
+            const uint32_t off = (uint32_t)((ks & 3) * 32 + (ks >> 2) * L::CHUNK_BYTES);
+            tc_mma_ss(tm_s[t], sw128_desc(q_addr[t] + off, 16, 1024), sw128_desc(k_addr + off, 16, 1024),
+                      IDESC_S, ks > 0 ? 1u : 0u);
+        }
+    };
+    // O_t += P_t V : A = P in TMEM (16-bit pairs packed per column, 8 columns per
+    // 16 keys), B = V tile read MN-major (D contiguous): 64-element chunks 16 KiB
+    // apart (leading byte offset; with D = 64 there is a single chunk and the
+    // field is unused), 8-key groups 1024 bytes apart (stride byte offset);
+    // K steps of 16 keys advance 2 KiB.
+    constexpr uint32_t V_LBO = (D == 128) ? (uint32_t)L::CHUNK_BYTES : 1024u;
+    auto issue_pv = [&](int t, int vslot, bool accumulate) {
+        const uint32_t v_addr = base + L::KV_OFF + vslot * L::TILE_BYTES;
+#pragma unroll
+        for (int ks = 0; ks < KSTEPS_PV; ++ks) {
+            tc_mma_ts(tm_o[t], tm_s[t] + (uint32_t)(ks * 8), sw128_desc(v_addr + ks * 2048, V_LBO, 1024),
+                      IDESC_PV, (accumulate || ks > 0) ? 1u : 0u);
+        }
+    };
+
+    int slot = 0;
+    uint32_t phase = 0;
+    uint32_t qf_phase = 0;
+    uint32_t p_phase[2] = {0u, 0u};
+    bool ok = true;
+
+    for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
+        const Unit U = decode_unit(p, u);
+        if (!mbar_wait(bar(L::B_QFULL), qf_phase, abort_flag, 3)) { ok = false; break; }
+        qf_phase ^= 1u;
+        tc_fence_after();
+        int vslot_prev = -1;
+        for (int j = 0; j < U.N; ++j) {
+            // ---- K_j
+            const int kslot = slot;
+            if (!mbar_wait(bar(L::B_KVFULL + kslot), phase, abort_flag, 4)) { ok = false; break; }
+            if (++slot == L::NSLOT) { slot = 0; phase ^= 1u; }
+            tc_fence_after();
+            if (j < U.n[0]) {
+                issue_s(0, kslot);
+                tc_commit(bar(L::B_SFULL + 0));
+            }
+            // ---- O_1 += P_1 V_{j-1} (tile 1 lags one step behind tile 0)
+            if (j >= 1 && j - 1 < U.n[1]) {
+                if (!mbar_wait(bar(L::B_PFULL + 1), p_phase[1], abort_flag, 5)) { ok = false; break; }
+                p_phase[1] ^= 1u;
+                tc_fence_after();
+                issue_pv(1, vslot_prev, j - 1 > 0);
+                tc_commit(bar(L::B_KVEMPTY + vslot_prev));
+                if (j - 1 == U.n[1] - 1) tc_commit(bar(L::B_OFULL + 1));
+            }
+            if (j < U.n[1]) {
+                issue_s(1, kslot);
+                tc_commit(bar(L::B_SFULL + 1));
+            }
+            tc_commit(bar(L::B_KVEMPTY + kslot));
+            if (j == U.N - 1) tc_commit(bar(L::B_QEMPTY));
+            // ---- V_j
+            const int vslot = slot;
+            if (!mbar_wait(bar(L::B_KVFULL + vslot), phase, abort_flag, 6)) { ok = false; break; }
+            if (++slot == L::NSLOT) { slot = 0; phase ^= 1u; }
+            tc_fence_after();
+            if (j < U.n[0]) {
+                if (!mbar_wait(bar(L::B_PFULL + 0), p_phase[0], abort_flag, 7)) { ok = false; break; }
+                p_phase[0] ^= 1u;
+                tc_fence_after();
+                issue_pv(0, vslot, j > 0);
+                if (j == U.n[0] - 1) tc_commit(bar(L::B_OFULL + 0));
+            }
+            if (j < U.n[1]) {
+                vslot_prev = vslot;
+            } else {
+                tc_commit(bar(L::B_KVEMPTY + vslot));
+            }
+        }
+        if (!ok) break;
+        if (U.n[1] > 0) {
+            // tail: O_1 += P_1 V_{N-1}
+            if (!mbar_wait(bar(L::B_PFULL + 1), p_phase[1], abort_flag, 8)) { ok = false; break; }
+            p_phase[1] ^= 1u;
+            tc_fence_after();
+            issue_pv(1, vslot_prev, U.N - 1 > 0);
+            tc_commit(bar(L::B_KVEMPTY + vslot_prev));
+            tc_commit(bar(L::B_OFULL + 1));
+        }
+    }
+    // all MMAs issued by this thread have completed once B_FIN fires
+    tc_commit(bar(L::B_FIN));
+    mbar_drain(bar(L::B_FIN), 0u);
+}
+
+template <int D, bool BF16>
+__device__ void softmax_role(const KParams& p, uint8_t* smem, uint32_t tmem, int t, int warp_in_group,
+                             volatile uint32_t* abort_flag) {
+    using L = Smem<D>;
+    const uint32_t base = smem_u32(smem);
+    const uint32_t bar0 = base + L::BAR_OFF;
+    auto bar = [&](int i) { return bar0 + 8u * (uint32_t)i; };
+    const int lane = threadIdx.x & 31;
+    const int row_in_tile = warp_in_group * 32 + lane;
+    const uint32_t lane_sel = (uint32_t)(warp_in_group * 32) << 16;
+    const uint32_t ts = tmem + lane_sel + (t == 0 ? COL_S0 : COL_S1);
+    const uint32_t to = tmem + lane_sel + (t == 0 ? COL_O0 : COL_O1);
+    const float sl2 = p.scale_log2;
+
+    uint32_t s_phase = 0, o_phase = 0;
+    for (int u = blockIdx.x; u < p.n_units; u += gridDim.x) {
+        const Unit U = decode_unit(p, u);
+        const int n = U.n[t];
+        if (n == 0) continue;
+        const int row = U.q0[t] + row_in_tile;
+        const int key_limit = p.causal ? min(row, p.S - 1) : p.S - 1;  // last visible key
+        float m_use = -INFINITY;  // running max in log2 units (lazy)
+        float l = 0.f;            // running sum relative to m_use
+        for (int j = 0; j < n; ++j) {
+            // the result is made warp-uniform: the TMEM accesses below need the whole warp
+            if (!__all_sync(0xffffffffu, mbar_wait(bar(L::B_SFULL + t), s_phase, abort_flag, 16 + t))) return;
+            s_phase ^= 1u;
+            tc_fence_after();
+            float s[BLOCK_N];
+#pragma unroll
+            for (int c = 0; c < BLOCK_N / 32; ++c) tmem_ld32(ts + 32 * c, s + 32 * c);
+            const int kbase = j * BLOCK_N;
+            const bool need_mask = (kbase + BLOCK_N > p.S) || (p.causal && kbase + BLOCK_N - 1 > U.q0[t]);
+            if (need_mask) {
+                const int lim = key_limit - kbase;
+#pragma unroll
+                for (int c = 0; c < BLOCK_N; ++c)
+                    if (c > lim) s[c] = -INFINITY;
+            }
+            float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
+#pragma unroll
+            for (int c = 4; c < BLOCK_N; c += 4) {
+                mx0 = fmaxf(mx0, s[c]);
+                mx1 = fmaxf(mx1, s[c + 1]);
+                mx2 = fmaxf(mx2, s[c + 2]);
+                mx3 = fmaxf(mx3, s[c + 3]);
+            }
+            const float m_blk = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
+            // lazy rescale: move the reference max only when it grew by more than TAU
+            const bool grow = m_blk > m_use + TAU;
+            float alpha = 1.f;
+            if (grow) {
+                alpha = (m_use == -INFINITY) ? 0.f : ex2(m_use - m_blk);
+                m_use = m_blk;
+                l *= alpha;
+            }
+            if (j > 0 && __any_sync(0xffffffffu, grow)) {
+                // O row *= alpha (1 for threads whose max did not move)
+#pragma unroll 1
+                for (int c = 0; c < D / 32; ++c) {
+                    float o[32];
+                    tmem_ld32(to + 32 * c, o);
+                    uint32_t w[32];
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) w[i] = __float_as_uint(o[i] * alpha);
+                    tmem_st32(to + 32 * c, w);
+                }
+            }
+            const float neg_m = (m_use == -INFINITY) ? 0.f : -m_use;
+            float l0 = 0.f, l1 = 0.f;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                uint32_t pk[32];
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const float p0 = ex2(fmaf(s[64 * h + 2 * i], sl2, neg_m));
+                    const float p1 = ex2(fmaf(s[64 * h + 2 * i + 1], sl2, neg_m));
+                    l0 += p0;
+                    l1 += p1;
+                    pk[i] = pack2<BF16>(p0, p1);
+                }
+                // P (16-bit, two per column) overwrites the first 64 columns of S
+                tmem_st32(ts + 32 * h, pk);
+            }
+            l += l0 + l1;
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(bar(L::B_PFULL + t));
+        }
+        // ---- epilogue: O = O_acc / l, LSE = (m + log2 l) ln 2
+        if (!__all_sync(0xffffffffu, mbar_wait(bar(L::B_OFULL + t), o_phase, abort_flag, 18 + t))) return;
+        o_phase ^= 1u;
+        tc_fence_after();
+        const float inv_l = 1.f / l;
+        const bool valid = row < p.S;
+        uint8_t* orow = p.o + ((size_t)U.bh * (size_t)p.S + (size_t)(valid ? row : 0)) * (size_t)(D * 2);
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+            float o[32];
+            tmem_ld32(to + 32 * c, o);
+            uint32_t w[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) w[i] = pack2<BF16>(o[2 * i] * inv_l, o[2 * i + 1] * inv_l);
+            if (valid) {
+                uint4* dst = reinterpret_cast<uint4*>(orow + c * 64);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+            }
+        }
+        if (valid) p.lse[(size_t)U.bh * (size_t)p.S + row] = (m_use + __log2f(l)) * 0.69314718055994530942f;
+        // the O reads above are ordered before the next unit's first PV by the
+        // fence + arrive of that unit's first P tile
+    }
+}
+
+template <int D, bool BF16>
+__global__ void __launch_bounds__(NUM_THREADS, 1) fa_fwd_kernel(const __grid_constant__ KParams p) {
+    using L = Smem<D>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t base = smem_u32(smem);
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    uint32_t* misc = reinterpret_cast<uint32_t*>(smem + L::MISC_OFF);
+    volatile uint32_t* abort_flag = misc + 1;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < L::NBAR; ++i) {
+            uint32_t count = 1;
+            if (i == L::B_PFULL || i == L::B_PFULL + 1) count = BLOCK_M;  // all softmax threads of a tile
+            mbar_init(base + L::BAR_OFF + 8 * i, count);
+        }
+        *abort_flag = 0u;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    }
+    if (warp == WARP_TMA && lane == 0) {
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&p.tmap_q)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&p.tmap_k)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&p.tmap_v)) : "memory");
+    }
+    if (warp == WARP_MMA) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_u32(misc)),
+                     "r"(TMEM_COLS)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = misc[0];
+
+    if (warp < 8) {
+        softmax_role<D, BF16>(p, smem, tmem, warp >> 2, warp & 3, abort_flag);
+    } else if (warp == WARP_TMA) {
+        if (lane == 0) producer_role<D>(p, smem, abort_flag);
+    } else if (warp == WARP_MMA) {
+        if (lane == 0) mma_role<D, BF16>(p, smem, tmem, abort_flag);
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == WARP_MMA) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS)
+                     : "memory");
+    }
+}
+
+template <int D, bool BF16>
+cudaError_t launch_impl(const LaunchArgs& a, cudaStream_t stream) {
+    using L = Smem<D>;
+    static_assert(L::ALLOC <= 232448, "shared memory budget exceeded");
+    auto kern = fa_fwd_kernel<D, BF16>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC);
+    if (e != cudaSuccess) return e;
+    KParams p;
+    p.tmap_q = a.tmap_q;
+    p.tmap_k = a.tmap_k;
+    p.tmap_v = a.tmap_v;
+    p.o = reinterpret_cast<uint8_t*>(a.o);
+    p.lse = a.lse;
+    p.BH = a.BH;
+    p.S = a.S;
+    p.n_mblk = (a.S + ROWS_PER_UNIT - 1) / ROWS_PER_UNIT;
+    p.n_units = (int)num_units(a.BH, a.S);
+    p.nkv = (a.S + BLOCK_N - 1) / BLOCK_N;
+    p.causal = a.causal;
+    p.scale_log2 = a.scale_log2;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)a.grid, 1, 1);
+    cfg.blockDim = dim3(NUM_THREADS, 1, 1);
+    cfg.dynamicSmemBytes = L::ALLOC;
+    cfg.stream = stream;
+    cfg.attrs = nullptr;
+    cfg.numAttrs = 0;
+    return cudaLaunchKernelEx(&cfg, kern, p);
+}
+
+}  // namespace
+
+cudaError_t launch_fwd_sm100(const LaunchArgs& a, cudaStream_t stream) {
+    if (a.D == 128) {
+        return a.dtype == 1 ? launch_impl<128, true>(a, stream) : launch_impl<128, false>(a, stream);
+    }
+    return a.dtype == 1 ? launch_impl<64, true>(a, stream) : launch_impl<64, false>(a, stream);
+}
+
+cudaError_t read_and_clear_status(cudaStream_t stream, int* status, int* site) {
+    cudaError_t e = cudaStreamSynchronize(stream);
+    if (e != cudaSuccess) return e;
+    int st = 0, si = 0;
+    e = cudaMemcpyFromSymbolAsync(&st, g_status, sizeof(int), 0, cudaMemcpyDeviceToHost, stream);
+    if (e == cudaSuccess)
+        e = cudaMemcpyFromSymbolAsync(&si, g_status_site, sizeof(int), 0, cudaMemcpyDeviceToHost, stream);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+    if (e != cudaSuccess) return e;
+    if (st != 0) {
+        const int zero = 0;
+        e = cudaMemcpyToSymbolAsync(g_status, &zero, sizeof(int), 0, cudaMemcpyHostToDevice, stream);
+        if (e == cudaSuccess)
+            e = cudaMemcpyToSymbolAsync(g_status_site, &zero, sizeof(int), 0, cudaMemcpyHostToDevice, stream);
+        if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+    }
+    *status = st;
+    *site = si;
+    return e;
+}
+
+}  // namespace fa

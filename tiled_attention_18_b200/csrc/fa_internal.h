@@ -1,0 +1,50 @@
+// fa_internal.h -- declarations shared by the host layer (fa_api.cpp) and the
+// sm_100a kernel translation unit (fa_fwd_sm100.cu).  Not part of the C ABI.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace fa {
+
+// Tile shape of the forward kernel: a CTA owns two query tiles of BLOCK_M
+// rows each and streams keys/values in tiles of BLOCK_N rows.
+constexpr int BLOCK_M = 128;
+constexpr int BLOCK_N = 128;
+constexpr int Q_TILES_PER_CTA = 2;
+constexpr int ROWS_PER_UNIT = BLOCK_M * Q_TILES_PER_CTA;
+
+// Device-side status codes written to the status word by the kernel.
+constexpr int DEV_OK = 0;
+constexpr int DEV_TIMEOUT = 1;
+
+struct LaunchArgs {
+    CUtensorMap tmap_q;     // 3-D maps over [B*H][S][D], box {64, 128, 1}, 128-byte swizzle
+    CUtensorMap tmap_k;
+    CUtensorMap tmap_v;
+    void* o;                // [B,H,S,D] 16-bit
+    float* lse;             // [B,H,S] fp32
+    int BH;
+    int S;
+    int D;
+    int dtype;              // 0 fp16, 1 bf16
+    int causal;
+    float scale_log2;       // scale * log2(e)
+    int grid;               // persistent CTAs
+};
+
+// Number of work units (b, h, 256-row query block).
+inline int64_t num_units(int64_t BH, int64_t S) {
+    return BH * ((S + ROWS_PER_UNIT - 1) / ROWS_PER_UNIT);
+}
+
+// Launch the persistent forward kernel on `stream`.  Returns a cudaError_t.
+cudaError_t launch_fwd_sm100(const LaunchArgs& a, cudaStream_t stream);
+
+// Read (after synchronising `stream`) and clear the device status word of
+// the current device.  *status receives DEV_OK or an error code; *site the
+// diagnostic word of the first failing wait.
+cudaError_t read_and_clear_status(cudaStream_t stream, int* status, int* site);
+
+}  // namespace fa
