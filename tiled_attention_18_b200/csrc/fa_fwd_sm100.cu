@@ -31,9 +31,9 @@
 //    thread owns one query row (one TMEM lane), reads its 128 scores, applies
 //    the diagonal/tail mask, updates m and l in the log2 domain with the
 //    scale folded into one FMA before ex2, writes P as packed 16-bit values
-//    back over the scores in TMEM, and rescales its O row only when the
-//    running max grew by more than TAU (lazy rescale); at the end of a unit it
-//    normalises O by 1/l, stores O and the LSE.
+//    back over the scores in TMEM, and rescales its O row when the running
+//    max grew (by more than 8 for fp16: lazy rescale; at all for bf16); at
+//    the end of a unit it normalises O by 1/l, stores O and the LSE.
 //
 // Every mbarrier wait is bounded: after WAIT_TIMEOUT_NS the waiting thread
 // raises the CTA's abort flag and the device status word, every role leaves
@@ -56,7 +56,18 @@ constexpr int NUM_THREADS = 320;   // 10 warps
 constexpr int WARP_TMA = 8;
 constexpr int WARP_MMA = 9;
 constexpr uint32_t TMEM_COLS = 512;
-constexpr float TAU = 8.0f;        // lazy-rescale threshold, log2 units
+// Rescale threshold of the running max, log2 units.  fp16 moves the reference
+// max only when it grew by more than 8 (lazy rescale; P <= 2^8 stays exact
+// enough at fp16's 11-bit precision).  bf16 (8-bit precision) keeps the exact
+// running max, so the largest weight of a row is exactly 1.0 and is not
+// rounded; with a sharp softmax that rounding would dominate the error of O.
+template <bool BF16>
+struct Policy {
+    static constexpr float TAU = BF16 ? 0.0f : 8.0f;
+    // bf16: l sums the rounded weights that the P.V product uses, so O is a
+    // convex combination of V rows (exact in the one-key limit).
+    static constexpr bool L_FROM_ROUNDED_P = BF16;
+};
 constexpr uint64_t WAIT_TIMEOUT_NS = 2000000000ull;
 constexpr uint64_t DRAIN_TIMEOUT_NS = 100000000ull;
 
@@ -218,8 +229,7 @@ __device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint
 
 // 32 lanes x 32 consecutive 32-bit columns; thread i gets lane (base + i).
 // The wait is inside the same statement so the results are valid on return.
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
-    uint32_t r[32];
+__device__ __forceinline__ void tmem_ld32u(uint32_t taddr, uint32_t (&r)[32]) {
     asm volatile(
         "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
         "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
@@ -232,6 +242,11 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
           "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
         : "r"(taddr)
         : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
+    uint32_t r[32];
+    tmem_ld32u(taddr, r);
 #pragma unroll
     for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
@@ -548,25 +563,13 @@ __device__ void softmax_role(const KParams& p, uint8_t* smem, uint32_t tmem, int
                 mx3 = fmaxf(mx3, s[c + 3]);
             }
             const float m_blk = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
-            // lazy rescale: move the reference max only when it grew by more than TAU
-            const bool grow = m_blk > m_use + TAU;
+            // move the reference max only when it grew by more than TAU
+            const bool grow = m_blk > m_use + Policy<BF16>::TAU;
             float alpha = 1.f;
             if (grow) {
                 alpha = (m_use == -INFINITY) ? 0.f : ex2(m_use - m_blk);
                 m_use = m_blk;
                 l *= alpha;
-            }
-            if (j > 0 && __any_sync(0xffffffffu, grow)) {
-                // O row *= alpha (1 for threads whose max did not move)
-#pragma unroll 1
-                for (int c = 0; c < D / 32; ++c) {
-                    float o[32];
-                    tmem_ld32(to + 32 * c, o);
-                    uint32_t w[32];
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) w[i] = __float_as_uint(o[i] * alpha);
-                    tmem_st32(to + 32 * c, w);
-                }
             }
             const float neg_m = (m_use == -INFINITY) ? 0.f : -m_use;
             float l0 = 0.f, l1 = 0.f;
@@ -577,14 +580,31 @@ __device__ void softmax_role(const KParams& p, uint8_t* smem, uint32_t tmem, int
                 for (int i = 0; i < 32; ++i) {
                     const float p0 = ex2(fmaf(s[64 * h + 2 * i], sl2, neg_m));
                     const float p1 = ex2(fmaf(s[64 * h + 2 * i + 1], sl2, neg_m));
-                    l0 += p0;
-                    l1 += p1;
                     pk[i] = pack2<BF16>(p0, p1);
+                    if constexpr (Policy<BF16>::L_FROM_ROUNDED_P) {
+                        l0 += __uint_as_float(pk[i] << 16);          // bf16 -> fp32 is exact
+                        l1 += __uint_as_float(pk[i] & 0xFFFF0000u);
+                    } else {
+                        l0 += p0;
+                        l1 += p1;
+                    }
                 }
                 // P (16-bit, two per column) overwrites the first 64 columns of S
                 tmem_st32(ts + 32 * h, pk);
             }
             l += l0 + l1;
+            if (j > 0 && __any_sync(0xffffffffu, grow)) {
+                // O row *= alpha (1 for threads whose max did not move); done after
+                // the scores are dead, before the P tile is published
+#pragma unroll 1
+                for (int c = 0; c < D / 32; ++c) {
+                    uint32_t r[32];
+                    tmem_ld32u(to + 32 * c, r);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+                    tmem_st32(to + 32 * c, r);
+                }
+            }
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(bar(L::B_PFULL + t));
