@@ -64,9 +64,11 @@ constexpr uint32_t TMEM_COLS = 512;
 template <bool BF16>
 struct Policy {
     static constexpr float TAU = BF16 ? 0.0f : 8.0f;
-    // bf16: l sums the rounded weights that the P.V product uses, so O is a
-    // convex combination of V rows (exact in the one-key limit).
-    static constexpr bool L_FROM_ROUNDED_P = BF16;
+    // bf16: O is normalised by the sum of the rounded weights that the P.V
+    // product uses (a second sum, lr), so O is a convex combination of V rows
+    // (exact in the one-key limit); the LSE keeps the fp32 sum l, whose
+    // rounding-free value the log needs on rows with few keys.
+    static constexpr bool NORM_BY_ROUNDED_P = BF16;
 };
 constexpr uint64_t WAIT_TIMEOUT_NS = 2000000000ull;
 constexpr uint64_t DRAIN_TIMEOUT_NS = 100000000ull;
@@ -536,8 +538,9 @@ __device__ void softmax_role(const KParams& p, uint8_t* smem, uint32_t tmem, int
         if (n == 0) continue;
         const int row = U.q0[t] + row_in_tile;
         const int key_limit = p.causal ? min(row, p.S - 1) : p.S - 1;  // last visible key
-        float m_use = -INFINITY;  // running max in log2 units (lazy)
-        float l = 0.f;            // running sum relative to m_use
+        float m_use = -INFINITY;  // reference max in log2 units
+        float l = 0.f;            // running sum of the weights relative to m_use (fp32)
+        float lr = 0.f;           // the same sum over the weights as rounded for P.V
         for (int j = 0; j < n; ++j) {
             // the result is made warp-uniform: the TMEM accesses below need the whole warp
             if (!__all_sync(0xffffffffu, mbar_wait(bar(L::B_SFULL + t), s_phase, abort_flag, 16 + t))) return;
@@ -570,9 +573,10 @@ __device__ void softmax_role(const KParams& p, uint8_t* smem, uint32_t tmem, int
                 alpha = (m_use == -INFINITY) ? 0.f : ex2(m_use - m_blk);
                 m_use = m_blk;
                 l *= alpha;
+                lr *= alpha;
             }
             const float neg_m = (m_use == -INFINITY) ? 0.f : -m_use;
-            float l0 = 0.f, l1 = 0.f;
+            float l0 = 0.f, l1 = 0.f, r0 = 0.f, r1 = 0.f;
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
                 uint32_t pk[32];
@@ -581,18 +585,18 @@ __device__ void softmax_role(const KParams& p, uint8_t* smem, uint32_t tmem, int
                     const float p0 = ex2(fmaf(s[64 * h + 2 * i], sl2, neg_m));
                     const float p1 = ex2(fmaf(s[64 * h + 2 * i + 1], sl2, neg_m));
                     pk[i] = pack2<BF16>(p0, p1);
-                    if constexpr (Policy<BF16>::L_FROM_ROUNDED_P) {
-                        l0 += __uint_as_float(pk[i] << 16);          // bf16 -> fp32 is exact
-                        l1 += __uint_as_float(pk[i] & 0xFFFF0000u);
-                    } else {
-                        l0 += p0;
-                        l1 += p1;
+                    l0 += p0;
+                    l1 += p1;
+                    if constexpr (Policy<BF16>::NORM_BY_ROUNDED_P) {
+                        r0 += __uint_as_float(pk[i] << 16);          // bf16 -> fp32 is exact
+                        r1 += __uint_as_float(pk[i] & 0xFFFF0000u);
                     }
                 }
                 // P (16-bit, two per column) overwrites the first 64 columns of S
                 tmem_st32(ts + 32 * h, pk);
             }
             l += l0 + l1;
+            lr += r0 + r1;
             if (j > 0 && __any_sync(0xffffffffu, grow)) {
                 // O row *= alpha (1 for threads whose max did not move); done after
                 // the scores are dead, before the P tile is published
@@ -613,7 +617,7 @@ __device__ void softmax_role(const KParams& p, uint8_t* smem, uint32_t tmem, int
         if (!__all_sync(0xffffffffu, mbar_wait(bar(L::B_OFULL + t), o_phase, abort_flag, 18 + t))) return;
         o_phase ^= 1u;
         tc_fence_after();
-        const float inv_l = 1.f / l;
+        const float inv_l = 1.f / (Policy<BF16>::NORM_BY_ROUNDED_P ? lr : l);
         const bool valid = row < p.S;
         uint8_t* orow = p.o + ((size_t)U.bh * (size_t)p.S + (size_t)(valid ? row : 0)) * (size_t)(D * 2);
 #pragma unroll 1
