@@ -14,26 +14,33 @@
 //    e^{m_old - m_new} rescale of the output: same page, section 2.2;
 //  - fusion of QK^T, softmax and PV in one kernel with only O written back:
 //    same page, sections 2.3 and 3.4;
+//  - the matrix unit and the vector unit working on different blocks at the
+//    same time (Cube/Vector pipelining): same page, sections 3.4 and 7.1;
 //  - causal masking by skipping key tiles above the diagonal inside the
 //    kernel (mode 2): the gsyq.cn catlass page, "Causal Mask的实现差异";
 //  - double-buffered loads overlapping compute: "ops-transformer
 //    FlashAttention 算子实战：让昇腾NPU算力彻底释放", section 5.
-// The pages target Ascend Cube/Vector units; this kernel is a B200 design:
+// The pages target Ascend Cube/Vector units; this kernel is a B200 design.
+// One persistent CTA per SM, 16 warps in four warpgroups:
 //
-//  * persistent CTAs (one per SM), each owning work units of two 128-row
-//    query tiles of one (b, h); units are ordered longest-first when causal;
-//  * warp 8 is the TMA producer: Q tiles once per unit, then K_j and V_j into
-//    a ring of shared-memory slots guarded by full/empty mbarriers;
-//  * warp 9 issues tcgen05.mma (one thread): S_t = Q_t K_j^T into TMEM, and
-//    O_t += P_t V_j with P_t read from TMEM; the two query tiles ping-pong so
-//    the tensor pipe works on one tile while the other's softmax runs;
-//  * warps 0-3 and 4-7 are the softmax warpgroups of tiles 0 and 1: each
-//    thread owns one query row (one TMEM lane), reads its 128 scores, applies
-//    the diagonal/tail mask, updates m and l in the log2 domain with the
-//    scale folded into one FMA before ex2, writes P as packed 16-bit values
-//    back over the scores in TMEM, and rescales its O row when the running
-//    max grew (by more than 8 for fp16: lazy rescale; at all for bf16); at
-//    the end of a unit it normalises O by 1/l, stores O and the LSE.
+//  * warpgroups 0 and 1 (softmax): one per 128-row query tile of the unit;
+//    each thread owns one query row (one TMEM lane). It reads its 128 scores,
+//    applies the diagonal/tail mask, updates the running max in the log2
+//    domain, hands the rescale factor of its O row to the correction
+//    warpgroup, computes the weights with the scale folded into one packed
+//    FMA before ex2, writes P as packed 16-bit pairs back over the scores in
+//    TMEM, and keeps the row sums.
+//  * warpgroup 2 (correction): rescales O rows in TMEM when a row's reference
+//    max moved (off the softmax's path), and runs the epilogue: O / l to
+//    16 bits, O and LSE stores.
+//  * warpgroup 3: warp 12 issues tcgen05.mma from one thread (S_t = Q_t K_j^T
+//    into TMEM; O_t += P_t V_j with P_t read from TMEM), warp 13 is the TMA
+//    producer (Q tiles once per unit, K_j and V_j through a ring of
+//    shared-memory slots with full/empty mbarriers), warps 14-15 idle.
+//    The two query tiles ping-pong: the tensor pipe works on one tile while
+//    the other tile's softmax runs.
+//  Registers are rebalanced with setmaxnreg: 184 for the softmax
+//  warpgroups, 88 for correction, 56 for warpgroup 3.
 //
 // Every mbarrier wait is bounded: after WAIT_TIMEOUT_NS the waiting thread
 // raises the CTA's abort flag and the device status word, every role leaves
@@ -52,10 +59,23 @@ __device__ int g_status_site = 0;  // (site) | (block << 8) of the first failing
 
 namespace {
 
-constexpr int NUM_THREADS = 320;   // 10 warps
-constexpr int WARP_TMA = 8;
-constexpr int WARP_MMA = 9;
+constexpr int NUM_THREADS = 512;   // 16 warps
+constexpr int WARP_MMA = 12;
+constexpr int WARP_TMA = 13;
+constexpr int REG_LAUNCH = 128;    // 65536 registers / 512 threads
+constexpr int REG_SOFTMAX = 184;
+constexpr int REG_CORR = 88;
+constexpr int REG_CTRL = 56;
+// setmaxnreg.inc waits until the registers are free: the split must fit the
+// launch allocation, and each SM sub-partition (one warp of every warpgroup).
+static_assert(2 * 128 * REG_SOFTMAX + 128 * REG_CORR + 128 * REG_CTRL <= NUM_THREADS * REG_LAUNCH,
+              "register split exceeds the launch allocation");
+static_assert(2 * REG_SOFTMAX + REG_CORR + REG_CTRL <= 512, "register split exceeds a sub-partition");
+
 constexpr uint32_t TMEM_COLS = 512;
+constexpr uint64_t WAIT_TIMEOUT_NS = 2000000000ull;
+constexpr uint64_t DRAIN_TIMEOUT_NS = 100000000ull;
+
 // Rescale threshold of the running max, log2 units.  fp16 moves the reference
 // max only when it grew by more than 8 (lazy rescale; P <= 2^8 stays exact
 // enough at fp16's 11-bit precision).  bf16 (8-bit precision) keeps the exact
@@ -70,8 +90,6 @@ struct Policy {
     // rounding-free value the log needs on rows with few keys.
     static constexpr bool NORM_BY_ROUNDED_P = BF16;
 };
-constexpr uint64_t WAIT_TIMEOUT_NS = 2000000000ull;
-constexpr uint64_t DRAIN_TIMEOUT_NS = 100000000ull;
 
 // TMEM column map: S/P of tile 0 and 1, then O of tile 0 and 1.
 constexpr uint32_t COL_S0 = 0;
@@ -87,16 +105,27 @@ struct Smem {
     static constexpr int NSLOT = (D == 128) ? 4 : 8;       // K/V ring depth
     static constexpr int Q_OFF = 0;
     static constexpr int KV_OFF = Q_OFF + Q_TILES_PER_CTA * TILE_BYTES;
-    static constexpr int BAR_OFF = KV_OFF + NSLOT * TILE_BYTES;
+    // per-row values handed from the softmax to the correction warpgroup
+    static constexpr int ALPHA_OFF = KV_OFF + NSLOT * TILE_BYTES;   // float [2][128]
+    // float2 [unit parity][tile][row] = (1/l, lse); double-buffered because a
+    // softmax warpgroup can finish the next unit before the epilogue of this
+    // one has read its values (never two units ahead: the unit after next
+    // needs this epilogue's O_t to have been read out)
+    static constexpr int FIN_OFF = ALPHA_OFF + 2 * BLOCK_M * 4;
+    static constexpr int BAR_OFF = FIN_OFF + 2 * 2 * BLOCK_M * 8;
     // barrier indices
     static constexpr int B_QFULL = 0;
     static constexpr int B_QEMPTY = 1;
     static constexpr int B_KVFULL = 2;
     static constexpr int B_KVEMPTY = B_KVFULL + NSLOT;
-    static constexpr int B_SFULL = B_KVEMPTY + NSLOT;      // [2]
-    static constexpr int B_PFULL = B_SFULL + 2;            // [2]
-    static constexpr int B_OFULL = B_PFULL + 2;            // [2]
-    static constexpr int B_FIN = B_OFULL + 2;
+    static constexpr int B_SFULL = B_KVEMPTY + NSLOT;      // [2] MMA -> softmax: S_t ready
+    static constexpr int B_PFULL = B_SFULL + 2;            // [2] softmax -> MMA: P_t ready
+    static constexpr int B_OFULL = B_PFULL + 2;            // [2] MMA -> correction: last O_t ready
+    static constexpr int B_STATS = B_OFULL + 2;            // [2] softmax -> correction: alpha ready
+    static constexpr int B_CORR = B_STATS + 2;             // [2] correction -> MMA: O_t rescaled
+    static constexpr int B_FINAL = B_CORR + 2;             // [parity][2] softmax -> correction: 1/l, lse ready
+    static constexpr int B_OFREE = B_FINAL + 4;            // [2] correction -> MMA: O_t read out
+    static constexpr int B_FIN = B_OFREE + 2;
     static constexpr int NBAR = B_FIN + 1;
     static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;    // tmem base (u32), abort flag (u32)
     static constexpr int BYTES = MISC_OFF + 16;
@@ -311,6 +340,21 @@ __host__ __device__ constexpr uint32_t make_idesc(bool bf16, int N, bool b_mn_ma
            | ((uint32_t)(BLOCK_M >> 4) << 24);         // M / 16
 }
 
+template <int N>
+__device__ __forceinline__ void setmaxnreg_inc() {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void setmaxnreg_dec() {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
+__device__ __forceinline__ float max3(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
 struct Unit {
     int bh;
     int q0[2];   // first query row of each tile
@@ -358,9 +402,8 @@ __device__ void producer_role(const KParams& p, uint8_t* smem, volatile uint32_t
     int slot = 0;
     uint32_t phase = 0;
     uint32_t qe_phase = 0;
-    int last_fill[L::NSLOT];
-#pragma unroll
-    for (int i = 0; i < L::NSLOT; ++i) last_fill[i] = -1;
+    uint32_t fill_mask = 0;    // slots with a fill issued
+    uint32_t fill_parity = 0;  // parity of each slot's last fill
     int last_q_fill = -1;
     bool ok = true;
 
@@ -384,7 +427,8 @@ __device__ void producer_role(const KParams& p, uint8_t* smem, volatile uint32_t
             for (int kv = 0; kv < 2; ++kv) {
                 if (!mbar_wait(bar(L::B_KVEMPTY + slot), phase ^ 1u, abort_flag, 2)) { ok = false; break; }
                 mbar_expect_tx(bar(L::B_KVFULL + slot), L::TILE_BYTES);
-                last_fill[slot] = (int)phase;
+                fill_mask |= 1u << slot;
+                fill_parity = (fill_parity & ~(1u << slot)) | (phase << slot);
                 const uint32_t dst = base + L::KV_OFF + slot * L::TILE_BYTES;
                 const CUtensorMap* map = kv ? &p.tmap_v : &p.tmap_k;
 #pragma unroll
@@ -399,7 +443,7 @@ __device__ void producer_role(const KParams& p, uint8_t* smem, volatile uint32_t
     if (!ok) {
         // drain the copies this thread issued before leaving
         for (int i = 0; i < L::NSLOT; ++i)
-            if (last_fill[i] >= 0) mbar_drain(bar(L::B_KVFULL + i), (uint32_t)last_fill[i]);
+            if (fill_mask & (1u << i)) mbar_drain(bar(L::B_KVFULL + i), (fill_parity >> i) & 1u);
         if (last_q_fill >= 0) mbar_drain(bar(L::B_QFULL), (uint32_t)last_q_fill);
     }
 }
@@ -415,20 +459,18 @@ __device__ void mma_role(const KParams& p, uint8_t* smem, uint32_t tmem, volatil
     constexpr int KSTEPS_S = D / 16;        // QK^T: K = D
     constexpr int KSTEPS_PV = BLOCK_N / 16; // PV: K = BLOCK_N keys
 
-    const uint32_t tm_s[2] = {tmem + COL_S0, tmem + COL_S1};
-    const uint32_t tm_o[2] = {tmem + COL_O0, tmem + COL_O1};
-    const uint32_t q_addr[2] = {base + L::Q_OFF, base + L::Q_OFF + L::TILE_BYTES};
-
     // S_t = Q_t K^T : A = Q tile (K-major), B = K tile (K-major), 128-byte swizzle,
     // 8-row groups 1024 bytes apart; K steps of 16 elements advance 32 bytes
     // inside a swizzle atom and 16 KiB across the 64-column chunks.
     auto issue_s = [&](int t, int kslot) {
+        const uint32_t q_addr = base + L::Q_OFF + (uint32_t)t * L::TILE_BYTES;
         const uint32_t k_addr = base + L::KV_OFF + kslot * L::TILE_BYTES;
+        const uint32_t d_tmem = tmem + (t == 0 ? COL_S0 : COL_S1);
 #pragma unroll
         for (int ks = 0; ks < KSTEPS_S; ++ks) {
             const uint32_t off = (uint32_t)((ks & 3) * 32 + (ks >> 2) * L::CHUNK_BYTES);
-            tc_mma_ss(tm_s[t], sw128_desc(q_addr[t] + off, 16, 1024), sw128_desc(k_addr + off, 16, 1024),
-                      IDESC_S, ks > 0 ? 1u : 0u);
+            tc_mma_ss(d_tmem, sw128_desc(q_addr + off, 16, 1024), sw128_desc(k_addr + off, 16, 1024), IDESC_S,
+                      ks > 0 ? 1u : 0u);
         }
     };
     // O_t += P_t V : A = P in TMEM (16-bit pairs packed per column, 8 columns per
@@ -439,10 +481,12 @@ __device__ void mma_role(const KParams& p, uint8_t* smem, uint32_t tmem, volatil
     constexpr uint32_t V_LBO = (D == 128) ? (uint32_t)L::CHUNK_BYTES : 1024u;
     auto issue_pv = [&](int t, int vslot, bool accumulate) {
         const uint32_t v_addr = base + L::KV_OFF + vslot * L::TILE_BYTES;
+        const uint32_t a_tmem = tmem + (t == 0 ? COL_S0 : COL_S1);
+        const uint32_t d_tmem = tmem + (t == 0 ? COL_O0 : COL_O1);
 #pragma unroll
         for (int ks = 0; ks < KSTEPS_PV; ++ks) {
-            tc_mma_ts(tm_o[t], tm_s[t] + (uint32_t)(ks * 8), sw128_desc(v_addr + ks * 2048, V_LBO, 1024),
-                      IDESC_PV, (accumulate || ks > 0) ? 1u : 0u);
+            tc_mma_ts(d_tmem, a_tmem + (uint32_t)(ks * 8), sw128_desc(v_addr + ks * 2048, V_LBO, 1024), IDESC_PV,
+                      (accumulate || ks > 0) ? 1u : 0u);
         }
     };
 
@@ -450,7 +494,29 @@ __device__ void mma_role(const KParams& p, uint8_t* smem, uint32_t tmem, volatil
     uint32_t phase = 0;
     uint32_t qf_phase = 0;
     uint32_t p_phase[2] = {0u, 0u};
+    uint32_t c_phase[2] = {0u, 0u};
+    uint32_t of_phase[2] = {0u, 0u};
+    bool o_used[2] = {false, false};
     bool ok = true;
+
+    // Wait for what PV_t of key tile j needs besides V: P_t, the O_t rescale
+    // (j > 0), or the previous unit's epilogue having read O_t (j == 0).
+    auto wait_pv_inputs = [&](int t, int j, int site) -> bool {
+        if (!mbar_wait(bar(L::B_PFULL + t), p_phase[t], abort_flag, site)) return false;
+        p_phase[t] ^= 1u;
+        if (j > 0) {
+            if (!mbar_wait(bar(L::B_CORR + t), c_phase[t], abort_flag, site + 1)) return false;
+            c_phase[t] ^= 1u;
+        } else {
+            if (o_used[t]) {
+                if (!mbar_wait(bar(L::B_OFREE + t), of_phase[t], abort_flag, site + 2)) return false;
+                of_phase[t] ^= 1u;
+            }
+            o_used[t] = true;
+        }
+        tc_fence_after();
+        return true;
+    };
 
     for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
         const Unit U = decode_unit(p, u);
@@ -470,12 +536,9 @@ __device__ void mma_role(const KParams& p, uint8_t* smem, uint32_t tmem, volatil
             }
             // ---- O_1 += P_1 V_{j-1} (tile 1 lags one step behind tile 0)
             if (j >= 1 && j - 1 < U.n[1]) {
-                if (!mbar_wait(bar(L::B_PFULL + 1), p_phase[1], abort_flag, 5)) { ok = false; break; }
-                p_phase[1] ^= 1u;
-                tc_fence_after();
+                if (!wait_pv_inputs(1, j - 1, 5)) { ok = false; break; }
                 issue_pv(1, vslot_prev, j - 1 > 0);
                 tc_commit(bar(L::B_KVEMPTY + vslot_prev));
-                if (j - 1 == U.n[1] - 1) tc_commit(bar(L::B_OFULL + 1));
             }
             if (j < U.n[1]) {
                 issue_s(1, kslot);
@@ -485,13 +548,11 @@ __device__ void mma_role(const KParams& p, uint8_t* smem, uint32_t tmem, volatil
             if (j == U.N - 1) tc_commit(bar(L::B_QEMPTY));
             // ---- V_j
             const int vslot = slot;
-            if (!mbar_wait(bar(L::B_KVFULL + vslot), phase, abort_flag, 6)) { ok = false; break; }
+            if (!mbar_wait(bar(L::B_KVFULL + vslot), phase, abort_flag, 8)) { ok = false; break; }
             if (++slot == L::NSLOT) { slot = 0; phase ^= 1u; }
             tc_fence_after();
             if (j < U.n[0]) {
-                if (!mbar_wait(bar(L::B_PFULL + 0), p_phase[0], abort_flag, 7)) { ok = false; break; }
-                p_phase[0] ^= 1u;
-                tc_fence_after();
+                if (!wait_pv_inputs(0, j, 9)) { ok = false; break; }
                 issue_pv(0, vslot, j > 0);
                 if (j == U.n[0] - 1) tc_commit(bar(L::B_OFULL + 0));
             }
@@ -504,9 +565,7 @@ __device__ void mma_role(const KParams& p, uint8_t* smem, uint32_t tmem, volatil
         if (!ok) break;
         if (U.n[1] > 0) {
             // tail: O_1 += P_1 V_{N-1}
-            if (!mbar_wait(bar(L::B_PFULL + 1), p_phase[1], abort_flag, 8)) { ok = false; break; }
-            p_phase[1] ^= 1u;
-            tc_fence_after();
+            if (!wait_pv_inputs(1, U.N - 1, 12)) { ok = false; break; }
             issue_pv(1, vslot_prev, U.N - 1 > 0);
             tc_commit(bar(L::B_KVEMPTY + vslot_prev));
             tc_commit(bar(L::B_OFULL + 1));
@@ -528,10 +587,13 @@ __device__ void softmax_role(const KParams& p, uint8_t* smem, uint32_t tmem, int
     const int row_in_tile = warp_in_group * 32 + lane;
     const uint32_t lane_sel = (uint32_t)(warp_in_group * 32) << 16;
     const uint32_t ts = tmem + lane_sel + (t == 0 ? COL_S0 : COL_S1);
-    const uint32_t to = tmem + lane_sel + (t == 0 ? COL_O0 : COL_O1);
+    float* alpha_buf = reinterpret_cast<float*>(smem + L::ALPHA_OFF) + t * BLOCK_M + row_in_tile;
+    float2* fin_buf = reinterpret_cast<float2*>(smem + L::FIN_OFF) + t * BLOCK_M + row_in_tile;
+    int fin_par = 0;  // parity of this tile's active units
     const float sl2 = p.scale_log2;
+    const float2 sl2x2 = make_float2(sl2, sl2);
 
-    uint32_t s_phase = 0, o_phase = 0;
+    uint32_t s_phase = 0;
     for (int u = blockIdx.x; u < p.n_units; u += gridDim.x) {
         const Unit U = decode_unit(p, u);
         const int n = U.n[t];
@@ -557,14 +619,17 @@ __device__ void softmax_role(const KParams& p, uint8_t* smem, uint32_t tmem, int
                 for (int c = 0; c < BLOCK_N; ++c)
                     if (c > lim) s[c] = -INFINITY;
             }
-            float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
+            float mx0 = max3(s[0], s[1], s[2]), mx1 = max3(s[3], s[4], s[5]);
+            float mx2 = max3(s[6], s[7], s[8]), mx3 = max3(s[9], s[10], s[11]);
 #pragma unroll
-            for (int c = 4; c < BLOCK_N; c += 4) {
-                mx0 = fmaxf(mx0, s[c]);
-                mx1 = fmaxf(mx1, s[c + 1]);
-                mx2 = fmaxf(mx2, s[c + 2]);
-                mx3 = fmaxf(mx3, s[c + 3]);
+            for (int c = 12; c < BLOCK_N - 4; c += 8) {
+                mx0 = max3(mx0, s[c], s[c + 1]);
+                mx1 = max3(mx1, s[c + 2], s[c + 3]);
+                mx2 = max3(mx2, s[c + 4], s[c + 5]);
+                mx3 = max3(mx3, s[c + 6], s[c + 7]);
             }
+            mx0 = max3(mx0, s[BLOCK_N - 4], s[BLOCK_N - 3]);
+            mx1 = max3(mx1, s[BLOCK_N - 2], s[BLOCK_N - 1]);
             const float m_blk = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
             // move the reference max only when it grew by more than TAU
             const bool grow = m_blk > m_use + Policy<BF16>::TAU;
@@ -575,67 +640,143 @@ __device__ void softmax_role(const KParams& p, uint8_t* smem, uint32_t tmem, int
                 l *= alpha;
                 lr *= alpha;
             }
+            if (j > 0) {
+                // the correction warpgroup rescales this O row by alpha before P.V
+                *alpha_buf = alpha;
+                mbar_arrive(bar(L::B_STATS + t));
+            }
             const float neg_m = (m_use == -INFINITY) ? 0.f : -m_use;
-            float l0 = 0.f, l1 = 0.f, r0 = 0.f, r1 = 0.f;
+            const float2 negm2 = make_float2(neg_m, neg_m);
+            float2 lsum0 = make_float2(0.f, 0.f), lsum1 = make_float2(0.f, 0.f);
+            float2 rsum0 = make_float2(0.f, 0.f), rsum1 = make_float2(0.f, 0.f);
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
                 uint32_t pk[32];
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
-                    const float p0 = ex2(fmaf(s[64 * h + 2 * i], sl2, neg_m));
-                    const float p1 = ex2(fmaf(s[64 * h + 2 * i + 1], sl2, neg_m));
-                    pk[i] = pack2<BF16>(p0, p1);
-                    l0 += p0;
-                    l1 += p1;
+                    const float2 x = __ffma2_rn(make_float2(s[64 * h + 2 * i], s[64 * h + 2 * i + 1]), sl2x2, negm2);
+                    const float2 e = make_float2(ex2(x.x), ex2(x.y));
+                    pk[i] = pack2<BF16>(e.x, e.y);
+                    if (i & 1) lsum1 = __fadd2_rn(lsum1, e); else lsum0 = __fadd2_rn(lsum0, e);
                     if constexpr (Policy<BF16>::NORM_BY_ROUNDED_P) {
-                        r0 += __uint_as_float(pk[i] << 16);          // bf16 -> fp32 is exact
-                        r1 += __uint_as_float(pk[i] & 0xFFFF0000u);
+                        // bf16 -> fp32 is exact: the rounded weights as the MMA sees them
+                        const float2 r = make_float2(__uint_as_float(pk[i] << 16), __uint_as_float(pk[i] & 0xFFFF0000u));
+                        if (i & 1) rsum1 = __fadd2_rn(rsum1, r); else rsum0 = __fadd2_rn(rsum0, r);
                     }
                 }
                 // P (16-bit, two per column) overwrites the first 64 columns of S
                 tmem_st32(ts + 32 * h, pk);
             }
-            l += l0 + l1;
-            lr += r0 + r1;
-            if (j > 0 && __any_sync(0xffffffffu, grow)) {
-                // O row *= alpha (1 for threads whose max did not move); done after
-                // the scores are dead, before the P tile is published
-#pragma unroll 1
-                for (int c = 0; c < D / 32; ++c) {
-                    uint32_t r[32];
-                    tmem_ld32u(to + 32 * c, r);
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-                    tmem_st32(to + 32 * c, r);
-                }
+            const float2 ls = __fadd2_rn(lsum0, lsum1);
+            l += ls.x + ls.y;
+            if constexpr (Policy<BF16>::NORM_BY_ROUNDED_P) {
+                const float2 rs = __fadd2_rn(rsum0, rsum1);
+                lr += rs.x + rs.y;
             }
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(bar(L::B_PFULL + t));
         }
-        // ---- epilogue: O = O_acc / l, LSE = (m + log2 l) ln 2
-        if (!__all_sync(0xffffffffu, mbar_wait(bar(L::B_OFULL + t), o_phase, abort_flag, 18 + t))) return;
-        o_phase ^= 1u;
+        // final statistics for the epilogue: 1/l for O, LSE = (m + log2 l) ln 2
+        const float norm = Policy<BF16>::NORM_BY_ROUNDED_P ? lr : l;
+        fin_buf[fin_par * 2 * BLOCK_M] = make_float2(1.f / norm, (m_use + __log2f(l)) * 0.69314718055994530942f);
+        mbar_arrive(bar(L::B_FINAL + 2 * fin_par + t));
+        fin_par ^= 1;
+    }
+}
+
+template <int D, bool BF16>
+__device__ void correction_role(const KParams& p, uint8_t* smem, uint32_t tmem, int warp_in_group,
+                                volatile uint32_t* abort_flag) {
+    using L = Smem<D>;
+    const uint32_t base = smem_u32(smem);
+    const uint32_t bar0 = base + L::BAR_OFF;
+    auto bar = [&](int i) { return bar0 + 8u * (uint32_t)i; };
+    const int lane = threadIdx.x & 31;
+    const int row_in_tile = warp_in_group * 32 + lane;
+    const uint32_t lane_sel = (uint32_t)(warp_in_group * 32) << 16;
+    const float* alpha_buf = reinterpret_cast<const float*>(smem + L::ALPHA_OFF);
+    const float2* fin_buf = reinterpret_cast<const float2*>(smem + L::FIN_OFF);
+    uint32_t st_phase[2] = {0u, 0u}, of_phase[2] = {0u, 0u};
+    uint32_t fi_phase[2][2] = {{0u, 0u}, {0u, 0u}};  // [unit parity][tile]
+    int fin_par[2] = {0, 0};
+
+    // O_t row *= alpha for iteration j of tile t (warp-uniform skip when all alpha == 1)
+    auto correct = [&](int t) -> bool {
+        if (!__all_sync(0xffffffffu, mbar_wait(bar(L::B_STATS + t), st_phase[t], abort_flag, 24 + t)))
+            return false;
+        st_phase[t] ^= 1u;
+        const float alpha = alpha_buf[t * BLOCK_M + row_in_tile];
+        if (__any_sync(0xffffffffu, alpha != 1.f)) {
+            tc_fence_after();
+            const uint32_t to = tmem + lane_sel + (t == 0 ? COL_O0 : COL_O1);
+#pragma unroll 1
+            for (int c = 0; c < D / 32; ++c) {
+                uint32_t r[32];
+                tmem_ld32u(to + 32 * c, r);
+#pragma unroll
+                for (int i = 0; i < 32; i += 2) {
+                    const float2 v = __fmul2_rn(make_float2(__uint_as_float(r[i]), __uint_as_float(r[i + 1])),
+                                                make_float2(alpha, alpha));
+                    r[i] = __float_as_uint(v.x);
+                    r[i + 1] = __float_as_uint(v.y);
+                }
+                tmem_st32(to + 32 * c, r);
+            }
+            tmem_wait_st();
+        }
+        tc_fence_before();
+        mbar_arrive(bar(L::B_CORR + t));
+        return true;
+    };
+
+    // O_t / l -> 16 bits -> global, LSE -> global; then O_t is free for the next unit
+    auto epilogue = [&](const Unit& U, int t) -> bool {
+        const int fp = fin_par[t];
+        if (!__all_sync(0xffffffffu, mbar_wait(bar(L::B_FINAL + 2 * fp + t), fi_phase[fp][t], abort_flag, 26 + t)))
+            return false;
+        fi_phase[fp][t] ^= 1u;
+        fin_par[t] ^= 1;
+        if (!__all_sync(0xffffffffu, mbar_wait(bar(L::B_OFULL + t), of_phase[t], abort_flag, 28 + t)))
+            return false;
+        of_phase[t] ^= 1u;
         tc_fence_after();
-        const float inv_l = 1.f / (Policy<BF16>::NORM_BY_ROUNDED_P ? lr : l);
+        const float2 fin = fin_buf[(fp * 2 + t) * BLOCK_M + row_in_tile];
+        const int row = U.q0[t] + row_in_tile;
         const bool valid = row < p.S;
         uint8_t* orow = p.o + ((size_t)U.bh * (size_t)p.S + (size_t)(valid ? row : 0)) * (size_t)(D * 2);
+        const uint32_t to = tmem + lane_sel + (t == 0 ? COL_O0 : COL_O1);
+        const float2 inv2 = make_float2(fin.x, fin.x);
 #pragma unroll 1
         for (int c = 0; c < D / 32; ++c) {
-            float o[32];
-            tmem_ld32(to + 32 * c, o);
+            uint32_t r[32];
+            tmem_ld32u(to + 32 * c, r);
             uint32_t w[16];
 #pragma unroll
-            for (int i = 0; i < 16; ++i) w[i] = pack2<BF16>(o[2 * i] * inv_l, o[2 * i + 1] * inv_l);
+            for (int i = 0; i < 16; ++i) {
+                const float2 v = __fmul2_rn(make_float2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1])), inv2);
+                w[i] = pack2<BF16>(v.x, v.y);
+            }
             if (valid) {
                 uint4* dst = reinterpret_cast<uint4*>(orow + c * 64);
 #pragma unroll
                 for (int i = 0; i < 4; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
             }
         }
-        if (valid) p.lse[(size_t)U.bh * (size_t)p.S + row] = (m_use + __log2f(l)) * 0.69314718055994530942f;
-        // the O reads above are ordered before the next unit's first PV by the
-        // fence + arrive of that unit's first P tile
+        if (valid) p.lse[(size_t)U.bh * (size_t)p.S + row] = fin.y;
+        tc_fence_before();
+        mbar_arrive(bar(L::B_OFREE + t));
+        return true;
+    };
+
+    for (int u = blockIdx.x; u < p.n_units; u += gridDim.x) {
+        const Unit U = decode_unit(p, u);
+        for (int j = 1; j < U.N; ++j) {
+            if (j < U.n[0] && !correct(0)) return;
+            if (j < U.n[1] && !correct(1)) return;
+        }
+        if (U.n[0] > 0 && !epilogue(U, 0)) return;
+        if (U.n[1] > 0 && !epilogue(U, 1)) return;
     }
 }
 
@@ -647,13 +788,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) fa_fwd_kernel(const __grid_con
     const uint32_t base = smem_u32(smem);
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
+    const int wg = warp >> 2;
     uint32_t* misc = reinterpret_cast<uint32_t*>(smem + L::MISC_OFF);
     volatile uint32_t* abort_flag = misc + 1;
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < L::NBAR; ++i) {
-            uint32_t count = 1;
-            if (i == L::B_PFULL || i == L::B_PFULL + 1) count = BLOCK_M;  // all softmax threads of a tile
+            uint32_t count = 1;  // TMA transaction or tcgen05.commit arrivals
+            if ((i >= L::B_PFULL && i < L::B_PFULL + 2) || (i >= L::B_STATS && i < L::B_STATS + 2) ||
+                (i >= L::B_CORR && i < L::B_CORR + 2) || (i >= L::B_FINAL && i < L::B_FINAL + 4) ||
+                (i >= L::B_OFREE && i < L::B_OFREE + 2))
+                count = BLOCK_M;  // one arrival per thread of a 128-thread warpgroup
             mbar_init(base + L::BAR_OFF + 8 * i, count);
         }
         *abort_flag = 0u;
@@ -666,8 +811,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) fa_fwd_kernel(const __grid_con
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&p.tmap_v)) : "memory");
     }
     if (warp == WARP_MMA) {
-        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                         smem_u32(misc)),
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(misc)),
                      "r"(TMEM_COLS)
                      : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
@@ -677,12 +821,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) fa_fwd_kernel(const __grid_con
     tc_fence_after();
     const uint32_t tmem = misc[0];
 
-    if (warp < 8) {
-        softmax_role<D, BF16>(p, smem, tmem, warp >> 2, warp & 3, abort_flag);
-    } else if (warp == WARP_TMA) {
-        if (lane == 0) producer_role<D>(p, smem, abort_flag);
-    } else if (warp == WARP_MMA) {
-        if (lane == 0) mma_role<D, BF16>(p, smem, tmem, abort_flag);
+    if (wg < 2) {
+        setmaxnreg_inc<REG_SOFTMAX>();
+        softmax_role<D, BF16>(p, smem, tmem, wg, warp & 3, abort_flag);
+    } else if (wg == 2) {
+        setmaxnreg_dec<REG_CORR>();
+        correction_role<D, BF16>(p, smem, tmem, warp & 3, abort_flag);
+    } else {
+        setmaxnreg_dec<REG_CTRL>();
+        if (warp == WARP_TMA) {
+            if (lane == 0) producer_role<D>(p, smem, abort_flag);
+        } else if (warp == WARP_MMA) {
+            if (lane == 0) mma_role<D, BF16>(p, smem, tmem, abort_flag);
+        }
     }
 
     tc_fence_before();
