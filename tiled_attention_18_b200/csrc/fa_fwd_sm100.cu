@@ -39,10 +39,10 @@
 //    shared-memory slots with full/empty mbarriers), warps 14-15 idle.
 //    The two query tiles ping-pong: the tensor pipe works on one tile while
 //    the other tile's softmax runs.
-//  Registers are rebalanced with setmaxnreg: 184 for the softmax
-//  warpgroups, 88 for correction, 56 for warpgroup 3.
+//  Registers are rebalanced with setmaxnreg: 176 for the softmax
+//  warpgroups, 88 for correction, 72 for warpgroup 3.
 //
-// Every mbarrier wait is bounded: after WAIT_TIMEOUT_NS the waiting thread
+// Every mbarrier wait is bounded: after WAIT_TIMEOUT_CYCLES the waiting thread
 // raises the CTA's abort flag and the device status word, every role leaves
 // its loop, outstanding TMA copies and MMAs are waited for (bounded), TMEM
 // is freed and the kernel returns.
@@ -63,9 +63,9 @@ constexpr int NUM_THREADS = 512;   // 16 warps
 constexpr int WARP_MMA = 12;
 constexpr int WARP_TMA = 13;
 constexpr int REG_LAUNCH = 128;    // 65536 registers / 512 threads
-constexpr int REG_SOFTMAX = 184;
+constexpr int REG_SOFTMAX = 176;
 constexpr int REG_CORR = 88;
-constexpr int REG_CTRL = 56;
+constexpr int REG_CTRL = 72;
 // setmaxnreg.inc waits until the registers are free: the split must fit the
 // launch allocation, and each SM sub-partition (one warp of every warpgroup).
 static_assert(2 * 128 * REG_SOFTMAX + 128 * REG_CORR + 128 * REG_CTRL <= NUM_THREADS * REG_LAUNCH,
@@ -73,8 +73,10 @@ static_assert(2 * 128 * REG_SOFTMAX + 128 * REG_CORR + 128 * REG_CTRL <= NUM_THR
 static_assert(2 * REG_SOFTMAX + REG_CORR + REG_CTRL <= 512, "register split exceeds a sub-partition");
 
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint64_t WAIT_TIMEOUT_NS = 2000000000ull;
-constexpr uint64_t DRAIN_TIMEOUT_NS = 100000000ull;
+// Bounds of a wait in SM clock cycles (SM clock <= 1.965 GHz): a wait gives up
+// after at least ~2 s, a drain of in-flight copies after at least ~0.1 s.
+constexpr long long WAIT_TIMEOUT_CYCLES = 4000000000ll;
+constexpr long long DRAIN_TIMEOUT_CYCLES = 200000000ll;
 
 // Rescale threshold of the running max, log2 units.  fp16 moves the reference
 // max only when it grew by more than 8 (lazy rescale; P <= 2^8 stays exact
@@ -119,13 +121,13 @@ struct Smem {
     static constexpr int B_KVFULL = 2;
     static constexpr int B_KVEMPTY = B_KVFULL + NSLOT;
     static constexpr int B_SFULL = B_KVEMPTY + NSLOT;      // [2] MMA -> softmax: S_t ready
-    static constexpr int B_PFULL = B_SFULL + 2;            // [2] softmax -> MMA: P_t ready
+    // [2] softmax + correction -> MMA: P_t written and O_t ready for it (rescaled,
+    // or read out by the previous unit's epilogue); 256 arrivals per phase
+    static constexpr int B_PFULL = B_SFULL + 2;
     static constexpr int B_OFULL = B_PFULL + 2;            // [2] MMA -> correction: last O_t ready
     static constexpr int B_STATS = B_OFULL + 2;            // [2] softmax -> correction: alpha ready
-    static constexpr int B_CORR = B_STATS + 2;             // [2] correction -> MMA: O_t rescaled
-    static constexpr int B_FINAL = B_CORR + 2;             // [parity][2] softmax -> correction: 1/l, lse ready
-    static constexpr int B_OFREE = B_FINAL + 4;            // [2] correction -> MMA: O_t read out
-    static constexpr int B_FIN = B_OFREE + 2;
+    static constexpr int B_FINAL = B_STATS + 2;            // [parity][2] softmax -> correction: 1/l, lse ready
+    static constexpr int B_FIN = B_FINAL + 4;
     static constexpr int NBAR = B_FIN + 1;
     static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;    // tmem base (u32), abort flag (u32)
     static constexpr int BYTES = MISC_OFF + 16;
@@ -153,11 +155,6 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
-__device__ __forceinline__ uint64_t globaltimer() {
-    uint64_t t;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    return t;
-}
 
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
@@ -192,16 +189,20 @@ __device__ __noinline__ void record_failure(int site) {
 
 // Wait for the phase of `bar` with the given parity.  Returns false when the
 // wait timed out (the abort flag and the status word are then set) or when
-// another role has already aborted.
+// another role has already aborted.  The deadline uses the SM cycle counter
+// (cheap to read); the common case costs only the polls themselves.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile uint32_t* abort_flag,
                                           int site) {
-    if (mbar_try_wait(bar, parity)) return true;
-    const uint64_t t0 = globaltimer();
+#pragma unroll 1
+    for (int i = 0; i < 8; ++i)
+        if (mbar_try_wait(bar, parity)) return true;
+    const long long t0 = clock64();
+#pragma unroll 1
     for (uint32_t it = 1; it < (1u << 30); ++it) {
         if (mbar_try_wait(bar, parity)) return true;
-        if ((it & 31u) == 0) {
+        if ((it & 15u) == 0) {
             if (*abort_flag) return false;
-            if (globaltimer() - t0 > WAIT_TIMEOUT_NS) break;
+            if (clock64() - t0 > WAIT_TIMEOUT_CYCLES) break;
         }
     }
     *abort_flag = 1u;
@@ -211,10 +212,10 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
 
 // Bounded wait that ignores the abort flag: used to drain in-flight copies.
 __device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity) {
-    const uint64_t t0 = globaltimer();
+    const long long t0 = clock64();
     for (uint32_t it = 0; it < (1u << 24); ++it) {
         if (mbar_try_wait(bar, parity)) return;
-        if (globaltimer() - t0 > DRAIN_TIMEOUT_NS) return;
+        if (clock64() - t0 > DRAIN_TIMEOUT_CYCLES) return;
     }
 }
 
@@ -245,6 +246,29 @@ __device__ __forceinline__ void tc_mma_ss(uint32_t d_tmem, uint64_t a_desc, uint
         "setp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
         "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+// The same with the descriptors given as 32-bit halves: the low half carries
+// the start address, so K steps are one 32-bit add each.
+__device__ __forceinline__ void tc_mma_ss2(uint32_t d_tmem, uint32_t a_lo, uint32_t a_hi, uint32_t b_lo,
+                                           uint32_t b_hi, uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t.reg .b64 a, b;\n\t"
+        "mov.b64 a, {%1, %2};\n\t"
+        "mov.b64 b, {%3, %4};\n\t"
+        "setp.ne.b32 p, %6, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %5, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_lo), "r"(a_hi), "r"(b_lo), "r"(b_hi), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+__device__ __forceinline__ void tc_mma_ts2(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_lo, uint32_t b_hi,
+                                           uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t.reg .b64 b;\n\t"
+        "mov.b64 b, {%2, %3};\n\t"
+        "setp.ne.b32 p, %5, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], b, %4, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "r"(b_lo), "r"(b_hi), "r"(idesc), "r"(accumulate)
         : "memory");
 }
 // D(tmem) (+)= A(tmem) * B(smem desc)
@@ -462,31 +486,40 @@ __device__ void mma_role(const KParams& p, uint8_t* smem, uint32_t tmem, volatil
     // S_t = Q_t K^T : A = Q tile (K-major), B = K tile (K-major), 128-byte swizzle,
     // 8-row groups 1024 bytes apart; K steps of 16 elements advance 32 bytes
     // inside a swizzle atom and 16 KiB across the 64-column chunks.
-    auto issue_s = [&](int t, int kslot) {
-        const uint32_t q_addr = base + L::Q_OFF + (uint32_t)t * L::TILE_BYTES;
-        const uint32_t k_addr = base + L::KV_OFF + kslot * L::TILE_BYTES;
-        const uint32_t d_tmem = tmem + (t == 0 ? COL_S0 : COL_S1);
-#pragma unroll
-        for (int ks = 0; ks < KSTEPS_S; ++ks) {
-            const uint32_t off = (uint32_t)((ks & 3) * 32 + (ks >> 2) * L::CHUNK_BYTES);
-            tc_mma_ss(d_tmem, sw128_desc(q_addr + off, 16, 1024), sw128_desc(k_addr + off, 16, 1024), IDESC_S,
-                      ks > 0 ? 1u : 0u);
-        }
-    };
     // O_t += P_t V : A = P in TMEM (16-bit pairs packed per column, 8 columns per
     // 16 keys), B = V tile read MN-major (D contiguous): 64-element chunks 16 KiB
     // apart (leading byte offset; with D = 64 there is a single chunk and the
     // field is unused), 8-key groups 1024 bytes apart (stride byte offset);
     // K steps of 16 keys advance 2 KiB.
+    // Descriptors are built once; a start address (< 256 KiB, 14 bits after >> 4)
+    // plus any offset used here stays inside the low half's field.
     constexpr uint32_t V_LBO = (D == 128) ? (uint32_t)L::CHUNK_BYTES : 1024u;
+    const uint64_t dq = sw128_desc(base + L::Q_OFF, 16, 1024);
+    const uint64_t dk = sw128_desc(base + L::KV_OFF, 16, 1024);
+    const uint64_t dv = sw128_desc(base + L::KV_OFF, V_LBO, 1024);
+    const uint32_t dq_lo = (uint32_t)dq, dq_hi = (uint32_t)(dq >> 32);
+    const uint32_t dk_lo = (uint32_t)dk, dk_hi = (uint32_t)(dk >> 32);
+    const uint32_t dv_lo = (uint32_t)dv, dv_hi = (uint32_t)(dv >> 32);
+    constexpr uint32_t TILE16 = (uint32_t)L::TILE_BYTES >> 4;
+
+    auto issue_s = [&](int t, int kslot) {
+        const uint32_t a_lo = dq_lo + (uint32_t)t * TILE16;
+        const uint32_t b_lo = dk_lo + (uint32_t)kslot * TILE16;
+        const uint32_t d_tmem = tmem + (t == 0 ? COL_S0 : COL_S1);
+#pragma unroll
+        for (int ks = 0; ks < KSTEPS_S; ++ks) {
+            const uint32_t off = (uint32_t)(((ks & 3) * 32 + (ks >> 2) * L::CHUNK_BYTES) >> 4);
+            tc_mma_ss2(d_tmem, a_lo + off, dq_hi, b_lo + off, dk_hi, IDESC_S, ks > 0 ? 1u : 0u);
+        }
+    };
     auto issue_pv = [&](int t, int vslot, bool accumulate) {
-        const uint32_t v_addr = base + L::KV_OFF + vslot * L::TILE_BYTES;
+        const uint32_t b_lo = dv_lo + (uint32_t)vslot * TILE16;
         const uint32_t a_tmem = tmem + (t == 0 ? COL_S0 : COL_S1);
         const uint32_t d_tmem = tmem + (t == 0 ? COL_O0 : COL_O1);
 #pragma unroll
         for (int ks = 0; ks < KSTEPS_PV; ++ks) {
-            tc_mma_ts(d_tmem, a_tmem + (uint32_t)(ks * 8), sw128_desc(v_addr + ks * 2048, V_LBO, 1024), IDESC_PV,
-                      (accumulate || ks > 0) ? 1u : 0u);
+            tc_mma_ts2(d_tmem, a_tmem + (uint32_t)(ks * 8), b_lo + (uint32_t)(ks * (2048 >> 4)), dv_hi, IDESC_PV,
+                       (accumulate || ks > 0) ? 1u : 0u);
         }
     };
 
@@ -494,27 +527,16 @@ __device__ void mma_role(const KParams& p, uint8_t* smem, uint32_t tmem, volatil
     uint32_t phase = 0;
     uint32_t qf_phase = 0;
     uint32_t p_phase[2] = {0u, 0u};
-    uint32_t c_phase[2] = {0u, 0u};
-    uint32_t of_phase[2] = {0u, 0u};
-    bool o_used[2] = {false, false};
     bool ok = true;
 
-    // Wait for what PV_t of key tile j needs besides V: P_t, the O_t rescale
-    // (j > 0), or the previous unit's epilogue having read O_t (j == 0).
-    auto wait_pv_inputs = [&](int t, int j, int site) -> bool {
+    // Wait for what PV_t needs besides V: P_t and O_t (one barrier, armed by the
+    // softmax and the correction warpgroups).  Waits of this thread queue behind
+    // its MMAs that the tensor pipe has not taken yet, so each wait point costs
+    // pipe time: the loop below has three per key tile (K, P1, V + P0).
+    auto wait_pv_inputs = [&](int t, int site) -> bool {
         if (!mbar_wait(bar(L::B_PFULL + t), p_phase[t], abort_flag, site)) return false;
         p_phase[t] ^= 1u;
-        if (j > 0) {
-            if (!mbar_wait(bar(L::B_CORR + t), c_phase[t], abort_flag, site + 1)) return false;
-            c_phase[t] ^= 1u;
-        } else {
-            if (o_used[t]) {
-                if (!mbar_wait(bar(L::B_OFREE + t), of_phase[t], abort_flag, site + 2)) return false;
-                of_phase[t] ^= 1u;
-            }
-            o_used[t] = true;
-        }
-        tc_fence_after();
+        tc_fence_after();  // P_t and O_t were written by tcgen05.st of other threads
         return true;
     };
 
@@ -522,21 +544,19 @@ __device__ void mma_role(const KParams& p, uint8_t* smem, uint32_t tmem, volatil
         const Unit U = decode_unit(p, u);
         if (!mbar_wait(bar(L::B_QFULL), qf_phase, abort_flag, 3)) { ok = false; break; }
         qf_phase ^= 1u;
-        tc_fence_after();
         int vslot_prev = -1;
         for (int j = 0; j < U.N; ++j) {
             // ---- K_j
             const int kslot = slot;
             if (!mbar_wait(bar(L::B_KVFULL + kslot), phase, abort_flag, 4)) { ok = false; break; }
             if (++slot == L::NSLOT) { slot = 0; phase ^= 1u; }
-            tc_fence_after();
             if (j < U.n[0]) {
                 issue_s(0, kslot);
                 tc_commit(bar(L::B_SFULL + 0));
             }
             // ---- O_1 += P_1 V_{j-1} (tile 1 lags one step behind tile 0)
             if (j >= 1 && j - 1 < U.n[1]) {
-                if (!wait_pv_inputs(1, j - 1, 5)) { ok = false; break; }
+                if (!wait_pv_inputs(1, 5)) { ok = false; break; }
                 issue_pv(1, vslot_prev, j - 1 > 0);
                 tc_commit(bar(L::B_KVEMPTY + vslot_prev));
             }
@@ -550,9 +570,8 @@ __device__ void mma_role(const KParams& p, uint8_t* smem, uint32_t tmem, volatil
             const int vslot = slot;
             if (!mbar_wait(bar(L::B_KVFULL + vslot), phase, abort_flag, 8)) { ok = false; break; }
             if (++slot == L::NSLOT) { slot = 0; phase ^= 1u; }
-            tc_fence_after();
             if (j < U.n[0]) {
-                if (!wait_pv_inputs(0, j, 9)) { ok = false; break; }
+                if (!wait_pv_inputs(0, 9)) { ok = false; break; }
                 issue_pv(0, vslot, j > 0);
                 if (j == U.n[0] - 1) tc_commit(bar(L::B_OFULL + 0));
             }
@@ -565,7 +584,7 @@ __device__ void mma_role(const KParams& p, uint8_t* smem, uint32_t tmem, volatil
         if (!ok) break;
         if (U.n[1] > 0) {
             // tail: O_1 += P_1 V_{N-1}
-            if (!wait_pv_inputs(1, U.N - 1, 12)) { ok = false; break; }
+            if (!wait_pv_inputs(1, 12)) { ok = false; break; }
             issue_pv(1, vslot_prev, U.N - 1 > 0);
             tc_commit(bar(L::B_KVEMPTY + vslot_prev));
             tc_commit(bar(L::B_OFULL + 1));
@@ -698,6 +717,9 @@ __device__ void correction_role(const KParams& p, uint8_t* smem, uint32_t tmem, 
     const float* alpha_buf = reinterpret_cast<const float*>(smem + L::ALPHA_OFF);
     const float2* fin_buf = reinterpret_cast<const float2*>(smem + L::FIN_OFF);
     uint32_t st_phase[2] = {0u, 0u}, of_phase[2] = {0u, 0u};
+    // O_t of the first unit needs no read-out: arm both tiles' first P barrier phase
+    mbar_arrive(bar(L::B_PFULL + 0));
+    mbar_arrive(bar(L::B_PFULL + 1));
     uint32_t fi_phase[2][2] = {{0u, 0u}, {0u, 0u}};  // [unit parity][tile]
     int fin_par[2] = {0, 0};
 
@@ -726,7 +748,7 @@ __device__ void correction_role(const KParams& p, uint8_t* smem, uint32_t tmem, 
             tmem_wait_st();
         }
         tc_fence_before();
-        mbar_arrive(bar(L::B_CORR + t));
+        mbar_arrive(bar(L::B_PFULL + t));
         return true;
     };
 
@@ -764,8 +786,9 @@ __device__ void correction_role(const KParams& p, uint8_t* smem, uint32_t tmem, 
             }
         }
         if (valid) p.lse[(size_t)U.bh * (size_t)p.S + row] = fin.y;
+        // O_t is free for the next unit's first P.V: arm that P barrier phase
         tc_fence_before();
-        mbar_arrive(bar(L::B_OFREE + t));
+        mbar_arrive(bar(L::B_PFULL + t));
         return true;
     };
 
@@ -795,10 +818,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) fa_fwd_kernel(const __grid_con
     if (threadIdx.x == 0) {
         for (int i = 0; i < L::NBAR; ++i) {
             uint32_t count = 1;  // TMA transaction or tcgen05.commit arrivals
-            if ((i >= L::B_PFULL && i < L::B_PFULL + 2) || (i >= L::B_STATS && i < L::B_STATS + 2) ||
-                (i >= L::B_CORR && i < L::B_CORR + 2) || (i >= L::B_FINAL && i < L::B_FINAL + 4) ||
-                (i >= L::B_OFREE && i < L::B_OFREE + 2))
-                count = BLOCK_M;  // one arrival per thread of a 128-thread warpgroup
+            if ((i >= L::B_STATS && i < L::B_STATS + 2) || (i >= L::B_FINAL && i < L::B_FINAL + 4))
+                count = BLOCK_M;      // one arrival per thread of a 128-thread warpgroup
+            if (i >= L::B_PFULL && i < L::B_PFULL + 2)
+                count = 2 * BLOCK_M;  // softmax and correction warpgroups
             mbar_init(base + L::BAR_OFF + 8 * i, count);
         }
         *abort_flag = 0u;
