@@ -40,7 +40,7 @@
 //    The two query tiles ping-pong: the tensor pipe works on one tile while
 //    the other tile's softmax runs.
 //  Registers are rebalanced with setmaxnreg: 176 for the softmax
-//  warpgroups, 88 for correction, 72 for warpgroup 3.
+//  warpgroups, 80 for correction, 80 for warpgroup 3.
 //
 // Every mbarrier wait is bounded: after WAIT_TIMEOUT_CYCLES the waiting thread
 // raises the CTA's abort flag and the device status word, every role leaves
@@ -64,8 +64,8 @@ constexpr int WARP_MMA = 12;
 constexpr int WARP_TMA = 13;
 constexpr int REG_LAUNCH = 128;    // 65536 registers / 512 threads
 constexpr int REG_SOFTMAX = 176;
-constexpr int REG_CORR = 88;
-constexpr int REG_CTRL = 72;
+constexpr int REG_CORR = 80;
+constexpr int REG_CTRL = 80;
 // setmaxnreg.inc waits until the registers are free: the split must fit the
 // launch allocation, and each SM sub-partition (one warp of every warpgroup).
 static_assert(2 * 128 * REG_SOFTMAX + 128 * REG_CORR + 128 * REG_CTRL <= NUM_THREADS * REG_LAUNCH,
@@ -73,19 +73,33 @@ static_assert(2 * 128 * REG_SOFTMAX + 128 * REG_CORR + 128 * REG_CTRL <= NUM_THR
 static_assert(2 * REG_SOFTMAX + REG_CORR + REG_CTRL <= 512, "register split exceeds a sub-partition");
 
 constexpr uint32_t TMEM_COLS = 512;
+// One weight pair in FMA_EXP2_PERIOD would be computed on the FMA pipe instead
+// of the MUFU (tiles without masking only); 0 disables it.  Measured on B200
+// with S = 16384, D = 128, bf16: period 0 -> 959 TFLOP/s, 4 -> 926, 2 -> 838:
+// the softmax warps are bound by instruction issue, not by the MUFU, so the
+// polynomial's extra instructions cost more than the ex2 they replace.
+constexpr int FMA_EXP2_PERIOD = 0;
 // Bounds of a wait in SM clock cycles (SM clock <= 1.965 GHz): a wait gives up
 // after at least ~2 s, a drain of in-flight copies after at least ~0.1 s.
 constexpr long long WAIT_TIMEOUT_CYCLES = 4000000000ll;
 constexpr long long DRAIN_TIMEOUT_CYCLES = 200000000ll;
 
-// Rescale threshold of the running max, log2 units.  fp16 moves the reference
-// max only when it grew by more than 8 (lazy rescale; P <= 2^8 stays exact
-// enough at fp16's 11-bit precision).  bf16 (8-bit precision) keeps the exact
-// running max, so the largest weight of a row is exactly 1.0 and is not
-// rounded; with a sharp softmax that rounding would dominate the error of O.
+// When the softmax moves a row's reference max m (log2 units) to the block max:
+//  - always when the block max exceeds m by more than TAU = 8 (weights stay
+//    <= 2^8, lazy rescale);
+//  - bf16 only: also when the block's largest weight 2^(max - m) exceeds
+//    KAPPA * l (l = the row sum so far).  Weights are rounded to bf16 (8-bit
+//    precision) before P.V, and the rounding of a row's largest weight
+//    2^d (0 < d <= 8) is what dominates the error of O when a few keys carry
+//    the row (a sharp softmax).  Moving m makes that weight exactly 1.0; when
+//    it is skipped, the weight is at most KAPPA/(1+KAPPA) of the row, so its
+//    rounding moves O by at most ~2^-9 * KAPPA * |v|.  Soft rows (large l)
+//    thus keep the lazy rescale, sharp rows the exact one.
+//  fp16 (11-bit precision) uses the lazy rule only.
 template <bool BF16>
 struct Policy {
-    static constexpr float TAU = BF16 ? 0.0f : 8.0f;
+    static constexpr float TAU = 8.0f;
+    [[maybe_unused]] static constexpr float KAPPA = 0.125f;
     // bf16: O is normalised by the sum of the rounded weights that the P.V
     // product uses (a second sum, lr), so O is a convex combination of V rows
     // (exact in the one-key limit); the LSE keeps the fp32 sum l, whose
@@ -238,18 +252,8 @@ __device__ __forceinline__ void tc_commit(uint32_t bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
                  : "memory");
 }
-// D(tmem) (+)= A(smem desc) * B(smem desc)
-__device__ __forceinline__ void tc_mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                          uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-// The same with the descriptors given as 32-bit halves: the low half carries
-// the start address, so K steps are one 32-bit add each.
+// D(tmem) (+)= A(smem desc) * B(smem desc), the descriptors given as 32-bit
+// halves: the low half carries the start address, so K steps are one 32-bit add.
 __device__ __forceinline__ void tc_mma_ss2(uint32_t d_tmem, uint32_t a_lo, uint32_t a_hi, uint32_t b_lo,
                                            uint32_t b_hi, uint32_t idesc, uint32_t accumulate) {
     asm volatile(
@@ -261,6 +265,7 @@ __device__ __forceinline__ void tc_mma_ss2(uint32_t d_tmem, uint32_t a_lo, uint3
         "r"(a_lo), "r"(a_hi), "r"(b_lo), "r"(b_hi), "r"(idesc), "r"(accumulate)
         : "memory");
 }
+// D(tmem) (+)= A(tmem) * B(smem desc)
 __device__ __forceinline__ void tc_mma_ts2(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_lo, uint32_t b_hi,
                                            uint32_t idesc, uint32_t accumulate) {
     asm volatile(
@@ -271,17 +276,6 @@ __device__ __forceinline__ void tc_mma_ts2(uint32_t d_tmem, uint32_t a_tmem, uin
         "r"(a_tmem), "r"(b_lo), "r"(b_hi), "r"(idesc), "r"(accumulate)
         : "memory");
 }
-// D(tmem) (+)= A(tmem) * B(smem desc)
-__device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
-                                          uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-
 // 32 lanes x 32 consecutive 32-bit columns; thread i gets lane (base + i).
 // The wait is inside the same statement so the results are valid on return.
 __device__ __forceinline__ void tmem_ld32u(uint32_t taddr, uint32_t (&r)[32]) {
@@ -299,11 +293,55 @@ __device__ __forceinline__ void tmem_ld32u(uint32_t taddr, uint32_t (&r)[32]) {
         : "memory");
 }
 
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
-    uint32_t r[32];
-    tmem_ld32u(taddr, r);
+// 32 lanes x 128 consecutive 32-bit columns (a whole score row per thread):
+// two 64-column loads and one wait.
+__device__ __forceinline__ void tmem_ld128(uint32_t taddr, float* v) {
+    uint32_t r[128];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x64.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%128];\n\t"
+        "tcgen05.ld.sync.aligned.32x32b.x64.b32 {%64,%65,%66,%67,%68,%69,%70,%71,%72,%73,%74,%75,%76,%77,%78,%79,%80,%81,%82,%83,%84,%85,%86,%87,%88,%89,%90,%91,%92,%93,%94,%95,%96,%97,%98,%99,%100,%101,%102,%103,%104,%105,%106,%107,%108,%109,%110,%111,%112,%113,%114,%115,%116,%117,%118,%119,%120,%121,%122,%123,%124,%125,%126,%127}, [%129];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]), "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]), "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]), "=r"(r[48]), "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]), "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63]), "=r"(r[64]), "=r"(r[65]), "=r"(r[66]), "=r"(r[67]), "=r"(r[68]), "=r"(r[69]), "=r"(r[70]), "=r"(r[71]), "=r"(r[72]), "=r"(r[73]), "=r"(r[74]), "=r"(r[75]), "=r"(r[76]), "=r"(r[77]), "=r"(r[78]), "=r"(r[79]), "=r"(r[80]), "=r"(r[81]), "=r"(r[82]), "=r"(r[83]), "=r"(r[84]), "=r"(r[85]), "=r"(r[86]), "=r"(r[87]), "=r"(r[88]), "=r"(r[89]), "=r"(r[90]), "=r"(r[91]), "=r"(r[92]), "=r"(r[93]), "=r"(r[94]), "=r"(r[95]), "=r"(r[96]), "=r"(r[97]), "=r"(r[98]), "=r"(r[99]), "=r"(r[100]), "=r"(r[101]), "=r"(r[102]), "=r"(r[103]), "=r"(r[104]), "=r"(r[105]), "=r"(r[106]), "=r"(r[107]), "=r"(r[108]), "=r"(r[109]), "=r"(r[110]), "=r"(r[111]), "=r"(r[112]), "=r"(r[113]), "=r"(r[114]), "=r"(r[115]), "=r"(r[116]), "=r"(r[117]), "=r"(r[118]), "=r"(r[119]), "=r"(r[120]), "=r"(r[121]), "=r"(r[122]), "=r"(r[123]), "=r"(r[124]), "=r"(r[125]), "=r"(r[126]), "=r"(r[127])
+        : "r"(taddr), "r"(taddr + 64u)
+        : "memory");
 #pragma unroll
-    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+    for (int i = 0; i < 128; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// 2^x for a pair of x <= 8 on the FMA pipe, used for part of the weights so the
+// MUFU is not the only unit producing them.  Method: Cody-Waite style range
+// reduction x = n + f with n = round(x) taken from the low mantissa bits of
+// x + 1.5*2^23 and f in [-1/2, 1/2]; 2^f by the degree-3 polynomial of least
+// maximum relative error on [-1/2, 1/2] (Remez exchange; coefficients from
+// exp2_poly_fit.py in this directory; max relative error 7.5e-5 evaluated in
+// float32); n is added to the float's exponent field.  x is clamped at -125 so
+// the result stays a normal float (2^-125 where the exact value underflows).
+__device__ __forceinline__ __attribute__((unused)) float2 exp2_fma2(float2 x) {
+    constexpr float SHIFT = 12582912.0f;  // 1.5 * 2^23
+    x.x = fmaxf(x.x, -125.0f);
+    x.y = fmaxf(x.y, -125.0f);
+    const float2 t = __fadd2_rn(x, make_float2(SHIFT, SHIFT));
+    const float2 r = __fadd2_rn(t, make_float2(-SHIFT, -SHIFT));          // round(x), exact
+    const float2 f = __ffma2_rn(r, make_float2(-1.0f, -1.0f), x);         // x - round(x), exact
+    float2 q = __ffma2_rn(make_float2(0.0551716685295105f, 0.0551716685295105f), f,
+                          make_float2(0.2426111251115799f, 0.2426111251115799f));
+    q = __ffma2_rn(q, f, make_float2(0.6932609677314758f, 0.6932609677314758f));
+    q = __ffma2_rn(q, f, make_float2(0.9999280571937561f, 0.9999280571937561f));
+    // bits(t) = bits(1.5 * 2^23) + n; shifting by 23 leaves n << 23 (mod 2^32)
+    return make_float2(__uint_as_float(__float_as_uint(q.x) + (__float_as_uint(t.x) << 23)),
+                       __uint_as_float(__float_as_uint(q.y) + (__float_as_uint(t.y) << 23)));
+}
+
+// acc + the two bf16 halves of a packed pair, each converted exactly (mixed-precision adds)
+__device__ __forceinline__ float2 add_bf16x2(float2 acc, uint32_t pk) {
+    float2 r;
+    asm("{\n\t.reg .b16 lo, hi;\n\t"
+        "mov.b32 {lo, hi}, %2;\n\t"
+        "add.rn.f32.bf16 %0, lo, %3;\n\t"
+        "add.rn.f32.bf16 %1, hi, %4;\n\t}"
+        : "=f"(r.x), "=f"(r.y)
+        : "r"(pk), "f"(acc.x), "f"(acc.y));
+    return r;
 }
 
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
@@ -540,46 +578,64 @@ __device__ void mma_role(const KParams& p, uint8_t* smem, uint32_t tmem, volatil
         return true;
     };
 
+    // Issue order per key tile j (tile 1 lags tile 0 by one step):
+    //   [P1] O1 += P1 V_{j-1};  S1 = Q1 K_j^T;   [V_j, K_{j+1}, P0] O0 += P0 V_j;  S0 = Q0 K_{j+1}^T
+    // Each P.V is followed directly by the next S of the same tile (the S/P
+    // columns are free once that P.V is issued, MMAs of one thread run in
+    // order), so the only gap the tensor pipe sees per tile is the wait for P.
     for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
         const Unit U = decode_unit(p, u);
+        const bool tile1_last = U.n[1] == U.N;  // which tile issues the unit's last S
         if (!mbar_wait(bar(L::B_QFULL), qf_phase, abort_flag, 3)) { ok = false; break; }
         qf_phase ^= 1u;
+        // prologue: K_0, S0 = Q0 K_0^T
+        int kslot = slot;
+        if (!mbar_wait(bar(L::B_KVFULL + kslot), phase, abort_flag, 4)) { ok = false; break; }
+        if (++slot == L::NSLOT) { slot = 0; phase ^= 1u; }
+        issue_s(0, kslot);
+        tc_commit(bar(L::B_SFULL + 0));
+        if (U.N == 1 && !tile1_last) tc_commit(bar(L::B_QEMPTY));
         int vslot_prev = -1;
         for (int j = 0; j < U.N; ++j) {
-            // ---- K_j
-            const int kslot = slot;
-            if (!mbar_wait(bar(L::B_KVFULL + kslot), phase, abort_flag, 4)) { ok = false; break; }
-            if (++slot == L::NSLOT) { slot = 0; phase ^= 1u; }
-            if (j < U.n[0]) {
-                issue_s(0, kslot);
-                tc_commit(bar(L::B_SFULL + 0));
-            }
-            // ---- O_1 += P_1 V_{j-1} (tile 1 lags one step behind tile 0)
-            if (j >= 1 && j - 1 < U.n[1]) {
+            // ---- tile 1: O1 += P1 V_{j-1}, then S1 = Q1 K_j^T
+            const bool pv1 = j >= 1 && j - 1 < U.n[1];
+            if (pv1) {
                 if (!wait_pv_inputs(1, 5)) { ok = false; break; }
                 issue_pv(1, vslot_prev, j - 1 > 0);
-                tc_commit(bar(L::B_KVEMPTY + vslot_prev));
             }
             if (j < U.n[1]) {
                 issue_s(1, kslot);
                 tc_commit(bar(L::B_SFULL + 1));
             }
-            tc_commit(bar(L::B_KVEMPTY + kslot));
-            if (j == U.N - 1) tc_commit(bar(L::B_QEMPTY));
-            // ---- V_j
+            if (pv1) tc_commit(bar(L::B_KVEMPTY + vslot_prev));  // V_{j-1}: last reader issued
+            tc_commit(bar(L::B_KVEMPTY + kslot));                // K_j: S0_j and S1_j issued
+            if (j == U.N - 1 && tile1_last) tc_commit(bar(L::B_QEMPTY));
+            // ---- tile 0: O0 += P0 V_j, then S0 = Q0 K_{j+1}^T
             const int vslot = slot;
-            if (!mbar_wait(bar(L::B_KVFULL + vslot), phase, abort_flag, 8)) { ok = false; break; }
+            if (!mbar_wait(bar(L::B_KVFULL + vslot), phase, abort_flag, 6)) { ok = false; break; }
             if (++slot == L::NSLOT) { slot = 0; phase ^= 1u; }
+            int knext = -1;
+            if (j + 1 < U.N) {
+                knext = slot;
+                if (!mbar_wait(bar(L::B_KVFULL + knext), phase, abort_flag, 7)) { ok = false; break; }
+                if (++slot == L::NSLOT) { slot = 0; phase ^= 1u; }
+            }
             if (j < U.n[0]) {
                 if (!wait_pv_inputs(0, 9)) { ok = false; break; }
                 issue_pv(0, vslot, j > 0);
                 if (j == U.n[0] - 1) tc_commit(bar(L::B_OFULL + 0));
+            }
+            if (j + 1 < U.n[0]) {
+                issue_s(0, knext);
+                tc_commit(bar(L::B_SFULL + 0));
+                if (j + 1 == U.N - 1 && !tile1_last) tc_commit(bar(L::B_QEMPTY));
             }
             if (j < U.n[1]) {
                 vslot_prev = vslot;
             } else {
                 tc_commit(bar(L::B_KVEMPTY + vslot));
             }
+            kslot = knext;
         }
         if (!ok) break;
         if (U.n[1] > 0) {
@@ -628,8 +684,7 @@ __device__ void softmax_role(const KParams& p, uint8_t* smem, uint32_t tmem, int
             s_phase ^= 1u;
             tc_fence_after();
             float s[BLOCK_N];
-#pragma unroll
-            for (int c = 0; c < BLOCK_N / 32; ++c) tmem_ld32(ts + 32 * c, s + 32 * c);
+            tmem_ld128(ts, s);
             const int kbase = j * BLOCK_N;
             const bool need_mask = (kbase + BLOCK_N > p.S) || (p.causal && kbase + BLOCK_N - 1 > U.q0[t]);
             if (need_mask) {
@@ -650,8 +705,8 @@ __device__ void softmax_role(const KParams& p, uint8_t* smem, uint32_t tmem, int
             mx0 = max3(mx0, s[BLOCK_N - 4], s[BLOCK_N - 3]);
             mx1 = max3(mx1, s[BLOCK_N - 2], s[BLOCK_N - 1]);
             const float m_blk = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
-            // move the reference max only when it grew by more than TAU
-            const bool grow = m_blk > m_use + Policy<BF16>::TAU;
+            bool grow = m_blk > m_use + Policy<BF16>::TAU;
+            if constexpr (BF16) grow = grow || (m_blk > m_use && ex2(m_blk - m_use) > Policy<BF16>::KAPPA * lr);
             float alpha = 1.f;
             if (grow) {
                 alpha = (m_use == -INFINITY) ? 0.f : ex2(m_use - m_blk);
@@ -668,23 +723,37 @@ __device__ void softmax_role(const KParams& p, uint8_t* smem, uint32_t tmem, int
             const float2 negm2 = make_float2(neg_m, neg_m);
             float2 lsum0 = make_float2(0.f, 0.f), lsum1 = make_float2(0.f, 0.f);
             float2 rsum0 = make_float2(0.f, 0.f), rsum1 = make_float2(0.f, 0.f);
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
+            // Weights of one half row (32 pairs) into packed 16-bit P; in tiles
+            // without masking, one pair in FMA_EXP2_PERIOD uses the FMA-pipe exp2.
+            auto half_row = [&](int h, bool use_fma_exp) {
                 uint32_t pk[32];
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
                     const float2 x = __ffma2_rn(make_float2(s[64 * h + 2 * i], s[64 * h + 2 * i + 1]), sl2x2, negm2);
-                    const float2 e = make_float2(ex2(x.x), ex2(x.y));
+                    float2 e;
+                    if constexpr (FMA_EXP2_PERIOD > 0) {
+                        constexpr int P = FMA_EXP2_PERIOD > 0 ? FMA_EXP2_PERIOD : 1;
+                        const bool fma_pair = use_fma_exp && (i % P) == P - 1;
+                        e = fma_pair ? exp2_fma2(x) : make_float2(ex2(x.x), ex2(x.y));
+                    } else {
+                        e = make_float2(ex2(x.x), ex2(x.y));
+                    }
                     pk[i] = pack2<BF16>(e.x, e.y);
                     if (i & 1) lsum1 = __fadd2_rn(lsum1, e); else lsum0 = __fadd2_rn(lsum0, e);
                     if constexpr (Policy<BF16>::NORM_BY_ROUNDED_P) {
-                        // bf16 -> fp32 is exact: the rounded weights as the MMA sees them
-                        const float2 r = make_float2(__uint_as_float(pk[i] << 16), __uint_as_float(pk[i] & 0xFFFF0000u));
-                        if (i & 1) rsum1 = __fadd2_rn(rsum1, r); else rsum0 = __fadd2_rn(rsum0, r);
+                        // the rounded weights as the MMA sees them (bf16 -> fp32 is exact)
+                        if (i & 1) rsum1 = add_bf16x2(rsum1, pk[i]); else rsum0 = add_bf16x2(rsum0, pk[i]);
                     }
                 }
                 // P (16-bit, two per column) overwrites the first 64 columns of S
                 tmem_st32(ts + 32 * h, pk);
+            };
+            if (need_mask) {
+                half_row(0, false);
+                half_row(1, false);
+            } else {
+                half_row(0, true);
+                half_row(1, true);
             }
             const float2 ls = __fadd2_rn(lsum0, lsum1);
             l += ls.x + ls.y;
