@@ -39,8 +39,8 @@
 //    shared-memory slots with full/empty mbarriers), warps 14-15 idle.
 //    The two query tiles ping-pong: the tensor pipe works on one tile while
 //    the other tile's softmax runs.
-//  Registers are rebalanced with setmaxnreg: 176 for the softmax
-//  warpgroups, 80 for correction, 80 for warpgroup 3.
+//  Registers are rebalanced with setmaxnreg: 184 for the softmax
+//  warpgroups, 72 for correction, 72 for warpgroup 3.
 //
 // Every mbarrier wait is bounded: after WAIT_TIMEOUT_CYCLES the waiting thread
 // raises the CTA's abort flag and the device status word, every role leaves
@@ -63,9 +63,9 @@ constexpr int NUM_THREADS = 512;   // 16 warps
 constexpr int WARP_MMA = 12;
 constexpr int WARP_TMA = 13;
 constexpr int REG_LAUNCH = 128;    // 65536 registers / 512 threads
-constexpr int REG_SOFTMAX = 176;
-constexpr int REG_CORR = 80;
-constexpr int REG_CTRL = 80;
+constexpr int REG_SOFTMAX = 184;
+constexpr int REG_CORR = 72;
+constexpr int REG_CTRL = 72;
 // setmaxnreg.inc waits until the registers are free: the split must fit the
 // launch allocation, and each SM sub-partition (one warp of every warpgroup).
 static_assert(2 * 128 * REG_SOFTMAX + 128 * REG_CORR + 128 * REG_CTRL <= NUM_THREADS * REG_LAUNCH,
@@ -75,9 +75,9 @@ static_assert(2 * REG_SOFTMAX + REG_CORR + REG_CTRL <= 512, "register split exce
 constexpr uint32_t TMEM_COLS = 512;
 // One weight pair in FMA_EXP2_PERIOD would be computed on the FMA pipe instead
 // of the MUFU (tiles without masking only); 0 disables it.  Measured on B200
-// with S = 16384, D = 128, bf16: period 0 -> 959 TFLOP/s, 4 -> 926, 2 -> 838:
-// the softmax warps are bound by instruction issue, not by the MUFU, so the
-// polynomial's extra instructions cost more than the ex2 they replace.
+// with S = 16384, D = 128, bf16 (no register spills in any variant):
+// period 0 -> 1034 TFLOP/s, 8 -> 1012, 4 -> 989: the polynomial's extra
+// instructions on the softmax warps cost more than the ex2 they replace.
 constexpr int FMA_EXP2_PERIOD = 0;
 // Bounds of a wait in SM clock cycles (SM clock <= 1.965 GHz): a wait gives up
 // after at least ~2 s, a drain of in-flight copies after at least ~0.1 s.
@@ -118,11 +118,19 @@ struct Smem {
     static constexpr int CHUNKS = D / 64;                  // 128-byte swizzle atoms along D
     static constexpr int CHUNK_BYTES = 128 * 128;          // 128 rows x 128 bytes
     static constexpr int TILE_BYTES = BLOCK_M * D * 2;     // one Q, K or V tile
-    static constexpr int NSLOT = (D == 128) ? 4 : 8;       // K/V ring depth
+    // K/V ring: a stage holds V_{s-1} and K_s, the two tiles that are first
+    // needed together (O0 += P0 V_{s-1}; S0 = Q0 K_s^T) and last used
+    // together (O1 += P1 V_{s-1}; S1 = Q1 K_s^T), so one wait and one release
+    // cover both.  A unit streams N + 1 stages (the first without V, the last
+    // without K).
+    static constexpr int STAGE_BYTES = 2 * TILE_BYTES;
+    static constexpr int NSTAGE = (D == 128) ? 2 : 4;
+    static constexpr int STAGE_K = 0;                      // offset of K_s in a stage
+    static constexpr int STAGE_V = TILE_BYTES;             // offset of V_{s-1}
     static constexpr int Q_OFF = 0;
     static constexpr int KV_OFF = Q_OFF + Q_TILES_PER_CTA * TILE_BYTES;
     // per-row values handed from the softmax to the correction warpgroup
-    static constexpr int ALPHA_OFF = KV_OFF + NSLOT * TILE_BYTES;   // float [2][128]
+    static constexpr int ALPHA_OFF = KV_OFF + NSTAGE * STAGE_BYTES;   // float [2][128]
     // float2 [unit parity][tile][row] = (1/l, lse); double-buffered because a
     // softmax warpgroup can finish the next unit before the epilogue of this
     // one has read its values (never two units ahead: the unit after next
@@ -132,9 +140,9 @@ struct Smem {
     // barrier indices
     static constexpr int B_QFULL = 0;
     static constexpr int B_QEMPTY = 1;
-    static constexpr int B_KVFULL = 2;
-    static constexpr int B_KVEMPTY = B_KVFULL + NSLOT;
-    static constexpr int B_SFULL = B_KVEMPTY + NSLOT;      // [2] MMA -> softmax: S_t ready
+    static constexpr int B_STFULL = 2;                     // [NSTAGE] TMA -> MMA
+    static constexpr int B_STEMPTY = B_STFULL + NSTAGE;    // [NSTAGE] MMA -> TMA
+    static constexpr int B_SFULL = B_STEMPTY + NSTAGE;     // [2] MMA -> softmax: S_t ready
     // [2] softmax + correction -> MMA: P_t written and O_t ready for it (rescaled,
     // or read out by the previous unit's epilogue); 256 arrivals per phase
     static constexpr int B_PFULL = B_SFULL + 2;
@@ -357,6 +365,15 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
         : "memory");
 }
 
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+        : "memory");
+}
+
 __device__ __forceinline__ void tmem_wait_st() {
     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
@@ -461,11 +478,11 @@ __device__ void producer_role(const KParams& p, uint8_t* smem, volatile uint32_t
     const uint32_t base = smem_u32(smem);
     const uint32_t bar0 = base + L::BAR_OFF;
     auto bar = [&](int i) { return bar0 + 8u * (uint32_t)i; };
-    int slot = 0;
+    int stage = 0;
     uint32_t phase = 0;
     uint32_t qe_phase = 0;
-    uint32_t fill_mask = 0;    // slots with a fill issued
-    uint32_t fill_parity = 0;  // parity of each slot's last fill
+    uint32_t fill_mask = 0;    // stages with a fill issued
+    uint32_t fill_parity = 0;  // parity of each stage's last fill
     int last_q_fill = -1;
     bool ok = true;
 
@@ -484,28 +501,33 @@ __device__ void producer_role(const KParams& p, uint8_t* smem, volatile uint32_t
             for (int c = 0; c < L::CHUNKS; ++c)
                 tma_load_3d(dst + c * L::CHUNK_BYTES, &p.tmap_q, bar(L::B_QFULL), c * 64, U.q0[t], U.bh);
         }
-        for (int j = 0; j < U.N; ++j) {
-#pragma unroll
-            for (int kv = 0; kv < 2; ++kv) {
-                if (!mbar_wait(bar(L::B_KVEMPTY + slot), phase ^ 1u, abort_flag, 2)) { ok = false; break; }
-                mbar_expect_tx(bar(L::B_KVFULL + slot), L::TILE_BYTES);
-                fill_mask |= 1u << slot;
-                fill_parity = (fill_parity & ~(1u << slot)) | (phase << slot);
-                const uint32_t dst = base + L::KV_OFF + slot * L::TILE_BYTES;
-                const CUtensorMap* map = kv ? &p.tmap_v : &p.tmap_k;
+        // stages 0..N: stage s = (V_{s-1} if s >= 1, K_s if s < N)
+        for (int st = 0; st <= U.N; ++st) {
+            if (!mbar_wait(bar(L::B_STEMPTY + stage), phase ^ 1u, abort_flag, 2)) { ok = false; break; }
+            const uint32_t bytes = (st >= 1 ? L::TILE_BYTES : 0) + (st < U.N ? L::TILE_BYTES : 0);
+            mbar_expect_tx(bar(L::B_STFULL + stage), bytes);
+            fill_mask |= 1u << stage;
+            fill_parity = (fill_parity & ~(1u << stage)) | (phase << stage);
+            const uint32_t dst = base + L::KV_OFF + stage * L::STAGE_BYTES;
+            if (st < U.N) {
 #pragma unroll
                 for (int c = 0; c < L::CHUNKS; ++c)
-                    tma_load_3d(dst + c * L::CHUNK_BYTES, map, bar(L::B_KVFULL + slot), c * 64, j * BLOCK_N,
-                                U.bh);
-                if (++slot == L::NSLOT) { slot = 0; phase ^= 1u; }
+                    tma_load_3d(dst + L::STAGE_K + c * L::CHUNK_BYTES, &p.tmap_k, bar(L::B_STFULL + stage), c * 64,
+                                st * BLOCK_N, U.bh);
             }
-            if (!ok) break;
+            if (st >= 1) {
+#pragma unroll
+                for (int c = 0; c < L::CHUNKS; ++c)
+                    tma_load_3d(dst + L::STAGE_V + c * L::CHUNK_BYTES, &p.tmap_v, bar(L::B_STFULL + stage), c * 64,
+                                (st - 1) * BLOCK_N, U.bh);
+            }
+            if (++stage == L::NSTAGE) { stage = 0; phase ^= 1u; }
         }
     }
     if (!ok) {
         // drain the copies this thread issued before leaving
-        for (int i = 0; i < L::NSLOT; ++i)
-            if (fill_mask & (1u << i)) mbar_drain(bar(L::B_KVFULL + i), (fill_parity >> i) & 1u);
+        for (int i = 0; i < L::NSTAGE; ++i)
+            if (fill_mask & (1u << i)) mbar_drain(bar(L::B_STFULL + i), (fill_parity >> i) & 1u);
         if (last_q_fill >= 0) mbar_drain(bar(L::B_QFULL), (uint32_t)last_q_fill);
     }
 }
@@ -540,9 +562,10 @@ __device__ void mma_role(const KParams& p, uint8_t* smem, uint32_t tmem, volatil
     const uint32_t dv_lo = (uint32_t)dv, dv_hi = (uint32_t)(dv >> 32);
     constexpr uint32_t TILE16 = (uint32_t)L::TILE_BYTES >> 4;
 
-    auto issue_s = [&](int t, int kslot) {
+    constexpr uint32_t STAGE16 = (uint32_t)L::STAGE_BYTES >> 4;
+    auto issue_s = [&](int t, int st) {
         const uint32_t a_lo = dq_lo + (uint32_t)t * TILE16;
-        const uint32_t b_lo = dk_lo + (uint32_t)kslot * TILE16;
+        const uint32_t b_lo = dk_lo + (uint32_t)st * STAGE16 + ((uint32_t)L::STAGE_K >> 4);
         const uint32_t d_tmem = tmem + (t == 0 ? COL_S0 : COL_S1);
 #pragma unroll
         for (int ks = 0; ks < KSTEPS_S; ++ks) {
@@ -550,8 +573,8 @@ __device__ void mma_role(const KParams& p, uint8_t* smem, uint32_t tmem, volatil
             tc_mma_ss2(d_tmem, a_lo + off, dq_hi, b_lo + off, dk_hi, IDESC_S, ks > 0 ? 1u : 0u);
         }
     };
-    auto issue_pv = [&](int t, int vslot, bool accumulate) {
-        const uint32_t b_lo = dv_lo + (uint32_t)vslot * TILE16;
+    auto issue_pv = [&](int t, int st, bool accumulate) {
+        const uint32_t b_lo = dv_lo + (uint32_t)st * STAGE16 + ((uint32_t)L::STAGE_V >> 4);
         const uint32_t a_tmem = tmem + (t == 0 ? COL_S0 : COL_S1);
         const uint32_t d_tmem = tmem + (t == 0 ? COL_O0 : COL_O1);
 #pragma unroll
@@ -561,7 +584,7 @@ __device__ void mma_role(const KParams& p, uint8_t* smem, uint32_t tmem, volatil
         }
     };
 
-    int slot = 0;
+    int stage = 0;
     uint32_t phase = 0;
     uint32_t qf_phase = 0;
     uint32_t p_phase[2] = {0u, 0u};
@@ -578,73 +601,67 @@ __device__ void mma_role(const KParams& p, uint8_t* smem, uint32_t tmem, volatil
         return true;
     };
 
-    // Issue order per key tile j (tile 1 lags tile 0 by one step):
-    //   [P1] O1 += P1 V_{j-1};  S1 = Q1 K_j^T;   [V_j, K_{j+1}, P0] O0 += P0 V_j;  S0 = Q0 K_{j+1}^T
+    // Issue order per key tile j (tile 1 lags tile 0 by one step), stage j
+    // holding V_{j-1} and K_j:
+    //   [P1] O1 += P1 V_{j-1};  S1 = Q1 K_j^T;  release stage j;
+    //   [stage j+1, P0] O0 += P0 V_j;  S0 = Q0 K_{j+1}^T
     // Each P.V is followed directly by the next S of the same tile (the S/P
-    // columns are free once that P.V is issued, MMAs of one thread run in
-    // order), so the only gap the tensor pipe sees per tile is the wait for P.
+    // columns are free once that P.V is issued; MMAs of one thread run in
+    // order).  Waits and commits of this thread queue behind its MMAs not yet
+    // taken by the tensor pipe, so there are as few of them as possible:
+    // per key tile three waits (P1, stage, P0) and three commits.
+    auto wait_stage = [&](int site) -> int {
+        const int st = stage;
+        if (!mbar_wait(bar(L::B_STFULL + st), phase, abort_flag, site)) return -1;
+        if (++stage == L::NSTAGE) { stage = 0; phase ^= 1u; }
+        return st;
+    };
     for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
         const Unit U = decode_unit(p, u);
         const bool tile1_last = U.n[1] == U.N;  // which tile issues the unit's last S
         if (!mbar_wait(bar(L::B_QFULL), qf_phase, abort_flag, 3)) { ok = false; break; }
         qf_phase ^= 1u;
-        // prologue: K_0, S0 = Q0 K_0^T
-        int kslot = slot;
-        if (!mbar_wait(bar(L::B_KVFULL + kslot), phase, abort_flag, 4)) { ok = false; break; }
-        if (++slot == L::NSLOT) { slot = 0; phase ^= 1u; }
-        issue_s(0, kslot);
+        // prologue: stage 0 (K_0), S0 = Q0 K_0^T
+        int cur = wait_stage(4);
+        if (cur < 0) { ok = false; break; }
+        issue_s(0, cur);
         tc_commit(bar(L::B_SFULL + 0));
         if (U.N == 1 && !tile1_last) tc_commit(bar(L::B_QEMPTY));
-        int vslot_prev = -1;
         for (int j = 0; j < U.N; ++j) {
-            // ---- tile 1: O1 += P1 V_{j-1}, then S1 = Q1 K_j^T
-            const bool pv1 = j >= 1 && j - 1 < U.n[1];
-            if (pv1) {
+            // ---- tile 1 on stage j: O1 += P1 V_{j-1}, S1 = Q1 K_j^T
+            if (j >= 1 && j - 1 < U.n[1]) {
                 if (!wait_pv_inputs(1, 5)) { ok = false; break; }
-                issue_pv(1, vslot_prev, j - 1 > 0);
+                issue_pv(1, cur, j - 1 > 0);
             }
             if (j < U.n[1]) {
-                issue_s(1, kslot);
+                issue_s(1, cur);
                 tc_commit(bar(L::B_SFULL + 1));
             }
-            if (pv1) tc_commit(bar(L::B_KVEMPTY + vslot_prev));  // V_{j-1}: last reader issued
-            tc_commit(bar(L::B_KVEMPTY + kslot));                // K_j: S0_j and S1_j issued
+            tc_commit(bar(L::B_STEMPTY + cur));  // V_{j-1} and K_j: last readers issued
             if (j == U.N - 1 && tile1_last) tc_commit(bar(L::B_QEMPTY));
-            // ---- tile 0: O0 += P0 V_j, then S0 = Q0 K_{j+1}^T
-            const int vslot = slot;
-            if (!mbar_wait(bar(L::B_KVFULL + vslot), phase, abort_flag, 6)) { ok = false; break; }
-            if (++slot == L::NSLOT) { slot = 0; phase ^= 1u; }
-            int knext = -1;
-            if (j + 1 < U.N) {
-                knext = slot;
-                if (!mbar_wait(bar(L::B_KVFULL + knext), phase, abort_flag, 7)) { ok = false; break; }
-                if (++slot == L::NSLOT) { slot = 0; phase ^= 1u; }
-            }
+            // ---- tile 0 on stage j+1: O0 += P0 V_j, S0 = Q0 K_{j+1}^T
+            const int nxt = wait_stage(6);
+            if (nxt < 0) { ok = false; break; }
             if (j < U.n[0]) {
                 if (!wait_pv_inputs(0, 9)) { ok = false; break; }
-                issue_pv(0, vslot, j > 0);
+                issue_pv(0, nxt, j > 0);
                 if (j == U.n[0] - 1) tc_commit(bar(L::B_OFULL + 0));
             }
             if (j + 1 < U.n[0]) {
-                issue_s(0, knext);
+                issue_s(0, nxt);
                 tc_commit(bar(L::B_SFULL + 0));
                 if (j + 1 == U.N - 1 && !tile1_last) tc_commit(bar(L::B_QEMPTY));
             }
-            if (j < U.n[1]) {
-                vslot_prev = vslot;
-            } else {
-                tc_commit(bar(L::B_KVEMPTY + vslot));
-            }
-            kslot = knext;
+            cur = nxt;
         }
         if (!ok) break;
+        // stage N holds V_{N-1}: O1 += P1 V_{N-1}, then release it
         if (U.n[1] > 0) {
-            // tail: O_1 += P_1 V_{N-1}
             if (!wait_pv_inputs(1, 12)) { ok = false; break; }
-            issue_pv(1, vslot_prev, U.N - 1 > 0);
-            tc_commit(bar(L::B_KVEMPTY + vslot_prev));
+            issue_pv(1, cur, U.N - 1 > 0);
             tc_commit(bar(L::B_OFULL + 1));
         }
+        tc_commit(bar(L::B_STEMPTY + cur));
     }
     // all MMAs issued by this thread have completed once B_FIN fires
     tc_commit(bar(L::B_FIN));
@@ -723,13 +740,14 @@ __device__ void softmax_role(const KParams& p, uint8_t* smem, uint32_t tmem, int
             const float2 negm2 = make_float2(neg_m, neg_m);
             float2 lsum0 = make_float2(0.f, 0.f), lsum1 = make_float2(0.f, 0.f);
             float2 rsum0 = make_float2(0.f, 0.f), rsum1 = make_float2(0.f, 0.f);
-            // Weights of one half row (32 pairs) into packed 16-bit P; in tiles
-            // without masking, one pair in FMA_EXP2_PERIOD uses the FMA-pipe exp2.
-            auto half_row = [&](int h, bool use_fma_exp) {
-                uint32_t pk[32];
+            // Weights of a quarter row (16 pairs) into packed 16-bit P, stored to
+            // TMEM right away (fewer live registers); in tiles without masking,
+            // one pair in FMA_EXP2_PERIOD uses the FMA-pipe exp2.
+            auto quarter_row = [&](int qr, bool use_fma_exp) {
+                uint32_t pk[16];
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const float2 x = __ffma2_rn(make_float2(s[64 * h + 2 * i], s[64 * h + 2 * i + 1]), sl2x2, negm2);
+                for (int i = 0; i < 16; ++i) {
+                    const float2 x = __ffma2_rn(make_float2(s[32 * qr + 2 * i], s[32 * qr + 2 * i + 1]), sl2x2, negm2);
                     float2 e;
                     if constexpr (FMA_EXP2_PERIOD > 0) {
                         constexpr int P = FMA_EXP2_PERIOD > 0 ? FMA_EXP2_PERIOD : 1;
@@ -746,14 +764,14 @@ __device__ void softmax_role(const KParams& p, uint8_t* smem, uint32_t tmem, int
                     }
                 }
                 // P (16-bit, two per column) overwrites the first 64 columns of S
-                tmem_st32(ts + 32 * h, pk);
+                tmem_st16(ts + 16 * qr, pk);
             };
             if (need_mask) {
-                half_row(0, false);
-                half_row(1, false);
+#pragma unroll
+                for (int qr = 0; qr < 4; ++qr) quarter_row(qr, false);
             } else {
-                half_row(0, true);
-                half_row(1, true);
+#pragma unroll
+                for (int qr = 0; qr < 4; ++qr) quarter_row(qr, true);
             }
             const float2 ls = __fadd2_rn(lsum0, lsum1);
             l += ls.x + ls.y;
