@@ -88,7 +88,7 @@ constexpr long long DRAIN_TIMEOUT_CYCLES = 200000000ll;
 //  - always when the block max exceeds m by more than TAU = 8 (weights stay
 //    <= 2^8, lazy rescale);
 //  - bf16 only: also when the block's largest weight 2^(max - m) exceeds
-//    KAPPA * l (l = the row sum so far).  Weights are rounded to bf16 (8-bit
+//    KAPPA * l (l = the row sum so far; KAPPA = RESCALE_KAPPA).  Weights are rounded to bf16 (8-bit
 //    precision) before P.V, and the rounding of a row's largest weight
 //    2^d (0 < d <= 8) is what dominates the error of O when a few keys carry
 //    the row (a sharp softmax).  Moving m makes that weight exactly 1.0; when
@@ -96,10 +96,10 @@ constexpr long long DRAIN_TIMEOUT_CYCLES = 200000000ll;
 //    rounding moves O by at most ~2^-9 * KAPPA * |v|.  Soft rows (large l)
 //    thus keep the lazy rescale, sharp rows the exact one.
 //  fp16 (11-bit precision) uses the lazy rule only.
+constexpr float RESCALE_KAPPA = 0.125f;
 template <bool BF16>
 struct Policy {
     static constexpr float TAU = 8.0f;
-    [[maybe_unused]] static constexpr float KAPPA = 0.125f;
     // bf16: O is normalised by the sum of the rounded weights that the P.V
     // product uses (a second sum, lr), so O is a convex combination of V rows
     // (exact in the one-key limit); the LSE keeps the fp32 sum l, whose
@@ -723,7 +723,7 @@ __device__ void softmax_role(const KParams& p, uint8_t* smem, uint32_t tmem, int
             mx1 = max3(mx1, s[BLOCK_N - 2], s[BLOCK_N - 1]);
             const float m_blk = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
             bool grow = m_blk > m_use + Policy<BF16>::TAU;
-            if constexpr (BF16) grow = grow || (m_blk > m_use && ex2(m_blk - m_use) > Policy<BF16>::KAPPA * lr);
+            if constexpr (BF16) grow = grow || (m_blk > m_use && ex2(m_blk - m_use) > RESCALE_KAPPA * lr);
             float alpha = 1.f;
             if (grow) {
                 alpha = (m_use == -INFINITY) ? 0.f : ex2(m_use - m_blk);
