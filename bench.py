@@ -35,7 +35,8 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
-from tiled_attention_18_b200.workloads import WORKLOADS, attention_flops, make_inputs, sample_rows  # noqa: E402
+from tiled_attention_18_b200.scaling import job_throughput, max_over_ranks, rank_env, rank_seed  # noqa: E402
+from tiled_attention_18_b200.workloads import WORKLOADS, make_inputs, sample_rows  # noqa: E402
 
 METRIC = "attention fwd TFLOPS (causal-adjusted) and % of B200 dense fp16/bf16 peak"
 UNIT = "TFLOP/s"
@@ -179,11 +180,8 @@ def run_reference(args):
     if rank != 0:
         return 0
     runs = workload_runs(args.workload)
-    for _ in range(args.warmup):
-        pass  # the oracle has no warm-up state; warm-up steps are not needed
-    cb = None
+    # the oracle keeps no state between calls: warm-up steps have nothing to warm
     times = []
-    flops_total = 0.0
     for _ in range(args.steps):
         cb = cpu_baseline(args.workload, target_s=max(2.0, 60.0 / max(args.steps, 1)))
         times.append(cb)
@@ -199,7 +197,6 @@ def run_reference(args):
         "cpu_baseline": cb,
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
-    del flops_total
     print(json.dumps(line), flush=True)
     return 0
 
@@ -225,9 +222,7 @@ def main(argv=None) -> int:
 
     import tiled_attention_18_b200 as fa
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    rank, world, local = rank_env()
     if world != args.gpus:
         print(f"warning: --gpus {args.gpus} but WORLD_SIZE={world}; using WORLD_SIZE", file=sys.stderr)
     torch.cuda.set_device(local)
@@ -253,7 +248,7 @@ def main(argv=None) -> int:
             host_in.append(host_in[0])
             dev_in.append(dev_in[0])
         else:
-            q, k, v = make_inputs(w.B, w.H, w.S, w.D, w.dtype, w.qk_mult, w.seed + rank)
+            q, k, v = make_inputs(w.B, w.H, w.S, w.D, w.dtype, w.qk_mult, rank_seed(w.seed, rank))
             host_in.append(tuple(t.pin_memory() for t in (q, k, v)))
             dev_in.append(tuple(t.to(dev) for t in (q, k, v)))
         o = torch.empty((w.B, w.H, w.S, w.D), dtype=w.torch_dtype, device=dev)
@@ -302,12 +297,9 @@ def main(argv=None) -> int:
         raise fa.FaError(st, "timed region")
     elapsed_ms = start.elapsed_time(stop)
     kern_ms = np.array([[a.elapsed_time(b) for (a, b) in row] for row in ev])  # [steps, runs]
-    t = torch.tensor([elapsed_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    max_ms = float(t.item())
+    max_ms = max_over_ranks(elapsed_ms, device=dev)
     step_flops = sum(w.flops for w in runs)
-    value = step_flops * world * args.steps / (max_ms * 1e-3) / 1e12
+    value = job_throughput(step_flops, args.steps, world, max_ms)
     peak, peak_src = peak_tflops()
 
     # roofline of the kernel: algorithmic flops per launch / mean launch duration
@@ -348,10 +340,7 @@ def main(argv=None) -> int:
         e1.record(stream)
         torch.cuda.synchronize(dev)
         barrier()
-        te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
-        if world > 1:
-            dist.all_reduce(te, op=dist.ReduceOp.MAX)
-        e2e_val = step_flops * world * args.e2e_steps / (float(te.item()) * 1e-3) / 1e12
+        e2e_val = job_throughput(step_flops, args.e2e_steps, world, max_over_ranks(e0.elapsed_time(e1), device=dev))
         e2e = {"value": e2e_val, "unit": UNIT, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
 
     cb = None

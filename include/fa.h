@@ -108,6 +108,16 @@ FA_API int fa_check_status(cudaStream_t stream);
  */
 FA_API int fa_last_timeout_site(void);
 
+/*
+ * fa_selftest_timeout -- diagnostic for the failure path (no counterpart on
+ * the pages): launches on `stream` a one-CTA kernel whose first mbarrier wait
+ * is never satisfied.  After about 50 ms the wait gives up, the kernel
+ * records a timeout in the device status word (wait site 100), releases its
+ * tensor memory and ends; the context stays usable.  A following
+ * fa_check_status returns FA_ERR_TIMEOUT.  Returns FA_OK when launched.
+ */
+FA_API int fa_selftest_timeout(cudaStream_t stream);
+
 /* fa_status_string -- static, NUL-terminated description of a status code. */
 FA_API const char* fa_status_string(int status);
 

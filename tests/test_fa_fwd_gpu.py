@@ -133,3 +133,18 @@ def test_host_side_errors_on_device():
     # empty problem: nothing launched, pointers not inspected
     assert fa.fa_fwd(0, 0, 0, 0, 0, 0, 4, 64, 64, 0.125, 0, fa.FA_FP16, st) == 0
     assert fa.fa_check_status(st) == 0
+
+
+def test_stuck_wait_reports_timeout_and_context_survives():
+    """A wait that nothing satisfies ends with FA_ERR_TIMEOUT (no hang, no fault),
+    and the library keeps working afterwards."""
+    st = torch.cuda.current_stream().cuda_stream
+    assert fa.fa_check_status(st) == 0
+    assert fa.fa_selftest_timeout(st) == 0
+    assert fa.fa_check_status(st) == -8           # FA_ERR_TIMEOUT
+    assert fa.fa_last_timeout_site() & 0xFF == 100
+    assert fa.fa_check_status(st) == 0            # the status word was cleared
+    q, k, v = make_inputs(1, 2, 300, 64, "fp16", seed=9)
+    o, lse = run_fa(q, k, v, softmax_scale(64), True)
+    o_ref, lse_ref = oracle.attn_fwd(q, k, v, softmax_scale(64), True, "fp16")
+    compare(o, lse, o_ref, lse_ref, "fp16")

@@ -37,6 +37,7 @@ SIGNATURES = [
       ctypes.c_int, ctypes.c_void_p]),
     ("fa_check_status", ctypes.c_int, [ctypes.c_void_p]),
     ("fa_last_timeout_site", ctypes.c_int, []),
+    ("fa_selftest_timeout", ctypes.c_int, [ctypes.c_void_p]),
     ("fa_status_string", ctypes.c_char_p, [ctypes.c_int]),
     ("fa_version", ctypes.c_int, []),
     ("fa_num_units", ctypes.c_longlong, [ctypes.c_int, ctypes.c_int, ctypes.c_int]),
@@ -83,6 +84,10 @@ def fa_check_status(stream: int = 0) -> int:
 
 def fa_last_timeout_site() -> int:
     return int(load().fa_last_timeout_site())
+
+
+def fa_selftest_timeout(stream: int = 0) -> int:
+    return int(load().fa_selftest_timeout(stream))
 
 
 def fa_status_string(status: int) -> str:

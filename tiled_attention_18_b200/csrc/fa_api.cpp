@@ -177,6 +177,18 @@ int fa_check_status(cudaStream_t stream) {
 
 int fa_last_timeout_site(void) { return t_last_site; }
 
+int fa_selftest_timeout(cudaStream_t stream) {
+    DeviceInfo dev;
+    int rc = device_info(&dev);
+    if (rc != FA_OK) return rc;
+    if (dev.major != 10 || dev.minor != 0) return FA_ERR_ARCH;
+    if (fa::launch_selftest_timeout(stream) != cudaSuccess) {
+        cudaGetLastError();
+        return FA_ERR_LAUNCH;
+    }
+    return FA_OK;
+}
+
 const char* fa_status_string(int status) {
     switch (status) {
         case FA_OK: return "ok";

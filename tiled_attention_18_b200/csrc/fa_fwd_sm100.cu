@@ -214,7 +214,7 @@ __device__ __noinline__ void record_failure(int site) {
 // another role has already aborted.  The deadline uses the SM cycle counter
 // (cheap to read); the common case costs only the polls themselves.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile uint32_t* abort_flag,
-                                          int site) {
+                                          int site, long long deadline_cycles = WAIT_TIMEOUT_CYCLES) {
 #pragma unroll 1
     for (int i = 0; i < 8; ++i)
         if (mbar_try_wait(bar, parity)) return true;
@@ -224,7 +224,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
         if (mbar_try_wait(bar, parity)) return true;
         if ((it & 15u) == 0) {
             if (*abort_flag) return false;
-            if (clock64() - t0 > WAIT_TIMEOUT_CYCLES) break;
+            if (clock64() - t0 > deadline_cycles) break;
         }
     }
     *abort_flag = 1u;
@@ -955,6 +955,41 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) fa_fwd_kernel(const __grid_con
     }
 }
 
+// Diagnostic kernel for the failure path: thread 0 waits on an mbarrier that
+// nothing arrives on, with a short deadline; it then raises the abort flag and
+// the status word.  Thread 32 waits on another barrier and leaves on the abort
+// flag; TMEM held by the CTA is released before the kernel ends.
+__global__ void __launch_bounds__(64, 1) selftest_timeout_kernel(long long deadline_cycles) {
+    __shared__ __align__(8) uint64_t bars[2];
+    __shared__ uint32_t tm;
+    __shared__ uint32_t abort_s;
+    const int warp = threadIdx.x >> 5;
+    const uint32_t b0 = smem_u32(&bars[0]), b1 = smem_u32(&bars[1]);
+    if (threadIdx.x == 0) {
+        mbar_init(b0, 1);
+        mbar_init(b1, 1);
+        abort_s = 0u;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 0) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&tm)), "r"(32u)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    volatile uint32_t* abort_flag = &abort_s;
+    if (threadIdx.x == 0) mbar_wait(b0, 0u, abort_flag, SELFTEST_SITE, deadline_cycles);
+    if (threadIdx.x == 32) mbar_wait(b1, 0u, abort_flag, SELFTEST_SITE + 1, 8 * deadline_cycles);
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tm), "r"(32u) : "memory");
+    }
+}
+
 template <int D, bool BF16>
 cudaError_t launch_impl(const LaunchArgs& a, cudaStream_t stream) {
     using L = Smem<D>;
@@ -992,6 +1027,12 @@ cudaError_t launch_fwd_sm100(const LaunchArgs& a, cudaStream_t stream) {
         return a.dtype == 1 ? launch_impl<128, true>(a, stream) : launch_impl<128, false>(a, stream);
     }
     return a.dtype == 1 ? launch_impl<64, true>(a, stream) : launch_impl<64, false>(a, stream);
+}
+
+cudaError_t launch_selftest_timeout(cudaStream_t stream) {
+    // about 50 ms at the maximum SM clock
+    selftest_timeout_kernel<<<1, 64, 0, stream>>>(100000000ll);
+    return cudaGetLastError();
 }
 
 cudaError_t read_and_clear_status(cudaStream_t stream, int* status, int* site) {

@@ -18,6 +18,8 @@ constexpr int ROWS_PER_UNIT = BLOCK_M * Q_TILES_PER_CTA;
 // Device-side status codes written to the status word by the kernel.
 constexpr int DEV_OK = 0;
 constexpr int DEV_TIMEOUT = 1;
+// Wait-site code of the diagnostic timeout kernel (low byte of the site word).
+constexpr int SELFTEST_SITE = 100;
 
 struct LaunchArgs {
     CUtensorMap tmap_q;     // 3-D maps over [B*H][S][D], box {64, 128, 1}, 128-byte swizzle
@@ -41,6 +43,9 @@ inline int64_t num_units(int64_t BH, int64_t S) {
 
 // Launch the persistent forward kernel on `stream`.  Returns a cudaError_t.
 cudaError_t launch_fwd_sm100(const LaunchArgs& a, cudaStream_t stream);
+
+// Launch the diagnostic kernel whose first wait is never satisfied.
+cudaError_t launch_selftest_timeout(cudaStream_t stream);
 
 // Read (after synchronising `stream`) and clear the device status word of
 // the current device.  *status receives DEV_OK or an error code; *site the
