@@ -83,8 +83,12 @@ typedef enum {
  *           nearest even.
  * stream  : the CUDA stream to launch on (0 = legacy default stream).
  *
- * Ownership: the caller owns every buffer and the stream; fa_fwd allocates
- * no device memory.  Synchronicity: asynchronous on `stream`; fa_fwd never
+ * Ownership: the caller owns every buffer and the stream.  With causal = 1
+ * the library's work scheduler uses a 4-byte counter in device scratch: one
+ * per (device, stream), allocated with cudaMalloc by the first causal call on
+ * that stream (so that call must not be inside a stream capture) and kept
+ * until the process exits; each causal call zeroes it with cudaMemsetAsync on
+ * `stream`.  Synchronicity: asynchronous on `stream`; fa_fwd never
  * synchronises.  Errors: argument checks run before any launch and return a
  * negative fa_status with nothing launched; a launch failure returns
  * FA_ERR_LAUNCH.  A device-side wait that exceeds its bound (about two

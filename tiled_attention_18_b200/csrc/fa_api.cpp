@@ -15,7 +15,9 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <map>
 #include <mutex>
+#include <utility>
 
 #include "fa_internal.h"
 
@@ -42,6 +44,27 @@ EncodeTiledFn g_encode = nullptr;
 std::once_flag g_encode_once;
 
 thread_local int t_last_site = 0;
+
+// Scratch of the causal work scheduler: one unit counter per (device, stream),
+// allocated on first use and kept for the life of the process.  Launches on
+// one stream are ordered, so they can share the counter; launches on
+// different streams never do.
+std::mutex g_ws_mu;
+std::map<std::pair<int, cudaStream_t>, unsigned int*> g_ws;
+
+unsigned int* sched_workspace(int dev, cudaStream_t stream) {
+    std::lock_guard<std::mutex> lock(g_ws_mu);
+    const auto key = std::make_pair(dev, stream);
+    auto it = g_ws.find(key);
+    if (it != g_ws.end()) return it->second;
+    void* ptr = nullptr;
+    if (cudaMalloc(&ptr, 256) != cudaSuccess) {
+        cudaGetLastError();
+        return nullptr;
+    }
+    g_ws[key] = static_cast<unsigned int*>(ptr);
+    return static_cast<unsigned int*>(ptr);
+}
 
 int device_info(DeviceInfo* out) {
     int dev = 0;
@@ -151,6 +174,17 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int
     a.scale_log2 = (float)((double)scale * 1.4426950408889634074);  // scale * log2(e)
     const int64_t units = fa::num_units(BH, S);
     a.grid = (int)(units < dev.sms ? units : dev.sms);
+    a.sched = nullptr;
+    if (causal) {
+        // units differ in length under the mask: CTAs claim them from a counter
+        unsigned int* ws = sched_workspace(cur, stream);
+        if (!ws) return FA_ERR_LAUNCH;
+        if (cudaMemsetAsync(ws, 0, sizeof(unsigned int), stream) != cudaSuccess) {
+            cudaGetLastError();
+            return FA_ERR_LAUNCH;
+        }
+        a.sched = ws;
+    }
     if (fa::launch_fwd_sm100(a, stream) != cudaSuccess) {
         cudaGetLastError();
         return FA_ERR_LAUNCH;

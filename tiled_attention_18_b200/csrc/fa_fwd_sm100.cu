@@ -36,7 +36,8 @@
 //  * warpgroup 3: warp 12 issues tcgen05.mma from one thread (S_t = Q_t K_j^T
 //    into TMEM; O_t += P_t V_j with P_t read from TMEM), warp 13 is the TMA
 //    producer (Q tiles once per unit, K_j and V_j through a ring of
-//    shared-memory slots with full/empty mbarriers), warps 14-15 idle.
+//    shared-memory stages with full/empty mbarriers; it also takes the work
+//    units, from a counter when causal, and publishes them), warps 14-15 idle.
 //    The two query tiles ping-pong: the tensor pipe works on one tile while
 //    the other tile's softmax runs.
 //  Registers are rebalanced with setmaxnreg: 184 for the softmax
@@ -150,9 +151,16 @@ struct Smem {
     static constexpr int B_STATS = B_OFULL + 2;            // [2] softmax -> correction: alpha ready
     static constexpr int B_FINAL = B_STATS + 2;            // [parity][2] softmax -> correction: 1/l, lse ready
     static constexpr int B_FIN = B_FINAL + 4;
-    static constexpr int NBAR = B_FIN + 1;
-    static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;    // tmem base (u32), abort flag (u32)
-    static constexpr int BYTES = MISC_OFF + 16;
+    // unit ring: the TMA lane publishes the work-unit indices it took, the MMA,
+    // softmax and correction roles read them
+    static constexpr int NUNIT = 2;
+    static constexpr int B_UFULL = B_FIN + 1;              // [NUNIT] TMA lane -> other roles
+    static constexpr int B_UEMPTY = B_UFULL + NUNIT;       // [NUNIT] other roles -> TMA lane
+    static constexpr int NBAR = B_UEMPTY + NUNIT;
+    // misc: tmem base (u32), abort flag (u32), pad, unit ring (int[NUNIT])
+    static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
+    static constexpr int UNIT_OFF = MISC_OFF + 16;
+    static constexpr int BYTES = UNIT_OFF + NUNIT * 4;
     static constexpr int ALLOC = BYTES + 1024;             // slack for 1 KiB alignment
 };
 
@@ -169,7 +177,12 @@ struct KParams {
     int nkv;       // key tiles per head
     int causal;
     float scale_log2;
+    unsigned int* sched;  // zeroed unit counter (claim order), or null for the static order
 };
+
+// Threads that read each published unit index: MMA lane, two softmax
+// warpgroups and the correction warpgroup.
+constexpr uint32_t UNIT_READERS = 1 + 2 * BLOCK_M + BLOCK_M;
 
 // ------------------------------------------------------------------ PTX helpers
 
@@ -472,6 +485,23 @@ __device__ __forceinline__ Unit decode_unit(const KParams& p, int u) {
 
 // ------------------------------------------------------------------ roles
 
+// Reads the work-unit indices published by the TMA lane, in order.
+// next() returns the unit, -1 when the CTA has no more work, -2 on abort.
+template <int D>
+struct UnitReader {
+    int slot = 0;
+    uint32_t phase = 0;
+    __device__ __forceinline__ int next(uint8_t* smem, volatile uint32_t* abort_flag, int site) {
+        using L = Smem<D>;
+        const uint32_t bar0 = smem_u32(smem) + L::BAR_OFF;
+        if (!mbar_wait(bar0 + 8u * (uint32_t)(L::B_UFULL + slot), phase, abort_flag, site)) return -2;
+        const int u = reinterpret_cast<volatile int*>(smem + L::UNIT_OFF)[slot];
+        mbar_arrive(bar0 + 8u * (uint32_t)(L::B_UEMPTY + slot));
+        if (++slot == L::NUNIT) { slot = 0; phase ^= 1u; }
+        return u;
+    }
+};
+
 template <int D>
 __device__ void producer_role(const KParams& p, uint8_t* smem, volatile uint32_t* abort_flag) {
     using L = Smem<D>;
@@ -485,8 +515,24 @@ __device__ void producer_role(const KParams& p, uint8_t* smem, volatile uint32_t
     uint32_t fill_parity = 0;  // parity of each stage's last fill
     int last_q_fill = -1;
     bool ok = true;
+    volatile int* ring = reinterpret_cast<volatile int*>(smem + L::UNIT_OFF);
+    int uslot = 0;
+    uint32_t uphase = 0;
 
-    for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
+    // Work units: with a counter (the causal mask, where units differ in
+    // length) the next unit is claimed when this CTA is about to start it, so
+    // CTAs that finish early take more units and the longest-first order of
+    // decode_unit holds across the grid; without one the CTA takes units
+    // blockIdx.x, blockIdx.x + gridDim.x, ...  Each index is published to the
+    // other roles through the unit ring.
+    for (int k = 0;; ++k) {
+        int u = p.sched ? (int)atomicAdd(p.sched, 1u) : (int)blockIdx.x + k * (int)gridDim.x;
+        if (u >= p.n_units) u = -1;
+        if (!mbar_wait(bar(L::B_UEMPTY + uslot), uphase ^ 1u, abort_flag, 30)) { ok = false; break; }
+        ring[uslot] = u;
+        mbar_arrive(bar(L::B_UFULL + uslot));
+        if (++uslot == L::NUNIT) { uslot = 0; uphase ^= 1u; }
+        if (u < 0) break;
         const Unit U = decode_unit(p, u);
         if (!mbar_wait(bar(L::B_QEMPTY), qe_phase ^ 1u, abort_flag, 1)) { ok = false; break; }
         qe_phase ^= 1u;
@@ -616,7 +662,10 @@ __device__ void mma_role(const KParams& p, uint8_t* smem, uint32_t tmem, volatil
         if (++stage == L::NSTAGE) { stage = 0; phase ^= 1u; }
         return st;
     };
-    for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
+    UnitReader<D> units;
+    for (;;) {
+        const int u = units.next(smem, abort_flag, 32);
+        if (u < 0) break;
         const Unit U = decode_unit(p, u);
         const bool tile1_last = U.n[1] == U.N;  // which tile issues the unit's last S
         if (!mbar_wait(bar(L::B_QFULL), qf_phase, abort_flag, 3)) { ok = false; break; }
@@ -686,7 +735,11 @@ __device__ void softmax_role(const KParams& p, uint8_t* smem, uint32_t tmem, int
     const float2 sl2x2 = make_float2(sl2, sl2);
 
     uint32_t s_phase = 0;
-    for (int u = blockIdx.x; u < p.n_units; u += gridDim.x) {
+    UnitReader<D> units;
+    for (;;) {
+        const int u = units.next(smem, abort_flag, 33);
+        if (!__all_sync(0xffffffffu, u != -2)) return;
+        if (u < 0) break;
         const Unit U = decode_unit(p, u);
         const int n = U.n[t];
         if (n == 0) continue;
@@ -879,7 +932,11 @@ __device__ void correction_role(const KParams& p, uint8_t* smem, uint32_t tmem, 
         return true;
     };
 
-    for (int u = blockIdx.x; u < p.n_units; u += gridDim.x) {
+    UnitReader<D> units;
+    for (;;) {
+        const int u = units.next(smem, abort_flag, 34);
+        if (!__all_sync(0xffffffffu, u != -2)) return;
+        if (u < 0) break;
         const Unit U = decode_unit(p, u);
         for (int j = 1; j < U.N; ++j) {
             if (j < U.n[0] && !correct(0)) return;
@@ -909,6 +966,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) fa_fwd_kernel(const __grid_con
                 count = BLOCK_M;      // one arrival per thread of a 128-thread warpgroup
             if (i >= L::B_PFULL && i < L::B_PFULL + 2)
                 count = 2 * BLOCK_M;  // softmax and correction warpgroups
+            if (i >= L::B_UEMPTY && i < L::B_UEMPTY + L::NUNIT) count = UNIT_READERS;
             mbar_init(base + L::BAR_OFF + 8 * i, count);
         }
         *abort_flag = 0u;
@@ -1010,6 +1068,7 @@ cudaError_t launch_impl(const LaunchArgs& a, cudaStream_t stream) {
     p.nkv = (a.S + BLOCK_N - 1) / BLOCK_N;
     p.causal = a.causal;
     p.scale_log2 = a.scale_log2;
+    p.sched = a.sched;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)a.grid, 1, 1);
     cfg.blockDim = dim3(NUM_THREADS, 1, 1);

@@ -34,6 +34,7 @@ struct LaunchArgs {
     int causal;
     float scale_log2;       // scale * log2(e)
     int grid;               // persistent CTAs
+    unsigned int* sched;    // zeroed device counter for claimed-unit scheduling, or null
 };
 
 // Number of work units (b, h, 256-row query block).
