@@ -98,6 +98,27 @@ FA_API int fa_fwd(const void* q, const void* k, const void* v, void* o, float* l
            int D, float scale, int causal, int dtype, cudaStream_t stream);
 
 /*
+ * fa_fwd_noalloc -- fa_fwd for callers that cannot allocate device memory
+ * (code that runs where cudaMalloc is unavailable or not allowed, such as
+ * inside a memory allocator, a runtime that works only in pre-allocated
+ * memory, or a process whose device footprint must not grow).  The pages have
+ * no counterpart; it is a deployment variant.  Same arguments, checks, result
+ * and error codes as fa_fwd, but it allocates nothing: the causal work
+ * scheduler's counter lives in a fixed 256-byte array inside libfa.so's own
+ * device memory, held on every GPU that loads the library until the process
+ * exits.  The first call on a device looks up that array's device address
+ * (once per device, with that device current), so make that first call
+ * before any stream capture.  Limit: the work units plus the CTAs of one call
+ * must stay below 2^31 (always true for shapes fa_fwd accepts); otherwise it
+ * returns FA_ERR_SHAPE.  Every call shares the one array, and each causal call
+ * zeroes its counter on `stream` before the launch: calls that overlap on the
+ * GPU (for example on two streams at once) race on it and may compute wrong
+ * results; issue them one after another.
+ */
+FA_API int fa_fwd_noalloc(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+                          int S, int D, float scale, int causal, int dtype, cudaStream_t stream);
+
+/*
  * fa_check_status -- synchronise `stream`, then report and clear the device
  * status word of the current device: FA_OK, FA_ERR_TIMEOUT if a kernel
  * stopped on a bounded wait since the last call, or FA_ERR_LAUNCH on a CUDA

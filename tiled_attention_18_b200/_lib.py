@@ -35,6 +35,10 @@ SIGNATURES = [
      [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
       ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_float, ctypes.c_int,
       ctypes.c_int, ctypes.c_void_p]),
+    ("fa_fwd_noalloc", ctypes.c_int,
+     [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+      ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_float, ctypes.c_int,
+      ctypes.c_int, ctypes.c_void_p]),
     ("fa_check_status", ctypes.c_int, [ctypes.c_void_p]),
     ("fa_last_timeout_site", ctypes.c_int, []),
     ("fa_selftest_timeout", ctypes.c_int, [ctypes.c_void_p]),
@@ -76,6 +80,13 @@ def fa_fwd(q_ptr: int, k_ptr: int, v_ptr: int, o_ptr: int, lse_ptr: int, B: int,
     """Raw C call: device pointers as integers, returns the fa_status code."""
     return int(load().fa_fwd(q_ptr, k_ptr, v_ptr, o_ptr, lse_ptr, B, H, S, D, float(scale), int(causal),
                              int(dtype), stream))
+
+
+def fa_fwd_noalloc(q_ptr: int, k_ptr: int, v_ptr: int, o_ptr: int, lse_ptr: int, B: int, H: int, S: int,
+                   D: int, scale: float, causal: int, dtype: int, stream: int) -> int:
+    """Raw C call of the variant that allocates no device memory (see include/fa.h)."""
+    return int(load().fa_fwd_noalloc(q_ptr, k_ptr, v_ptr, o_ptr, lse_ptr, B, H, S, D, float(scale),
+                                     int(causal), int(dtype), stream))
 
 
 def fa_check_status(stream: int = 0) -> int:

@@ -196,6 +196,81 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int
     return FA_OK;
 }
 
+// For callers that cannot allocate device memory (for example code running
+// where cudaMalloc is unavailable or forbidden: inside an allocator, a
+// pre-allocated-memory runtime, or a process that must not grow its device
+// footprint).  Same computation and arguments as fa_fwd; the causal scheduler's
+// counter lives in the library's static scratch array instead of memory the
+// library allocates.  Nothing here allocates.
+int fa_fwd_noalloc(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int S, int D,
+                   float scale, int causal, int dtype, cudaStream_t stream) {
+    if (B < 0 || H < 0 || S < 0) return FA_ERR_SHAPE;
+    if (D != 64 && D != 128) return FA_ERR_HEADDIM;
+    if (dtype != FA_FP16 && dtype != FA_BF16) return FA_ERR_DTYPE;
+    if (!(std::isfinite(scale) && scale > 0.f)) return FA_ERR_SCALE;
+    if (causal != 0 && causal != 1) return FA_ERR_ARG;
+    if (B == 0 || H == 0 || S == 0) return FA_OK;  // empty problem
+    const int64_t BH = (int64_t)B * H;
+    if (BH > INT_MAX || BH * (int64_t)S > INT_MAX) return FA_ERR_SHAPE;
+    if (!q || !k || !v || !o || !lse) return FA_ERR_NULL;
+    const uintptr_t a16 = (uintptr_t)q | (uintptr_t)k | (uintptr_t)v | (uintptr_t)o;
+    if ((a16 & 15u) != 0 || ((uintptr_t)lse & 3u) != 0) return FA_ERR_ALIGN;
+
+    DeviceInfo dev;
+    int rc = device_info(&dev);
+    if (rc != FA_OK) return rc;
+    if (dev.major != 10 || dev.minor != 0) return FA_ERR_ARCH;
+    int cur = 0;
+    cudaGetDevice(&cur);
+    const void* ptrs[5] = {q, k, v, o, lse};
+    for (const void* p : ptrs) {
+        rc = check_device_pointer(p, cur);
+        if (rc != FA_OK) return rc;
+    }
+    const int64_t units = fa::num_units(BH, S);
+    const int grid = (int)(units < dev.sms ? units : dev.sms);
+    // the counter is read back as an int: the claims of all CTAs must fit
+    if (units + grid > fa::NOALLOC_MAX_CLAIMS) return FA_ERR_SHAPE;
+
+    fa::LaunchArgs a;
+    std::memset(&a, 0, sizeof(a));
+    if (!encode_bhsd(&a.tmap_q, q, (int)BH, S, D, dtype) || !encode_bhsd(&a.tmap_k, k, (int)BH, S, D, dtype) ||
+        !encode_bhsd(&a.tmap_v, v, (int)BH, S, D, dtype))
+        return FA_ERR_LAUNCH;
+    a.o = o;
+    a.lse = lse;
+    a.BH = (int)BH;
+    a.S = S;
+    a.D = D;
+    a.dtype = dtype;
+    a.causal = causal;
+    a.scale_log2 = (float)((double)scale * 1.4426950408889634074);  // scale * log2(e)
+    a.grid = grid;
+    a.sched = nullptr;
+    if (causal) {
+        unsigned int* scratch = nullptr;
+        if (fa::noalloc_scratch_address(&scratch) != cudaSuccess) {
+            cudaGetLastError();
+            return FA_ERR_LAUNCH;
+        }
+        // the array keeps the previous call's counter: clear it on this stream
+        if (cudaMemsetAsync(scratch, 0, sizeof(unsigned int), stream) != cudaSuccess) {
+            cudaGetLastError();
+            return FA_ERR_LAUNCH;
+        }
+        a.sched = scratch;
+    }
+    if (fa::launch_fwd_sm100(a, stream) != cudaSuccess) {
+        cudaGetLastError();
+        return FA_ERR_LAUNCH;
+    }
+    if (cudaPeekAtLastError() != cudaSuccess) {
+        cudaGetLastError();
+        return FA_ERR_LAUNCH;
+    }
+    return FA_OK;
+}
+
 int fa_check_status(cudaStream_t stream) {
     int st = 0, site = 0;
     if (fa::read_and_clear_status(stream, &st, &site) != cudaSuccess) {

@@ -51,12 +51,20 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <mutex>
+
 #include "fa_internal.h"
 
 namespace fa {
 
 __device__ int g_status = 0;       // first error code, 0 if none
 __device__ int g_status_site = 0;  // (site) | (block << 8) of the first failing wait
+
+// Scratch of fa_fwd_noalloc, for callers that cannot allocate device memory:
+// a fixed 256-byte array in the library's own device memory (every GPU that
+// loads the library holds it until the process exits).  Word 0 is the causal
+// work-unit counter.  All fa_fwd_noalloc calls share it.
+static __device__ __align__(256) unsigned int g_noalloc_scratch[NOALLOC_SCRATCH_WORDS];
 
 namespace {
 
@@ -1092,6 +1100,26 @@ cudaError_t launch_selftest_timeout(cudaStream_t stream) {
     // about 50 ms at the maximum SM clock
     selftest_timeout_kernel<<<1, 64, 0, stream>>>(100000000ll);
     return cudaGetLastError();
+}
+
+cudaError_t noalloc_scratch_address(unsigned int** out) {
+    // The array's name in host code is only a stand-in; the device address is
+    // looked up once per device, with that device current.
+    static std::mutex mu;
+    static unsigned int* addr[64] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!addr[dev]) {
+        void* ptr = nullptr;
+        e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+        if (e != cudaSuccess) return e;
+        addr[dev] = static_cast<unsigned int*>(ptr);
+    }
+    *out = addr[dev];
+    return cudaSuccess;
 }
 
 cudaError_t read_and_clear_status(cudaStream_t stream, int* status, int* site) {

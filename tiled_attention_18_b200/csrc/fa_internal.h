@@ -45,6 +45,16 @@ inline int64_t num_units(int64_t BH, int64_t S) {
 // Launch the persistent forward kernel on `stream`.  Returns a cudaError_t.
 cudaError_t launch_fwd_sm100(const LaunchArgs& a, cudaStream_t stream);
 
+// fa_fwd_noalloc: size of its static scratch array (256 bytes; word 0 is the
+// causal unit counter) and the largest number of unit claims the counter
+// serves (work units + CTAs, read back as a non-negative int).
+constexpr int NOALLOC_SCRATCH_WORDS = 64;
+constexpr long long NOALLOC_MAX_CLAIMS = 0x7FFFFFFFll;
+
+// Device address of the static scratch array on the current device (looked
+// up once per device).
+cudaError_t noalloc_scratch_address(unsigned int** out);
+
 // Launch the diagnostic kernel whose first wait is never satisfied.
 cudaError_t launch_selftest_timeout(cudaStream_t stream);
 
