@@ -462,15 +462,30 @@ struct Unit {
     int N;       // key tiles streamed for the unit
 };
 
+// Causal units are ordered longest first within groups of CAUSAL_HEAD_GROUP
+// heads (0: one group of all heads): the K/V of the heads that CTAs work on at
+// the same time then fit in L2 (8 heads x 2 x S x D x 2 bytes = 64 MiB at
+// S = 16384, D = 128) while claimed scheduling keeps the makespan balanced.
+constexpr int CAUSAL_HEAD_GROUP = 8;
+
 // Work-unit order: with the causal mask, longest units first (query block
-// descending), heads innermost; without it, heads outermost so that CTAs
-// running together share one head's K/V in L2.
+// descending) within head groups, heads innermost; without it, heads
+// outermost so that CTAs running together share one head's K/V in L2.
 __device__ __forceinline__ Unit decode_unit(const KParams& p, int u) {
     Unit U;
     int mb;
     if (p.causal) {
-        mb = p.n_mblk - 1 - u / p.BH;
-        U.bh = u % p.BH;
+        if (CAUSAL_HEAD_GROUP > 0 && p.BH > CAUSAL_HEAD_GROUP) {
+            const int per_group = CAUSAL_HEAD_GROUP * p.n_mblk;
+            const int g = u / per_group;
+            const int within = u - g * per_group;
+            const int gh = min(CAUSAL_HEAD_GROUP, p.BH - g * CAUSAL_HEAD_GROUP);  // heads in this group
+            mb = p.n_mblk - 1 - within / gh;
+            U.bh = g * CAUSAL_HEAD_GROUP + within % gh;
+        } else {
+            mb = p.n_mblk - 1 - u / p.BH;
+            U.bh = u % p.BH;
+        }
     } else {
         U.bh = u / p.n_mblk;
         mb = u % p.n_mblk;
