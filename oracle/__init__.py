@@ -19,8 +19,12 @@ ctypes.  Function-level citations are in the C file's header:
   page, "Causal Mask的实现差异", mode 2).
 - ``attn_probs`` : the softmax matrix P of one head (tiny sizes).
 - ``causal_tile_count`` : element-wise enumeration of computed/skipped tile pairs.
+- ``attn_fwd_gen`` / ``attn_rows_gen`` : the same definition with Sq queries and
+  Sk keys (cross-attention) and the causal mask aligned to the last Sq keys.
 
-Parity pins: every function above is pinned by tests in tests/test_oracle.py.
+Parity pins: every function above is pinned by tests in tests/test_oracle.py and
+tests/test_oracle_general.py (torch SDPA in float64 with an explicit mask, the
+Q = 0 closed form, agreement with attn_fwd when Sq = Sk).
 """
 from __future__ import annotations
 
@@ -82,6 +86,12 @@ def _load():
                                           ctypes.c_int, ctypes.c_int, i64, i64, ctypes.c_int,
                                           f64p, f64p]
         lib.oracle_attn_tiled.restype = ctypes.c_int
+        lib.oracle_attn_fwd_gen.argtypes = [u16p, u16p, u16p, i64, i64, i64, i64, i64, ctypes.c_float,
+                                            ctypes.c_int, ctypes.c_int, f64p, f64p]
+        lib.oracle_attn_fwd_gen.restype = ctypes.c_int
+        lib.oracle_attn_rows_gen.argtypes = [u16p, u16p, u16p, i64, i64, i64, i64, i64, ctypes.c_float,
+                                             ctypes.c_int, ctypes.c_int, i64p, i64p, i64, f64p, f64p]
+        lib.oracle_attn_rows_gen.restype = ctypes.c_int
         lib.oracle_causal_tile_count.argtypes = [i64, i64, i64, i64p, i64p, i64p]
         lib.oracle_causal_tile_count.restype = None
         lib.oracle_num_threads.argtypes = []
@@ -159,6 +169,47 @@ def attn_rows(q, k, v, scale: float, causal: bool, dtype, bh_idx, row_idx):
                               _ptr(o, ctypes.c_double), _ptr(lse, ctypes.c_double))
     if rc != 0:
         raise RuntimeError(f"oracle_attn_rows failed with {rc}")
+    return o, lse
+
+
+def attn_fwd_gen(q, k, v, scale: float, causal: bool, dtype):
+    """Naive fp64 attention with Sq = q.shape[2] queries and Sk = k.shape[2] keys
+    (contiguous BHSD); causal means query i sees keys j <= i + Sk - Sq."""
+    lib = _load()
+    qb, kb, vb = _bits(q), _bits(k), _bits(v)
+    B, H, Sq, D = qb.shape
+    Sk = kb.shape[2]
+    if kb.shape != (B, H, Sk, D) or vb.shape != kb.shape:
+        raise ValueError("k and v must be [B, H, Sk, D] with q's B, H, D")
+    o = np.empty((B, H, Sq, D), dtype=np.float64)
+    lse = np.empty((B, H, Sq), dtype=np.float64)
+    rc = lib.oracle_attn_fwd_gen(_ptr(qb, ctypes.c_uint16), _ptr(kb, ctypes.c_uint16),
+                                 _ptr(vb, ctypes.c_uint16), B, H, Sq, Sk, D, float(np.float32(scale)),
+                                 int(bool(causal)), _dtype_code(dtype),
+                                 _ptr(o, ctypes.c_double), _ptr(lse, ctypes.c_double))
+    if rc != 0:
+        raise RuntimeError(f"oracle_attn_fwd_gen failed with {rc}")
+    return o, lse
+
+
+def attn_rows_gen(q, k, v, scale: float, causal: bool, dtype, bh_idx, row_idx):
+    """attn_fwd_gen for selected (bh, query row) pairs. Returns (O [n,D], LSE [n])."""
+    lib = _load()
+    qb, kb, vb = _bits(q), _bits(k), _bits(v)
+    B, H, Sq, D = qb.shape
+    Sk = kb.shape[2]
+    bh = np.ascontiguousarray(bh_idx, dtype=np.int64)
+    ri = np.ascontiguousarray(row_idx, dtype=np.int64)
+    n = bh.size
+    o = np.empty((n, D), dtype=np.float64)
+    lse = np.empty((n,), dtype=np.float64)
+    rc = lib.oracle_attn_rows_gen(_ptr(qb, ctypes.c_uint16), _ptr(kb, ctypes.c_uint16),
+                                  _ptr(vb, ctypes.c_uint16), B, H, Sq, Sk, D, float(np.float32(scale)),
+                                  int(bool(causal)), _dtype_code(dtype),
+                                  _ptr(bh, ctypes.c_int64), _ptr(ri, ctypes.c_int64), n,
+                                  _ptr(o, ctypes.c_double), _ptr(lse, ctypes.c_double))
+    if rc != 0:
+        raise RuntimeError(f"oracle_attn_rows_gen failed with {rc}")
     return o, lse
 
 

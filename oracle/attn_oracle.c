@@ -403,3 +403,123 @@ int oracle_num_threads(void)
     return 1;
 #endif
 }
+
+/* -------------------------------------------- general shapes (Sq != Sk) */
+
+/*
+ * Cross-attention and offset causal masking: queries [B,H,Sq,D], keys and
+ * values [B,H,Sk,D] (contiguous).  With the causal mask query i sees key j iff
+ * j <= i + (Sk - Sq): the queries are the last Sq positions of the Sk keys
+ * (bottom-right alignment; with Sq = Sk this is the mask above).  A query that
+ * sees no key gets O = 0 and LSE = -inf (the log of an empty sum).
+ * Same definition as oracle_attn_fwd otherwise.  Sources: text-to-image
+ * cross-attention with 77 text tokens ("解析CANN ops-transformer的FlashAttention
+ * 算子：注意力机制的内存优化", section "Stable Diffusion中的优化"); the causal
+ * mask as in oracle_attn_fwd.  The pages do not say how a causal mask aligns
+ * when Sq != Sk; the bottom-right reading (queries are the newest positions,
+ * as in decoding with a cache) is taken.
+ */
+static void naive_row_gen(const double *qi, const double *kh, const double *vh, int64_t nj, int64_t D,
+                          double scale, double *srow, double *o, double *lse)
+{
+    if (nj <= 0) {
+        for (int64_t d = 0; d < D; ++d) o[d] = 0.0;
+        *lse = -INFINITY;
+        return;
+    }
+    for (int64_t j = 0; j < nj; ++j) {
+        double dot = 0.0;
+        for (int64_t d = 0; d < D; ++d) dot += qi[d] * kh[j * D + d];
+        srow[j] = scale * dot;
+    }
+    double m = -INFINITY;
+    for (int64_t j = 0; j < nj; ++j)
+        if (srow[j] > m) m = srow[j];
+    double l = 0.0;
+    for (int64_t j = 0; j < nj; ++j) {
+        srow[j] = exp(srow[j] - m);
+        l += srow[j];
+    }
+    for (int64_t d = 0; d < D; ++d) o[d] = 0.0;
+    for (int64_t j = 0; j < nj; ++j)
+        for (int64_t d = 0; d < D; ++d) o[d] += srow[j] * vh[j * D + d];
+    for (int64_t d = 0; d < D; ++d) o[d] /= l;
+    *lse = m + log(l);
+}
+
+static int64_t visible_keys(int64_t i, int64_t Sq, int64_t Sk, int causal)
+{
+    if (!causal) return Sk;
+    int64_t n = i + (Sk - Sq) + 1;
+    if (n < 0) n = 0;
+    if (n > Sk) n = Sk;
+    return n;
+}
+
+int oracle_attn_fwd_gen(const uint16_t *q, const uint16_t *k, const uint16_t *v, int64_t B, int64_t H,
+                        int64_t Sq, int64_t Sk, int64_t D, float scale, int causal, int dtype, double *o,
+                        double *lse)
+{
+    if (B < 0 || H < 0 || Sq < 0 || Sk < 0 || D <= 0) return -2;
+    if (dtype != ORACLE_F16 && dtype != ORACLE_BF16) return -4;
+    const double sc = (double)scale;
+    for (int64_t bh = 0; bh < B * H; ++bh) {
+        double *qh = (double *)malloc(sizeof(double) * (size_t)(Sq * D > 0 ? Sq * D : 1));
+        double *kh = (double *)malloc(sizeof(double) * (size_t)(Sk * D > 0 ? Sk * D : 1));
+        double *vh = (double *)malloc(sizeof(double) * (size_t)(Sk * D > 0 ? Sk * D : 1));
+        if (!qh || !kh || !vh) { free(qh); free(kh); free(vh); return -10; }
+        oracle_decode(q + bh * Sq * D, qh, Sq * D, dtype);
+        oracle_decode(k + bh * Sk * D, kh, Sk * D, dtype);
+        oracle_decode(v + bh * Sk * D, vh, Sk * D, dtype);
+#pragma omp parallel
+        {
+            double *srow = (double *)malloc(sizeof(double) * (size_t)(Sk > 0 ? Sk : 1));
+#pragma omp for schedule(dynamic, 16)
+            for (int64_t i = 0; i < Sq; ++i)
+                naive_row_gen(qh + i * D, kh, vh, visible_keys(i, Sq, Sk, causal), D, sc, srow,
+                              o + (bh * Sq + i) * D, lse + bh * Sq + i);
+            free(srow);
+        }
+        free(qh); free(kh); free(vh);
+    }
+    return 0;
+}
+
+/* The general definition for a list of (bh, i) query rows only. */
+int oracle_attn_rows_gen(const uint16_t *q, const uint16_t *k, const uint16_t *v, int64_t B, int64_t H,
+                         int64_t Sq, int64_t Sk, int64_t D, float scale, int causal, int dtype,
+                         const int64_t *bh_idx, const int64_t *row_idx, int64_t nrows, double *o, double *lse)
+{
+    if (B < 0 || H < 0 || Sq < 0 || Sk < 0 || D <= 0) return -2;
+    if (dtype != ORACLE_F16 && dtype != ORACLE_BF16) return -4;
+    for (int64_t r = 0; r < nrows; ++r)
+        if (bh_idx[r] < 0 || bh_idx[r] >= B * H || row_idx[r] < 0 || row_idx[r] >= Sq) return -2;
+    const double sc = (double)scale;
+    int bad = 0;
+#pragma omp parallel
+    {
+        double *srow = (double *)malloc(sizeof(double) * (size_t)(Sk > 0 ? Sk : 1));
+        double *qi = (double *)malloc(sizeof(double) * (size_t)D);
+        double *kh = (double *)malloc(sizeof(double) * (size_t)(Sk * D > 0 ? Sk * D : 1));
+        double *vh = (double *)malloc(sizeof(double) * (size_t)(Sk * D > 0 ? Sk * D : 1));
+        int64_t cur_bh = -1;
+        if (!srow || !qi || !kh || !vh) {
+#pragma omp atomic write
+            bad = 1;
+        }
+#pragma omp for schedule(static)
+        for (int64_t r = 0; r < nrows; ++r) {
+            if (!srow || !qi || !kh || !vh) continue;
+            int64_t bh = bh_idx[r], i = row_idx[r];
+            if (bh != cur_bh) {
+                oracle_decode(k + bh * Sk * D, kh, Sk * D, dtype);
+                oracle_decode(v + bh * Sk * D, vh, Sk * D, dtype);
+                cur_bh = bh;
+            }
+            oracle_decode(q + (bh * Sq + i) * D, qi, D, dtype);
+            naive_row_gen(qi, kh, vh, visible_keys(i, Sq, Sk, causal), D, sc, srow, o + r * D, lse + r);
+        }
+        free(srow); free(qi); free(kh); free(vh);
+    }
+    return bad ? -10 : 0;
+}
