@@ -1,13 +1,19 @@
 """Benchmark of the fused attention forward pass on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl fa|reference]
-                    [--workload c5|c1|c2|c3|c4|c5a|c5b] [--no-e2e] [--no-cpu-baseline]
+                    [--workload c5|c1|c2|c3|c4|c5a|c5b|sdxl_xattn|bert_large|prefill_cached]
+                    [--no-e2e] [--no-cpu-baseline]
 
 A step is one pass of the whole forward path over one batch of synthetic
 input.  The default workload is the long-context configuration
 B=1, H=32, S=16384, D=128, bf16, run both without and with the causal mask
 (two fa_fwd launches per step).  Inputs (512 MiB) are larger than the 126 MB
 L2, so no L2 flush is needed between steps.
+
+The general-shape workloads (sdxl_xattn: 4096 queries over 77 keys;
+bert_large: B=32, H=16, S=512, D=64 in the BSHD layout; prefill_cached:
+4096 causal queries over 16384 keys) run through fa_fwd_ex; their inputs are
+rotated over enough copies that one rotation touches more than twice the L2.
 
 Throughput is attention TFLOP/s with the causal case counted at half
 (4*B*H*S^2*D per non-causal run), over the whole job: with N GPUs (one
@@ -22,6 +28,7 @@ same workload (rank 0 only) and prints the same JSON line with
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import json
 import os
 import subprocess
@@ -36,7 +43,8 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 from tiled_attention_18_b200.scaling import job_throughput, max_over_ranks, rank_env, rank_seed  # noqa: E402
-from tiled_attention_18_b200.workloads import WORKLOADS, make_inputs, sample_rows  # noqa: E402
+from tiled_attention_18_b200.workloads import (GENERAL_WORKLOADS, WORKLOADS, sample_rows,  # noqa: E402
+                                               workload_inputs)
 
 METRIC = "attention fwd TFLOPS (causal-adjusted) and % of B200 dense fp16/bf16 peak"
 UNIT = "TFLOP/s"
@@ -44,13 +52,15 @@ FALLBACK_BF16_TFLOPS = 1590.0
 PEAKS_PATH = os.path.join(ROOT, "MEASURED_PEAKS.json")
 TRAFFIC_PATH = os.path.join(ROOT, "profiles", "fa_fwd_traffic.json")
 KERNEL_SRC = os.path.join(ROOT, "tiled_attention_18_b200", "csrc", "fa_fwd_sm100.cu")
+L2_BYTES = 126 * 1024 * 1024
+ALL_WORKLOADS = {**WORKLOADS, **GENERAL_WORKLOADS}
 
 
 def workload_runs(name: str):
     """The fa_fwd runs of one step: (Workload, ...)."""
     if name == "c5":
         return [WORKLOADS["c5a"], WORKLOADS["c5b"]]
-    return [WORKLOADS[name]]
+    return [ALL_WORKLOADS[name]]
 
 
 def workload_label(name: str) -> str:
@@ -58,6 +68,9 @@ def workload_label(name: str) -> str:
     w = runs[0]
     causal = "non-causal + causal" if len(runs) == 2 else ("causal" if w.causal else "non-causal")
     extra = f", Q,K x{w.qk_mult:g}" if w.qk_mult != 1.0 else ""
+    if w.general:
+        lay = f", {w.layout.upper()} layout" if w.layout != "bhsd" else ""
+        return f"attention fwd {w.dtype} B={w.B} H={w.H} Sq={w.S} Sk={w.Skv} D={w.D}, {causal}{extra}{lay}"
     return f"attention fwd {w.dtype} B={w.B} H={w.H} S={w.S} D={w.D}, {causal}{extra}"
 
 
@@ -76,12 +89,12 @@ def kernel_source_hash() -> str:
         return hashlib.sha256(f.read()).hexdigest()[:16]
 
 
-def traffic_per_launch():
-    """DRAM bytes per launch from the committed ncu summary, if taken on this kernel source."""
+def traffic_per_launch(workload: str):
+    """DRAM bytes per step from the committed ncu summary, if taken on this kernel source and workload."""
     try:
         with open(TRAFFIC_PATH) as f:
             t = json.load(f)
-        if t.get("kernel_source_sha256_16") != kernel_source_hash():
+        if t.get("kernel_source_sha256_16") != kernel_source_hash() or t.get("workload_key", "c5") != workload:
             return None
         return float(t["dram_bytes_per_step"])
     except Exception:
@@ -153,18 +166,21 @@ def cpu_baseline(name: str, target_s: float = 12.0):
     flops_total, t_total, rows_total = 0.0, 0.0, 0
     desc = []
     for w in runs:
-        q, k, v = make_inputs(w.B, w.H, w.S, w.D, w.dtype, w.qk_mult, w.seed)
+        q, k, v = workload_inputs(w)
         # rows of the sample: random rows over all heads; cost per row = 4*D*(keys seen)
         n = 64
         while True:
             bh, rows = sample_rows(w.B, w.H, w.S, n_random=n, edge=0, seed=99)
             t0 = time.perf_counter()
-            oracle.attn_rows(q, k, v, w.scale, w.causal, w.dtype, bh, rows)
+            if w.general:
+                oracle.attn_rows_gen(q, k, v, w.scale, w.causal, w.dtype, bh, rows)
+            else:
+                oracle.attn_rows(q, k, v, w.scale, w.causal, w.dtype, bh, rows)
             dt = time.perf_counter() - t0
             if dt >= per_run_s * 0.5 or n >= (1 << 20):
                 break
             n = int(n * min(16.0, max(2.0, per_run_s / max(dt, 1e-3))))
-        keys = (rows + 1) if w.causal else np.full_like(rows, w.S)
+        keys = np.minimum(rows + (w.Skv - w.S) + 1, w.Skv) if w.causal else np.full_like(rows, w.Skv)
         flops = float(4.0 * w.D * keys.sum())
         flops_total += flops
         t_total += dt
@@ -207,7 +223,7 @@ def main(argv=None) -> int:
     ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["fa", "reference"], default="fa")
-    ap.add_argument("--workload", default="c5", choices=["c5"] + list(WORKLOADS))
+    ap.add_argument("--workload", default="c5", choices=["c5"] + list(ALL_WORKLOADS))
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -240,34 +256,56 @@ def main(argv=None) -> int:
     stream = torch.cuda.current_stream(dev)
     sid = stream.cuda_stream
 
-    # inputs: each rank draws its own independent batch (seed = workload seed + rank)
-    host_in, dev_in, dev_out = [], [], []
+    # inputs: each rank draws its own independent batch (seed = workload seed + rank).
+    # Each tensor is held as "storage" contiguous in the workload's layout
+    # (BHSD, or BSHD read through a transposed view); inputs smaller than twice
+    # the L2 are rotated over several device copies so that every step reads
+    # them from DRAM.
+    def storage(w, t):
+        return t.contiguous() if w.layout == "bhsd" else t.transpose(1, 2).contiguous()
+
+    def view(w, t):
+        return t if w.layout == "bhsd" else t.transpose(1, 2)
+
+    host_in, dev_in, dev_out, n_copies = [], [], [], []
     for i, w in enumerate(runs):
-        if i > 0 and (w.B, w.H, w.S, w.D, w.dtype, w.qk_mult) == (runs[0].B, runs[0].H, runs[0].S, runs[0].D,
-                                                                   runs[0].dtype, runs[0].qk_mult):
+        if i > 0 and not w.general and (w.B, w.H, w.S, w.D, w.dtype, w.qk_mult) == (
+                runs[0].B, runs[0].H, runs[0].S, runs[0].D, runs[0].dtype, runs[0].qk_mult):
             host_in.append(host_in[0])
             dev_in.append(dev_in[0])
+            n_copies.append(n_copies[0])
         else:
-            q, k, v = make_inputs(w.B, w.H, w.S, w.D, w.dtype, w.qk_mult, rank_seed(w.seed, rank))
+            wr = dataclasses.replace(w, seed=rank_seed(w.seed, rank))
+            q, k, v = (storage(w, t) for t in workload_inputs(wr))
+            set_bytes = sum(t.numel() * t.element_size() for t in (q, k, v))
+            copies = 1 if set_bytes >= 2 * L2_BYTES else min(64, -(-2 * L2_BYTES // set_bytes))
             host_in.append(tuple(t.pin_memory() for t in (q, k, v)))
-            dev_in.append(tuple(t.to(dev) for t in (q, k, v)))
-        o = torch.empty((w.B, w.H, w.S, w.D), dtype=w.torch_dtype, device=dev)
+            dev_in.append([tuple(t.to(dev) for t in (q, k, v)) for _ in range(copies)])
+            n_copies.append(copies)
+        o = storage(w, torch.empty((w.B, w.H, w.S, w.D), dtype=w.torch_dtype)).to(dev)
         lse = torch.empty((w.B, w.H, w.S), dtype=torch.float32, device=dev)
         dev_out.append((o, lse))
 
-    def launch(i):
+    def launch(i, step=0):
         w = runs[i]
-        q, k, v = dev_in[i]
+        q, k, v = (view(w, t) for t in dev_in[i][step % n_copies[i]])
         o, lse = dev_out[i]
-        st = fa.fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), w.B, w.H, w.S, w.D,
-                       w.scale, int(w.causal), fa.FA_BF16 if w.dtype == "bf16" else fa.FA_FP16, sid)
+        o = view(w, o)
+        dt = fa.FA_BF16 if w.dtype == "bf16" else fa.FA_FP16
+        if w.general:
+            st = fa.fa_fwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), w.B, w.H, w.S,
+                              w.Skv, w.D, q.stride()[:3], k.stride()[:3], v.stride()[:3], o.stride()[:3], w.scale,
+                              int(w.causal), dt, sid)
+        else:
+            st = fa.fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), w.B, w.H, w.S,
+                           w.D, w.scale, int(w.causal), dt, sid)
         if st != 0:
             raise fa.FaError(st)
 
     # warm-up
-    for _ in range(args.warmup):
+    for s_ in range(args.warmup):
         for i in range(len(runs)):
-            launch(i)
+            launch(i, s_)
     torch.cuda.synchronize(dev)
     st = fa.fa_check_status(sid)
     if st != 0:
@@ -286,7 +324,7 @@ def main(argv=None) -> int:
     for s in range(args.steps):
         for i in range(len(runs)):
             ev[s][i][0].record(stream)
-            launch(i)
+            launch(i, s)
             ev[s][i][1].record(stream)
     stop.record(stream)
     torch.cuda.synchronize(dev)
@@ -308,7 +346,7 @@ def main(argv=None) -> int:
         mean_ms = float(kern_ms[:, i].mean())
         per_run.append({"run": w.describe(), "mean_ms": mean_ms, "tflops": w.flops / (mean_ms * 1e-3) / 1e12})
     achieved = step_flops / (float(kern_ms.sum(axis=1).mean()) * 1e-3) / 1e12
-    traffic = traffic_per_launch()
+    traffic = traffic_per_launch(args.workload)
 
     # end to end through the public call with host buffers
     e2e = None
@@ -322,7 +360,7 @@ def main(argv=None) -> int:
         def e2e_step():
             for i, w in enumerate(runs):
                 if i == 0 or host_in[i] is not host_in[0]:
-                    for hsrc, dsrc in zip(host_in[i], dev_in[i]):
+                    for hsrc, dsrc in zip(host_in[i], dev_in[i][0]):
                         dsrc.copy_(hsrc, non_blocking=True)
                 launch(i)
                 dev_out_o, dev_out_l = dev_out[i]
@@ -354,7 +392,10 @@ def main(argv=None) -> int:
             "warmup": args.warmup, "ms_per_step": max_ms / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": w0.dtype, "data": "synthetic",
             "config": {"workload": workload_label(args.workload), "B": w0.B, "H": w0.H, "S": w0.S, "D": w0.D,
-                       "runs_per_step": len(runs), "l2": "inputs larger than L2 (no flush)",
+                       **({"Sk": w0.Skv, "layout": w0.layout} if w0.general else {}),
+                       "runs_per_step": len(runs),
+                       "l2": ("inputs larger than L2 (no flush)" if max(n_copies) == 1 else
+                              f"inputs rotated over {max(n_copies)} device copies (> 2x L2 per rotation, no flush)"),
                        "parallelism": f"independent batch per GPU x{world}"},
             "pct_of_peak": 100.0 * value / (peak * world),
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": UNIT,

@@ -2,8 +2,8 @@
  * fa.h -- C ABI of libfa.so: fused attention forward (FlashAttention-2 style)
  * for NVIDIA B200 (sm_100a).
  *
- * The operation, per batch b, head h and query row i of contiguous BHSD
- * tensors:
+ * The operation, per batch b, head h and query row i of BHSD tensors
+ * (contiguous for fa_fwd; any b, h, s strides and Sq != Sk for fa_fwd_ex):
  *
  *   O[b,h,i,:]  = sum_j softmax_j( scale * Q[b,h,i,:] . K[b,h,j,:] ) * V[b,h,j,:]
  *   LSE[b,h,i]  = log( sum_j exp( scale * Q[b,h,i,:] . K[b,h,j,:] ) )   (natural log)
@@ -59,7 +59,9 @@ typedef enum {
     FA_ERR_TIMEOUT = -8,  /* a device-side wait exceeded its bound (reported by fa_check_status) */
     FA_ERR_SCALE = -9,    /* scale is not finite and > 0 */
     FA_ERR_ARG = -10,     /* causal is not 0 or 1 */
-    FA_ERR_PTR = -11      /* a pointer is not device memory of the current device */
+    FA_ERR_PTR = -11,     /* a pointer is not device memory of the current device */
+    FA_ERR_STRIDE = -12   /* fa_fwd_ex: a stride is negative, zero over an extent > 1, not a
+                             multiple of 8 elements (16 bytes), or not below 2^36 elements */
 } fa_status;
 
 /*
@@ -117,6 +119,44 @@ FA_API int fa_fwd(const void* q, const void* k, const void* v, void* o, float* l
  */
 FA_API int fa_fwd_noalloc(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
                           int S, int D, float scale, int causal, int dtype, cudaStream_t stream);
+
+/*
+ * fa_fwd_ex -- fa_fwd for general shapes: Sq queries and Sk keys per head
+ * (cross-attention, e.g. image tokens attending to 77 text tokens:
+ * "解析CANN ops-transformer的FlashAttention算子：注意力机制的内存优化",
+ * section "Stable Diffusion中的优化") and tensors at arbitrary b, h, s strides,
+ * so that [batch, seq_len, heads, head_dim] (BSHD) data is read in place
+ * instead of being transposed and copied first (the layout pitfall of the
+ * gsyq.cn catlass FlashAttention page, section on data layout).
+ *
+ *   O[b,h,i,:] = sum_j softmax_j( scale * Q[b,h,i,:] . K[b,h,j,:] ) * V[b,h,j,:]
+ *
+ * with j over [0, Sk); with causal = 1, j over [0, i + Sk - Sq]: the queries
+ * are the last Sq of the Sk positions (bottom-right alignment; with Sq = Sk
+ * this is fa_fwd's mask).  The pages do not say how the mask aligns when
+ * Sq != Sk; this is the reading taken.
+ *
+ * q       : [B, H, Sq, D] elements at q_stride; k, v : [B, H, Sk, D] at
+ *           k_stride, v_stride; o : [B, H, Sq, D] at o_stride.  Each *_stride
+ *           is a host array of 3 element strides for the b, h and s
+ *           dimensions (d is contiguous), or NULL for the contiguous BHSD
+ *           layout of that shape.  A stride over an extent of 1 is ignored.
+ *           Every other stride must be > 0, a multiple of 8 elements (16
+ *           bytes) and below 2^36 elements (else FA_ERR_STRIDE).  o must not
+ *           overlap itself, q, k, v or lse.
+ * lse     : [B, H, Sq] contiguous fp32 (natural log).  Required.
+ * B, H, Sq: B, H or Sq 0 is an empty problem (FA_OK, nothing launched,
+ *           pointers not inspected).  Sk must be >= 1, and >= Sq when
+ *           causal = 1 (else FA_ERR_SHAPE: some query would see no key).
+ *           B*H*Sq must fit in 31 bits and Sq, Sk must stay below 2^31 - 512.
+ * D, scale, causal, dtype, stream, ownership, scheduler scratch, errors:
+ *           as fa_fwd.  fa_fwd(q, k, v, o, lse, B, H, S, D, ...) computes the
+ *           same as fa_fwd_ex with Sq = Sk = S and NULL strides.
+ */
+FA_API int fa_fwd_ex(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Sq,
+                     int Sk, int D, const long long* q_stride, const long long* k_stride,
+                     const long long* v_stride, const long long* o_stride, float scale, int causal, int dtype,
+                     cudaStream_t stream);
 
 /*
  * fa_check_status -- synchronise `stream`, then report and clear the device

@@ -56,3 +56,40 @@ def compare(o_gpu: torch.Tensor, lse_gpu: torch.Tensor, o_ref: np.ndarray, lse_r
     assert lse_err <= LSE_TOL, f"max |dLSE| {lse_err:.3g} > {LSE_TOL}"
     return {"max_abs_o": max_err, "max_abs_o_representable": max_err_repr, "n_below_floor": n_floor,
             "max_abs_lse": lse_err}
+
+
+def run_fa_ex(q, k, v, scale: float, causal: bool, layouts=("bhsd", "bhsd", "bhsd", "bhsd"), o_pad: int = 0):
+    """fa_fwd_ex through the C ABI on CPU BHSD inputs placed on the GPU in the
+    given layouts (q, k, v, o: "bhsd" | "bshd").  ``o_pad`` > 0 writes O into a
+    view of a wider NaN-filled buffer (rows o_pad elements apart from the next
+    row's start beyond D) and checks that the gaps stay NaN.
+    Returns CPU (O contiguous BHSD, LSE)."""
+    from tiled_attention_18_b200.workloads import to_layout
+    B, H, Sq, D = q.shape
+    Sk = k.shape[2]
+    dq, dk, dv = (to_layout(t, lay).to("cuda") if lay == "bhsd" else
+                  t.transpose(1, 2).contiguous().to("cuda").transpose(1, 2)
+                  for t, lay in zip((q, k, v), layouts[:3]))
+    if o_pad:
+        if layouts[3] == "bhsd":
+            buf = torch.full((B, H, Sq, D + o_pad), float("nan"), dtype=q.dtype, device="cuda")
+            o = buf[..., :D]
+        else:
+            buf = torch.full((B, Sq, H, D + o_pad), float("nan"), dtype=q.dtype, device="cuda")
+            o = buf[..., :D].transpose(1, 2)
+    else:
+        shape = (B, H, Sq, D) if layouts[3] == "bhsd" else (B, Sq, H, D)
+        buf = torch.full(shape, float("nan"), dtype=q.dtype, device="cuda")
+        o = buf if layouts[3] == "bhsd" else buf.transpose(1, 2)
+    lse = torch.full((B, H, Sq), float("nan"), dtype=torch.float32, device="cuda")
+    st = torch.cuda.current_stream().cuda_stream
+    dt = fa.FA_BF16 if q.dtype == torch.bfloat16 else fa.FA_FP16
+    rc = fa.fa_fwd_ex(dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), o.data_ptr(), lse.data_ptr(), B, H, Sq, Sk, D,
+                      dq.stride()[:3], dk.stride()[:3], dv.stride()[:3], o.stride()[:3], scale, int(causal), dt, st)
+    assert rc == 0, f"fa_fwd_ex returned {rc} ({fa.fa_status_string(rc)})"
+    s = fa.fa_check_status(st)
+    assert s == 0, f"device status {s} ({fa.fa_status_string(s)}), site {fa.fa_last_timeout_site():#x}"
+    torch.cuda.synchronize()
+    if o_pad:
+        assert torch.isnan(buf[..., D:]).all(), "fa_fwd_ex wrote outside O's view"
+    return o.contiguous().cpu(), lse.cpu()

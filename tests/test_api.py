@@ -102,3 +102,44 @@ def test_missing_library_fails_loudly(tmp_path, monkeypatch):
     monkeypatch.setattr(_lib, "_lib", None)
     with pytest.raises(OSError):
         _lib.load()
+
+
+@pytest.mark.parametrize("args,code", [
+    (dict(Sq=-1), _lib.FA_ERR_SHAPE),
+    (dict(Sk=-1), _lib.FA_ERR_SHAPE),
+    (dict(Sk=0), _lib.FA_ERR_SHAPE),                      # a query would see no key
+    (dict(Sq=200, Sk=100, causal=1), _lib.FA_ERR_SHAPE),  # bottom-right mask: first rows see nothing
+    (dict(Sk=(1 << 31) - 100), _lib.FA_ERR_SHAPE),
+    (dict(D=32), _lib.FA_ERR_HEADDIM),
+    (dict(dtype=-1), _lib.FA_ERR_DTYPE),
+    (dict(scale=0.0), _lib.FA_ERR_SCALE),
+    (dict(causal=-1), _lib.FA_ERR_ARG),
+    (dict(v=0), _lib.FA_ERR_NULL),
+    (dict(qs=(128 * 64 * 2, 64, 2 * 64 + 4)), _lib.FA_ERR_STRIDE),   # s stride not 16 bytes
+    (dict(ks=(0, 64, 128)), _lib.FA_ERR_STRIDE),                     # zero over B = 2
+    (dict(vs=(-8, 64, 128)), _lib.FA_ERR_STRIDE),
+    (dict(os=(1 << 36, 64, 128)), _lib.FA_ERR_STRIDE),
+    (dict(k=A + 2), _lib.FA_ERR_ALIGN),
+])
+def test_fa_fwd_ex_invalid_arguments(lib, args, code):
+    a = dict(q=A, k=A, v=A, o=A, lse=A, B=2, H=3, Sq=100, Sk=300, D=64, qs=None, ks=None, vs=None, os=None,
+             scale=0.125, causal=0, dtype=1)
+    a.update(args)
+    st = fa.fa_fwd_ex(a["q"], a["k"], a["v"], a["o"], a["lse"], a["B"], a["H"], a["Sq"], a["Sk"], a["D"],
+                      a["qs"], a["ks"], a["vs"], a["os"], a["scale"], a["causal"], a["dtype"], 0)
+    assert st == code
+
+
+def test_fa_fwd_ex_stride_over_unit_extent_is_ignored(lib):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a device is present")
+    # B = 1 and H = 1: the (invalid) b and h strides are never used; the call
+    # gets past every argument check and stops at the missing device
+    st = fa.fa_fwd_ex(A, A, A, A, A, 1, 1, 64, 64, 64, (3, -5, 64), (0, 0, 64), None, None, 0.125, 1, 0, 0)
+    assert st == _lib.FA_ERR_LAUNCH
+
+
+def test_fa_fwd_ex_empty_problems(lib):
+    for B, H, Sq, Sk in ((0, 2, 10, 10), (1, 0, 10, 10), (1, 2, 0, 10), (1, 2, 0, 0)):
+        assert fa.fa_fwd_ex(0, 0, 0, 0, 0, B, H, Sq, Sk, 64, None, None, None, None, 0.1, 1, 0, 0) == _lib.FA_OK

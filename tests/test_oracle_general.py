@@ -5,13 +5,8 @@ import pytest
 import torch
 
 import oracle
+from tiled_attention_18_b200.workloads import make_cross_inputs as _qkv
 from tiled_attention_18_b200.workloads import make_inputs, softmax_scale
-
-
-def _qkv(B, H, Sq, Sk, D, dtype, seed):
-    q, _, _ = make_inputs(B, H, Sq, D, dtype, seed=seed)
-    _, k, v = make_inputs(B, H, Sk, D, dtype, seed=seed + 1)
-    return q, k, v
 
 
 def _bottom_right_mask(Sq, Sk):

@@ -8,11 +8,11 @@ in Python or PyTorch, and there is no fallback path.
 """
 from __future__ import annotations
 
-from ._lib import (FA_BF16, FA_FP16, FaError, fa_check_status, fa_fwd, fa_fwd_noalloc, fa_last_timeout_site,
-                   fa_num_units, fa_selftest_timeout, fa_status_string, fa_version, load)
+from ._lib import (FA_BF16, FA_FP16, FaError, fa_check_status, fa_fwd, fa_fwd_ex, fa_fwd_noalloc,
+                   fa_last_timeout_site, fa_num_units, fa_selftest_timeout, fa_status_string, fa_version, load)
 
 __all__ = [
-    "FA_BF16", "FA_FP16", "FaError", "fa_check_status", "fa_fwd", "fa_fwd_noalloc", "fa_last_timeout_site",
+    "FA_BF16", "FA_FP16", "FaError", "fa_check_status", "fa_fwd", "fa_fwd_ex", "fa_fwd_noalloc", "fa_last_timeout_site",
     "fa_num_units", "fa_selftest_timeout", "fa_status_string", "fa_version", "flash_attention_forward", "load",
 ]
 
@@ -27,35 +27,50 @@ def _dtype_code(t) -> int:
 
 
 def flash_attention_forward(q, k, v, scale: float, causal: bool = False, out=None, lse=None, stream=None):
-    """O, LSE for contiguous BHSD CUDA tensors ``q, k, v`` ([B, H, S, D], fp16/bf16).
+    """O, LSE for CUDA tensors ``q`` [B, H, Sq, D] and ``k, v`` [B, H, Sk, D] (fp16/bf16).
 
-    ``scale`` is required (commonly 1/sqrt(D)).  ``out``/``lse`` may be given
-    to reuse buffers.  Launches on ``stream`` (default: torch's current
-    stream) and returns without synchronising.
+    The tensors may be any strided views whose last dimension is contiguous
+    (for example ``x.transpose(1, 2)`` of a [B, S, H, D] tensor); b, h and s
+    strides must be multiples of 8 elements.  With ``causal`` query i sees
+    keys j <= i + Sk - Sq (requires Sq <= Sk).  ``scale`` is required
+    (commonly 1/sqrt(D)).  ``out`` (like ``q``, any such strides) and ``lse``
+    (contiguous float32 [B, H, Sq]) may be given to reuse buffers; by default
+    ``out`` takes ``q``'s memory layout.  Launches on ``stream`` (default:
+    torch's current stream) and returns without synchronising.
     """
     import torch
-    if q.dim() != 4 or k.shape != q.shape or v.shape != q.shape:
-        raise ValueError("q, k, v must all be [B, H, S, D] with the same shape")
+    if q.dim() != 4 or k.dim() != 4 or v.shape != k.shape:
+        raise ValueError("q must be [B, H, Sq, D] and k, v [B, H, Sk, D]")
+    B, H, Sq, D = q.shape
+    Sk = k.shape[2]
+    if k.shape[0] != B or k.shape[1] != H or k.shape[3] != D:
+        raise ValueError("k and v must share q's B, H and D")
     if not (q.is_cuda and k.is_cuda and v.is_cuda):
         raise ValueError("q, k, v must be CUDA tensors")
     if k.dtype != q.dtype or v.dtype != q.dtype:
         raise TypeError("q, k, v must share one dtype")
     for name, t in (("q", q), ("k", k), ("v", v)):
-        if not t.is_contiguous():
-            raise ValueError(f"{name} must be contiguous BHSD")
-    B, H, S, D = q.shape
+        if t.stride(3) != 1 and D > 1:
+            raise ValueError(f"{name} must be contiguous in its last dimension")
     if out is None:
         out = torch.empty_like(q)
     if lse is None:
-        lse = torch.empty((B, H, S), dtype=torch.float32, device=q.device)
-    if out.shape != q.shape or out.dtype != q.dtype or not out.is_contiguous():
-        raise ValueError("out must be a contiguous tensor like q")
-    if lse.shape != (B, H, S) or lse.dtype != torch.float32 or not lse.is_contiguous():
-        raise ValueError("lse must be a contiguous float32 [B, H, S] tensor")
+        lse = torch.empty((B, H, Sq), dtype=torch.float32, device=q.device)
+    if out.shape != q.shape or out.dtype != q.dtype or out.stride(3) != 1:
+        raise ValueError("out must be like q, contiguous in its last dimension")
+    if lse.shape != (B, H, Sq) or lse.dtype != torch.float32 or not lse.is_contiguous():
+        raise ValueError("lse must be a contiguous float32 [B, H, Sq] tensor")
     if stream is None:
         stream = torch.cuda.current_stream(q.device)
-    st = fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(), B, H, S, D,
-                float(scale), int(bool(causal)), _dtype_code(q), int(stream.cuda_stream))
-    if st != 0:
-        raise FaError(st)
+    st = int(stream.cuda_stream)
+    dt = _dtype_code(q)
+    if Sq == Sk and all(t.is_contiguous() for t in (q, k, v, out)):
+        rc = fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(), B, H, Sq, D,
+                    float(scale), int(bool(causal)), dt, st)
+    else:
+        rc = fa_fwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(), B, H, Sq, Sk, D,
+                       q.stride()[:3], k.stride()[:3], v.stride()[:3], out.stride()[:3], float(scale),
+                       int(bool(causal)), dt, st)
+    if rc != 0:
+        raise FaError(rc)
     return out, lse

@@ -28,6 +28,9 @@ FA_ERR_TIMEOUT = -8
 FA_ERR_SCALE = -9
 FA_ERR_ARG = -10
 FA_ERR_PTR = -11
+FA_ERR_STRIDE = -12
+
+_LL3 = ctypes.POINTER(ctypes.c_longlong)
 
 # (name, restype, argtypes) of every symbol include/fa.h declares
 SIGNATURES = [
@@ -39,6 +42,10 @@ SIGNATURES = [
      [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
       ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_float, ctypes.c_int,
       ctypes.c_int, ctypes.c_void_p]),
+    ("fa_fwd_ex", ctypes.c_int,
+     [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+      ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+      _LL3, _LL3, _LL3, _LL3, ctypes.c_float, ctypes.c_int, ctypes.c_int, ctypes.c_void_p]),
     ("fa_check_status", ctypes.c_int, [ctypes.c_void_p]),
     ("fa_last_timeout_site", ctypes.c_int, []),
     ("fa_selftest_timeout", ctypes.c_int, [ctypes.c_void_p]),
@@ -87,6 +94,25 @@ def fa_fwd_noalloc(q_ptr: int, k_ptr: int, v_ptr: int, o_ptr: int, lse_ptr: int,
     """Raw C call of the variant that allocates no device memory (see include/fa.h)."""
     return int(load().fa_fwd_noalloc(q_ptr, k_ptr, v_ptr, o_ptr, lse_ptr, B, H, S, D, float(scale),
                                      int(causal), int(dtype), stream))
+
+
+def _strides(st):
+    if st is None:
+        return None
+    vals = [int(x) for x in st]
+    if len(vals) != 3:
+        raise ValueError("a stride triple (b, h, s) is expected")
+    return (ctypes.c_longlong * 3)(*vals)
+
+
+def fa_fwd_ex(q_ptr: int, k_ptr: int, v_ptr: int, o_ptr: int, lse_ptr: int, B: int, H: int, Sq: int, Sk: int,
+              D: int, q_stride, k_stride, v_stride, o_stride, scale: float, causal: int, dtype: int,
+              stream: int) -> int:
+    """Raw C call of the general-shape entry: each *_stride is a (b, h, s) element-stride
+    triple or None for contiguous BHSD."""
+    return int(load().fa_fwd_ex(q_ptr, k_ptr, v_ptr, o_ptr, lse_ptr, B, H, Sq, Sk, D, _strides(q_stride),
+                                _strides(k_stride), _strides(v_stride), _strides(o_stride), float(scale),
+                                int(causal), int(dtype), stream))
 
 
 def fa_check_status(stream: int = 0) -> int:

@@ -93,23 +93,44 @@ EncodeTiledFn encoder() {
     return g_encode;
 }
 
-// 3-D map over a BHSD tensor viewed as [B*H][S][D] (innermost first: D, S, B*H),
-// box {64, 128, 1}: one 128-byte-wide column chunk of 128 rows, 128-byte swizzle
-// (the swizzle atom the tcgen05 operand descriptors expect).  Rows past S read
-// as zeros and never bleed into the next head.
-bool encode_bhsd(CUtensorMap* map, const void* ptr, int BH, int S, int D, int dtype) {
+// 4-D map over a [B][H][S][D] tensor with the given element strides
+// (innermost first: D, S, H, B), box {64, 128, 1, 1}: one 128-byte-wide column
+// chunk of 128 rows of one head, 128-byte swizzle (the swizzle atom the
+// tcgen05 operand descriptors expect).  Rows past S read as zeros and never
+// bleed into the next head, whatever the layout.
+bool encode_tensor(CUtensorMap* map, const void* ptr, int B, int H, int S, int D, const long long st[3],
+                   int dtype) {
     EncodeTiledFn enc = encoder();
     if (!enc) return false;
-    const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)S, (cuuint64_t)BH};
-    const cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)S * (cuuint64_t)D * 2};
-    const cuuint32_t box[3] = {64, (cuuint32_t)fa::BLOCK_M, 1};
-    const cuuint32_t elem[3] = {1, 1, 1};
+    const cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)S, (cuuint64_t)H, (cuuint64_t)B};
+    const cuuint64_t strides[3] = {(cuuint64_t)st[2] * 2, (cuuint64_t)st[1] * 2, (cuuint64_t)st[0] * 2};
+    const cuuint32_t box[4] = {64, (cuuint32_t)fa::BLOCK_M, 1, 1};
+    const cuuint32_t elem[4] = {1, 1, 1, 1};
     const CUtensorMapDataType dt =
         dtype == FA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
-    CUresult r = enc(map, dt, 3, const_cast<void*>(ptr), dims, strides, box, elem, CU_TENSOR_MAP_INTERLEAVE_NONE,
+    CUresult r = enc(map, dt, 4, const_cast<void*>(ptr), dims, strides, box, elem, CU_TENSOR_MAP_INTERLEAVE_NONE,
                      CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
+}
+
+// Element strides (b, h, s) of one tensor: the caller's, or contiguous BHSD
+// when `given` is null.  A stride over an extent of 1 never moves the address
+// and is replaced by the contiguous one.  Returns FA_OK or FA_ERR_STRIDE.
+constexpr long long MAX_STRIDE = 1ll << 36;  // elements: 2^37 bytes, well inside TMA's 2^40
+int resolve_strides(const long long* given, int B, int H, int S, int D, long long out[3]) {
+    const long long contig[3] = {(long long)H * S * D, (long long)S * D, (long long)D};
+    const int ext[3] = {B, H, S};
+    for (int i = 0; i < 3; ++i) {
+        if (!given || ext[i] == 1) {
+            out[i] = contig[i];
+            continue;
+        }
+        const long long x = given[i];
+        if (x <= 0 || x % 8 != 0 || x >= MAX_STRIDE) return FA_ERR_STRIDE;
+        out[i] = x;
+    }
+    return FA_OK;
 }
 
 int check_device_pointer(const void* p, int dev) {
@@ -133,22 +154,40 @@ long long fa_num_units(int B, int H, int S) {
     return (long long)fa::num_units((int64_t)B * H, S);
 }
 
-int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int S, int D,
-           float scale, int causal, int dtype, cudaStream_t stream) {
-    if (B < 0 || H < 0 || S < 0) return FA_ERR_SHAPE;
+}  // extern "C"
+
+namespace {
+
+// Where the causal scheduler's counter lives.
+enum class Scratch { Allocated, Static };
+
+// The one implementation behind fa_fwd, fa_fwd_ex and fa_fwd_noalloc: checks
+// in the documented order, tensor maps, grid size, scheduler counter, launch.
+int forward(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Sq, int Sk, int D,
+            const long long* q_stride, const long long* k_stride, const long long* v_stride,
+            const long long* o_stride, float scale, int causal, int dtype, cudaStream_t stream, Scratch scratch) {
+    if (B < 0 || H < 0 || Sq < 0 || Sk < 0) return FA_ERR_SHAPE;
     if (D != 64 && D != 128) return FA_ERR_HEADDIM;
     if (dtype != FA_FP16 && dtype != FA_BF16) return FA_ERR_DTYPE;
     if (!(std::isfinite(scale) && scale > 0.f)) return FA_ERR_SCALE;
     if (causal != 0 && causal != 1) return FA_ERR_ARG;
-    if (B == 0 || H == 0 || S == 0) return FA_OK;  // empty problem
+    if (B == 0 || H == 0 || Sq == 0) return FA_OK;  // empty problem
+    // every query row must see at least one key
+    if (Sk == 0 || (causal && Sq > Sk)) return FA_ERR_SHAPE;
     const int64_t BH = (int64_t)B * H;
-    if (BH > INT_MAX || BH * (int64_t)S > INT_MAX) return FA_ERR_SHAPE;
+    if (BH > INT_MAX || BH * (int64_t)Sq > INT_MAX || Sq > INT_MAX - 512 || Sk > INT_MAX - 512) return FA_ERR_SHAPE;
     if (!q || !k || !v || !o || !lse) return FA_ERR_NULL;
+    long long qs[3], ks[3], vs[3], os[3];
+    int rc = resolve_strides(q_stride, B, H, Sq, D, qs);
+    if (rc == FA_OK) rc = resolve_strides(k_stride, B, H, Sk, D, ks);
+    if (rc == FA_OK) rc = resolve_strides(v_stride, B, H, Sk, D, vs);
+    if (rc == FA_OK) rc = resolve_strides(o_stride, B, H, Sq, D, os);
+    if (rc != FA_OK) return rc;
     const uintptr_t a16 = (uintptr_t)q | (uintptr_t)k | (uintptr_t)v | (uintptr_t)o;
     if ((a16 & 15u) != 0 || ((uintptr_t)lse & 3u) != 0) return FA_ERR_ALIGN;
 
     DeviceInfo dev;
-    int rc = device_info(&dev);
+    rc = device_info(&dev);
     if (rc != FA_OK) return rc;
     if (dev.major != 10 || dev.minor != 0) return FA_ERR_ARCH;
     int cur = 0;
@@ -158,32 +197,47 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int
         rc = check_device_pointer(p, cur);
         if (rc != FA_OK) return rc;
     }
+    const int64_t units = fa::num_units(BH, Sq);
+    const int grid = (int)(units < dev.sms ? units : dev.sms);
+    // fa_fwd_noalloc's counter is read back as an int: the claims of all CTAs must fit
+    if (scratch == Scratch::Static && units + grid > fa::NOALLOC_MAX_CLAIMS) return FA_ERR_SHAPE;
 
     fa::LaunchArgs a;
     std::memset(&a, 0, sizeof(a));
-    if (!encode_bhsd(&a.tmap_q, q, (int)BH, S, D, dtype) || !encode_bhsd(&a.tmap_k, k, (int)BH, S, D, dtype) ||
-        !encode_bhsd(&a.tmap_v, v, (int)BH, S, D, dtype))
+    if (!encode_tensor(&a.tmap_q, q, B, H, Sq, D, qs, dtype) || !encode_tensor(&a.tmap_k, k, B, H, Sk, D, ks, dtype) ||
+        !encode_tensor(&a.tmap_v, v, B, H, Sk, D, vs, dtype))
         return FA_ERR_LAUNCH;
     a.o = o;
     a.lse = lse;
-    a.BH = (int)BH;
-    a.S = S;
+    for (int i = 0; i < 3; ++i) a.o_stride[i] = os[i];
+    a.B = B;
+    a.H = H;
+    a.Sq = Sq;
+    a.Sk = Sk;
     a.D = D;
     a.dtype = dtype;
     a.causal = causal;
     a.scale_log2 = (float)((double)scale * 1.4426950408889634074);  // scale * log2(e)
-    const int64_t units = fa::num_units(BH, S);
-    a.grid = (int)(units < dev.sms ? units : dev.sms);
+    a.grid = grid;
     a.sched = nullptr;
     if (causal) {
         // units differ in length under the mask: CTAs claim them from a counter
-        unsigned int* ws = sched_workspace(cur, stream);
-        if (!ws) return FA_ERR_LAUNCH;
-        if (cudaMemsetAsync(ws, 0, sizeof(unsigned int), stream) != cudaSuccess) {
+        unsigned int* ctr = nullptr;
+        if (scratch == Scratch::Static) {
+            if (fa::noalloc_scratch_address(&ctr) != cudaSuccess) {
+                cudaGetLastError();
+                return FA_ERR_LAUNCH;
+            }
+        } else {
+            ctr = sched_workspace(cur, stream);
+            if (!ctr) return FA_ERR_LAUNCH;
+        }
+        // the counter keeps the previous call's value: clear it on this stream
+        if (cudaMemsetAsync(ctr, 0, sizeof(unsigned int), stream) != cudaSuccess) {
             cudaGetLastError();
             return FA_ERR_LAUNCH;
         }
-        a.sched = ws;
+        a.sched = ctr;
     }
     if (fa::launch_fwd_sm100(a, stream) != cudaSuccess) {
         cudaGetLastError();
@@ -196,6 +250,23 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int
     return FA_OK;
 }
 
+}  // namespace
+
+extern "C" {
+
+int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int S, int D,
+           float scale, int causal, int dtype, cudaStream_t stream) {
+    return forward(q, k, v, o, lse, B, H, S, S, D, nullptr, nullptr, nullptr, nullptr, scale, causal, dtype, stream,
+                   Scratch::Allocated);
+}
+
+int fa_fwd_ex(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Sq, int Sk, int D,
+              const long long* q_stride, const long long* k_stride, const long long* v_stride,
+              const long long* o_stride, float scale, int causal, int dtype, cudaStream_t stream) {
+    return forward(q, k, v, o, lse, B, H, Sq, Sk, D, q_stride, k_stride, v_stride, o_stride, scale, causal, dtype,
+                   stream, Scratch::Allocated);
+}
+
 // For callers that cannot allocate device memory (for example code running
 // where cudaMalloc is unavailable or forbidden: inside an allocator, a
 // pre-allocated-memory runtime, or a process that must not grow its device
@@ -204,71 +275,8 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int
 // library allocates.  Nothing here allocates.
 int fa_fwd_noalloc(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int S, int D,
                    float scale, int causal, int dtype, cudaStream_t stream) {
-    if (B < 0 || H < 0 || S < 0) return FA_ERR_SHAPE;
-    if (D != 64 && D != 128) return FA_ERR_HEADDIM;
-    if (dtype != FA_FP16 && dtype != FA_BF16) return FA_ERR_DTYPE;
-    if (!(std::isfinite(scale) && scale > 0.f)) return FA_ERR_SCALE;
-    if (causal != 0 && causal != 1) return FA_ERR_ARG;
-    if (B == 0 || H == 0 || S == 0) return FA_OK;  // empty problem
-    const int64_t BH = (int64_t)B * H;
-    if (BH > INT_MAX || BH * (int64_t)S > INT_MAX) return FA_ERR_SHAPE;
-    if (!q || !k || !v || !o || !lse) return FA_ERR_NULL;
-    const uintptr_t a16 = (uintptr_t)q | (uintptr_t)k | (uintptr_t)v | (uintptr_t)o;
-    if ((a16 & 15u) != 0 || ((uintptr_t)lse & 3u) != 0) return FA_ERR_ALIGN;
-
-    DeviceInfo dev;
-    int rc = device_info(&dev);
-    if (rc != FA_OK) return rc;
-    if (dev.major != 10 || dev.minor != 0) return FA_ERR_ARCH;
-    int cur = 0;
-    cudaGetDevice(&cur);
-    const void* ptrs[5] = {q, k, v, o, lse};
-    for (const void* p : ptrs) {
-        rc = check_device_pointer(p, cur);
-        if (rc != FA_OK) return rc;
-    }
-    const int64_t units = fa::num_units(BH, S);
-    const int grid = (int)(units < dev.sms ? units : dev.sms);
-    // the counter is read back as an int: the claims of all CTAs must fit
-    if (units + grid > fa::NOALLOC_MAX_CLAIMS) return FA_ERR_SHAPE;
-
-    fa::LaunchArgs a;
-    std::memset(&a, 0, sizeof(a));
-    if (!encode_bhsd(&a.tmap_q, q, (int)BH, S, D, dtype) || !encode_bhsd(&a.tmap_k, k, (int)BH, S, D, dtype) ||
-        !encode_bhsd(&a.tmap_v, v, (int)BH, S, D, dtype))
-        return FA_ERR_LAUNCH;
-    a.o = o;
-    a.lse = lse;
-    a.BH = (int)BH;
-    a.S = S;
-    a.D = D;
-    a.dtype = dtype;
-    a.causal = causal;
-    a.scale_log2 = (float)((double)scale * 1.4426950408889634074);  // scale * log2(e)
-    a.grid = grid;
-    a.sched = nullptr;
-    if (causal) {
-        unsigned int* scratch = nullptr;
-        if (fa::noalloc_scratch_address(&scratch) != cudaSuccess) {
-            cudaGetLastError();
-            return FA_ERR_LAUNCH;
-        }
-        // the array keeps the previous call's counter: clear it on this stream
-        if (cudaMemsetAsync(scratch, 0, sizeof(unsigned int), stream) != cudaSuccess) {
-            cudaGetLastError();
-            return FA_ERR_LAUNCH;
-        }
-        a.sched = scratch;
-    }
-    if (fa::launch_fwd_sm100(a, stream) != cudaSuccess) {
-        cudaGetLastError();
-        return FA_ERR_LAUNCH;
-    }
-    if (cudaPeekAtLastError() != cudaSuccess) {
-        cudaGetLastError();
-        return FA_ERR_LAUNCH;
-    }
-    return FA_OK;
+    return forward(q, k, v, o, lse, B, H, S, S, D, nullptr, nullptr, nullptr, nullptr, scale, causal, dtype, stream,
+                   Scratch::Static);
 }
 
 int fa_check_status(cudaStream_t stream) {
@@ -302,7 +310,7 @@ const char* fa_status_string(int status) {
     switch (status) {
         case FA_OK: return "ok";
         case FA_ERR_NULL: return "a required pointer is NULL";
-        case FA_ERR_SHAPE: return "invalid B, H or S";
+        case FA_ERR_SHAPE: return "invalid B, H, Sq or Sk (or causal with Sq > Sk)";
         case FA_ERR_HEADDIM: return "head dimension must be 64 or 128";
         case FA_ERR_DTYPE: return "dtype must be FA_FP16 or FA_BF16";
         case FA_ERR_ALIGN: return "q, k, v, o must be 16-byte aligned and lse 4-byte aligned";
@@ -312,6 +320,7 @@ const char* fa_status_string(int status) {
         case FA_ERR_SCALE: return "scale must be finite and > 0";
         case FA_ERR_ARG: return "causal must be 0 or 1";
         case FA_ERR_PTR: return "pointer is not device memory of the current device";
+        case FA_ERR_STRIDE: return "a stride is not positive, a multiple of 8 elements and below 2^36";
         default: return "unknown status";
     }
 }

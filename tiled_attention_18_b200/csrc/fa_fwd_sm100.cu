@@ -177,13 +177,17 @@ struct KParams {
     CUtensorMap tmap_k;
     CUtensorMap tmap_v;
     uint8_t* o;
-    float* lse;
+    float* lse;    // [B, H, Sq] contiguous
+    long long o_sb, o_sh, o_ss;  // byte strides of O over b, h and the query row
     int BH;
-    int S;
+    int H;
+    int Sq;        // query rows per head
+    int Sk;        // keys per head
     int n_mblk;    // 256-row query blocks per head
     int n_units;
     int nkv;       // key tiles per head
     int causal;
+    int causal_off;  // Sk - Sq: query i sees keys j <= i + causal_off under the mask
     float scale_log2;
     unsigned int* sched;  // zeroed unit counter (claim order), or null for the static order
 };
@@ -262,12 +266,12 @@ __device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity) {
     }
 }
 
-__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, uint32_t bar, int c0,
-                                            int c1, int c2) {
+__device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* map, uint32_t bar, int c0,
+                                            int c1, int c2, int c3) {
     asm volatile(
-        "cp.async.bulk.tensor.3d.shared::cta.global.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
+        "cp.async.bulk.tensor.4d.shared::cta.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5, %6}], [%2];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
         : "memory");
 }
 
@@ -495,10 +499,11 @@ __device__ __forceinline__ Unit decode_unit(const KParams& p, int u) {
         const int q0 = mb * ROWS_PER_UNIT + t * BLOCK_M;
         U.q0[t] = q0;
         int n = 0;
-        if (q0 < p.S) {
+        if (q0 < p.Sq) {
             // diagonal bound: key tile j is visited iff its first key j*BLOCK_N is
-            // not after the tile's last query row q0 + BLOCK_M - 1
-            n = p.causal ? min((q0 + BLOCK_M - 1) / BLOCK_N + 1, p.nkv) : p.nkv;
+            // not after the last key that the tile's last query row sees,
+            // q0 + BLOCK_M - 1 + causal_off
+            n = p.causal ? min((q0 + BLOCK_M - 1 + p.causal_off) / BLOCK_N + 1, p.nkv) : p.nkv;
         }
         U.n[t] = n;
     }
@@ -557,6 +562,7 @@ __device__ void producer_role(const KParams& p, uint8_t* smem, volatile uint32_t
         if (++uslot == L::NUNIT) { uslot = 0; uphase ^= 1u; }
         if (u < 0) break;
         const Unit U = decode_unit(p, u);
+        const int ub = U.bh / p.H, uh = U.bh - ub * p.H;  // tensor-map coordinates of the head
         if (!mbar_wait(bar(L::B_QEMPTY), qe_phase ^ 1u, abort_flag, 1)) { ok = false; break; }
         qe_phase ^= 1u;
         const uint32_t qbytes = (U.n[0] > 0 ? L::TILE_BYTES : 0) + (U.n[1] > 0 ? L::TILE_BYTES : 0);
@@ -568,7 +574,7 @@ __device__ void producer_role(const KParams& p, uint8_t* smem, volatile uint32_t
             const uint32_t dst = base + L::Q_OFF + t * L::TILE_BYTES;
 #pragma unroll
             for (int c = 0; c < L::CHUNKS; ++c)
-                tma_load_3d(dst + c * L::CHUNK_BYTES, &p.tmap_q, bar(L::B_QFULL), c * 64, U.q0[t], U.bh);
+                tma_load_4d(dst + c * L::CHUNK_BYTES, &p.tmap_q, bar(L::B_QFULL), c * 64, U.q0[t], uh, ub);
         }
         // stages 0..N: stage s = (V_{s-1} if s >= 1, K_s if s < N)
         for (int st = 0; st <= U.N; ++st) {
@@ -581,14 +587,14 @@ __device__ void producer_role(const KParams& p, uint8_t* smem, volatile uint32_t
             if (st < U.N) {
 #pragma unroll
                 for (int c = 0; c < L::CHUNKS; ++c)
-                    tma_load_3d(dst + L::STAGE_K + c * L::CHUNK_BYTES, &p.tmap_k, bar(L::B_STFULL + stage), c * 64,
-                                st * BLOCK_N, U.bh);
+                    tma_load_4d(dst + L::STAGE_K + c * L::CHUNK_BYTES, &p.tmap_k, bar(L::B_STFULL + stage), c * 64,
+                                st * BLOCK_N, uh, ub);
             }
             if (st >= 1) {
 #pragma unroll
                 for (int c = 0; c < L::CHUNKS; ++c)
-                    tma_load_3d(dst + L::STAGE_V + c * L::CHUNK_BYTES, &p.tmap_v, bar(L::B_STFULL + stage), c * 64,
-                                (st - 1) * BLOCK_N, U.bh);
+                    tma_load_4d(dst + L::STAGE_V + c * L::CHUNK_BYTES, &p.tmap_v, bar(L::B_STFULL + stage), c * 64,
+                                (st - 1) * BLOCK_N, uh, ub);
             }
             if (++stage == L::NSTAGE) { stage = 0; phase ^= 1u; }
         }
@@ -767,7 +773,7 @@ __device__ void softmax_role(const KParams& p, uint8_t* smem, uint32_t tmem, int
         const int n = U.n[t];
         if (n == 0) continue;
         const int row = U.q0[t] + row_in_tile;
-        const int key_limit = p.causal ? min(row, p.S - 1) : p.S - 1;  // last visible key
+        const int key_limit = p.causal ? min(row + p.causal_off, p.Sk - 1) : p.Sk - 1;  // last visible key
         float m_use = -INFINITY;  // reference max in log2 units
         float l = 0.f;            // running sum of the weights relative to m_use (fp32)
         float lr = 0.f;           // the same sum over the weights as rounded for P.V
@@ -779,7 +785,8 @@ __device__ void softmax_role(const KParams& p, uint8_t* smem, uint32_t tmem, int
             float s[BLOCK_N];
             tmem_ld128(ts, s);
             const int kbase = j * BLOCK_N;
-            const bool need_mask = (kbase + BLOCK_N > p.S) || (p.causal && kbase + BLOCK_N - 1 > U.q0[t]);
+            const bool need_mask =
+                (kbase + BLOCK_N > p.Sk) || (p.causal && kbase + BLOCK_N - 1 > U.q0[t] + p.causal_off);
             if (need_mask) {
                 const int lim = key_limit - kbase;
 #pragma unroll
@@ -928,8 +935,9 @@ __device__ void correction_role(const KParams& p, uint8_t* smem, uint32_t tmem, 
         tc_fence_after();
         const float2 fin = fin_buf[(fp * 2 + t) * BLOCK_M + row_in_tile];
         const int row = U.q0[t] + row_in_tile;
-        const bool valid = row < p.S;
-        uint8_t* orow = p.o + ((size_t)U.bh * (size_t)p.S + (size_t)(valid ? row : 0)) * (size_t)(D * 2);
+        const bool valid = row < p.Sq;
+        const int ub = U.bh / p.H, uh = U.bh - ub * p.H;
+        uint8_t* orow = p.o + (long long)ub * p.o_sb + (long long)uh * p.o_sh + (long long)(valid ? row : 0) * p.o_ss;
         const uint32_t to = tmem + lane_sel + (t == 0 ? COL_O0 : COL_O1);
         const float2 inv2 = make_float2(fin.x, fin.x);
 #pragma unroll 1
@@ -948,7 +956,7 @@ __device__ void correction_role(const KParams& p, uint8_t* smem, uint32_t tmem, 
                 for (int i = 0; i < 4; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
             }
         }
-        if (valid) p.lse[(size_t)U.bh * (size_t)p.S + row] = fin.y;
+        if (valid) p.lse[(size_t)U.bh * (size_t)p.Sq + row] = fin.y;
         // O_t is free for the next unit's first P.V: arm that P barrier phase
         tc_fence_before();
         mbar_arrive(bar(L::B_PFULL + t));
@@ -1084,12 +1092,18 @@ cudaError_t launch_impl(const LaunchArgs& a, cudaStream_t stream) {
     p.tmap_v = a.tmap_v;
     p.o = reinterpret_cast<uint8_t*>(a.o);
     p.lse = a.lse;
-    p.BH = a.BH;
-    p.S = a.S;
-    p.n_mblk = (a.S + ROWS_PER_UNIT - 1) / ROWS_PER_UNIT;
-    p.n_units = (int)num_units(a.BH, a.S);
-    p.nkv = (a.S + BLOCK_N - 1) / BLOCK_N;
+    p.o_sb = a.o_stride[0] * 2;
+    p.o_sh = a.o_stride[1] * 2;
+    p.o_ss = a.o_stride[2] * 2;
+    p.BH = a.B * a.H;
+    p.H = a.H;
+    p.Sq = a.Sq;
+    p.Sk = a.Sk;
+    p.n_mblk = (a.Sq + ROWS_PER_UNIT - 1) / ROWS_PER_UNIT;
+    p.n_units = (int)num_units(p.BH, a.Sq);
+    p.nkv = (a.Sk + BLOCK_N - 1) / BLOCK_N;
     p.causal = a.causal;
+    p.causal_off = a.Sk - a.Sq;
     p.scale_log2 = a.scale_log2;
     p.sched = a.sched;
     cudaLaunchConfig_t cfg = {};

@@ -22,13 +22,16 @@ constexpr int DEV_TIMEOUT = 1;
 constexpr int SELFTEST_SITE = 100;
 
 struct LaunchArgs {
-    CUtensorMap tmap_q;     // 3-D maps over [B*H][S][D], box {64, 128, 1}, 128-byte swizzle
-    CUtensorMap tmap_k;
+    CUtensorMap tmap_q;     // 4-D maps over [B][H][S][D] (innermost first: D, S, H, B) with
+    CUtensorMap tmap_k;     // the tensors' own strides, box {64, 128, 1, 1}, 128-byte swizzle
     CUtensorMap tmap_v;
-    void* o;                // [B,H,S,D] 16-bit
-    float* lse;             // [B,H,S] fp32
-    int BH;
-    int S;
+    void* o;                // [B,H,Sq,D] 16-bit at o_stride
+    float* lse;             // [B,H,Sq] fp32, contiguous
+    long long o_stride[3];  // element strides of O over b, h, s (d is contiguous)
+    int B;
+    int H;
+    int Sq;                 // query rows per head
+    int Sk;                 // key/value rows per head (Sk >= Sq under the causal mask)
     int D;
     int dtype;              // 0 fp16, 1 bf16
     int causal;

@@ -39,6 +39,17 @@ class Workload:
     causal: bool
     qk_mult: float = 1.0
     seed: int = 0
+    Sk: int = 0            # keys per head; 0 = S (self-attention)
+    layout: str = "bhsd"   # memory layout of Q, K, V and O: "bhsd" or "bshd"
+
+    @property
+    def Skv(self) -> int:
+        return self.Sk if self.Sk else self.S
+
+    @property
+    def general(self) -> bool:
+        """True when the workload needs fa_fwd_ex (Sq != Sk or a non-BHSD layout)."""
+        return self.Skv != self.S or self.layout != "bhsd"
 
     @property
     def torch_dtype(self) -> torch.dtype:
@@ -50,11 +61,17 @@ class Workload:
 
     @property
     def flops(self) -> float:
-        return attention_flops(self.B, self.H, self.S, self.D, self.causal)
+        if not self.general:
+            return attention_flops(self.B, self.H, self.S, self.D, self.causal)
+        return attention_flops_general(self.B, self.H, self.S, self.Skv, self.D, self.causal)
 
     def describe(self) -> str:
         c = "causal" if self.causal else "non-causal"
         extra = f", Q,K x{self.qk_mult:g}" if self.qk_mult != 1.0 else ""
+        if self.general:
+            lay = f", {self.layout.upper()}" if self.layout != "bhsd" else ""
+            return (f"attn-fwd {self.dtype} B={self.B} H={self.H} Sq={self.S} Sk={self.Skv} D={self.D} "
+                    f"{c}{extra}{lay}")
         return f"attn-fwd {self.dtype} B={self.B} H={self.H} S={self.S} D={self.D} {c}{extra}"
 
 
@@ -69,6 +86,16 @@ def attention_flops(B: int, H: int, S: int, D: int, causal: bool) -> float:
     return f / 2.0 if causal else f
 
 
+def attention_flops_general(B: int, H: int, Sq: int, Sk: int, D: int, causal: bool) -> float:
+    """4*B*H*Sq*Sk*D; with the bottom-right causal mask the Sq x Sq corner above
+    the diagonal is not counted (half of it), which gives attention_flops when
+    Sq = Sk."""
+    f = 4.0 * B * H * Sq * Sk * D
+    if causal:
+        f -= 4.0 * B * H * D * Sq * Sq / 2.0
+    return f
+
+
 # The five workload configurations; the last one runs both with and without the mask.
 WORKLOADS = {
     "c1": Workload("c1", 1, 2, 256, 64, "fp16", False),
@@ -77,6 +104,22 @@ WORKLOADS = {
     "c4": Workload("c4", 1, 40, 8192, 128, "bf16", True, qk_mult=2.0),
     "c5a": Workload("c5a", 1, 32, 16384, 128, "bf16", False),
     "c5b": Workload("c5b", 1, 32, 16384, 128, "bf16", True),
+}
+
+# General-shape workloads (fa_fwd_ex):
+# - sdxl_xattn: text-to-image cross-attention, 4096 image tokens (a 64 x 64
+#   latent grid) attending to 77 text tokens, 10 heads of 64 (the SDXL case of
+#   "解析CANN ops-transformer的FlashAttention算子：注意力机制的内存优化");
+# - bert_large: the BERT-Large shape B=32, H=16, S=512, D=64 of the
+#   FlashAttention-2 page's section 4.3, with the tensors in the
+#   [batch, seq_len, heads, head_dim] layout that the gsyq.cn catlass page warns
+#   about, read in place;
+# - prefill_cached: a causal chunk of 4096 new queries over 16384 cached keys
+#   (queries aligned to the last keys), bf16 as the catlass page advises above 4K.
+GENERAL_WORKLOADS = {
+    "sdxl_xattn": Workload("sdxl_xattn", 2, 10, 4096, 64, "fp16", False, Sk=77),
+    "bert_large": Workload("bert_large", 32, 16, 512, 64, "fp16", False, layout="bshd"),
+    "prefill_cached": Workload("prefill_cached", 1, 32, 4096, 128, "bf16", True, Sk=16384),
 }
 
 # Parity tolerances (max-abs) on O by dtype, and on the LSE.
@@ -100,7 +143,27 @@ def make_inputs(B: int, H: int, S: int, D: int, dtype: str, qk_mult: float = 1.0
     return (q.to(tdt).contiguous(), k.to(tdt).contiguous(), v.to(tdt).contiguous())
 
 
+def make_cross_inputs(B: int, H: int, Sq: int, Sk: int, D: int, dtype: str, seed: int = 0):
+    """Q [B,H,Sq,D] drawn as make_inputs(seed) draws Q; K, V [B,H,Sk,D] drawn as
+    make_inputs(seed + 1) draws K and V.  Contiguous BHSD CPU tensors."""
+    q, _, _ = make_inputs(B, H, Sq, D, dtype, seed=seed)
+    _, k, v = make_inputs(B, H, Sk, D, dtype, seed=seed + 1)
+    return q, k, v
+
+
+def to_layout(x: torch.Tensor, layout: str) -> torch.Tensor:
+    """The same [B,H,S,D] values stored in ``layout``, returned as a [B,H,S,D] view."""
+    if layout == "bhsd":
+        return x.contiguous()
+    if layout == "bshd":
+        return x.transpose(1, 2).contiguous().transpose(1, 2)
+    raise ValueError(f"unknown layout {layout!r}")
+
+
 def workload_inputs(w: Workload):
+    """Contiguous BHSD CPU tensors of the workload (see to_layout for its layout)."""
+    if w.Skv != w.S:
+        return make_cross_inputs(w.B, w.H, w.S, w.Skv, w.D, w.dtype, w.seed)
     return make_inputs(w.B, w.H, w.S, w.D, w.dtype, w.qk_mult, w.seed)
 
 
