@@ -21,10 +21,14 @@ ctypes.  Function-level citations are in the C file's header:
 - ``causal_tile_count`` : element-wise enumeration of computed/skipped tile pairs.
 - ``attn_fwd_gen`` / ``attn_rows_gen`` : the same definition with Sq queries and
   Sk keys (cross-attention) and the causal mask aligned to the last Sq keys.
+- ``attn_bwd`` : dQ, dK, dV by the chain rule through the definition (the
+  softmax Jacobian), with optional absolute-value error scales.
 
 Parity pins: every function above is pinned by tests in tests/test_oracle.py and
 tests/test_oracle_general.py (torch SDPA in float64 with an explicit mask, the
-Q = 0 closed form, agreement with attn_fwd when Sq = Sk).
+Q = 0 closed form, agreement with attn_fwd when Sq = Sk) and
+tests/test_oracle_bwd.py (float64 autograd, central finite differences of
+attn_fwd_gen, closed forms and column-sum identities).
 """
 from __future__ import annotations
 
@@ -92,6 +96,9 @@ def _load():
         lib.oracle_attn_rows_gen.argtypes = [u16p, u16p, u16p, i64, i64, i64, i64, i64, ctypes.c_float,
                                              ctypes.c_int, ctypes.c_int, i64p, i64p, i64, f64p, f64p]
         lib.oracle_attn_rows_gen.restype = ctypes.c_int
+        lib.oracle_attn_bwd.argtypes = [u16p, u16p, u16p, u16p, i64, i64, i64, i64, i64, ctypes.c_float,
+                                        ctypes.c_int, ctypes.c_int, f64p, f64p, f64p, f64p, f64p, f64p]
+        lib.oracle_attn_bwd.restype = ctypes.c_int
         lib.oracle_causal_tile_count.argtypes = [i64, i64, i64, i64p, i64p, i64p]
         lib.oracle_causal_tile_count.restype = None
         lib.oracle_num_threads.argtypes = []
@@ -211,6 +218,31 @@ def attn_rows_gen(q, k, v, scale: float, causal: bool, dtype, bh_idx, row_idx):
     if rc != 0:
         raise RuntimeError(f"oracle_attn_rows_gen failed with {rc}")
     return o, lse
+
+
+def attn_bwd(q, k, v, dout, scale: float, causal: bool, dtype, magnitudes: bool = False):
+    """fp64 gradients (dQ, dK, dV) of attention for the upstream gradient ``dout``
+    (q, dout: [B,H,Sq,D]; k, v: [B,H,Sk,D]; bottom-right causal).  With
+    ``magnitudes`` also returns the absolute-value sums (mag_dQ, mag_dK, mag_dV)
+    that scale each element's 16-bit rounding error (see attn_oracle.c)."""
+    lib = _load()
+    qb, kb, vb, gb = _bits(q), _bits(k), _bits(v), _bits(dout)
+    B, H, Sq, D = qb.shape
+    Sk = kb.shape[2]
+    if gb.shape != qb.shape or kb.shape != (B, H, Sk, D) or vb.shape != kb.shape:
+        raise ValueError("dout must be like q and k, v [B, H, Sk, D]")
+    dq = np.empty((B, H, Sq, D))
+    dk = np.empty((B, H, Sk, D))
+    dv = np.empty((B, H, Sk, D))
+    mags = tuple(np.empty(a.shape) for a in (dq, dk, dv)) if magnitudes else (None, None, None)
+    fp = lambda a: _ptr(a, ctypes.c_double) if a is not None else None  # noqa: E731
+    rc = lib.oracle_attn_bwd(_ptr(qb, ctypes.c_uint16), _ptr(kb, ctypes.c_uint16), _ptr(vb, ctypes.c_uint16),
+                             _ptr(gb, ctypes.c_uint16), B, H, Sq, Sk, D, float(np.float32(scale)),
+                             int(bool(causal)), _dtype_code(dtype), fp(dq), fp(dk), fp(dv),
+                             fp(mags[0]), fp(mags[1]), fp(mags[2]))
+    if rc != 0:
+        raise RuntimeError(f"oracle_attn_bwd failed with {rc}")
+    return (dq, dk, dv) + (mags if magnitudes else ())
 
 
 def attn_tiled(q, k, v, scale: float, causal: bool, dtype, Br: int, Bc: int, form: int = 0):

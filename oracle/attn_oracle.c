@@ -523,3 +523,149 @@ int oracle_attn_rows_gen(const uint16_t *q, const uint16_t *k, const uint16_t *v
     }
     return bad ? -10 : 0;
 }
+
+/* ------------------------------------------------------------ backward pass */
+
+/*
+ * Gradients of the attention forward pass (general shapes, bottom-right causal
+ * mask as in oracle_attn_fwd_gen) for an upstream gradient dO = dL/dO:
+ *
+ *   P_ij  = softmax_j(s_ij),  s_ij = scale * q_i . k_j  over the visible keys
+ *   dV_j  = sum_i P_ij dO_i
+ *   dP_ij = dO_i . v_j
+ *   dS_ij = P_ij (dP_ij - sum_k P_ik dP_ik)      (the softmax Jacobian)
+ *   dQ_i  = scale * sum_j dS_ij k_j
+ *   dK_j  = scale * sum_i dS_ij q_i
+ *
+ * This is the chain rule through the definition, written out; the backward
+ * pass recomputes S and P from Q, K and the saved row statistics instead of
+ * storing P ("FlashAttention-2 在昇腾 NPU 上如何做到 3 倍加速？", the
+ * recomputation row of the core-optimisation table and section 6.2; the
+ * backward configuration with a deterministic switch on the gsyq.cn catlass
+ * page, "反向传播的特殊处理").  Here nothing is recomputed from saved state: every
+ * quantity comes from q, k, v and dO in fp64.
+ *
+ * Optional outputs mag_dq, mag_dk, mag_dv (NULL to skip) hold the same sums
+ * over absolute values, the scale of the rounding error a 16-bit evaluation
+ * of each element can carry:
+ *   mag_dV_j = sum_i P_ij |dO_i|
+ *   mag_dQ_i = scale * sum_j P_ij (|dP_ij| + a_i) |k_j|
+ *   mag_dK_j = scale * sum_i P_ij (|dP_ij| + a_i) |q_i|,
+ *   a_i = sum_k P_ik |dP_ik|.
+ * Rows with no visible key have zero gradients.
+ */
+int oracle_attn_bwd(const uint16_t *q, const uint16_t *k, const uint16_t *v, const uint16_t *dout, int64_t B,
+                    int64_t H, int64_t Sq, int64_t Sk, int64_t D, float scale, int causal, int dtype, double *dq,
+                    double *dk, double *dv, double *mag_dq, double *mag_dk, double *mag_dv)
+{
+    if (B < 0 || H < 0 || Sq < 0 || Sk < 0 || D <= 0) return -2;
+    if (dtype != ORACLE_F16 && dtype != ORACLE_BF16) return -4;
+    const double sc = (double)scale;
+    const size_t szq = (size_t)(Sq * D > 0 ? Sq * D : 1), szk = (size_t)(Sk * D > 0 ? Sk * D : 1);
+    for (int64_t bh = 0; bh < B * H; ++bh) {
+        double *qh = (double *)malloc(sizeof(double) * szq);
+        double *oh = (double *)malloc(sizeof(double) * szq);
+        double *kh = (double *)malloc(sizeof(double) * szk);
+        double *vh = (double *)malloc(sizeof(double) * szk);
+        double *lse = (double *)malloc(sizeof(double) * (size_t)(Sq > 0 ? Sq : 1));
+        double *dsum = (double *)malloc(sizeof(double) * (size_t)(Sq > 0 ? Sq : 1));
+        double *asum = (double *)malloc(sizeof(double) * (size_t)(Sq > 0 ? Sq : 1));
+        if (!qh || !oh || !kh || !vh || !lse || !dsum || !asum) {
+            free(qh); free(oh); free(kh); free(vh); free(lse); free(dsum); free(asum);
+            return -10;
+        }
+        oracle_decode(q + bh * Sq * D, qh, Sq * D, dtype);
+        oracle_decode(dout + bh * Sq * D, oh, Sq * D, dtype);  /* oh holds dO */
+        oracle_decode(k + bh * Sk * D, kh, Sk * D, dtype);
+        oracle_decode(v + bh * Sk * D, vh, Sk * D, dtype);
+        double *dqh = dq + bh * Sq * D, *dkh = dk + bh * Sk * D, *dvh = dv + bh * Sk * D;
+        double *mqh = mag_dq ? mag_dq + bh * Sq * D : NULL;
+        double *mkh = mag_dk ? mag_dk + bh * Sk * D : NULL;
+        double *mvh = mag_dv ? mag_dv + bh * Sk * D : NULL;
+
+        /* pass 1, per query row: P row, dP row, the row's softmax-Jacobian sum, dQ */
+#pragma omp parallel
+        {
+            double *prow = (double *)malloc(sizeof(double) * (size_t)(Sk > 0 ? Sk : 1));
+            double *dprow = (double *)malloc(sizeof(double) * (size_t)(Sk > 0 ? Sk : 1));
+#pragma omp for schedule(dynamic, 8)
+            for (int64_t i = 0; i < Sq; ++i) {
+                const int64_t nj = visible_keys(i, Sq, Sk, causal);
+                const double *qi = qh + i * D, *doi = oh + i * D;
+                for (int64_t d = 0; d < D; ++d) {
+                    dqh[i * D + d] = 0.0;
+                    if (mqh) mqh[i * D + d] = 0.0;
+                }
+                if (nj <= 0) {
+                    lse[i] = -INFINITY; dsum[i] = 0.0; asum[i] = 0.0;
+                    continue;
+                }
+                double m = -INFINITY;
+                for (int64_t j = 0; j < nj; ++j) {
+                    double dot = 0.0, dp = 0.0;
+                    for (int64_t d = 0; d < D; ++d) {
+                        dot += qi[d] * kh[j * D + d];
+                        dp += doi[d] * vh[j * D + d];
+                    }
+                    prow[j] = sc * dot;
+                    dprow[j] = dp;
+                    if (prow[j] > m) m = prow[j];
+                }
+                double l = 0.0;
+                for (int64_t j = 0; j < nj; ++j) {
+                    prow[j] = exp(prow[j] - m);
+                    l += prow[j];
+                }
+                double ds = 0.0, as = 0.0;
+                for (int64_t j = 0; j < nj; ++j) {
+                    prow[j] /= l;
+                    ds += prow[j] * dprow[j];
+                    as += prow[j] * fabs(dprow[j]);
+                }
+                lse[i] = m + log(l);
+                dsum[i] = ds;
+                asum[i] = as;
+                for (int64_t j = 0; j < nj; ++j) {
+                    const double g = sc * prow[j] * (dprow[j] - ds);
+                    const double gm = sc * prow[j] * (fabs(dprow[j]) + as);
+                    for (int64_t d = 0; d < D; ++d) {
+                        dqh[i * D + d] += g * kh[j * D + d];
+                        if (mqh) mqh[i * D + d] += gm * fabs(kh[j * D + d]);
+                    }
+                }
+            }
+            free(prow); free(dprow);
+        }
+        /* pass 2, per key: dK and dV over the queries that see it */
+#pragma omp parallel for schedule(dynamic, 8)
+        for (int64_t j = 0; j < Sk; ++j) {
+            const double *kj = kh + j * D, *vj = vh + j * D;
+            for (int64_t d = 0; d < D; ++d) {
+                dkh[j * D + d] = 0.0;
+                dvh[j * D + d] = 0.0;
+                if (mkh) mkh[j * D + d] = 0.0;
+                if (mvh) mvh[j * D + d] = 0.0;
+            }
+            for (int64_t i = 0; i < Sq; ++i) {
+                if (j >= visible_keys(i, Sq, Sk, causal)) continue;
+                const double *qi = qh + i * D, *doi = oh + i * D;
+                double dot = 0.0, dp = 0.0;
+                for (int64_t d = 0; d < D; ++d) {
+                    dot += qi[d] * kj[d];
+                    dp += doi[d] * vj[d];
+                }
+                const double p = exp(sc * dot - lse[i]);
+                const double g = sc * p * (dp - dsum[i]);
+                const double gm = sc * p * (fabs(dp) + asum[i]);
+                for (int64_t d = 0; d < D; ++d) {
+                    dkh[j * D + d] += g * qi[d];
+                    dvh[j * D + d] += p * doi[d];
+                    if (mkh) mkh[j * D + d] += gm * fabs(qi[d]);
+                    if (mvh) mvh[j * D + d] += p * fabs(doi[d]);
+                }
+            }
+        }
+        free(qh); free(oh); free(kh); free(vh); free(lse); free(dsum); free(asum);
+    }
+    return 0;
+}
