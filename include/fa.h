@@ -60,8 +60,9 @@ typedef enum {
     FA_ERR_SCALE = -9,    /* scale is not finite and > 0 */
     FA_ERR_ARG = -10,     /* causal is not 0 or 1 */
     FA_ERR_PTR = -11,     /* a pointer is not device memory of the current device */
-    FA_ERR_STRIDE = -12   /* fa_fwd_ex: a stride is negative, zero over an extent > 1, not a
+    FA_ERR_STRIDE = -12,  /* fa_fwd_ex: a stride is negative, zero over an extent > 1, not a
                              multiple of 8 elements (16 bytes), or not below 2^36 elements */
+    FA_ERR_WORKSPACE = -13 /* fa_bwd: workspace NULL, not 256-byte aligned or too small */
 } fa_status;
 
 /*
@@ -157,6 +158,52 @@ FA_API int fa_fwd_ex(const void* q, const void* k, const void* v, void* o, float
                      int Sk, int D, const long long* q_stride, const long long* k_stride,
                      const long long* v_stride, const long long* o_stride, float scale, int causal, int dtype,
                      cudaStream_t stream);
+
+/*
+ * fa_bwd_workspace_size -- bytes of device workspace fa_bwd needs for B*H
+ * heads of Sq query rows of dimension D: an fp32 dQ accumulator
+ * [B*H][Sq][D], two fp32 row-statistic arrays [B*H][Sq rounded up to 128]
+ * and a 256-byte scheduler counter, each part 256-byte aligned.  0 for an
+ * empty problem, a negative fa_status on invalid sizes.  Host only.
+ */
+FA_API long long fa_bwd_workspace_size(int B, int H, int Sq, int D);
+
+/*
+ * fa_bwd -- backward pass of fa_fwd / fa_fwd_ex (contiguous BHSD tensors):
+ * the gradients dQ, dK, dV of the attention output for the upstream gradient
+ * dO, recomputing the scores and weights tile by tile from Q, K and the
+ * forward pass's LSE instead of storing them ("FlashAttention-2 在昇腾 NPU 上
+ * 如何做到 3 倍加速？", the recomputation row of the core-optimisation table
+ * and section 6.2; the backward configuration on the gsyq.cn catlass page,
+ * "反向传播的特殊处理").  With P_ij = exp(scale q_i.k_j - LSE_i) over the keys
+ * query i sees (the mask of fa_fwd_ex: all keys, or j <= i + Sk - Sq) and
+ * Delta_i = sum_d dO_id O_id:
+ *
+ *   dV_j = sum_i P_ij dO_i,    dS_ij = P_ij (dO_i.v_j - Delta_i),
+ *   dQ_i = scale sum_j dS_ij k_j,    dK_j = scale sum_i dS_ij q_i.
+ *
+ * q, o, dout : device, [B, H, Sq, D] contiguous, dtype.  o and lse must be the
+ *              forward outputs for these q, k, v, scale and mask.
+ * k, v       : device, [B, H, Sk, D] contiguous, dtype.
+ * lse        : device, [B, H, Sq] contiguous fp32 (natural log).
+ * dq         : device, [B, H, Sq, D] contiguous, dtype.  Written.
+ * dk, dv     : device, [B, H, Sk, D] contiguous, dtype.  Written.
+ * workspace  : device, at least fa_bwd_workspace_size(B, H, Sq, D) bytes,
+ *              256-byte aligned (else FA_ERR_WORKSPACE); contents on entry do
+ *              not matter; used only during the call's kernels on `stream`, so
+ *              calls that may overlap on the GPU need separate workspaces.
+ * B, H, Sq, Sk, D, scale, causal, dtype: as fa_fwd_ex.  B or H 0 is an empty
+ *              problem (FA_OK, nothing launched); Sq = 0 zeroes dK and dV.
+ * Numerics: S, P, dP, dS, Delta and all accumulation in fp32; P and dS are
+ * rounded to dtype before their products; dQ is accumulated in fp32 across
+ * key tiles with atomic adds (so its last bits may differ between runs; dK and
+ * dV are deterministic); the outputs are rounded to nearest even.
+ * Three kernels run on `stream` (row statistics, the fused backward, dQ
+ * conversion); nothing is allocated; asynchronous.  Errors as fa_fwd.
+ */
+FA_API int fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
+                  void* dq, void* dk, void* dv, void* workspace, long long workspace_bytes, int B, int H, int Sq,
+                  int Sk, int D, float scale, int causal, int dtype, cudaStream_t stream);
 
 /*
  * fa_check_status -- synchronise `stream`, then report and clear the device

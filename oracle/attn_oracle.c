@@ -551,7 +551,11 @@ int oracle_attn_rows_gen(const uint16_t *q, const uint16_t *k, const uint16_t *v
  *   mag_dV_j = sum_i P_ij |dO_i|
  *   mag_dQ_i = scale * sum_j P_ij (|dP_ij| + a_i) |k_j|
  *   mag_dK_j = scale * sum_i P_ij (|dP_ij| + a_i) |q_i|,
- *   a_i = sum_k P_ik |dP_ik|.
+ *   a_i = sum_k P_ik |dP_ik| + 2 sum_d |dO_id| sum_k P_ik |v_kd|
+ * (the second part of a_i scales the error of sum_k P_ik dP_ik when it is
+ * formed as sum_d dO_id O_id from a forward output O whose own error is at
+ * most twice the unit roundoff times sum_k P_ik |v_kd|: its weights and its
+ * result are each rounded once).
  * Rows with no visible key have zero gradients.
  */
 int oracle_attn_bwd(const uint16_t *q, const uint16_t *k, const uint16_t *v, const uint16_t *dout, int64_t B,
@@ -574,6 +578,7 @@ int oracle_attn_bwd(const uint16_t *q, const uint16_t *k, const uint16_t *v, con
             free(qh); free(oh); free(kh); free(vh); free(lse); free(dsum); free(asum);
             return -10;
         }
+        const int64_t Dd = D;
         oracle_decode(q + bh * Sq * D, qh, Sq * D, dtype);
         oracle_decode(dout + bh * Sq * D, oh, Sq * D, dtype);  /* oh holds dO */
         oracle_decode(k + bh * Sk * D, kh, Sk * D, dtype);
@@ -621,6 +626,12 @@ int oracle_attn_bwd(const uint16_t *q, const uint16_t *k, const uint16_t *v, con
                     prow[j] /= l;
                     ds += prow[j] * dprow[j];
                     as += prow[j] * fabs(dprow[j]);
+                }
+                /* 2 sum_d |dO_id| sum_j P_ij |v_jd| */
+                for (int64_t d = 0; d < Dd; ++d) {
+                    double od = 0.0;
+                    for (int64_t j = 0; j < nj; ++j) od += prow[j] * fabs(vh[j * D + d]);
+                    as += 2.0 * fabs(doi[d]) * od;
                 }
                 lse[i] = m + log(l);
                 dsum[i] = ds;

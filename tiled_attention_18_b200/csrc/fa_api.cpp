@@ -279,14 +279,108 @@ int fa_fwd_noalloc(const void* q, const void* k, const void* v, void* o, float* 
                    Scratch::Static);
 }
 
+long long fa_bwd_workspace_size(int B, int H, int Sq, int D) {
+    if (B < 0 || H < 0 || Sq < 0) return FA_ERR_SHAPE;
+    if (D != 64 && D != 128) return FA_ERR_HEADDIM;
+    if (B == 0 || H == 0 || Sq == 0) return 0;
+    return (long long)fa::bwd_workspace_layout((int64_t)B * H, Sq, D).total;
+}
+
+int fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse, void* dq,
+           void* dk, void* dv, void* workspace, long long workspace_bytes, int B, int H, int Sq, int Sk, int D,
+           float scale, int causal, int dtype, cudaStream_t stream) {
+    if (B < 0 || H < 0 || Sq < 0 || Sk < 0) return FA_ERR_SHAPE;
+    if (D != 64 && D != 128) return FA_ERR_HEADDIM;
+    if (dtype != FA_FP16 && dtype != FA_BF16) return FA_ERR_DTYPE;
+    if (!(std::isfinite(scale) && scale > 0.f)) return FA_ERR_SCALE;
+    if (causal != 0 && causal != 1) return FA_ERR_ARG;
+    if (B == 0 || H == 0 || (Sq == 0 && Sk == 0)) return FA_OK;  // empty problem
+    if (Sk == 0 || (causal && Sq > Sk)) return FA_ERR_SHAPE;     // a query would see no key
+    const int64_t BH = (int64_t)B * H;
+    if (BH > INT_MAX || BH * (int64_t)Sq > INT_MAX || BH * (int64_t)Sk > INT_MAX || Sq > INT_MAX - 512 ||
+        Sk > INT_MAX - 512)
+        return FA_ERR_SHAPE;
+    if (Sq == 0) {
+        // no query: the key and value gradients are zero
+        if (!dk || !dv) return FA_ERR_NULL;
+        const size_t bytes = (size_t)BH * (size_t)Sk * (size_t)D * 2;
+        if (cudaMemsetAsync(dk, 0, bytes, stream) != cudaSuccess || cudaMemsetAsync(dv, 0, bytes, stream) != cudaSuccess) {
+            cudaGetLastError();
+            return FA_ERR_LAUNCH;
+        }
+        return FA_OK;
+    }
+    if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv) return FA_ERR_NULL;
+    const fa::BwdWorkspace ws = fa::bwd_workspace_layout(BH, Sq, D);
+    if (!workspace || ((uintptr_t)workspace & 255u) != 0 || workspace_bytes < ws.total) return FA_ERR_WORKSPACE;
+    const uintptr_t a16 = (uintptr_t)q | (uintptr_t)k | (uintptr_t)v | (uintptr_t)o | (uintptr_t)dout |
+                          (uintptr_t)dq | (uintptr_t)dk | (uintptr_t)dv;
+    if ((a16 & 15u) != 0 || ((uintptr_t)lse & 3u) != 0) return FA_ERR_ALIGN;
+
+    DeviceInfo dev;
+    int rc = device_info(&dev);
+    if (rc != FA_OK) return rc;
+    if (dev.major != 10 || dev.minor != 0) return FA_ERR_ARCH;
+    int cur = 0;
+    cudaGetDevice(&cur);
+    const void* ptrs[10] = {q, k, v, o, dout, lse, dq, dk, dv, workspace};
+    for (const void* p : ptrs) {
+        rc = check_device_pointer(p, cur);
+        if (rc != FA_OK) return rc;
+    }
+    long long qs[3], ks[3];
+    resolve_strides(nullptr, B, H, Sq, D, qs);
+    resolve_strides(nullptr, B, H, Sk, D, ks);
+    fa::BwdLaunchArgs a;
+    std::memset(&a, 0, sizeof(a));
+    if (!encode_tensor(&a.tmap_q, q, B, H, Sq, D, qs, dtype) || !encode_tensor(&a.tmap_do, dout, B, H, Sq, D, qs, dtype) ||
+        !encode_tensor(&a.tmap_k, k, B, H, Sk, D, ks, dtype) || !encode_tensor(&a.tmap_v, v, B, H, Sk, D, ks, dtype))
+        return FA_ERR_LAUNCH;
+    uint8_t* w = static_cast<uint8_t*>(workspace);
+    a.o = o;
+    a.dout = dout;
+    a.lse = lse;
+    a.dq = dq;
+    a.dk = dk;
+    a.dv = dv;
+    a.dq_acc = reinterpret_cast<float*>(w + ws.dq_acc);
+    a.lse2 = reinterpret_cast<float*>(w + ws.lse2);
+    a.delta = reinterpret_cast<float*>(w + ws.delta);
+    a.sched = reinterpret_cast<unsigned int*>(w + ws.sched);
+    a.B = B;
+    a.H = H;
+    a.Sq = Sq;
+    a.Sk = Sk;
+    a.D = D;
+    a.dtype = dtype;
+    a.causal = causal;
+    a.scale = scale;
+    const int64_t units = BH * ((Sk + 127) / 128);
+    a.grid = (int)(units < dev.sms ? units : dev.sms);
+    if (fa::launch_bwd_sm100(a, stream) != cudaSuccess) {
+        cudaGetLastError();
+        return FA_ERR_LAUNCH;
+    }
+    if (cudaPeekAtLastError() != cudaSuccess) {
+        cudaGetLastError();
+        return FA_ERR_LAUNCH;
+    }
+    return FA_OK;
+}
+
 int fa_check_status(cudaStream_t stream) {
-    int st = 0, site = 0;
-    if (fa::read_and_clear_status(stream, &st, &site) != cudaSuccess) {
+    int st = 0, site = 0, st_b = 0, site_b = 0;
+    if (fa::read_and_clear_status(stream, &st, &site) != cudaSuccess ||
+        fa::read_and_clear_status_bwd(stream, &st_b, &site_b) != cudaSuccess) {
         cudaGetLastError();
         return FA_ERR_LAUNCH;
     }
     if (st != fa::DEV_OK) {
         t_last_site = site;
+        return FA_ERR_TIMEOUT;
+    }
+    if (st_b != fa::DEV_OK) {
+        t_last_site = site_b;
         return FA_ERR_TIMEOUT;
     }
     return FA_OK;
@@ -321,6 +415,7 @@ const char* fa_status_string(int status) {
         case FA_ERR_ARG: return "causal must be 0 or 1";
         case FA_ERR_PTR: return "pointer is not device memory of the current device";
         case FA_ERR_STRIDE: return "a stride is not positive, a multiple of 8 elements and below 2^36";
+        case FA_ERR_WORKSPACE: return "workspace is NULL, not 256-byte aligned or smaller than fa_bwd_workspace_size";
         default: return "unknown status";
     }
 }

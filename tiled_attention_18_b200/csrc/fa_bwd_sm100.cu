@@ -1,0 +1,728 @@
+// fa_bwd_sm100.cu -- attention backward pass (dQ, dK, dV) for B200 (sm_100a).
+//
+// Gradients of O = softmax(scale * Q K^T [+ causal]) V for an upstream
+// gradient dO, by the FlashAttention-2 recomputation scheme: the forward pass
+// keeps only O and the per-row log-sum-exp; the backward pass recomputes the
+// scores and weights tile by tile instead of storing the S x S matrix
+// ("FlashAttention-2 在昇腾 NPU 上如何做到 3 倍加速？深度拆解 ops-transformer 的实现",
+// the recomputation row of the core-optimisation table and section 6.2; the
+// backward configuration of the gsyq.cn catlass FlashAttention page,
+// "反向传播的特殊处理", whose non-deterministic mode accumulates with atomic
+// adds, as dQ does here).
+//
+// With P_ij = exp(scale * q_i.k_j - LSE_i), dP_ij = dO_i.v_j and
+// Delta_i = sum_d dO_id O_id (= sum_j P_ij dP_ij):
+//   dV_j = sum_i P_ij dO_i
+//   dS_ij = P_ij (dP_ij - Delta_i)
+//   dK_j = scale * sum_i dS_ij q_i
+//   dQ_i = scale * sum_j dS_ij k_j
+//
+// Three launches on the caller's stream:
+//   1. bwd_prep_kernel: Delta_i, LSE_i * log2(e) (rows padded to a multiple of
+//      128: +inf, so that their weights are 0) and a zeroed fp32 dQ accumulator;
+//   2. fa_bwd_kernel: one persistent CTA per SM; a work unit is (b, h, 128-key
+//      tile).  The CTA keeps K_n, V_n in shared memory and dK, dV in tensor
+//      memory and walks the 128-row query tiles that see its keys:
+//        S^T = K Q_m^T, dP^T = V dO_m^T   (tcgen05.mma, fp32 in TMEM)
+//        P^T, dS^T                          (one key row per thread, packed to
+//                                            16 bits in TMEM; dS^T also to SMEM)
+//        dV += P^T dO_m, dK += dS^T Q_m     (A operand from TMEM)
+//        dQ_m = dS K                        (A = dS from SMEM, MN-major)
+//      dQ_m is added to the fp32 accumulator with vector reductions; dK, dV
+//      are written once per unit;
+//   3. bwd_post_kernel: dQ = scale * accumulator, rounded to the 16-bit dtype.
+//
+// Every mbarrier wait is bounded like the forward kernel's (abort flag, status
+// word read by fa_check_status, drained copies, TMEM freed).
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "fa_internal.h"
+
+namespace fa {
+namespace {
+
+// Status words of this translation unit (see read_and_clear_status_bwd).
+__device__ int g_status = 0;
+__device__ int g_status_site = 0;
+
+#include "sm100_helpers.cuh"
+
+constexpr int BWD_THREADS = 384;   // 12 warps
+constexpr int BW_TMA = 0;          // warp 0 lane 0: TMA loads and unit claims
+constexpr int BW_MMA = 1;          // warp 1 lane 0: every tcgen05.mma; TMEM owner
+constexpr int TILE = 128;          // keys per unit and query rows per step
+constexpr uint32_t BWD_TMEM_COLS = 512;
+constexpr uint32_t UNIT_READERS_BWD = 1 + 2 * TILE;  // MMA lane + two warpgroups
+
+// Tensor-memory columns: S^T/P^T, dP^T/dS^T, the dV and dK accumulators and
+// dQ of one step.  At D = 128 the 512 columns are used up, so dQ_m lands in
+// the dP^T columns (free once dK has read dS^T); at D = 64 it has its own.
+constexpr uint32_t COL_S = 0;
+constexpr uint32_t COL_DP = 128;
+constexpr uint32_t COL_DV = 256;
+template <int D>
+struct Cols {
+    static constexpr uint32_t DK = COL_DV + D;
+    static constexpr uint32_t DQ = (D == 128) ? COL_DP : COL_DV + 2 * D;
+    static_assert(DQ + D <= BWD_TMEM_COLS || DQ == COL_DP, "tensor memory budget");
+};
+
+template <int D>
+struct BwdSmem {
+    static constexpr int CHUNKS = D / 64;           // 128-byte column chunks of a tile
+    static constexpr int CHUNK_BYTES = TILE * 128;  // 128 rows x 64 elements x 2 bytes
+    static constexpr int TILE_BYTES = TILE * D * 2;
+    static constexpr int NSTAGE = (D == 128) ? 1 : 2;
+    static constexpr int K_OFF = 0;
+    static constexpr int V_OFF = TILE_BYTES;
+    static constexpr int STAGE_OFF = 2 * TILE_BYTES;        // stage: Q_m, dO_m
+    static constexpr int STAGE_BYTES = 2 * TILE_BYTES;
+    static constexpr int DS_OFF = STAGE_OFF + NSTAGE * STAGE_BYTES;  // dS^T [128 keys][128 queries]
+    static constexpr int DS_BYTES = TILE * TILE * 2;
+    static constexpr int STATS_OFF = DS_OFF + DS_BYTES;      // per stage: lse2[128], delta[128]
+    static constexpr int STATS_BYTES = 2 * TILE * 4;
+    static constexpr int BAR_OFF = STATS_OFF + NSTAGE * STATS_BYTES;
+    enum {
+        B_KVFULL = 0,
+        B_KVEMPTY,
+        B_SFULL,
+        B_PFULL,
+        B_DSEMPTY,
+        B_DQFULL,
+        B_DQEMPTY,
+        B_DKVFULL,
+        B_DKVEMPTY,
+        B_FIN,
+        B_UFULL,               // [2]
+        B_UEMPTY = B_UFULL + 2,  // [2]
+        B_QFULL = B_UEMPTY + 2,  // [NSTAGE]
+        B_QEMPTY = B_QFULL + NSTAGE,
+        NBAR = B_QEMPTY + NSTAGE
+    };
+    static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;  // [0] TMEM base, [1] abort flag
+    static constexpr int UNIT_OFF = MISC_OFF + 16;       // unit ring, int[2]
+    static constexpr int BYTES = UNIT_OFF + 8;
+    static constexpr int ALLOC = BYTES + 1024;           // slack for 1 KiB alignment
+};
+
+struct BwdParams {
+    CUtensorMap tmap_q;
+    CUtensorMap tmap_k;
+    CUtensorMap tmap_v;
+    CUtensorMap tmap_do;
+    const float* lse2;    // [BH][Sq_pad] LSE * log2(e), +inf on padded rows
+    const float* delta;   // [BH][Sq_pad] rowsum(dO * O), 0 on padded rows
+    float* dq_acc;        // [BH][Sq][D] fp32, zeroed by the prep kernel
+    uint8_t* dk;          // [BH][Sk][D] 16-bit
+    uint8_t* dv;
+    int BH, H, Sq, Sk, Sq_pad, n_mtiles, n_ktiles, n_units, causal, causal_off;
+    float scale_log2;     // scale * log2(e)
+    float scale;
+    unsigned int* sched;  // zeroed unit counter (causal), or null
+};
+
+struct BUnit {
+    int bh;
+    int n;      // key tile
+    int m_lo;   // first query tile that sees a key of the tile
+    int T;      // query tiles visited
+};
+
+// Units: with the causal mask the number of query tiles falls with the key
+// tile index, so units are claimed in key-tile order (longest first), heads
+// innermost; without it, heads outermost (CTAs running together share one
+// head's Q and dO in L2).
+__device__ __forceinline__ BUnit decode_bwd_unit(const BwdParams& p, int u) {
+    BUnit U;
+    if (p.causal) {
+        U.n = u / p.BH;
+        U.bh = u - U.n * p.BH;
+        // query q sees key j iff j <= q + causal_off: the first query that sees
+        // key n*128 is n*128 - causal_off
+        const int q_first = U.n * TILE - p.causal_off;
+        U.m_lo = q_first > 0 ? q_first / TILE : 0;
+    } else {
+        U.bh = u / p.n_ktiles;
+        U.n = u - U.bh * p.n_ktiles;
+        U.m_lo = 0;
+    }
+    U.T = p.n_mtiles - U.m_lo;
+    return U;
+}
+
+__host__ __device__ constexpr uint32_t make_idesc_bwd(bool bf16, int N, bool a_mn_major, bool b_mn_major) {
+    return (1u << 4)                                   // D format: f32
+           | ((bf16 ? 1u : 0u) << 7)                   // A format
+           | ((bf16 ? 1u : 0u) << 10)                  // B format
+           | ((a_mn_major ? 1u : 0u) << 15)            // A major
+           | ((b_mn_major ? 1u : 0u) << 16)            // B major
+           | ((uint32_t)(N >> 3) << 17)                // N / 8
+           | ((uint32_t)(TILE >> 4) << 24);            // M / 16 (M = 128)
+}
+
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+    asm volatile("cp.async.bulk.shared::cta.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+                 "l"(src), "r"(bytes), "r"(bar)
+                 : "memory");
+}
+
+__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
+    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
+                 : "memory");
+}
+
+__device__ __forceinline__ void fence_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Reads the work-unit indices published by the TMA lane (same protocol as the
+// forward kernel's ring): -1 when the CTA has no more work, -2 on abort.
+template <int D>
+struct BwdUnitReader {
+    int slot = 0;
+    uint32_t phase = 0;
+    __device__ __forceinline__ int next(uint8_t* smem, volatile uint32_t* abort_flag, int site) {
+        using L = BwdSmem<D>;
+        const uint32_t bar0 = smem_u32(smem) + L::BAR_OFF;
+        if (!mbar_wait(bar0 + 8u * (uint32_t)(L::B_UFULL + slot), phase, abort_flag, site)) return -2;
+        const int u = reinterpret_cast<volatile int*>(smem + L::UNIT_OFF)[slot];
+        mbar_arrive(bar0 + 8u * (uint32_t)(L::B_UEMPTY + slot));
+        if (++slot == 2) { slot = 0; phase ^= 1u; }
+        return u;
+    }
+};
+
+template <int D>
+__device__ void bwd_producer(const BwdParams& p, uint8_t* smem, volatile uint32_t* abort_flag) {
+    using L = BwdSmem<D>;
+    const uint32_t base = smem_u32(smem);
+    const uint32_t bar0 = base + L::BAR_OFF;
+    auto bar = [&](int i) { return bar0 + 8u * (uint32_t)i; };
+    volatile int* ring = reinterpret_cast<volatile int*>(smem + L::UNIT_OFF);
+    int uslot = 0;
+    uint32_t uphase = 0, kv_phase = 0, phase = 0;
+    int stage = 0;
+    bool ok = true;
+    int kv_fill = -1;             // parity of the last K/V fill, -1 if none
+    uint32_t fill_mask = 0, fill_parity = 0;
+    for (int k = 0;; ++k) {
+        int u = p.sched ? (int)atomicAdd(p.sched, 1u) : (int)blockIdx.x + k * (int)gridDim.x;
+        if (u >= p.n_units) u = -1;
+        if (!mbar_wait(bar(L::B_UEMPTY + uslot), uphase ^ 1u, abort_flag, 40)) { ok = false; break; }
+        ring[uslot] = u;
+        mbar_arrive(bar(L::B_UFULL + uslot));
+        if (++uslot == 2) { uslot = 0; uphase ^= 1u; }
+        if (u < 0) break;
+        const BUnit U = decode_bwd_unit(p, u);
+        const int b = U.bh / p.H, h = U.bh - b * p.H;
+        if (!mbar_wait(bar(L::B_KVEMPTY), kv_phase ^ 1u, abort_flag, 41)) { ok = false; break; }
+        mbar_expect_tx(bar(L::B_KVFULL), 2 * L::TILE_BYTES);
+        kv_fill = (int)kv_phase;
+        kv_phase ^= 1u;
+#pragma unroll
+        for (int c = 0; c < L::CHUNKS; ++c) {
+            tma_load_4d(base + L::K_OFF + c * L::CHUNK_BYTES, &p.tmap_k, bar(L::B_KVFULL), c * 64, U.n * TILE, h, b);
+            tma_load_4d(base + L::V_OFF + c * L::CHUNK_BYTES, &p.tmap_v, bar(L::B_KVFULL), c * 64, U.n * TILE, h, b);
+        }
+        for (int t = 0; t < U.T; ++t) {
+            const int m = U.m_lo + t;
+            if (!mbar_wait(bar(L::B_QEMPTY + stage), phase ^ 1u, abort_flag, 42)) { ok = false; break; }
+            mbar_expect_tx(bar(L::B_QFULL + stage), 2 * L::TILE_BYTES + L::STATS_BYTES);
+            fill_mask |= 1u << stage;
+            fill_parity = (fill_parity & ~(1u << stage)) | (phase << stage);
+            const uint32_t dst = base + L::STAGE_OFF + stage * L::STAGE_BYTES;
+#pragma unroll
+            for (int c = 0; c < L::CHUNKS; ++c) {
+                tma_load_4d(dst + c * L::CHUNK_BYTES, &p.tmap_q, bar(L::B_QFULL + stage), c * 64, m * TILE, h, b);
+                tma_load_4d(dst + L::TILE_BYTES + c * L::CHUNK_BYTES, &p.tmap_do, bar(L::B_QFULL + stage), c * 64,
+                            m * TILE, h, b);
+            }
+            const size_t srow = (size_t)U.bh * (size_t)p.Sq_pad + (size_t)m * TILE;
+            const uint32_t sdst = base + L::STATS_OFF + stage * L::STATS_BYTES;
+            bulk_load(sdst, p.lse2 + srow, TILE * 4, bar(L::B_QFULL + stage));
+            bulk_load(sdst + TILE * 4, p.delta + srow, TILE * 4, bar(L::B_QFULL + stage));
+            if (++stage == L::NSTAGE) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+    }
+    if (!ok) {
+        for (int i = 0; i < L::NSTAGE; ++i)
+            if (fill_mask & (1u << i)) mbar_drain(bar(L::B_QFULL + i), (fill_parity >> i) & 1u);
+        if (kv_fill >= 0) mbar_drain(bar(L::B_KVFULL), (uint32_t)kv_fill);
+    }
+}
+
+template <int D, bool BF16>
+__device__ void bwd_mma(const BwdParams& p, uint8_t* smem, uint32_t tmem, volatile uint32_t* abort_flag) {
+    using L = BwdSmem<D>;
+    using C = Cols<D>;
+    const uint32_t base = smem_u32(smem);
+    const uint32_t bar0 = base + L::BAR_OFF;
+    auto bar = [&](int i) { return bar0 + 8u * (uint32_t)i; };
+    constexpr uint32_t IDESC_S = make_idesc_bwd(BF16, TILE, false, false);  // S^T, dP^T: N = 128 queries
+    constexpr uint32_t IDESC_KV = make_idesc_bwd(BF16, D, false, true);     // dV, dK: A in TMEM, B MN-major
+    constexpr uint32_t IDESC_DQ = make_idesc_bwd(BF16, D, true, true);      // dQ: A = dS MN-major, B = K MN-major
+    constexpr uint32_t MN_LBO = (D == 128) ? (uint32_t)L::CHUNK_BYTES : 1024u;
+
+    // K-major operands (K, V, Q, dO as [rows][D], 128-byte swizzle): a K step of
+    // 16 elements advances 32 bytes inside a swizzle atom and 16 KiB across
+    // 64-column chunks.  MN-major operands (Q, dO, K as [rows][D] read along D;
+    // dS^T as [keys][queries] read along the queries): 64-element chunks 16 KiB
+    // apart (leading byte offset), 8-row groups 1024 bytes apart; a K step of 16
+    // rows advances 2 KiB.
+    const uint64_t dk_k = sw128_desc(base + L::K_OFF, 16, 1024);
+    const uint64_t dv_k = sw128_desc(base + L::V_OFF, 16, 1024);
+    const uint64_t dstage_k = sw128_desc(base + L::STAGE_OFF, 16, 1024);
+    const uint64_t dstage_mn = sw128_desc(base + L::STAGE_OFF, MN_LBO, 1024);
+    const uint64_t dk_mn = sw128_desc(base + L::K_OFF, MN_LBO, 1024);
+    const uint64_t ds_mn = sw128_desc(base + L::DS_OFF, (uint32_t)L::CHUNK_BYTES, 1024);
+    constexpr uint32_t STAGE16 = (uint32_t)L::STAGE_BYTES >> 4;
+    constexpr uint32_t TILE16 = (uint32_t)L::TILE_BYTES >> 4;
+
+    // D(tmem) = A(smem, K-major over D) B(smem, K-major over D)^T
+    auto issue_kmajor = [&](uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t b_off16) {
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+            const uint32_t off = (uint32_t)(((ks & 3) * 32 + (ks >> 2) * L::CHUNK_BYTES) >> 4);
+            tc_mma_ss2(d_tmem, (uint32_t)a + off, (uint32_t)(a >> 32), (uint32_t)b + b_off16 + off,
+                       (uint32_t)(b >> 32), IDESC_S, ks > 0 ? 1u : 0u);
+        }
+    };
+    // D(tmem) (+)= A(tmem, 16-bit pairs) B(smem, MN-major), K = 128 rows
+    auto issue_ts = [&](uint32_t d_tmem, uint32_t a_tmem, uint64_t b, uint32_t b_off16, bool accumulate) {
+#pragma unroll
+        for (int ks = 0; ks < TILE / 16; ++ks)
+            tc_mma_ts2(d_tmem, a_tmem + (uint32_t)(ks * 8), (uint32_t)b + b_off16 + (uint32_t)(ks * (2048 >> 4)),
+                       (uint32_t)(b >> 32), IDESC_KV, (accumulate || ks > 0) ? 1u : 0u);
+    };
+
+    uint32_t kv_phase = 0, phase = 0, p_phase = 0, dqe_phase = 0, dkve_phase = 0;
+    int stage = 0;
+    BwdUnitReader<D> units;
+    for (;;) {
+        const int u = units.next(smem, abort_flag, 43);
+        if (u < 0) break;
+        const BUnit U = decode_bwd_unit(p, u);
+        if (!mbar_wait(bar(L::B_KVFULL), kv_phase, abort_flag, 44)) break;
+        kv_phase ^= 1u;
+        bool ok = true;
+        for (int t = 0; t < U.T; ++t) {
+            const int st = stage;
+            if (!mbar_wait(bar(L::B_QFULL + st), phase, abort_flag, 45)) { ok = false; break; }
+            if (++stage == L::NSTAGE) { stage = 0; phase ^= 1u; }
+            const uint32_t q_off16 = (uint32_t)st * STAGE16;
+            const uint32_t do_off16 = q_off16 + TILE16;
+            // S^T = K Q_m^T
+            issue_kmajor(tmem + COL_S, dk_k, dstage_k, q_off16);
+            // dP^T = V dO_m^T (at D = 128 these columns hold the previous dQ: wait for its read-out)
+            if (C::DQ == COL_DP) {
+                if (!mbar_wait(bar(L::B_DQEMPTY), dqe_phase ^ 1u, abort_flag, 46)) { ok = false; break; }
+                dqe_phase ^= 1u;
+                tc_fence_after();
+            }
+            issue_kmajor(tmem + COL_DP, dv_k, dstage_k, do_off16);
+            tc_commit(bar(L::B_SFULL));
+            // P^T and dS^T from the dS warpgroup
+            if (!mbar_wait(bar(L::B_PFULL), p_phase, abort_flag, 47)) { ok = false; break; }
+            p_phase ^= 1u;
+            tc_fence_after();
+            if (t == 0) {
+                // the previous unit's dK and dV have been read out
+                if (!mbar_wait(bar(L::B_DKVEMPTY), dkve_phase ^ 1u, abort_flag, 48)) { ok = false; break; }
+                dkve_phase ^= 1u;
+                tc_fence_after();
+            }
+            issue_ts(tmem + COL_DV, tmem + COL_S, dstage_mn, do_off16, t > 0);  // dV += P^T dO_m
+            issue_ts(tmem + C::DK, tmem + COL_DP, dstage_mn, q_off16, t > 0);  // dK += dS^T Q_m
+            tc_commit(bar(L::B_QEMPTY + st));
+            if (C::DQ != COL_DP) {
+                if (!mbar_wait(bar(L::B_DQEMPTY), dqe_phase ^ 1u, abort_flag, 46)) { ok = false; break; }
+                dqe_phase ^= 1u;
+                tc_fence_after();
+            }
+            // dQ_m = dS K: A = dS (queries x keys) read MN-major from dS^T, B = K read MN-major
+#pragma unroll
+            for (int ks = 0; ks < TILE / 16; ++ks) {
+                const uint32_t off = (uint32_t)(ks * (2048 >> 4));
+                tc_mma_ss2(tmem + C::DQ, (uint32_t)ds_mn + off, (uint32_t)(ds_mn >> 32), (uint32_t)dk_mn + off,
+                           (uint32_t)(dk_mn >> 32), IDESC_DQ, ks > 0 ? 1u : 0u);
+            }
+            tc_commit(bar(L::B_DQFULL));
+            tc_commit(bar(L::B_DSEMPTY));
+        }
+        if (!ok) break;
+        tc_commit(bar(L::B_DKVFULL));
+        tc_commit(bar(L::B_KVEMPTY));
+    }
+    // all MMAs issued by this thread have completed once B_FIN fires
+    tc_commit(bar(L::B_FIN));
+    mbar_drain(bar(L::B_FIN), 0u);
+}
+
+// P^T and dS^T: one key row per thread (TMEM lane), 32 queries at a time.
+template <int D, bool BF16>
+__device__ void bwd_ds_role(const BwdParams& p, uint8_t* smem, uint32_t tmem, int warp_in_group,
+                            volatile uint32_t* abort_flag) {
+    using L = BwdSmem<D>;
+    const uint32_t base = smem_u32(smem);
+    const uint32_t bar0 = base + L::BAR_OFF;
+    auto bar = [&](int i) { return bar0 + 8u * (uint32_t)i; };
+    const int lane = threadIdx.x & 31;
+    const int row = warp_in_group * 32 + lane;  // key row within the tile
+    const uint32_t lane_sel = (uint32_t)(warp_in_group * 32) << 16;
+    const float sl2 = p.scale_log2;
+    uint32_t s_phase = 0, dse_phase = 0, phase = 0;
+    int stage = 0;
+    // this thread's row of the dS^T tile: 128-byte rows, 8-row groups 1 KiB apart,
+    // 16-byte granules XOR-swizzled by the row index (the TMA/UMMA 128-byte swizzle)
+    uint8_t* ds_row = smem + L::DS_OFF + (row >> 3) * 1024 + (row & 7) * 128;
+    const int sw = row & 7;
+    BwdUnitReader<D> units;
+    for (;;) {
+        const int u = units.next(smem, abort_flag, 49);
+        if (!__all_sync(0xffffffffu, u != -2)) return;
+        if (u < 0) break;
+        const BUnit U = decode_bwd_unit(p, u);
+        const int key = U.n * TILE + row;
+        const bool key_ok = key < p.Sk;
+        const int q_min = p.causal ? key - p.causal_off : 0;  // first query that sees this key
+        for (int t = 0; t < U.T; ++t) {
+            const int m = U.m_lo + t;
+            const int st = stage;
+            const uint32_t st_phase = phase;
+            if (++stage == L::NSTAGE) { stage = 0; phase ^= 1u; }
+            if (!__all_sync(0xffffffffu, mbar_wait(bar(L::B_SFULL), s_phase, abort_flag, 50))) return;
+            s_phase ^= 1u;
+            // the stage's row statistics came with its TMA fill: observe that fill
+            // here too (the phase cannot move on before this warpgroup arrives on
+            // B_PFULL, since the stage is released only after the P.V / dS.Q MMAs)
+            if (!__all_sync(0xffffffffu, mbar_wait(bar(L::B_QFULL + st), st_phase, abort_flag, 55))) return;
+            // the previous dQ MMA has read the dS^T tile
+            if (!__all_sync(0xffffffffu, mbar_wait(bar(L::B_DSEMPTY), dse_phase ^ 1u, abort_flag, 51))) return;
+            dse_phase ^= 1u;
+            tc_fence_after();
+            const float* lse2s = reinterpret_cast<const float*>(smem + L::STATS_OFF + st * L::STATS_BYTES);
+            const float* dls = lse2s + TILE;
+            const bool need_mask = !key_ok || (m * TILE < q_min);
+#pragma unroll 1
+            for (int c = 0; c < 4; ++c) {
+                uint32_t sr[32], dr[32];
+                tmem_ld32u(tmem + lane_sel + COL_S + 32 * c, sr);
+                tmem_ld32u(tmem + lane_sel + COL_DP + 32 * c, dr);
+                uint32_t pk[16], dk[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const int j = 32 * c + 2 * i;
+                    const float2 l2 = *reinterpret_cast<const float2*>(lse2s + j);
+                    const float2 dl = *reinterpret_cast<const float2*>(dls + j);
+                    float p0 = ex2(fmaf(__uint_as_float(sr[2 * i]), sl2, -l2.x));
+                    float p1 = ex2(fmaf(__uint_as_float(sr[2 * i + 1]), sl2, -l2.y));
+                    if (need_mask) {
+                        const int q = m * TILE + j;
+                        if (!key_ok || q < q_min) p0 = 0.f;
+                        if (!key_ok || q + 1 < q_min) p1 = 0.f;
+                    }
+                    const float d0 = p0 * (__uint_as_float(dr[2 * i]) - dl.x);
+                    const float d1 = p1 * (__uint_as_float(dr[2 * i + 1]) - dl.y);
+                    pk[i] = pack2<BF16>(p0, p1);
+                    dk[i] = pack2<BF16>(d0, d1);
+                }
+                tmem_st16(tmem + lane_sel + COL_S + 16 * c, pk);
+                tmem_st16(tmem + lane_sel + COL_DP + 16 * c, dk);
+                // queries 32c .. 32c+31 of this key row: chunk c/2, granules (c%2)*4 .. +3
+                uint8_t* chunk = ds_row + (c >> 1) * L::CHUNK_BYTES;
+#pragma unroll
+                for (int g = 0; g < 4; ++g) {
+                    const int gr = ((c & 1) * 4 + g) ^ sw;
+                    *reinterpret_cast<uint4*>(chunk + gr * 16) =
+                        make_uint4(dk[4 * g], dk[4 * g + 1], dk[4 * g + 2], dk[4 * g + 3]);
+                }
+            }
+            tmem_wait_st();
+            fence_async_smem();
+            tc_fence_before();
+            mbar_arrive(bar(L::B_PFULL));
+        }
+    }
+}
+
+// dQ_m read-out (one query row per thread) into the fp32 accumulator, and the
+// unit's dK, dV (one key row per thread) to global memory.
+template <int D, bool BF16>
+__device__ void bwd_out_role(const BwdParams& p, uint8_t* smem, uint32_t tmem, int warp_in_group,
+                             volatile uint32_t* abort_flag) {
+    using L = BwdSmem<D>;
+    using C = Cols<D>;
+    const uint32_t base = smem_u32(smem);
+    const uint32_t bar0 = base + L::BAR_OFF;
+    auto bar = [&](int i) { return bar0 + 8u * (uint32_t)i; };
+    const int lane = threadIdx.x & 31;
+    const int row = warp_in_group * 32 + lane;
+    const uint32_t lane_sel = (uint32_t)(warp_in_group * 32) << 16;
+    uint32_t dq_phase = 0, dkv_phase = 0;
+    BwdUnitReader<D> units;
+    for (;;) {
+        const int u = units.next(smem, abort_flag, 52);
+        if (!__all_sync(0xffffffffu, u != -2)) return;
+        if (u < 0) break;
+        const BUnit U = decode_bwd_unit(p, u);
+        for (int t = 0; t < U.T; ++t) {
+            const int m = U.m_lo + t;
+            if (!__all_sync(0xffffffffu, mbar_wait(bar(L::B_DQFULL), dq_phase, abort_flag, 53))) return;
+            dq_phase ^= 1u;
+            tc_fence_after();
+            const int q = m * TILE + row;
+            const bool valid = q < p.Sq;
+            float* dst = p.dq_acc + ((size_t)U.bh * (size_t)p.Sq + (size_t)(valid ? q : 0)) * D;
+#pragma unroll 1
+            for (int c = 0; c < D / 32; ++c) {
+                uint32_t r[32];
+                tmem_ld32u(tmem + lane_sel + C::DQ + 32 * c, r);
+                if (valid) {
+#pragma unroll
+                    for (int i = 0; i < 8; ++i)
+                        red_add_v4(dst + 32 * c + 4 * i, __uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]),
+                                   __uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3]));
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(bar(L::B_DQEMPTY));
+        }
+        if (!__all_sync(0xffffffffu, mbar_wait(bar(L::B_DKVFULL), dkv_phase, abort_flag, 54))) return;
+        dkv_phase ^= 1u;
+        tc_fence_after();
+        const int key = U.n * TILE + row;
+        const bool valid = key < p.Sk;
+        const size_t off = ((size_t)U.bh * (size_t)p.Sk + (size_t)(valid ? key : 0)) * (size_t)(D * 2);
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+            uint32_t r[32];
+            uint32_t w[16];
+            tmem_ld32u(tmem + lane_sel + COL_DV + 32 * c, r);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) w[i] = pack2<BF16>(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
+            if (valid) {
+                uint4* d = reinterpret_cast<uint4*>(p.dv + off + c * 64);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) d[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+            }
+            tmem_ld32u(tmem + lane_sel + C::DK + 32 * c, r);
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+                w[i] = pack2<BF16>(__uint_as_float(r[2 * i]) * p.scale, __uint_as_float(r[2 * i + 1]) * p.scale);
+            if (valid) {
+                uint4* d = reinterpret_cast<uint4*>(p.dk + off + c * 64);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) d[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+            }
+        }
+        tc_fence_before();
+        mbar_arrive(bar(L::B_DKVEMPTY));
+    }
+}
+
+template <int D, bool BF16>
+__global__ void __launch_bounds__(BWD_THREADS, 1) fa_bwd_kernel(const __grid_constant__ BwdParams p) {
+    using L = BwdSmem<D>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t base = smem_u32(smem);
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int wg = warp >> 2;
+    uint32_t* misc = reinterpret_cast<uint32_t*>(smem + L::MISC_OFF);
+    volatile uint32_t* abort_flag = misc + 1;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < L::NBAR; ++i) {
+            uint32_t count = 1;  // TMA transaction or tcgen05.commit arrivals
+            if (i == L::B_PFULL || i == L::B_DQEMPTY || i == L::B_DKVEMPTY) count = TILE;  // one warpgroup
+            if (i >= L::B_UEMPTY && i < L::B_UEMPTY + 2) count = UNIT_READERS_BWD;
+            mbar_init(base + L::BAR_OFF + 8 * i, count);
+        }
+        *abort_flag = 0u;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    }
+    if (warp == BW_TMA && lane == 0) {
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&p.tmap_q)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&p.tmap_k)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&p.tmap_v)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&p.tmap_do)) : "memory");
+    }
+    if (warp == BW_MMA) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(misc)),
+                     "r"(BWD_TMEM_COLS)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = misc[0];
+
+    if (wg == 0) {
+        if (warp == BW_TMA && lane == 0) bwd_producer<D>(p, smem, abort_flag);
+        if (warp == BW_MMA && lane == 0) bwd_mma<D, BF16>(p, smem, tmem, abort_flag);
+    } else if (wg == 1) {
+        bwd_ds_role<D, BF16>(p, smem, tmem, warp & 3, abort_flag);
+    } else {
+        bwd_out_role<D, BF16>(p, smem, tmem, warp & 3, abort_flag);
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == BW_MMA) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(BWD_TMEM_COLS)
+                     : "memory");
+    }
+}
+
+template <bool BF16>
+__device__ __forceinline__ float load16(const uint16_t* p) {
+    const uint16_t x = *p;
+    if constexpr (BF16) return __bfloat162float(__ushort_as_bfloat16(x));
+    else return __half2float(__ushort_as_half(x));
+}
+
+// One warp per (bh, query row) of the padded row range: Delta = sum_d dO O in
+// fp32, LSE * log2(e), and the row of the dQ accumulator cleared.  Padded rows
+// get +inf (weight 0) and Delta = 0.  Block (0, 0) also clears the scheduler
+// counter, which the main kernel (next on the stream) reads.
+template <int D, bool BF16>
+__global__ void __launch_bounds__(256) bwd_prep_kernel(const uint16_t* __restrict__ o, const uint16_t* __restrict__ dout,
+                                                       const float* __restrict__ lse, float* __restrict__ lse2,
+                                                       float* __restrict__ delta, float* __restrict__ dq_acc, int Sq,
+                                                       int Sq_pad, unsigned int* sched) {
+    constexpr int PER_LANE = D / 32;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int row = blockIdx.x * 8 + warp;
+    const size_t bh = blockIdx.y;
+    if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0 && sched) *sched = 0u;
+    if (row >= Sq_pad) return;
+    if (row >= Sq) {
+        if (lane == 0) {
+            lse2[bh * Sq_pad + row] = __int_as_float(0x7f800000);  // +inf
+            delta[bh * Sq_pad + row] = 0.f;
+        }
+        return;
+    }
+    const size_t e0 = (bh * (size_t)Sq + (size_t)row) * D + (size_t)lane * PER_LANE;
+    float acc = 0.f;
+#pragma unroll
+    for (int i = 0; i < PER_LANE; ++i) acc = fmaf(load16<BF16>(o + e0 + i), load16<BF16>(dout + e0 + i), acc);
+#pragma unroll
+    for (int s = 16; s > 0; s >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, s);
+#pragma unroll
+    for (int i = 0; i < PER_LANE; ++i) dq_acc[e0 + i] = 0.f;
+    if (lane == 0) {
+        lse2[bh * Sq_pad + row] = lse[bh * (size_t)Sq + row] * 1.4426950408889634f;
+        delta[bh * Sq_pad + row] = acc;
+    }
+}
+
+// dQ = scale * accumulator, rounded to the 16-bit dtype (4 elements per thread).
+template <bool BF16>
+__global__ void __launch_bounds__(256) bwd_post_kernel(const float4* __restrict__ acc, uint2* __restrict__ dq,
+                                                       size_t n4, float scale) {
+    for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n4; i += (size_t)gridDim.x * blockDim.x) {
+        const float4 a = acc[i];
+        dq[i] = make_uint2(pack2<BF16>(a.x * scale, a.y * scale), pack2<BF16>(a.z * scale, a.w * scale));
+    }
+}
+
+template <int D, bool BF16>
+cudaError_t launch_bwd_impl(const BwdLaunchArgs& a, cudaStream_t stream) {
+    using L = BwdSmem<D>;
+    static_assert(L::ALLOC <= 232448, "shared memory budget exceeded");
+    const int BH = a.B * a.H;
+    const int n_mtiles = (a.Sq + TILE - 1) / TILE;
+    const int Sq_pad = n_mtiles * TILE;
+    {
+        dim3 grid((unsigned)(Sq_pad / 8), (unsigned)BH, 1);
+        bwd_prep_kernel<D, BF16><<<grid, 256, 0, stream>>>(
+            static_cast<const uint16_t*>(a.o), static_cast<const uint16_t*>(a.dout), a.lse, a.lse2, a.delta,
+            a.dq_acc, a.Sq, Sq_pad, a.sched);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    {
+        auto kern = fa_bwd_kernel<D, BF16>;
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC);
+        if (e != cudaSuccess) return e;
+        BwdParams p;
+        p.tmap_q = a.tmap_q;
+        p.tmap_k = a.tmap_k;
+        p.tmap_v = a.tmap_v;
+        p.tmap_do = a.tmap_do;
+        p.lse2 = a.lse2;
+        p.delta = a.delta;
+        p.dq_acc = a.dq_acc;
+        p.dk = static_cast<uint8_t*>(a.dk);
+        p.dv = static_cast<uint8_t*>(a.dv);
+        p.BH = BH;
+        p.H = a.H;
+        p.Sq = a.Sq;
+        p.Sk = a.Sk;
+        p.Sq_pad = Sq_pad;
+        p.n_mtiles = n_mtiles;
+        p.n_ktiles = (a.Sk + TILE - 1) / TILE;
+        p.n_units = BH * p.n_ktiles;
+        p.causal = a.causal;
+        p.causal_off = a.Sk - a.Sq;
+        p.scale_log2 = a.scale * 1.4426950408889634f;
+        p.scale = a.scale;
+        p.sched = a.causal ? a.sched : nullptr;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)a.grid, 1, 1);
+        cfg.blockDim = dim3(BWD_THREADS, 1, 1);
+        cfg.dynamicSmemBytes = L::ALLOC;
+        cfg.stream = stream;
+        e = cudaLaunchKernelEx(&cfg, kern, p);
+        if (e != cudaSuccess) return e;
+    }
+    {
+        const size_t n4 = (size_t)BH * (size_t)a.Sq * D / 4;
+        const unsigned blocks = (unsigned)((n4 + 255) / 256 < 148u * 16u ? (n4 + 255) / 256 : 148u * 16u);
+        bwd_post_kernel<BF16><<<blocks, 256, 0, stream>>>(reinterpret_cast<const float4*>(a.dq_acc),
+                                                           static_cast<uint2*>(a.dq), n4, a.scale);
+        return cudaGetLastError();
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_bwd_sm100(const BwdLaunchArgs& a, cudaStream_t stream) {
+    if (a.D == 128) {
+        return a.dtype == 1 ? launch_bwd_impl<128, true>(a, stream) : launch_bwd_impl<128, false>(a, stream);
+    }
+    return a.dtype == 1 ? launch_bwd_impl<64, true>(a, stream) : launch_bwd_impl<64, false>(a, stream);
+}
+
+cudaError_t read_and_clear_status_bwd(cudaStream_t stream, int* status, int* site) {
+    cudaError_t e = cudaStreamSynchronize(stream);
+    if (e != cudaSuccess) return e;
+    int st = 0, si = 0;
+    e = cudaMemcpyFromSymbolAsync(&st, g_status, sizeof(int), 0, cudaMemcpyDeviceToHost, stream);
+    if (e == cudaSuccess)
+        e = cudaMemcpyFromSymbolAsync(&si, g_status_site, sizeof(int), 0, cudaMemcpyDeviceToHost, stream);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+    if (e != cudaSuccess) return e;
+    if (st != 0) {
+        const int zero = 0;
+        e = cudaMemcpyToSymbolAsync(g_status, &zero, sizeof(int), 0, cudaMemcpyHostToDevice, stream);
+        if (e == cudaSuccess)
+            e = cudaMemcpyToSymbolAsync(g_status_site, &zero, sizeof(int), 0, cudaMemcpyHostToDevice, stream);
+        if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+    }
+    *status = st;
+    *site = si;
+    return e;
+}
+
+}  // namespace fa

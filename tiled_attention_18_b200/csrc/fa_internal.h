@@ -40,6 +40,58 @@ struct LaunchArgs {
     unsigned int* sched;    // zeroed device counter for claimed-unit scheduling, or null
 };
 
+// Backward pass (fa_bwd): tensor maps as for the forward pass (Q, dO over
+// [B][H][Sq][D]; K, V over [B][H][Sk][D]), the forward outputs O and LSE, the
+// gradients, and the caller's workspace carved as bwd_workspace_layout says.
+struct BwdLaunchArgs {
+    CUtensorMap tmap_q;
+    CUtensorMap tmap_k;
+    CUtensorMap tmap_v;
+    CUtensorMap tmap_do;
+    const void* o;          // [B,H,Sq,D] 16-bit
+    const void* dout;       // [B,H,Sq,D] 16-bit
+    const float* lse;       // [B,H,Sq] fp32 (natural log)
+    void* dq;               // [B,H,Sq,D] 16-bit
+    void* dk;               // [B,H,Sk,D] 16-bit
+    void* dv;               // [B,H,Sk,D] 16-bit
+    float* dq_acc;          // workspace: [B*H][Sq][D] fp32
+    float* lse2;            // workspace: [B*H][Sq_pad] fp32
+    float* delta;           // workspace: [B*H][Sq_pad] fp32
+    unsigned int* sched;    // workspace: unit counter
+    int B;
+    int H;
+    int Sq;
+    int Sk;
+    int D;
+    int dtype;
+    int causal;
+    float scale;
+    int grid;
+};
+
+// Byte offsets of the backward workspace parts (each 256-byte aligned) and
+// its total size.  Sq_pad = Sq rounded up to a multiple of 128.
+struct BwdWorkspace {
+    int64_t dq_acc, lse2, delta, sched, total;
+};
+inline BwdWorkspace bwd_workspace_layout(int64_t BH, int64_t Sq, int64_t D) {
+    auto up = [](int64_t x) { return (x + 255) / 256 * 256; };
+    const int64_t Sq_pad = (Sq + 127) / 128 * 128;
+    BwdWorkspace w;
+    w.dq_acc = 0;
+    w.lse2 = up(BH * Sq * D * 4);
+    w.delta = w.lse2 + up(BH * Sq_pad * 4);
+    w.sched = w.delta + up(BH * Sq_pad * 4);
+    w.total = w.sched + 256;
+    return w;
+}
+
+// Launch the three backward kernels (prep, main, post) on `stream`.
+cudaError_t launch_bwd_sm100(const BwdLaunchArgs& a, cudaStream_t stream);
+
+// Status words of the backward kernels (same protocol as read_and_clear_status).
+cudaError_t read_and_clear_status_bwd(cudaStream_t stream, int* status, int* site);
+
 // Number of work units (b, h, 256-row query block).
 inline int64_t num_units(int64_t BH, int64_t S) {
     return BH * ((S + ROWS_PER_UNIT - 1) / ROWS_PER_UNIT);
