@@ -217,6 +217,186 @@ def run_reference(args):
     return 0
 
 
+BWD_FLOP_FACTOR = 2.5  # five S x S x D products in the backward pass against two in the forward pass
+
+
+def cpu_baseline_bwd(name: str, target_s: float = 12.0):
+    """The fp64 backward oracle on one head of the workload's first run with the
+    sequence cut to a length whose cost fits ``target_s``; TFLOP/s of that sample
+    (2.5x the forward's algorithmic flops of the sample)."""
+    import dataclasses as dc
+
+    import oracle
+    import torch
+    w = workload_runs(name)[-1]
+    S = 256
+    while True:
+        ws = dc.replace(w, B=1, H=1, S=min(S, w.S), Sk=(min(S, w.Skv) if w.Sk else 0))
+        q, k, v = workload_inputs(ws)
+        g = torch.Generator().manual_seed(5)
+        dout = torch.randn(q.shape, generator=g).to(q.dtype)
+        t0 = time.perf_counter()
+        oracle.attn_bwd(q, k, v, dout, ws.scale, ws.causal, ws.dtype)
+        dt = time.perf_counter() - t0
+        if dt >= target_s / 8 or S >= w.S:
+            break
+        S *= 2
+    flops = BWD_FLOP_FACTOR * ws.flops
+    return {"value": flops / dt / 1e12, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"fp64 backward oracle on one head of {ws.describe()} ({dt:.1f} s on the host cores)"}
+
+
+def run_bwd(args) -> int:
+    """Time fa_bwd (the backward pass) on the workload; O and LSE come from one
+    forward call before the timed region, dO is seeded random."""
+    import torch
+    import torch.distributed as dist
+
+    import tiled_attention_18_b200 as fa
+
+    rank, world, local = rank_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    fa.load()
+    runs = workload_runs(args.workload)
+    for w in runs:
+        if w.layout != "bhsd":
+            raise SystemExit("fa_bwd takes contiguous BHSD tensors; pick a BHSD workload")
+    stream = torch.cuda.current_stream(dev)
+    sid = stream.cuda_stream
+    bufs = []
+    for w in runs:
+        wr = dataclasses.replace(w, seed=rank_seed(w.seed, rank))
+        q, k, v = (t.to(dev) for t in workload_inputs(wr))
+        g = torch.Generator().manual_seed(rank_seed(w.seed, rank) + 7)
+        dout = torch.randn(q.shape, generator=g).to(q.dtype).to(dev)
+        o = torch.empty_like(q)
+        lse = torch.empty(q.shape[:3], dtype=torch.float32, device=dev)
+        dt = fa.FA_BF16 if w.dtype == "bf16" else fa.FA_FP16
+        st = fa.fa_fwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), w.B, w.H, w.S,
+                          w.Skv, w.D, None, None, None, None, w.scale, int(w.causal), dt, sid)
+        if st != 0:
+            raise fa.FaError(st)
+        nbytes = fa.fa_bwd_workspace_size(w.B, w.H, w.S, w.D)
+        bufs.append(dict(q=q, k=k, v=v, o=o, lse=lse, dout=dout, dq=torch.empty_like(q), dk=torch.empty_like(k),
+                         dv=torch.empty_like(v), ws=torch.empty(nbytes, dtype=torch.uint8, device=dev),
+                         nbytes=nbytes, dt=dt))
+
+    def launch(i):
+        w, b = runs[i], bufs[i]
+        st = fa.fa_bwd(b["q"].data_ptr(), b["k"].data_ptr(), b["v"].data_ptr(), b["o"].data_ptr(),
+                       b["dout"].data_ptr(), b["lse"].data_ptr(), b["dq"].data_ptr(), b["dk"].data_ptr(),
+                       b["dv"].data_ptr(), b["ws"].data_ptr(), b["nbytes"], w.B, w.H, w.S, w.Skv, w.D, w.scale,
+                       int(w.causal), b["dt"], sid)
+        if st != 0:
+            raise fa.FaError(st, "fa_bwd")
+
+    for _ in range(args.warmup):
+        for i in range(len(runs)):
+            launch(i)
+    torch.cuda.synchronize(dev)
+    st = fa.fa_check_status(sid)
+    if st != 0:
+        raise fa.FaError(st, "warm-up")
+    ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in runs]
+          for _ in range(args.steps)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.3)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    start.record(stream)
+    for s_ in range(args.steps):
+        for i in range(len(runs)):
+            ev[s_][i][0].record(stream)
+            launch(i)
+            ev[s_][i][1].record(stream)
+    stop.record(stream)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    sampler.stop()
+    st = fa.fa_check_status(sid)
+    if st != 0:
+        raise fa.FaError(st, "timed region")
+    kern_ms = np.array([[a.elapsed_time(b) for (a, b) in row] for row in ev])
+    max_ms = max_over_ranks(start.elapsed_time(stop), device=dev)
+    step_flops = BWD_FLOP_FACTOR * sum(w.flops for w in runs)
+    value = job_throughput(step_flops, args.steps, world, max_ms)
+    peak, peak_src = peak_tflops()
+    per_run = [{"run": w.describe(), "mean_ms": float(kern_ms[:, i].mean()),
+                "tflops": BWD_FLOP_FACTOR * w.flops / (float(kern_ms[:, i].mean()) * 1e-3) / 1e12}
+               for i, w in enumerate(runs)]
+    achieved = step_flops / (float(kern_ms.sum(axis=1).mean()) * 1e-3) / 1e12
+
+    e2e = None
+    if not args.no_e2e:
+        names_in = ("q", "k", "v", "o", "dout", "lse")
+        names_out = ("dq", "dk", "dv")
+        host = [{n: torch.empty(b[n].shape, dtype=b[n].dtype).pin_memory() for n in names_in + names_out}
+                for b in bufs]
+        for hb, b in zip(host, bufs):
+            for n in names_in:
+                hb[n].copy_(b[n])
+        h2d = sum(hb[n].numel() * hb[n].element_size() for hb in host for n in names_in)
+        d2h = sum(hb[n].numel() * hb[n].element_size() for hb in host for n in names_out)
+
+        def e2e_step():
+            for i, (hb, b) in enumerate(zip(host, bufs)):
+                for n in names_in:
+                    b[n].copy_(hb[n], non_blocking=True)
+                launch(i)
+                for n in names_out:
+                    hb[n].copy_(b[n], non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        e2e = {"value": job_throughput(step_flops, args.e2e_steps, world,
+                                       max_over_ranks(e0.elapsed_time(e1), device=dev)),
+               "unit": UNIT, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+    cb = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cb = cpu_baseline_bwd(args.workload)
+    if rank == 0:
+        w0 = runs[0]
+        line = {
+            "metric": "attention bwd TFLOPS (2.5x forward flops, causal-adjusted) and % of B200 dense bf16 peak",
+            "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": max_ms / args.steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": w0.dtype, "data": "synthetic",
+            "config": {"workload": "backward of " + workload_label(args.workload), "B": w0.B, "H": w0.H,
+                       "S": w0.S, "D": w0.D, "runs_per_step": len(runs),
+                       "l2": "inputs larger than L2 (no flush)" if sum(
+                           t.numel() * t.element_size() for t in (bufs[0]["q"], bufs[0]["k"], bufs[0]["v"],
+                                                                  bufs[0]["dout"])) > L2_BYTES
+                       else "inputs smaller than L2 (warm)",
+                       "parallelism": f"independent batch per GPU x{world}"},
+            "pct_of_peak": 100.0 * value / (peak * world),
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": UNIT,
+                         "frac": achieved / peak, "traffic": None, "peak_source": peak_src, "per_run": per_run},
+            "clocks": sampler.summary(),
+            "e2e": e2e,
+            "gpu_launches": 3 * len(runs) * args.steps,
+            "cpu_baseline": cb,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
 def main(argv=None) -> int:
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -227,11 +407,15 @@ def main(argv=None) -> int:
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--pass", dest="pass_", choices=["fwd", "bwd"], default="fwd",
+                    help="fwd: the forward pass (default); bwd: the backward pass fa_bwd")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":
         return run_reference(args)
+    if args.pass_ == "bwd":
+        return run_bwd(args)
 
     import torch
     import torch.distributed as dist
