@@ -99,12 +99,12 @@ EncodeTiledFn encoder() {
 // tcgen05 operand descriptors expect).  Rows past S read as zeros and never
 // bleed into the next head, whatever the layout.
 bool encode_tensor(CUtensorMap* map, const void* ptr, int B, int H, int S, int D, const long long st[3],
-                   int dtype) {
+                   int dtype, int box_rows = fa::BLOCK_M) {
     EncodeTiledFn enc = encoder();
     if (!enc) return false;
     const cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)S, (cuuint64_t)H, (cuuint64_t)B};
     const cuuint64_t strides[3] = {(cuuint64_t)st[2] * 2, (cuuint64_t)st[1] * 2, (cuuint64_t)st[0] * 2};
-    const cuuint32_t box[4] = {64, (cuuint32_t)fa::BLOCK_M, 1, 1};
+    const cuuint32_t box[4] = {64, (cuuint32_t)box_rows, 1, 1};
     const cuuint32_t elem[4] = {1, 1, 1, 1};
     const CUtensorMapDataType dt =
         dtype == FA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
@@ -333,7 +333,10 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const voi
     resolve_strides(nullptr, B, H, Sk, D, ks);
     fa::BwdLaunchArgs a;
     std::memset(&a, 0, sizeof(a));
-    if (!encode_tensor(&a.tmap_q, q, B, H, Sq, D, qs, dtype) || !encode_tensor(&a.tmap_do, dout, B, H, Sq, D, qs, dtype) ||
+    // the D = 128 backward kernel steps through 64 query rows at a time
+    const int q_box = (D == 128) ? 64 : fa::BLOCK_M;
+    if (!encode_tensor(&a.tmap_q, q, B, H, Sq, D, qs, dtype, q_box) ||
+        !encode_tensor(&a.tmap_do, dout, B, H, Sq, D, qs, dtype, q_box) ||
         !encode_tensor(&a.tmap_k, k, B, H, Sk, D, ks, dtype) || !encode_tensor(&a.tmap_v, v, B, H, Sk, D, ks, dtype))
         return FA_ERR_LAUNCH;
     uint8_t* w = static_cast<uint8_t*>(workspace);

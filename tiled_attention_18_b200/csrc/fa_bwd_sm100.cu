@@ -20,9 +20,11 @@
 // Three launches on the caller's stream:
 //   1. bwd_prep_kernel: Delta_i, LSE_i * log2(e) (rows padded to a multiple of
 //      128: +inf, so that their weights are 0) and a zeroed fp32 dQ accumulator;
-//   2. fa_bwd_kernel: one persistent CTA per SM; a work unit is (b, h, 128-key
-//      tile).  The CTA keeps K_n, V_n in shared memory and dK, dV in tensor
-//      memory and walks the 128-row query tiles that see its keys:
+//   2. the fused kernel: one persistent CTA per SM; a work unit is (b, h,
+//      128-key tile).  The CTA keeps K_n, V_n in shared memory and dK, dV in
+//      tensor memory and walks the query rows that see its keys (D = 64,
+//      fa_bwd_kernel: 128-row steps; D = 128, fa_bwd_kernel_d128: 64-row steps
+//      with double-buffered scores, see below):
 //        S^T = K Q_m^T, dP^T = V dO_m^T   (tcgen05.mma, fp32 in TMEM)
 //        P^T, dS^T                          (one key row per thread, packed to
 //                                            16 bits in TMEM; dS^T also to SMEM)
@@ -58,9 +60,9 @@ constexpr int TILE = 128;          // keys per unit and query rows per step
 constexpr uint32_t BWD_TMEM_COLS = 512;
 constexpr uint32_t UNIT_READERS_BWD = 1 + 2 * TILE;  // MMA lane + two warpgroups
 
-// Tensor-memory columns: S^T/P^T, dP^T/dS^T, the dV and dK accumulators and
-// dQ of one step.  At D = 128 the 512 columns are used up, so dQ_m lands in
-// the dP^T columns (free once dK has read dS^T); at D = 64 it has its own.
+// Tensor-memory columns of fa_bwd_kernel (D = 64): S^T/P^T, dP^T/dS^T, the dV
+// and dK accumulators and dQ of one step (the template also fits D = 128 by
+// putting dQ_m in the dP^T columns, but D = 128 runs fa_bwd_kernel_d128).
 constexpr uint32_t COL_S = 0;
 constexpr uint32_t COL_DP = 128;
 constexpr uint32_t COL_DV = 256;
@@ -76,7 +78,7 @@ struct BwdSmem {
     static constexpr int CHUNKS = D / 64;           // 128-byte column chunks of a tile
     static constexpr int CHUNK_BYTES = TILE * 128;  // 128 rows x 64 elements x 2 bytes
     static constexpr int TILE_BYTES = TILE * D * 2;
-    static constexpr int NSTAGE = (D == 128) ? 1 : 2;
+    static constexpr int NSTAGE = 2;
     static constexpr int K_OFF = 0;
     static constexpr int V_OFF = TILE_BYTES;
     static constexpr int STAGE_OFF = 2 * TILE_BYTES;        // stage: Q_m, dO_m
@@ -583,6 +585,466 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) fa_bwd_kernel(const __grid_con
     }
 }
 
+// ------------------------------------------------------------------------
+// D = 128: 64-row query steps with double-buffered S^T / dP^T.
+//
+// Tensor memory: S0 [0,64) dP0 [64,128) S1 [128,192) dP1 [192,256), dV
+// [256,384), dK [384,512).  While the dS warpgroup turns step g's S^T, dP^T
+// (buffer g&1) into P^T, dS^T, the MMA lane already computes step g+1's into
+// the other buffer; then dV += P^T dO, dK += dS^T Q and dQ^T = K^T dS^T (M = D
+// = 128 lanes, N = 64 queries) into step g's S columns, which the output
+// warpgroup reads out (one head-dimension lane per thread) into the fp32 dQ
+// accumulator.  Q and dO stream through three 32 KiB stages.  Every role
+// derives buffer, stage and barrier parities from the global step count g.
+constexpr int QM = 64;  // query rows per step
+
+struct Bwd2Smem {
+    static constexpr int D = 128;
+    static constexpr int KCHUNK = TILE * 128;        // K/V: [128 rows][64 cols] per chunk
+    static constexpr int QCHUNK = QM * 128;          // Q/dO: [64 rows][64 cols] per chunk
+    static constexpr int KV_TILE = TILE * D * 2;     // 32 KiB
+    static constexpr int Q_TILE = QM * D * 2;        // 16 KiB
+    static constexpr int NSTAGE = 3;
+    static constexpr int K_OFF = 0;
+    static constexpr int V_OFF = KV_TILE;
+    static constexpr int STAGE_OFF = 2 * KV_TILE;    // stage: Q_m, dO_m
+    static constexpr int STAGE_BYTES = 2 * Q_TILE;
+    static constexpr int DS_OFF = STAGE_OFF + NSTAGE * STAGE_BYTES;  // dS^T [2][128 keys][64 queries]
+    static constexpr int DS_BYTES = TILE * QM * 2;                 // 16 KiB
+    static constexpr int STATS_OFF = DS_OFF + 2 * DS_BYTES;          // per stage: lse2[64], delta[64]
+    static constexpr int STATS_BYTES = 2 * QM * 4;
+    static constexpr int BAR_OFF = STATS_OFF + NSTAGE * STATS_BYTES;
+    enum {
+        B_KVFULL = 0,
+        B_KVEMPTY,
+        B_DKVFULL,
+        B_DKVEMPTY,
+        B_FIN,
+        B_UFULL,                    // [2]
+        B_UEMPTY = B_UFULL + 2,     // [2]
+        B_SFULL = B_UEMPTY + 2,     // [2] per buffer
+        B_PFULL = B_SFULL + 2,      // [2]
+        B_DQFULL = B_PFULL + 2,     // [2]
+        B_DQEMPTY = B_DQFULL + 2,   // [2]
+        B_DSEMPTY = B_DQEMPTY + 2,  // [2]
+        B_QFULL = B_DSEMPTY + 2,    // [NSTAGE]
+        B_QEMPTY = B_QFULL + NSTAGE,
+        NBAR = B_QEMPTY + NSTAGE
+    };
+    static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
+    static constexpr int UNIT_OFF = MISC_OFF + 16;
+    static constexpr int BYTES = UNIT_OFF + 8;
+    static constexpr int ALLOC = BYTES + 1024;
+};
+
+constexpr uint32_t COL2_DV = 256;
+constexpr uint32_t COL2_DK = 384;
+__device__ __forceinline__ uint32_t col2_s(uint32_t b) { return 128u * b; }
+__device__ __forceinline__ uint32_t col2_dp(uint32_t b) { return 128u * b + 64u; }
+
+// Units for 64-row steps: m_lo counts steps.
+__device__ __forceinline__ BUnit decode_bwd2_unit(const BwdParams& p, int u) {
+    BUnit U;
+    if (p.causal) {
+        U.n = u / p.BH;
+        U.bh = u - U.n * p.BH;
+        const int q_first = U.n * TILE - p.causal_off;
+        U.m_lo = q_first > 0 ? q_first / QM : 0;
+    } else {
+        U.bh = u / p.n_ktiles;
+        U.n = u - U.bh * p.n_ktiles;
+        U.m_lo = 0;
+    }
+    U.T = p.n_mtiles - U.m_lo;  // n_mtiles counts 64-row steps here
+    return U;
+}
+
+struct Bwd2UnitReader {
+    int slot = 0;
+    uint32_t phase = 0;
+    __device__ __forceinline__ int next(uint8_t* smem, volatile uint32_t* abort_flag, int site) {
+        using L = Bwd2Smem;
+        const uint32_t bar0 = smem_u32(smem) + L::BAR_OFF;
+        if (!mbar_wait(bar0 + 8u * (uint32_t)(L::B_UFULL + slot), phase, abort_flag, site)) return -2;
+        const int u = reinterpret_cast<volatile int*>(smem + L::UNIT_OFF)[slot];
+        mbar_arrive(bar0 + 8u * (uint32_t)(L::B_UEMPTY + slot));
+        if (++slot == 2) { slot = 0; phase ^= 1u; }
+        return u;
+    }
+};
+
+__device__ void bwd2_producer(const BwdParams& p, uint8_t* smem, volatile uint32_t* abort_flag) {
+    using L = Bwd2Smem;
+    const uint32_t base = smem_u32(smem);
+    const uint32_t bar0 = base + L::BAR_OFF;
+    auto bar = [&](int i) { return bar0 + 8u * (uint32_t)i; };
+    volatile int* ring = reinterpret_cast<volatile int*>(smem + L::UNIT_OFF);
+    int uslot = 0;
+    uint32_t uphase = 0;
+    bool ok = true;
+    int kv_fill = -1;
+    uint32_t fill_mask = 0, fill_parity = 0;
+    uint32_t g = 0;  // global step count
+    int nunit = 0;
+    for (int k = 0;; ++k) {
+        int u = p.sched ? (int)atomicAdd(p.sched, 1u) : (int)blockIdx.x + k * (int)gridDim.x;
+        if (u >= p.n_units) u = -1;
+        if (!mbar_wait(bar(L::B_UEMPTY + uslot), uphase ^ 1u, abort_flag, 60)) { ok = false; break; }
+        ring[uslot] = u;
+        mbar_arrive(bar(L::B_UFULL + uslot));
+        if (++uslot == 2) { uslot = 0; uphase ^= 1u; }
+        if (u < 0) break;
+        const BUnit U = decode_bwd2_unit(p, u);
+        const int b = U.bh / p.H, h = U.bh - b * p.H;
+        const uint32_t kvp = (uint32_t)nunit & 1u;
+        if (!mbar_wait(bar(L::B_KVEMPTY), kvp ^ 1u, abort_flag, 61)) { ok = false; break; }
+        mbar_expect_tx(bar(L::B_KVFULL), 2 * L::KV_TILE);
+        kv_fill = (int)kvp;
+        ++nunit;
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+            tma_load_4d(base + L::K_OFF + c * L::KCHUNK, &p.tmap_k, bar(L::B_KVFULL), c * 64, U.n * TILE, h, b);
+            tma_load_4d(base + L::V_OFF + c * L::KCHUNK, &p.tmap_v, bar(L::B_KVFULL), c * 64, U.n * TILE, h, b);
+        }
+        for (int t = 0; t < U.T; ++t, ++g) {
+            const int m = U.m_lo + t;
+            const int st = (int)(g % L::NSTAGE);
+            const uint32_t sp = (g / L::NSTAGE) & 1u;
+            if (!mbar_wait(bar(L::B_QEMPTY + st), sp ^ 1u, abort_flag, 62)) { ok = false; break; }
+            mbar_expect_tx(bar(L::B_QFULL + st), 2 * L::Q_TILE + L::STATS_BYTES);
+            fill_mask |= 1u << st;
+            fill_parity = (fill_parity & ~(1u << st)) | (sp << st);
+            const uint32_t dst = base + L::STAGE_OFF + st * L::STAGE_BYTES;
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+                tma_load_4d(dst + c * L::QCHUNK, &p.tmap_q, bar(L::B_QFULL + st), c * 64, m * QM, h, b);
+                tma_load_4d(dst + L::Q_TILE + c * L::QCHUNK, &p.tmap_do, bar(L::B_QFULL + st), c * 64, m * QM, h, b);
+            }
+            const size_t srow = (size_t)U.bh * (size_t)p.Sq_pad + (size_t)m * QM;
+            const uint32_t sdst = base + L::STATS_OFF + st * L::STATS_BYTES;
+            bulk_load(sdst, p.lse2 + srow, QM * 4, bar(L::B_QFULL + st));
+            bulk_load(sdst + QM * 4, p.delta + srow, QM * 4, bar(L::B_QFULL + st));
+        }
+        if (!ok) break;
+    }
+    if (!ok) {
+        for (int i = 0; i < L::NSTAGE; ++i)
+            if (fill_mask & (1u << i)) mbar_drain(bar(L::B_QFULL + i), (fill_parity >> i) & 1u);
+        if (kv_fill >= 0) mbar_drain(bar(L::B_KVFULL), (uint32_t)kv_fill);
+    }
+}
+
+template <bool BF16>
+__device__ void bwd2_mma(const BwdParams& p, uint8_t* smem, uint32_t tmem, volatile uint32_t* abort_flag) {
+    using L = Bwd2Smem;
+    const uint32_t base = smem_u32(smem);
+    const uint32_t bar0 = base + L::BAR_OFF;
+    auto bar = [&](int i) { return bar0 + 8u * (uint32_t)i; };
+    constexpr uint32_t IDESC_S = make_idesc_bwd(BF16, QM, false, false);   // S^T, dP^T: N = 64 queries
+    constexpr uint32_t IDESC_KV = make_idesc_bwd(BF16, 128, false, true);  // dV, dK: A in TMEM, B MN-major
+    constexpr uint32_t IDESC_DQ = make_idesc_bwd(BF16, QM, true, true);    // dQ^T: A = K^T, B = dS^T
+    // K-major: K, V ([128 rows][128], chunks 16 KiB apart), Q, dO ([64 rows][128],
+    // chunks 8 KiB apart); a K step of 16 elements is +32 bytes in a chunk.
+    // MN-major: Q, dO along D (2 chunks 8 KiB apart), K along D (2 chunks 16 KiB
+    // apart), dS^T along the queries (one 64-wide chunk); 8-row groups 1 KiB
+    // apart and a K step of 16 rows +2 KiB throughout.
+    const uint64_t a_k = sw128_desc(base + L::K_OFF, 16, 1024);
+    const uint64_t a_v = sw128_desc(base + L::V_OFF, 16, 1024);
+    const uint64_t b_stage_k = sw128_desc(base + L::STAGE_OFF, 16, 1024);
+    const uint64_t b_stage_mn = sw128_desc(base + L::STAGE_OFF, (uint32_t)L::QCHUNK, 1024);
+    const uint64_t a_kt = sw128_desc(base + L::K_OFF, (uint32_t)L::KCHUNK, 1024);
+    const uint64_t b_ds = sw128_desc(base + L::DS_OFF, 1024, 1024);
+    constexpr uint32_t STAGE16 = (uint32_t)L::STAGE_BYTES >> 4;
+    constexpr uint32_t QTILE16 = (uint32_t)L::Q_TILE >> 4;
+    constexpr uint32_t DS16 = (uint32_t)L::DS_BYTES >> 4;
+    auto lo = [](uint64_t d) { return (uint32_t)d; };
+    auto hi = [](uint64_t d) { return (uint32_t)(d >> 32); };
+
+    // S^T or dP^T of one step: A = K or V (128 keys), B = Q or dO (64 queries), K = D
+    auto issue_sp = [&](uint32_t d_tmem, uint64_t a, uint32_t b_off16) {
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+            const uint32_t in_chunk = (uint32_t)((ks & 3) * 32) >> 4;
+            const uint32_t a_off = in_chunk + (uint32_t)(((ks >> 2) * L::KCHUNK) >> 4);
+            const uint32_t b_off = in_chunk + (uint32_t)(((ks >> 2) * L::QCHUNK) >> 4);
+            tc_mma_ss2(d_tmem, lo(a) + a_off, hi(a), lo(b_stage_k) + b_off16 + b_off, hi(b_stage_k), IDESC_S,
+                       ks > 0 ? 1u : 0u);
+        }
+    };
+    // dV or dK += A(tmem, 64 queries packed) B(smem MN-major, 64 rows x 128)
+    auto issue_kv = [&](uint32_t d_tmem, uint32_t a_tmem, uint32_t b_off16, bool accumulate) {
+#pragma unroll
+        for (int ks = 0; ks < QM / 16; ++ks)
+            tc_mma_ts2(d_tmem, a_tmem + (uint32_t)(ks * 8), lo(b_stage_mn) + b_off16 + (uint32_t)(ks * (2048 >> 4)),
+                       hi(b_stage_mn), IDESC_KV, (accumulate || ks > 0) ? 1u : 0u);
+    };
+    auto wait_p = [&](uint32_t bar_idx, uint32_t parity, int site) -> bool {
+        return mbar_wait(bar(bar_idx), parity, abort_flag, site);
+    };
+
+    uint32_t g = 0;
+    int nunit = 0;
+    bool ok = true;
+    Bwd2UnitReader units;
+    for (;;) {
+        const int u = units.next(smem, abort_flag, 63);
+        if (u < 0) break;
+        const BUnit U = decode_bwd2_unit(p, u);
+        const uint32_t kvp = (uint32_t)nunit & 1u;
+        ++nunit;
+        if (!wait_p(L::B_KVFULL, kvp, 64)) { ok = false; break; }
+        // step g's S^T and dP^T into buffer g & 1
+        auto issue_step = [&](uint32_t gs) -> bool {
+            const uint32_t b = gs & 1u;
+            const int st = (int)(gs % L::NSTAGE);
+            if (!wait_p(L::B_QFULL + st, (gs / L::NSTAGE) & 1u, 65)) return false;
+            // the buffer's previous dQ^T (step gs - 2) has been read out
+            if (!wait_p(L::B_DQEMPTY + b, ((gs >> 1) & 1u) ^ 1u, 66)) return false;
+            tc_fence_after();
+            const uint32_t q16 = (uint32_t)st * STAGE16;
+            issue_sp(tmem + col2_s(b), a_k, q16);
+            issue_sp(tmem + col2_dp(b), a_v, q16 + QTILE16);
+            tc_commit(bar(L::B_SFULL + b));
+            return true;
+        };
+        if (!issue_step(g)) { ok = false; break; }
+        for (int t = 0; t < U.T; ++t, ++g) {
+            const uint32_t b = g & 1u;
+            const int st = (int)(g % L::NSTAGE);
+            if (t + 1 < U.T && !issue_step(g + 1)) { ok = false; break; }
+            if (!wait_p(L::B_PFULL + b, (g >> 1) & 1u, 67)) { ok = false; break; }
+            tc_fence_after();
+            if (t == 0) {
+                if (!wait_p(L::B_DKVEMPTY, kvp ^ 1u, 68)) { ok = false; break; }
+                tc_fence_after();
+            }
+            const uint32_t q16 = (uint32_t)st * STAGE16;
+            issue_kv(tmem + COL2_DV, tmem + col2_s(b), q16 + QTILE16, t > 0);  // dV += P^T dO_m
+            issue_kv(tmem + COL2_DK, tmem + col2_dp(b), q16, t > 0);          // dK += dS^T Q_m
+            tc_commit(bar(L::B_QEMPTY + st));
+            // dQ^T = K^T dS^T into this step's S columns
+#pragma unroll
+            for (int ks = 0; ks < TILE / 16; ++ks) {
+                const uint32_t off = (uint32_t)(ks * (2048 >> 4));
+                tc_mma_ss2(tmem + col2_s(b), lo(a_kt) + off, hi(a_kt), lo(b_ds) + b * DS16 + off, hi(b_ds), IDESC_DQ,
+                           ks > 0 ? 1u : 0u);
+            }
+            tc_commit(bar(L::B_DQFULL + b));
+            tc_commit(bar(L::B_DSEMPTY + b));
+        }
+        if (!ok) break;
+        tc_commit(bar(L::B_DKVFULL));
+        tc_commit(bar(L::B_KVEMPTY));
+    }
+    (void)ok;
+    tc_commit(bar(L::B_FIN));
+    mbar_drain(bar(L::B_FIN), 0u);
+}
+
+template <bool BF16>
+__device__ void bwd2_ds_role(const BwdParams& p, uint8_t* smem, uint32_t tmem, int warp_in_group,
+                             volatile uint32_t* abort_flag) {
+    using L = Bwd2Smem;
+    const uint32_t base = smem_u32(smem);
+    const uint32_t bar0 = base + L::BAR_OFF;
+    auto bar = [&](int i) { return bar0 + 8u * (uint32_t)i; };
+    const int lane = threadIdx.x & 31;
+    const int row = warp_in_group * 32 + lane;  // key row
+    const uint32_t lane_sel = (uint32_t)(warp_in_group * 32) << 16;
+    const float sl2 = p.scale_log2;
+    const int sw = row & 7;
+    uint32_t g = 0;
+    Bwd2UnitReader units;
+    for (;;) {
+        const int u = units.next(smem, abort_flag, 69);
+        if (!__all_sync(0xffffffffu, u != -2)) return;
+        if (u < 0) break;
+        const BUnit U = decode_bwd2_unit(p, u);
+        const int key = U.n * TILE + row;
+        const bool key_ok = key < p.Sk;
+        const int q_min = p.causal ? key - p.causal_off : 0;
+        for (int t = 0; t < U.T; ++t, ++g) {
+            const int m = U.m_lo + t;
+            const uint32_t b = g & 1u;
+            const int st = (int)(g % L::NSTAGE);
+            if (!__all_sync(0xffffffffu, mbar_wait(bar(L::B_SFULL + b), (g >> 1) & 1u, abort_flag, 70))) return;
+            if (!__all_sync(0xffffffffu, mbar_wait(bar(L::B_QFULL + st), (g / L::NSTAGE) & 1u, abort_flag, 71)))
+                return;
+            if (!__all_sync(0xffffffffu, mbar_wait(bar(L::B_DSEMPTY + b), ((g >> 1) & 1u) ^ 1u, abort_flag, 72)))
+                return;
+            tc_fence_after();
+            const float* lse2s = reinterpret_cast<const float*>(smem + L::STATS_OFF + st * L::STATS_BYTES);
+            const float* dls = lse2s + QM;
+            const bool need_mask = !key_ok || (m * QM < q_min);
+            uint8_t* ds_row = smem + L::DS_OFF + b * L::DS_BYTES + (row >> 3) * 1024 + (row & 7) * 128;
+#pragma unroll 1
+            for (int c = 0; c < QM / 32; ++c) {
+                uint32_t sr[32], dr[32];
+                tmem_ld32u(tmem + lane_sel + col2_s(b) + 32 * c, sr);
+                tmem_ld32u(tmem + lane_sel + col2_dp(b) + 32 * c, dr);
+                uint32_t pk[16], dk[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const int j = 32 * c + 2 * i;
+                    const float2 l2 = *reinterpret_cast<const float2*>(lse2s + j);
+                    const float2 dl = *reinterpret_cast<const float2*>(dls + j);
+                    float p0 = ex2(fmaf(__uint_as_float(sr[2 * i]), sl2, -l2.x));
+                    float p1 = ex2(fmaf(__uint_as_float(sr[2 * i + 1]), sl2, -l2.y));
+                    if (need_mask) {
+                        const int q = m * QM + j;
+                        if (!key_ok || q < q_min) p0 = 0.f;
+                        if (!key_ok || q + 1 < q_min) p1 = 0.f;
+                    }
+                    pk[i] = pack2<BF16>(p0, p1);
+                    dk[i] = pack2<BF16>(p0 * (__uint_as_float(dr[2 * i]) - dl.x),
+                                        p1 * (__uint_as_float(dr[2 * i + 1]) - dl.y));
+                }
+                tmem_st16(tmem + lane_sel + col2_s(b) + 16 * c, pk);
+                tmem_st16(tmem + lane_sel + col2_dp(b) + 16 * c, dk);
+#pragma unroll
+                for (int gi = 0; gi < 4; ++gi) {
+                    const int gr = (c * 4 + gi) ^ sw;
+                    *reinterpret_cast<uint4*>(ds_row + gr * 16) =
+                        make_uint4(dk[4 * gi], dk[4 * gi + 1], dk[4 * gi + 2], dk[4 * gi + 3]);
+                }
+            }
+            tmem_wait_st();
+            fence_async_smem();
+            tc_fence_before();
+            mbar_arrive(bar(L::B_PFULL + b));
+        }
+    }
+}
+
+template <bool BF16>
+__device__ void bwd2_out_role(const BwdParams& p, uint8_t* smem, uint32_t tmem, int warp_in_group,
+                              volatile uint32_t* abort_flag) {
+    using L = Bwd2Smem;
+    const uint32_t base = smem_u32(smem);
+    const uint32_t bar0 = base + L::BAR_OFF;
+    auto bar = [&](int i) { return bar0 + 8u * (uint32_t)i; };
+    const int lane = threadIdx.x & 31;
+    const int row = warp_in_group * 32 + lane;  // head-dimension index for dQ^T, key row for dK/dV
+    const uint32_t lane_sel = (uint32_t)(warp_in_group * 32) << 16;
+    uint32_t g = 0;
+    int nunit = 0;
+    Bwd2UnitReader units;
+    for (;;) {
+        const int u = units.next(smem, abort_flag, 73);
+        if (!__all_sync(0xffffffffu, u != -2)) return;
+        if (u < 0) break;
+        const BUnit U = decode_bwd2_unit(p, u);
+        const uint32_t kvp = (uint32_t)nunit & 1u;
+        ++nunit;
+        for (int t = 0; t < U.T; ++t, ++g) {
+            const int m = U.m_lo + t;
+            const uint32_t b = g & 1u;
+            if (!__all_sync(0xffffffffu, mbar_wait(bar(L::B_DQFULL + b), (g >> 1) & 1u, abort_flag, 74))) return;
+            tc_fence_after();
+            uint32_t r0[32], r1[32];
+            tmem_ld32u(tmem + lane_sel + col2_s(b), r0);
+            tmem_ld32u(tmem + lane_sel + col2_s(b) + 32, r1);
+            tc_fence_before();
+            mbar_arrive(bar(L::B_DQEMPTY + b));
+            // dQ[q][d] += dQ^T[d][q]: consecutive threads take consecutive d (coalesced)
+            float* dst = p.dq_acc + ((size_t)U.bh * (size_t)p.Sq + (size_t)m * QM) * 128 + row;
+            const int nq = min(QM, p.Sq - m * QM);
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+                if (j < nq) atomicAdd(dst + (size_t)j * 128, __uint_as_float(r0[j]));
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+                if (32 + j < nq) atomicAdd(dst + (size_t)(32 + j) * 128, __uint_as_float(r1[j]));
+        }
+        if (!__all_sync(0xffffffffu, mbar_wait(bar(L::B_DKVFULL), kvp, abort_flag, 75))) return;
+        tc_fence_after();
+        const int key = U.n * TILE + row;
+        const bool valid = key < p.Sk;
+        const size_t off = ((size_t)U.bh * (size_t)p.Sk + (size_t)(valid ? key : 0)) * 256;
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+            uint32_t r[32];
+            uint32_t w[16];
+            tmem_ld32u(tmem + lane_sel + COL2_DV + 32 * c, r);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) w[i] = pack2<BF16>(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
+            if (valid) {
+                uint4* d = reinterpret_cast<uint4*>(p.dv + off + c * 64);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) d[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+            }
+            tmem_ld32u(tmem + lane_sel + COL2_DK + 32 * c, r);
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+                w[i] = pack2<BF16>(__uint_as_float(r[2 * i]) * p.scale, __uint_as_float(r[2 * i + 1]) * p.scale);
+            if (valid) {
+                uint4* d = reinterpret_cast<uint4*>(p.dk + off + c * 64);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) d[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+            }
+        }
+        tc_fence_before();
+        mbar_arrive(bar(L::B_DKVEMPTY));
+    }
+}
+
+template <bool BF16>
+__global__ void __launch_bounds__(BWD_THREADS, 1) fa_bwd_kernel_d128(const __grid_constant__ BwdParams p) {
+    using L = Bwd2Smem;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t base = smem_u32(smem);
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int wg = warp >> 2;
+    uint32_t* misc = reinterpret_cast<uint32_t*>(smem + L::MISC_OFF);
+    volatile uint32_t* abort_flag = misc + 1;
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < L::NBAR; ++i) {
+            uint32_t count = 1;
+            if ((i >= L::B_PFULL && i < L::B_PFULL + 2) || (i >= L::B_DQEMPTY && i < L::B_DQEMPTY + 2) ||
+                i == L::B_DKVEMPTY)
+                count = TILE;  // one warpgroup
+            if (i >= L::B_UEMPTY && i < L::B_UEMPTY + 2) count = UNIT_READERS_BWD;
+            mbar_init(base + L::BAR_OFF + 8 * i, count);
+        }
+        *abort_flag = 0u;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    }
+    if (warp == BW_TMA && lane == 0) {
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&p.tmap_q)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&p.tmap_k)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&p.tmap_v)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&p.tmap_do)) : "memory");
+    }
+    if (warp == BW_MMA) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(misc)),
+                     "r"(BWD_TMEM_COLS)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = misc[0];
+    if (wg == 0) {
+        if (warp == BW_TMA && lane == 0) bwd2_producer(p, smem, abort_flag);
+        if (warp == BW_MMA && lane == 0) bwd2_mma<BF16>(p, smem, tmem, abort_flag);
+    } else if (wg == 1) {
+        bwd2_ds_role<BF16>(p, smem, tmem, warp & 3, abort_flag);
+    } else {
+        bwd2_out_role<BF16>(p, smem, tmem, warp & 3, abort_flag);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == BW_MMA) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(BWD_TMEM_COLS)
+                     : "memory");
+    }
+}
+
 template <bool BF16>
 __device__ __forceinline__ float load16(const uint16_t* p) {
     const uint16_t x = *p;
@@ -638,8 +1100,8 @@ __global__ void __launch_bounds__(256) bwd_post_kernel(const float4* __restrict_
 
 template <int D, bool BF16>
 cudaError_t launch_bwd_impl(const BwdLaunchArgs& a, cudaStream_t stream) {
-    using L = BwdSmem<D>;
-    static_assert(L::ALLOC <= 232448, "shared memory budget exceeded");
+    static_assert(BwdSmem<64>::ALLOC <= 232448, "shared memory budget exceeded");
+    static_assert(Bwd2Smem::ALLOC <= 232448, "shared memory budget exceeded");
     const int BH = a.B * a.H;
     const int n_mtiles = (a.Sq + TILE - 1) / TILE;
     const int Sq_pad = n_mtiles * TILE;
@@ -652,8 +1114,12 @@ cudaError_t launch_bwd_impl(const BwdLaunchArgs& a, cudaStream_t stream) {
         if (e != cudaSuccess) return e;
     }
     {
-        auto kern = fa_bwd_kernel<D, BF16>;
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC);
+        // D = 128 runs the 64-row-step kernel (its Q/dO maps have 64-row boxes)
+        void (*kern)(const BwdParams);
+        if constexpr (D == 128) kern = fa_bwd_kernel_d128<BF16>;
+        else kern = fa_bwd_kernel<D, BF16>;
+        const int alloc = (D == 128) ? Bwd2Smem::ALLOC : BwdSmem<64>::ALLOC;
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, alloc);
         if (e != cudaSuccess) return e;
         BwdParams p;
         p.tmap_q = a.tmap_q;
@@ -670,7 +1136,7 @@ cudaError_t launch_bwd_impl(const BwdLaunchArgs& a, cudaStream_t stream) {
         p.Sq = a.Sq;
         p.Sk = a.Sk;
         p.Sq_pad = Sq_pad;
-        p.n_mtiles = n_mtiles;
+        p.n_mtiles = (D == 128) ? (a.Sq + QM - 1) / QM : n_mtiles;
         p.n_ktiles = (a.Sk + TILE - 1) / TILE;
         p.n_units = BH * p.n_ktiles;
         p.causal = a.causal;
@@ -681,7 +1147,7 @@ cudaError_t launch_bwd_impl(const BwdLaunchArgs& a, cudaStream_t stream) {
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3((unsigned)a.grid, 1, 1);
         cfg.blockDim = dim3(BWD_THREADS, 1, 1);
-        cfg.dynamicSmemBytes = L::ALLOC;
+        cfg.dynamicSmemBytes = alloc;
         cfg.stream = stream;
         e = cudaLaunchKernelEx(&cfg, kern, p);
         if (e != cudaSuccess) return e;
