@@ -84,9 +84,13 @@ def peak_tflops():
 
 
 def kernel_source_hash() -> str:
+    """Hash of the forward kernel's sources (its file and the shared device helpers)."""
     import hashlib
-    with open(KERNEL_SRC, "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+    h = hashlib.sha256()
+    for path in (KERNEL_SRC, os.path.join(os.path.dirname(KERNEL_SRC), "sm100_helpers.cuh")):
+        with open(path, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
 
 
 def traffic_per_launch(workload: str):

@@ -122,6 +122,7 @@ struct BwdParams {
     uint8_t* dk;          // [BH][Sk][D] 16-bit
     uint8_t* dv;
     int BH, H, Sq, Sk, Sq_pad, n_mtiles, n_ktiles, n_units, causal, causal_off;
+    int head_group;       // causal claim order: heads per group (their Q, dO, dQ fit in L2)
     float scale_log2;     // scale * log2(e)
     float scale;
     unsigned int* sched;  // zeroed unit counter (causal), or null
@@ -136,13 +137,22 @@ struct BUnit {
 
 // Units: with the causal mask the number of query tiles falls with the key
 // tile index, so units are claimed in key-tile order (longest first), heads
-// innermost; without it, heads outermost (CTAs running together share one
-// head's Q and dO in L2).
+// innermost, within groups of head_group heads whose Q, dO and dQ accumulator
+// stay in L2 together; without the mask, heads outermost (CTAs running
+// together share one head's Q, dO and dQ in L2).
+__device__ __forceinline__ void causal_unit_order(const BwdParams& p, int u, int* bh, int* n) {
+    const int per_group = p.head_group * p.n_ktiles;
+    const int g = u / per_group;
+    const int within = u - g * per_group;
+    const int gh = min(p.head_group, p.BH - g * p.head_group);  // heads in this group
+    *n = within / gh;
+    *bh = g * p.head_group + (within - *n * gh);
+}
+
 __device__ __forceinline__ BUnit decode_bwd_unit(const BwdParams& p, int u) {
     BUnit U;
     if (p.causal) {
-        U.n = u / p.BH;
-        U.bh = u - U.n * p.BH;
+        causal_unit_order(p, u, &U.bh, &U.n);
         // query q sees key j iff j <= q + causal_off: the first query that sees
         // key n*128 is n*128 - causal_off
         const int q_first = U.n * TILE - p.causal_off;
@@ -592,11 +602,25 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) fa_bwd_kernel(const __grid_con
 // [256,384), dK [384,512).  While the dS warpgroup turns step g's S^T, dP^T
 // (buffer g&1) into P^T, dS^T, the MMA lane already computes step g+1's into
 // the other buffer; then dV += P^T dO, dK += dS^T Q and dQ^T = K^T dS^T (M = D
-// = 128 lanes, N = 64 queries) into step g's S columns, which the output
-// warpgroup reads out (one head-dimension lane per thread) into the fp32 dQ
-// accumulator.  Q and dO stream through three 32 KiB stages.  Every role
+// = 128 lanes, N = 64 queries) into step g's dP columns (after dK has read
+// dS^T there), which the output warpgroup reads out (one head-dimension lane
+// per thread) into the fp32 dQ accumulator.  The next S^T into a buffer needs
+// no wait; only its dP^T waits for that buffer's dQ^T read-out, and the S^T
+// MMAs issued before it cover that latency.  Q and dO stream through three 32 KiB stages.  Every role
 // derives buffer, stage and barrier parities from the global step count g.
 constexpr int QM = 64;  // query rows per step
+// 16 warps: warpgroup 0 = TMA lane (warp 0) and MMA lane (warp 1); warpgroups 1
+// and 3 = the dS work of query columns [0, 32) and [32, 64) of each step (two
+// warps per SM sub-partition hide each other's latencies); warpgroup 2 = dQ^T
+// read-out and the dK/dV epilogue.
+constexpr int BWD2_THREADS = 512;
+constexpr uint32_t UNIT_READERS_BWD2 = 1 + 3 * TILE;
+// Register split (launch: 128 per thread): control 64, dS 176 each, output 96;
+// per SM sub-partition one warp of each warpgroup: 64 + 176 + 96 + 176 = 512.
+constexpr int REG2_CTRL = 64;
+constexpr int REG2_DS = 176;
+constexpr int REG2_OUT = 96;
+static_assert(REG2_CTRL + 2 * REG2_DS + REG2_OUT <= 4 * 128, "register split exceeds the launch budget");
 
 struct Bwd2Smem {
     static constexpr int D = 128;
@@ -646,8 +670,7 @@ __device__ __forceinline__ uint32_t col2_dp(uint32_t b) { return 128u * b + 64u;
 __device__ __forceinline__ BUnit decode_bwd2_unit(const BwdParams& p, int u) {
     BUnit U;
     if (p.causal) {
-        U.n = u / p.BH;
-        U.bh = u - U.n * p.BH;
+        causal_unit_order(p, u, &U.bh, &U.n);
         const int q_first = U.n * TILE - p.causal_off;
         U.m_lo = q_first > 0 ? q_first / QM : 0;
     } else {
@@ -771,12 +794,16 @@ __device__ void bwd2_mma(const BwdParams& p, uint8_t* smem, uint32_t tmem, volat
                        ks > 0 ? 1u : 0u);
         }
     };
-    // dV or dK += A(tmem, 64 queries packed) B(smem MN-major, 64 rows x 128)
+    // dV or dK += A(tmem, 64 queries packed) B(smem MN-major, 64 rows x 128).  The
+    // packed pairs of queries [32c, 32c + 32) sit in columns 32c .. 32c + 15 of
+    // the buffer (each dS warpgroup packs into its own columns), so the K step
+    // of queries 16 ks .. 16 ks + 15 reads columns 32 (ks / 2) + 8 (ks % 2).
     auto issue_kv = [&](uint32_t d_tmem, uint32_t a_tmem, uint32_t b_off16, bool accumulate) {
 #pragma unroll
         for (int ks = 0; ks < QM / 16; ++ks)
-            tc_mma_ts2(d_tmem, a_tmem + (uint32_t)(ks * 8), lo(b_stage_mn) + b_off16 + (uint32_t)(ks * (2048 >> 4)),
-                       hi(b_stage_mn), IDESC_KV, (accumulate || ks > 0) ? 1u : 0u);
+            tc_mma_ts2(d_tmem, a_tmem + (uint32_t)((ks >> 1) * 32 + (ks & 1) * 8),
+                       lo(b_stage_mn) + b_off16 + (uint32_t)(ks * (2048 >> 4)), hi(b_stage_mn), IDESC_KV,
+                       (accumulate || ks > 0) ? 1u : 0u);
     };
     auto wait_p = [&](uint32_t bar_idx, uint32_t parity, int site) -> bool {
         return mbar_wait(bar(bar_idx), parity, abort_flag, site);
@@ -798,11 +825,11 @@ __device__ void bwd2_mma(const BwdParams& p, uint8_t* smem, uint32_t tmem, volat
             const uint32_t b = gs & 1u;
             const int st = (int)(gs % L::NSTAGE);
             if (!wait_p(L::B_QFULL + st, (gs / L::NSTAGE) & 1u, 65)) return false;
-            // the buffer's previous dQ^T (step gs - 2) has been read out
-            if (!wait_p(L::B_DQEMPTY + b, ((gs >> 1) & 1u) ^ 1u, 66)) return false;
-            tc_fence_after();
             const uint32_t q16 = (uint32_t)st * STAGE16;
             issue_sp(tmem + col2_s(b), a_k, q16);
+            // the buffer's previous dQ^T (step gs - 2, in its dP columns) has been read out
+            if (!wait_p(L::B_DQEMPTY + b, ((gs >> 1) & 1u) ^ 1u, 66)) return false;
+            tc_fence_after();
             issue_sp(tmem + col2_dp(b), a_v, q16 + QTILE16);
             tc_commit(bar(L::B_SFULL + b));
             return true;
@@ -822,11 +849,11 @@ __device__ void bwd2_mma(const BwdParams& p, uint8_t* smem, uint32_t tmem, volat
             issue_kv(tmem + COL2_DV, tmem + col2_s(b), q16 + QTILE16, t > 0);  // dV += P^T dO_m
             issue_kv(tmem + COL2_DK, tmem + col2_dp(b), q16, t > 0);          // dK += dS^T Q_m
             tc_commit(bar(L::B_QEMPTY + st));
-            // dQ^T = K^T dS^T into this step's S columns
+            // dQ^T = K^T dS^T into this step's dP columns
 #pragma unroll
             for (int ks = 0; ks < TILE / 16; ++ks) {
                 const uint32_t off = (uint32_t)(ks * (2048 >> 4));
-                tc_mma_ss2(tmem + col2_s(b), lo(a_kt) + off, hi(a_kt), lo(b_ds) + b * DS16 + off, hi(b_ds), IDESC_DQ,
+                tc_mma_ss2(tmem + col2_dp(b), lo(a_kt) + off, hi(a_kt), lo(b_ds) + b * DS16 + off, hi(b_ds), IDESC_DQ,
                            ks > 0 ? 1u : 0u);
             }
             tc_commit(bar(L::B_DQFULL + b));
@@ -842,7 +869,7 @@ __device__ void bwd2_mma(const BwdParams& p, uint8_t* smem, uint32_t tmem, volat
 }
 
 template <bool BF16>
-__device__ void bwd2_ds_role(const BwdParams& p, uint8_t* smem, uint32_t tmem, int warp_in_group,
+__device__ void bwd2_ds_role(const BwdParams& p, uint8_t* smem, uint32_t tmem, int warp_in_group, int c,
                              volatile uint32_t* abort_flag) {
     using L = Bwd2Smem;
     const uint32_t base = smem_u32(smem);
@@ -867,18 +894,19 @@ __device__ void bwd2_ds_role(const BwdParams& p, uint8_t* smem, uint32_t tmem, i
             const int m = U.m_lo + t;
             const uint32_t b = g & 1u;
             const int st = (int)(g % L::NSTAGE);
-            if (!__all_sync(0xffffffffu, mbar_wait(bar(L::B_SFULL + b), (g >> 1) & 1u, abort_flag, 70))) return;
+            // the stage's statistics and the free dS^T buffer are normally ready long
+            // before the scores: take those waits first
             if (!__all_sync(0xffffffffu, mbar_wait(bar(L::B_QFULL + st), (g / L::NSTAGE) & 1u, abort_flag, 71)))
                 return;
             if (!__all_sync(0xffffffffu, mbar_wait(bar(L::B_DSEMPTY + b), ((g >> 1) & 1u) ^ 1u, abort_flag, 72)))
                 return;
+            if (!__all_sync(0xffffffffu, mbar_wait(bar(L::B_SFULL + b), (g >> 1) & 1u, abort_flag, 70))) return;
             tc_fence_after();
             const float* lse2s = reinterpret_cast<const float*>(smem + L::STATS_OFF + st * L::STATS_BYTES);
             const float* dls = lse2s + QM;
-            const bool need_mask = !key_ok || (m * QM < q_min);
+            const bool need_mask = !key_ok || (m * QM + 32 * c < q_min);
             uint8_t* ds_row = smem + L::DS_OFF + b * L::DS_BYTES + (row >> 3) * 1024 + (row & 7) * 128;
-#pragma unroll 1
-            for (int c = 0; c < QM / 32; ++c) {
+            {
                 uint32_t sr[32], dr[32];
                 tmem_ld32u(tmem + lane_sel + col2_s(b) + 32 * c, sr);
                 tmem_ld32u(tmem + lane_sel + col2_dp(b) + 32 * c, dr);
@@ -899,8 +927,10 @@ __device__ void bwd2_ds_role(const BwdParams& p, uint8_t* smem, uint32_t tmem, i
                     dk[i] = pack2<BF16>(p0 * (__uint_as_float(dr[2 * i]) - dl.x),
                                         p1 * (__uint_as_float(dr[2 * i + 1]) - dl.y));
                 }
-                tmem_st16(tmem + lane_sel + col2_s(b) + 16 * c, pk);
-                tmem_st16(tmem + lane_sel + col2_dp(b) + 16 * c, dk);
+                // packed into the first 16 of this warpgroup's own 32 columns: the other
+                // dS warpgroup may still be reading its raw scores from the rest
+                tmem_st16(tmem + lane_sel + col2_s(b) + 32 * c, pk);
+                tmem_st16(tmem + lane_sel + col2_dp(b) + 32 * c, dk);
 #pragma unroll
                 for (int gi = 0; gi < 4; ++gi) {
                     const int gr = (c * 4 + gi) ^ sw;
@@ -942,8 +972,8 @@ __device__ void bwd2_out_role(const BwdParams& p, uint8_t* smem, uint32_t tmem, 
             if (!__all_sync(0xffffffffu, mbar_wait(bar(L::B_DQFULL + b), (g >> 1) & 1u, abort_flag, 74))) return;
             tc_fence_after();
             uint32_t r0[32], r1[32];
-            tmem_ld32u(tmem + lane_sel + col2_s(b), r0);
-            tmem_ld32u(tmem + lane_sel + col2_s(b) + 32, r1);
+            tmem_ld32u(tmem + lane_sel + col2_dp(b), r0);
+            tmem_ld32u(tmem + lane_sel + col2_dp(b) + 32, r1);
             tc_fence_before();
             mbar_arrive(bar(L::B_DQEMPTY + b));
             // dQ[q][d] += dQ^T[d][q]: consecutive threads take consecutive d (coalesced)
@@ -989,7 +1019,7 @@ __device__ void bwd2_out_role(const BwdParams& p, uint8_t* smem, uint32_t tmem, 
 }
 
 template <bool BF16>
-__global__ void __launch_bounds__(BWD_THREADS, 1) fa_bwd_kernel_d128(const __grid_constant__ BwdParams p) {
+__global__ void __launch_bounds__(BWD2_THREADS, 1) fa_bwd_kernel_d128(const __grid_constant__ BwdParams p) {
     using L = Bwd2Smem;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -1002,10 +1032,9 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) fa_bwd_kernel_d128(const __gri
     if (threadIdx.x == 0) {
         for (int i = 0; i < L::NBAR; ++i) {
             uint32_t count = 1;
-            if ((i >= L::B_PFULL && i < L::B_PFULL + 2) || (i >= L::B_DQEMPTY && i < L::B_DQEMPTY + 2) ||
-                i == L::B_DKVEMPTY)
-                count = TILE;  // one warpgroup
-            if (i >= L::B_UEMPTY && i < L::B_UEMPTY + 2) count = UNIT_READERS_BWD;
+            if ((i >= L::B_DQEMPTY && i < L::B_DQEMPTY + 2) || i == L::B_DKVEMPTY) count = TILE;  // one warpgroup
+            if (i >= L::B_PFULL && i < L::B_PFULL + 2) count = 2 * TILE;  // both dS warpgroups
+            if (i >= L::B_UEMPTY && i < L::B_UEMPTY + 2) count = UNIT_READERS_BWD2;
             mbar_init(base + L::BAR_OFF + 8 * i, count);
         }
         *abort_flag = 0u;
@@ -1029,11 +1058,14 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) fa_bwd_kernel_d128(const __gri
     tc_fence_after();
     const uint32_t tmem = misc[0];
     if (wg == 0) {
+        setmaxnreg_dec<REG2_CTRL>();
         if (warp == BW_TMA && lane == 0) bwd2_producer(p, smem, abort_flag);
         if (warp == BW_MMA && lane == 0) bwd2_mma<BF16>(p, smem, tmem, abort_flag);
-    } else if (wg == 1) {
-        bwd2_ds_role<BF16>(p, smem, tmem, warp & 3, abort_flag);
+    } else if (wg == 1 || wg == 3) {
+        setmaxnreg_inc<REG2_DS>();
+        bwd2_ds_role<BF16>(p, smem, tmem, warp & 3, wg == 1 ? 0 : 1, abort_flag);
     } else {
+        setmaxnreg_dec<REG2_OUT>();
         bwd2_out_role<BF16>(p, smem, tmem, warp & 3, abort_flag);
     }
     tc_fence_before();
@@ -1141,12 +1173,18 @@ cudaError_t launch_bwd_impl(const BwdLaunchArgs& a, cudaStream_t stream) {
         p.n_units = BH * p.n_ktiles;
         p.causal = a.causal;
         p.causal_off = a.Sk - a.Sq;
+        {
+            // heads whose Q, dO (16-bit) and dQ accumulator (fp32) take <= 48 MiB
+            const long long per_head = (long long)a.Sq * D * 8;
+            const long long g = (48ll << 20) / (per_head > 0 ? per_head : 1);
+            p.head_group = (int)(g < 1 ? 1 : (g > BH ? BH : g));
+        }
         p.scale_log2 = a.scale * 1.4426950408889634f;
         p.scale = a.scale;
         p.sched = a.causal ? a.sched : nullptr;
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3((unsigned)a.grid, 1, 1);
-        cfg.blockDim = dim3(BWD_THREADS, 1, 1);
+        cfg.blockDim = dim3(D == 128 ? BWD2_THREADS : BWD_THREADS, 1, 1);
         cfg.dynamicSmemBytes = alloc;
         cfg.stream = stream;
         e = cudaLaunchKernelEx(&cfg, kern, p);
