@@ -294,7 +294,7 @@ def run_bwd(args) -> int:
         st = fa.fa_bwd(b["q"].data_ptr(), b["k"].data_ptr(), b["v"].data_ptr(), b["o"].data_ptr(),
                        b["dout"].data_ptr(), b["lse"].data_ptr(), b["dq"].data_ptr(), b["dk"].data_ptr(),
                        b["dv"].data_ptr(), b["ws"].data_ptr(), b["nbytes"], w.B, w.H, w.S, w.Skv, w.D, w.scale,
-                       int(w.causal), b["dt"], sid)
+                       int(w.causal), int(args.deterministic), b["dt"], sid)
         if st != 0:
             raise fa.FaError(st, "fa_bwd")
 
@@ -380,7 +380,8 @@ def run_bwd(args) -> int:
             "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": max_ms / args.steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": w0.dtype, "data": "synthetic",
-            "config": {"workload": "backward of " + workload_label(args.workload), "B": w0.B, "H": w0.H,
+            "config": {"workload": ("deterministic " if args.deterministic else "") + "backward of "
+                       + workload_label(args.workload), "B": w0.B, "H": w0.H,
                        "S": w0.S, "D": w0.D, "runs_per_step": len(runs),
                        "l2": "inputs larger than L2 (no flush)" if sum(
                            t.numel() * t.element_size() for t in (bufs[0]["q"], bufs[0]["k"], bufs[0]["v"],
@@ -413,6 +414,8 @@ def main(argv=None) -> int:
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--pass", dest="pass_", choices=["fwd", "bwd"], default="fwd",
                     help="fwd: the forward pass (default); bwd: the backward pass fa_bwd")
+    ap.add_argument("--deterministic", action="store_true",
+                    help="with --pass bwd: the deterministic dQ mode (key tiles add in order)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -58,7 +58,7 @@ typedef enum {
     FA_ERR_LAUNCH = -7,   /* a CUDA runtime error (launch, tensor-map encoding, sync) */
     FA_ERR_TIMEOUT = -8,  /* a device-side wait exceeded its bound (reported by fa_check_status) */
     FA_ERR_SCALE = -9,    /* scale is not finite and > 0 */
-    FA_ERR_ARG = -10,     /* causal is not 0 or 1 */
+    FA_ERR_ARG = -10,     /* causal (or fa_bwd's deterministic) is not 0 or 1 */
     FA_ERR_PTR = -11,     /* a pointer is not device memory of the current device */
     FA_ERR_STRIDE = -12,  /* fa_fwd_ex: a stride is negative, zero over an extent > 1, not a
                              multiple of 8 elements (16 bytes), or not below 2^36 elements */
@@ -162,8 +162,9 @@ FA_API int fa_fwd_ex(const void* q, const void* k, const void* v, void* o, float
 /*
  * fa_bwd_workspace_size -- bytes of device workspace fa_bwd needs for B*H
  * heads of Sq query rows of dimension D: an fp32 dQ accumulator
- * [B*H][Sq][D], two fp32 row-statistic arrays [B*H][Sq rounded up to 128]
- * and a 256-byte scheduler counter, each part 256-byte aligned.  0 for an
+ * [B*H][Sq][D], two fp32 row-statistic arrays [B*H][Sq rounded up to 128],
+ * the deterministic mode's turn counters [B*H][Sq/64 rounded up][4] int and a
+ * 256-byte scheduler counter, each part 256-byte aligned.  0 for an
  * empty problem, a negative fa_status on invalid sizes.  Host only.
  */
 FA_API long long fa_bwd_workspace_size(int B, int H, int Sq, int D);
@@ -194,16 +195,24 @@ FA_API long long fa_bwd_workspace_size(int B, int H, int Sq, int D);
  *              calls that may overlap on the GPU need separate workspaces.
  * B, H, Sq, Sk, D, scale, causal, dtype: as fa_fwd_ex.  B or H 0 is an empty
  *              problem (FA_OK, nothing launched); Sq = 0 zeroes dK and dV.
+ * deterministic: 0 = dQ is accumulated in fp32 across key tiles with atomic
+ *              adds (fastest; its last bits may differ between runs); 1 = the
+ *              key tiles of a head add their dQ parts in key-tile order (the
+ *              catlass page's deterministic mode), so every output is bitwise
+ *              repeatable.  Mode 1 makes CTAs wait (bounded) for one another, so
+ *              all of the call's CTAs must be able to run at once: do not run
+ *              other kernels beside it that hold SMs it needs, or the waits may
+ *              time out (reported by fa_check_status as FA_ERR_TIMEOUT).  dK and
+ *              dV are bitwise repeatable in both modes.
  * Numerics: S, P, dP, dS, Delta and all accumulation in fp32; P and dS are
- * rounded to dtype before their products; dQ is accumulated in fp32 across
- * key tiles with atomic adds (so its last bits may differ between runs; dK and
- * dV are deterministic); the outputs are rounded to nearest even.
+ * rounded to dtype before their products; the outputs are rounded to nearest
+ * even.
  * Three kernels run on `stream` (row statistics, the fused backward, dQ
  * conversion); nothing is allocated; asynchronous.  Errors as fa_fwd.
  */
 FA_API int fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
                   void* dq, void* dk, void* dv, void* workspace, long long workspace_bytes, int B, int H, int Sq,
-                  int Sk, int D, float scale, int causal, int dtype, cudaStream_t stream);
+                  int Sk, int D, float scale, int causal, int deterministic, int dtype, cudaStream_t stream);
 
 /*
  * fa_check_status -- synchronise `stream`, then report and clear the device

@@ -140,7 +140,7 @@ def _abs_sums(q, k, dout, scale, causal):
     return sc * abs_dq, sc * abs_dk, abs_dv
 
 
-def run_fa_bwd(q, k, v, dout, scale: float, causal: bool):
+def run_fa_bwd(q, k, v, dout, scale: float, causal: bool, deterministic: bool = False):
     """Forward (fa_fwd_ex) then backward (fa_bwd) through the C ABI on CPU
     contiguous inputs; returns CPU (dQ, dK, dV, O, LSE)."""
     B, H, Sq, D = q.shape
@@ -160,7 +160,7 @@ def run_fa_bwd(q, k, v, dout, scale: float, causal: bool):
     ws = torch.full((max(ws_bytes, 1),), 0xAB, dtype=torch.uint8, device="cuda")  # garbage on entry
     rc = fa.fa_bwd(dq_.data_ptr(), dk_.data_ptr(), dv_.data_ptr(), o.data_ptr(), ddo.data_ptr(), lse.data_ptr(),
                    gq.data_ptr(), gk.data_ptr(), gv.data_ptr(), ws.data_ptr(), ws_bytes, B, H, Sq, Sk, D, scale,
-                   int(causal), dt, st)
+                   int(causal), int(deterministic), dt, st)
     assert rc == 0, f"fa_bwd returned {rc} ({fa.fa_status_string(rc)})"
     s = fa.fa_check_status(st)
     assert s == 0, f"device status {s} ({fa.fa_status_string(s)}), site {fa.fa_last_timeout_site():#x}"

@@ -149,11 +149,14 @@ def test_bwd_workspace_size(lib):
     assert fa.fa_bwd_workspace_size(0, 4, 100, 64) == 0
     assert fa.fa_bwd_workspace_size(1, 1, -1, 64) == _lib.FA_ERR_SHAPE
     assert fa.fa_bwd_workspace_size(1, 1, 10, 96) == _lib.FA_ERR_HEADDIM
-    # dQ accumulator (fp32) + two padded fp32 row arrays + 256-byte counter, 256-aligned parts
+    # dQ accumulator (fp32) + two padded fp32 row arrays + turn counters + 256-byte
+    # scheduler counter, 256-aligned parts
     B, H, S, D = 2, 3, 300, 128
-    acc = -(-(B * H * S * D * 4) // 256) * 256
-    rows = -(-(B * H * 384 * 4) // 256) * 256
-    assert fa.fa_bwd_workspace_size(B, H, S, D) == acc + 2 * rows + 256
+    up = lambda x: -(-x // 256) * 256  # noqa: E731
+    acc = up(B * H * S * D * 4)
+    rows = up(B * H * 384 * 4)
+    flags = up(B * H * 5 * 4 * 4)
+    assert fa.fa_bwd_workspace_size(B, H, S, D) == acc + 2 * rows + flags + 256
 
 
 @pytest.mark.parametrize("args,code", [
@@ -164,6 +167,7 @@ def test_bwd_workspace_size(lib):
     (dict(dtype=3), _lib.FA_ERR_DTYPE),
     (dict(scale=math.nan), _lib.FA_ERR_SCALE),
     (dict(causal=5), _lib.FA_ERR_ARG),
+    (dict(det=2), _lib.FA_ERR_ARG),
     (dict(dout=0), _lib.FA_ERR_NULL),
     (dict(dq=0), _lib.FA_ERR_NULL),
     (dict(ws=0), _lib.FA_ERR_WORKSPACE),
@@ -174,13 +178,14 @@ def test_bwd_workspace_size(lib):
 ])
 def test_fa_bwd_invalid_arguments(lib, args, code):
     a = dict(q=A, k=A, v=A, o=A, dout=A, lse=A, dq=A, dk=A, dv=A, ws=A, ws_bytes=1 << 30, B=1, H=2, Sq=100, Sk=300,
-             D=64, scale=0.125, causal=0, dtype=0)
+             D=64, scale=0.125, causal=0, det=0, dtype=0)
     a.update(args)
     st = fa.fa_bwd(a["q"], a["k"], a["v"], a["o"], a["dout"], a["lse"], a["dq"], a["dk"], a["dv"], a["ws"],
-                   a["ws_bytes"], a["B"], a["H"], a["Sq"], a["Sk"], a["D"], a["scale"], a["causal"], a["dtype"], 0)
+                   a["ws_bytes"], a["B"], a["H"], a["Sq"], a["Sk"], a["D"], a["scale"], a["causal"], a["det"],
+                   a["dtype"], 0)
     assert st == code
 
 
 def test_fa_bwd_empty_problems(lib):
     for B, H, Sq, Sk in ((0, 2, 10, 10), (1, 0, 10, 10), (1, 2, 0, 0)):
-        assert fa.fa_bwd(0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0, B, H, Sq, Sk, 64, 0.1, 0, 0, 0) == _lib.FA_OK
+        assert fa.fa_bwd(0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0, B, H, Sq, Sk, 64, 0.1, 0, 0, 0, 0) == _lib.FA_OK

@@ -87,7 +87,7 @@ def test_bwd_zero_queries_zero_key_gradients():
     dv = torch.full_like(k, float("nan"))
     st = torch.cuda.current_stream().cuda_stream
     rc = fa.fa_bwd(0, k.data_ptr(), k.data_ptr(), 0, 0, 0, 0, dk.data_ptr(), dv.data_ptr(), 0, 0, 1, 2, 0, 100, 64,
-                   0.125, 0, fa.FA_FP16, st)
+                   0.125, 0, 0, fa.FA_FP16, st)
     assert rc == 0
     torch.cuda.synchronize()
     assert torch.all(dk == 0) and torch.all(dv == 0)
@@ -101,6 +101,35 @@ def test_bwd_rejects_small_workspace():
     st = torch.cuda.current_stream().cuda_stream
     p = q.data_ptr()
     assert fa.fa_bwd(p, p, p, p, p, lse.data_ptr(), p, p, p, ws.data_ptr(), need - 1, 1, 1, 128, 128, 64, 0.125, 0,
-                     fa.FA_FP16, st) == -13
+                     0, fa.FA_FP16, st) == -13
     assert fa.fa_bwd(p, p, p, p, p, lse.data_ptr(), p, p, p, ws.data_ptr() + 16, need, 1, 1, 128, 128, 64, 0.125, 0,
-                     fa.FA_FP16, st) == -13
+                     0, fa.FA_FP16, st) == -13
+
+
+@pytest.mark.parametrize("shape", [(1, 2, 300, 300, 128), (2, 2, 200, 456, 64), (1, 1, 513, 513, 64),
+                                   (1, 2, 640, 1000, 128)], ids=lambda s: "x".join(map(str, s)))
+@pytest.mark.parametrize("causal", [False, True], ids=["full", "causal"])
+def test_bwd_deterministic_mode_matches_oracle(shape, causal):
+    B, H, Sq, Sk, D = shape
+    q, k, v = make_cross_inputs(B, H, Sq, Sk, D, "bf16", seed=Sq + Sk)
+    dout = _dout(q.shape, "bf16", seed=Sq)
+    scale = softmax_scale(D)
+    gq, gk, gv, _, _ = run_fa_bwd(q, k, v, dout, scale, causal, deterministic=True)
+    dq, dk, dv, mq, mk, mv = oracle.attn_bwd(q, k, v, dout, scale, causal, "bf16", magnitudes=True)
+    print(compare_bwd((gq, gk, gv), (dq, dk, dv), (mq, mk, mv), "bf16", q, k, dout, scale, causal))
+
+
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("causal", [False, True], ids=["full", "causal"])
+def test_bwd_deterministic_mode_is_bitwise_repeatable(D, causal):
+    """S = 4096 (32 key tiles per head): dQ, dK, dV identical over three runs."""
+    q, k, v = make_inputs(1, 6, 4096, D, "bf16", seed=21)
+    dout = _dout(q.shape, "bf16", seed=22)
+    runs = [run_fa_bwd(q, k, v, dout, softmax_scale(D), causal, deterministic=True)[:3] for _ in range(3)]
+    for r in runs[1:]:
+        for a, b in zip(r, runs[0]):
+            assert torch.equal(a, b)
+    # and it agrees with the atomic mode to rounding (same products, another order of dQ sums)
+    ga = run_fa_bwd(q, k, v, dout, softmax_scale(D), causal)[:3]
+    assert torch.equal(ga[1], runs[0][1]) and torch.equal(ga[2], runs[0][2])
+    assert torch.allclose(ga[0].float(), runs[0][0].float(), rtol=2e-2, atol=2e-3)

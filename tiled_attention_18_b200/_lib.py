@@ -50,7 +50,8 @@ SIGNATURES = [
     ("fa_bwd_workspace_size", ctypes.c_longlong, [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int]),
     ("fa_bwd", ctypes.c_int,
      [ctypes.c_void_p] * 10 + [ctypes.c_longlong, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
-                               ctypes.c_int, ctypes.c_float, ctypes.c_int, ctypes.c_int, ctypes.c_void_p]),
+                               ctypes.c_int, ctypes.c_float, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                               ctypes.c_void_p]),
     ("fa_check_status", ctypes.c_int, [ctypes.c_void_p]),
     ("fa_last_timeout_site", ctypes.c_int, []),
     ("fa_selftest_timeout", ctypes.c_int, [ctypes.c_void_p]),
@@ -126,10 +127,11 @@ def fa_bwd_workspace_size(B: int, H: int, Sq: int, D: int) -> int:
 
 def fa_bwd(q_ptr: int, k_ptr: int, v_ptr: int, o_ptr: int, do_ptr: int, lse_ptr: int, dq_ptr: int, dk_ptr: int,
            dv_ptr: int, ws_ptr: int, ws_bytes: int, B: int, H: int, Sq: int, Sk: int, D: int, scale: float,
-           causal: int, dtype: int, stream: int) -> int:
+           causal: int, deterministic: int, dtype: int, stream: int) -> int:
     """Raw C call of the backward pass (see include/fa.h)."""
     return int(load().fa_bwd(q_ptr, k_ptr, v_ptr, o_ptr, do_ptr, lse_ptr, dq_ptr, dk_ptr, dv_ptr, ws_ptr,
-                             int(ws_bytes), B, H, Sq, Sk, D, float(scale), int(causal), int(dtype), stream))
+                             int(ws_bytes), B, H, Sq, Sk, D, float(scale), int(causal), int(deterministic),
+                             int(dtype), stream))
 
 
 def fa_check_status(stream: int = 0) -> int:

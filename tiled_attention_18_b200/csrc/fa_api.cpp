@@ -288,12 +288,13 @@ long long fa_bwd_workspace_size(int B, int H, int Sq, int D) {
 
 int fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse, void* dq,
            void* dk, void* dv, void* workspace, long long workspace_bytes, int B, int H, int Sq, int Sk, int D,
-           float scale, int causal, int dtype, cudaStream_t stream) {
+           float scale, int causal, int deterministic, int dtype, cudaStream_t stream) {
     if (B < 0 || H < 0 || Sq < 0 || Sk < 0) return FA_ERR_SHAPE;
     if (D != 64 && D != 128) return FA_ERR_HEADDIM;
     if (dtype != FA_FP16 && dtype != FA_BF16) return FA_ERR_DTYPE;
     if (!(std::isfinite(scale) && scale > 0.f)) return FA_ERR_SCALE;
     if (causal != 0 && causal != 1) return FA_ERR_ARG;
+    if (deterministic != 0 && deterministic != 1) return FA_ERR_ARG;
     if (B == 0 || H == 0 || (Sq == 0 && Sk == 0)) return FA_OK;  // empty problem
     if (Sk == 0 || (causal && Sq > Sk)) return FA_ERR_SHAPE;     // a query would see no key
     const int64_t BH = (int64_t)B * H;
@@ -350,6 +351,14 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const voi
     a.lse2 = reinterpret_cast<float*>(w + ws.lse2);
     a.delta = reinterpret_cast<float*>(w + ws.delta);
     a.sched = reinterpret_cast<unsigned int*>(w + ws.sched);
+    a.dq_flags = nullptr;
+    if (deterministic) {
+        a.dq_flags = reinterpret_cast<int*>(w + ws.flags);
+        if (cudaMemsetAsync(a.dq_flags, 0, (size_t)ws.flags_bytes, stream) != cudaSuccess) {
+            cudaGetLastError();
+            return FA_ERR_LAUNCH;
+        }
+    }
     a.B = B;
     a.H = H;
     a.Sq = Sq;
@@ -415,7 +424,7 @@ const char* fa_status_string(int status) {
         case FA_ERR_LAUNCH: return "CUDA runtime error";
         case FA_ERR_TIMEOUT: return "a device-side wait exceeded its bound";
         case FA_ERR_SCALE: return "scale must be finite and > 0";
-        case FA_ERR_ARG: return "causal must be 0 or 1";
+        case FA_ERR_ARG: return "causal (and deterministic) must be 0 or 1";
         case FA_ERR_PTR: return "pointer is not device memory of the current device";
         case FA_ERR_STRIDE: return "a stride is not positive, a multiple of 8 elements and below 2^36";
         case FA_ERR_WORKSPACE: return "workspace is NULL, not 256-byte aligned or smaller than fa_bwd_workspace_size";

@@ -123,6 +123,9 @@ struct BwdParams {
     uint8_t* dv;
     int BH, H, Sq, Sk, Sq_pad, n_mtiles, n_ktiles, n_units, causal, causal_off;
     int head_group;       // causal claim order: heads per group (their Q, dO, dQ fit in L2)
+    int* dq_flags;        // deterministic mode: [BH][flag_steps][4] key tiles added so far per
+                          // (head, query step, warp); null: dQ is added with atomics
+    int flag_steps;
     float scale_log2;     // scale * log2(e)
     float scale;
     unsigned int* sched;  // zeroed unit counter (causal), or null
@@ -185,6 +188,45 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_
 __device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
     asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
                  : "memory");
+}
+
+// Deterministic dQ: the key tiles of one head add their dQ contributions to
+// each query step in key-tile order.  A warp waits (bounded) until the step's
+// counter for it equals its key tile, adds with plain loads and stores that
+// bypass L1, and passes the turn on with a release store.  Units are claimed
+// from the counter in key-tile order, so the tile a warp waits for belongs to a
+// CTA that is already running.
+__device__ __forceinline__ bool wait_turn(const int* flag, int target, volatile uint32_t* abort_flag, int site) {
+    int ok = 1;
+    if ((threadIdx.x & 31) == 0) {
+        const long long t0 = clock64();
+        for (uint32_t it = 0;; ++it) {
+            int v;
+            asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(flag) : "memory");
+            if (v == target) break;
+            if ((it & 15u) == 15u) {
+                if (*abort_flag) { ok = 0; break; }
+                if (clock64() - t0 > WAIT_TIMEOUT_CYCLES) {
+                    *abort_flag = 1u;
+                    record_failure(site);
+                    ok = 0;
+                    break;
+                }
+            }
+            __nanosleep(32);
+        }
+    }
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    __syncwarp();
+    return ok != 0;
+}
+
+__device__ __forceinline__ void pass_turn(int* flag, int next) {
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) {
+        __threadfence();
+        asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(flag), "r"(next) : "memory");
+    }
 }
 
 __device__ __forceinline__ void fence_async_smem() {
@@ -490,17 +532,33 @@ __device__ void bwd_out_role(const BwdParams& p, uint8_t* smem, uint32_t tmem, i
             const int q = m * TILE + row;
             const bool valid = q < p.Sq;
             float* dst = p.dq_acc + ((size_t)U.bh * (size_t)p.Sq + (size_t)(valid ? q : 0)) * D;
+            int* flag = p.dq_flags ? p.dq_flags + ((size_t)U.bh * p.flag_steps + m) * 4 + warp_in_group : nullptr;
+            if (flag && !wait_turn(flag, U.n, abort_flag, 56)) return;
 #pragma unroll 1
             for (int c = 0; c < D / 32; ++c) {
                 uint32_t r[32];
                 tmem_ld32u(tmem + lane_sel + C::DQ + 32 * c, r);
                 if (valid) {
+                    if (flag) {
 #pragma unroll
-                    for (int i = 0; i < 8; ++i)
-                        red_add_v4(dst + 32 * c + 4 * i, __uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]),
-                                   __uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3]));
+                        for (int i = 0; i < 8; ++i) {
+                            float4* a4 = reinterpret_cast<float4*>(dst + 32 * c + 4 * i);
+                            float4 v = __ldcg(a4);
+                            v.x += __uint_as_float(r[4 * i]);
+                            v.y += __uint_as_float(r[4 * i + 1]);
+                            v.z += __uint_as_float(r[4 * i + 2]);
+                            v.w += __uint_as_float(r[4 * i + 3]);
+                            __stcg(a4, v);
+                        }
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 8; ++i)
+                            red_add_v4(dst + 32 * c + 4 * i, __uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]),
+                                       __uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3]));
+                    }
                 }
             }
+            if (flag) pass_turn(flag, U.n + 1);
             tc_fence_before();
             mbar_arrive(bar(L::B_DQEMPTY));
         }
@@ -971,20 +1029,52 @@ __device__ void bwd2_out_role(const BwdParams& p, uint8_t* smem, uint32_t tmem, 
             const uint32_t b = g & 1u;
             if (!__all_sync(0xffffffffu, mbar_wait(bar(L::B_DQFULL + b), (g >> 1) & 1u, abort_flag, 74))) return;
             tc_fence_after();
-            uint32_t r0[32], r1[32];
-            tmem_ld32u(tmem + lane_sel + col2_dp(b), r0);
-            tmem_ld32u(tmem + lane_sel + col2_dp(b) + 32, r1);
-            tc_fence_before();
-            mbar_arrive(bar(L::B_DQEMPTY + b));
             // dQ[q][d] += dQ^T[d][q]: consecutive threads take consecutive d (coalesced)
             float* dst = p.dq_acc + ((size_t)U.bh * (size_t)p.Sq + (size_t)m * QM) * 128 + row;
             const int nq = min(QM, p.Sq - m * QM);
+            if (!p.dq_flags) {
+                // read the whole step, free the columns, then add with atomics
+                uint32_t r0[32], r1[32];
+                tmem_ld32u(tmem + lane_sel + col2_dp(b), r0);
+                tmem_ld32u(tmem + lane_sel + col2_dp(b) + 32, r1);
+                tc_fence_before();
+                mbar_arrive(bar(L::B_DQEMPTY + b));
 #pragma unroll
-            for (int j = 0; j < 32; ++j)
-                if (j < nq) atomicAdd(dst + (size_t)j * 128, __uint_as_float(r0[j]));
+                for (int j = 0; j < 32; ++j)
+                    if (j < nq) atomicAdd(dst + (size_t)j * 128, __uint_as_float(r0[j]));
 #pragma unroll
-            for (int j = 0; j < 32; ++j)
-                if (32 + j < nq) atomicAdd(dst + (size_t)(32 + j) * 128, __uint_as_float(r1[j]));
+                for (int j = 0; j < 32; ++j)
+                    if (32 + j < nq) atomicAdd(dst + (size_t)(32 + j) * 128, __uint_as_float(r1[j]));
+            } else {
+                // this key tile's turn for the step, then 32 queries at a time:
+                // read-modify-write in batches of 16 (loads in flight together)
+                int* flag = p.dq_flags + ((size_t)U.bh * p.flag_steps + m) * 4 + warp_in_group;
+                if (!wait_turn(flag, U.n, abort_flag, 57)) return;
+#pragma unroll 1
+                for (int hh = 0; hh < 2; ++hh) {
+                    uint32_t r[32];
+                    tmem_ld32u(tmem + lane_sel + col2_dp(b) + 32 * hh, r);
+                    if (hh == 1) {
+                        tc_fence_before();
+                        mbar_arrive(bar(L::B_DQEMPTY + b));
+                    }
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        float v[16];
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) {
+                            const int jq = 32 * hh + 16 * h + j;
+                            v[j] = jq < nq ? __ldcg(dst + (size_t)jq * 128) : 0.f;
+                        }
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) {
+                            const int jq = 32 * hh + 16 * h + j;
+                            if (jq < nq) __stcg(dst + (size_t)jq * 128, v[j] + __uint_as_float(r[16 * h + j]));
+                        }
+                    }
+                }
+                pass_turn(flag, U.n + 1);
+            }
         }
         if (!__all_sync(0xffffffffu, mbar_wait(bar(L::B_DKVFULL), kvp, abort_flag, 75))) return;
         tc_fence_after();
@@ -1181,7 +1271,11 @@ cudaError_t launch_bwd_impl(const BwdLaunchArgs& a, cudaStream_t stream) {
         }
         p.scale_log2 = a.scale * 1.4426950408889634f;
         p.scale = a.scale;
-        p.sched = a.causal ? a.sched : nullptr;
+        // units are claimed from the counter with the mask (they differ in length)
+        // and in deterministic mode (the order of dQ additions follows the claims)
+        p.sched = (a.causal || a.dq_flags) ? a.sched : nullptr;
+        p.dq_flags = a.dq_flags;
+        p.flag_steps = (D == 128) ? (a.Sq + QM - 1) / QM : n_mtiles;
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3((unsigned)a.grid, 1, 1);
         cfg.blockDim = dim3(D == 128 ? BWD2_THREADS : BWD_THREADS, 1, 1);

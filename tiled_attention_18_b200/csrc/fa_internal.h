@@ -58,6 +58,7 @@ struct BwdLaunchArgs {
     float* lse2;            // workspace: [B*H][Sq_pad] fp32
     float* delta;           // workspace: [B*H][Sq_pad] fp32
     unsigned int* sched;    // workspace: unit counter
+    int* dq_flags;          // workspace: deterministic-mode turn counters, or null (atomic mode)
     int B;
     int H;
     int Sq;
@@ -72,7 +73,7 @@ struct BwdLaunchArgs {
 // Byte offsets of the backward workspace parts (each 256-byte aligned) and
 // its total size.  Sq_pad = Sq rounded up to a multiple of 128.
 struct BwdWorkspace {
-    int64_t dq_acc, lse2, delta, sched, total;
+    int64_t dq_acc, lse2, delta, flags, flags_bytes, sched, total;
 };
 inline BwdWorkspace bwd_workspace_layout(int64_t BH, int64_t Sq, int64_t D) {
     auto up = [](int64_t x) { return (x + 255) / 256 * 256; };
@@ -81,7 +82,9 @@ inline BwdWorkspace bwd_workspace_layout(int64_t BH, int64_t Sq, int64_t D) {
     w.dq_acc = 0;
     w.lse2 = up(BH * Sq * D * 4);
     w.delta = w.lse2 + up(BH * Sq_pad * 4);
-    w.sched = w.delta + up(BH * Sq_pad * 4);
+    w.flags = w.delta + up(BH * Sq_pad * 4);
+    w.flags_bytes = BH * ((Sq + 63) / 64) * 4 * 4;  // [BH][64-row steps][4 warps] int
+    w.sched = w.flags + up(w.flags_bytes);
     w.total = w.sched + 256;
     return w;
 }
