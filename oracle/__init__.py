@@ -23,12 +23,15 @@ ctypes.  Function-level citations are in the C file's header:
   Sk keys (cross-attention) and the causal mask aligned to the last Sq keys.
 - ``attn_bwd`` : dQ, dK, dV by the chain rule through the definition (the
   softmax Jacobian), with optional absolute-value error scales.
+- ``attn_fwd_masked`` : the definition with an explicit boolean mask.
 
 Parity pins: every function above is pinned by tests in tests/test_oracle.py and
 tests/test_oracle_general.py (torch SDPA in float64 with an explicit mask, the
 Q = 0 closed form, agreement with attn_fwd when Sq = Sk) and
 tests/test_oracle_bwd.py (float64 autograd, central finite differences of
-attn_fwd_gen, closed forms and column-sum identities).
+attn_fwd_gen, closed forms and column-sum identities) and
+tests/test_oracle_mask.py (SDPA fp64 with a boolean mask, all-ones mask =
+no mask, lower-triangular mask = the causal flag, fully masked rows).
 """
 from __future__ import annotations
 
@@ -99,6 +102,10 @@ def _load():
         lib.oracle_attn_bwd.argtypes = [u16p, u16p, u16p, u16p, i64, i64, i64, i64, i64, ctypes.c_float,
                                         ctypes.c_int, ctypes.c_int, f64p, f64p, f64p, f64p, f64p, f64p]
         lib.oracle_attn_bwd.restype = ctypes.c_int
+        lib.oracle_attn_fwd_masked.argtypes = [u16p, u16p, u16p, i64, i64, i64, i64, i64, ctypes.c_float,
+                                               ctypes.c_int, ctypes.c_int, ctypes.POINTER(ctypes.c_uint8), i64, i64,
+                                               i64, f64p, f64p]
+        lib.oracle_attn_fwd_masked.restype = ctypes.c_int
         lib.oracle_causal_tile_count.argtypes = [i64, i64, i64, i64p, i64p, i64p]
         lib.oracle_causal_tile_count.restype = None
         lib.oracle_num_threads.argtypes = []
@@ -217,6 +224,32 @@ def attn_rows_gen(q, k, v, scale: float, causal: bool, dtype, bh_idx, row_idx):
                                   _ptr(o, ctypes.c_double), _ptr(lse, ctypes.c_double))
     if rc != 0:
         raise RuntimeError(f"oracle_attn_rows_gen failed with {rc}")
+    return o, lse
+
+
+def attn_fwd_masked(q, k, v, mask, scale: float, causal: bool, dtype):
+    """attn_fwd_gen with an explicit boolean mask: ``mask`` broadcasts to
+    [B, H, Sq, Sk] (a bool/uint8 tensor or array whose b and h dimensions may
+    be 1); query i sees key j iff mask[..., i, j] (and the causal rule).  Rows
+    that see no key give O = 0 and LSE = -inf."""
+    lib = _load()
+    qb, kb, vb = _bits(q), _bits(k), _bits(v)
+    B, H, Sq, D = qb.shape
+    Sk = kb.shape[2]
+    m = np.asarray(mask.cpu().numpy() if hasattr(mask, "cpu") else mask).astype(np.uint8)
+    if m.ndim != 4 or m.shape[2:] != (Sq, Sk) or m.shape[0] not in (1, B) or m.shape[1] not in (1, H):
+        raise ValueError("mask must be [B|1, H|1, Sq, Sk]")
+    m = np.ascontiguousarray(m)
+    sb = 0 if m.shape[0] == 1 else m.shape[1] * Sq * Sk
+    sh = 0 if m.shape[1] == 1 else Sq * Sk
+    o = np.empty((B, H, Sq, D))
+    lse = np.empty((B, H, Sq))
+    rc = lib.oracle_attn_fwd_masked(_ptr(qb, ctypes.c_uint16), _ptr(kb, ctypes.c_uint16), _ptr(vb, ctypes.c_uint16),
+                                    B, H, Sq, Sk, D, float(np.float32(scale)), int(bool(causal)), _dtype_code(dtype),
+                                    _ptr(m, ctypes.c_uint8), sb, sh, Sk, _ptr(o, ctypes.c_double),
+                                    _ptr(lse, ctypes.c_double))
+    if rc != 0:
+        raise RuntimeError(f"oracle_attn_fwd_masked failed with {rc}")
     return o, lse
 
 

@@ -680,3 +680,75 @@ int oracle_attn_bwd(const uint16_t *q, const uint16_t *k, const uint16_t *v, con
     }
     return 0;
 }
+
+/* ------------------------------------------------------------ explicit mask */
+
+/*
+ * The general definition with an explicit boolean mask: query i of head (b, h)
+ * sees key j iff mask[b][h][i][j] != 0 (and, with causal = 1, j <= i + Sk - Sq).
+ * The mask is uint8 with element strides mask_sb, mask_sh, mask_si over b, h
+ * and the query row (0 broadcasts) and contiguous keys.  A row that sees no key
+ * gets O = 0 and LSE = -inf.  Sources: the fused mask of the FlashAttention-2
+ * page, section 3.4 (a score whose mask entry is false becomes -infinity
+ * before the softmax); the explicit mask matrix of the gsyq.cn catlass page
+ * ("Causal Mask的实现差异", mode 1).
+ */
+int oracle_attn_fwd_masked(const uint16_t *q, const uint16_t *k, const uint16_t *v, int64_t B, int64_t H,
+                           int64_t Sq, int64_t Sk, int64_t D, float scale, int causal, int dtype,
+                           const uint8_t *mask, int64_t mask_sb, int64_t mask_sh, int64_t mask_si, double *o,
+                           double *lse)
+{
+    if (B < 0 || H < 0 || Sq < 0 || Sk < 0 || D <= 0) return -2;
+    if (dtype != ORACLE_F16 && dtype != ORACLE_BF16) return -4;
+    const double sc = (double)scale;
+    for (int64_t b = 0; b < B; ++b)
+        for (int64_t h = 0; h < H; ++h) {
+            const int64_t bh = b * H + h;
+            double *qh = (double *)malloc(sizeof(double) * (size_t)(Sq * D > 0 ? Sq * D : 1));
+            double *kh = (double *)malloc(sizeof(double) * (size_t)(Sk * D > 0 ? Sk * D : 1));
+            double *vh = (double *)malloc(sizeof(double) * (size_t)(Sk * D > 0 ? Sk * D : 1));
+            if (!qh || !kh || !vh) { free(qh); free(kh); free(vh); return -10; }
+            oracle_decode(q + bh * Sq * D, qh, Sq * D, dtype);
+            oracle_decode(k + bh * Sk * D, kh, Sk * D, dtype);
+            oracle_decode(v + bh * Sk * D, vh, Sk * D, dtype);
+#pragma omp parallel
+            {
+                double *srow = (double *)malloc(sizeof(double) * (size_t)(Sk > 0 ? Sk : 1));
+                int64_t *idx = (int64_t *)malloc(sizeof(int64_t) * (size_t)(Sk > 0 ? Sk : 1));
+#pragma omp for schedule(dynamic, 16)
+                for (int64_t i = 0; i < Sq; ++i) {
+                    const uint8_t *mrow = mask + b * mask_sb + h * mask_sh + i * mask_si;
+                    const int64_t nvis = visible_keys(i, Sq, Sk, causal);
+                    int64_t n = 0;
+                    for (int64_t j = 0; j < nvis; ++j)
+                        if (mrow[j]) idx[n++] = j;
+                    double *oi = o + (bh * Sq + i) * D;
+                    if (n == 0) {
+                        for (int64_t d = 0; d < D; ++d) oi[d] = 0.0;
+                        lse[bh * Sq + i] = -INFINITY;
+                        continue;
+                    }
+                    double m = -INFINITY;
+                    for (int64_t t = 0; t < n; ++t) {
+                        double dot = 0.0;
+                        for (int64_t d = 0; d < D; ++d) dot += qh[i * D + d] * kh[idx[t] * D + d];
+                        srow[t] = sc * dot;
+                        if (srow[t] > m) m = srow[t];
+                    }
+                    double l = 0.0;
+                    for (int64_t t = 0; t < n; ++t) {
+                        srow[t] = exp(srow[t] - m);
+                        l += srow[t];
+                    }
+                    for (int64_t d = 0; d < D; ++d) oi[d] = 0.0;
+                    for (int64_t t = 0; t < n; ++t)
+                        for (int64_t d = 0; d < D; ++d) oi[d] += srow[t] * vh[idx[t] * D + d];
+                    for (int64_t d = 0; d < D; ++d) oi[d] /= l;
+                    lse[bh * Sq + i] = m + log(l);
+                }
+                free(srow); free(idx);
+            }
+            free(qh); free(kh); free(vh);
+        }
+    return 0;
+}
