@@ -160,6 +160,29 @@ FA_API int fa_fwd_ex(const void* q, const void* k, const void* v, void* o, float
                      cudaStream_t stream);
 
 /*
+ * fa_fwd_mask -- fa_fwd_ex (contiguous BHSD, Sq queries, Sk keys) with an
+ * explicit boolean mask fused into the kernel: query i of head (b, h) attends
+ * to key j only where mask[b][h][i][j] != 0 (and, with causal = 1, j <= i + Sk
+ * - Sq).  A masked score becomes -infinity before the softmax
+ * ("FlashAttention-2 在昇腾 NPU 上如何做到 3 倍加速？", section 3.4, the fused
+ * mask; the explicit mask matrix of the gsyq.cn catlass page, "Causal Mask的
+ * 实现差异", mode 1).  A row that sees no key gets O = 0 and LSE = -infinity
+ * (the pages do not say; this is the reading taken).
+ *
+ * mask        : device, uint8 (0 = masked, nonzero = attend), keys contiguous.
+ * mask_stride : host array of 3 element strides over b, h and the query row;
+ *               0 over b or h broadcasts one mask to every batch or head.  All
+ *               three must be multiples of 16 and the row stride >= Sk (else
+ *               FA_ERR_STRIDE); mask must be 16-byte aligned (FA_ERR_ALIGN).
+ * Other arguments, ownership and errors: as fa_fwd_ex.  The mask costs a
+ * 16-byte load per 16 keys of every query row and tile; key tiles above the
+ * causal diagonal are still skipped.
+ */
+FA_API int fa_fwd_mask(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Sq,
+                       int Sk, int D, const void* mask, const long long* mask_stride, float scale, int causal,
+                       int dtype, cudaStream_t stream);
+
+/*
  * fa_bwd_workspace_size -- bytes of device workspace fa_bwd needs for B*H
  * heads of Sq query rows of dimension D: an fp32 dQ accumulator
  * [B*H][Sq][D], two fp32 row-statistic arrays [B*H][Sq rounded up to 128],

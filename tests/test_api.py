@@ -189,3 +189,23 @@ def test_fa_bwd_invalid_arguments(lib, args, code):
 def test_fa_bwd_empty_problems(lib):
     for B, H, Sq, Sk in ((0, 2, 10, 10), (1, 0, 10, 10), (1, 2, 0, 0)):
         assert fa.fa_bwd(0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0, B, H, Sq, Sk, 64, 0.1, 0, 0, 0, 0) == _lib.FA_OK
+
+
+@pytest.mark.parametrize("args,code", [
+    (dict(mask=0), _lib.FA_ERR_NULL),
+    (dict(ms=None), _lib.FA_ERR_NULL),
+    (dict(ms=(0, 0, 100)), _lib.FA_ERR_STRIDE),         # row stride below Sk
+    (dict(ms=(0, 0, 328)), _lib.FA_ERR_STRIDE),         # row stride not a multiple of 16
+    (dict(ms=(-16, 0, 336)), _lib.FA_ERR_STRIDE),
+    (dict(ms=(8, 0, 336)), _lib.FA_ERR_STRIDE),
+    (dict(mask=A + 4), _lib.FA_ERR_ALIGN),
+    (dict(D=80), _lib.FA_ERR_HEADDIM),
+    (dict(Sq=400, Sk=300, causal=1), _lib.FA_ERR_SHAPE),
+])
+def test_fa_fwd_mask_invalid_arguments(lib, args, code):
+    a = dict(q=A, k=A, v=A, o=A, lse=A, B=2, H=3, Sq=100, Sk=330, D=64, mask=A, ms=(0, 0, 336), scale=0.125,
+             causal=0, dtype=1)
+    a.update(args)
+    st = fa.fa_fwd_mask(a["q"], a["k"], a["v"], a["o"], a["lse"], a["B"], a["H"], a["Sq"], a["Sk"], a["D"], a["mask"],
+                        a["ms"], a["scale"], a["causal"], a["dtype"], 0)
+    assert st == code

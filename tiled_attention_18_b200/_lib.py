@@ -47,6 +47,9 @@ SIGNATURES = [
      [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
       ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
       _LL3, _LL3, _LL3, _LL3, ctypes.c_float, ctypes.c_int, ctypes.c_int, ctypes.c_void_p]),
+    ("fa_fwd_mask", ctypes.c_int,
+     [ctypes.c_void_p] * 5 + [ctypes.c_int] * 5 + [ctypes.c_void_p, _LL3, ctypes.c_float, ctypes.c_int, ctypes.c_int,
+                                                ctypes.c_void_p]),
     ("fa_bwd_workspace_size", ctypes.c_longlong, [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int]),
     ("fa_bwd", ctypes.c_int,
      [ctypes.c_void_p] * 10 + [ctypes.c_longlong, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
@@ -119,6 +122,13 @@ def fa_fwd_ex(q_ptr: int, k_ptr: int, v_ptr: int, o_ptr: int, lse_ptr: int, B: i
     return int(load().fa_fwd_ex(q_ptr, k_ptr, v_ptr, o_ptr, lse_ptr, B, H, Sq, Sk, D, _strides(q_stride),
                                 _strides(k_stride), _strides(v_stride), _strides(o_stride), float(scale),
                                 int(causal), int(dtype), stream))
+
+
+def fa_fwd_mask(q_ptr: int, k_ptr: int, v_ptr: int, o_ptr: int, lse_ptr: int, B: int, H: int, Sq: int, Sk: int,
+                D: int, mask_ptr: int, mask_stride, scale: float, causal: int, dtype: int, stream: int) -> int:
+    """Raw C call of the explicit-mask forward: mask_stride is a (b, h, row) element-stride triple."""
+    return int(load().fa_fwd_mask(q_ptr, k_ptr, v_ptr, o_ptr, lse_ptr, B, H, Sq, Sk, D, mask_ptr,
+                                  _strides(mask_stride), float(scale), int(causal), int(dtype), stream))
 
 
 def fa_bwd_workspace_size(B: int, H: int, Sq: int, D: int) -> int:

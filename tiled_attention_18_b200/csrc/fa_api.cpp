@@ -165,7 +165,8 @@ enum class Scratch { Allocated, Static };
 // in the documented order, tensor maps, grid size, scheduler counter, launch.
 int forward(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Sq, int Sk, int D,
             const long long* q_stride, const long long* k_stride, const long long* v_stride,
-            const long long* o_stride, float scale, int causal, int dtype, cudaStream_t stream, Scratch scratch) {
+            const long long* o_stride, float scale, int causal, int dtype, cudaStream_t stream, Scratch scratch,
+            const uint8_t* mask = nullptr, const long long* mask_stride = nullptr) {
     if (B < 0 || H < 0 || Sq < 0 || Sk < 0) return FA_ERR_SHAPE;
     if (D != 64 && D != 128) return FA_ERR_HEADDIM;
     if (dtype != FA_FP16 && dtype != FA_BF16) return FA_ERR_DTYPE;
@@ -183,7 +184,16 @@ int forward(const void* q, const void* k, const void* v, void* o, float* lse, in
     if (rc == FA_OK) rc = resolve_strides(v_stride, B, H, Sk, D, vs);
     if (rc == FA_OK) rc = resolve_strides(o_stride, B, H, Sq, D, os);
     if (rc != FA_OK) return rc;
-    const uintptr_t a16 = (uintptr_t)q | (uintptr_t)k | (uintptr_t)v | (uintptr_t)o;
+    long long ms[3] = {0, 0, 0};
+    if (mask) {
+        // element strides over b, h, query row: 0 broadcasts over b or h; rows
+        // at least Sk apart and 16-byte aligned (whole 16-byte loads)
+        for (int i = 0; i < 3; ++i) ms[i] = mask_stride[i];
+        if (ms[0] < 0 || ms[1] < 0 || ms[0] >= MAX_STRIDE || ms[1] >= MAX_STRIDE || ms[2] >= MAX_STRIDE)
+            return FA_ERR_STRIDE;
+        if ((ms[2] < Sk && Sq > 1) || ms[2] % 16 != 0 || ms[0] % 16 != 0 || ms[1] % 16 != 0) return FA_ERR_STRIDE;
+    }
+    const uintptr_t a16 = (uintptr_t)q | (uintptr_t)k | (uintptr_t)v | (uintptr_t)o | (uintptr_t)mask;
     if ((a16 & 15u) != 0 || ((uintptr_t)lse & 3u) != 0) return FA_ERR_ALIGN;
 
     DeviceInfo dev;
@@ -192,7 +202,7 @@ int forward(const void* q, const void* k, const void* v, void* o, float* lse, in
     if (dev.major != 10 || dev.minor != 0) return FA_ERR_ARCH;
     int cur = 0;
     cudaGetDevice(&cur);
-    const void* ptrs[5] = {q, k, v, o, lse};
+    const void* ptrs[6] = {q, k, v, o, lse, mask ? (const void*)mask : (const void*)q};
     for (const void* p : ptrs) {
         rc = check_device_pointer(p, cur);
         if (rc != FA_OK) return rc;
@@ -210,6 +220,8 @@ int forward(const void* q, const void* k, const void* v, void* o, float* lse, in
     a.o = o;
     a.lse = lse;
     for (int i = 0; i < 3; ++i) a.o_stride[i] = os[i];
+    a.mask = mask;
+    for (int i = 0; i < 3; ++i) a.mask_stride[i] = ms[i];
     a.B = B;
     a.H = H;
     a.Sq = Sq;
@@ -258,6 +270,15 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int
            float scale, int causal, int dtype, cudaStream_t stream) {
     return forward(q, k, v, o, lse, B, H, S, S, D, nullptr, nullptr, nullptr, nullptr, scale, causal, dtype, stream,
                    Scratch::Allocated);
+}
+
+int fa_fwd_mask(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Sq, int Sk,
+                int D, const void* mask, const long long* mask_stride, float scale, int causal, int dtype,
+                cudaStream_t stream) {
+    if (B < 0 || H < 0 || Sq < 0 || Sk < 0) return FA_ERR_SHAPE;
+    if (B > 0 && H > 0 && Sq > 0 && (!mask || !mask_stride)) return FA_ERR_NULL;
+    return forward(q, k, v, o, lse, B, H, Sq, Sk, D, nullptr, nullptr, nullptr, nullptr, scale, causal, dtype, stream,
+                   Scratch::Allocated, static_cast<const uint8_t*>(mask), mask_stride);
 }
 
 int fa_fwd_ex(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Sq, int Sk, int D,

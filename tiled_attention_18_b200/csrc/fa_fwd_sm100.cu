@@ -184,6 +184,8 @@ struct KParams {
     int nkv;       // key tiles per head
     int causal;
     int causal_off;  // Sk - Sq: query i sees keys j <= i + causal_off under the mask
+    const uint8_t* mask;         // explicit boolean mask (nonzero = attend), or null
+    long long m_sb, m_sh, m_ss;  // its element strides over b, h and the query row (keys contiguous)
     float scale_log2;
     unsigned int* sched;  // zeroed unit counter (claim order), or null for the static order
 };
@@ -262,6 +264,40 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
     float r;
     asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
     return r;
+}
+
+// The 128 mask bytes of keys [kbase, kbase + 128) of one query row as a 128-bit
+// mask (bit c of word c / 32 = key kbase + c may be attended).  Keys at or past
+// Sk read as 0.  Whole 16-byte loads when the tile is complete (the row and the
+// tile start are 16-byte aligned), byte loads on the ragged last tile.
+__device__ __forceinline__ void load_mask_bits(const uint8_t* mrow, int kbase, int Sk, uint32_t (&bits)[4]) {
+    if (kbase + BLOCK_N <= Sk) {
+        const uint4* src = reinterpret_cast<const uint4*>(mrow + kbase);
+        uint4 w[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) w[i] = __ldg(src + i);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            uint32_t acc = 0;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const uint4 x = w[2 * q + h];
+                const uint32_t ws[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    // one bit per nonzero byte, gathered into a nibble (byte i -> bit i)
+                    const uint32_t t = __vcmpne4(ws[e], 0u) & 0x01010101u;
+                    acc |= ((t * 0x01020408u) >> 24 & 0xFu) << (16 * h + 4 * e);
+                }
+            }
+            bits[q] = acc;
+        }
+    } else {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) bits[q] = 0u;
+        for (int c = 0; c < Sk - kbase; ++c)
+            if (mrow[kbase + c]) bits[c >> 5] |= 1u << (c & 31);
+    }
 }
 
 struct Unit {
@@ -551,7 +587,7 @@ __device__ void mma_role(const KParams& p, uint8_t* smem, uint32_t tmem, volatil
     mbar_drain(bar(L::B_FIN), 0u);
 }
 
-template <int D, bool BF16>
+template <int D, bool BF16, bool MASK>
 __device__ void softmax_role(const KParams& p, uint8_t* smem, uint32_t tmem, int t, int warp_in_group,
                              volatile uint32_t* abort_flag) {
     using L = Smem<D>;
@@ -582,6 +618,15 @@ __device__ void softmax_role(const KParams& p, uint8_t* smem, uint32_t tmem, int
         float m_use = -INFINITY;  // reference max in log2 units
         float l = 0.f;            // running sum of the weights relative to m_use (fp32)
         float lr = 0.f;           // the same sum over the weights as rounded for P.V
+        // explicit mask: this row's bits for the next key tile, loaded while the
+        // previous tile's MMAs run (rows past Sq read the last row)
+        const uint8_t* mrow = nullptr;
+        uint32_t mbits[4] = {0u, 0u, 0u, 0u};
+        if constexpr (MASK) {
+            const int ub = U.bh / p.H, uh = U.bh - ub * p.H;
+            mrow = p.mask + (long long)ub * p.m_sb + (long long)uh * p.m_sh + (long long)min(row, p.Sq - 1) * p.m_ss;
+            load_mask_bits(mrow, 0, p.Sk, mbits);
+        }
         for (int j = 0; j < n; ++j) {
             // the result is made warp-uniform: the TMEM accesses below need the whole warp
             if (!__all_sync(0xffffffffu, mbar_wait(bar(L::B_SFULL + t), s_phase, abort_flag, 16 + t))) return;
@@ -597,6 +642,11 @@ __device__ void softmax_role(const KParams& p, uint8_t* smem, uint32_t tmem, int
 #pragma unroll
                 for (int c = 0; c < BLOCK_N; ++c)
                     if (c > lim) s[c] = -INFINITY;
+            }
+            if constexpr (MASK) {
+#pragma unroll
+                for (int c = 0; c < BLOCK_N; ++c)
+                    if (!((mbits[c >> 5] >> (c & 31)) & 1u)) s[c] = -INFINITY;
             }
             float mx0 = max3(s[0], s[1], s[2]), mx1 = max3(s[3], s[4], s[5]);
             float mx2 = max3(s[6], s[7], s[8]), mx3 = max3(s[9], s[10], s[11]);
@@ -670,10 +720,17 @@ __device__ void softmax_role(const KParams& p, uint8_t* smem, uint32_t tmem, int
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(bar(L::B_PFULL + t));
+            if constexpr (MASK) {
+                if (j + 1 < n) load_mask_bits(mrow, kbase + BLOCK_N, p.Sk, mbits);
+            }
         }
-        // final statistics for the epilogue: 1/l for O, LSE = (m + log2 l) ln 2
+        // final statistics for the epilogue: 1/l for O, LSE = (m + log2 l) ln 2;
+        // a row with no visible key (possible only with an explicit mask) gets
+        // O = 0 and LSE = -inf
         const float norm = Policy<BF16>::NORM_BY_ROUNDED_P ? lr : l;
-        fin_buf[fin_par * 2 * BLOCK_M] = make_float2(1.f / norm, (m_use + __log2f(l)) * 0.69314718055994530942f);
+        fin_buf[fin_par * 2 * BLOCK_M] = (l > 0.f)
+            ? make_float2(1.f / norm, (m_use + __log2f(l)) * 0.69314718055994530942f)
+            : make_float2(0.f, -INFINITY);
         mbar_arrive(bar(L::B_FINAL + 2 * fin_par + t));
         fin_par ^= 1;
     }
@@ -783,7 +840,7 @@ __device__ void correction_role(const KParams& p, uint8_t* smem, uint32_t tmem, 
     }
 }
 
-template <int D, bool BF16>
+template <int D, bool BF16, bool MASK>
 __global__ void __launch_bounds__(NUM_THREADS, 1) fa_fwd_kernel(const __grid_constant__ KParams p) {
     using L = Smem<D>;
     extern __shared__ uint8_t smem_raw[];
@@ -827,7 +884,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) fa_fwd_kernel(const __grid_con
 
     if (wg < 2) {
         setmaxnreg_inc<REG_SOFTMAX>();
-        softmax_role<D, BF16>(p, smem, tmem, wg, warp & 3, abort_flag);
+        softmax_role<D, BF16, MASK>(p, smem, tmem, wg, warp & 3, abort_flag);
     } else if (wg == 2) {
         setmaxnreg_dec<REG_CORR>();
         correction_role<D, BF16>(p, smem, tmem, warp & 3, abort_flag);
@@ -884,11 +941,11 @@ __global__ void __launch_bounds__(64, 1) selftest_timeout_kernel(long long deadl
     }
 }
 
-template <int D, bool BF16>
+template <int D, bool BF16, bool MASK>
 cudaError_t launch_impl(const LaunchArgs& a, cudaStream_t stream) {
     using L = Smem<D>;
     static_assert(L::ALLOC <= 232448, "shared memory budget exceeded");
-    auto kern = fa_fwd_kernel<D, BF16>;
+    auto kern = fa_fwd_kernel<D, BF16, MASK>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC);
     if (e != cudaSuccess) return e;
     KParams p;
@@ -909,6 +966,10 @@ cudaError_t launch_impl(const LaunchArgs& a, cudaStream_t stream) {
     p.nkv = (a.Sk + BLOCK_N - 1) / BLOCK_N;
     p.causal = a.causal;
     p.causal_off = a.Sk - a.Sq;
+    p.mask = a.mask;
+    p.m_sb = a.mask_stride[0];
+    p.m_sh = a.mask_stride[1];
+    p.m_ss = a.mask_stride[2];
     p.scale_log2 = a.scale_log2;
     p.sched = a.sched;
     cudaLaunchConfig_t cfg = {};
@@ -925,9 +986,11 @@ cudaError_t launch_impl(const LaunchArgs& a, cudaStream_t stream) {
 
 cudaError_t launch_fwd_sm100(const LaunchArgs& a, cudaStream_t stream) {
     if (a.D == 128) {
-        return a.dtype == 1 ? launch_impl<128, true>(a, stream) : launch_impl<128, false>(a, stream);
+        if (a.mask) return a.dtype == 1 ? launch_impl<128, true, true>(a, stream) : launch_impl<128, false, true>(a, stream);
+        return a.dtype == 1 ? launch_impl<128, true, false>(a, stream) : launch_impl<128, false, false>(a, stream);
     }
-    return a.dtype == 1 ? launch_impl<64, true>(a, stream) : launch_impl<64, false>(a, stream);
+    if (a.mask) return a.dtype == 1 ? launch_impl<64, true, true>(a, stream) : launch_impl<64, false, true>(a, stream);
+    return a.dtype == 1 ? launch_impl<64, true, false>(a, stream) : launch_impl<64, false, false>(a, stream);
 }
 
 cudaError_t launch_selftest_timeout(cudaStream_t stream) {

@@ -28,6 +28,8 @@ struct LaunchArgs {
     void* o;                // [B,H,Sq,D] 16-bit at o_stride
     float* lse;             // [B,H,Sq] fp32, contiguous
     long long o_stride[3];  // element strides of O over b, h, s (d is contiguous)
+    const uint8_t* mask;    // explicit boolean mask (nonzero = attend) or null
+    long long mask_stride[3];  // its element strides over b, h, query row (keys contiguous)
     int B;
     int H;
     int Sq;                 // query rows per head
