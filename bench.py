@@ -414,6 +414,9 @@ def main(argv=None) -> int:
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--pass", dest="pass_", choices=["fwd", "bwd"], default="fwd",
                     help="fwd: the forward pass (default); bwd: the backward pass fa_bwd")
+    ap.add_argument("--mask", choices=["none", "tril"], default="none",
+                    help="tril: causal runs go through fa_fwd_mask with an explicit lower-triangular mask "
+                         "(the catlass page's mode 1) instead of the in-kernel diagonal skip (mode 2)")
     ap.add_argument("--deterministic", action="store_true",
                     help="with --pass bwd: the deterministic dQ mode (key tiles add in order)")
     args = ap.parse_args(argv)
@@ -477,13 +480,29 @@ def main(argv=None) -> int:
         lse = torch.empty((w.B, w.H, w.S), dtype=torch.float32, device=dev)
         dev_out.append((o, lse))
 
+    # --mask tril: one shared [1, 1, Sq, Sk] uint8 lower-triangular mask (rows padded to 16 bytes)
+    tril = {}
+    if args.mask == "tril":
+        for i, w in enumerate(runs):
+            if w.causal:
+                pad = -(-w.Skv // 16) * 16
+                ii = torch.arange(w.S, device=dev)[:, None]
+                jj = torch.arange(pad, device=dev)[None, :]
+                tril[i] = ((jj <= ii + (w.Skv - w.S)) & (jj < w.Skv)).to(torch.uint8).contiguous()
+
     def launch(i, step=0):
         w = runs[i]
         q, k, v = (view(w, t) for t in dev_in[i][step % n_copies[i]])
         o, lse = dev_out[i]
         o = view(w, o)
         dt = fa.FA_BF16 if w.dtype == "bf16" else fa.FA_FP16
-        if w.general:
+        if i in tril:
+            if w.layout != "bhsd":
+                raise SystemExit("--mask takes BHSD workloads")
+            m = tril[i]
+            st = fa.fa_fwd_mask(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), w.B, w.H,
+                                w.S, w.Skv, w.D, m.data_ptr(), (0, 0, m.stride(0)), w.scale, 0, dt, sid)
+        elif w.general:
             st = fa.fa_fwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), w.B, w.H, w.S,
                               w.Skv, w.D, q.stride()[:3], k.stride()[:3], v.stride()[:3], o.stride()[:3], w.scale,
                               int(w.causal), dt, sid)
@@ -582,7 +601,9 @@ def main(argv=None) -> int:
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": max_ms / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": w0.dtype, "data": "synthetic",
-            "config": {"workload": workload_label(args.workload), "B": w0.B, "H": w0.H, "S": w0.S, "D": w0.D,
+            "config": {"workload": workload_label(args.workload)
+                       + (" (causal as an explicit lower-triangular mask, no tile skipping)" if tril else ""),
+                       "B": w0.B, "H": w0.H, "S": w0.S, "D": w0.D,
                        **({"Sk": w0.Skv, "layout": w0.layout} if w0.general else {}),
                        "runs_per_step": len(runs),
                        "l2": ("inputs larger than L2 (no flush)" if max(n_copies) == 1 else
