@@ -51,7 +51,7 @@ typedef enum {
     FA_OK = 0,
     FA_ERR_NULL = -1,     /* a required pointer is NULL */
     FA_ERR_SHAPE = -2,    /* B, H or S negative, or too large for 32-bit indexing */
-    FA_ERR_HEADDIM = -3,  /* D is not 64 or 128 */
+    FA_ERR_HEADDIM = -3,  /* D is not 64, 128 or 256 (64 or 128 for fa_fwd_mask and fa_bwd) */
     FA_ERR_DTYPE = -4,    /* dtype is not FA_FP16 or FA_BF16 */
     FA_ERR_ALIGN = -5,    /* q, k, v, o not 16-byte aligned, or lse not 4-byte aligned */
     FA_ERR_ARCH = -6,     /* the current device is not compute capability 10.0 (sm_100) */
@@ -77,7 +77,10 @@ typedef enum {
  * B, H, S : batch, heads, sequence length (queries = keys = S).  Any of them
  *           0 is an empty problem: FA_OK, nothing is launched and the pointers
  *           are not inspected.  B*H*S must fit in 31 bits.
- * D       : head dimension, 64 or 128.
+ * D       : head dimension, 64, 128 or 256.  D = 256 runs a kernel of its own
+ *           (one 128-row query tile per work unit, 64-key tiles); the pages
+ *           name 64, 128 and 256 as the common head dimensions
+ *           ("FlashAttention-2 在昇腾 NPU 上如何做到 3 倍加速？", section 3.2).
  * scale   : softmax scale (commonly 1/sqrt(D)); finite and > 0.
  * causal  : 0 = attend to all keys; 1 = key j attends to query i iff j <= i.
  * dtype   : FA_FP16 or FA_BF16 (inputs and output).  Scores, the softmax

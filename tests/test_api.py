@@ -63,7 +63,7 @@ A = 0x10000  # an aligned, non-null address (never dereferenced: checks fail fir
     (dict(B=-1), _lib.FA_ERR_SHAPE),
     (dict(S=-5), _lib.FA_ERR_SHAPE),
     (dict(D=96), _lib.FA_ERR_HEADDIM),
-    (dict(D=256), _lib.FA_ERR_HEADDIM),
+    (dict(D=512), _lib.FA_ERR_HEADDIM),
     (dict(dtype=2), _lib.FA_ERR_DTYPE),
     (dict(scale=0.0), _lib.FA_ERR_SCALE),
     (dict(scale=-1.0), _lib.FA_ERR_SCALE),
@@ -200,6 +200,7 @@ def test_fa_bwd_empty_problems(lib):
     (dict(ms=(8, 0, 336)), _lib.FA_ERR_STRIDE),
     (dict(mask=A + 4), _lib.FA_ERR_ALIGN),
     (dict(D=80), _lib.FA_ERR_HEADDIM),
+    (dict(D=256), _lib.FA_ERR_HEADDIM),               # the mask is fused into the D = 64/128 kernel only
     (dict(Sq=400, Sk=300, causal=1), _lib.FA_ERR_SHAPE),
 ])
 def test_fa_fwd_mask_invalid_arguments(lib, args, code):

@@ -168,7 +168,7 @@ int forward(const void* q, const void* k, const void* v, void* o, float* lse, in
             const long long* o_stride, float scale, int causal, int dtype, cudaStream_t stream, Scratch scratch,
             const uint8_t* mask = nullptr, const long long* mask_stride = nullptr) {
     if (B < 0 || H < 0 || Sq < 0 || Sk < 0) return FA_ERR_SHAPE;
-    if (D != 64 && D != 128) return FA_ERR_HEADDIM;
+    if (D != 64 && D != 128 && !(D == 256 && !mask)) return FA_ERR_HEADDIM;
     if (dtype != FA_FP16 && dtype != FA_BF16) return FA_ERR_DTYPE;
     if (!(std::isfinite(scale) && scale > 0.f)) return FA_ERR_SCALE;
     if (causal != 0 && causal != 1) return FA_ERR_ARG;
@@ -207,15 +207,18 @@ int forward(const void* q, const void* k, const void* v, void* o, float* lse, in
         rc = check_device_pointer(p, cur);
         if (rc != FA_OK) return rc;
     }
-    const int64_t units = fa::num_units(BH, Sq);
+    const int64_t units = (D == 256) ? fa::num_units_d256(BH, Sq) : fa::num_units(BH, Sq);
     const int grid = (int)(units < dev.sms ? units : dev.sms);
     // fa_fwd_noalloc's counter is read back as an int: the claims of all CTAs must fit
     if (scratch == Scratch::Static && units + grid > fa::NOALLOC_MAX_CLAIMS) return FA_ERR_SHAPE;
 
     fa::LaunchArgs a;
     std::memset(&a, 0, sizeof(a));
-    if (!encode_tensor(&a.tmap_q, q, B, H, Sq, D, qs, dtype) || !encode_tensor(&a.tmap_k, k, B, H, Sk, D, ks, dtype) ||
-        !encode_tensor(&a.tmap_v, v, B, H, Sk, D, vs, dtype))
+    // the D = 256 kernel streams keys and values in 64-row tiles
+    const int kv_box = (D == 256) ? 64 : fa::BLOCK_N;
+    if (!encode_tensor(&a.tmap_q, q, B, H, Sq, D, qs, dtype) ||
+        !encode_tensor(&a.tmap_k, k, B, H, Sk, D, ks, dtype, kv_box) ||
+        !encode_tensor(&a.tmap_v, v, B, H, Sk, D, vs, dtype, kv_box))
         return FA_ERR_LAUNCH;
     a.o = o;
     a.lse = lse;
@@ -251,7 +254,8 @@ int forward(const void* q, const void* k, const void* v, void* o, float* lse, in
         }
         a.sched = ctr;
     }
-    if (fa::launch_fwd_sm100(a, stream) != cudaSuccess) {
+    const cudaError_t le = (D == 256) ? fa::launch_fwd_d256_sm100(a, stream) : fa::launch_fwd_sm100(a, stream);
+    if (le != cudaSuccess) {
         cudaGetLastError();
         return FA_ERR_LAUNCH;
     }
@@ -402,19 +406,19 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const voi
 }
 
 int fa_check_status(cudaStream_t stream) {
-    int st = 0, site = 0, st_b = 0, site_b = 0;
-    if (fa::read_and_clear_status(stream, &st, &site) != cudaSuccess ||
-        fa::read_and_clear_status_bwd(stream, &st_b, &site_b) != cudaSuccess) {
+    // one status word per kernel translation unit; all are read and cleared
+    int st[3] = {0, 0, 0}, site[3] = {0, 0, 0};
+    if (fa::read_and_clear_status(stream, &st[0], &site[0]) != cudaSuccess ||
+        fa::read_and_clear_status_bwd(stream, &st[1], &site[1]) != cudaSuccess ||
+        fa::read_and_clear_status_d256(stream, &st[2], &site[2]) != cudaSuccess) {
         cudaGetLastError();
         return FA_ERR_LAUNCH;
     }
-    if (st != fa::DEV_OK) {
-        t_last_site = site;
-        return FA_ERR_TIMEOUT;
-    }
-    if (st_b != fa::DEV_OK) {
-        t_last_site = site_b;
-        return FA_ERR_TIMEOUT;
+    for (int i = 0; i < 3; ++i) {
+        if (st[i] != fa::DEV_OK) {
+            t_last_site = site[i];
+            return FA_ERR_TIMEOUT;
+        }
     }
     return FA_OK;
 }
@@ -438,7 +442,7 @@ const char* fa_status_string(int status) {
         case FA_OK: return "ok";
         case FA_ERR_NULL: return "a required pointer is NULL";
         case FA_ERR_SHAPE: return "invalid B, H, Sq or Sk (or causal with Sq > Sk)";
-        case FA_ERR_HEADDIM: return "head dimension must be 64 or 128";
+        case FA_ERR_HEADDIM: return "head dimension must be 64, 128 or 256 (64 or 128 for fa_fwd_mask and fa_bwd)";
         case FA_ERR_DTYPE: return "dtype must be FA_FP16 or FA_BF16";
         case FA_ERR_ALIGN: return "q, k, v, o must be 16-byte aligned and lse 4-byte aligned";
         case FA_ERR_ARCH: return "the current device is not sm_100 (B200)";

@@ -105,6 +105,12 @@ inline int64_t num_units(int64_t BH, int64_t S) {
 // Launch the persistent forward kernel on `stream`.  Returns a cudaError_t.
 cudaError_t launch_fwd_sm100(const LaunchArgs& a, cudaStream_t stream);
 
+// Head dimension 256: its own kernel (one 128-row query tile per work unit,
+// 64-key tiles; K/V tensor maps with 64-row boxes), its units and status words.
+cudaError_t launch_fwd_d256_sm100(const LaunchArgs& a, cudaStream_t stream);
+int64_t num_units_d256(int64_t BH, int64_t Sq);
+cudaError_t read_and_clear_status_d256(cudaStream_t stream, int* status, int* site);
+
 // fa_fwd_noalloc: size of its static scratch array (256 bytes; word 0 is the
 // causal unit counter) and the largest number of unit claims the counter
 // serves (work units + CTAs, read back as a non-negative int).

@@ -115,11 +115,14 @@ WORKLOADS = {
 #   [batch, seq_len, heads, head_dim] layout that the gsyq.cn catlass page warns
 #   about, read in place;
 # - prefill_cached: a causal chunk of 4096 new queries over 16384 cached keys
-#   (queries aligned to the last keys), bf16 as the catlass page advises above 4K.
+#   (queries aligned to the last keys), bf16 as the catlass page advises above 4K;
+# - d256_long: head dimension 256, S = 8192, causal, bf16.
 GENERAL_WORKLOADS = {
     "sdxl_xattn": Workload("sdxl_xattn", 2, 10, 4096, 64, "fp16", False, Sk=77),
     "bert_large": Workload("bert_large", 32, 16, 512, 64, "fp16", False, layout="bshd"),
     "prefill_cached": Workload("prefill_cached", 1, 32, 4096, 128, "bf16", True, Sk=16384),
+    # head dimension 256 (the third of the pages' common head dimensions), long context
+    "d256_long": Workload("d256_long", 1, 16, 8192, 256, "bf16", True),
 }
 
 # Parity tolerances (max-abs) on O by dtype, and on the LSE.
