@@ -23,7 +23,8 @@ ctypes.  Function-level citations are in the C file's header:
   Sk keys (cross-attention) and the causal mask aligned to the last Sq keys.
 - ``attn_bwd`` : dQ, dK, dV by the chain rule through the definition (the
   softmax Jacobian), with optional absolute-value error scales.
-- ``attn_fwd_masked`` : the definition with an explicit boolean mask.
+- ``attn_fwd_masked`` / ``attn_bwd_masked`` : the definition with an explicit
+  boolean mask, and its gradients.
 
 Parity pins: every function above is pinned by tests in tests/test_oracle.py and
 tests/test_oracle_general.py (torch SDPA in float64 with an explicit mask, the
@@ -106,6 +107,10 @@ def _load():
                                                ctypes.c_int, ctypes.c_int, ctypes.POINTER(ctypes.c_uint8), i64, i64,
                                                i64, f64p, f64p]
         lib.oracle_attn_fwd_masked.restype = ctypes.c_int
+        lib.oracle_attn_bwd_masked.argtypes = [u16p, u16p, u16p, u16p, i64, i64, i64, i64, i64, ctypes.c_float,
+                                               ctypes.c_int, ctypes.c_int, ctypes.POINTER(ctypes.c_uint8), i64, i64,
+                                               i64, f64p, f64p, f64p, f64p, f64p, f64p]
+        lib.oracle_attn_bwd_masked.restype = ctypes.c_int
         lib.oracle_causal_tile_count.argtypes = [i64, i64, i64, i64p, i64p, i64p]
         lib.oracle_causal_tile_count.restype = None
         lib.oracle_num_threads.argtypes = []
@@ -275,6 +280,32 @@ def attn_bwd(q, k, v, dout, scale: float, causal: bool, dtype, magnitudes: bool 
                              fp(mags[0]), fp(mags[1]), fp(mags[2]))
     if rc != 0:
         raise RuntimeError(f"oracle_attn_bwd failed with {rc}")
+    return (dq, dk, dv) + (mags if magnitudes else ())
+
+
+def attn_bwd_masked(q, k, v, dout, mask, scale: float, causal: bool, dtype, magnitudes: bool = False):
+    """attn_bwd for the masked attention of attn_fwd_masked (mask [B|1, H|1, Sq, Sk])."""
+    lib = _load()
+    qb, kb, vb, gb = _bits(q), _bits(k), _bits(v), _bits(dout)
+    B, H, Sq, D = qb.shape
+    Sk = kb.shape[2]
+    m = np.asarray(mask.cpu().numpy() if hasattr(mask, "cpu") else mask).astype(np.uint8)
+    if m.ndim != 4 or m.shape[2:] != (Sq, Sk) or m.shape[0] not in (1, B) or m.shape[1] not in (1, H):
+        raise ValueError("mask must be [B|1, H|1, Sq, Sk]")
+    m = np.ascontiguousarray(m)
+    sb = 0 if m.shape[0] == 1 else m.shape[1] * Sq * Sk
+    sh = 0 if m.shape[1] == 1 else Sq * Sk
+    dq = np.empty((B, H, Sq, D))
+    dk = np.empty((B, H, Sk, D))
+    dv = np.empty((B, H, Sk, D))
+    mags = tuple(np.empty(a.shape) for a in (dq, dk, dv)) if magnitudes else (None, None, None)
+    fp = lambda a: _ptr(a, ctypes.c_double) if a is not None else None  # noqa: E731
+    rc = lib.oracle_attn_bwd_masked(_ptr(qb, ctypes.c_uint16), _ptr(kb, ctypes.c_uint16), _ptr(vb, ctypes.c_uint16),
+                                    _ptr(gb, ctypes.c_uint16), B, H, Sq, Sk, D, float(np.float32(scale)),
+                                    int(bool(causal)), _dtype_code(dtype), _ptr(m, ctypes.c_uint8), sb, sh, Sk,
+                                    fp(dq), fp(dk), fp(dv), fp(mags[0]), fp(mags[1]), fp(mags[2]))
+    if rc != 0:
+        raise RuntimeError(f"oracle_attn_bwd_masked failed with {rc}")
     return (dq, dk, dv) + (mags if magnitudes else ())
 
 

@@ -558,15 +558,25 @@ int oracle_attn_rows_gen(const uint16_t *q, const uint16_t *k, const uint16_t *v
  * result are each rounded once).
  * Rows with no visible key have zero gradients.
  */
-int oracle_attn_bwd(const uint16_t *q, const uint16_t *k, const uint16_t *v, const uint16_t *dout, int64_t B,
-                    int64_t H, int64_t Sq, int64_t Sk, int64_t D, float scale, int causal, int dtype, double *dq,
-                    double *dk, double *dv, double *mag_dq, double *mag_dk, double *mag_dv)
+/* Key j is visible to query i of head (b, h): the causal rule, and the mask
+ * entry when a mask is given (see oracle_attn_fwd_masked). */
+static int bwd_visible(int64_t i, int64_t j, int64_t Sq, int64_t Sk, int causal, const uint8_t *mrow)
+{
+    if (j >= visible_keys(i, Sq, Sk, causal)) return 0;
+    return mrow ? mrow[j] != 0 : 1;
+}
+
+static int attn_bwd_impl(const uint16_t *q, const uint16_t *k, const uint16_t *v, const uint16_t *dout, int64_t B,
+                         int64_t H, int64_t Sq, int64_t Sk, int64_t D, float scale, int causal, int dtype,
+                         const uint8_t *mask, int64_t mask_sb, int64_t mask_sh, int64_t mask_si, double *dq,
+                         double *dk, double *dv, double *mag_dq, double *mag_dk, double *mag_dv)
 {
     if (B < 0 || H < 0 || Sq < 0 || Sk < 0 || D <= 0) return -2;
     if (dtype != ORACLE_F16 && dtype != ORACLE_BF16) return -4;
     const double sc = (double)scale;
     const size_t szq = (size_t)(Sq * D > 0 ? Sq * D : 1), szk = (size_t)(Sk * D > 0 ? Sk * D : 1);
     for (int64_t bh = 0; bh < B * H; ++bh) {
+        const uint8_t *mhead = mask ? mask + (bh / H) * mask_sb + (bh % H) * mask_sh : NULL;
         double *qh = (double *)malloc(sizeof(double) * szq);
         double *oh = (double *)malloc(sizeof(double) * szq);
         double *kh = (double *)malloc(sizeof(double) * szk);
@@ -595,18 +605,26 @@ int oracle_attn_bwd(const uint16_t *q, const uint16_t *k, const uint16_t *v, con
             double *dprow = (double *)malloc(sizeof(double) * (size_t)(Sk > 0 ? Sk : 1));
 #pragma omp for schedule(dynamic, 8)
             for (int64_t i = 0; i < Sq; ++i) {
+                const uint8_t *mrow = mhead ? mhead + i * mask_si : NULL;
                 const int64_t nj = visible_keys(i, Sq, Sk, causal);
                 const double *qi = qh + i * D, *doi = oh + i * D;
                 for (int64_t d = 0; d < D; ++d) {
                     dqh[i * D + d] = 0.0;
                     if (mqh) mqh[i * D + d] = 0.0;
                 }
-                if (nj <= 0) {
+                int64_t nvis = 0;
+                for (int64_t j = 0; j < nj; ++j) nvis += bwd_visible(i, j, Sq, Sk, causal, mrow);
+                if (nvis == 0) {
                     lse[i] = -INFINITY; dsum[i] = 0.0; asum[i] = 0.0;
                     continue;
                 }
                 double m = -INFINITY;
                 for (int64_t j = 0; j < nj; ++j) {
+                    if (!bwd_visible(i, j, Sq, Sk, causal, mrow)) {
+                        prow[j] = -INFINITY;
+                        dprow[j] = 0.0;
+                        continue;
+                    }
                     double dot = 0.0, dp = 0.0;
                     for (int64_t d = 0; d < D; ++d) {
                         dot += qi[d] * kh[j * D + d];
@@ -658,7 +676,7 @@ int oracle_attn_bwd(const uint16_t *q, const uint16_t *k, const uint16_t *v, con
                 if (mvh) mvh[j * D + d] = 0.0;
             }
             for (int64_t i = 0; i < Sq; ++i) {
-                if (j >= visible_keys(i, Sq, Sk, causal)) continue;
+                if (!bwd_visible(i, j, Sq, Sk, causal, mhead ? mhead + i * mask_si : NULL)) continue;
                 const double *qi = qh + i * D, *doi = oh + i * D;
                 double dot = 0.0, dp = 0.0;
                 for (int64_t d = 0; d < D; ++d) {
@@ -679,6 +697,26 @@ int oracle_attn_bwd(const uint16_t *q, const uint16_t *k, const uint16_t *v, con
         free(qh); free(oh); free(kh); free(vh); free(lse); free(dsum); free(asum);
     }
     return 0;
+}
+
+int oracle_attn_bwd(const uint16_t *q, const uint16_t *k, const uint16_t *v, const uint16_t *dout, int64_t B,
+                    int64_t H, int64_t Sq, int64_t Sk, int64_t D, float scale, int causal, int dtype, double *dq,
+                    double *dk, double *dv, double *mag_dq, double *mag_dk, double *mag_dv)
+{
+    return attn_bwd_impl(q, k, v, dout, B, H, Sq, Sk, D, scale, causal, dtype, NULL, 0, 0, 0, dq, dk, dv, mag_dq,
+                         mag_dk, mag_dv);
+}
+
+/* The gradients of the masked attention of oracle_attn_fwd_masked (same mask
+ * convention); masked pairs contribute nothing, rows with no visible key get no
+ * gradient. */
+int oracle_attn_bwd_masked(const uint16_t *q, const uint16_t *k, const uint16_t *v, const uint16_t *dout,
+                           int64_t B, int64_t H, int64_t Sq, int64_t Sk, int64_t D, float scale, int causal,
+                           int dtype, const uint8_t *mask, int64_t mask_sb, int64_t mask_sh, int64_t mask_si,
+                           double *dq, double *dk, double *dv, double *mag_dq, double *mag_dk, double *mag_dv)
+{
+    return attn_bwd_impl(q, k, v, dout, B, H, Sq, Sk, D, scale, causal, dtype, mask, mask_sb, mask_sh, mask_si, dq,
+                         dk, dv, mag_dq, mag_dk, mag_dv);
 }
 
 /* ------------------------------------------------------------ explicit mask */
