@@ -241,6 +241,20 @@ FA_API int fa_bwd(const void* q, const void* k, const void* v, const void* o, co
                   int Sk, int D, float scale, int causal, int deterministic, int dtype, cudaStream_t stream);
 
 /*
+ * fa_bwd_mask -- fa_bwd for the explicitly masked attention of fa_fwd_mask:
+ * the same mask (device uint8, nonzero = attend; mask_stride = element strides
+ * over b, h and the query row, 0 broadcasting over b or h; all multiples of 16,
+ * row stride >= Sk; 16-byte aligned).  Masked (query, key) pairs contribute no
+ * gradient; rows that saw no key (LSE = -inf) get dQ = 0.  o and lse must come
+ * from fa_fwd_mask with the same mask.  D = 64 or 128; other arguments, modes
+ * and errors as fa_bwd.
+ */
+FA_API int fa_bwd_mask(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                       const float* lse, void* dq, void* dk, void* dv, void* workspace, long long workspace_bytes,
+                       int B, int H, int Sq, int Sk, int D, const void* mask, const long long* mask_stride,
+                       float scale, int causal, int deterministic, int dtype, cudaStream_t stream);
+
+/*
  * fa_check_status -- synchronise `stream`, then report and clear the device
  * status word of the current device: FA_OK, FA_ERR_TIMEOUT if a kernel
  * stopped on a bounded wait since the last call, or FA_ERR_LAUNCH on a CUDA

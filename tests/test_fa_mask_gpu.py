@@ -126,3 +126,73 @@ def test_block_sparse_mask_long_sequence():
     o, lse = run_masked(q, k, v, mask, softmax_scale(D), False)
     o_ref, lse_ref = oracle.attn_fwd_masked(q, k, v, mask, softmax_scale(D), False, "bf16")
     print(compare(o, lse, o_ref, lse_ref, "bf16"))
+
+
+def _dout(shape, dtype, seed):
+    g = torch.Generator().manual_seed(seed)
+    return torch.randn(shape, generator=g).to(torch.float16 if dtype == "fp16" else torch.bfloat16)
+
+
+def run_masked_bwd(q, k, v, dout, mask_bool, scale, causal, deterministic=False):
+    B, H, Sq, D = q.shape
+    Sk = k.shape[2]
+    dq_, dk_, dv_, ddo = (t.cuda() for t in (q, k, v, dout))
+    o = torch.empty_like(dq_)
+    lse = torch.empty((B, H, Sq), dtype=torch.float32, device="cuda")
+    dm, ms = _device_mask(mask_bool)
+    st = torch.cuda.current_stream().cuda_stream
+    dt = fa.FA_BF16 if q.dtype == torch.bfloat16 else fa.FA_FP16
+    assert fa.fa_fwd_mask(dq_.data_ptr(), dk_.data_ptr(), dv_.data_ptr(), o.data_ptr(), lse.data_ptr(), B, H, Sq, Sk,
+                          D, dm.data_ptr(), ms, scale, int(causal), dt, st) == 0
+    gq, gk, gv = (torch.full_like(t, float("nan")) for t in (dq_, dk_, dv_))
+    nb = fa.fa_bwd_workspace_size(B, H, Sq, D)
+    ws = torch.empty(nb, dtype=torch.uint8, device="cuda")
+    rc = fa.fa_bwd_mask(dq_.data_ptr(), dk_.data_ptr(), dv_.data_ptr(), o.data_ptr(), ddo.data_ptr(), lse.data_ptr(),
+                        gq.data_ptr(), gk.data_ptr(), gv.data_ptr(), ws.data_ptr(), nb, B, H, Sq, Sk, D,
+                        dm.data_ptr(), ms, scale, int(causal), int(deterministic), dt, st)
+    assert rc == 0, f"fa_bwd_mask returned {rc}"
+    assert fa.fa_check_status(st) == 0
+    torch.cuda.synchronize()
+    return gq.cpu(), gk.cpu(), gv.cpu()
+
+
+BWD_CASES = [(1, 2, 200, 200, 64, "full"), (2, 2, 129, 300, 128, "bcast_b"), (1, 3, 300, 333, 64, "bcast_both"),
+             (1, 2, 256, 700, 128, "full")]
+
+
+@pytest.mark.parametrize("case", BWD_CASES, ids=lambda c: "x".join(map(str, c)))
+@pytest.mark.parametrize("dtype", ["fp16", "bf16"])
+@pytest.mark.parametrize("causal", [False, True], ids=["full", "causal"])
+def test_masked_bwd_matches_oracle(case, dtype, causal):
+    from gpu_helpers import compare_bwd
+    B, H, Sq, Sk, D, md = case
+    q, k, v = make_cross_inputs(B, H, Sq, Sk, D, dtype, seed=Sq + 2 * Sk)
+    shape = {"full": (B, H, Sq, Sk), "bcast_b": (1, H, Sq, Sk), "bcast_both": (1, 1, Sq, Sk)}[md]
+    mask = _mask(shape, seed=Sq + Sk)
+    if causal:
+        i = torch.arange(Sq)
+        mask[..., i, torch.clamp(i + (Sk - Sq), max=Sk - 1)] = True
+    mask[..., 5, :] = False                      # a row that sees no key
+    dout = _dout(q.shape, dtype, seed=Sq)
+    scale = softmax_scale(D)
+    gq, gk, gv = run_masked_bwd(q, k, v, dout, mask, scale, causal)
+    dq, dk, dv, mq, mk, mv = oracle.attn_bwd_masked(q, k, v, dout, mask, scale, causal, dtype, magnitudes=True)
+    # the subnormal term's absolute sums run over every causally visible pair, masked
+    # ones included: a looser, still valid bound
+    print(compare_bwd((gq, gk, gv), (dq, dk, dv), (mq, mk, mv), dtype, q, k, dout, scale, causal))
+    assert torch.all(gq[:, :, 5] == 0)
+
+
+def test_masked_bwd_deterministic_repeatable():
+    q, k, v = make_inputs(1, 4, 2048, 128, "bf16", seed=31)
+    dout = _dout(q.shape, "bf16", seed=32)
+    i = torch.arange(2048)[:, None]
+    j = torch.arange(2048)[None, :]
+    mask = (((i // 128) == (j // 128)) | (j < 32))[None, None]
+    a = run_masked_bwd(q, k, v, dout, mask, 0.088, False, deterministic=True)
+    b = run_masked_bwd(q, k, v, dout, mask, 0.088, False, deterministic=True)
+    for x, y in zip(a, b):
+        assert torch.equal(x, y)
+    from gpu_helpers import compare_bwd
+    dq, dk, dv, mq, mk, mv = oracle.attn_bwd_masked(q, k, v, dout, mask, 0.088, False, "bf16", magnitudes=True)
+    print(compare_bwd(a, (dq, dk, dv), (mq, mk, mv), "bf16", q, k, dout, 0.088, False))

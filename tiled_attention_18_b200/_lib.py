@@ -55,6 +55,10 @@ SIGNATURES = [
      [ctypes.c_void_p] * 10 + [ctypes.c_longlong, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                ctypes.c_int, ctypes.c_float, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                ctypes.c_void_p]),
+    ("fa_bwd_mask", ctypes.c_int,
+     [ctypes.c_void_p] * 10 + [ctypes.c_longlong, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                               ctypes.c_int, ctypes.c_void_p, _LL3, ctypes.c_float, ctypes.c_int, ctypes.c_int,
+                               ctypes.c_int, ctypes.c_void_p]),
     ("fa_check_status", ctypes.c_int, [ctypes.c_void_p]),
     ("fa_last_timeout_site", ctypes.c_int, []),
     ("fa_selftest_timeout", ctypes.c_int, [ctypes.c_void_p]),
@@ -142,6 +146,16 @@ def fa_bwd(q_ptr: int, k_ptr: int, v_ptr: int, o_ptr: int, do_ptr: int, lse_ptr:
     return int(load().fa_bwd(q_ptr, k_ptr, v_ptr, o_ptr, do_ptr, lse_ptr, dq_ptr, dk_ptr, dv_ptr, ws_ptr,
                              int(ws_bytes), B, H, Sq, Sk, D, float(scale), int(causal), int(deterministic),
                              int(dtype), stream))
+
+
+def fa_bwd_mask(q_ptr: int, k_ptr: int, v_ptr: int, o_ptr: int, do_ptr: int, lse_ptr: int, dq_ptr: int,
+                dk_ptr: int, dv_ptr: int, ws_ptr: int, ws_bytes: int, B: int, H: int, Sq: int, Sk: int, D: int,
+                mask_ptr: int, mask_stride, scale: float, causal: int, deterministic: int, dtype: int,
+                stream: int) -> int:
+    """Raw C call of the masked backward pass (see include/fa.h)."""
+    return int(load().fa_bwd_mask(q_ptr, k_ptr, v_ptr, o_ptr, do_ptr, lse_ptr, dq_ptr, dk_ptr, dv_ptr, ws_ptr,
+                                  int(ws_bytes), B, H, Sq, Sk, D, mask_ptr, _strides(mask_stride), float(scale),
+                                  int(causal), int(deterministic), int(dtype), stream))
 
 
 def fa_check_status(stream: int = 0) -> int:

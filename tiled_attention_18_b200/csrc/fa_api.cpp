@@ -311,9 +311,14 @@ long long fa_bwd_workspace_size(int B, int H, int Sq, int D) {
     return (long long)fa::bwd_workspace_layout((int64_t)B * H, Sq, D).total;
 }
 
-int fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse, void* dq,
-           void* dk, void* dv, void* workspace, long long workspace_bytes, int B, int H, int Sq, int Sk, int D,
-           float scale, int causal, int deterministic, int dtype, cudaStream_t stream) {
+}  // extern "C"
+
+namespace {
+
+int backward(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse, void* dq,
+             void* dk, void* dv, void* workspace, long long workspace_bytes, int B, int H, int Sq, int Sk, int D,
+             float scale, int causal, int deterministic, int dtype, cudaStream_t stream, const uint8_t* mask,
+             const long long* mask_stride) {
     if (B < 0 || H < 0 || Sq < 0 || Sk < 0) return FA_ERR_SHAPE;
     if (D != 64 && D != 128) return FA_ERR_HEADDIM;
     if (dtype != FA_FP16 && dtype != FA_BF16) return FA_ERR_DTYPE;
@@ -337,6 +342,14 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const voi
         return FA_OK;
     }
     if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv) return FA_ERR_NULL;
+    long long ms[3] = {0, 0, 0};
+    if (mask) {
+        for (int i = 0; i < 3; ++i) ms[i] = mask_stride[i];
+        if (ms[0] < 0 || ms[1] < 0 || ms[0] >= MAX_STRIDE || ms[1] >= MAX_STRIDE || ms[2] >= MAX_STRIDE)
+            return FA_ERR_STRIDE;
+        if ((ms[2] < Sk && Sq > 1) || ms[2] % 16 != 0 || ms[0] % 16 != 0 || ms[1] % 16 != 0) return FA_ERR_STRIDE;
+        if (((uintptr_t)mask & 15u) != 0) return FA_ERR_ALIGN;
+    }
     const fa::BwdWorkspace ws = fa::bwd_workspace_layout(BH, Sq, D);
     if (!workspace || ((uintptr_t)workspace & 255u) != 0 || workspace_bytes < ws.total) return FA_ERR_WORKSPACE;
     const uintptr_t a16 = (uintptr_t)q | (uintptr_t)k | (uintptr_t)v | (uintptr_t)o | (uintptr_t)dout |
@@ -349,7 +362,7 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const voi
     if (dev.major != 10 || dev.minor != 0) return FA_ERR_ARCH;
     int cur = 0;
     cudaGetDevice(&cur);
-    const void* ptrs[10] = {q, k, v, o, dout, lse, dq, dk, dv, workspace};
+    const void* ptrs[11] = {q, k, v, o, dout, lse, dq, dk, dv, workspace, mask ? (const void*)mask : q};
     for (const void* p : ptrs) {
         rc = check_device_pointer(p, cur);
         if (rc != FA_OK) return rc;
@@ -376,6 +389,8 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const voi
     a.lse2 = reinterpret_cast<float*>(w + ws.lse2);
     a.delta = reinterpret_cast<float*>(w + ws.delta);
     a.sched = reinterpret_cast<unsigned int*>(w + ws.sched);
+    a.mask = mask;
+    for (int i = 0; i < 3; ++i) a.mask_stride[i] = ms[i];
     a.dq_flags = nullptr;
     if (deterministic) {
         a.dq_flags = reinterpret_cast<int*>(w + ws.flags);
@@ -403,6 +418,27 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const voi
         return FA_ERR_LAUNCH;
     }
     return FA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse, void* dq,
+           void* dk, void* dv, void* workspace, long long workspace_bytes, int B, int H, int Sq, int Sk, int D,
+           float scale, int causal, int deterministic, int dtype, cudaStream_t stream) {
+    return backward(q, k, v, o, dout, lse, dq, dk, dv, workspace, workspace_bytes, B, H, Sq, Sk, D, scale, causal,
+                    deterministic, dtype, stream, nullptr, nullptr);
+}
+
+int fa_bwd_mask(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
+                void* dq, void* dk, void* dv, void* workspace, long long workspace_bytes, int B, int H, int Sq, int Sk,
+                int D, const void* mask, const long long* mask_stride, float scale, int causal, int deterministic,
+                int dtype, cudaStream_t stream) {
+    if (B < 0 || H < 0 || Sq < 0 || Sk < 0) return FA_ERR_SHAPE;
+    if (B > 0 && H > 0 && Sq > 0 && (!mask || !mask_stride)) return FA_ERR_NULL;
+    return backward(q, k, v, o, dout, lse, dq, dk, dv, workspace, workspace_bytes, B, H, Sq, Sk, D, scale, causal,
+                    deterministic, dtype, stream, static_cast<const uint8_t*>(mask), mask_stride);
 }
 
 int fa_check_status(cudaStream_t stream) {

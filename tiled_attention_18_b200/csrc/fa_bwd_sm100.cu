@@ -126,6 +126,8 @@ struct BwdParams {
     int* dq_flags;        // deterministic mode: [BH][flag_steps][4] key tiles added so far per
                           // (head, query step, warp); null: dQ is added with atomics
     int flag_steps;
+    const uint8_t* mask;         // explicit boolean mask (nonzero = attend), or null
+    long long m_sb, m_sh, m_ss;  // its element strides over b, h and the query row
     float scale_log2;     // scale * log2(e)
     float scale;
     unsigned int* sched;  // zeroed unit counter (causal), or null
@@ -227,6 +229,40 @@ __device__ __forceinline__ void pass_turn(int* flag, int next) {
         __threadfence();
         asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(flag), "r"(next) : "memory");
     }
+}
+
+// Explicit mask, transposed for a warp that owns keys key0 .. key0 + 31 (one
+// per lane): returns for this lane's key the bits of queries q0 .. q0 + 31
+// (bit i set = query q0 + i may attend).  Lane i reads query row q0 + i's 32
+// mask bytes (two 16-byte loads; byte loads on the ragged last keys; rows past
+// Sq read the last row), folds them into 32 bits, and 32 ballots transpose the
+// warp's 32 x 32 bit block.
+__device__ __forceinline__ uint32_t mask_col_bits(const uint8_t* mhead, long long ss, int Sq, int Sk, int q0,
+                                                  int key0) {
+    const int lane = threadIdx.x & 31;
+    const uint8_t* r = mhead + (long long)min(q0 + lane, Sq - 1) * ss + key0;
+    uint32_t rowbits = 0u;
+    if (key0 + 32 <= Sk) {
+        const uint4 a = __ldg(reinterpret_cast<const uint4*>(r));
+        const uint4 b = __ldg(reinterpret_cast<const uint4*>(r + 16));
+        const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            // one bit per nonzero byte, gathered into a nibble (byte i -> bit i)
+            const uint32_t t = __vcmpne4(w[e], 0u) & 0x01010101u;
+            rowbits |= ((t * 0x01020408u) >> 24 & 0xFu) << (4 * e);
+        }
+    } else {
+        for (int c = 0; c < Sk - key0; ++c)
+            if (r[c]) rowbits |= 1u << c;
+    }
+    uint32_t col = 0u;
+#pragma unroll
+    for (int kk = 0; kk < 32; ++kk) {
+        const uint32_t bal = __ballot_sync(0xffffffffu, (rowbits >> kk) & 1u);
+        if (lane == kk) col = bal;
+    }
+    return col;
 }
 
 __device__ __forceinline__ void fence_async_smem() {
@@ -444,6 +480,8 @@ __device__ void bwd_ds_role(const BwdParams& p, uint8_t* smem, uint32_t tmem, in
         const int key = U.n * TILE + row;
         const bool key_ok = key < p.Sk;
         const int q_min = p.causal ? key - p.causal_off : 0;  // first query that sees this key
+        const uint8_t* mhead =
+            p.mask ? p.mask + (long long)(U.bh / p.H) * p.m_sb + (long long)(U.bh % p.H) * p.m_sh : nullptr;
         for (int t = 0; t < U.T; ++t) {
             const int m = U.m_lo + t;
             const int st = stage;
@@ -461,9 +499,13 @@ __device__ void bwd_ds_role(const BwdParams& p, uint8_t* smem, uint32_t tmem, in
             tc_fence_after();
             const float* lse2s = reinterpret_cast<const float*>(smem + L::STATS_OFF + st * L::STATS_BYTES);
             const float* dls = lse2s + TILE;
-            const bool need_mask = !key_ok || (m * TILE < q_min);
+            const bool need_mask = !key_ok || (m * TILE < q_min) || p.mask != nullptr;
 #pragma unroll 1
             for (int c = 0; c < 4; ++c) {
+                // explicit mask: this key's bits over the chunk's 32 queries
+                const uint32_t mbits = p.mask ? mask_col_bits(mhead, p.m_ss, p.Sq, p.Sk, m * TILE + 32 * c,
+                                                              U.n * TILE + warp_in_group * 32)
+                                              : 0xffffffffu;
                 uint32_t sr[32], dr[32];
                 tmem_ld32u(tmem + lane_sel + COL_S + 32 * c, sr);
                 tmem_ld32u(tmem + lane_sel + COL_DP + 32 * c, dr);
@@ -477,8 +519,8 @@ __device__ void bwd_ds_role(const BwdParams& p, uint8_t* smem, uint32_t tmem, in
                     float p1 = ex2(fmaf(__uint_as_float(sr[2 * i + 1]), sl2, -l2.y));
                     if (need_mask) {
                         const int q = m * TILE + j;
-                        if (!key_ok || q < q_min) p0 = 0.f;
-                        if (!key_ok || q + 1 < q_min) p1 = 0.f;
+                        if (!key_ok || q < q_min || !((mbits >> (2 * i)) & 1u)) p0 = 0.f;
+                        if (!key_ok || q + 1 < q_min || !((mbits >> (2 * i + 1)) & 1u)) p1 = 0.f;
                     }
                     const float d0 = p0 * (__uint_as_float(dr[2 * i]) - dl.x);
                     const float d1 = p1 * (__uint_as_float(dr[2 * i + 1]) - dl.y);
@@ -926,7 +968,7 @@ __device__ void bwd2_mma(const BwdParams& p, uint8_t* smem, uint32_t tmem, volat
     mbar_drain(bar(L::B_FIN), 0u);
 }
 
-template <bool BF16>
+template <bool BF16, bool MASK>
 __device__ void bwd2_ds_role(const BwdParams& p, uint8_t* smem, uint32_t tmem, int warp_in_group, int c,
                              volatile uint32_t* abort_flag) {
     using L = Bwd2Smem;
@@ -948,6 +990,8 @@ __device__ void bwd2_ds_role(const BwdParams& p, uint8_t* smem, uint32_t tmem, i
         const int key = U.n * TILE + row;
         const bool key_ok = key < p.Sk;
         const int q_min = p.causal ? key - p.causal_off : 0;
+        const uint8_t* mhead =
+            MASK ? p.mask + (long long)(U.bh / p.H) * p.m_sb + (long long)(U.bh % p.H) * p.m_sh : nullptr;
         for (int t = 0; t < U.T; ++t, ++g) {
             const int m = U.m_lo + t;
             const uint32_t b = g & 1u;
@@ -962,7 +1006,11 @@ __device__ void bwd2_ds_role(const BwdParams& p, uint8_t* smem, uint32_t tmem, i
             tc_fence_after();
             const float* lse2s = reinterpret_cast<const float*>(smem + L::STATS_OFF + st * L::STATS_BYTES);
             const float* dls = lse2s + QM;
-            const bool need_mask = !key_ok || (m * QM + 32 * c < q_min);
+            const bool need_mask = !key_ok || (m * QM + 32 * c < q_min) || MASK;
+            // explicit mask: this key's bits over the 32 queries of this warpgroup
+            uint32_t mbits = 0xffffffffu;
+            if constexpr (MASK)
+                mbits = mask_col_bits(mhead, p.m_ss, p.Sq, p.Sk, m * QM + 32 * c, U.n * TILE + warp_in_group * 32);
             uint8_t* ds_row = smem + L::DS_OFF + b * L::DS_BYTES + (row >> 3) * 1024 + (row & 7) * 128;
             {
                 uint32_t sr[32], dr[32];
@@ -978,8 +1026,8 @@ __device__ void bwd2_ds_role(const BwdParams& p, uint8_t* smem, uint32_t tmem, i
                     float p1 = ex2(fmaf(__uint_as_float(sr[2 * i + 1]), sl2, -l2.y));
                     if (need_mask) {
                         const int q = m * QM + j;
-                        if (!key_ok || q < q_min) p0 = 0.f;
-                        if (!key_ok || q + 1 < q_min) p1 = 0.f;
+                        if (!key_ok || q < q_min || !((mbits >> (2 * i)) & 1u)) p0 = 0.f;
+                        if (!key_ok || q + 1 < q_min || !((mbits >> (2 * i + 1)) & 1u)) p1 = 0.f;
                     }
                     pk[i] = pack2<BF16>(p0, p1);
                     dk[i] = pack2<BF16>(p0 * (__uint_as_float(dr[2 * i]) - dl.x),
@@ -1108,7 +1156,7 @@ __device__ void bwd2_out_role(const BwdParams& p, uint8_t* smem, uint32_t tmem, 
     }
 }
 
-template <bool BF16>
+template <bool BF16, bool MASK>
 __global__ void __launch_bounds__(BWD2_THREADS, 1) fa_bwd_kernel_d128(const __grid_constant__ BwdParams p) {
     using L = Bwd2Smem;
     extern __shared__ uint8_t smem_raw[];
@@ -1153,7 +1201,7 @@ __global__ void __launch_bounds__(BWD2_THREADS, 1) fa_bwd_kernel_d128(const __gr
         if (warp == BW_MMA && lane == 0) bwd2_mma<BF16>(p, smem, tmem, abort_flag);
     } else if (wg == 1 || wg == 3) {
         setmaxnreg_inc<REG2_DS>();
-        bwd2_ds_role<BF16>(p, smem, tmem, warp & 3, wg == 1 ? 0 : 1, abort_flag);
+        bwd2_ds_role<BF16, MASK>(p, smem, tmem, warp & 3, wg == 1 ? 0 : 1, abort_flag);
     } else {
         setmaxnreg_dec<REG2_OUT>();
         bwd2_out_role<BF16>(p, smem, tmem, warp & 3, abort_flag);
@@ -1205,7 +1253,9 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const uint16_t* __restric
 #pragma unroll
     for (int i = 0; i < PER_LANE; ++i) dq_acc[e0 + i] = 0.f;
     if (lane == 0) {
-        lse2[bh * Sq_pad + row] = lse[bh * (size_t)Sq + row] * 1.4426950408889634f;
+        // a row that saw no key (LSE = -inf) gets +inf, i.e. weights 0
+        const float lv = lse[bh * (size_t)Sq + row];
+        lse2[bh * Sq_pad + row] = (lv == -INFINITY) ? __int_as_float(0x7f800000) : lv * 1.4426950408889634f;
         delta[bh * Sq_pad + row] = acc;
     }
 }
@@ -1238,7 +1288,7 @@ cudaError_t launch_bwd_impl(const BwdLaunchArgs& a, cudaStream_t stream) {
     {
         // D = 128 runs the 64-row-step kernel (its Q/dO maps have 64-row boxes)
         void (*kern)(const BwdParams);
-        if constexpr (D == 128) kern = fa_bwd_kernel_d128<BF16>;
+        if constexpr (D == 128) kern = a.mask ? fa_bwd_kernel_d128<BF16, true> : fa_bwd_kernel_d128<BF16, false>;
         else kern = fa_bwd_kernel<D, BF16>;
         const int alloc = (D == 128) ? Bwd2Smem::ALLOC : BwdSmem<64>::ALLOC;
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, alloc);
@@ -1275,6 +1325,10 @@ cudaError_t launch_bwd_impl(const BwdLaunchArgs& a, cudaStream_t stream) {
         // and in deterministic mode (the order of dQ additions follows the claims)
         p.sched = (a.causal || a.dq_flags) ? a.sched : nullptr;
         p.dq_flags = a.dq_flags;
+        p.mask = a.mask;
+        p.m_sb = a.mask_stride[0];
+        p.m_sh = a.mask_stride[1];
+        p.m_ss = a.mask_stride[2];
         p.flag_steps = (D == 128) ? (a.Sq + QM - 1) / QM : n_mtiles;
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3((unsigned)a.grid, 1, 1);

@@ -61,6 +61,8 @@ struct BwdLaunchArgs {
     float* delta;           // workspace: [B*H][Sq_pad] fp32
     unsigned int* sched;    // workspace: unit counter
     int* dq_flags;          // workspace: deterministic-mode turn counters, or null (atomic mode)
+    const uint8_t* mask;    // explicit boolean mask or null
+    long long mask_stride[3];
     int B;
     int H;
     int Sq;
