@@ -14,7 +14,7 @@ from ._lib import (FA_BF16, FA_FP16, FaError, fa_bwd, fa_bwd_mask, fa_bwd_worksp
 
 __all__ = [
     "FA_BF16", "FA_FP16", "FaError", "fa_bwd", "fa_bwd_mask", "fa_bwd_workspace_size", "fa_check_status", "fa_fwd", "fa_fwd_ex",
-    "fa_fwd_mask",
+    "fa_fwd_mask", "flash_attention_backward",
     "fa_fwd_noalloc", "fa_last_timeout_site",
     "fa_num_units", "fa_selftest_timeout", "fa_status_string", "fa_version", "flash_attention_forward", "load",
 ]
@@ -77,3 +77,38 @@ def flash_attention_forward(q, k, v, scale: float, causal: bool = False, out=Non
     if rc != 0:
         raise FaError(rc)
     return out, lse
+
+
+def flash_attention_backward(q, k, v, o, lse, dout, scale: float, causal: bool = False, deterministic: bool = False,
+                             dq=None, dk=None, dv=None, workspace=None, stream=None):
+    """dQ, dK, dV for contiguous BHSD CUDA tensors (q, o, dout [B, H, Sq, D];
+    k, v [B, H, Sk, D]; lse [B, H, Sq] fp32 from the forward call).  The
+    workspace (fa_bwd_workspace_size bytes) is allocated with torch unless
+    given.  Launches on ``stream`` (default: torch's current stream) and
+    returns without synchronising."""
+    import torch
+    B, H, Sq, D = q.shape
+    Sk = k.shape[2]
+    for name, t in (("q", q), ("k", k), ("v", v), ("o", o), ("dout", dout)):
+        if not (t.is_cuda and t.is_contiguous() and t.dtype == q.dtype):
+            raise ValueError(f"{name} must be a contiguous CUDA tensor of q's dtype")
+    if o.shape != q.shape or dout.shape != q.shape or k.shape != (B, H, Sk, D) or v.shape != k.shape:
+        raise ValueError("q, o, dout must be [B, H, Sq, D] and k, v [B, H, Sk, D]")
+    if lse.shape != (B, H, Sq) or lse.dtype != torch.float32 or not lse.is_contiguous():
+        raise ValueError("lse must be a contiguous float32 [B, H, Sq] tensor")
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    nbytes = fa_bwd_workspace_size(B, H, Sq, D)
+    if nbytes < 0:
+        raise FaError(nbytes, "fa_bwd_workspace_size")
+    if workspace is None:
+        workspace = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=q.device)
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device)
+    rc = fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), dout.data_ptr(), lse.data_ptr(),
+                dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), workspace.data_ptr(), workspace.numel(), B, H, Sq, Sk, D,
+                float(scale), int(bool(causal)), int(bool(deterministic)), _dtype_code(q), int(stream.cuda_stream))
+    if rc != 0:
+        raise FaError(rc, "fa_bwd")
+    return dq, dk, dv
