@@ -255,6 +255,33 @@ FA_API int fa_bwd_mask(const void* q, const void* k, const void* v, const void* 
                        float scale, int causal, int deterministic, int dtype, cudaStream_t stream);
 
 /*
+ * fa_merge_partial -- fold a partial attention result into a running one by
+ * log-sum-exp weights.  For two disjoint key sets with results (O_a, L_a) and
+ * (O_b, L_b): L = log(e^L_a + e^L_b), O = e^(L_a - L) O_a + e^(L_b - L) O_b, the
+ * attention over their union.  This combines the blocks of a sequence split
+ * across devices ("FlashAttention-2 在昇腾 NPU 上如何做到 3 倍加速？", section
+ * 6.4) and is the rescaling the online softmax applies tile by tile (section
+ * 2.2).
+ *
+ * o_acc   : device, [rows][D] fp32, the running O; updated in place.
+ * lse_acc : device, [rows] fp32 (natural log), the running LSE; updated.  Start
+ *           with -inf (no key yet); a row whose sides are both -inf is left
+ *           unchanged.
+ * o_part  : device, [rows][D] 16-bit (dtype), a partial O, e.g. from fa_fwd_ex.
+ * lse_part: device, [rows] fp32, its LSE (-inf: the partial saw no key).
+ * rows, D : contiguous rows of D values (1 <= D <= 1024).
+ * Asynchronous on stream; errors as fa_fwd (argument checks first).
+ */
+FA_API int fa_merge_partial(float* o_acc, float* lse_acc, const void* o_part, const float* lse_part, long long rows,
+                            int D, int dtype, cudaStream_t stream);
+
+/*
+ * fa_merge_finalize -- round n fp32 values (a running O) to the 16-bit dtype
+ * (nearest even) into o.  Device pointers; asynchronous on stream.
+ */
+FA_API int fa_merge_finalize(const float* o_acc, void* o, long long n, int dtype, cudaStream_t stream);
+
+/*
  * fa_check_status -- synchronise `stream`, then report and clear the device
  * status word of the current device: FA_OK, FA_ERR_TIMEOUT if a kernel
  * stopped on a bounded wait since the last call, or FA_ERR_LAUNCH on a CUDA

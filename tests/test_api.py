@@ -210,3 +210,15 @@ def test_fa_fwd_mask_invalid_arguments(lib, args, code):
     st = fa.fa_fwd_mask(a["q"], a["k"], a["v"], a["o"], a["lse"], a["B"], a["H"], a["Sq"], a["Sk"], a["D"], a["mask"],
                         a["ms"], a["scale"], a["causal"], a["dtype"], 0)
     assert st == code
+
+
+def test_merge_entries_reject_bad_arguments(lib):
+    assert fa.fa_merge_partial(A, A, A, A, -1, 64, 1, 0) == _lib.FA_ERR_SHAPE
+    assert fa.fa_merge_partial(A, A, A, A, 10, 0, 1, 0) == _lib.FA_ERR_HEADDIM
+    assert fa.fa_merge_partial(A, A, A, A, 10, 64, 5, 0) == _lib.FA_ERR_DTYPE
+    assert fa.fa_merge_partial(0, A, A, A, 10, 64, 1, 0) == _lib.FA_ERR_NULL
+    assert fa.fa_merge_partial(A + 2, A, A, A, 10, 64, 1, 0) == _lib.FA_ERR_ALIGN
+    assert fa.fa_merge_partial(0, 0, 0, 0, 0, 64, 1, 0) == _lib.FA_OK
+    assert fa.fa_merge_finalize(A, A, -1, 1, 0) == _lib.FA_ERR_SHAPE
+    assert fa.fa_merge_finalize(A, A + 1, 10, 1, 0) == _lib.FA_ERR_ALIGN
+    assert fa.fa_merge_finalize(0, 0, 0, 1, 0) == _lib.FA_OK

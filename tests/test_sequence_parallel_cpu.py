@@ -1,0 +1,91 @@
+"""Multi-rank sequence-parallel attention on CPU: gloo ranks (spawned
+processes) run the ring and all-gather schedules of
+tiled_attention_18_b200.sequence_parallel with an fp64 oracle stand-in for the
+kernels; the gathered result must equal full attention."""
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+from tiled_attention_18_b200.sequence_parallel import (allgather_attention_forward, ring_attention_forward,
+                                                       ring_schedule)
+
+
+class OracleOps:
+    """Partial attention by the fp64 oracle, fp64 LSE merge (test stand-in)."""
+
+    def __init__(self, scale, dtype):
+        self.scale, self.dtype = scale, dtype
+
+    def partial(self, q, k, v, causal):
+        import oracle
+        o, lse = oracle.attn_fwd_gen(q, k, v, self.scale, causal, self.dtype)
+        return torch.from_numpy(o), torch.from_numpy(lse)
+
+    def init(self, q):
+        B, H, S, D = q.shape
+        return [torch.zeros((B, H, S, D), dtype=torch.float64), torch.full((B, H, S), float("-inf"),
+                                                                           dtype=torch.float64)]
+
+    def merge(self, state, o_p, lse_p):
+        o, lse = state
+        m = torch.maximum(lse, lse_p)
+        wa = torch.where(torch.isneginf(lse), torch.zeros_like(lse), torch.exp(lse - m))
+        wb = torch.where(torch.isneginf(lse_p), torch.zeros_like(lse_p), torch.exp(lse_p - m))
+        state[0] = (wa[..., None] * o + wb[..., None] * o_p) / (wa + wb)[..., None]
+        state[1] = m + torch.log(wa + wb)
+
+    def finalize(self, state):
+        return state[0], state[1]
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, mode, causal, out_dir):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        from tiled_attention_18_b200.workloads import make_inputs
+        B, H, c, D = 1, 2, 24, 16
+        q, k, v = make_inputs(B, H, world * c, D, "fp16", seed=5)
+        sl = slice(rank * c, (rank + 1) * c)
+        ops = OracleOps(0.25, "fp16")
+        fn = ring_attention_forward if mode == "ring" else allgather_attention_forward
+        o, lse = fn(q[:, :, sl].contiguous(), k[:, :, sl].contiguous(), v[:, :, sl].contiguous(), 0.25, causal,
+                    ops=ops)
+        np.save(os.path.join(out_dir, f"o{rank}.npy"), o.numpy())
+        np.save(os.path.join(out_dir, f"l{rank}.npy"), lse.numpy())
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 3])
+@pytest.mark.parametrize("mode", ["ring", "allgather"])
+@pytest.mark.parametrize("causal", [False, True])
+def test_sequence_parallel_ranks_equal_full_attention(tmp_path, world, mode, causal):
+    import oracle
+    from tiled_attention_18_b200.workloads import make_inputs
+    mp.spawn(_worker, args=(world, _free_port(), mode, causal, str(tmp_path)), nprocs=world, join=True)
+    B, H, c, D = 1, 2, 24, 16
+    q, k, v = make_inputs(B, H, world * c, D, "fp16", seed=5)
+    o_ref, lse_ref = oracle.attn_fwd(q, k, v, 0.25, causal, "fp16")
+    o = np.concatenate([np.load(tmp_path / f"o{r}.npy") for r in range(world)], axis=2)
+    lse = np.concatenate([np.load(tmp_path / f"l{r}.npy") for r in range(world)], axis=2)
+    assert np.max(np.abs(o - o_ref)) <= 1e-12
+    assert np.max(np.abs(lse - lse_ref)) <= 1e-12
+
+
+def test_ring_schedule():
+    assert ring_schedule(0, 3, False) == [(0, "full"), (2, "full"), (1, "full")]
+    assert ring_schedule(2, 3, True) == [(2, "causal"), (1, "full"), (0, "full")]
+    assert ring_schedule(0, 3, True) == [(0, "causal"), (2, "skip"), (1, "skip")]
+    assert ring_schedule(1, 4, True) == [(1, "causal"), (0, "full"), (3, "skip"), (2, "skip")]

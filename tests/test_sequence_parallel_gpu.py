@@ -1,0 +1,77 @@
+"""Sequence-parallel attention through the library's kernels on one GPU: the
+ring and all-gather schedules of every rank of a W-rank group are run in one
+process (the K/V block each rank would receive is handed to it directly), and
+the concatenated result is compared with the fp64 oracle's full attention.
+Covers fa_merge_partial / fa_merge_finalize and the block-causal logic; the
+P2P/all-gather communication itself is covered by the gloo tests."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import tiled_attention_18_b200 as fa
+from tiled_attention_18_b200.sequence_parallel import CudaOps, allgather_attention_forward, ring_attention_forward
+from tiled_attention_18_b200.workloads import make_inputs, softmax_scale
+
+from gpu_helpers import compare
+
+pytestmark = pytest.mark.gpu
+
+
+def _run_all_ranks(mode, q, k, v, world, scale, causal):
+    B, H, S, D = q.shape
+    c = S // world
+    dq, dk, dv = (t.cuda() for t in (q, k, v))
+    chunks = [(dq[:, :, r * c:(r + 1) * c].contiguous(), dk[:, :, r * c:(r + 1) * c].contiguous(),
+               dv[:, :, r * c:(r + 1) * c].contiguous()) for r in range(world)]
+    kv_blocks = [torch.stack([ck, cv]) for (_, ck, cv) in chunks]
+    outs, lses = [], []
+    for r in range(world):
+        qr, kr, vr = chunks[r]
+        ops = CudaOps(scale)
+        if mode == "ring":
+            # at step s the rank holds rank (r - s)'s block and receives rank (r - s - 1)'s
+            o, lse = ring_attention_forward(qr, kr, vr, scale, causal, ops=ops, rank=r, world=world,
+                                            exchange=lambda s, kv, r=r: (None, kv_blocks[(r - s - 1) % world]))
+        else:
+            o, lse = allgather_attention_forward(qr, kr, vr, scale, causal, ops=ops, rank=r, world=world,
+                                                 gather=lambda kv: torch.stack(kv_blocks))
+        outs.append(o)
+        lses.append(lse)
+    st = torch.cuda.current_stream().cuda_stream
+    assert fa.fa_check_status(st) == 0
+    torch.cuda.synchronize()
+    return torch.cat(outs, dim=2).cpu(), torch.cat(lses, dim=2).cpu()
+
+
+@pytest.mark.parametrize("mode", ["ring", "allgather"])
+@pytest.mark.parametrize("world", [2, 4])
+@pytest.mark.parametrize("causal", [False, True], ids=["full", "causal"])
+@pytest.mark.parametrize("dtype,D", [("bf16", 128), ("fp16", 64)])
+def test_sequence_parallel_schedules_match_full_attention(mode, world, causal, dtype, D):
+    q, k, v = make_inputs(1, 4, 1024, D, dtype, seed=world + D)
+    scale = softmax_scale(D)
+    o, lse = _run_all_ranks(mode, q, k, v, world, scale, causal)
+    o_ref, lse_ref = oracle.attn_fwd(q, k, v, scale, causal, dtype)
+    print(mode, world, causal, dtype, compare(o, lse, o_ref, lse_ref, dtype))
+
+
+def test_merge_partial_matches_union_and_empty_sides():
+    """Two disjoint key halves merged equal attention over all keys; an empty
+    partial (LSE = -inf) leaves the running result unchanged."""
+    q, k, v = make_inputs(2, 3, 384, 128, "bf16", seed=7)
+    dq, dk, dv = (t.cuda() for t in (q, k, v))
+    ops = CudaOps(0.09)
+    state = ops.init(dq)
+    for lo, hi in ((0, 200), (200, 384)):
+        o_p, lse_p = fa.flash_attention_forward(dq, dk[:, :, lo:hi].contiguous(), dv[:, :, lo:hi].contiguous(), 0.09)
+        ops.merge(state, o_p, lse_p)
+    before = state[0].clone(), state[1].clone()
+    empty_o = torch.zeros_like(dq)
+    empty_l = torch.full(dq.shape[:3], float("-inf"), device="cuda")
+    ops.merge(state, empty_o, empty_l)
+    assert torch.equal(state[0], before[0]) and torch.equal(state[1], before[1])
+    o, lse = ops.finalize(state)
+    torch.cuda.synchronize()
+    o_ref, lse_ref = oracle.attn_fwd(q, k, v, 0.09, False, "bf16")
+    compare(o.cpu(), lse.cpu(), o_ref, lse_ref, "bf16")

@@ -59,6 +59,10 @@ SIGNATURES = [
      [ctypes.c_void_p] * 10 + [ctypes.c_longlong, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                ctypes.c_int, ctypes.c_void_p, _LL3, ctypes.c_float, ctypes.c_int, ctypes.c_int,
                                ctypes.c_int, ctypes.c_void_p]),
+    ("fa_merge_partial", ctypes.c_int,
+     [ctypes.c_void_p] * 4 + [ctypes.c_longlong, ctypes.c_int, ctypes.c_int, ctypes.c_void_p]),
+    ("fa_merge_finalize", ctypes.c_int,
+     [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_longlong, ctypes.c_int, ctypes.c_void_p]),
     ("fa_check_status", ctypes.c_int, [ctypes.c_void_p]),
     ("fa_last_timeout_site", ctypes.c_int, []),
     ("fa_selftest_timeout", ctypes.c_int, [ctypes.c_void_p]),
@@ -156,6 +160,16 @@ def fa_bwd_mask(q_ptr: int, k_ptr: int, v_ptr: int, o_ptr: int, do_ptr: int, lse
     return int(load().fa_bwd_mask(q_ptr, k_ptr, v_ptr, o_ptr, do_ptr, lse_ptr, dq_ptr, dk_ptr, dv_ptr, ws_ptr,
                                   int(ws_bytes), B, H, Sq, Sk, D, mask_ptr, _strides(mask_stride), float(scale),
                                   int(causal), int(deterministic), int(dtype), stream))
+
+
+def fa_merge_partial(o_acc_ptr: int, lse_acc_ptr: int, o_part_ptr: int, lse_part_ptr: int, rows: int, D: int,
+                     dtype: int, stream: int) -> int:
+    return int(load().fa_merge_partial(o_acc_ptr, lse_acc_ptr, o_part_ptr, lse_part_ptr, int(rows), D, int(dtype),
+                                       stream))
+
+
+def fa_merge_finalize(o_acc_ptr: int, o_ptr: int, n: int, dtype: int, stream: int) -> int:
+    return int(load().fa_merge_finalize(o_acc_ptr, o_ptr, int(n), int(dtype), stream))
 
 
 def fa_check_status(stream: int = 0) -> int:

@@ -23,7 +23,8 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libfa.so")
 SOURCES = [os.path.join(CSRC, "fa_fwd_sm100.cu"), os.path.join(CSRC, "fa_fwd_d256_sm100.cu"),
-           os.path.join(CSRC, "fa_bwd_sm100.cu"), os.path.join(CSRC, "fa_api.cpp")]
+           os.path.join(CSRC, "fa_bwd_sm100.cu"), os.path.join(CSRC, "fa_merge_sm100.cu"),
+           os.path.join(CSRC, "fa_api.cpp")]
 HEADERS = [os.path.join(CSRC, "fa_internal.h"), os.path.join(CSRC, "sm100_helpers.cuh"),
            os.path.join(INCLUDE, "fa.h")]
 

@@ -441,6 +441,53 @@ int fa_bwd_mask(const void* q, const void* k, const void* v, const void* o, cons
                     deterministic, dtype, stream, static_cast<const uint8_t*>(mask), mask_stride);
 }
 
+int fa_merge_partial(float* o_acc, float* lse_acc, const void* o_part, const float* lse_part, long long rows, int D,
+                     int dtype, cudaStream_t stream) {
+    if (rows < 0) return FA_ERR_SHAPE;
+    if (D < 1 || D > 1024) return FA_ERR_HEADDIM;
+    if (dtype != FA_FP16 && dtype != FA_BF16) return FA_ERR_DTYPE;
+    if (rows == 0) return FA_OK;
+    if (!o_acc || !lse_acc || !o_part || !lse_part) return FA_ERR_NULL;
+    if ((((uintptr_t)o_acc | (uintptr_t)lse_acc | (uintptr_t)lse_part) & 3u) != 0 || ((uintptr_t)o_part & 1u) != 0)
+        return FA_ERR_ALIGN;
+    int cur = 0;
+    if (cudaGetDevice(&cur) != cudaSuccess) {
+        cudaGetLastError();
+        return FA_ERR_LAUNCH;
+    }
+    const void* ptrs[4] = {o_acc, lse_acc, o_part, lse_part};
+    for (const void* p : ptrs) {
+        const int rc = check_device_pointer(p, cur);
+        if (rc != FA_OK) return rc;
+    }
+    if (fa::launch_merge_partial(o_acc, lse_acc, o_part, lse_part, rows, D, dtype, stream) != cudaSuccess) {
+        cudaGetLastError();
+        return FA_ERR_LAUNCH;
+    }
+    return FA_OK;
+}
+
+int fa_merge_finalize(const float* o_acc, void* o, long long n, int dtype, cudaStream_t stream) {
+    if (n < 0) return FA_ERR_SHAPE;
+    if (dtype != FA_FP16 && dtype != FA_BF16) return FA_ERR_DTYPE;
+    if (n == 0) return FA_OK;
+    if (!o_acc || !o) return FA_ERR_NULL;
+    if (((uintptr_t)o_acc & 3u) != 0 || ((uintptr_t)o & 1u) != 0) return FA_ERR_ALIGN;
+    int cur = 0;
+    if (cudaGetDevice(&cur) != cudaSuccess) {
+        cudaGetLastError();
+        return FA_ERR_LAUNCH;
+    }
+    int rc = check_device_pointer(o_acc, cur);
+    if (rc == FA_OK) rc = check_device_pointer(o, cur);
+    if (rc != FA_OK) return rc;
+    if (fa::launch_merge_finalize(o_acc, o, n, dtype, stream) != cudaSuccess) {
+        cudaGetLastError();
+        return FA_ERR_LAUNCH;
+    }
+    return FA_OK;
+}
+
 int fa_check_status(cudaStream_t stream) {
     // one status word per kernel translation unit; all are read and cleared
     int st[3] = {0, 0, 0}, site[3] = {0, 0, 0};

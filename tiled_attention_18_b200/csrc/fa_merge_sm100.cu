@@ -1,0 +1,90 @@
+// fa_merge_sm100.cu -- merging partial attention results by their log-sum-exp
+// (declared in include/fa.h: fa_merge_partial, fa_merge_finalize).
+//
+// Attention over a key set split into blocks is the LSE-weighted combination
+// of the attention over each block: with (O_a, L_a) and (O_b, L_b) for two
+// disjoint key sets, L = log(e^L_a + e^L_b) and O = (e^(L_a - L) O_a +
+// e^(L_b - L) O_b).  This is what lets the sequence be split across devices
+// ("FlashAttention-2 在昇腾 NPU 上如何做到 3 倍加速？", section 6.4: each device
+// computes the attention of its part of the sequence while K/V move between
+// devices) and is the same rescaling the online softmax applies tile by tile
+// inside one kernel (section 2.2).
+//
+// One warp per row, its lanes striding over the row's D values.  The running
+// result is fp32 (o_acc, lse_acc); a partial is 16-bit O with fp32 LSE, as
+// fa_fwd_ex produces them.  An empty side (LSE = -inf) contributes nothing.
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "fa_internal.h"
+
+namespace fa {
+namespace {
+
+template <bool BF16>
+__device__ __forceinline__ float to_f32(uint16_t x) {
+    if constexpr (BF16) return __bfloat162float(__ushort_as_bfloat16(x));
+    else return __half2float(__ushort_as_half(x));
+}
+
+template <bool BF16>
+__device__ __forceinline__ uint16_t from_f32(float x) {
+    if constexpr (BF16) return __bfloat16_as_ushort(__float2bfloat16_rn(x));
+    else return __half_as_ushort(__float2half_rn(x));
+}
+
+template <bool BF16>
+__global__ void __launch_bounds__(256) merge_kernel(float* __restrict__ o_acc, float* __restrict__ lse_acc,
+                                                    const uint16_t* __restrict__ o_part,
+                                                    const float* __restrict__ lse_part, long long rows, int D) {
+    const long long row = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (row >= rows) return;
+    const float la = lse_acc[row], lb = lse_part[row];
+    const float m = fmaxf(la, lb);
+    if (m == -INFINITY) return;  // neither side saw a key
+    const float wa = (la == -INFINITY) ? 0.f : expf(la - m);
+    const float wb = (lb == -INFINITY) ? 0.f : expf(lb - m);
+    const float inv = 1.f / (wa + wb);
+    const float ca = wa * inv, cb = wb * inv;
+    float* oa = o_acc + row * D;
+    const uint16_t* ob = o_part + row * D;
+    for (int d = lane; d < D; d += 32) oa[d] = ca * oa[d] + cb * to_f32<BF16>(ob[d]);
+    __syncwarp();
+    if (lane == 0) lse_acc[row] = m + logf(wa + wb);
+}
+
+template <bool BF16>
+__global__ void __launch_bounds__(256) finalize_kernel(const float* __restrict__ o_acc, uint16_t* __restrict__ o,
+                                                       long long n) {
+    for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x)
+        o[i] = from_f32<BF16>(o_acc[i]);
+}
+
+}  // namespace
+
+cudaError_t launch_merge_partial(float* o_acc, float* lse_acc, const void* o_part, const float* lse_part,
+                                 long long rows, int D, int dtype, cudaStream_t stream) {
+    const unsigned blocks = (unsigned)((rows + 7) / 8);
+    if (dtype == 1)
+        merge_kernel<true><<<blocks, 256, 0, stream>>>(o_acc, lse_acc, static_cast<const uint16_t*>(o_part), lse_part,
+                                                       rows, D);
+    else
+        merge_kernel<false><<<blocks, 256, 0, stream>>>(o_acc, lse_acc, static_cast<const uint16_t*>(o_part),
+                                                        lse_part, rows, D);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_merge_finalize(const float* o_acc, void* o, long long n, int dtype, cudaStream_t stream) {
+    const long long want = (n + 255) / 256;
+    const unsigned blocks = (unsigned)(want < 148 * 32 ? want : 148 * 32);
+    if (dtype == 1)
+        finalize_kernel<true><<<blocks, 256, 0, stream>>>(o_acc, static_cast<uint16_t*>(o), n);
+    else
+        finalize_kernel<false><<<blocks, 256, 0, stream>>>(o_acc, static_cast<uint16_t*>(o), n);
+    return cudaGetLastError();
+}
+
+}  // namespace fa

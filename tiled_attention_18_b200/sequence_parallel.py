@@ -1,0 +1,180 @@
+"""Sequence-parallel attention forward across the ranks of a torch.distributed group.
+
+The sequence is split into equal contiguous chunks, one per rank in rank
+order; every rank holds its chunk of Q, K and V ([B, H, c, D]) and computes
+the attention of its queries over the whole sequence, the K/V it lacks coming
+from the other ranks ("FlashAttention-2 在昇腾 NPU 上如何做到 3 倍加速？",
+section 6.4: each device computes the attention of its part of the sequence,
+K/V synchronised between devices by collective communication).  Two ways:
+
+- ``allgather_attention_forward``: one all-gather of K and V, then one
+  ``fa_fwd_ex`` over the keys this rank's queries can see (all of them, or,
+  with the causal mask, the first (rank + 1) * c: bottom-right alignment puts
+  query i of the chunk at global position rank * c + i).  Memory: the whole
+  sequence's K/V on every rank.
+- ``ring_attention_forward``: the K/V blocks travel around the ring (P2P to
+  rank + 1, from rank - 1) while each rank computes the attention of its
+  queries over the block it holds and folds the partial (O, LSE) into a
+  running fp32 result with ``fa_merge_partial`` (the log-sum-exp merge).
+  With the causal mask a rank skips the blocks that come after its own and
+  uses the causal kernel on its own block.  Memory: two K/V blocks.
+
+Every step of the attention runs in the library's kernels; this module only
+orders the launches and the communication.  The ``ops`` and ``exchange``
+parameters exist so that tests can drive the same schedule with stand-ins
+(CPU ranks over gloo, or all ranks in one process on one GPU).
+"""
+from __future__ import annotations
+
+from typing import Callable, List, Optional, Tuple
+
+
+def ring_schedule(rank: int, world: int, causal: bool) -> List[Tuple[int, str]]:
+    """(source rank, mode) for ring steps s = 0 .. world - 1: at step s this rank
+    holds the K/V block of rank (rank - s) mod world; mode is "full", "causal"
+    (its own block under the mask) or "skip" (a block after its own under the
+    mask)."""
+    out = []
+    for s in range(world):
+        src = (rank - s) % world
+        if not causal:
+            out.append((src, "full"))
+        elif src == rank:
+            out.append((src, "causal"))
+        elif src < rank:
+            out.append((src, "full"))
+        else:
+            out.append((src, "skip"))
+    return out
+
+
+class CudaOps:
+    """The library's kernels: fa_fwd_ex for a partial, fa_merge_partial /
+    fa_merge_finalize for the running result (fp32 O, fp32 LSE)."""
+
+    def __init__(self, scale: float, stream=None):
+        self.scale = float(scale)
+        self.stream = stream
+
+    def _sid(self, t):
+        import torch
+        st = self.stream if self.stream is not None else torch.cuda.current_stream(t.device)
+        return int(st.cuda_stream)
+
+    def partial(self, q, k, v, causal: bool):
+        from . import flash_attention_forward
+        return flash_attention_forward(q, k, v, self.scale, causal, stream=self.stream)
+
+    def init(self, q):
+        import torch
+        B, H, S, D = q.shape
+        o = torch.zeros((B, H, S, D), dtype=torch.float32, device=q.device)
+        lse = torch.full((B, H, S), float("-inf"), dtype=torch.float32, device=q.device)
+        return [o, lse, q.dtype]
+
+    def merge(self, state, o_part, lse_part):
+        from . import FaError, fa_merge_partial
+        from . import _dtype_code
+        o_acc, lse_acc, _ = state
+        rows = lse_acc.numel()
+        rc = fa_merge_partial(o_acc.data_ptr(), lse_acc.data_ptr(), o_part.data_ptr(), lse_part.data_ptr(), rows,
+                              o_acc.shape[-1], _dtype_code(o_part), self._sid(o_acc))
+        if rc != 0:
+            raise FaError(rc, "fa_merge_partial")
+
+    def finalize(self, state):
+        import torch
+        from . import FaError, fa_merge_finalize
+        o_acc, lse_acc, dtype = state
+        o = torch.empty(o_acc.shape, dtype=dtype, device=o_acc.device)
+        code = 1 if dtype == torch.bfloat16 else 0
+        rc = fa_merge_finalize(o_acc.data_ptr(), o.data_ptr(), o_acc.numel(), code, self._sid(o_acc))
+        if rc != 0:
+            raise FaError(rc, "fa_merge_finalize")
+        return o, lse_acc
+
+
+def _p2p_ring_exchange(group, rank: int, world: int):
+    """Send the held K/V block to rank + 1 and receive the next from rank - 1
+    (one packed buffer per step)."""
+    import torch
+    import torch.distributed as dist
+
+    nxt = dist.get_global_rank(group, (rank + 1) % world) if group is not None else (rank + 1) % world
+    prv = dist.get_global_rank(group, (rank - 1) % world) if group is not None else (rank - 1) % world
+
+    def exchange(step: int, kv):
+        recv = torch.empty_like(kv)
+        ops = [dist.P2POp(dist.isend, kv, nxt, group), dist.P2POp(dist.irecv, recv, prv, group)]
+        reqs = dist.batch_isend_irecv(ops)
+        return reqs, recv
+
+    return exchange
+
+
+def ring_attention_forward(q, k, v, scale: float, causal: bool = False, group=None, ops=None,
+                           exchange: Optional[Callable] = None, rank: Optional[int] = None,
+                           world: Optional[int] = None):
+    """O and LSE of this rank's query chunk over the whole sequence.
+
+    q, k, v: this rank's contiguous chunks [B, H, c, D] (equal c on every rank).
+    With the default ``exchange`` the K/V blocks move by NCCL (or gloo) P2P on
+    ``group``; the transfer of step s + 1's block is started before step s's
+    attention and waited for after it, so the two overlap.
+    """
+    import torch
+    import torch.distributed as dist
+
+    if rank is None:
+        rank = dist.get_rank(group)
+    if world is None:
+        world = dist.get_world_size(group)
+    ops = ops if ops is not None else CudaOps(scale)
+    if exchange is None:
+        exchange = _p2p_ring_exchange(group, rank, world)
+    c = k.shape[2]
+    kv = torch.stack([k, v])  # one buffer per step: [2, B, H, c, D]
+    state = ops.init(q)
+    for s, (src, mode) in enumerate(ring_schedule(rank, world, causal)):
+        pending = exchange(s, kv) if s + 1 < world else None
+        if mode != "skip":
+            o_p, lse_p = ops.partial(q, kv[0], kv[1], mode == "causal")
+            ops.merge(state, o_p, lse_p)
+        if pending is not None:
+            reqs, nxt = pending
+            for r in reqs or []:
+                r.wait()
+            kv = nxt
+    assert kv.shape[3] == c
+    return ops.finalize(state)
+
+
+def allgather_attention_forward(q, k, v, scale: float, causal: bool = False, group=None, ops=None,
+                                gather: Optional[Callable] = None, rank: Optional[int] = None,
+                                world: Optional[int] = None):
+    """O and LSE of this rank's query chunk: all-gather K and V, then one
+    partial over the visible keys (all of them, or the first (rank + 1) * c
+    with the causal mask, aligned bottom-right)."""
+    import torch
+    import torch.distributed as dist
+
+    if rank is None:
+        rank = dist.get_rank(group)
+    if world is None:
+        world = dist.get_world_size(group)
+    ops = ops if ops is not None else CudaOps(scale)
+    B, H, c, D = k.shape
+    kv = torch.stack([k, v]).contiguous()
+    if gather is None:
+        # the concatenated form [world * 2, ...] (every backend accepts it)
+        out = torch.empty((world * 2,) + tuple(kv.shape[1:]), dtype=kv.dtype, device=kv.device)
+        dist.all_gather_into_tensor(out, kv, group=group)
+        out = out.view((world,) + tuple(kv.shape))
+    else:
+        out = gather(kv)
+    # [world, 2, B, H, c, D] -> K, V [B, H, world * c, D] (rank-ordered chunks)
+    full = out.permute(1, 2, 3, 0, 4, 5).reshape(2, B, H, world * c, D)
+    n_keys = (rank + 1) * c if causal else world * c
+    kf = full[0, :, :, :n_keys].contiguous()
+    vf = full[1, :, :, :n_keys].contiguous()
+    return ops.partial(q, kf, vf, causal)
