@@ -49,6 +49,7 @@ from tiled_attention_18_b200.workloads import (GENERAL_WORKLOADS, WORKLOADS, sam
 METRIC = "attention fwd TFLOPS (causal-adjusted) and % of B200 dense fp16/bf16 peak"
 UNIT = "TFLOP/s"
 FALLBACK_BF16_TFLOPS = 1590.0
+FALLBACK_HBM_GBS = 6650.0
 PEAKS_PATH = os.path.join(ROOT, "MEASURED_PEAKS.json")
 TRAFFIC_PATH = os.path.join(ROOT, "profiles", "fa_fwd_traffic.json")
 KERNEL_SRC = os.path.join(ROOT, "tiled_attention_18_b200", "csrc", "fa_fwd_sm100.cu")
@@ -402,6 +403,150 @@ def run_bwd(args) -> int:
     return 0
 
 
+def hbm_peak():
+    try:
+        with open(PEAKS_PATH) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured (MEASURED_PEAKS.json hbm_gbs)"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback (6.65 TB/s pool measurement)"
+
+
+def run_sp(args) -> int:
+    """Sequence-parallel forward: the ring (or all-gather) schedule of
+    sequence_parallel.py for --sp-world ranks, run one rank after another on
+    this GPU with the K/V blocks handed over in memory -- every partial
+    attention, merge and finalize launch of all ranks, no communication.  The
+    value is the attention throughput of the split computation (whole-sequence
+    flops over the summed device time), to set beside the single-kernel
+    forward; the merge kernel's HBM roofline is reported beside it."""
+    import torch
+
+    import tiled_attention_18_b200 as fa
+    from tiled_attention_18_b200.sequence_parallel import CudaOps, allgather_attention_forward, ring_attention_forward
+
+    rank, world, local = rank_env()
+    if world > 1:
+        raise SystemExit("--pass sp runs every rank's schedule in one process on one GPU; launch it without torchrun")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    fa.load()
+    W = args.sp_world
+    runs = workload_runs(args.workload)
+    for w in runs:
+        if w.layout != "bhsd" or w.S != w.Skv or w.S % W:
+            raise SystemExit("--pass sp needs a self-attention BHSD workload whose S divides into --sp-world chunks")
+    stream = torch.cuda.current_stream(dev)
+    sid = stream.cuda_stream
+    data = []
+    for w in runs:
+        q, k, v = (t.to(dev) for t in workload_inputs(w))
+        c = w.S // W
+        qs = [q[:, :, r * c:(r + 1) * c].contiguous() for r in range(W)]
+        kv = [torch.stack([k[:, :, r * c:(r + 1) * c], v[:, :, r * c:(r + 1) * c]]).contiguous() for r in range(W)]
+        data.append((w, qs, kv, torch.stack(kv) if args.sp_mode == "allgather" else None))
+        del q, k, v
+
+    class TimedOps(CudaOps):
+        def __init__(self, scale, log):
+            super().__init__(scale)
+            self.log = log
+
+        def _timed(self, kind, nbytes, fn, *a):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            out = fn(*a)
+            e1.record(stream)
+            self.log.append((kind, e0, e1, nbytes))
+            return out
+
+        def partial(self, q, k, v, causal):
+            return self._timed("partial", 0, super().partial, q, k, v, causal)
+
+        def merge(self, state, o_p, lse_p):
+            # per row: fp32 O read and written (8 D bytes), the 16-bit partial O (2 D), three fp32 LSE words
+            nbytes = (10 * o_p.shape[-1] + 12) * lse_p.numel()
+            return self._timed("merge", nbytes, super().merge, state, o_p, lse_p)
+
+        def finalize(self, state):
+            return self._timed("finalize", 0, super().finalize, state)
+
+    def step(log):
+        for (w, qs, kv, stacked) in data:
+            ops = TimedOps(w.scale, log)
+            for r in range(W):
+                qk = qs[r]
+                if args.sp_mode == "ring":
+                    ring_attention_forward(qk, kv[r][0], kv[r][1], w.scale, w.causal, ops=ops, rank=r, world=W,
+                                           exchange=lambda s, cur, r=r: (None, kv[(r - s - 1) % W]))
+                else:
+                    allgather_attention_forward(qk, kv[r][0], kv[r][1], w.scale, w.causal, ops=ops, rank=r,
+                                                world=W, gather=lambda cur, st=stacked: st)
+
+    for _ in range(args.warmup):
+        step([])
+    torch.cuda.synchronize(dev)
+    st = fa.fa_check_status(sid)
+    if st != 0:
+        raise fa.FaError(st, "warm-up")
+    log = []
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.3)
+    torch.cuda.synchronize(dev)
+    start.record(stream)
+    for _ in range(args.steps):
+        step(log)
+    stop.record(stream)
+    torch.cuda.synchronize(dev)
+    sampler.stop()
+    st = fa.fa_check_status(sid)
+    if st != 0:
+        raise fa.FaError(st, "timed region")
+    total_ms = start.elapsed_time(stop)
+    ms = {"partial": 0.0, "merge": 0.0, "finalize": 0.0}
+    n = {"partial": 0, "merge": 0, "finalize": 0}
+    merge_bytes = 0
+    for kind, a, b, nbytes in log:
+        ms[kind] += a.elapsed_time(b)
+        n[kind] += 1
+        merge_bytes += nbytes
+    step_flops = sum(w.flops for w in runs)
+    value = step_flops * args.steps / (total_ms * 1e-3) / 1e12
+    peak, peak_src = peak_tflops()
+    achieved = step_flops * args.steps / (ms["partial"] * 1e-3) / 1e12
+    hbm, hbm_src = hbm_peak()
+    merge_info = None
+    if n["merge"]:
+        gbs = merge_bytes / (ms["merge"] * 1e-3) / 1e9
+        merge_info = {"bytes_per_launch": merge_bytes / n["merge"], "mean_us": 1e3 * ms["merge"] / n["merge"],
+                      "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm, "peak_source": hbm_src,
+                      "launches_per_step": n["merge"] // args.steps}
+    launches = sum(n.values())  # partials, merges, finalizes; the all-gather's K/V copies are torch's
+    cb = None if args.no_cpu_baseline else cpu_baseline(args.workload)
+    w0 = runs[0]
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": total_ms / args.steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": w0.dtype, "data": "synthetic",
+        "config": {"workload": f"sequence-parallel ({args.sp_mode}, {W} ranks run in turn on one GPU, no "
+                               f"communication) " + workload_label(args.workload),
+                   "B": w0.B, "H": w0.H, "S": w0.S, "D": w0.D, "chunk": w0.S // W,
+                   "l2": "inputs larger than L2 (no flush)"},
+        "pct_of_peak": 100.0 * value / peak,
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": UNIT, "frac": achieved / peak,
+                     "traffic": None, "peak_source": peak_src, "kernel": "fa_fwd_ex partials"},
+        "time_split_ms_per_step": {k: v / args.steps for k, v in ms.items()},
+        "merge": merge_info,
+        "clocks": sampler.summary(),
+        "e2e": None,
+        "gpu_launches": launches,
+        "cpu_baseline": cb,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main(argv=None) -> int:
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -412,8 +557,11 @@ def main(argv=None) -> int:
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--pass", dest="pass_", choices=["fwd", "bwd"], default="fwd",
-                    help="fwd: the forward pass (default); bwd: the backward pass fa_bwd")
+    ap.add_argument("--pass", dest="pass_", choices=["fwd", "bwd", "sp"], default="fwd",
+                    help="fwd: the forward pass (default); bwd: the backward pass fa_bwd; sp: the "
+                         "sequence-parallel schedule of --sp-world ranks run in turn on one GPU")
+    ap.add_argument("--sp-world", type=int, default=4, help="with --pass sp: ranks of the schedule")
+    ap.add_argument("--sp-mode", choices=["ring", "allgather"], default="ring", help="with --pass sp")
     ap.add_argument("--mask", choices=["none", "tril"], default="none",
                     help="tril: causal runs go through fa_fwd_mask with an explicit lower-triangular mask "
                          "(the catlass page's mode 1) instead of the in-kernel diagonal skip (mode 2)")
@@ -426,6 +574,8 @@ def main(argv=None) -> int:
         return run_reference(args)
     if args.pass_ == "bwd":
         return run_bwd(args)
+    if args.pass_ == "sp":
+        return run_sp(args)
 
     import torch
     import torch.distributed as dist

@@ -269,7 +269,7 @@ FA_API int fa_bwd_mask(const void* q, const void* k, const void* v, const void* 
  *           unchanged.
  * o_part  : device, [rows][D] 16-bit (dtype), a partial O, e.g. from fa_fwd_ex.
  * lse_part: device, [rows] fp32, its LSE (-inf: the partial saw no key).
- * rows, D : contiguous rows of D values (1 <= D <= 1024).
+ * rows, D : contiguous rows of D values (0 <= rows <= 2^33, 1 <= D <= 1024).
  * Asynchronous on stream; errors as fa_fwd (argument checks first).
  */
 FA_API int fa_merge_partial(float* o_acc, float* lse_acc, const void* o_part, const float* lse_part, long long rows,

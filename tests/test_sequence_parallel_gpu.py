@@ -75,3 +75,55 @@ def test_merge_partial_matches_union_and_empty_sides():
     torch.cuda.synchronize()
     o_ref, lse_ref = oracle.attn_fwd(q, k, v, 0.09, False, "bf16")
     compare(o.cpu(), lse.cpu(), o_ref, lse_ref, "bf16")
+
+
+@pytest.mark.parametrize("D,offset", [(128, 0), (64, 0), (98, 0), (128, 1)], ids=["d128", "d64", "d98", "unaligned"])
+@pytest.mark.parametrize("dtype", ["bf16", "fp16"])
+def test_merge_partial_kernel_matches_fp64_merge(D, offset, dtype):
+    """fa_merge_partial against the log-sum-exp combination written out in
+    fp64, with rows where either side or both sides are empty (LSE = -inf);
+    D = 98 and a buffer offset by one element take the scalar variant."""
+    tdt = torch.bfloat16 if dtype == "bf16" else torch.float16
+    rows = 1000
+    g = torch.Generator().manual_seed(D + offset)
+    o_acc = torch.randn(rows * D + offset, generator=g)
+    l_acc = torch.randn(rows, generator=g) * 4
+    o_p = torch.randn(rows * D + offset, generator=g).to(tdt)
+    l_p = torch.randn(rows, generator=g) * 4
+    l_acc[::7] = float("-inf")
+    l_p[::11] = float("-inf")
+    a0 = o_acc[offset:].view(rows, D).double().numpy()
+    b0 = o_p[offset:].view(rows, D).double().numpy()
+    la, lb = l_acc.double().numpy(), l_p.double().numpy()
+    m = np.maximum(la, lb)
+    with np.errstate(invalid="ignore"):
+        wa = np.where(np.isinf(la), 0.0, np.exp(la - m))
+        wb = np.where(np.isinf(lb), 0.0, np.exp(lb - m))
+        s = wa + wb
+        o_ref = np.where((s > 0)[:, None], (wa[:, None] * a0 + wb[:, None] * b0) / np.where(s > 0, s, 1)[:, None], a0)
+        l_ref = np.where(s > 0, m + np.log(np.where(s > 0, s, 1)), la)
+    d_acc, d_lacc, d_p, d_lp = (t.cuda() for t in (o_acc, l_acc, o_p, l_p))
+    rc = fa.fa_merge_partial(d_acc.data_ptr() + 4 * offset, d_lacc.data_ptr(), d_p.data_ptr() + 2 * offset,
+                             d_lp.data_ptr(), rows, D, 1 if dtype == "bf16" else 0,
+                             torch.cuda.current_stream().cuda_stream)
+    assert rc == 0
+    torch.cuda.synchronize()
+    got_o = d_acc.cpu()[offset:].view(rows, D).double().numpy()
+    got_l = d_lacc.cpu().double().numpy()
+    # fp32 weights and products: a few ulps of fp32 relative to the row's magnitude
+    scale_o = np.abs(a0).max(axis=1, keepdims=True) + np.abs(b0).max(axis=1, keepdims=True)
+    assert np.all(np.abs(got_o - o_ref) <= 4e-6 * scale_o)
+    both_empty = np.isinf(la) & np.isinf(lb)
+    assert np.all(np.isneginf(got_l[both_empty]))
+    assert np.all(np.abs(got_l[~both_empty] - l_ref[~both_empty]) <= 4e-6 * (1 + np.abs(l_ref[~both_empty])))
+
+
+def test_merge_finalize_rounds_to_nearest_even():
+    x = torch.randn(4099, generator=torch.Generator().manual_seed(3)) * 10
+    for tdt, code in ((torch.bfloat16, 1), (torch.float16, 0)):
+        dx = x.cuda()
+        out = torch.empty(4099, dtype=tdt, device="cuda")
+        assert fa.fa_merge_finalize(dx.data_ptr(), out.data_ptr(), 4099, code,
+                                    torch.cuda.current_stream().cuda_stream) == 0
+        torch.cuda.synchronize()
+        assert torch.equal(out.cpu(), x.to(tdt))

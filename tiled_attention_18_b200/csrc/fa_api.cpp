@@ -443,7 +443,7 @@ int fa_bwd_mask(const void* q, const void* k, const void* v, const void* o, cons
 
 int fa_merge_partial(float* o_acc, float* lse_acc, const void* o_part, const float* lse_part, long long rows, int D,
                      int dtype, cudaStream_t stream) {
-    if (rows < 0) return FA_ERR_SHAPE;
+    if (rows < 0 || rows > (1LL << 33)) return FA_ERR_SHAPE;  // 8 rows per block, grid < 2^31
     if (D < 1 || D > 1024) return FA_ERR_HEADDIM;
     if (dtype != FA_FP16 && dtype != FA_BF16) return FA_ERR_DTYPE;
     if (rows == 0) return FA_OK;

@@ -36,6 +36,15 @@ __device__ __forceinline__ uint16_t from_f32(float x) {
 }
 
 template <bool BF16>
+__device__ __forceinline__ float4 load4_f32(const uint16_t* p) {
+    const uint2 raw = *reinterpret_cast<const uint2*>(p);
+    return make_float4(to_f32<BF16>((uint16_t)(raw.x & 0xffffu)), to_f32<BF16>((uint16_t)(raw.x >> 16)),
+                       to_f32<BF16>((uint16_t)(raw.y & 0xffffu)), to_f32<BF16>((uint16_t)(raw.y >> 16)));
+}
+
+// VEC: D % 4 == 0 with 16-byte aligned o_acc and 8-byte aligned o_part, so a
+// lane moves four consecutive values per access (one float4, one 8-byte load).
+template <bool BF16, bool VEC>
 __global__ void __launch_bounds__(256) merge_kernel(float* __restrict__ o_acc, float* __restrict__ lse_acc,
                                                     const uint16_t* __restrict__ o_part,
                                                     const float* __restrict__ lse_part, long long rows, int D) {
@@ -51,7 +60,23 @@ __global__ void __launch_bounds__(256) merge_kernel(float* __restrict__ o_acc, f
     const float ca = wa * inv, cb = wb * inv;
     float* oa = o_acc + row * D;
     const uint16_t* ob = o_part + row * D;
-    for (int d = lane; d < D; d += 32) oa[d] = ca * oa[d] + cb * to_f32<BF16>(ob[d]);
+    // an accumulator that has seen no key yet (ca = 0) is overwritten, not read
+    if constexpr (VEC) {
+        for (int d = 4 * lane; d < D; d += 128) {
+            const float4 b = load4_f32<BF16>(ob + d);
+            float4 r;
+            if (ca != 0.f) {
+                const float4 a = *reinterpret_cast<const float4*>(oa + d);
+                r = make_float4(ca * a.x + cb * b.x, ca * a.y + cb * b.y, ca * a.z + cb * b.z, ca * a.w + cb * b.w);
+            } else {
+                r = make_float4(cb * b.x, cb * b.y, cb * b.z, cb * b.w);
+            }
+            *reinterpret_cast<float4*>(oa + d) = r;
+        }
+    } else {
+        for (int d = lane; d < D; d += 32)
+            oa[d] = (ca != 0.f ? ca * oa[d] : 0.f) + cb * to_f32<BF16>(ob[d]);
+    }
     __syncwarp();
     if (lane == 0) lse_acc[row] = m + logf(wa + wb);
 }
@@ -68,12 +93,15 @@ __global__ void __launch_bounds__(256) finalize_kernel(const float* __restrict__
 cudaError_t launch_merge_partial(float* o_acc, float* lse_acc, const void* o_part, const float* lse_part,
                                  long long rows, int D, int dtype, cudaStream_t stream) {
     const unsigned blocks = (unsigned)((rows + 7) / 8);
-    if (dtype == 1)
-        merge_kernel<true><<<blocks, 256, 0, stream>>>(o_acc, lse_acc, static_cast<const uint16_t*>(o_part), lse_part,
-                                                       rows, D);
-    else
-        merge_kernel<false><<<blocks, 256, 0, stream>>>(o_acc, lse_acc, static_cast<const uint16_t*>(o_part),
-                                                        lse_part, rows, D);
+    const uint16_t* ob = static_cast<const uint16_t*>(o_part);
+    const bool vec = (D % 4 == 0) && ((uintptr_t)o_acc % 16 == 0) && ((uintptr_t)o_part % 8 == 0);
+    if (dtype == 1) {
+        if (vec) merge_kernel<true, true><<<blocks, 256, 0, stream>>>(o_acc, lse_acc, ob, lse_part, rows, D);
+        else merge_kernel<true, false><<<blocks, 256, 0, stream>>>(o_acc, lse_acc, ob, lse_part, rows, D);
+    } else {
+        if (vec) merge_kernel<false, true><<<blocks, 256, 0, stream>>>(o_acc, lse_acc, ob, lse_part, rows, D);
+        else merge_kernel<false, false><<<blocks, 256, 0, stream>>>(o_acc, lse_acc, ob, lse_part, rows, D);
+    }
     return cudaGetLastError();
 }
 
