@@ -25,6 +25,11 @@ ctypes.  Function-level citations are in the C file's header:
   softmax Jacobian), with optional absolute-value error scales.
 - ``attn_fwd_masked`` / ``attn_bwd_masked`` : the definition with an explicit
   boolean mask, and its gradients.
+- ``philox4x32_10`` / ``dropout_keep_mask`` : the counter-based generator
+  (Salmon et al., SC 2011) and the keep decisions of attention dropout.
+- ``attn_fwd_dropout`` / ``attn_rows_dropout`` / ``attn_bwd_dropout`` :
+  attention with dropout after the softmax (FlashAttention-2 page, sections
+  3.4 and 6.3) and its gradients.
 
 Parity pins: every function above is pinned by tests in tests/test_oracle.py and
 tests/test_oracle_general.py (torch SDPA in float64 with an explicit mask, the
@@ -32,7 +37,9 @@ Q = 0 closed form, agreement with attn_fwd when Sq = Sk) and
 tests/test_oracle_bwd.py (float64 autograd, central finite differences of
 attn_fwd_gen, closed forms and column-sum identities) and
 tests/test_oracle_mask.py (SDPA fp64 with a boolean mask, all-ones mask =
-no mask, lower-triangular mask = the causal flag, fully masked rows).
+no mask, lower-triangular mask = the causal flag, fully masked rows) and
+tests/test_oracle_dropout.py (Philox known-answer vectors, keep rates, p = 0
+equals no dropout, unbiasedness over offsets, float64 autograd).
 """
 from __future__ import annotations
 
@@ -111,6 +118,24 @@ def _load():
                                                ctypes.c_int, ctypes.c_int, ctypes.POINTER(ctypes.c_uint8), i64, i64,
                                                i64, f64p, f64p, f64p, f64p, f64p, f64p]
         lib.oracle_attn_bwd_masked.restype = ctypes.c_int
+        u32 = ctypes.c_uint32
+        u32p = ctypes.POINTER(ctypes.c_uint32)
+        lib.oracle_philox4x32_10.argtypes = [u32p, u32p, u32p]
+        lib.oracle_philox4x32_10.restype = None
+        lib.oracle_dropout_keep_mask.argtypes = [i64, i64, i64, u32, ctypes.c_uint64, u32,
+                                                 ctypes.POINTER(ctypes.c_uint8)]
+        lib.oracle_dropout_keep_mask.restype = ctypes.c_int
+        lib.oracle_attn_fwd_dropout.argtypes = [u16p, u16p, u16p, i64, i64, i64, i64, i64, ctypes.c_float,
+                                                ctypes.c_int, ctypes.c_int, u32, ctypes.c_uint64, u32, f64p, f64p]
+        lib.oracle_attn_fwd_dropout.restype = ctypes.c_int
+        lib.oracle_attn_rows_dropout.argtypes = [u16p, u16p, u16p, i64, i64, i64, i64, i64, ctypes.c_float,
+                                                 ctypes.c_int, ctypes.c_int, u32, ctypes.c_uint64, u32, i64p, i64p,
+                                                 i64, f64p, f64p]
+        lib.oracle_attn_rows_dropout.restype = ctypes.c_int
+        lib.oracle_attn_bwd_dropout.argtypes = [u16p, u16p, u16p, u16p, i64, i64, i64, i64, i64, ctypes.c_float,
+                                                ctypes.c_int, ctypes.c_int, u32, ctypes.c_uint64, u32, f64p, f64p,
+                                                f64p, f64p, f64p, f64p]
+        lib.oracle_attn_bwd_dropout.restype = ctypes.c_int
         lib.oracle_causal_tile_count.argtypes = [i64, i64, i64, i64p, i64p, i64p]
         lib.oracle_causal_tile_count.restype = None
         lib.oracle_num_threads.argtypes = []
@@ -306,6 +331,91 @@ def attn_bwd_masked(q, k, v, dout, mask, scale: float, causal: bool, dtype, magn
                                     fp(dq), fp(dk), fp(dv), fp(mags[0]), fp(mags[1]), fp(mags[2]))
     if rc != 0:
         raise RuntimeError(f"oracle_attn_bwd_masked failed with {rc}")
+    return (dq, dk, dv) + (mags if magnitudes else ())
+
+
+def philox4x32_10(counter, key):
+    """Philox4x32-10 of one 128-bit counter (4 words) under a 64-bit key (2 words)."""
+    lib = _load()
+    c = np.ascontiguousarray(counter, dtype=np.uint32)
+    k = np.ascontiguousarray(key, dtype=np.uint32)
+    if c.shape != (4,) or k.shape != (2,):
+        raise ValueError("counter: 4 words, key: 2 words")
+    out = np.empty(4, dtype=np.uint32)
+    lib.oracle_philox4x32_10(_ptr(c, ctypes.c_uint32), _ptr(k, ctypes.c_uint32), _ptr(out, ctypes.c_uint32))
+    return out
+
+
+def dropout_keep_mask(BH: int, Sq: int, Sk: int, p8: int, seed: int, offset: int) -> np.ndarray:
+    """keep[bh, i, j] (1 = kept) of attention dropout with threshold p8 (1/256 units)."""
+    lib = _load()
+    keep = np.empty((BH, Sq, Sk), dtype=np.uint8)
+    rc = lib.oracle_dropout_keep_mask(BH, Sq, Sk, int(p8), int(seed) & (2**64 - 1), int(offset) & 0xffffffff,
+                                      _ptr(keep, ctypes.c_uint8))
+    if rc != 0:
+        raise RuntimeError(f"oracle_dropout_keep_mask failed with {rc}")
+    return keep
+
+
+def attn_fwd_dropout(q, k, v, scale: float, causal: bool, dtype, p8: int, seed: int, offset: int):
+    """attn_fwd_gen with dropout after the softmax: weights kept by the Philox rule
+    of attn_oracle.c (threshold p8 in 1/256 units), kept weights scaled by
+    256 / (256 - p8); LSE of the undropped softmax."""
+    lib = _load()
+    qb, kb, vb = _bits(q), _bits(k), _bits(v)
+    B, H, Sq, D = qb.shape
+    Sk = kb.shape[2]
+    o = np.empty((B, H, Sq, D))
+    lse = np.empty((B, H, Sq))
+    rc = lib.oracle_attn_fwd_dropout(_ptr(qb, ctypes.c_uint16), _ptr(kb, ctypes.c_uint16), _ptr(vb, ctypes.c_uint16),
+                                     B, H, Sq, Sk, D, float(np.float32(scale)), int(bool(causal)), _dtype_code(dtype),
+                                     int(p8), int(seed) & (2**64 - 1), int(offset) & 0xffffffff,
+                                     _ptr(o, ctypes.c_double), _ptr(lse, ctypes.c_double))
+    if rc != 0:
+        raise RuntimeError(f"oracle_attn_fwd_dropout failed with {rc}")
+    return o, lse
+
+
+def attn_rows_dropout(q, k, v, scale: float, causal: bool, dtype, p8: int, seed: int, offset: int, bh_idx, row_idx):
+    """attn_fwd_dropout for selected (bh, query row) pairs. Returns (O [n,D], LSE [n])."""
+    lib = _load()
+    qb, kb, vb = _bits(q), _bits(k), _bits(v)
+    B, H, Sq, D = qb.shape
+    Sk = kb.shape[2]
+    bh = np.ascontiguousarray(bh_idx, dtype=np.int64)
+    ri = np.ascontiguousarray(row_idx, dtype=np.int64)
+    n = bh.size
+    o = np.empty((n, D))
+    lse = np.empty((n,))
+    rc = lib.oracle_attn_rows_dropout(_ptr(qb, ctypes.c_uint16), _ptr(kb, ctypes.c_uint16), _ptr(vb, ctypes.c_uint16),
+                                      B, H, Sq, Sk, D, float(np.float32(scale)), int(bool(causal)),
+                                      _dtype_code(dtype), int(p8), int(seed) & (2**64 - 1), int(offset) & 0xffffffff,
+                                      _ptr(bh, ctypes.c_int64), _ptr(ri, ctypes.c_int64), n,
+                                      _ptr(o, ctypes.c_double), _ptr(lse, ctypes.c_double))
+    if rc != 0:
+        raise RuntimeError(f"oracle_attn_rows_dropout failed with {rc}")
+    return o, lse
+
+
+def attn_bwd_dropout(q, k, v, dout, scale: float, causal: bool, dtype, p8: int, seed: int, offset: int,
+                     magnitudes: bool = False):
+    """attn_bwd for the attention with dropout of attn_fwd_dropout."""
+    lib = _load()
+    qb, kb, vb, gb = _bits(q), _bits(k), _bits(v), _bits(dout)
+    B, H, Sq, D = qb.shape
+    Sk = kb.shape[2]
+    dq = np.empty((B, H, Sq, D))
+    dk = np.empty((B, H, Sk, D))
+    dv = np.empty((B, H, Sk, D))
+    mags = tuple(np.empty(a.shape) for a in (dq, dk, dv)) if magnitudes else (None, None, None)
+    fp = lambda a: _ptr(a, ctypes.c_double) if a is not None else None  # noqa: E731
+    rc = lib.oracle_attn_bwd_dropout(_ptr(qb, ctypes.c_uint16), _ptr(kb, ctypes.c_uint16), _ptr(vb, ctypes.c_uint16),
+                                     _ptr(gb, ctypes.c_uint16), B, H, Sq, Sk, D, float(np.float32(scale)),
+                                     int(bool(causal)), _dtype_code(dtype), int(p8), int(seed) & (2**64 - 1),
+                                     int(offset) & 0xffffffff, fp(dq), fp(dk), fp(dv), fp(mags[0]), fp(mags[1]),
+                                     fp(mags[2]))
+    if rc != 0:
+        raise RuntimeError(f"oracle_attn_bwd_dropout failed with {rc}")
     return (dq, dk, dv) + (mags if magnitudes else ())
 
 

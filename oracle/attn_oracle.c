@@ -524,6 +524,185 @@ int oracle_attn_rows_gen(const uint16_t *q, const uint16_t *k, const uint16_t *v
     return bad ? -10 : 0;
 }
 
+/* ------------------------------------------------------------------ dropout */
+
+/*
+ * Attention dropout: after the softmax each weight P_ij is kept with
+ * probability 1 - p and zeroed otherwise, and the kept weights are scaled by
+ * 1 / (1 - p), so O_i = sum_j P_ij z_ij v_j with z_ij = keep_ij / (1 - p)
+ * (an unbiased estimate of the undropped O).  The normalisation l and the
+ * LSE are those of the undropped softmax.  Source: the fused dropout of the
+ * FlashAttention-2 page, sections 3.4 and 6.3 (dropout_prob = 0.1 inside the
+ * kernel, random numbers drawn on the device).  That page's listing writes
+ * -infinity into the score before the softmax instead; that variant is the
+ * explicit mask of oracle_attn_fwd_masked with a random mask.  The standard
+ * reading (drop after the softmax, rescale the kept weights) is the one
+ * taken here.
+ *
+ * The pages name no generator.  The keep decisions come from Philox4x32-10
+ * (Salmon, Moraes, Dror and Shaw, "Parallel Random Numbers: As Easy as 1, 2,
+ * 3", SC 2011): for head bh = b * H + h, query row i and key j,
+ *   counter = (j / 16, i, bh, offset), key = (seed mod 2^32, seed / 2^32),
+ * and element j takes byte j mod 16 of the four 32-bit output words (word
+ * (j mod 16) / 4, bits 8 (j mod 4) .. 8 (j mod 4) + 7).  It is kept iff that
+ * byte is >= p8, the drop threshold in 1/256 units; the drop probability is
+ * p8 / 256 and the kept weights are scaled by 256 / (256 - p8).
+ */
+#define PHILOX_M0 0xD2511F53u
+#define PHILOX_M1 0xCD9E8D57u
+#define PHILOX_W0 0x9E3779B9u
+#define PHILOX_W1 0xBB67AE85u
+
+/* Ten rounds of the Philox-4x32 bijection; the key is bumped by the Weyl
+ * constants before every round after the first. */
+void oracle_philox4x32_10(const uint32_t ctr[4], const uint32_t key[2], uint32_t out[4])
+{
+    uint32_t x0 = ctr[0], x1 = ctr[1], x2 = ctr[2], x3 = ctr[3];
+    uint32_t k0 = key[0], k1 = key[1];
+    for (int r = 0; r < 10; ++r) {
+        if (r > 0) {
+            k0 += PHILOX_W0;
+            k1 += PHILOX_W1;
+        }
+        const uint64_t a = (uint64_t)PHILOX_M0 * x0;  /* hi/lo products of the two multipliers */
+        const uint64_t b = (uint64_t)PHILOX_M1 * x2;
+        const uint32_t y0 = (uint32_t)(b >> 32) ^ x1 ^ k0;
+        const uint32_t y1 = (uint32_t)b;
+        const uint32_t y2 = (uint32_t)(a >> 32) ^ x3 ^ k1;
+        const uint32_t y3 = (uint32_t)a;
+        x0 = y0; x1 = y1; x2 = y2; x3 = y3;
+    }
+    out[0] = x0; out[1] = x1; out[2] = x2; out[3] = x3;
+}
+
+static int dropout_keep(uint64_t seed, uint32_t offset, uint32_t p8, int64_t bh, int64_t i, int64_t j)
+{
+    const uint32_t ctr[4] = {(uint32_t)(j >> 4), (uint32_t)i, (uint32_t)bh, offset};
+    const uint32_t key[2] = {(uint32_t)seed, (uint32_t)(seed >> 32)};
+    uint32_t w[4];
+    oracle_philox4x32_10(ctr, key, w);
+    const uint32_t byte = (w[(j & 15) >> 2] >> (8 * (j & 3))) & 0xffu;
+    return byte >= p8;
+}
+
+/* keep[bh][i][j] (1 = kept) for tests; BH * Sq * Sk bytes. */
+int oracle_dropout_keep_mask(int64_t BH, int64_t Sq, int64_t Sk, uint32_t p8, uint64_t seed, uint32_t offset,
+                             uint8_t *keep)
+{
+    if (BH < 0 || Sq < 0 || Sk < 0 || p8 > 255) return -2;
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < BH * Sq; ++r)
+        for (int64_t j = 0; j < Sk; ++j) keep[r * Sk + j] = (uint8_t)dropout_keep(seed, offset, p8, r / Sq, r % Sq, j);
+    return 0;
+}
+
+/* One query row with dropout: the softmax over the nj visible keys, then
+ * O = sum_j P_j z_j v_j.  An empty row gets O = 0, LSE = -inf. */
+static void dropout_row(const double *qi, const double *kh, const double *vh, int64_t nj, int64_t D, double scale,
+                        uint64_t seed, uint32_t offset, uint32_t p8, int64_t bh, int64_t i, double *srow, double *o,
+                        double *lse)
+{
+    if (nj <= 0) {
+        for (int64_t d = 0; d < D; ++d) o[d] = 0.0;
+        *lse = -INFINITY;
+        return;
+    }
+    const double zs = 256.0 / (256.0 - (double)p8);
+    for (int64_t j = 0; j < nj; ++j) {
+        double dot = 0.0;
+        for (int64_t d = 0; d < D; ++d) dot += qi[d] * kh[j * D + d];
+        srow[j] = scale * dot;
+    }
+    double m = -INFINITY;
+    for (int64_t j = 0; j < nj; ++j)
+        if (srow[j] > m) m = srow[j];
+    double l = 0.0;
+    for (int64_t j = 0; j < nj; ++j) {
+        srow[j] = exp(srow[j] - m);
+        l += srow[j];
+    }
+    for (int64_t d = 0; d < D; ++d) o[d] = 0.0;
+    for (int64_t j = 0; j < nj; ++j) {
+        if (!dropout_keep(seed, offset, p8, bh, i, j)) continue;
+        const double w = srow[j] * zs;
+        for (int64_t d = 0; d < D; ++d) o[d] += w * vh[j * D + d];
+    }
+    for (int64_t d = 0; d < D; ++d) o[d] /= l;
+    *lse = m + log(l);
+}
+
+/* Attention with dropout, general shapes and the bottom-right causal mask of
+ * oracle_attn_fwd_gen.  o: [B,H,Sq,D], lse: [B,H,Sq]. */
+int oracle_attn_fwd_dropout(const uint16_t *q, const uint16_t *k, const uint16_t *v, int64_t B, int64_t H,
+                            int64_t Sq, int64_t Sk, int64_t D, float scale, int causal, int dtype, uint32_t p8,
+                            uint64_t seed, uint32_t offset, double *o, double *lse)
+{
+    if (B < 0 || H < 0 || Sq < 0 || Sk < 0 || D <= 0 || p8 > 255) return -2;
+    if (dtype != ORACLE_F16 && dtype != ORACLE_BF16) return -4;
+    const double sc = (double)scale;
+    for (int64_t bh = 0; bh < B * H; ++bh) {
+        double *qh = (double *)malloc(sizeof(double) * (size_t)(Sq * D > 0 ? Sq * D : 1));
+        double *kh = (double *)malloc(sizeof(double) * (size_t)(Sk * D > 0 ? Sk * D : 1));
+        double *vh = (double *)malloc(sizeof(double) * (size_t)(Sk * D > 0 ? Sk * D : 1));
+        if (!qh || !kh || !vh) { free(qh); free(kh); free(vh); return -10; }
+        oracle_decode(q + bh * Sq * D, qh, Sq * D, dtype);
+        oracle_decode(k + bh * Sk * D, kh, Sk * D, dtype);
+        oracle_decode(v + bh * Sk * D, vh, Sk * D, dtype);
+#pragma omp parallel
+        {
+            double *srow = (double *)malloc(sizeof(double) * (size_t)(Sk > 0 ? Sk : 1));
+#pragma omp for schedule(dynamic, 16)
+            for (int64_t i = 0; i < Sq; ++i)
+                dropout_row(qh + i * D, kh, vh, visible_keys(i, Sq, Sk, causal), D, sc, seed, offset, p8, bh, i,
+                            srow, o + (bh * Sq + i) * D, lse + bh * Sq + i);
+            free(srow);
+        }
+        free(qh); free(kh); free(vh);
+    }
+    return 0;
+}
+
+/* The dropout definition for a list of (bh, i) query rows only. */
+int oracle_attn_rows_dropout(const uint16_t *q, const uint16_t *k, const uint16_t *v, int64_t B, int64_t H,
+                             int64_t Sq, int64_t Sk, int64_t D, float scale, int causal, int dtype, uint32_t p8,
+                             uint64_t seed, uint32_t offset, const int64_t *bh_idx, const int64_t *row_idx,
+                             int64_t nrows, double *o, double *lse)
+{
+    if (B < 0 || H < 0 || Sq < 0 || Sk < 0 || D <= 0 || p8 > 255) return -2;
+    if (dtype != ORACLE_F16 && dtype != ORACLE_BF16) return -4;
+    for (int64_t r = 0; r < nrows; ++r)
+        if (bh_idx[r] < 0 || bh_idx[r] >= B * H || row_idx[r] < 0 || row_idx[r] >= Sq) return -2;
+    const double sc = (double)scale;
+    int bad = 0;
+#pragma omp parallel
+    {
+        double *srow = (double *)malloc(sizeof(double) * (size_t)(Sk > 0 ? Sk : 1));
+        double *qi = (double *)malloc(sizeof(double) * (size_t)D);
+        double *kh = (double *)malloc(sizeof(double) * (size_t)(Sk * D > 0 ? Sk * D : 1));
+        double *vh = (double *)malloc(sizeof(double) * (size_t)(Sk * D > 0 ? Sk * D : 1));
+        int64_t cur_bh = -1;
+        if (!srow || !qi || !kh || !vh) {
+#pragma omp atomic write
+            bad = 1;
+        }
+#pragma omp for schedule(static)
+        for (int64_t r = 0; r < nrows; ++r) {
+            if (!srow || !qi || !kh || !vh) continue;
+            const int64_t bh = bh_idx[r], i = row_idx[r];
+            if (bh != cur_bh) {
+                oracle_decode(k + bh * Sk * D, kh, Sk * D, dtype);
+                oracle_decode(v + bh * Sk * D, vh, Sk * D, dtype);
+                cur_bh = bh;
+            }
+            oracle_decode(q + (bh * Sq + i) * D, qi, D, dtype);
+            dropout_row(qi, kh, vh, visible_keys(i, Sq, Sk, causal), D, sc, seed, offset, p8, bh, i, srow,
+                        o + r * D, lse + r);
+        }
+        free(srow); free(qi); free(kh); free(vh);
+    }
+    return bad ? -10 : 0;
+}
+
 /* ------------------------------------------------------------ backward pass */
 
 /*
@@ -566,14 +745,25 @@ static int bwd_visible(int64_t i, int64_t j, int64_t Sq, int64_t Sk, int causal,
     return mrow ? mrow[j] != 0 : 1;
 }
 
+/*
+ * With dropout (drop != 0; the keep rule and scaling z_ij of the dropout
+ * section above) the forward output is O_i = sum_j P_ij z_ij v_j, so
+ *   dV_j  = sum_i P_ij z_ij dO_i
+ *   dP_ij = z_ij (dO_i . v_j)       (the gradient reaching the weight P_ij)
+ *   dS_ij = P_ij (dP_ij - sum_k P_ik dP_ik)
+ * and sum_k P_ik dP_ik is again dO_i . O_i.  The magnitudes use the same
+ * weights (P z in place of P where a value is multiplied by V or dO).
+ */
 static int attn_bwd_impl(const uint16_t *q, const uint16_t *k, const uint16_t *v, const uint16_t *dout, int64_t B,
                          int64_t H, int64_t Sq, int64_t Sk, int64_t D, float scale, int causal, int dtype,
-                         const uint8_t *mask, int64_t mask_sb, int64_t mask_sh, int64_t mask_si, double *dq,
-                         double *dk, double *dv, double *mag_dq, double *mag_dk, double *mag_dv)
+                         const uint8_t *mask, int64_t mask_sb, int64_t mask_sh, int64_t mask_si, int drop,
+                         uint32_t p8, uint64_t seed, uint32_t offset, double *dq, double *dk, double *dv,
+                         double *mag_dq, double *mag_dk, double *mag_dv)
 {
-    if (B < 0 || H < 0 || Sq < 0 || Sk < 0 || D <= 0) return -2;
+    if (B < 0 || H < 0 || Sq < 0 || Sk < 0 || D <= 0 || p8 > 255) return -2;
     if (dtype != ORACLE_F16 && dtype != ORACLE_BF16) return -4;
     const double sc = (double)scale;
+    const double zs = 256.0 / (256.0 - (double)p8);
     const size_t szq = (size_t)(Sq * D > 0 ? Sq * D : 1), szk = (size_t)(Sk * D > 0 ? Sk * D : 1);
     for (int64_t bh = 0; bh < B * H; ++bh) {
         const uint8_t *mhead = mask ? mask + (bh / H) * mask_sb + (bh % H) * mask_sh : NULL;
@@ -603,6 +793,7 @@ static int attn_bwd_impl(const uint16_t *q, const uint16_t *k, const uint16_t *v
         {
             double *prow = (double *)malloc(sizeof(double) * (size_t)(Sk > 0 ? Sk : 1));
             double *dprow = (double *)malloc(sizeof(double) * (size_t)(Sk > 0 ? Sk : 1));
+            double *zrow = (double *)malloc(sizeof(double) * (size_t)(Sk > 0 ? Sk : 1));
 #pragma omp for schedule(dynamic, 8)
             for (int64_t i = 0; i < Sq; ++i) {
                 const uint8_t *mrow = mhead ? mhead + i * mask_si : NULL;
@@ -623,6 +814,7 @@ static int attn_bwd_impl(const uint16_t *q, const uint16_t *k, const uint16_t *v
                     if (!bwd_visible(i, j, Sq, Sk, causal, mrow)) {
                         prow[j] = -INFINITY;
                         dprow[j] = 0.0;
+                        zrow[j] = 0.0;
                         continue;
                     }
                     double dot = 0.0, dp = 0.0;
@@ -630,8 +822,9 @@ static int attn_bwd_impl(const uint16_t *q, const uint16_t *k, const uint16_t *v
                         dot += qi[d] * kh[j * D + d];
                         dp += doi[d] * vh[j * D + d];
                     }
+                    zrow[j] = drop ? (dropout_keep(seed, offset, p8, bh, i, j) ? zs : 0.0) : 1.0;
                     prow[j] = sc * dot;
-                    dprow[j] = dp;
+                    dprow[j] = zrow[j] * dp;
                     if (prow[j] > m) m = prow[j];
                 }
                 double l = 0.0;
@@ -648,7 +841,8 @@ static int attn_bwd_impl(const uint16_t *q, const uint16_t *k, const uint16_t *v
                 /* 2 sum_d |dO_id| sum_j P_ij |v_jd| */
                 for (int64_t d = 0; d < Dd; ++d) {
                     double od = 0.0;
-                    for (int64_t j = 0; j < nj; ++j) od += prow[j] * fabs(vh[j * D + d]);
+                    for (int64_t j = 0; j < nj; ++j)
+                        if (prow[j] > 0.0) od += prow[j] * zrow[j] * fabs(vh[j * D + d]);
                     as += 2.0 * fabs(doi[d]) * od;
                 }
                 lse[i] = m + log(l);
@@ -663,7 +857,7 @@ static int attn_bwd_impl(const uint16_t *q, const uint16_t *k, const uint16_t *v
                     }
                 }
             }
-            free(prow); free(dprow);
+            free(prow); free(dprow); free(zrow);
         }
         /* pass 2, per key: dK and dV over the queries that see it */
 #pragma omp parallel for schedule(dynamic, 8)
@@ -684,13 +878,15 @@ static int attn_bwd_impl(const uint16_t *q, const uint16_t *k, const uint16_t *v
                     dp += doi[d] * vj[d];
                 }
                 const double p = exp(sc * dot - lse[i]);
+                const double z = drop ? (dropout_keep(seed, offset, p8, bh, i, j) ? zs : 0.0) : 1.0;
+                dp *= z;
                 const double g = sc * p * (dp - dsum[i]);
                 const double gm = sc * p * (fabs(dp) + asum[i]);
                 for (int64_t d = 0; d < D; ++d) {
                     dkh[j * D + d] += g * qi[d];
-                    dvh[j * D + d] += p * doi[d];
+                    dvh[j * D + d] += p * z * doi[d];
                     if (mkh) mkh[j * D + d] += gm * fabs(qi[d]);
-                    if (mvh) mvh[j * D + d] += p * fabs(doi[d]);
+                    if (mvh) mvh[j * D + d] += p * z * fabs(doi[d]);
                 }
             }
         }
@@ -703,8 +899,18 @@ int oracle_attn_bwd(const uint16_t *q, const uint16_t *k, const uint16_t *v, con
                     int64_t H, int64_t Sq, int64_t Sk, int64_t D, float scale, int causal, int dtype, double *dq,
                     double *dk, double *dv, double *mag_dq, double *mag_dk, double *mag_dv)
 {
-    return attn_bwd_impl(q, k, v, dout, B, H, Sq, Sk, D, scale, causal, dtype, NULL, 0, 0, 0, dq, dk, dv, mag_dq,
-                         mag_dk, mag_dv);
+    return attn_bwd_impl(q, k, v, dout, B, H, Sq, Sk, D, scale, causal, dtype, NULL, 0, 0, 0, 0, 0, 0, 0, dq, dk, dv,
+                         mag_dq, mag_dk, mag_dv);
+}
+
+/* The gradients of the attention with dropout of oracle_attn_fwd_dropout. */
+int oracle_attn_bwd_dropout(const uint16_t *q, const uint16_t *k, const uint16_t *v, const uint16_t *dout,
+                            int64_t B, int64_t H, int64_t Sq, int64_t Sk, int64_t D, float scale, int causal,
+                            int dtype, uint32_t p8, uint64_t seed, uint32_t offset, double *dq, double *dk,
+                            double *dv, double *mag_dq, double *mag_dk, double *mag_dv)
+{
+    return attn_bwd_impl(q, k, v, dout, B, H, Sq, Sk, D, scale, causal, dtype, NULL, 0, 0, 0, 1, p8, seed, offset,
+                         dq, dk, dv, mag_dq, mag_dk, mag_dv);
 }
 
 /* The gradients of the masked attention of oracle_attn_fwd_masked (same mask
@@ -715,8 +921,8 @@ int oracle_attn_bwd_masked(const uint16_t *q, const uint16_t *k, const uint16_t 
                            int dtype, const uint8_t *mask, int64_t mask_sb, int64_t mask_sh, int64_t mask_si,
                            double *dq, double *dk, double *dv, double *mag_dq, double *mag_dk, double *mag_dv)
 {
-    return attn_bwd_impl(q, k, v, dout, B, H, Sq, Sk, D, scale, causal, dtype, mask, mask_sb, mask_sh, mask_si, dq,
-                         dk, dv, mag_dq, mag_dk, mag_dv);
+    return attn_bwd_impl(q, k, v, dout, B, H, Sq, Sk, D, scale, causal, dtype, mask, mask_sb, mask_sh, mask_si, 0, 0,
+                         0, 0, dq, dk, dv, mag_dq, mag_dk, mag_dv);
 }
 
 /* ------------------------------------------------------------ explicit mask */
