@@ -58,7 +58,7 @@ typedef enum {
     FA_ERR_LAUNCH = -7,   /* a CUDA runtime error (launch, tensor-map encoding, sync) */
     FA_ERR_TIMEOUT = -8,  /* a device-side wait exceeded its bound (reported by fa_check_status) */
     FA_ERR_SCALE = -9,    /* scale is not finite and > 0 */
-    FA_ERR_ARG = -10,     /* causal (or fa_bwd's deterministic) is not 0 or 1 */
+    FA_ERR_ARG = -10,     /* causal (or fa_bwd's deterministic) is not 0 or 1, or dropout_p is out of range */
     FA_ERR_PTR = -11,     /* a pointer is not device memory of the current device */
     FA_ERR_STRIDE = -12,  /* fa_fwd_ex: a stride is negative, zero over an extent > 1, not a
                              multiple of 8 elements (16 bytes), or not below 2^36 elements */
@@ -253,6 +253,49 @@ FA_API int fa_bwd_mask(const void* q, const void* k, const void* v, const void* 
                        const float* lse, void* dq, void* dk, void* dv, void* workspace, long long workspace_bytes,
                        int B, int H, int Sq, int Sk, int D, const void* mask, const long long* mask_stride,
                        float scale, int causal, int deterministic, int dtype, cudaStream_t stream);
+
+/*
+ * fa_fwd_dropout -- fa_fwd_ex (contiguous BHSD, Sq queries, Sk keys, bottom-right
+ * causal mask) with attention dropout fused into the kernel: after the softmax
+ * each weight P_ij is kept or zeroed, and the kept weights are scaled by
+ * 1 / (1 - p), so O_i = sum_j P_ij z_ij v_j with z_ij in {0, 1 / (1 - p)}
+ * ("FlashAttention-2 在昇腾 NPU 上如何做到 3 倍加速？", sections 3.4 and 6.3: dropout
+ * fused into the kernel with random numbers drawn on the device).  The LSE is
+ * that of the undropped softmax (what fa_bwd_dropout needs).
+ *
+ * The keep decisions are reproducible from (seed, offset): for head
+ * bh = b * H + h, query row i and key j, Philox4x32-10 (Salmon, Moraes, Dror,
+ * Shaw, "Parallel Random Numbers: As Easy as 1, 2, 3", SC 2011) of the
+ * counter (j / 16, i, bh, offset) under the key (seed mod 2^32, seed / 2^32)
+ * gives four 32-bit words; key j takes byte j mod 16 of them (word
+ * (j mod 16) / 4, little-endian byte j mod 4) and is kept iff that byte is
+ * >= p8 = floor(256 dropout_p + 1/2).  The drop probability is therefore
+ * p8 / 256 and the kept weights are scaled by 256 / (256 - p8).
+ *
+ * dropout_p : 0 <= dropout_p and p8 <= 255 (else FA_ERR_ARG); 0 keeps every
+ *             weight (the result equals fa_fwd_ex's).
+ * seed, offset : the generator's key and the counter's last word; use a new
+ *             offset (or seed) for every call that needs fresh decisions.
+ * D = 64 or 128 (else FA_ERR_HEADDIM).  Other arguments, ownership and errors
+ * as fa_fwd_ex with NULL strides.
+ */
+FA_API int fa_fwd_dropout(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Sq,
+                          int Sk, int D, float scale, int causal, float dropout_p, unsigned long long seed,
+                          unsigned int offset, int dtype, cudaStream_t stream);
+
+/*
+ * fa_bwd_dropout -- fa_bwd for the attention with dropout of fa_fwd_dropout:
+ * with the same dropout_p, seed and offset the kernel regenerates the same
+ * keep decisions, and dV_j = sum_i P_ij z_ij dO_i, dP_ij = z_ij dO_i . v_j,
+ * dS_ij = P_ij (dP_ij - dO_i . O_i).  o and lse must come from fa_fwd_dropout
+ * with the same arguments.  D = 64 or 128; other arguments, modes and errors
+ * as fa_bwd; dropout_p as fa_fwd_dropout.
+ */
+FA_API int fa_bwd_dropout(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                          const float* lse, void* dq, void* dk, void* dv, void* workspace, long long workspace_bytes,
+                          int B, int H, int Sq, int Sk, int D, float scale, int causal, float dropout_p,
+                          unsigned long long seed, unsigned int offset, int deterministic, int dtype,
+                          cudaStream_t stream);
 
 /*
  * fa_merge_partial -- fold a partial attention result into a running one by

@@ -222,3 +222,18 @@ def test_merge_entries_reject_bad_arguments(lib):
     assert fa.fa_merge_finalize(A, A, -1, 1, 0) == _lib.FA_ERR_SHAPE
     assert fa.fa_merge_finalize(A, A + 1, 10, 1, 0) == _lib.FA_ERR_ALIGN
     assert fa.fa_merge_finalize(0, 0, 0, 1, 0) == _lib.FA_OK
+
+
+def test_dropout_entries_reject_bad_arguments(lib):
+    ok = dict(B=1, H=1, Sq=128, Sk=128, D=128)
+    args = lambda p, D=128, B=1: (A, A, A, A, A, B, 1, 128, 128, D, 0.1, 0, p, 1, 0, 1, 0)  # noqa: E731
+    for p in (-0.1, float("nan"), float("inf"), 1.0, 255.5 / 256):
+        assert fa.fa_fwd_dropout(*args(p)) == _lib.FA_ERR_ARG, p
+    assert fa.fa_fwd_dropout(*args(0.2, D=256)) == _lib.FA_ERR_HEADDIM
+    assert fa.fa_fwd_dropout(*args(0.2, B=0)) == _lib.FA_OK  # empty problem, nothing launched
+    assert fa.fa_fwd_dropout(*args(0.2, B=-1)) == _lib.FA_ERR_SHAPE
+    bargs = lambda p, D=128: (A,) * 10 + (1 << 20, 1, 1, 128, 128, D, 0.1, 0, p, 1, 0, 0, 1, 0)  # noqa: E731
+    for p in (-0.5, float("nan"), 1.0):
+        assert fa.fa_bwd_dropout(*bargs(p)) == _lib.FA_ERR_ARG, p
+    assert fa.fa_bwd_dropout(*bargs(0.1, D=256)) == _lib.FA_ERR_HEADDIM
+    assert ok  # the shapes above are otherwise valid

@@ -8,12 +8,13 @@ in Python or PyTorch, and there is no fallback path.
 """
 from __future__ import annotations
 
-from ._lib import (FA_BF16, FA_FP16, FaError, fa_bwd, fa_bwd_mask, fa_bwd_workspace_size, fa_check_status, fa_fwd, fa_fwd_ex,
-                   fa_fwd_mask, fa_fwd_noalloc, fa_merge_finalize, fa_merge_partial, fa_last_timeout_site, fa_num_units, fa_selftest_timeout, fa_status_string,
+from ._lib import (FA_BF16, FA_FP16, FaError, fa_bwd, fa_bwd_dropout, fa_bwd_mask, fa_bwd_workspace_size,
+                   fa_check_status, fa_fwd, fa_fwd_dropout, fa_fwd_ex, fa_fwd_mask, fa_fwd_noalloc, fa_merge_finalize, fa_merge_partial, fa_last_timeout_site, fa_num_units, fa_selftest_timeout, fa_status_string,
                    fa_version, load)
 
 __all__ = [
-    "FA_BF16", "FA_FP16", "FaError", "fa_bwd", "fa_bwd_mask", "fa_bwd_workspace_size", "fa_check_status", "fa_fwd", "fa_fwd_ex",
+    "FA_BF16", "FA_FP16", "FaError", "fa_bwd", "fa_bwd_dropout", "fa_bwd_mask", "fa_bwd_workspace_size",
+    "fa_check_status", "fa_fwd", "fa_fwd_dropout", "fa_fwd_ex",
     "fa_fwd_mask", "fa_merge_finalize", "fa_merge_partial", "flash_attention_backward",
     "fa_fwd_noalloc", "fa_last_timeout_site",
     "fa_num_units", "fa_selftest_timeout", "fa_status_string", "fa_version", "flash_attention_forward", "load",
@@ -29,7 +30,8 @@ def _dtype_code(t) -> int:
     raise TypeError(f"unsupported dtype {t.dtype}; expected float16 or bfloat16")
 
 
-def flash_attention_forward(q, k, v, scale: float, causal: bool = False, out=None, lse=None, stream=None):
+def flash_attention_forward(q, k, v, scale: float, causal: bool = False, out=None, lse=None, stream=None,
+                            dropout_p: float = 0.0, seed: int = 0, offset: int = 0):
     """O, LSE for CUDA tensors ``q`` [B, H, Sq, D] and ``k, v`` [B, H, Sk, D] (fp16/bf16).
 
     The tensors may be any strided views whose last dimension is contiguous
@@ -40,6 +42,10 @@ def flash_attention_forward(q, k, v, scale: float, causal: bool = False, out=Non
     (contiguous float32 [B, H, Sq]) may be given to reuse buffers; by default
     ``out`` takes ``q``'s memory layout.  Launches on ``stream`` (default:
     torch's current stream) and returns without synchronising.
+
+    ``dropout_p`` > 0 applies attention dropout after the softmax
+    (fa_fwd_dropout: contiguous tensors; the keep decisions are fixed by
+    ``seed`` and ``offset``, which flash_attention_backward must be given too).
     """
     import torch
     if q.dim() != 4 or k.dim() != 4 or v.shape != k.shape:
@@ -67,6 +73,14 @@ def flash_attention_forward(q, k, v, scale: float, causal: bool = False, out=Non
         stream = torch.cuda.current_stream(q.device)
     st = int(stream.cuda_stream)
     dt = _dtype_code(q)
+    if dropout_p != 0.0:
+        if not all(t.is_contiguous() for t in (q, k, v, out)):
+            raise ValueError("dropout needs contiguous q, k, v and out")
+        rc = fa_fwd_dropout(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(), B, H, Sq, Sk,
+                            D, float(scale), int(bool(causal)), float(dropout_p), int(seed), int(offset), dt, st)
+        if rc != 0:
+            raise FaError(rc, "fa_fwd_dropout")
+        return out, lse
     if Sq == Sk and all(t.is_contiguous() for t in (q, k, v, out)):
         rc = fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(), B, H, Sq, D,
                     float(scale), int(bool(causal)), dt, st)
@@ -80,12 +94,14 @@ def flash_attention_forward(q, k, v, scale: float, causal: bool = False, out=Non
 
 
 def flash_attention_backward(q, k, v, o, lse, dout, scale: float, causal: bool = False, deterministic: bool = False,
-                             dq=None, dk=None, dv=None, workspace=None, stream=None):
+                             dq=None, dk=None, dv=None, workspace=None, stream=None, dropout_p: float = 0.0,
+                             seed: int = 0, offset: int = 0):
     """dQ, dK, dV for contiguous BHSD CUDA tensors (q, o, dout [B, H, Sq, D];
     k, v [B, H, Sk, D]; lse [B, H, Sq] fp32 from the forward call).  The
     workspace (fa_bwd_workspace_size bytes) is allocated with torch unless
     given.  Launches on ``stream`` (default: torch's current stream) and
-    returns without synchronising."""
+    returns without synchronising.  ``dropout_p``, ``seed`` and ``offset``
+    must be those of the forward call (fa_bwd_dropout when dropout_p > 0)."""
     import torch
     B, H, Sq, D = q.shape
     Sk = k.shape[2]
@@ -106,6 +122,14 @@ def flash_attention_backward(q, k, v, o, lse, dout, scale: float, causal: bool =
         workspace = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=q.device)
     if stream is None:
         stream = torch.cuda.current_stream(q.device)
+    if dropout_p != 0.0:
+        rc = fa_bwd_dropout(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), dout.data_ptr(), lse.data_ptr(),
+                            dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), workspace.data_ptr(), workspace.numel(), B, H,
+                            Sq, Sk, D, float(scale), int(bool(causal)), float(dropout_p), int(seed), int(offset),
+                            int(bool(deterministic)), _dtype_code(q), int(stream.cuda_stream))
+        if rc != 0:
+            raise FaError(rc, "fa_bwd_dropout")
+        return dq, dk, dv
     rc = fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), dout.data_ptr(), lse.data_ptr(),
                 dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), workspace.data_ptr(), workspace.numel(), B, H, Sq, Sk, D,
                 float(scale), int(bool(causal)), int(bool(deterministic)), _dtype_code(q), int(stream.cuda_stream))

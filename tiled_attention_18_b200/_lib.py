@@ -59,6 +59,13 @@ SIGNATURES = [
      [ctypes.c_void_p] * 10 + [ctypes.c_longlong, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                ctypes.c_int, ctypes.c_void_p, _LL3, ctypes.c_float, ctypes.c_int, ctypes.c_int,
                                ctypes.c_int, ctypes.c_void_p]),
+    ("fa_fwd_dropout", ctypes.c_int,
+     [ctypes.c_void_p] * 5 + [ctypes.c_int] * 5 + [ctypes.c_float, ctypes.c_int, ctypes.c_float, ctypes.c_ulonglong,
+                                                ctypes.c_uint, ctypes.c_int, ctypes.c_void_p]),
+    ("fa_bwd_dropout", ctypes.c_int,
+     [ctypes.c_void_p] * 10 + [ctypes.c_longlong, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                               ctypes.c_int, ctypes.c_float, ctypes.c_int, ctypes.c_float, ctypes.c_ulonglong,
+                               ctypes.c_uint, ctypes.c_int, ctypes.c_int, ctypes.c_void_p]),
     ("fa_merge_partial", ctypes.c_int,
      [ctypes.c_void_p] * 4 + [ctypes.c_longlong, ctypes.c_int, ctypes.c_int, ctypes.c_void_p]),
     ("fa_merge_finalize", ctypes.c_int,
@@ -160,6 +167,26 @@ def fa_bwd_mask(q_ptr: int, k_ptr: int, v_ptr: int, o_ptr: int, do_ptr: int, lse
     return int(load().fa_bwd_mask(q_ptr, k_ptr, v_ptr, o_ptr, do_ptr, lse_ptr, dq_ptr, dk_ptr, dv_ptr, ws_ptr,
                                   int(ws_bytes), B, H, Sq, Sk, D, mask_ptr, _strides(mask_stride), float(scale),
                                   int(causal), int(deterministic), int(dtype), stream))
+
+
+def fa_fwd_dropout(q_ptr: int, k_ptr: int, v_ptr: int, o_ptr: int, lse_ptr: int, B: int, H: int, Sq: int, Sk: int,
+                   D: int, scale: float, causal: int, dropout_p: float, seed: int, offset: int, dtype: int,
+                   stream: int) -> int:
+    """Raw C call of the forward pass with dropout (see include/fa.h)."""
+    return int(load().fa_fwd_dropout(q_ptr, k_ptr, v_ptr, o_ptr, lse_ptr, B, H, Sq, Sk, D, float(scale), int(causal),
+                                     float(dropout_p), int(seed) & (2**64 - 1), int(offset) & 0xffffffff, int(dtype),
+                                     stream))
+
+
+def fa_bwd_dropout(q_ptr: int, k_ptr: int, v_ptr: int, o_ptr: int, do_ptr: int, lse_ptr: int, dq_ptr: int,
+                   dk_ptr: int, dv_ptr: int, ws_ptr: int, ws_bytes: int, B: int, H: int, Sq: int, Sk: int, D: int,
+                   scale: float, causal: int, dropout_p: float, seed: int, offset: int, deterministic: int,
+                   dtype: int, stream: int) -> int:
+    """Raw C call of the backward pass with dropout (see include/fa.h)."""
+    return int(load().fa_bwd_dropout(q_ptr, k_ptr, v_ptr, o_ptr, do_ptr, lse_ptr, dq_ptr, dk_ptr, dv_ptr, ws_ptr,
+                                     int(ws_bytes), B, H, Sq, Sk, D, float(scale), int(causal), float(dropout_p),
+                                     int(seed) & (2**64 - 1), int(offset) & 0xffffffff, int(deterministic),
+                                     int(dtype), stream))
 
 
 def fa_merge_partial(o_acc_ptr: int, lse_acc_ptr: int, o_part_ptr: int, lse_part_ptr: int, rows: int, D: int,

@@ -158,6 +158,22 @@ long long fa_num_units(int B, int H, int S) {
 
 namespace {
 
+// Dropout probability -> threshold in 1/256 units (nearest, halves up) and the
+// scale of the kept weights; false when p is not finite, negative or rounds to
+// 256 (every weight dropped).
+bool make_dropout(float p, unsigned long long seed, unsigned int offset, fa::DropoutArgs* d) {
+    if (!std::isfinite(p) || p < 0.f) return false;
+    const double t = std::floor((double)p * 256.0 + 0.5);
+    if (t > 255.0) return false;
+    d->enabled = 1;
+    d->p8 = (uint32_t)t;
+    d->seed_lo = (uint32_t)(seed & 0xffffffffull);
+    d->seed_hi = (uint32_t)(seed >> 32);
+    d->offset = offset;
+    d->keep_scale = (float)(256.0 / (256.0 - t));
+    return true;
+}
+
 // Where the causal scheduler's counter lives.
 enum class Scratch { Allocated, Static };
 
@@ -166,9 +182,10 @@ enum class Scratch { Allocated, Static };
 int forward(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Sq, int Sk, int D,
             const long long* q_stride, const long long* k_stride, const long long* v_stride,
             const long long* o_stride, float scale, int causal, int dtype, cudaStream_t stream, Scratch scratch,
-            const uint8_t* mask = nullptr, const long long* mask_stride = nullptr) {
+            const uint8_t* mask = nullptr, const long long* mask_stride = nullptr,
+            const fa::DropoutArgs* drop = nullptr) {
     if (B < 0 || H < 0 || Sq < 0 || Sk < 0) return FA_ERR_SHAPE;
-    if (D != 64 && D != 128 && !(D == 256 && !mask)) return FA_ERR_HEADDIM;
+    if (D != 64 && D != 128 && !(D == 256 && !mask && !drop)) return FA_ERR_HEADDIM;
     if (dtype != FA_FP16 && dtype != FA_BF16) return FA_ERR_DTYPE;
     if (!(std::isfinite(scale) && scale > 0.f)) return FA_ERR_SCALE;
     if (causal != 0 && causal != 1) return FA_ERR_ARG;
@@ -225,6 +242,7 @@ int forward(const void* q, const void* k, const void* v, void* o, float* lse, in
     for (int i = 0; i < 3; ++i) a.o_stride[i] = os[i];
     a.mask = mask;
     for (int i = 0; i < 3; ++i) a.mask_stride[i] = ms[i];
+    if (drop) a.drop = *drop;
     a.B = B;
     a.H = H;
     a.Sq = Sq;
@@ -285,6 +303,17 @@ int fa_fwd_mask(const void* q, const void* k, const void* v, void* o, float* lse
                    Scratch::Allocated, static_cast<const uint8_t*>(mask), mask_stride);
 }
 
+int fa_fwd_dropout(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Sq, int Sk,
+                   int D, float scale, int causal, float dropout_p, unsigned long long seed, unsigned int offset,
+                   int dtype, cudaStream_t stream) {
+    fa::DropoutArgs d;
+    std::memset(&d, 0, sizeof(d));
+    if (!make_dropout(dropout_p, seed, offset, &d)) return FA_ERR_ARG;
+    if (D == 256) return FA_ERR_HEADDIM;
+    return forward(q, k, v, o, lse, B, H, Sq, Sk, D, nullptr, nullptr, nullptr, nullptr, scale, causal, dtype, stream,
+                   Scratch::Allocated, nullptr, nullptr, &d);
+}
+
 int fa_fwd_ex(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Sq, int Sk, int D,
               const long long* q_stride, const long long* k_stride, const long long* v_stride,
               const long long* o_stride, float scale, int causal, int dtype, cudaStream_t stream) {
@@ -318,7 +347,7 @@ namespace {
 int backward(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse, void* dq,
              void* dk, void* dv, void* workspace, long long workspace_bytes, int B, int H, int Sq, int Sk, int D,
              float scale, int causal, int deterministic, int dtype, cudaStream_t stream, const uint8_t* mask,
-             const long long* mask_stride) {
+             const long long* mask_stride, const fa::DropoutArgs* drop = nullptr) {
     if (B < 0 || H < 0 || Sq < 0 || Sk < 0) return FA_ERR_SHAPE;
     if (D != 64 && D != 128) return FA_ERR_HEADDIM;
     if (dtype != FA_FP16 && dtype != FA_BF16) return FA_ERR_DTYPE;
@@ -391,6 +420,7 @@ int backward(const void* q, const void* k, const void* v, const void* o, const v
     a.sched = reinterpret_cast<unsigned int*>(w + ws.sched);
     a.mask = mask;
     for (int i = 0; i < 3; ++i) a.mask_stride[i] = ms[i];
+    if (drop) a.drop = *drop;
     a.dq_flags = nullptr;
     if (deterministic) {
         a.dq_flags = reinterpret_cast<int*>(w + ws.flags);
@@ -439,6 +469,17 @@ int fa_bwd_mask(const void* q, const void* k, const void* v, const void* o, cons
     if (B > 0 && H > 0 && Sq > 0 && (!mask || !mask_stride)) return FA_ERR_NULL;
     return backward(q, k, v, o, dout, lse, dq, dk, dv, workspace, workspace_bytes, B, H, Sq, Sk, D, scale, causal,
                     deterministic, dtype, stream, static_cast<const uint8_t*>(mask), mask_stride);
+}
+
+int fa_bwd_dropout(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
+                   void* dq, void* dk, void* dv, void* workspace, long long workspace_bytes, int B, int H, int Sq,
+                   int Sk, int D, float scale, int causal, float dropout_p, unsigned long long seed,
+                   unsigned int offset, int deterministic, int dtype, cudaStream_t stream) {
+    fa::DropoutArgs d;
+    std::memset(&d, 0, sizeof(d));
+    if (!make_dropout(dropout_p, seed, offset, &d)) return FA_ERR_ARG;
+    return backward(q, k, v, o, dout, lse, dq, dk, dv, workspace, workspace_bytes, B, H, Sq, Sk, D, scale, causal,
+                    deterministic, dtype, stream, nullptr, nullptr, &d);
 }
 
 int fa_merge_partial(float* o_acc, float* lse_acc, const void* o_part, const float* lse_part, long long rows, int D,

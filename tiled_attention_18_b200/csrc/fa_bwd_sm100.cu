@@ -131,6 +131,10 @@ struct BwdParams {
     float scale_log2;     // scale * log2(e)
     float scale;
     unsigned int* sched;  // zeroed unit counter (causal), or null
+    // dropout: on/off, threshold in every byte, generator key, counter word 3, 1 / (1 - p)
+    int drop;
+    uint32_t drop_p8x4, seed_lo, seed_hi, drop_offset;
+    float keep_scale;
 };
 
 struct BUnit {
@@ -255,6 +259,32 @@ __device__ __forceinline__ uint32_t mask_col_bits(const uint8_t* mhead, long lon
     } else {
         for (int c = 0; c < Sk - key0; ++c)
             if (r[c]) rowbits |= 1u << c;
+    }
+    uint32_t col = 0u;
+#pragma unroll
+    for (int kk = 0; kk < 32; ++kk) {
+        const uint32_t bal = __ballot_sync(0xffffffffu, (rowbits >> kk) & 1u);
+        if (lane == kk) col = bal;
+    }
+    return col;
+}
+
+// Dropout keep decisions in the same transposed form: for this lane's key
+// (key0 + lane) the bits of queries q0 .. q0 + 31 (bit i set = the weight of
+// query q0 + i is kept).  Lane i draws the two generator blocks of query
+// q0 + i over keys key0 .. key0 + 31 (key0 a multiple of 16), folds their
+// keep bytes into 32 bits, and 32 ballots transpose the warp's block.
+__device__ __forceinline__ uint32_t dropout_col_bits(const BwdParams& p, int bh, int q0, int key0) {
+    const int lane = threadIdx.x & 31;
+    const uint32_t q = (uint32_t)(q0 + lane), g = (uint32_t)key0 >> 4;
+    const uint4 a = dropout_keep_bytes(g, q, (uint32_t)bh, p.drop_offset, p.seed_lo, p.seed_hi, p.drop_p8x4);
+    const uint4 b = dropout_keep_bytes(g + 1u, q, (uint32_t)bh, p.drop_offset, p.seed_lo, p.seed_hi, p.drop_p8x4);
+    const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+    uint32_t rowbits = 0u;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+        const uint32_t t = w[e] & 0x01010101u;  // one byte per key: 1 kept, 0 dropped
+        rowbits |= ((t * 0x01020408u) >> 24 & 0xFu) << (4 * e);
     }
     uint32_t col = 0u;
 #pragma unroll
@@ -506,6 +536,10 @@ __device__ void bwd_ds_role(const BwdParams& p, uint8_t* smem, uint32_t tmem, in
                 const uint32_t mbits = p.mask ? mask_col_bits(mhead, p.m_ss, p.Sq, p.Sk, m * TILE + 32 * c,
                                                               U.n * TILE + warp_in_group * 32)
                                               : 0xffffffffu;
+                // dropout: this key's keep bits over the chunk's 32 queries
+                const uint32_t zbits =
+                    p.drop ? dropout_col_bits(p, U.bh, m * TILE + 32 * c, U.n * TILE + warp_in_group * 32)
+                           : 0xffffffffu;
                 uint32_t sr[32], dr[32];
                 tmem_ld32u(tmem + lane_sel + COL_S + 32 * c, sr);
                 tmem_ld32u(tmem + lane_sel + COL_DP + 32 * c, dr);
@@ -522,9 +556,15 @@ __device__ void bwd_ds_role(const BwdParams& p, uint8_t* smem, uint32_t tmem, in
                         if (!key_ok || q < q_min || !((mbits >> (2 * i)) & 1u)) p0 = 0.f;
                         if (!key_ok || q + 1 < q_min || !((mbits >> (2 * i + 1)) & 1u)) p1 = 0.f;
                     }
-                    const float d0 = p0 * (__uint_as_float(dr[2 * i]) - dl.x);
-                    const float d1 = p1 * (__uint_as_float(dr[2 * i + 1]) - dl.y);
-                    pk[i] = pack2<BF16>(p0, p1);
+                    // dropout factors: 1 / (1 - p) for a kept weight, 0 for a dropped one
+                    float z0 = 1.f, z1 = 1.f;
+                    if (p.drop) {
+                        z0 = ((zbits >> (2 * i)) & 1u) ? p.keep_scale : 0.f;
+                        z1 = ((zbits >> (2 * i + 1)) & 1u) ? p.keep_scale : 0.f;
+                    }
+                    const float d0 = p0 * (__uint_as_float(dr[2 * i]) * z0 - dl.x);
+                    const float d1 = p1 * (__uint_as_float(dr[2 * i + 1]) * z1 - dl.y);
+                    pk[i] = pack2<BF16>(p0 * z0, p1 * z1);
                     dk[i] = pack2<BF16>(d0, d1);
                 }
                 tmem_st16(tmem + lane_sel + COL_S + 16 * c, pk);
@@ -968,7 +1008,7 @@ __device__ void bwd2_mma(const BwdParams& p, uint8_t* smem, uint32_t tmem, volat
     mbar_drain(bar(L::B_FIN), 0u);
 }
 
-template <bool BF16, bool MASK>
+template <bool BF16, bool MASK, bool DROP>
 __device__ void bwd2_ds_role(const BwdParams& p, uint8_t* smem, uint32_t tmem, int warp_in_group, int c,
                              volatile uint32_t* abort_flag) {
     using L = Bwd2Smem;
@@ -1011,6 +1051,9 @@ __device__ void bwd2_ds_role(const BwdParams& p, uint8_t* smem, uint32_t tmem, i
             uint32_t mbits = 0xffffffffu;
             if constexpr (MASK)
                 mbits = mask_col_bits(mhead, p.m_ss, p.Sq, p.Sk, m * QM + 32 * c, U.n * TILE + warp_in_group * 32);
+            // dropout: this key's keep bits over the same 32 queries
+            uint32_t zbits = 0xffffffffu;
+            if constexpr (DROP) zbits = dropout_col_bits(p, U.bh, m * QM + 32 * c, U.n * TILE + warp_in_group * 32);
             uint8_t* ds_row = smem + L::DS_OFF + b * L::DS_BYTES + (row >> 3) * 1024 + (row & 7) * 128;
             {
                 uint32_t sr[32], dr[32];
@@ -1029,9 +1072,15 @@ __device__ void bwd2_ds_role(const BwdParams& p, uint8_t* smem, uint32_t tmem, i
                         if (!key_ok || q < q_min || !((mbits >> (2 * i)) & 1u)) p0 = 0.f;
                         if (!key_ok || q + 1 < q_min || !((mbits >> (2 * i + 1)) & 1u)) p1 = 0.f;
                     }
-                    pk[i] = pack2<BF16>(p0, p1);
-                    dk[i] = pack2<BF16>(p0 * (__uint_as_float(dr[2 * i]) - dl.x),
-                                        p1 * (__uint_as_float(dr[2 * i + 1]) - dl.y));
+                    // dropout factors: 1 / (1 - p) for a kept weight, 0 for a dropped one
+                    float z0 = 1.f, z1 = 1.f;
+                    if constexpr (DROP) {
+                        z0 = ((zbits >> (2 * i)) & 1u) ? p.keep_scale : 0.f;
+                        z1 = ((zbits >> (2 * i + 1)) & 1u) ? p.keep_scale : 0.f;
+                    }
+                    pk[i] = pack2<BF16>(p0 * z0, p1 * z1);
+                    dk[i] = pack2<BF16>(p0 * (__uint_as_float(dr[2 * i]) * z0 - dl.x),
+                                        p1 * (__uint_as_float(dr[2 * i + 1]) * z1 - dl.y));
                 }
                 // packed into the first 16 of this warpgroup's own 32 columns: the other
                 // dS warpgroup may still be reading its raw scores from the rest
@@ -1156,7 +1205,7 @@ __device__ void bwd2_out_role(const BwdParams& p, uint8_t* smem, uint32_t tmem, 
     }
 }
 
-template <bool BF16, bool MASK>
+template <bool BF16, bool MASK, bool DROP>
 __global__ void __launch_bounds__(BWD2_THREADS, 1) fa_bwd_kernel_d128(const __grid_constant__ BwdParams p) {
     using L = Bwd2Smem;
     extern __shared__ uint8_t smem_raw[];
@@ -1201,7 +1250,7 @@ __global__ void __launch_bounds__(BWD2_THREADS, 1) fa_bwd_kernel_d128(const __gr
         if (warp == BW_MMA && lane == 0) bwd2_mma<BF16>(p, smem, tmem, abort_flag);
     } else if (wg == 1 || wg == 3) {
         setmaxnreg_inc<REG2_DS>();
-        bwd2_ds_role<BF16, MASK>(p, smem, tmem, warp & 3, wg == 1 ? 0 : 1, abort_flag);
+        bwd2_ds_role<BF16, MASK, DROP>(p, smem, tmem, warp & 3, wg == 1 ? 0 : 1, abort_flag);
     } else {
         setmaxnreg_dec<REG2_OUT>();
         bwd2_out_role<BF16>(p, smem, tmem, warp & 3, abort_flag);
@@ -1288,7 +1337,9 @@ cudaError_t launch_bwd_impl(const BwdLaunchArgs& a, cudaStream_t stream) {
     {
         // D = 128 runs the 64-row-step kernel (its Q/dO maps have 64-row boxes)
         void (*kern)(const BwdParams);
-        if constexpr (D == 128) kern = a.mask ? fa_bwd_kernel_d128<BF16, true> : fa_bwd_kernel_d128<BF16, false>;
+        if constexpr (D == 128)
+            kern = a.drop.enabled ? fa_bwd_kernel_d128<BF16, false, true>
+                                  : (a.mask ? fa_bwd_kernel_d128<BF16, true, false> : fa_bwd_kernel_d128<BF16, false, false>);
         else kern = fa_bwd_kernel<D, BF16>;
         const int alloc = (D == 128) ? Bwd2Smem::ALLOC : BwdSmem<64>::ALLOC;
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, alloc);
@@ -1329,6 +1380,12 @@ cudaError_t launch_bwd_impl(const BwdLaunchArgs& a, cudaStream_t stream) {
         p.m_sb = a.mask_stride[0];
         p.m_sh = a.mask_stride[1];
         p.m_ss = a.mask_stride[2];
+        p.drop = a.drop.enabled;
+        p.drop_p8x4 = a.drop.p8 * 0x01010101u;
+        p.seed_lo = a.drop.seed_lo;
+        p.seed_hi = a.drop.seed_hi;
+        p.drop_offset = a.drop.offset;
+        p.keep_scale = a.drop.enabled ? a.drop.keep_scale : 1.f;
         p.flag_steps = (D == 128) ? (a.Sq + QM - 1) / QM : n_mtiles;
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3((unsigned)a.grid, 1, 1);

@@ -188,6 +188,9 @@ struct KParams {
     long long m_sb, m_sh, m_ss;  // its element strides over b, h and the query row (keys contiguous)
     float scale_log2;
     unsigned int* sched;  // zeroed unit counter (claim order), or null for the static order
+    // dropout (DROP kernels): threshold in every byte, generator key, counter word 3, 1 / (1 - p)
+    uint32_t drop_p8x4, seed_lo, seed_hi, drop_offset;
+    float keep_scale;
 };
 
 // Threads that read each published unit index: MMA lane, two softmax
@@ -587,7 +590,7 @@ __device__ void mma_role(const KParams& p, uint8_t* smem, uint32_t tmem, volatil
     mbar_drain(bar(L::B_FIN), 0u);
 }
 
-template <int D, bool BF16, bool MASK>
+template <int D, bool BF16, bool MASK, bool DROP>
 __device__ void softmax_role(const KParams& p, uint8_t* smem, uint32_t tmem, int t, int warp_in_group,
                              volatile uint32_t* abort_flag) {
     using L = Smem<D>;
@@ -683,6 +686,17 @@ __device__ void softmax_role(const KParams& p, uint8_t* smem, uint32_t tmem, int
             // one pair in FMA_EXP2_PERIOD uses the FMA-pipe exp2.
             auto quarter_row = [&](int qr, bool use_fma_exp) {
                 uint32_t pk[16];
+                // dropout: keep masks of the quarter's 32 keys (two 16-key generator blocks)
+                uint32_t km[8];
+                if constexpr (DROP) {
+                    const uint32_t g0 = (uint32_t)(kbase + 32 * qr) >> 4;
+                    const uint4 a = dropout_keep_bytes(g0, (uint32_t)row, (uint32_t)U.bh, p.drop_offset, p.seed_lo,
+                                                       p.seed_hi, p.drop_p8x4);
+                    const uint4 b = dropout_keep_bytes(g0 + 1u, (uint32_t)row, (uint32_t)U.bh, p.drop_offset,
+                                                       p.seed_lo, p.seed_hi, p.drop_p8x4);
+                    km[0] = a.x; km[1] = a.y; km[2] = a.z; km[3] = a.w;
+                    km[4] = b.x; km[5] = b.y; km[6] = b.z; km[7] = b.w;
+                }
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
                     const float2 x = __ffma2_rn(make_float2(s[32 * qr + 2 * i], s[32 * qr + 2 * i + 1]), sl2x2, negm2);
@@ -700,6 +714,9 @@ __device__ void softmax_role(const KParams& p, uint8_t* smem, uint32_t tmem, int
                         // the rounded weights as the MMA sees them (bf16 -> fp32 is exact)
                         if (i & 1) rsum1 = add_bf16x2(rsum1, pk[i]); else rsum0 = add_bf16x2(rsum0, pk[i]);
                     }
+                    // the sums keep every weight; P.V sees only the kept ones (keys 2i and
+                    // 2i + 1 are bytes 2i and 2i + 1 of the quarter's mask: each byte fills a half)
+                    if constexpr (DROP) pk[i] &= __byte_perm(km[i >> 1], 0u, (i & 1) ? 0x3322u : 0x1100u);
                 }
                 // P (16-bit, two per column) overwrites the first 64 columns of S
                 tmem_st16(ts + 16 * qr, pk);
@@ -729,7 +746,7 @@ __device__ void softmax_role(const KParams& p, uint8_t* smem, uint32_t tmem, int
         // O = 0 and LSE = -inf
         const float norm = Policy<BF16>::NORM_BY_ROUNDED_P ? lr : l;
         fin_buf[fin_par * 2 * BLOCK_M] = (l > 0.f)
-            ? make_float2(1.f / norm, (m_use + __log2f(l)) * 0.69314718055994530942f)
+            ? make_float2((DROP ? p.keep_scale : 1.f) / norm, (m_use + __log2f(l)) * 0.69314718055994530942f)
             : make_float2(0.f, -INFINITY);
         mbar_arrive(bar(L::B_FINAL + 2 * fin_par + t));
         fin_par ^= 1;
@@ -840,7 +857,7 @@ __device__ void correction_role(const KParams& p, uint8_t* smem, uint32_t tmem, 
     }
 }
 
-template <int D, bool BF16, bool MASK>
+template <int D, bool BF16, bool MASK, bool DROP>
 __global__ void __launch_bounds__(NUM_THREADS, 1) fa_fwd_kernel(const __grid_constant__ KParams p) {
     using L = Smem<D>;
     extern __shared__ uint8_t smem_raw[];
@@ -884,7 +901,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) fa_fwd_kernel(const __grid_con
 
     if (wg < 2) {
         setmaxnreg_inc<REG_SOFTMAX>();
-        softmax_role<D, BF16, MASK>(p, smem, tmem, wg, warp & 3, abort_flag);
+        softmax_role<D, BF16, MASK, DROP>(p, smem, tmem, wg, warp & 3, abort_flag);
     } else if (wg == 2) {
         setmaxnreg_dec<REG_CORR>();
         correction_role<D, BF16>(p, smem, tmem, warp & 3, abort_flag);
@@ -941,11 +958,11 @@ __global__ void __launch_bounds__(64, 1) selftest_timeout_kernel(long long deadl
     }
 }
 
-template <int D, bool BF16, bool MASK>
+template <int D, bool BF16, bool MASK, bool DROP = false>
 cudaError_t launch_impl(const LaunchArgs& a, cudaStream_t stream) {
     using L = Smem<D>;
     static_assert(L::ALLOC <= 232448, "shared memory budget exceeded");
-    auto kern = fa_fwd_kernel<D, BF16, MASK>;
+    auto kern = fa_fwd_kernel<D, BF16, MASK, DROP>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC);
     if (e != cudaSuccess) return e;
     KParams p;
@@ -972,6 +989,11 @@ cudaError_t launch_impl(const LaunchArgs& a, cudaStream_t stream) {
     p.m_ss = a.mask_stride[2];
     p.scale_log2 = a.scale_log2;
     p.sched = a.sched;
+    p.drop_p8x4 = a.drop.p8 * 0x01010101u;
+    p.seed_lo = a.drop.seed_lo;
+    p.seed_hi = a.drop.seed_hi;
+    p.drop_offset = a.drop.offset;
+    p.keep_scale = a.drop.enabled ? a.drop.keep_scale : 1.f;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)a.grid, 1, 1);
     cfg.blockDim = dim3(NUM_THREADS, 1, 1);
@@ -985,6 +1007,12 @@ cudaError_t launch_impl(const LaunchArgs& a, cudaStream_t stream) {
 }  // namespace
 
 cudaError_t launch_fwd_sm100(const LaunchArgs& a, cudaStream_t stream) {
+    if (a.drop.enabled) {
+        if (a.D == 128)
+            return a.dtype == 1 ? launch_impl<128, true, false, true>(a, stream)
+                                : launch_impl<128, false, false, true>(a, stream);
+        return a.dtype == 1 ? launch_impl<64, true, false, true>(a, stream) : launch_impl<64, false, false, true>(a, stream);
+    }
     if (a.D == 128) {
         if (a.mask) return a.dtype == 1 ? launch_impl<128, true, true>(a, stream) : launch_impl<128, false, true>(a, stream);
         return a.dtype == 1 ? launch_impl<128, true, false>(a, stream) : launch_impl<128, false, false>(a, stream);

@@ -21,6 +21,18 @@ constexpr int DEV_TIMEOUT = 1;
 // Wait-site code of the diagnostic timeout kernel (low byte of the site word).
 constexpr int SELFTEST_SITE = 100;
 
+// Attention dropout after the softmax: the weight of query q and key j of
+// head bh is kept iff byte j mod 16 of Philox4x32-10(counter (j / 16, q, bh,
+// offset), key (seed_lo, seed_hi)) is >= p8; kept weights are scaled by
+// keep_scale = 256 / (256 - p8).
+struct DropoutArgs {
+    int enabled;
+    uint32_t p8;            // drop threshold in 1/256 units, 0 .. 255
+    uint32_t seed_lo, seed_hi;
+    uint32_t offset;
+    float keep_scale;
+};
+
 struct LaunchArgs {
     CUtensorMap tmap_q;     // 4-D maps over [B][H][S][D] (innermost first: D, S, H, B) with
     CUtensorMap tmap_k;     // the tensors' own strides, box {64, 128, 1, 1}, 128-byte swizzle
@@ -30,6 +42,7 @@ struct LaunchArgs {
     long long o_stride[3];  // element strides of O over b, h, s (d is contiguous)
     const uint8_t* mask;    // explicit boolean mask (nonzero = attend) or null
     long long mask_stride[3];  // its element strides over b, h, query row (keys contiguous)
+    DropoutArgs drop;       // dropout (drop.enabled = 0: none)
     int B;
     int H;
     int Sq;                 // query rows per head
@@ -63,6 +76,7 @@ struct BwdLaunchArgs {
     int* dq_flags;          // workspace: deterministic-mode turn counters, or null (atomic mode)
     const uint8_t* mask;    // explicit boolean mask or null
     long long mask_stride[3];
+    DropoutArgs drop;       // dropout (drop.enabled = 0: none)
     int B;
     int H;
     int Sq;

@@ -169,6 +169,33 @@ __device__ __forceinline__ void tmem_wait_st() {
     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
+// Philox4x32-10, the counter-based generator of Salmon, Moraes, Dror and Shaw
+// ("Parallel Random Numbers: As Easy as 1, 2, 3", SC 2011): ten rounds that
+// multiply words 0 and 2 by two fixed odd constants, keep the low halves and
+// fold the high halves into words 1 and 3 and the key; the key advances by
+// two Weyl increments between rounds.
+__device__ __forceinline__ uint4 philox4x32_10(uint4 c, uint32_t k0, uint32_t k1) {
+#pragma unroll
+    for (int r = 0; r < 10; ++r) {
+        const uint32_t lo0 = 0xD2511F53u * c.x, hi0 = __umulhi(0xD2511F53u, c.x);
+        const uint32_t lo1 = 0xCD9E8D57u * c.z, hi1 = __umulhi(0xCD9E8D57u, c.z);
+        c = make_uint4(hi1 ^ c.y ^ k0, lo1, hi0 ^ c.w ^ k1, lo0);
+        k0 += 0x9E3779B9u;
+        k1 += 0xBB67AE85u;
+    }
+    return c;
+}
+
+// Dropout keep masks of the 16 keys [16 g, 16 g + 16) of query q in head bh:
+// byte b of the result (word b / 4, little-endian byte b mod 4) is 0xFF when
+// key 16 g + b is kept (its random byte >= the threshold; p8x4 = the
+// threshold in every byte), 0x00 when it is dropped.
+__device__ __forceinline__ uint4 dropout_keep_bytes(uint32_t g, uint32_t q, uint32_t bh, uint32_t offset,
+                                                    uint32_t seed_lo, uint32_t seed_hi, uint32_t p8x4) {
+    const uint4 r = philox4x32_10(make_uint4(g, q, bh, offset), seed_lo, seed_hi);
+    return make_uint4(__vcmpgeu4(r.x, p8x4), __vcmpgeu4(r.y, p8x4), __vcmpgeu4(r.z, p8x4), __vcmpgeu4(r.w, p8x4));
+}
+
 __device__ __forceinline__ float ex2(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
