@@ -50,6 +50,7 @@ METRIC = "attention fwd TFLOPS (causal-adjusted) and % of B200 dense fp16/bf16 p
 UNIT = "TFLOP/s"
 FALLBACK_BF16_TFLOPS = 1590.0
 FALLBACK_HBM_GBS = 6650.0
+DROPOUT_SEED = 0x5EED5EED5EED
 PEAKS_PATH = os.path.join(ROOT, "MEASURED_PEAKS.json")
 TRAFFIC_PATH = os.path.join(ROOT, "profiles", "fa_fwd_traffic.json")
 KERNEL_SRC = os.path.join(ROOT, "tiled_attention_18_b200", "csrc", "fa_fwd_sm100.cu")
@@ -163,7 +164,7 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(self.samples)}
 
 
-def cpu_baseline(name: str, target_s: float = 12.0):
+def cpu_baseline(name: str, target_s: float = 12.0, dropout: float = 0.0):
     """Time the oracle on a bounded row sample of the workload; TFLOP/s of the sample."""
     import oracle
     runs = workload_runs(name)
@@ -177,7 +178,10 @@ def cpu_baseline(name: str, target_s: float = 12.0):
         while True:
             bh, rows = sample_rows(w.B, w.H, w.S, n_random=n, edge=0, seed=99)
             t0 = time.perf_counter()
-            if w.general:
+            if dropout > 0.0:
+                oracle.attn_rows_dropout(q, k, v, w.scale, w.causal, w.dtype, int(np.floor(dropout * 256 + 0.5)),
+                                         DROPOUT_SEED, 0, bh, rows)
+            elif w.general:
                 oracle.attn_rows_gen(q, k, v, w.scale, w.causal, w.dtype, bh, rows)
             else:
                 oracle.attn_rows(q, k, v, w.scale, w.causal, w.dtype, bh, rows)
@@ -281,8 +285,12 @@ def run_bwd(args) -> int:
         o = torch.empty_like(q)
         lse = torch.empty(q.shape[:3], dtype=torch.float32, device=dev)
         dt = fa.FA_BF16 if w.dtype == "bf16" else fa.FA_FP16
-        st = fa.fa_fwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), w.B, w.H, w.S,
-                          w.Skv, w.D, None, None, None, None, w.scale, int(w.causal), dt, sid)
+        if args.dropout > 0.0:
+            st = fa.fa_fwd_dropout(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), w.B, w.H,
+                                   w.S, w.Skv, w.D, w.scale, int(w.causal), args.dropout, DROPOUT_SEED, 0, dt, sid)
+        else:
+            st = fa.fa_fwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), w.B, w.H, w.S,
+                              w.Skv, w.D, None, None, None, None, w.scale, int(w.causal), dt, sid)
         if st != 0:
             raise fa.FaError(st)
         nbytes = fa.fa_bwd_workspace_size(w.B, w.H, w.S, w.D)
@@ -292,6 +300,16 @@ def run_bwd(args) -> int:
 
     def launch(i):
         w, b = runs[i], bufs[i]
+        if args.dropout > 0.0:
+            # the forward's decisions (offset 0), regenerated by the backward
+            st = fa.fa_bwd_dropout(b["q"].data_ptr(), b["k"].data_ptr(), b["v"].data_ptr(), b["o"].data_ptr(),
+                                   b["dout"].data_ptr(), b["lse"].data_ptr(), b["dq"].data_ptr(), b["dk"].data_ptr(),
+                                   b["dv"].data_ptr(), b["ws"].data_ptr(), b["nbytes"], w.B, w.H, w.S, w.Skv, w.D,
+                                   w.scale, int(w.causal), args.dropout, DROPOUT_SEED, 0, int(args.deterministic),
+                                   b["dt"], sid)
+            if st != 0:
+                raise fa.FaError(st, "fa_bwd_dropout")
+            return
         st = fa.fa_bwd(b["q"].data_ptr(), b["k"].data_ptr(), b["v"].data_ptr(), b["o"].data_ptr(),
                        b["dout"].data_ptr(), b["lse"].data_ptr(), b["dq"].data_ptr(), b["dk"].data_ptr(),
                        b["dv"].data_ptr(), b["ws"].data_ptr(), b["nbytes"], w.B, w.H, w.S, w.Skv, w.D, w.scale,
@@ -382,7 +400,8 @@ def run_bwd(args) -> int:
             "ms_per_step": max_ms / args.steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": w0.dtype, "data": "synthetic",
             "config": {"workload": ("deterministic " if args.deterministic else "") + "backward of "
-                       + workload_label(args.workload), "B": w0.B, "H": w0.H,
+                       + workload_label(args.workload)
+                       + (f", attention dropout p = {args.dropout:g}" if args.dropout > 0 else ""), "B": w0.B, "H": w0.H,
                        "S": w0.S, "D": w0.D, "runs_per_step": len(runs),
                        "l2": "inputs larger than L2 (no flush)" if sum(
                            t.numel() * t.element_size() for t in (bufs[0]["q"], bufs[0]["k"], bufs[0]["v"],
@@ -565,6 +584,8 @@ def main(argv=None) -> int:
     ap.add_argument("--mask", choices=["none", "tril"], default="none",
                     help="tril: causal runs go through fa_fwd_mask with an explicit lower-triangular mask "
                          "(the catlass page's mode 1) instead of the in-kernel diagonal skip (mode 2)")
+    ap.add_argument("--dropout", type=float, default=0.0,
+                    help="attention dropout probability (fa_fwd_dropout / fa_bwd_dropout); 0 = none")
     ap.add_argument("--deterministic", action="store_true",
                     help="with --pass bwd: the deterministic dQ mode (key tiles add in order)")
     args = ap.parse_args(argv)
@@ -646,7 +667,13 @@ def main(argv=None) -> int:
         o, lse = dev_out[i]
         o = view(w, o)
         dt = fa.FA_BF16 if w.dtype == "bf16" else fa.FA_FP16
-        if i in tril:
+        if args.dropout > 0.0:
+            if w.layout != "bhsd":
+                raise SystemExit("--dropout takes BHSD workloads")
+            # a fresh offset per step: new keep decisions, as in training
+            st = fa.fa_fwd_dropout(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), w.B, w.H,
+                                   w.S, w.Skv, w.D, w.scale, int(w.causal), args.dropout, DROPOUT_SEED, step, dt, sid)
+        elif i in tril:
             if w.layout != "bhsd":
                 raise SystemExit("--mask takes BHSD workloads")
             m = tril[i]
@@ -706,7 +733,8 @@ def main(argv=None) -> int:
         mean_ms = float(kern_ms[:, i].mean())
         per_run.append({"run": w.describe(), "mean_ms": mean_ms, "tflops": w.flops / (mean_ms * 1e-3) / 1e12})
     achieved = step_flops / (float(kern_ms.sum(axis=1).mean()) * 1e-3) / 1e12
-    traffic = traffic_per_launch(args.workload)
+    # the committed DRAM capture is of the kernels without dropout or an explicit mask
+    traffic = traffic_per_launch(args.workload) if (args.dropout == 0.0 and not tril) else None
 
     # end to end through the public call with host buffers
     e2e = None
@@ -743,7 +771,7 @@ def main(argv=None) -> int:
 
     cb = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cb = cpu_baseline(args.workload)
+        cb = cpu_baseline(args.workload, dropout=args.dropout)
 
     if rank == 0:
         w0 = runs[0]
@@ -752,7 +780,8 @@ def main(argv=None) -> int:
             "warmup": args.warmup, "ms_per_step": max_ms / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": w0.dtype, "data": "synthetic",
             "config": {"workload": workload_label(args.workload)
-                       + (" (causal as an explicit lower-triangular mask, no tile skipping)" if tril else ""),
+                       + (" (causal as an explicit lower-triangular mask, no tile skipping)" if tril else "")
+                       + (f", attention dropout p = {args.dropout:g} (fresh offset per step)" if args.dropout > 0 else ""),
                        "B": w0.B, "H": w0.H, "S": w0.S, "D": w0.D,
                        **({"Sk": w0.Skv, "layout": w0.layout} if w0.general else {}),
                        "runs_per_step": len(runs),
