@@ -241,6 +241,25 @@ FA_API int fa_bwd(const void* q, const void* k, const void* v, const void* o, co
                   int Sk, int D, float scale, int causal, int deterministic, int dtype, cudaStream_t stream);
 
 /*
+ * fa_bwd_ex -- fa_bwd with each tensor at its own (b, h, s) element strides,
+ * d contiguous, as fa_fwd_ex takes them (NULL = contiguous BHSD): BSHD data,
+ * packed QKV and padded gradient buffers are read and written in place.
+ * q_stride, o_stride, do_stride, dq_stride: host arrays of 3 strides for the
+ * [B][H][Sq][D] tensors; k_stride, v_stride, dk_stride, dv_stride for the
+ * [B][H][Sk][D] ones.  Each stride > 0, a multiple of 8 elements and below
+ * 2^36 (a stride over an extent of 1 is ignored), else FA_ERR_STRIDE; with
+ * Sq = 0 the dK/dV strides must be NULL.  The gradients must not overlap
+ * each other or the inputs.  Other arguments, workspace, modes and errors as
+ * fa_bwd (the workspace size does not depend on the strides).
+ */
+FA_API int fa_bwd_ex(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
+                     void* dq, void* dk, void* dv, void* workspace, long long workspace_bytes, int B, int H, int Sq,
+                     int Sk, int D, const long long* q_stride, const long long* k_stride,
+                     const long long* v_stride, const long long* o_stride, const long long* do_stride,
+                     const long long* dq_stride, const long long* dk_stride, const long long* dv_stride,
+                     float scale, int causal, int deterministic, int dtype, cudaStream_t stream);
+
+/*
  * fa_bwd_mask -- fa_bwd for the explicitly masked attention of fa_fwd_mask:
  * the same mask (device uint8, nonzero = attend; mask_stride = element strides
  * over b, h and the query row, 0 broadcasting over b or h; all multiples of 16,

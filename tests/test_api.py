@@ -237,3 +237,21 @@ def test_dropout_entries_reject_bad_arguments(lib):
         assert fa.fa_bwd_dropout(*bargs(p)) == _lib.FA_ERR_ARG, p
     assert fa.fa_bwd_dropout(*bargs(0.1, D=256)) == _lib.FA_ERR_HEADDIM
     assert ok  # the shapes above are otherwise valid
+
+
+def test_bwd_ex_rejects_bad_strides(lib):
+    def call(B=1, H=2, Sq=128, Sk=128, strides=(None,) * 8):
+        return fa.fa_bwd_ex(A, A, A, A, A, A, A, A, A, A, 1 << 30, B, H, Sq, Sk, 64, *strides, 0.1, 0, 0, 1, 0)
+    for bad in ((7, 64, 64), (0, 64, 64), (-8, 64, 64), (1 << 36, 64, 64)):
+        for t in range(8):
+            st = [None] * 8
+            st[t] = bad
+            assert call(B=2, strides=st) == _lib.FA_ERR_STRIDE, (t, bad)
+    # a stride over an extent of 1 is ignored (B = 1: the batch stride)
+    st = [None] * 8
+    st[0] = (3, 2 * 128 * 64, 64)
+    assert call(Sq=0, Sk=0, strides=st) == _lib.FA_OK
+    # no query: dK/dV are zeroed as contiguous blocks, so their strides must be NULL
+    st = [None] * 8
+    st[6] = (2 * 128 * 64, 128 * 64, 64)
+    assert call(Sq=0, strides=st) == _lib.FA_ERR_STRIDE

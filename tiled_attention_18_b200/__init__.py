@@ -8,12 +8,12 @@ in Python or PyTorch, and there is no fallback path.
 """
 from __future__ import annotations
 
-from ._lib import (FA_BF16, FA_FP16, FaError, fa_bwd, fa_bwd_dropout, fa_bwd_mask, fa_bwd_workspace_size,
+from ._lib import (FA_BF16, FA_FP16, FaError, fa_bwd, fa_bwd_dropout, fa_bwd_ex, fa_bwd_mask, fa_bwd_workspace_size,
                    fa_check_status, fa_fwd, fa_fwd_dropout, fa_fwd_ex, fa_fwd_mask, fa_fwd_noalloc, fa_merge_finalize, fa_merge_partial, fa_last_timeout_site, fa_num_units, fa_selftest_timeout, fa_status_string,
                    fa_version, load)
 
 __all__ = [
-    "FA_BF16", "FA_FP16", "FaError", "fa_bwd", "fa_bwd_dropout", "fa_bwd_mask", "fa_bwd_workspace_size",
+    "FA_BF16", "FA_FP16", "FaError", "fa_bwd", "fa_bwd_dropout", "fa_bwd_ex", "fa_bwd_mask", "fa_bwd_workspace_size",
     "fa_check_status", "fa_fwd", "fa_fwd_dropout", "fa_fwd_ex",
     "fa_fwd_mask", "fa_merge_finalize", "fa_merge_partial", "flash_attention_backward",
     "fa_fwd_noalloc", "fa_last_timeout_site",
@@ -96,8 +96,10 @@ def flash_attention_forward(q, k, v, scale: float, causal: bool = False, out=Non
 def flash_attention_backward(q, k, v, o, lse, dout, scale: float, causal: bool = False, deterministic: bool = False,
                              dq=None, dk=None, dv=None, workspace=None, stream=None, dropout_p: float = 0.0,
                              seed: int = 0, offset: int = 0):
-    """dQ, dK, dV for contiguous BHSD CUDA tensors (q, o, dout [B, H, Sq, D];
-    k, v [B, H, Sk, D]; lse [B, H, Sq] fp32 from the forward call).  The
+    """dQ, dK, dV for CUDA tensors q, o, dout [B, H, Sq, D] and k, v [B, H, Sk, D]
+    (lse [B, H, Sq] fp32 from the forward call).  The tensors may be strided
+    views contiguous in their last dimension (fa_bwd_ex), like the forward's;
+    the gradients take the layouts of q, k, v unless given.  The
     workspace (fa_bwd_workspace_size bytes) is allocated with torch unless
     given.  Launches on ``stream`` (default: torch's current stream) and
     returns without synchronising.  ``dropout_p``, ``seed`` and ``offset``
@@ -106,8 +108,8 @@ def flash_attention_backward(q, k, v, o, lse, dout, scale: float, causal: bool =
     B, H, Sq, D = q.shape
     Sk = k.shape[2]
     for name, t in (("q", q), ("k", k), ("v", v), ("o", o), ("dout", dout)):
-        if not (t.is_cuda and t.is_contiguous() and t.dtype == q.dtype):
-            raise ValueError(f"{name} must be a contiguous CUDA tensor of q's dtype")
+        if not (t.is_cuda and t.dtype == q.dtype and (t.stride(3) == 1 or D == 1)):
+            raise ValueError(f"{name} must be a CUDA tensor of q's dtype, contiguous in its last dimension")
     if o.shape != q.shape or dout.shape != q.shape or k.shape != (B, H, Sk, D) or v.shape != k.shape:
         raise ValueError("q, o, dout must be [B, H, Sq, D] and k, v [B, H, Sk, D]")
     if lse.shape != (B, H, Sq) or lse.dtype != torch.float32 or not lse.is_contiguous():
@@ -122,6 +124,17 @@ def flash_attention_backward(q, k, v, o, lse, dout, scale: float, causal: bool =
         workspace = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=q.device)
     if stream is None:
         stream = torch.cuda.current_stream(q.device)
+    tensors = (q, k, v, o, dout, dq, dk, dv)
+    if not all(t.is_contiguous() for t in tensors):
+        if dropout_p != 0.0:
+            raise ValueError("dropout needs contiguous tensors")
+        rc = fa_bwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), dout.data_ptr(), lse.data_ptr(),
+                       dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), workspace.data_ptr(), workspace.numel(), B, H, Sq,
+                       Sk, D, *(t.stride()[:3] for t in tensors), float(scale), int(bool(causal)),
+                       int(bool(deterministic)), _dtype_code(q), int(stream.cuda_stream))
+        if rc != 0:
+            raise FaError(rc, "fa_bwd_ex")
+        return dq, dk, dv
     if dropout_p != 0.0:
         rc = fa_bwd_dropout(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), dout.data_ptr(), lse.data_ptr(),
                             dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), workspace.data_ptr(), workspace.numel(), B, H,

@@ -55,6 +55,10 @@ SIGNATURES = [
      [ctypes.c_void_p] * 10 + [ctypes.c_longlong, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                ctypes.c_int, ctypes.c_float, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                ctypes.c_void_p]),
+    ("fa_bwd_ex", ctypes.c_int,
+     [ctypes.c_void_p] * 10 + [ctypes.c_longlong, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                               ctypes.c_int] + [_LL3] * 8 + [ctypes.c_float, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                                           ctypes.c_void_p]),
     ("fa_bwd_mask", ctypes.c_int,
      [ctypes.c_void_p] * 10 + [ctypes.c_longlong, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                ctypes.c_int, ctypes.c_void_p, _LL3, ctypes.c_float, ctypes.c_int, ctypes.c_int,
@@ -157,6 +161,19 @@ def fa_bwd(q_ptr: int, k_ptr: int, v_ptr: int, o_ptr: int, do_ptr: int, lse_ptr:
     return int(load().fa_bwd(q_ptr, k_ptr, v_ptr, o_ptr, do_ptr, lse_ptr, dq_ptr, dk_ptr, dv_ptr, ws_ptr,
                              int(ws_bytes), B, H, Sq, Sk, D, float(scale), int(causal), int(deterministic),
                              int(dtype), stream))
+
+
+def fa_bwd_ex(q_ptr: int, k_ptr: int, v_ptr: int, o_ptr: int, do_ptr: int, lse_ptr: int, dq_ptr: int, dk_ptr: int,
+              dv_ptr: int, ws_ptr: int, ws_bytes: int, B: int, H: int, Sq: int, Sk: int, D: int, q_stride, k_stride,
+              v_stride, o_stride, do_stride, dq_stride, dk_stride, dv_stride, scale: float, causal: int,
+              deterministic: int, dtype: int, stream: int) -> int:
+    """Raw C call of the strided backward pass: each stride argument is a (b, h, s)
+    element-stride triple or None (contiguous)."""
+    return int(load().fa_bwd_ex(q_ptr, k_ptr, v_ptr, o_ptr, do_ptr, lse_ptr, dq_ptr, dk_ptr, dv_ptr, ws_ptr,
+                                int(ws_bytes), B, H, Sq, Sk, D, _strides(q_stride), _strides(k_stride),
+                                _strides(v_stride), _strides(o_stride), _strides(do_stride), _strides(dq_stride),
+                                _strides(dk_stride), _strides(dv_stride), float(scale), int(causal),
+                                int(deterministic), int(dtype), stream))
 
 
 def fa_bwd_mask(q_ptr: int, k_ptr: int, v_ptr: int, o_ptr: int, do_ptr: int, lse_ptr: int, dq_ptr: int,

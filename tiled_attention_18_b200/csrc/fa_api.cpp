@@ -347,7 +347,8 @@ namespace {
 int backward(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse, void* dq,
              void* dk, void* dv, void* workspace, long long workspace_bytes, int B, int H, int Sq, int Sk, int D,
              float scale, int causal, int deterministic, int dtype, cudaStream_t stream, const uint8_t* mask,
-             const long long* mask_stride, const fa::DropoutArgs* drop = nullptr) {
+             const long long* mask_stride, const fa::DropoutArgs* drop = nullptr,
+             const long long* const* strides = nullptr) {
     if (B < 0 || H < 0 || Sq < 0 || Sk < 0) return FA_ERR_SHAPE;
     if (D != 64 && D != 128) return FA_ERR_HEADDIM;
     if (dtype != FA_FP16 && dtype != FA_BF16) return FA_ERR_DTYPE;
@@ -360,9 +361,19 @@ int backward(const void* q, const void* k, const void* v, const void* o, const v
     if (BH > INT_MAX || BH * (int64_t)Sq > INT_MAX || BH * (int64_t)Sk > INT_MAX || Sq > INT_MAX - 512 ||
         Sk > INT_MAX - 512)
         return FA_ERR_SHAPE;
+    // strides (elements over b, h, row) of q, k, v, o, dout, dq, dk, dv; NULL = contiguous
+    long long st[8][3];
+    {
+        const int rows[8] = {Sq, Sk, Sk, Sq, Sq, Sq, Sk, Sk};
+        for (int t = 0; t < 8; ++t) {
+            const int rc = resolve_strides(strides ? strides[t] : nullptr, B, H, rows[t], D, st[t]);
+            if (rc != FA_OK) return rc;
+        }
+    }
     if (Sq == 0) {
         // no query: the key and value gradients are zero
         if (!dk || !dv) return FA_ERR_NULL;
+        if (strides && (strides[6] || strides[7])) return FA_ERR_STRIDE;  // zeroed as whole contiguous blocks
         const size_t bytes = (size_t)BH * (size_t)Sk * (size_t)D * 2;
         if (cudaMemsetAsync(dk, 0, bytes, stream) != cudaSuccess || cudaMemsetAsync(dv, 0, bytes, stream) != cudaSuccess) {
             cudaGetLastError();
@@ -396,17 +407,22 @@ int backward(const void* q, const void* k, const void* v, const void* o, const v
         rc = check_device_pointer(p, cur);
         if (rc != FA_OK) return rc;
     }
-    long long qs[3], ks[3];
-    resolve_strides(nullptr, B, H, Sq, D, qs);
-    resolve_strides(nullptr, B, H, Sk, D, ks);
     fa::BwdLaunchArgs a;
     std::memset(&a, 0, sizeof(a));
     // the D = 128 backward kernel steps through 64 query rows at a time
     const int q_box = (D == 128) ? 64 : fa::BLOCK_M;
-    if (!encode_tensor(&a.tmap_q, q, B, H, Sq, D, qs, dtype, q_box) ||
-        !encode_tensor(&a.tmap_do, dout, B, H, Sq, D, qs, dtype, q_box) ||
-        !encode_tensor(&a.tmap_k, k, B, H, Sk, D, ks, dtype) || !encode_tensor(&a.tmap_v, v, B, H, Sk, D, ks, dtype))
+    if (!encode_tensor(&a.tmap_q, q, B, H, Sq, D, st[0], dtype, q_box) ||
+        !encode_tensor(&a.tmap_do, dout, B, H, Sq, D, st[4], dtype, q_box) ||
+        !encode_tensor(&a.tmap_k, k, B, H, Sk, D, st[1], dtype) ||
+        !encode_tensor(&a.tmap_v, v, B, H, Sk, D, st[2], dtype))
         return FA_ERR_LAUNCH;
+    for (int i = 0; i < 3; ++i) {
+        a.o_stride[i] = st[3][i];
+        a.do_stride[i] = st[4][i];
+        a.dq_stride[i] = st[5][i];
+        a.dk_stride[i] = st[6][i];
+        a.dv_stride[i] = st[7][i];
+    }
     uint8_t* w = static_cast<uint8_t*>(workspace);
     a.o = o;
     a.dout = dout;
@@ -459,6 +475,18 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const voi
            float scale, int causal, int deterministic, int dtype, cudaStream_t stream) {
     return backward(q, k, v, o, dout, lse, dq, dk, dv, workspace, workspace_bytes, B, H, Sq, Sk, D, scale, causal,
                     deterministic, dtype, stream, nullptr, nullptr);
+}
+
+int fa_bwd_ex(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse, void* dq,
+              void* dk, void* dv, void* workspace, long long workspace_bytes, int B, int H, int Sq, int Sk, int D,
+              const long long* q_stride, const long long* k_stride, const long long* v_stride,
+              const long long* o_stride, const long long* do_stride, const long long* dq_stride,
+              const long long* dk_stride, const long long* dv_stride, float scale, int causal, int deterministic,
+              int dtype, cudaStream_t stream) {
+    const long long* const strides[8] = {q_stride, k_stride, v_stride, o_stride, do_stride, dq_stride, dk_stride,
+                                         dv_stride};
+    return backward(q, k, v, o, dout, lse, dq, dk, dv, workspace, workspace_bytes, B, H, Sq, Sk, D, scale, causal,
+                    deterministic, dtype, stream, nullptr, nullptr, nullptr, strides);
 }
 
 int fa_bwd_mask(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,

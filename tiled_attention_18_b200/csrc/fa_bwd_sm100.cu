@@ -111,6 +111,10 @@ struct BwdSmem {
     static constexpr int ALLOC = BYTES + 1024;           // slack for 1 KiB alignment
 };
 
+struct Strides3 {
+    long long s[3];  // element strides over b, h and the row
+};
+
 struct BwdParams {
     CUtensorMap tmap_q;
     CUtensorMap tmap_k;
@@ -119,8 +123,9 @@ struct BwdParams {
     const float* lse2;    // [BH][Sq_pad] LSE * log2(e), +inf on padded rows
     const float* delta;   // [BH][Sq_pad] rowsum(dO * O), 0 on padded rows
     float* dq_acc;        // [BH][Sq][D] fp32, zeroed by the prep kernel
-    uint8_t* dk;          // [BH][Sk][D] 16-bit
-    uint8_t* dv;
+    uint8_t* dk;          // [B][H][Sk][D] 16-bit at byte strides dk_s (over b, h, key row)
+    uint8_t* dv;          // the same at dv_s
+    long long dk_s[3], dv_s[3];
     int BH, H, Sq, Sk, Sq_pad, n_mtiles, n_ktiles, n_units, causal, causal_off;
     int head_group;       // causal claim order: heads per group (their Q, dO, dQ fit in L2)
     int* dq_flags;        // deterministic mode: [BH][flag_steps][4] key tiles added so far per
@@ -649,7 +654,10 @@ __device__ void bwd_out_role(const BwdParams& p, uint8_t* smem, uint32_t tmem, i
         tc_fence_after();
         const int key = U.n * TILE + row;
         const bool valid = key < p.Sk;
-        const size_t off = ((size_t)U.bh * (size_t)p.Sk + (size_t)(valid ? key : 0)) * (size_t)(D * 2);
+        const int ub = U.bh / p.H, uh = U.bh - ub * p.H;
+        const long long kr = valid ? key : 0;
+        uint8_t* dv_row = p.dv + ub * p.dv_s[0] + uh * p.dv_s[1] + kr * p.dv_s[2];
+        uint8_t* dk_row = p.dk + ub * p.dk_s[0] + uh * p.dk_s[1] + kr * p.dk_s[2];
 #pragma unroll 1
         for (int c = 0; c < D / 32; ++c) {
             uint32_t r[32];
@@ -658,7 +666,7 @@ __device__ void bwd_out_role(const BwdParams& p, uint8_t* smem, uint32_t tmem, i
 #pragma unroll
             for (int i = 0; i < 16; ++i) w[i] = pack2<BF16>(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
             if (valid) {
-                uint4* d = reinterpret_cast<uint4*>(p.dv + off + c * 64);
+                uint4* d = reinterpret_cast<uint4*>(dv_row + c * 64);
 #pragma unroll
                 for (int i = 0; i < 4; ++i) d[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
             }
@@ -667,7 +675,7 @@ __device__ void bwd_out_role(const BwdParams& p, uint8_t* smem, uint32_t tmem, i
             for (int i = 0; i < 16; ++i)
                 w[i] = pack2<BF16>(__uint_as_float(r[2 * i]) * p.scale, __uint_as_float(r[2 * i + 1]) * p.scale);
             if (valid) {
-                uint4* d = reinterpret_cast<uint4*>(p.dk + off + c * 64);
+                uint4* d = reinterpret_cast<uint4*>(dk_row + c * 64);
 #pragma unroll
                 for (int i = 0; i < 4; ++i) d[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
             }
@@ -1177,7 +1185,10 @@ __device__ void bwd2_out_role(const BwdParams& p, uint8_t* smem, uint32_t tmem, 
         tc_fence_after();
         const int key = U.n * TILE + row;
         const bool valid = key < p.Sk;
-        const size_t off = ((size_t)U.bh * (size_t)p.Sk + (size_t)(valid ? key : 0)) * 256;
+        const int ub = U.bh / p.H, uh = U.bh - ub * p.H;
+        const long long kr = valid ? key : 0;
+        uint8_t* dv_row = p.dv + ub * p.dv_s[0] + uh * p.dv_s[1] + kr * p.dv_s[2];
+        uint8_t* dk_row = p.dk + ub * p.dk_s[0] + uh * p.dk_s[1] + kr * p.dk_s[2];
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
             uint32_t r[32];
@@ -1186,7 +1197,7 @@ __device__ void bwd2_out_role(const BwdParams& p, uint8_t* smem, uint32_t tmem, 
 #pragma unroll
             for (int i = 0; i < 16; ++i) w[i] = pack2<BF16>(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
             if (valid) {
-                uint4* d = reinterpret_cast<uint4*>(p.dv + off + c * 64);
+                uint4* d = reinterpret_cast<uint4*>(dv_row + c * 64);
 #pragma unroll
                 for (int i = 0; i < 4; ++i) d[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
             }
@@ -1195,7 +1206,7 @@ __device__ void bwd2_out_role(const BwdParams& p, uint8_t* smem, uint32_t tmem, 
             for (int i = 0; i < 16; ++i)
                 w[i] = pack2<BF16>(__uint_as_float(r[2 * i]) * p.scale, __uint_as_float(r[2 * i + 1]) * p.scale);
             if (valid) {
-                uint4* d = reinterpret_cast<uint4*>(p.dk + off + c * 64);
+                uint4* d = reinterpret_cast<uint4*>(dk_row + c * 64);
 #pragma unroll
                 for (int i = 0; i < 4; ++i) d[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
             }
@@ -1279,7 +1290,8 @@ template <int D, bool BF16>
 __global__ void __launch_bounds__(256) bwd_prep_kernel(const uint16_t* __restrict__ o, const uint16_t* __restrict__ dout,
                                                        const float* __restrict__ lse, float* __restrict__ lse2,
                                                        float* __restrict__ delta, float* __restrict__ dq_acc, int Sq,
-                                                       int Sq_pad, unsigned int* sched) {
+                                                       int Sq_pad, unsigned int* sched, int H, Strides3 os,
+                                                       Strides3 dos) {
     constexpr int PER_LANE = D / 32;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int row = blockIdx.x * 8 + warp;
@@ -1293,10 +1305,13 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const uint16_t* __restric
         }
         return;
     }
-    const size_t e0 = (bh * (size_t)Sq + (size_t)row) * D + (size_t)lane * PER_LANE;
+    const size_t e0 = (bh * (size_t)Sq + (size_t)row) * D + (size_t)lane * PER_LANE;  // dQ accumulator (contiguous)
+    const long long ub = (long long)(bh / H), uh = (long long)(bh % H);
+    const long long eo = ub * os.s[0] + uh * os.s[1] + row * os.s[2] + lane * PER_LANE;
+    const long long ed = ub * dos.s[0] + uh * dos.s[1] + row * dos.s[2] + lane * PER_LANE;
     float acc = 0.f;
 #pragma unroll
-    for (int i = 0; i < PER_LANE; ++i) acc = fmaf(load16<BF16>(o + e0 + i), load16<BF16>(dout + e0 + i), acc);
+    for (int i = 0; i < PER_LANE; ++i) acc = fmaf(load16<BF16>(o + eo + i), load16<BF16>(dout + ed + i), acc);
 #pragma unroll
     for (int s = 16; s > 0; s >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, s);
 #pragma unroll
@@ -1309,13 +1324,20 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const uint16_t* __restric
     }
 }
 
-// dQ = scale * accumulator, rounded to the 16-bit dtype (4 elements per thread).
-template <bool BF16>
-__global__ void __launch_bounds__(256) bwd_post_kernel(const float4* __restrict__ acc, uint2* __restrict__ dq,
-                                                       size_t n4, float scale) {
+// dQ = scale * accumulator, rounded to the 16-bit dtype (4 elements per
+// thread), written at dQ's element strides over b, h and the query row.
+template <int D, bool BF16>
+__global__ void __launch_bounds__(256) bwd_post_kernel(const float4* __restrict__ acc, uint16_t* __restrict__ dq,
+                                                       size_t n4, float scale, int H, int Sq, Strides3 qs) {
+    constexpr int G = D / 4;  // 4-element groups per row
     for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n4; i += (size_t)gridDim.x * blockDim.x) {
         const float4 a = acc[i];
-        dq[i] = make_uint2(pack2<BF16>(a.x * scale, a.y * scale), pack2<BF16>(a.z * scale, a.w * scale));
+        const size_t rowi = i / G;  // (bh, query row), rows of the contiguous accumulator
+        const int d = (int)(i - rowi * G) * 4;
+        const long long bh = (long long)(rowi / (size_t)Sq), row = (long long)(rowi - (size_t)bh * Sq);
+        const long long e = (bh / H) * qs.s[0] + (bh % H) * qs.s[1] + row * qs.s[2] + d;
+        *reinterpret_cast<uint2*>(dq + e) =
+            make_uint2(pack2<BF16>(a.x * scale, a.y * scale), pack2<BF16>(a.z * scale, a.w * scale));
     }
 }
 
@@ -1330,7 +1352,8 @@ cudaError_t launch_bwd_impl(const BwdLaunchArgs& a, cudaStream_t stream) {
         dim3 grid((unsigned)(Sq_pad / 8), (unsigned)BH, 1);
         bwd_prep_kernel<D, BF16><<<grid, 256, 0, stream>>>(
             static_cast<const uint16_t*>(a.o), static_cast<const uint16_t*>(a.dout), a.lse, a.lse2, a.delta,
-            a.dq_acc, a.Sq, Sq_pad, a.sched);
+            a.dq_acc, a.Sq, Sq_pad, a.sched, a.H, Strides3{{a.o_stride[0], a.o_stride[1], a.o_stride[2]}},
+            Strides3{{a.do_stride[0], a.do_stride[1], a.do_stride[2]}});
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
@@ -1354,6 +1377,10 @@ cudaError_t launch_bwd_impl(const BwdLaunchArgs& a, cudaStream_t stream) {
         p.dq_acc = a.dq_acc;
         p.dk = static_cast<uint8_t*>(a.dk);
         p.dv = static_cast<uint8_t*>(a.dv);
+        for (int i = 0; i < 3; ++i) {
+            p.dk_s[i] = a.dk_stride[i] * 2;
+            p.dv_s[i] = a.dv_stride[i] * 2;
+        }
         p.BH = BH;
         p.H = a.H;
         p.Sq = a.Sq;
@@ -1398,8 +1425,9 @@ cudaError_t launch_bwd_impl(const BwdLaunchArgs& a, cudaStream_t stream) {
     {
         const size_t n4 = (size_t)BH * (size_t)a.Sq * D / 4;
         const unsigned blocks = (unsigned)((n4 + 255) / 256 < 148u * 16u ? (n4 + 255) / 256 : 148u * 16u);
-        bwd_post_kernel<BF16><<<blocks, 256, 0, stream>>>(reinterpret_cast<const float4*>(a.dq_acc),
-                                                           static_cast<uint2*>(a.dq), n4, a.scale);
+        bwd_post_kernel<D, BF16><<<blocks, 256, 0, stream>>>(
+            reinterpret_cast<const float4*>(a.dq_acc), static_cast<uint16_t*>(a.dq), n4, a.scale, a.H, a.Sq,
+            Strides3{{a.dq_stride[0], a.dq_stride[1], a.dq_stride[2]}});
         return cudaGetLastError();
     }
 }

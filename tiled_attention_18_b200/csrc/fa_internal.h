@@ -63,8 +63,10 @@ struct BwdLaunchArgs {
     CUtensorMap tmap_k;
     CUtensorMap tmap_v;
     CUtensorMap tmap_do;
-    const void* o;          // [B,H,Sq,D] 16-bit
-    const void* dout;       // [B,H,Sq,D] 16-bit
+    const void* o;          // [B,H,Sq,D] 16-bit at o_stride
+    const void* dout;       // [B,H,Sq,D] 16-bit at do_stride
+    // element strides over b, h and the row (d contiguous) of O, dO and the gradients
+    long long o_stride[3], do_stride[3], dq_stride[3], dk_stride[3], dv_stride[3];
     const float* lse;       // [B,H,Sq] fp32 (natural log)
     void* dq;               // [B,H,Sq,D] 16-bit
     void* dk;               // [B,H,Sk,D] 16-bit
