@@ -270,18 +270,20 @@ def run_bwd(args) -> int:
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
     fa.load()
+    from tiled_attention_18_b200.workloads import to_layout
     runs = workload_runs(args.workload)
     for w in runs:
-        if w.layout != "bhsd":
-            raise SystemExit("fa_bwd takes contiguous BHSD tensors; pick a BHSD workload")
+        if w.layout != "bhsd" and (args.dropout > 0.0 or args.deterministic):
+            raise SystemExit("--dropout and --deterministic take BHSD workloads")
     stream = torch.cuda.current_stream(dev)
     sid = stream.cuda_stream
     bufs = []
     for w in runs:
         wr = dataclasses.replace(w, seed=rank_seed(w.seed, rank))
-        q, k, v = (t.to(dev) for t in workload_inputs(wr))
+        # BSHD workloads: every tensor (inputs, O, dO, gradients) in that layout, through fa_bwd_ex
+        q, k, v = (to_layout(t.to(dev), w.layout) for t in workload_inputs(wr))
         g = torch.Generator().manual_seed(rank_seed(w.seed, rank) + 7)
-        dout = torch.randn(q.shape, generator=g).to(q.dtype).to(dev)
+        dout = to_layout(torch.randn(q.shape, generator=g).to(q.dtype).to(dev), w.layout)
         o = torch.empty_like(q)
         lse = torch.empty(q.shape[:3], dtype=torch.float32, device=dev)
         dt = fa.FA_BF16 if w.dtype == "bf16" else fa.FA_FP16
@@ -290,10 +292,13 @@ def run_bwd(args) -> int:
                                    w.S, w.Skv, w.D, w.scale, int(w.causal), args.dropout, DROPOUT_SEED, 0, dt, sid)
         else:
             st = fa.fa_fwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), w.B, w.H, w.S,
-                              w.Skv, w.D, None, None, None, None, w.scale, int(w.causal), dt, sid)
+                              w.Skv, w.D, q.stride()[:3], k.stride()[:3], v.stride()[:3], o.stride()[:3], w.scale,
+                              int(w.causal), dt, sid)
         if st != 0:
             raise fa.FaError(st)
         nbytes = fa.fa_bwd_workspace_size(w.B, w.H, w.S, w.D)
+        if nbytes < 0:
+            raise SystemExit(f"the backward pass takes D = 64 or 128 ({fa.fa_status_string(int(nbytes))})")
         bufs.append(dict(q=q, k=k, v=v, o=o, lse=lse, dout=dout, dq=torch.empty_like(q), dk=torch.empty_like(k),
                          dv=torch.empty_like(v), ws=torch.empty(nbytes, dtype=torch.uint8, device=dev),
                          nbytes=nbytes, dt=dt))
@@ -309,6 +314,15 @@ def run_bwd(args) -> int:
                                    b["dt"], sid)
             if st != 0:
                 raise fa.FaError(st, "fa_bwd_dropout")
+            return
+        if w.layout != "bhsd":
+            names = ("q", "k", "v", "o", "dout", "dq", "dk", "dv")
+            st = fa.fa_bwd_ex(*(b[n].data_ptr() for n in names[:5]), b["lse"].data_ptr(),
+                              *(b[n].data_ptr() for n in names[5:]), b["ws"].data_ptr(), b["nbytes"], w.B, w.H, w.S,
+                              w.Skv, w.D, *(b[n].stride()[:3] for n in names), w.scale, int(w.causal), 0, b["dt"],
+                              sid)
+            if st != 0:
+                raise fa.FaError(st, "fa_bwd_ex")
             return
         st = fa.fa_bwd(b["q"].data_ptr(), b["k"].data_ptr(), b["v"].data_ptr(), b["o"].data_ptr(),
                        b["dout"].data_ptr(), b["lse"].data_ptr(), b["dq"].data_ptr(), b["dk"].data_ptr(),
