@@ -1,6 +1,10 @@
 /*
- * fa.h -- C ABI of libfa.so: fused attention forward (FlashAttention-2 style)
- * for NVIDIA B200 (sm_100a).
+ * fa.h -- C ABI of libfa.so: fused attention (FlashAttention-2 style) for
+ * NVIDIA B200 (sm_100a): the forward pass (fa_fwd, fa_fwd_ex, fa_fwd_noalloc,
+ * head dimension 64/128/256), its explicit-mask and dropout variants
+ * (fa_fwd_mask, fa_fwd_dropout), the backward pass (fa_bwd, fa_bwd_ex,
+ * fa_bwd_mask, fa_bwd_dropout) and the log-sum-exp merge of partial results
+ * for a sequence split across devices (fa_merge_partial, fa_merge_finalize).
  *
  * The operation, per batch b, head h and query row i of BHSD tensors
  * (contiguous for fa_fwd; any b, h, s strides and Sq != Sk for fa_fwd_ex):
@@ -51,7 +55,7 @@ typedef enum {
     FA_OK = 0,
     FA_ERR_NULL = -1,     /* a required pointer is NULL */
     FA_ERR_SHAPE = -2,    /* B, H or S negative, or too large for 32-bit indexing */
-    FA_ERR_HEADDIM = -3,  /* D is not 64, 128 or 256 (64 or 128 for fa_fwd_mask and fa_bwd) */
+    FA_ERR_HEADDIM = -3,  /* D is not 64, 128 or 256 (64 or 128 for the mask, dropout and backward entries) */
     FA_ERR_DTYPE = -4,    /* dtype is not FA_FP16 or FA_BF16 */
     FA_ERR_ALIGN = -5,    /* q, k, v, o not 16-byte aligned, or lse not 4-byte aligned */
     FA_ERR_ARCH = -6,     /* the current device is not compute capability 10.0 (sm_100) */
@@ -60,9 +64,10 @@ typedef enum {
     FA_ERR_SCALE = -9,    /* scale is not finite and > 0 */
     FA_ERR_ARG = -10,     /* causal (or fa_bwd's deterministic) is not 0 or 1, or dropout_p is out of range */
     FA_ERR_PTR = -11,     /* a pointer is not device memory of the current device */
-    FA_ERR_STRIDE = -12,  /* fa_fwd_ex: a stride is negative, zero over an extent > 1, not a
-                             multiple of 8 elements (16 bytes), or not below 2^36 elements */
-    FA_ERR_WORKSPACE = -13 /* fa_bwd: workspace NULL, not 256-byte aligned or too small */
+    FA_ERR_STRIDE = -12,  /* fa_fwd_ex, fa_bwd_ex: a stride is negative, zero over an extent > 1,
+                             not a multiple of 8 elements (16 bytes), or not below 2^36 elements;
+                             the mask entries: a mask stride breaks their rules */
+    FA_ERR_WORKSPACE = -13 /* the fa_bwd entries: workspace NULL, not 256-byte aligned or too small */
 } fa_status;
 
 /*
