@@ -205,20 +205,26 @@ def run_reference(args):
     if rank != 0:
         return 0
     runs = workload_runs(args.workload)
+    bwd = args.pass_ == "bwd"
     # the oracle keeps no state between calls: warm-up steps have nothing to warm
     times = []
     for _ in range(args.steps):
-        cb = cpu_baseline(args.workload, target_s=max(2.0, 60.0 / max(args.steps, 1)))
+        budget = max(2.0, 60.0 / max(args.steps, 1))
+        cb = (cpu_baseline_bwd(args.workload, target_s=budget, dropout=args.dropout) if bwd else
+              cpu_baseline(args.workload, target_s=budget, dropout=args.dropout))
         times.append(cb)
     value = float(np.median([c["value"] for c in times]))
     cb = dict(times[-1])
     cb["value"] = value
-    step_flops = sum(w.flops for w in runs)
+    step_flops = (BWD_FLOP_FACTOR if bwd else 1.0) * sum(w.flops for w in runs)
+    label = ("backward of " if bwd else "") + workload_label(args.workload) + (
+        f", attention dropout p = {args.dropout:g}" if args.dropout > 0 else "")
     line = {
-        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "impl": "reference", "metric": BWD_METRIC if bwd else METRIC, "value": value, "unit": UNIT,
+        "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_flops / (value * 1e12) * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": workload_label(args.workload), "note": "fp64 CPU oracle on bounded row samples"},
+        "config": {"workload": label, "note": "fp64 CPU oracle on bounded samples"},
         "cpu_baseline": cb,
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -227,9 +233,10 @@ def run_reference(args):
 
 
 BWD_FLOP_FACTOR = 2.5  # five S x S x D products in the backward pass against two in the forward pass
+BWD_METRIC = "attention bwd TFLOPS (2.5x forward flops, causal-adjusted) and % of B200 dense bf16 peak"
 
 
-def cpu_baseline_bwd(name: str, target_s: float = 12.0):
+def cpu_baseline_bwd(name: str, target_s: float = 12.0, dropout: float = 0.0):
     """The fp64 backward oracle on one head of the workload's first run with the
     sequence cut to a length whose cost fits ``target_s``; TFLOP/s of that sample
     (2.5x the forward's algorithmic flops of the sample)."""
@@ -245,7 +252,11 @@ def cpu_baseline_bwd(name: str, target_s: float = 12.0):
         g = torch.Generator().manual_seed(5)
         dout = torch.randn(q.shape, generator=g).to(q.dtype)
         t0 = time.perf_counter()
-        oracle.attn_bwd(q, k, v, dout, ws.scale, ws.causal, ws.dtype)
+        if dropout > 0.0:
+            oracle.attn_bwd_dropout(q, k, v, dout, ws.scale, ws.causal, ws.dtype, int(np.floor(dropout * 256 + 0.5)),
+                                    DROPOUT_SEED, 0)
+        else:
+            oracle.attn_bwd(q, k, v, dout, ws.scale, ws.causal, ws.dtype)
         dt = time.perf_counter() - t0
         if dt >= target_s / 8 or S >= w.S:
             break
@@ -405,11 +416,11 @@ def run_bwd(args) -> int:
                "unit": UNIT, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
     cb = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cb = cpu_baseline_bwd(args.workload)
+        cb = cpu_baseline_bwd(args.workload, dropout=args.dropout)
     if rank == 0:
         w0 = runs[0]
         line = {
-            "metric": "attention bwd TFLOPS (2.5x forward flops, causal-adjusted) and % of B200 dense bf16 peak",
+            "metric": BWD_METRIC,
             "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": max_ms / args.steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": w0.dtype, "data": "synthetic",
