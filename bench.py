@@ -209,7 +209,7 @@ def run_reference(args):
     # the oracle keeps no state between calls: warm-up steps have nothing to warm
     times = []
     for _ in range(args.steps):
-        budget = max(2.0, 60.0 / max(args.steps, 1))
+        budget = args.cpu_seconds if args.cpu_seconds > 0 else max(2.0, 60.0 / max(args.steps, 1))
         cb = (cpu_baseline_bwd(args.workload, target_s=budget, dropout=args.dropout) if bwd else
               cpu_baseline(args.workload, target_s=budget, dropout=args.dropout))
         times.append(cb)
@@ -601,6 +601,8 @@ def main(argv=None) -> int:
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=0.0,
+                    help="--impl reference: CPU seconds per step (default: about a minute per run)")
     ap.add_argument("--pass", dest="pass_", choices=["fwd", "bwd", "sp"], default="fwd",
                     help="fwd: the forward pass (default); bwd: the backward pass fa_bwd; sp: the "
                          "sequence-parallel schedule of --sp-world ranks run in turn on one GPU")
