@@ -349,6 +349,15 @@ FA_API int fa_merge_partial(float* o_acc, float* lse_acc, const void* o_part, co
 FA_API int fa_merge_finalize(const float* o_acc, void* o, long long n, int dtype, cudaStream_t stream);
 
 /*
+ * fa_accumulate -- acc[i] += x[i] for n values: fp32 accumulators (device,
+ * 4-byte aligned) of 16-bit partial results x (device, dtype), e.g. the
+ * gradients of one K/V block in the sequence-parallel backward pass, which
+ * sums the contributions of every block.  Asynchronous on stream; errors as
+ * fa_merge_partial.
+ */
+FA_API int fa_accumulate(float* acc, const void* x, long long n, int dtype, cudaStream_t stream);
+
+/*
  * fa_check_status -- synchronise `stream`, then report and clear the device
  * status word of the current device: FA_OK, FA_ERR_TIMEOUT if a kernel
  * stopped on a bounded wait since the last call, or FA_ERR_LAUNCH on a CUDA

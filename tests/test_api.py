@@ -255,3 +255,12 @@ def test_bwd_ex_rejects_bad_strides(lib):
     st = [None] * 8
     st[6] = (2 * 128 * 64, 128 * 64, 64)
     assert call(Sq=0, strides=st) == _lib.FA_ERR_STRIDE
+
+
+def test_accumulate_rejects_bad_arguments(lib):
+    assert fa.fa_accumulate(A, A, -1, 1, 0) == _lib.FA_ERR_SHAPE
+    assert fa.fa_accumulate(A, A, 10, 7, 0) == _lib.FA_ERR_DTYPE
+    assert fa.fa_accumulate(0, A, 10, 1, 0) == _lib.FA_ERR_NULL
+    assert fa.fa_accumulate(A + 2, A, 10, 1, 0) == _lib.FA_ERR_ALIGN
+    assert fa.fa_accumulate(A, A + 1, 10, 1, 0) == _lib.FA_ERR_ALIGN
+    assert fa.fa_accumulate(0, 0, 0, 1, 0) == _lib.FA_OK

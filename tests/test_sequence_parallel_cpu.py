@@ -89,3 +89,70 @@ def test_ring_schedule():
     assert ring_schedule(2, 3, True) == [(2, "causal"), (1, "full"), (0, "full")]
     assert ring_schedule(0, 3, True) == [(0, "causal"), (2, "skip"), (1, "skip")]
     assert ring_schedule(1, 4, True) == [(1, "causal"), (0, "full"), (3, "skip"), (2, "skip")]
+
+
+class GradOps:
+    """Stand-in for the kernels in the ring backward: a block's share of the
+    gradients for the rows' global O and LSE, in float64 (test stand-in)."""
+
+    def __init__(self, scale):
+        self.scale = scale
+
+    def zeros_f32(self, t):
+        return torch.zeros(t.shape, dtype=torch.float64)
+
+    def bwd_partial(self, q, k, v, o, lse, dout, causal, deterministic=False):
+        qd, kd, vd, dod = (t.double() for t in (q, k, v, dout))
+        s = self.scale * qd @ kd.transpose(-1, -2)
+        if causal:
+            n = s.shape[-1]
+            s = s.masked_fill(torch.ones(n, n, dtype=torch.bool).triu(1), float("-inf"))
+        p = torch.exp(s - lse[..., None])
+        ds = p * (dod @ vd.transpose(-1, -2) - (dod * o).sum(-1, keepdim=True))
+        return self.scale * ds @ kd, self.scale * ds.transpose(-1, -2) @ qd, p.transpose(-1, -2) @ dod
+
+    def accumulate(self, acc, x):
+        acc += x
+
+    def to16(self, acc, dtype):
+        return acc
+
+
+def _bwd_worker(rank, world, port, causal, out_dir):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        import oracle
+        from tiled_attention_18_b200.sequence_parallel import ring_attention_backward
+        from tiled_attention_18_b200.workloads import make_inputs
+        B, H, c, D = 1, 2, 20, 16
+        q, k, v = make_inputs(B, H, world * c, D, "bf16", seed=6)
+        dout = torch.randn(q.shape, generator=torch.Generator().manual_seed(7)).to(torch.bfloat16)
+        o, lse = oracle.attn_fwd(q, k, v, 0.25, causal, "bf16")  # the forward's global rows
+        sl = slice(rank * c, (rank + 1) * c)
+        part = lambda t: t[:, :, sl].contiguous()  # noqa: E731
+        dq, dk, dv = ring_attention_backward(part(q), part(k), part(v), torch.from_numpy(o[:, :, sl].copy()),
+                                             torch.from_numpy(lse[:, :, sl].copy()), part(dout), 0.25, causal,
+                                             ops=GradOps(0.25))
+        for name, t in (("dq", dq), ("dk", dk), ("dv", dv)):
+            np.save(os.path.join(out_dir, f"{name}{rank}.npy"), t.numpy())
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 3])
+@pytest.mark.parametrize("causal", [False, True])
+def test_ring_backward_ranks_equal_full_gradients(tmp_path, world, causal):
+    """The gradients gathered from the ranks equal the oracle's gradients of
+    attention over the whole sequence."""
+    import oracle
+    from tiled_attention_18_b200.workloads import make_inputs
+    mp.spawn(_bwd_worker, args=(world, _free_port(), causal, str(tmp_path)), nprocs=world, join=True)
+    B, H, c, D = 1, 2, 20, 16
+    q, k, v = make_inputs(B, H, world * c, D, "bf16", seed=6)
+    dout = torch.randn(q.shape, generator=torch.Generator().manual_seed(7)).to(torch.bfloat16)
+    refs = oracle.attn_bwd(q, k, v, dout, 0.25, causal, "bf16")
+    for name, ref in zip(("dq", "dk", "dv"), refs):
+        got = np.concatenate([np.load(tmp_path / f"{name}{r}.npy") for r in range(world)], axis=2)
+        assert np.max(np.abs(got - ref)) <= 1e-10, name

@@ -127,3 +127,77 @@ def test_merge_finalize_rounds_to_nearest_even():
                                     torch.cuda.current_stream().cuda_stream) == 0
         torch.cuda.synchronize()
         assert torch.equal(out.cpu(), x.to(tdt))
+
+
+def _run_ranks_in_threads(world, fn):
+    """fn(rank, exchange) for every rank, each in its own thread; exchange hands a
+    payload to rank + 1 and returns the one from rank - 1.  All threads launch on
+    the same CUDA stream, so the launch order orders the work."""
+    import queue
+    import threading
+    boxes = [queue.Queue() for _ in range(world)]
+    results, errors = [None] * world, []
+
+    def make_exchange(r):
+        def exchange(step, payload):
+            boxes[(r + 1) % world].put(payload)
+            return None, boxes[r].get(timeout=120)
+        return exchange
+
+    def body(r):
+        try:
+            results[r] = fn(r, make_exchange(r))
+        except Exception as e:  # re-raised in the test thread
+            errors.append(e)
+
+    threads = [threading.Thread(target=body, args=(r,)) for r in range(world)]
+    for t in threads:
+        t.start()
+    for t in threads:
+        t.join(timeout=300)
+    if errors:
+        raise errors[0]
+    return results
+
+
+@pytest.mark.parametrize("world", [2, 4])
+@pytest.mark.parametrize("causal", [False, True], ids=["full", "causal"])
+@pytest.mark.parametrize("dtype,D", [("bf16", 128), ("fp16", 64)])
+def test_ring_backward_through_the_kernels(world, causal, dtype, D):
+    """Every rank's ring backward (fa_bwd partials for the global O and LSE,
+    fa_accumulate, fa_merge_finalize) on one GPU; the gathered gradients against
+    the oracle's gradients over the whole sequence.  Each rank rounds its 16-bit
+    partials once before the fp32 sums and the sums once at the end: together at
+    most 2 more units of u * mag than one fa_bwd call, hence the bound c = 4."""
+    from gpu_helpers import compare_bwd
+    from tiled_attention_18_b200.sequence_parallel import ring_attention_backward
+    B, H, S = 1, 3, 512
+    c = S // world
+    q, k, v = make_inputs(B, H, S, D, dtype, seed=world + D)
+    dout = torch.randn(q.shape, generator=torch.Generator().manual_seed(5)).to(q.dtype)
+    scale = softmax_scale(D)
+    dq, dk, dv, ddo = (t.cuda() for t in (q, k, v, dout))
+    o, lse = fa.flash_attention_forward(dq, dk, dv, scale, causal)  # the forward's global rows
+    part = lambda t, r: t[:, :, r * c:(r + 1) * c].contiguous()  # noqa: E731
+
+    def rank_fn(r, exchange):
+        return ring_attention_backward(part(dq, r), part(dk, r), part(dv, r), part(o, r), part(lse, r),
+                                       part(ddo, r), scale, causal, ops=CudaOps(scale), exchange=exchange, rank=r,
+                                       world=world)
+
+    res = _run_ranks_in_threads(world, rank_fn)
+    assert fa.fa_check_status(torch.cuda.current_stream().cuda_stream) == 0
+    torch.cuda.synchronize()
+    grads = tuple(torch.cat([res[r][i] for r in range(world)], dim=2).cpu() for i in range(3))
+    refs = oracle.attn_bwd(q, k, v, dout, scale, causal, dtype, magnitudes=True)
+    print(compare_bwd(grads, refs[:3], refs[3:], dtype, q, k, dout, scale, causal, c=4.0))
+
+
+def test_accumulate_kernel():
+    for tdt, code, n in ((torch.bfloat16, 1, 4096), (torch.float16, 0, 1001)):
+        x = torch.randn(n, generator=torch.Generator().manual_seed(n)).to(tdt)
+        acc0 = torch.randn(n, generator=torch.Generator().manual_seed(n + 1))
+        dacc, dx = acc0.cuda(), x.cuda()
+        assert fa.fa_accumulate(dacc.data_ptr(), dx.data_ptr(), n, code, torch.cuda.current_stream().cuda_stream) == 0
+        torch.cuda.synchronize()
+        assert torch.equal(dacc.cpu(), acc0 + x.float())

@@ -8,12 +8,12 @@ in Python or PyTorch, and there is no fallback path.
 """
 from __future__ import annotations
 
-from ._lib import (FA_BF16, FA_FP16, FaError, fa_bwd, fa_bwd_dropout, fa_bwd_ex, fa_bwd_mask, fa_bwd_workspace_size,
+from ._lib import (FA_BF16, FA_FP16, FaError, fa_accumulate, fa_bwd, fa_bwd_dropout, fa_bwd_ex, fa_bwd_mask, fa_bwd_workspace_size,
                    fa_check_status, fa_fwd, fa_fwd_dropout, fa_fwd_ex, fa_fwd_mask, fa_fwd_noalloc, fa_merge_finalize, fa_merge_partial, fa_last_timeout_site, fa_num_units, fa_selftest_timeout, fa_status_string,
                    fa_version, load)
 
 __all__ = [
-    "FA_BF16", "FA_FP16", "FaError", "fa_bwd", "fa_bwd_dropout", "fa_bwd_ex", "fa_bwd_mask", "fa_bwd_workspace_size",
+    "FA_BF16", "FA_FP16", "FaError", "fa_accumulate", "fa_bwd", "fa_bwd_dropout", "fa_bwd_ex", "fa_bwd_mask", "fa_bwd_workspace_size",
     "fa_check_status", "fa_fwd", "fa_fwd_dropout", "fa_fwd_ex",
     "fa_fwd_mask", "fa_merge_finalize", "fa_merge_partial", "flash_attention_backward",
     "fa_fwd_noalloc", "fa_last_timeout_site",

@@ -70,6 +70,7 @@ SIGNATURES = [
      [ctypes.c_void_p] * 10 + [ctypes.c_longlong, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                ctypes.c_int, ctypes.c_float, ctypes.c_int, ctypes.c_float, ctypes.c_ulonglong,
                                ctypes.c_uint, ctypes.c_int, ctypes.c_int, ctypes.c_void_p]),
+    ("fa_accumulate", ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_longlong, ctypes.c_int, ctypes.c_void_p]),
     ("fa_merge_partial", ctypes.c_int,
      [ctypes.c_void_p] * 4 + [ctypes.c_longlong, ctypes.c_int, ctypes.c_int, ctypes.c_void_p]),
     ("fa_merge_finalize", ctypes.c_int,
@@ -204,6 +205,11 @@ def fa_bwd_dropout(q_ptr: int, k_ptr: int, v_ptr: int, o_ptr: int, do_ptr: int, 
                                      int(ws_bytes), B, H, Sq, Sk, D, float(scale), int(causal), float(dropout_p),
                                      int(seed) & (2**64 - 1), int(offset) & 0xffffffff, int(deterministic),
                                      int(dtype), stream))
+
+
+def fa_accumulate(acc_ptr: int, x_ptr: int, n: int, dtype: int, stream: int) -> int:
+    """Raw C call: acc (fp32) += x (16-bit) over n values."""
+    return int(load().fa_accumulate(acc_ptr, x_ptr, int(n), int(dtype), stream))
 
 
 def fa_merge_partial(o_acc_ptr: int, lse_acc_ptr: int, o_part_ptr: int, lse_part_ptr: int, rows: int, D: int,

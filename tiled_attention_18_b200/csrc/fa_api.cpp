@@ -557,6 +557,27 @@ int fa_merge_finalize(const float* o_acc, void* o, long long n, int dtype, cudaS
     return FA_OK;
 }
 
+int fa_accumulate(float* acc, const void* x, long long n, int dtype, cudaStream_t stream) {
+    if (n < 0) return FA_ERR_SHAPE;
+    if (dtype != FA_FP16 && dtype != FA_BF16) return FA_ERR_DTYPE;
+    if (n == 0) return FA_OK;
+    if (!acc || !x) return FA_ERR_NULL;
+    if (((uintptr_t)acc & 3u) != 0 || ((uintptr_t)x & 1u) != 0) return FA_ERR_ALIGN;
+    int cur = 0;
+    if (cudaGetDevice(&cur) != cudaSuccess) {
+        cudaGetLastError();
+        return FA_ERR_LAUNCH;
+    }
+    int rc = check_device_pointer(acc, cur);
+    if (rc == FA_OK) rc = check_device_pointer(x, cur);
+    if (rc != FA_OK) return rc;
+    if (fa::launch_accumulate(acc, x, n, dtype, stream) != cudaSuccess) {
+        cudaGetLastError();
+        return FA_ERR_LAUNCH;
+    }
+    return FA_OK;
+}
+
 int fa_check_status(cudaStream_t stream) {
     // one status word per kernel translation unit; all are read and cleared
     int st[3] = {0, 0, 0}, site[3] = {0, 0, 0};

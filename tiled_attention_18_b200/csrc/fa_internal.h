@@ -113,6 +113,7 @@ inline BwdWorkspace bwd_workspace_layout(int64_t BH, int64_t Sq, int64_t D) {
 // and the conversion of the running O to 16 bits (fa_merge_sm100.cu).
 cudaError_t launch_merge_partial(float* o_acc, float* lse_acc, const void* o_part, const float* lse_part,
                                  long long rows, int D, int dtype, cudaStream_t stream);
+cudaError_t launch_accumulate(float* acc, const void* x, long long n, int dtype, cudaStream_t stream);
 cudaError_t launch_merge_finalize(const float* o_acc, void* o, long long n, int dtype, cudaStream_t stream);
 
 // Launch the three backward kernels (prep, main, post) on `stream`.

@@ -1,5 +1,6 @@
 // fa_merge_sm100.cu -- merging partial attention results by their log-sum-exp
-// (declared in include/fa.h: fa_merge_partial, fa_merge_finalize).
+// and accumulating partial gradients (declared in include/fa.h:
+// fa_merge_partial, fa_merge_finalize, fa_accumulate).
 //
 // Attention over a key set split into blocks is the LSE-weighted combination
 // of the attention over each block: with (O_a, L_a) and (O_b, L_b) for two
@@ -88,7 +89,39 @@ __global__ void __launch_bounds__(256) finalize_kernel(const float* __restrict__
         o[i] = from_f32<BF16>(o_acc[i]);
 }
 
+// acc += x for n values: fp32 accumulators of partial gradients (16-bit x),
+// four per thread when n, acc and x allow it.
+template <bool BF16>
+__global__ void __launch_bounds__(256) accumulate_kernel(float* __restrict__ acc, const uint16_t* __restrict__ x,
+                                                         long long n) {
+    const long long step = (long long)gridDim.x * blockDim.x;
+    long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if ((n & 3) == 0 && ((uintptr_t)acc & 15) == 0 && ((uintptr_t)x & 7) == 0) {
+        for (; i < n / 4; i += step) {
+            const uint2 r = reinterpret_cast<const uint2*>(x)[i];
+            float4 a = reinterpret_cast<float4*>(acc)[i];
+            a.x += to_f32<BF16>((uint16_t)(r.x & 0xffffu));
+            a.y += to_f32<BF16>((uint16_t)(r.x >> 16));
+            a.z += to_f32<BF16>((uint16_t)(r.y & 0xffffu));
+            a.w += to_f32<BF16>((uint16_t)(r.y >> 16));
+            reinterpret_cast<float4*>(acc)[i] = a;
+        }
+    } else {
+        for (; i < n; i += step) acc[i] += to_f32<BF16>(x[i]);
+    }
+}
+
 }  // namespace
+
+cudaError_t launch_accumulate(float* acc, const void* x, long long n, int dtype, cudaStream_t stream) {
+    const long long want = (n / 4 + 255) / 256 + 1;
+    const unsigned blocks = (unsigned)(want < 148 * 32 ? want : 148 * 32);
+    if (dtype == 1)
+        accumulate_kernel<true><<<blocks, 256, 0, stream>>>(acc, static_cast<const uint16_t*>(x), n);
+    else
+        accumulate_kernel<false><<<blocks, 256, 0, stream>>>(acc, static_cast<const uint16_t*>(x), n);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_merge_partial(float* o_acc, float* lse_acc, const void* o_part, const float* lse_part,
                                  long long rows, int D, int dtype, cudaStream_t stream) {

@@ -19,6 +19,13 @@ K/V synchronised between devices by collective communication).  Two ways:
   With the causal mask a rank skips the blocks that come after its own and
   uses the causal kernel on its own block.  Memory: two K/V blocks.
 
+``ring_attention_backward`` gives the gradients of the ring forward (the
+section's setting is distributed training): with the global O and LSE of the
+forward, ``fa_bwd`` on (this rank's queries, one K/V block) yields exactly that
+block's share of dQ, dK and dV, so dQ accumulates locally while every K/V
+block travels the ring together with fp32 accumulators of its dK and dV
+(``fa_accumulate``), one more step than the forward, back to its owner.
+
 Every step of the attention runs in the library's kernels; this module only
 orders the launches and the communication.  The ``ops`` and ``exchange``
 parameters exist so that tests can drive the same schedule with stand-ins
@@ -81,6 +88,43 @@ class CudaOps:
                               o_acc.shape[-1], _dtype_code(o_part), self._sid(o_acc))
         if rc != 0:
             raise FaError(rc, "fa_merge_partial")
+
+    # -- backward
+    def __init_bwd(self, q):
+        import torch
+        from . import fa_bwd_workspace_size
+        B, H, S, D = q.shape
+        n = fa_bwd_workspace_size(B, H, S, D)
+        if getattr(self, "_ws", None) is None or self._ws.numel() < n:
+            self._ws = torch.empty(max(n, 1), dtype=torch.uint8, device=q.device)
+
+    def zeros_f32(self, t):
+        import torch
+        return torch.zeros(t.shape, dtype=torch.float32, device=t.device)
+
+    def bwd_partial(self, q, k, v, o, lse, dout, causal: bool, deterministic: bool = False):
+        """This block's share of dQ, dK, dV (16-bit) for the rows' global O and LSE."""
+        from . import flash_attention_backward
+        self.__init_bwd(q)
+        return flash_attention_backward(q, k.contiguous(), v.contiguous(), o, lse, dout, self.scale, causal,
+                                        deterministic=deterministic, workspace=self._ws, stream=self.stream)
+
+    def accumulate(self, acc, x):
+        from . import FaError, fa_accumulate
+        code = 1 if str(x.dtype) == "torch.bfloat16" else 0
+        rc = fa_accumulate(acc.data_ptr(), x.data_ptr(), x.numel(), code, self._sid(acc))
+        if rc != 0:
+            raise FaError(rc, "fa_accumulate")
+
+    def to16(self, acc, dtype):
+        import torch
+        from . import FaError, fa_merge_finalize
+        out = torch.empty(acc.shape, dtype=dtype, device=acc.device)
+        code = 1 if dtype == torch.bfloat16 else 0
+        rc = fa_merge_finalize(acc.data_ptr(), out.data_ptr(), acc.numel(), code, self._sid(acc))
+        if rc != 0:
+            raise FaError(rc, "fa_merge_finalize")
+        return out
 
     def finalize(self, state):
         import torch
@@ -178,3 +222,59 @@ def allgather_attention_forward(q, k, v, scale: float, causal: bool = False, gro
     kf = full[0, :, :, :n_keys].contiguous()
     vf = full[1, :, :, :n_keys].contiguous()
     return ops.partial(q, kf, vf, causal)
+
+
+def _p2p_ring_exchange_tuple(group, rank: int, world: int):
+    """Send a tuple of tensors to rank + 1 and receive tensors of the same shapes
+    from rank - 1 (one batched P2P call per step)."""
+    import torch
+    import torch.distributed as dist
+
+    nxt = dist.get_global_rank(group, (rank + 1) % world) if group is not None else (rank + 1) % world
+    prv = dist.get_global_rank(group, (rank - 1) % world) if group is not None else (rank - 1) % world
+
+    def exchange(step: int, payload):
+        recv = tuple(torch.empty_like(t) for t in payload)
+        ops = [dist.P2POp(dist.isend, t, nxt, group) for t in payload]
+        ops += [dist.P2POp(dist.irecv, r, prv, group) for r in recv]
+        return dist.batch_isend_irecv(ops), recv
+
+    return exchange
+
+
+def ring_attention_backward(q, k, v, o, lse, dout, scale: float, causal: bool = False, group=None, ops=None,
+                            exchange: Optional[Callable] = None, rank: Optional[int] = None,
+                            world: Optional[int] = None, deterministic: bool = False):
+    """dQ, dK, dV of this rank's chunks for the ring forward.
+
+    q, k, v, dout: this rank's chunks [B, H, c, D]; o, lse: this rank's rows of
+    the forward over the whole sequence (ring_attention_forward's output).  At
+    step s the rank holds the K/V block of rank (rank - s) mod world with the
+    fp32 dK/dV accumulated for it so far, adds its queries' share, and passes
+    both on; after world exchanges each rank holds its own block again with
+    every rank's share added.  dQ is summed locally in fp32.  The causal mask
+    skips blocks after the rank's own and uses the causal kernel on its own.
+    """
+    import torch
+    import torch.distributed as dist
+
+    if rank is None:
+        rank = dist.get_rank(group)
+    if world is None:
+        world = dist.get_world_size(group)
+    ops = ops if ops is not None else CudaOps(scale)
+    if exchange is None:
+        exchange = _p2p_ring_exchange_tuple(group, rank, world)
+    kv = torch.stack([k, v])                 # the block being carried: [2, B, H, c, D]
+    acc = ops.zeros_f32(kv)                  # its dK, dV so far (fp32)
+    dq_acc = ops.zeros_f32(q)
+    for s, (src, mode) in enumerate(ring_schedule(rank, world, causal)):
+        if mode != "skip":
+            dq_p, dk_p, dv_p = ops.bwd_partial(q, kv[0], kv[1], o, lse, dout, mode == "causal", deterministic)
+            ops.accumulate(dq_acc, dq_p)
+            ops.accumulate(acc[0], dk_p)
+            ops.accumulate(acc[1], dv_p)
+        reqs, (kv, acc) = exchange(s, (kv, acc))
+        for r in reqs or []:
+            r.wait()
+    return ops.to16(dq_acc, q.dtype), ops.to16(acc[0], k.dtype), ops.to16(acc[1], v.dtype)
