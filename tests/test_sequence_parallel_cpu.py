@@ -156,3 +156,48 @@ def test_ring_backward_ranks_equal_full_gradients(tmp_path, world, causal):
     for name, ref in zip(("dq", "dk", "dv"), refs):
         got = np.concatenate([np.load(tmp_path / f"{name}{r}.npy") for r in range(world)], axis=2)
         assert np.max(np.abs(got - ref)) <= 1e-10, name
+
+
+def _ulysses_worker(rank, world, port, causal, out_dir):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        import oracle
+        from tiled_attention_18_b200.sequence_parallel import ulysses_attention_backward, ulysses_attention_forward
+        from tiled_attention_18_b200.workloads import make_inputs
+        B, H, c, D = 1, 2 * world, 16, 8
+        q, k, v = make_inputs(B, H, world * c, D, "bf16", seed=8)
+        dout = torch.randn(q.shape, generator=torch.Generator().manual_seed(9)).to(torch.bfloat16)
+        sl = slice(rank * c, (rank + 1) * c)
+        part = lambda t: t[:, :, sl].contiguous()  # noqa: E731
+        o, lse = ulysses_attention_forward(part(q), part(k), part(v), 0.25, causal, ops=OracleOps(0.25, "bf16"))
+        # the backward with the oracle's global rows as the forward output (float64 stand-in)
+        o_full, lse_full = oracle.attn_fwd(q, k, v, 0.25, causal, "bf16")
+        dq, dk, dv = ulysses_attention_backward(part(q), part(k), part(v),
+                                                torch.from_numpy(o_full[:, :, sl].copy()),
+                                                torch.from_numpy(lse_full[:, :, sl].copy()), part(dout), 0.25,
+                                                causal, ops=GradOps(0.25))
+        for name, t in (("o", o), ("l", lse), ("dq", dq), ("dk", dk), ("dv", dv)):
+            np.save(os.path.join(out_dir, f"u{name}{rank}.npy"), t.numpy())
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 3])
+@pytest.mark.parametrize("causal", [False, True])
+def test_ulysses_ranks_equal_full_attention(tmp_path, world, causal):
+    """Head-parallel sequence parallelism over gloo: forward and backward equal
+    the oracle over the whole sequence."""
+    import oracle
+    from tiled_attention_18_b200.workloads import make_inputs
+    mp.spawn(_ulysses_worker, args=(world, _free_port(), causal, str(tmp_path)), nprocs=world, join=True)
+    B, H, c, D = 1, 2 * world, 16, 8
+    q, k, v = make_inputs(B, H, world * c, D, "bf16", seed=8)
+    dout = torch.randn(q.shape, generator=torch.Generator().manual_seed(9)).to(torch.bfloat16)
+    o_ref, lse_ref = oracle.attn_fwd(q, k, v, 0.25, causal, "bf16")
+    refs = dict(zip(("dq", "dk", "dv"), oracle.attn_bwd(q, k, v, dout, 0.25, causal, "bf16")))
+    refs.update(o=o_ref, l=lse_ref)
+    for name, ref in refs.items():
+        got = np.concatenate([np.load(tmp_path / f"u{name}{r}.npy") for r in range(world)], axis=2)
+        assert np.max(np.abs(got - ref)) <= 1e-10, name

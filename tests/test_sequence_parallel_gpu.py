@@ -201,3 +201,61 @@ def test_accumulate_kernel():
         assert fa.fa_accumulate(dacc.data_ptr(), dx.data_ptr(), n, code, torch.cuda.current_stream().cuda_stream) == 0
         torch.cuda.synchronize()
         assert torch.equal(dacc.cpu(), acc0 + x.float())
+
+
+class _ThreadAllToAll:
+    """all-to-all among threads: rank r's x[p] goes to rank p, which gets them
+    stacked by source rank.  Two barriers per call: all have written, all
+    have read."""
+
+    def __init__(self, world):
+        import threading
+        self.world = world
+        self.slots = [[None] * world for _ in range(world)]
+        self.barrier = threading.Barrier(world)
+
+    def make(self, r):
+        def a2a(x):
+            for p in range(self.world):
+                self.slots[p][r] = x[p]
+            self.barrier.wait(timeout=120)
+            out = torch.stack([self.slots[r][p] for p in range(self.world)])
+            self.barrier.wait(timeout=120)
+            return out
+        return a2a
+
+
+@pytest.mark.parametrize("world", [2, 4])
+@pytest.mark.parametrize("causal", [False, True], ids=["full", "causal"])
+@pytest.mark.parametrize("dtype,D", [("bf16", 128), ("fp16", 64)])
+def test_ulysses_through_the_kernels(world, causal, dtype, D):
+    """Head-parallel forward and backward, every rank in its own thread on one
+    GPU: the kernels run on whole heads, so the results are those of single
+    calls on the full sequence (forward tolerance; backward bound of fa_bwd)."""
+    from gpu_helpers import compare, compare_bwd
+    from tiled_attention_18_b200.sequence_parallel import ulysses_attention_backward, ulysses_attention_forward
+    B, H, S = 1, 4, 512
+    c = S // world
+    q, k, v = make_inputs(B, H, S, D, dtype, seed=world + 2 * D)
+    dout = torch.randn(q.shape, generator=torch.Generator().manual_seed(6)).to(q.dtype)
+    scale = softmax_scale(D)
+    dq, dk, dv, ddo = (t.cuda() for t in (q, k, v, dout))
+    part = lambda t, r: t[:, :, r * c:(r + 1) * c].contiguous()  # noqa: E731
+    comm = _ThreadAllToAll(world)
+
+    def rank_fn(r, _exchange):
+        ops = CudaOps(scale)
+        o, lse = ulysses_attention_forward(part(dq, r), part(dk, r), part(dv, r), scale, causal, ops=ops,
+                                           alltoall=comm.make(r), rank=r, world=world)
+        grads = ulysses_attention_backward(part(dq, r), part(dk, r), part(dv, r), o, lse, part(ddo, r), scale,
+                                           causal, ops=ops, alltoall=comm.make(r), rank=r, world=world)
+        return (o, lse) + grads
+
+    res = _run_ranks_in_threads(world, rank_fn)
+    assert fa.fa_check_status(torch.cuda.current_stream().cuda_stream) == 0
+    torch.cuda.synchronize()
+    cat = [torch.cat([res[r][i] for r in range(world)], dim=2).cpu() for i in range(5)]
+    o_ref, lse_ref = oracle.attn_fwd(q, k, v, scale, causal, dtype)
+    compare(cat[0], cat[1], o_ref, lse_ref, dtype)
+    refs = oracle.attn_bwd(q, k, v, dout, scale, causal, dtype, magnitudes=True)
+    print(compare_bwd(tuple(cat[2:]), refs[:3], refs[3:], dtype, q, k, dout, scale, causal))

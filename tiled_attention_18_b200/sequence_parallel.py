@@ -19,6 +19,11 @@ K/V synchronised between devices by collective communication).  Two ways:
   With the causal mask a rank skips the blocks that come after its own and
   uses the causal kernel on its own block.  Memory: two K/V blocks.
 
+- ``ulysses_attention_forward`` / ``ulysses_attention_backward``: head
+  parallelism inside the sequence-parallel group: one all-to-all gives each
+  rank H / world heads over the whole sequence, the unmodified kernels run on
+  them, and one all-to-all returns the results (no merge).
+
 ``ring_attention_backward`` gives the gradients of the ring forward (the
 section's setting is distributed training): with the global O and LSE of the
 forward, ``fa_bwd`` on (this rank's queries, one K/V block) yields exactly that
@@ -278,3 +283,104 @@ def ring_attention_backward(q, k, v, o, lse, dout, scale: float, causal: bool = 
         for r in reqs or []:
             r.wait()
     return ops.to16(dq_acc, q.dtype), ops.to16(acc[0], k.dtype), ops.to16(acc[1], v.dtype)
+
+
+# ------------------------------------------------------------------ all-to-all (head-parallel)
+
+def _alltoall_default(group, world: int):
+    """all_to_all over ``group`` of a tensor whose leading dimension indexes the
+    destination rank; returns the tensor whose leading dimension indexes the source."""
+    import torch
+    import torch.distributed as dist
+
+    def a2a(x):
+        out = torch.empty_like(x)
+        dist.all_to_all_single(out, x.contiguous(), group=group)
+        return out
+
+    return a2a
+
+
+def _to_heads(x, world: int, c: int):
+    """[B, H, c, D] chunk (this rank's positions, all heads) -> [world, B, H/world, c, D],
+    leading dimension = the rank that owns that head group."""
+    B, H, _, D = x.shape
+    return x.reshape(B, world, H // world, c, D).permute(1, 0, 2, 3, 4)
+
+
+def _gather_positions(y, world: int, c: int):
+    """[world(source), B, Hw, c, D] -> [B, Hw, world * c, D]: the source ranks' chunks in
+    sequence order."""
+    W, B, Hw, _, D = y.shape
+    return y.permute(1, 2, 0, 3, 4).reshape(B, Hw, W * c, D)
+
+
+def _scatter_positions(x, world: int, c: int):
+    """[B, Hw, world * c, ...] -> [world(destination), B, Hw, c, ...]."""
+    B, Hw = x.shape[:2]
+    rest = tuple(x.shape[3:])
+    return x.reshape((B, Hw, world, c) + rest).permute((2, 0, 1, 3) + tuple(range(4, 4 + len(rest))))
+
+
+def _back_to_chunk(y, world: int):
+    """[world(source = head group), B, Hw, c, ...] -> [B, world * Hw, c, ...] (all heads
+    of this rank's positions)."""
+    W, B, Hw, c = y.shape[:4]
+    rest = tuple(y.shape[4:])
+    return y.permute((1, 0, 2, 3) + tuple(range(4, 4 + len(rest)))).reshape((B, W * Hw, c) + rest)
+
+
+def ulysses_attention_forward(q, k, v, scale: float, causal: bool = False, group=None, ops=None,
+                              alltoall: Optional[Callable] = None, rank: Optional[int] = None,
+                              world: Optional[int] = None):
+    """O and LSE of this rank's query chunk by head-parallel attention: one
+    all-to-all turns the sequence-sharded Q, K, V ([B, H, c, D] per rank) into
+    head-sharded full sequences ([B, H / world, world * c, D]), each rank runs
+    the attention of its heads over the whole sequence (causal mask included,
+    the positions being in order), and one all-to-all returns O and LSE to the
+    ranks that own the positions.  H must be a multiple of world.  No merge is
+    needed: each head's attention runs in one kernel call."""
+    import torch
+    import torch.distributed as dist
+
+    if rank is None:
+        rank = dist.get_rank(group)
+    if world is None:
+        world = dist.get_world_size(group)
+    B, H, c, D = q.shape
+    if H % world:
+        raise ValueError("the head count must be a multiple of the group size")
+    ops = ops if ops is not None else CudaOps(scale)
+    a2a = alltoall if alltoall is not None else _alltoall_default(group, world)
+    recv = a2a(torch.stack([_to_heads(t, world, c) for t in (q, k, v)], dim=1))  # [W, 3, B, Hw, c, D]
+    qh, kh, vh = (_gather_positions(recv[:, i], world, c).contiguous() for i in range(3))
+    o, lse = ops.partial(qh, kh, vh, causal)
+    o_back = a2a(_scatter_positions(o, world, c).contiguous())             # [W, B, Hw, c, D]
+    l_back = a2a(_scatter_positions(lse, world, c).contiguous())           # [W, B, Hw, c]
+    return _back_to_chunk(o_back, world).contiguous(), _back_to_chunk(l_back, world).contiguous()
+
+
+def ulysses_attention_backward(q, k, v, o, lse, dout, scale: float, causal: bool = False, group=None, ops=None,
+                               alltoall: Optional[Callable] = None, rank: Optional[int] = None,
+                               world: Optional[int] = None, deterministic: bool = False):
+    """dQ, dK, dV of this rank's chunks for ulysses_attention_forward: the
+    inputs, O, dO and LSE go to the head owners by one all-to-all, each rank
+    runs the backward of its heads over the whole sequence, and the gradients
+    come back by another."""
+    import torch
+    import torch.distributed as dist
+
+    if rank is None:
+        rank = dist.get_rank(group)
+    if world is None:
+        world = dist.get_world_size(group)
+    B, H, c, D = q.shape
+    ops = ops if ops is not None else CudaOps(scale)
+    a2a = alltoall if alltoall is not None else _alltoall_default(group, world)
+    recv = a2a(torch.stack([_to_heads(t, world, c) for t in (q, k, v, o, dout)], dim=1))  # [W, 5, B, Hw, c, D]
+    qh, kh, vh, oh, doh = (_gather_positions(recv[:, i], world, c).contiguous() for i in range(5))
+    lh = a2a(lse.reshape(B, world, H // world, c).permute(1, 0, 2, 3).contiguous())      # [W, B, Hw, c]
+    lh = lh.permute(1, 2, 0, 3).reshape(B, H // world, world * c).contiguous()
+    dq, dk, dv = ops.bwd_partial(qh, kh, vh, oh, lh, doh, causal, deterministic)
+    grads = a2a(torch.stack([_scatter_positions(g, world, c) for g in (dq, dk, dv)], dim=1).contiguous())
+    return tuple(_back_to_chunk(grads[:, i], world).contiguous() for i in range(3))
