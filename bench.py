@@ -485,9 +485,18 @@ def run_sp(args) -> int:
     for w in runs:
         q, k, v = (t.to(dev) for t in workload_inputs(w))
         c = w.S // W
-        qs = [q[:, :, r * c:(r + 1) * c].contiguous() for r in range(W)]
-        kv = [torch.stack([k[:, :, r * c:(r + 1) * c], v[:, :, r * c:(r + 1) * c]]).contiguous() for r in range(W)]
-        data.append((w, qs, kv, torch.stack(kv) if args.sp_mode == "allgather" else None))
+        if args.sp_mode == "ulysses":
+            if w.H % W:
+                raise SystemExit("--sp-mode ulysses needs H divisible by --sp-world")
+            hw = w.H // W
+            # each rank's head group over the whole sequence (what the all-to-all delivers)
+            heads = [tuple(t[:, r * hw:(r + 1) * hw].contiguous() for t in (q, k, v)) for r in range(W)]
+            data.append((w, heads, None, None))
+        else:
+            qs = [q[:, :, r * c:(r + 1) * c].contiguous() for r in range(W)]
+            kv = [torch.stack([k[:, :, r * c:(r + 1) * c], v[:, :, r * c:(r + 1) * c]]).contiguous()
+                  for r in range(W)]
+            data.append((w, qs, kv, torch.stack(kv) if args.sp_mode == "allgather" else None))
         del q, k, v
 
     class TimedOps(CudaOps):
@@ -518,6 +527,9 @@ def run_sp(args) -> int:
         for (w, qs, kv, stacked) in data:
             ops = TimedOps(w.scale, log)
             for r in range(W):
+                if args.sp_mode == "ulysses":
+                    ops.partial(*qs[r], w.causal)
+                    continue
                 qk = qs[r]
                 if args.sp_mode == "ring":
                     ring_attention_forward(qk, kv[r][0], kv[r][1], w.scale, w.causal, ops=ops, rank=r, world=W,
@@ -607,7 +619,7 @@ def main(argv=None) -> int:
                     help="fwd: the forward pass (default); bwd: the backward pass fa_bwd; sp: the "
                          "sequence-parallel schedule of --sp-world ranks run in turn on one GPU")
     ap.add_argument("--sp-world", type=int, default=4, help="with --pass sp: ranks of the schedule")
-    ap.add_argument("--sp-mode", choices=["ring", "allgather"], default="ring", help="with --pass sp")
+    ap.add_argument("--sp-mode", choices=["ring", "allgather", "ulysses"], default="ring", help="with --pass sp")
     ap.add_argument("--mask", choices=["none", "tril"], default="none",
                     help="tril: causal runs go through fa_fwd_mask with an explicit lower-triangular mask "
                          "(the catlass page's mode 1) instead of the in-kernel diagonal skip (mode 2)")
