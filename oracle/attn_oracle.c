@@ -1,5 +1,8 @@
 /*
- * attn_oracle.c -- plain, slow, fp64 CPU oracle for the attention forward pass.
+ * attn_oracle.c -- plain, slow, fp64 CPU oracle for attention: the forward
+ * pass (square and general shapes, causal, explicit mask, dropout) and its
+ * gradients (the backward section below), with each function's definition
+ * and sources stated where it is defined.
  *
  * TEST INFRASTRUCTURE ONLY.  Nothing on the product path (the CUDA library
  * and its Python binding) may link, load or call this file.  It is used by
