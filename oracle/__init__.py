@@ -128,6 +128,16 @@ def _load():
         lib.oracle_attn_fwd_dropout.argtypes = [u16p, u16p, u16p, i64, i64, i64, i64, i64, ctypes.c_float,
                                                 ctypes.c_int, ctypes.c_int, u32, ctypes.c_uint64, u32, f64p, f64p]
         lib.oracle_attn_fwd_dropout.restype = ctypes.c_int
+        u8p = ctypes.POINTER(ctypes.c_uint8)
+        lib.oracle_attn_fwd_dropout_masked.argtypes = [u16p, u16p, u16p, i64, i64, i64, i64, i64, ctypes.c_float,
+                                                       ctypes.c_int, ctypes.c_int, u32, ctypes.c_uint64, u32, u8p,
+                                                       i64, i64, i64, f64p, f64p]
+        lib.oracle_attn_fwd_dropout_masked.restype = ctypes.c_int
+        lib.oracle_attn_bwd_dropout_masked.argtypes = [u16p, u16p, u16p, u16p, i64, i64, i64, i64, i64,
+                                                       ctypes.c_float, ctypes.c_int, ctypes.c_int, u32,
+                                                       ctypes.c_uint64, u32, u8p, i64, i64, i64, f64p, f64p, f64p,
+                                                       f64p, f64p, f64p]
+        lib.oracle_attn_bwd_dropout_masked.restype = ctypes.c_int
         lib.oracle_attn_rows_dropout.argtypes = [u16p, u16p, u16p, i64, i64, i64, i64, i64, ctypes.c_float,
                                                  ctypes.c_int, ctypes.c_int, u32, ctypes.c_uint64, u32, i64p, i64p,
                                                  i64, f64p, f64p]
@@ -357,20 +367,35 @@ def dropout_keep_mask(BH: int, Sq: int, Sk: int, p8: int, seed: int, offset: int
     return keep
 
 
-def attn_fwd_dropout(q, k, v, scale: float, causal: bool, dtype, p8: int, seed: int, offset: int):
+def _mask_args(mask, B, H, Sq, Sk):
+    """(array, strides over b, h, row) of a [B|1, H|1, Sq, Sk] mask, or (None, 0, 0, 0)."""
+    if mask is None:
+        return None, 0, 0, 0
+    m = np.asarray(mask.cpu().numpy() if hasattr(mask, "cpu") else mask).astype(np.uint8)
+    if m.ndim != 4 or m.shape[2:] != (Sq, Sk) or m.shape[0] not in (1, B) or m.shape[1] not in (1, H):
+        raise ValueError("mask must be [B|1, H|1, Sq, Sk]")
+    m = np.ascontiguousarray(m)
+    return m, (0 if m.shape[0] == 1 else m.shape[1] * Sq * Sk), (0 if m.shape[1] == 1 else Sq * Sk), Sk
+
+
+def attn_fwd_dropout(q, k, v, scale: float, causal: bool, dtype, p8: int, seed: int, offset: int, mask=None):
     """attn_fwd_gen with dropout after the softmax: weights kept by the Philox rule
     of attn_oracle.c (threshold p8 in 1/256 units), kept weights scaled by
-    256 / (256 - p8); LSE of the undropped softmax."""
+    256 / (256 - p8); LSE of the undropped softmax.  ``mask`` (optional, as
+    attn_fwd_masked's) restricts the keys each row sees."""
     lib = _load()
     qb, kb, vb = _bits(q), _bits(k), _bits(v)
     B, H, Sq, D = qb.shape
     Sk = kb.shape[2]
     o = np.empty((B, H, Sq, D))
     lse = np.empty((B, H, Sq))
-    rc = lib.oracle_attn_fwd_dropout(_ptr(qb, ctypes.c_uint16), _ptr(kb, ctypes.c_uint16), _ptr(vb, ctypes.c_uint16),
-                                     B, H, Sq, Sk, D, float(np.float32(scale)), int(bool(causal)), _dtype_code(dtype),
-                                     int(p8), int(seed) & (2**64 - 1), int(offset) & 0xffffffff,
-                                     _ptr(o, ctypes.c_double), _ptr(lse, ctypes.c_double))
+    m, sb, sh, si = _mask_args(mask, B, H, Sq, Sk)
+    rc = lib.oracle_attn_fwd_dropout_masked(_ptr(qb, ctypes.c_uint16), _ptr(kb, ctypes.c_uint16),
+                                            _ptr(vb, ctypes.c_uint16), B, H, Sq, Sk, D, float(np.float32(scale)),
+                                            int(bool(causal)), _dtype_code(dtype), int(p8), int(seed) & (2**64 - 1),
+                                            int(offset) & 0xffffffff,
+                                            _ptr(m, ctypes.c_uint8) if m is not None else None, sb, sh, si,
+                                            _ptr(o, ctypes.c_double), _ptr(lse, ctypes.c_double))
     if rc != 0:
         raise RuntimeError(f"oracle_attn_fwd_dropout failed with {rc}")
     return o, lse
@@ -398,8 +423,8 @@ def attn_rows_dropout(q, k, v, scale: float, causal: bool, dtype, p8: int, seed:
 
 
 def attn_bwd_dropout(q, k, v, dout, scale: float, causal: bool, dtype, p8: int, seed: int, offset: int,
-                     magnitudes: bool = False):
-    """attn_bwd for the attention with dropout of attn_fwd_dropout."""
+                     magnitudes: bool = False, mask=None):
+    """attn_bwd for the attention with dropout (and optional mask) of attn_fwd_dropout."""
     lib = _load()
     qb, kb, vb, gb = _bits(q), _bits(k), _bits(v), _bits(dout)
     B, H, Sq, D = qb.shape
@@ -409,11 +434,13 @@ def attn_bwd_dropout(q, k, v, dout, scale: float, causal: bool, dtype, p8: int, 
     dv = np.empty((B, H, Sk, D))
     mags = tuple(np.empty(a.shape) for a in (dq, dk, dv)) if magnitudes else (None, None, None)
     fp = lambda a: _ptr(a, ctypes.c_double) if a is not None else None  # noqa: E731
-    rc = lib.oracle_attn_bwd_dropout(_ptr(qb, ctypes.c_uint16), _ptr(kb, ctypes.c_uint16), _ptr(vb, ctypes.c_uint16),
-                                     _ptr(gb, ctypes.c_uint16), B, H, Sq, Sk, D, float(np.float32(scale)),
-                                     int(bool(causal)), _dtype_code(dtype), int(p8), int(seed) & (2**64 - 1),
-                                     int(offset) & 0xffffffff, fp(dq), fp(dk), fp(dv), fp(mags[0]), fp(mags[1]),
-                                     fp(mags[2]))
+    m, sb, sh, si = _mask_args(mask, B, H, Sq, Sk)
+    rc = lib.oracle_attn_bwd_dropout_masked(_ptr(qb, ctypes.c_uint16), _ptr(kb, ctypes.c_uint16),
+                                            _ptr(vb, ctypes.c_uint16), _ptr(gb, ctypes.c_uint16), B, H, Sq, Sk, D,
+                                            float(np.float32(scale)), int(bool(causal)), _dtype_code(dtype), int(p8),
+                                            int(seed) & (2**64 - 1), int(offset) & 0xffffffff,
+                                            _ptr(m, ctypes.c_uint8) if m is not None else None, sb, sh, si,
+                                            fp(dq), fp(dk), fp(dv), fp(mags[0]), fp(mags[1]), fp(mags[2]))
     if rc != 0:
         raise RuntimeError(f"oracle_attn_bwd_dropout failed with {rc}")
     return (dq, dk, dv) + (mags if magnitudes else ())

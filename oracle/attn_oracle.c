@@ -602,10 +602,13 @@ int oracle_dropout_keep_mask(int64_t BH, int64_t Sq, int64_t Sk, uint32_t p8, ui
 /* One query row with dropout: the softmax over the nj visible keys, then
  * O = sum_j P_j z_j v_j.  An empty row gets O = 0, LSE = -inf. */
 static void dropout_row(const double *qi, const double *kh, const double *vh, int64_t nj, int64_t D, double scale,
-                        uint64_t seed, uint32_t offset, uint32_t p8, int64_t bh, int64_t i, double *srow, double *o,
-                        double *lse)
+                        uint64_t seed, uint32_t offset, uint32_t p8, int64_t bh, int64_t i, const uint8_t *mrow,
+                        double *srow, double *o, double *lse)
 {
-    if (nj <= 0) {
+    /* with an explicit mask the row sees only the keys its mask row allows */
+    int64_t nvis = 0;
+    for (int64_t j = 0; j < nj; ++j) nvis += mrow ? (mrow[j] != 0) : 1;
+    if (nvis == 0) {
         for (int64_t d = 0; d < D; ++d) o[d] = 0.0;
         *lse = -INFINITY;
         return;
@@ -614,7 +617,7 @@ static void dropout_row(const double *qi, const double *kh, const double *vh, in
     for (int64_t j = 0; j < nj; ++j) {
         double dot = 0.0;
         for (int64_t d = 0; d < D; ++d) dot += qi[d] * kh[j * D + d];
-        srow[j] = scale * dot;
+        srow[j] = (mrow && !mrow[j]) ? -INFINITY : scale * dot;
     }
     double m = -INFINITY;
     for (int64_t j = 0; j < nj; ++j)
@@ -626,6 +629,7 @@ static void dropout_row(const double *qi, const double *kh, const double *vh, in
     }
     for (int64_t d = 0; d < D; ++d) o[d] = 0.0;
     for (int64_t j = 0; j < nj; ++j) {
+        if (mrow && !mrow[j]) continue;
         if (!dropout_keep(seed, offset, p8, bh, i, j)) continue;
         const double w = srow[j] * zs;
         for (int64_t d = 0; d < D; ++d) o[d] += w * vh[j * D + d];
@@ -635,10 +639,12 @@ static void dropout_row(const double *qi, const double *kh, const double *vh, in
 }
 
 /* Attention with dropout, general shapes and the bottom-right causal mask of
- * oracle_attn_fwd_gen.  o: [B,H,Sq,D], lse: [B,H,Sq]. */
-int oracle_attn_fwd_dropout(const uint16_t *q, const uint16_t *k, const uint16_t *v, int64_t B, int64_t H,
-                            int64_t Sq, int64_t Sk, int64_t D, float scale, int causal, int dtype, uint32_t p8,
-                            uint64_t seed, uint32_t offset, double *o, double *lse)
+ * oracle_attn_fwd_gen, and optionally an explicit mask (the convention of
+ * oracle_attn_fwd_masked; mask = NULL: none).  o: [B,H,Sq,D], lse: [B,H,Sq]. */
+int oracle_attn_fwd_dropout_masked(const uint16_t *q, const uint16_t *k, const uint16_t *v, int64_t B, int64_t H,
+                                   int64_t Sq, int64_t Sk, int64_t D, float scale, int causal, int dtype,
+                                   uint32_t p8, uint64_t seed, uint32_t offset, const uint8_t *mask, int64_t mask_sb,
+                                   int64_t mask_sh, int64_t mask_si, double *o, double *lse)
 {
     if (B < 0 || H < 0 || Sq < 0 || Sk < 0 || D <= 0 || p8 > 255) return -2;
     if (dtype != ORACLE_F16 && dtype != ORACLE_BF16) return -4;
@@ -657,12 +663,21 @@ int oracle_attn_fwd_dropout(const uint16_t *q, const uint16_t *k, const uint16_t
 #pragma omp for schedule(dynamic, 16)
             for (int64_t i = 0; i < Sq; ++i)
                 dropout_row(qh + i * D, kh, vh, visible_keys(i, Sq, Sk, causal), D, sc, seed, offset, p8, bh, i,
-                            srow, o + (bh * Sq + i) * D, lse + bh * Sq + i);
+                            mask ? mask + (bh / H) * mask_sb + (bh % H) * mask_sh + i * mask_si : NULL, srow,
+                            o + (bh * Sq + i) * D, lse + bh * Sq + i);
             free(srow);
         }
         free(qh); free(kh); free(vh);
     }
     return 0;
+}
+
+int oracle_attn_fwd_dropout(const uint16_t *q, const uint16_t *k, const uint16_t *v, int64_t B, int64_t H,
+                            int64_t Sq, int64_t Sk, int64_t D, float scale, int causal, int dtype, uint32_t p8,
+                            uint64_t seed, uint32_t offset, double *o, double *lse)
+{
+    return oracle_attn_fwd_dropout_masked(q, k, v, B, H, Sq, Sk, D, scale, causal, dtype, p8, seed, offset, NULL, 0,
+                                          0, 0, o, lse);
 }
 
 /* The dropout definition for a list of (bh, i) query rows only. */
@@ -698,7 +713,7 @@ int oracle_attn_rows_dropout(const uint16_t *q, const uint16_t *k, const uint16_
                 cur_bh = bh;
             }
             oracle_decode(q + (bh * Sq + i) * D, qi, D, dtype);
-            dropout_row(qi, kh, vh, visible_keys(i, Sq, Sk, causal), D, sc, seed, offset, p8, bh, i, srow,
+            dropout_row(qi, kh, vh, visible_keys(i, Sq, Sk, causal), D, sc, seed, offset, p8, bh, i, NULL, srow,
                         o + r * D, lse + r);
         }
         free(srow); free(qi); free(kh); free(vh);
@@ -904,6 +919,17 @@ int oracle_attn_bwd(const uint16_t *q, const uint16_t *k, const uint16_t *v, con
 {
     return attn_bwd_impl(q, k, v, dout, B, H, Sq, Sk, D, scale, causal, dtype, NULL, 0, 0, 0, 0, 0, 0, 0, dq, dk, dv,
                          mag_dq, mag_dk, mag_dv);
+}
+
+/* The gradients of oracle_attn_fwd_dropout_masked (mask = NULL: none). */
+int oracle_attn_bwd_dropout_masked(const uint16_t *q, const uint16_t *k, const uint16_t *v, const uint16_t *dout,
+                                   int64_t B, int64_t H, int64_t Sq, int64_t Sk, int64_t D, float scale, int causal,
+                                   int dtype, uint32_t p8, uint64_t seed, uint32_t offset, const uint8_t *mask,
+                                   int64_t mask_sb, int64_t mask_sh, int64_t mask_si, double *dq, double *dk,
+                                   double *dv, double *mag_dq, double *mag_dk, double *mag_dv)
+{
+    return attn_bwd_impl(q, k, v, dout, B, H, Sq, Sk, D, scale, causal, dtype, mask, mask_sb, mask_sh, mask_si, 1, p8,
+                         seed, offset, dq, dk, dv, mag_dq, mag_dk, mag_dv);
 }
 
 /* The gradients of the attention with dropout of oracle_attn_fwd_dropout. */

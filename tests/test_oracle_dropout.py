@@ -128,3 +128,64 @@ def test_gradients_match_float64_autograd(causal, shape):
     (o * dout.double()).sum().backward()
     for name, mine, ref in (("dQ", dq, tq.grad), ("dK", dk, tk.grad), ("dV", dv, tv.grad)):
         assert np.allclose(mine, ref.numpy(), rtol=1e-10, atol=1e-12), name
+
+
+def _padding_mask(B, Sq, Sk, seed):
+    """A key-padding mask [B, 1, Sq, Sk]: batch b sees its first L_b keys."""
+    g = np.random.default_rng(seed)
+    lens = g.integers(Sk // 3, Sk + 1, size=B)
+    m = np.zeros((B, 1, Sq, Sk), dtype=np.uint8)
+    for b in range(B):
+        m[b, :, :, :lens[b]] = 1
+    return m
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_mask_and_dropout_together(causal):
+    """With a mask and dropout: an all-ones mask equals dropout alone and p8 = 0
+    equals the mask alone (bitwise); O = (P_masked * keep * zs) V."""
+    B, H, Sq, Sk, D, p8 = 2, 2, 24, 40, 8, 60
+    q, k, v = make_cross_inputs(B, H, Sq, Sk, D, "bf16", seed=31)
+    ones = np.ones((1, 1, Sq, Sk), dtype=np.uint8)
+    a = oracle.attn_fwd_dropout(q, k, v, 0.5, causal, "bf16", p8, 3, 4)
+    b = oracle.attn_fwd_dropout(q, k, v, 0.5, causal, "bf16", p8, 3, 4, mask=ones)
+    assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
+    m = _padding_mask(B, Sq, Sk, 5)
+    c = oracle.attn_fwd_dropout(q, k, v, 0.5, causal, "bf16", 0, 3, 4, mask=m)
+    d = oracle.attn_fwd_masked(q, k, v, m, 0.5, causal, "bf16")
+    assert np.array_equal(c[0], d[0]) and np.array_equal(c[1], d[1])
+    # the combination against its definition written with numpy
+    o, lse = oracle.attn_fwd_dropout(q, k, v, 0.5, causal, "bf16", p8, 3, 4, mask=m)
+    keep = oracle.dropout_keep_mask(B * H, Sq, Sk, p8, 3, 4).reshape(B, H, Sq, Sk)
+    qd, kd, vd = (t.double().numpy() for t in (q, k, v))
+    s = 0.5 * qd @ kd.swapaxes(-1, -2)
+    vis = np.broadcast_to(m.astype(bool), s.shape).copy()
+    if causal:
+        vis &= (np.arange(Sk)[None, :] <= np.arange(Sq)[:, None] + (Sk - Sq))
+    s = np.where(vis, s, -np.inf)
+    mx = s.max(-1, keepdims=True)
+    p = np.exp(s - mx)
+    l = p.sum(-1, keepdims=True)
+    want = (p / l * keep * (256.0 / (256.0 - p8))) @ vd
+    assert np.allclose(o, want, rtol=0, atol=1e-12)
+    assert np.allclose(lse, (mx + np.log(l))[..., 0], rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_mask_and_dropout_gradients_match_autograd(causal):
+    B, H, Sq, Sk, D, p8, scale = 2, 2, 20, 33, 8, 77, 0.375
+    q, k, v = make_cross_inputs(B, H, Sq, Sk, D, "fp16", seed=41)
+    dout = torch.randn(q.shape, generator=torch.Generator().manual_seed(42)).to(torch.float16)
+    m = _padding_mask(B, Sq, Sk, 6)
+    dq, dk, dv = oracle.attn_bwd_dropout(q, k, v, dout, scale, causal, "fp16", p8, 8, 9, mask=m)
+    keep = torch.from_numpy(oracle.dropout_keep_mask(B * H, Sq, Sk, p8, 8, 9).astype(np.float64)).view(B, H, Sq, Sk)
+    tq, tk, tv = (t.double().requires_grad_(True) for t in (q, k, v))
+    s = scale * tq @ tk.transpose(-1, -2)
+    vis = torch.from_numpy(m.astype(bool)).expand(B, H, Sq, Sk)
+    if causal:
+        vis = vis & (torch.arange(Sk)[None, :] <= torch.arange(Sq)[:, None] + (Sk - Sq))
+    s = s.masked_fill(~vis, float("-inf"))
+    o = (torch.softmax(s, dim=-1) * keep * (256.0 / (256.0 - p8))) @ tv
+    (o * dout.double()).sum().backward()
+    for name, mine, ref in (("dQ", dq, tq.grad), ("dK", dk, tk.grad), ("dV", dv, tv.grad)):
+        assert np.allclose(mine, ref.numpy(), rtol=1e-10, atol=1e-12), name
