@@ -322,6 +322,75 @@ FA_API int fa_bwd_dropout(const void* q, const void* k, const void* v, const voi
                           cudaStream_t stream);
 
 /*
+ * fa_forward / fa_backward -- every option of the forward and backward
+ * passes in one call, in any combination: Sq != Sk with the bottom-right
+ * causal mask, per-tensor (b, h, s) strides, an explicit mask, dropout.
+ * The fields mean what the arguments of the same names mean for fa_fwd_ex,
+ * fa_fwd_mask and fa_fwd_dropout (fa_bwd_ex, fa_bwd_mask, fa_bwd_dropout):
+ * a NULL stride array is contiguous, a NULL mask is no mask, dropout_p = 0 is
+ * no dropout.  With a mask or dropout, D = 64 or 128.  The caller owns the
+ * struct (read during the call only) and everything it points to.  Errors:
+ * FA_ERR_NULL for a NULL params pointer, else those of the separate entries.
+ * o and lse given to fa_backward must come from fa_forward with the same
+ * mask and dropout arguments.
+ */
+typedef struct fa_fwd_params {
+    const void* q;
+    const void* k;
+    const void* v;
+    void* o;
+    float* lse;
+    int B, H, Sq, Sk, D;
+    const long long* q_stride; /* each: 3 element strides over b, h, s, or NULL */
+    const long long* k_stride;
+    const long long* v_stride;
+    const long long* o_stride;
+    const void* mask;          /* uint8 [B|1][H|1][Sq][Sk], nonzero = attend, or NULL */
+    const long long* mask_stride;
+    float dropout_p;           /* 0: no dropout */
+    unsigned long long seed;
+    unsigned int offset;
+    float scale;
+    int causal;
+    int dtype;
+} fa_fwd_params;
+
+typedef struct fa_bwd_params {
+    const void* q;
+    const void* k;
+    const void* v;
+    const void* o;
+    const void* dout;
+    const float* lse;
+    void* dq;
+    void* dk;
+    void* dv;
+    void* workspace;           /* fa_bwd_workspace_size(B, H, Sq, D) bytes, 256-byte aligned */
+    long long workspace_bytes;
+    int B, H, Sq, Sk, D;
+    const long long* q_stride; /* each: 3 element strides over b, h, s, or NULL */
+    const long long* k_stride;
+    const long long* v_stride;
+    const long long* o_stride;
+    const long long* do_stride;
+    const long long* dq_stride;
+    const long long* dk_stride;
+    const long long* dv_stride;
+    const void* mask;
+    const long long* mask_stride;
+    float dropout_p;
+    unsigned long long seed;
+    unsigned int offset;
+    float scale;
+    int causal;
+    int deterministic;
+    int dtype;
+} fa_bwd_params;
+
+FA_API int fa_forward(const fa_fwd_params* p, cudaStream_t stream);
+FA_API int fa_backward(const fa_bwd_params* p, cudaStream_t stream);
+
+/*
  * fa_merge_partial -- fold a partial attention result into a running one by
  * log-sum-exp weights.  For two disjoint key sets with results (O_a, L_a) and
  * (O_b, L_b): L = log(e^L_a + e^L_b), O = e^(L_a - L) O_a + e^(L_b - L) O_b, the

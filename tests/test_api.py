@@ -264,3 +264,47 @@ def test_accumulate_rejects_bad_arguments(lib):
     assert fa.fa_accumulate(A + 2, A, 10, 1, 0) == _lib.FA_ERR_ALIGN
     assert fa.fa_accumulate(A, A + 1, 10, 1, 0) == _lib.FA_ERR_ALIGN
     assert fa.fa_accumulate(0, 0, 0, 1, 0) == _lib.FA_OK
+
+
+def test_params_structs_match_the_header(tmp_path):
+    """The ctypes mirrors of fa_fwd_params / fa_bwd_params have the C layout:
+    a small C program built against include/fa.h prints every field's offset."""
+    import shutil
+    import subprocess
+    if not shutil.which("gcc"):
+        pytest.skip("gcc not available")
+    fields = {"fa_fwd_params": _lib.FwdParams, "fa_bwd_params": _lib.BwdParams}
+    lines = ['#include <stdio.h>', '#include <stddef.h>', '#include "fa.h"', "int main(void) {"]
+    for cname, cls in fields.items():
+        lines.append(f'printf("{cname} size %zu\\n", sizeof({cname}));')
+        for f, _ in cls._fields_:
+            lines.append(f'printf("{cname} {f} %zu\\n", offsetof({cname}, {f}));')
+    lines.append("return 0; }")
+    src = tmp_path / "layout.c"
+    src.write_text("\n".join(lines))
+    exe = tmp_path / "layout"
+    cuda_inc = "/usr/local/cuda/include"
+    subprocess.run(["gcc", "-I", os.path.join(ROOT, "include"), "-I", cuda_inc, "-o", str(exe), str(src)], check=True)
+    out = subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split("\n")
+    got = {tuple(l.split()[:2]): int(l.split()[2]) for l in out if l.strip()}
+    for cname, cls in fields.items():
+        assert got[(cname, "size")] == ctypes.sizeof(cls), cname
+        for f, _ in cls._fields_:
+            assert got[(cname, f)] == getattr(cls, f).offset, (cname, f)
+
+
+def test_unified_entries_reject_bad_arguments(lib):
+    assert _lib.load().fa_forward(None, None) == _lib.FA_ERR_NULL
+    assert _lib.load().fa_backward(None, None) == _lib.FA_ERR_NULL
+    base = dict(q=A, k=A, v=A, o=A, lse=A, B=1, H=1, Sq=128, Sk=128, D=128, scale=0.1, causal=0, dtype=1)
+    assert fa.fa_forward(0, **base, dropout_p=-0.1) == _lib.FA_ERR_ARG
+    assert fa.fa_forward(0, **base, dropout_p=1.0) == _lib.FA_ERR_ARG
+    assert fa.fa_forward(0, **base, mask=A) == _lib.FA_ERR_NULL          # a mask needs its strides
+    assert fa.fa_forward(0, **{**base, "D": 256}, dropout_p=0.1) == _lib.FA_ERR_HEADDIM
+    assert fa.fa_forward(0, **{**base, "B": 0}, dropout_p=0.1) == _lib.FA_OK
+    assert fa.fa_forward(0, **{**base, "B": 2}, q_stride=(7, 64, 64)) == _lib.FA_ERR_STRIDE
+    bb = dict(q=A, k=A, v=A, o=A, dout=A, lse=A, dq=A, dk=A, dv=A, workspace=A, workspace_bytes=1 << 30, B=1, H=1,
+              Sq=128, Sk=128, D=128, scale=0.1, causal=0, deterministic=0, dtype=1)
+    assert fa.fa_backward(0, **bb, dropout_p=float("nan")) == _lib.FA_ERR_ARG
+    assert fa.fa_backward(0, **{**bb, "D": 256}) == _lib.FA_ERR_HEADDIM
+    assert fa.fa_backward(0, **{**bb, "B": 2, "H": 2}, dq_stride=(64, 0, 64)) == _lib.FA_ERR_STRIDE

@@ -8,12 +8,12 @@ in Python or PyTorch, and there is no fallback path.
 """
 from __future__ import annotations
 
-from ._lib import (FA_BF16, FA_FP16, FaError, fa_accumulate, fa_bwd, fa_bwd_dropout, fa_bwd_ex, fa_bwd_mask, fa_bwd_workspace_size,
+from ._lib import (FA_BF16, FA_FP16, FaError, fa_accumulate, fa_backward, fa_bwd, fa_forward, fa_bwd_dropout, fa_bwd_ex, fa_bwd_mask, fa_bwd_workspace_size,
                    fa_check_status, fa_fwd, fa_fwd_dropout, fa_fwd_ex, fa_fwd_mask, fa_fwd_noalloc, fa_merge_finalize, fa_merge_partial, fa_last_timeout_site, fa_num_units, fa_selftest_timeout, fa_status_string,
                    fa_version, load)
 
 __all__ = [
-    "FA_BF16", "FA_FP16", "FaError", "fa_accumulate", "fa_bwd", "fa_bwd_dropout", "fa_bwd_ex", "fa_bwd_mask", "fa_bwd_workspace_size",
+    "FA_BF16", "FA_FP16", "FaError", "fa_accumulate", "fa_backward", "fa_bwd", "fa_forward", "fa_bwd_dropout", "fa_bwd_ex", "fa_bwd_mask", "fa_bwd_workspace_size",
     "fa_check_status", "fa_fwd", "fa_fwd_dropout", "fa_fwd_ex",
     "fa_fwd_mask", "fa_merge_finalize", "fa_merge_partial", "flash_attention_backward",
     "fa_fwd_noalloc", "fa_last_timeout_site",
@@ -30,8 +30,18 @@ def _dtype_code(t) -> int:
     raise TypeError(f"unsupported dtype {t.dtype}; expected float16 or bfloat16")
 
 
+def _mask_stride(mask, B, H, Sq, Sk):
+    """(b, h, row) element strides of a [B|1, H|1, Sq, Sk] uint8/bool CUDA mask (0 broadcasts)."""
+    if mask.dim() != 4 or tuple(mask.shape[2:]) != (Sq, Sk) or mask.shape[0] not in (1, B) or \
+            mask.shape[1] not in (1, H):
+        raise ValueError("mask must be [B|1, H|1, Sq, Sk]")
+    if mask.element_size() != 1 or not mask.is_cuda or (mask.stride(3) != 1 and Sk > 1):
+        raise ValueError("mask must be a uint8/bool CUDA tensor with contiguous keys")
+    return (mask.stride(0) if mask.shape[0] > 1 else 0, mask.stride(1) if mask.shape[1] > 1 else 0, mask.stride(2))
+
+
 def flash_attention_forward(q, k, v, scale: float, causal: bool = False, out=None, lse=None, stream=None,
-                            dropout_p: float = 0.0, seed: int = 0, offset: int = 0):
+                            dropout_p: float = 0.0, seed: int = 0, offset: int = 0, mask=None):
     """O, LSE for CUDA tensors ``q`` [B, H, Sq, D] and ``k, v`` [B, H, Sk, D] (fp16/bf16).
 
     The tensors may be any strided views whose last dimension is contiguous
@@ -43,9 +53,12 @@ def flash_attention_forward(q, k, v, scale: float, causal: bool = False, out=Non
     ``out`` takes ``q``'s memory layout.  Launches on ``stream`` (default:
     torch's current stream) and returns without synchronising.
 
-    ``dropout_p`` > 0 applies attention dropout after the softmax
-    (fa_fwd_dropout: contiguous tensors; the keep decisions are fixed by
-    ``seed`` and ``offset``, which flash_attention_backward must be given too).
+    ``dropout_p`` > 0 applies attention dropout after the softmax (the keep
+    decisions are fixed by ``seed`` and ``offset``, which
+    flash_attention_backward must be given too).  ``mask`` (a uint8/bool CUDA
+    tensor [B|1, H|1, Sq, Sk], nonzero = attend, keys contiguous, row stride a
+    multiple of 16 and >= Sk) restricts the keys each query sees.  Mask,
+    dropout, strides and Sq != Sk combine freely (fa_forward).
     """
     import torch
     if q.dim() != 4 or k.dim() != 4 or v.shape != k.shape:
@@ -73,13 +86,16 @@ def flash_attention_forward(q, k, v, scale: float, causal: bool = False, out=Non
         stream = torch.cuda.current_stream(q.device)
     st = int(stream.cuda_stream)
     dt = _dtype_code(q)
-    if dropout_p != 0.0:
-        if not all(t.is_contiguous() for t in (q, k, v, out)):
-            raise ValueError("dropout needs contiguous q, k, v and out")
-        rc = fa_fwd_dropout(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(), B, H, Sq, Sk,
-                            D, float(scale), int(bool(causal)), float(dropout_p), int(seed), int(offset), dt, st)
+    if dropout_p != 0.0 or mask is not None:
+        rc = fa_forward(st, q=q.data_ptr(), k=k.data_ptr(), v=v.data_ptr(), o=out.data_ptr(), lse=lse.data_ptr(),
+                        B=B, H=H, Sq=Sq, Sk=Sk, D=D, q_stride=q.stride()[:3], k_stride=k.stride()[:3],
+                        v_stride=v.stride()[:3], o_stride=out.stride()[:3],
+                        mask=mask.data_ptr() if mask is not None else None,
+                        mask_stride=_mask_stride(mask, B, H, Sq, Sk) if mask is not None else None,
+                        dropout_p=float(dropout_p), seed=seed, offset=offset, scale=float(scale),
+                        causal=int(bool(causal)), dtype=dt)
         if rc != 0:
-            raise FaError(rc, "fa_fwd_dropout")
+            raise FaError(rc, "fa_forward")
         return out, lse
     if Sq == Sk and all(t.is_contiguous() for t in (q, k, v, out)):
         rc = fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(), B, H, Sq, D,
@@ -95,15 +111,16 @@ def flash_attention_forward(q, k, v, scale: float, causal: bool = False, out=Non
 
 def flash_attention_backward(q, k, v, o, lse, dout, scale: float, causal: bool = False, deterministic: bool = False,
                              dq=None, dk=None, dv=None, workspace=None, stream=None, dropout_p: float = 0.0,
-                             seed: int = 0, offset: int = 0):
+                             seed: int = 0, offset: int = 0, mask=None):
     """dQ, dK, dV for CUDA tensors q, o, dout [B, H, Sq, D] and k, v [B, H, Sk, D]
     (lse [B, H, Sq] fp32 from the forward call).  The tensors may be strided
     views contiguous in their last dimension (fa_bwd_ex), like the forward's;
     the gradients take the layouts of q, k, v unless given.  The
     workspace (fa_bwd_workspace_size bytes) is allocated with torch unless
     given.  Launches on ``stream`` (default: torch's current stream) and
-    returns without synchronising.  ``dropout_p``, ``seed`` and ``offset``
-    must be those of the forward call (fa_bwd_dropout when dropout_p > 0)."""
+    returns without synchronising.  ``dropout_p``, ``seed``, ``offset`` and
+    ``mask`` must be those of the forward call (fa_backward when a mask or
+    dropout is given)."""
     import torch
     B, H, Sq, D = q.shape
     Sk = k.shape[2]
@@ -125,9 +142,20 @@ def flash_attention_backward(q, k, v, o, lse, dout, scale: float, causal: bool =
     if stream is None:
         stream = torch.cuda.current_stream(q.device)
     tensors = (q, k, v, o, dout, dq, dk, dv)
+    if dropout_p != 0.0 or mask is not None:
+        names = ("q", "k", "v", "o", "dout", "dq", "dk", "dv")
+        rc = fa_backward(int(stream.cuda_stream), **{n: t.data_ptr() for n, t in zip(names, tensors)},
+                         lse=lse.data_ptr(), workspace=workspace.data_ptr(), workspace_bytes=workspace.numel(),
+                         B=B, H=H, Sq=Sq, Sk=Sk, D=D,
+                         **{("do" if n == "dout" else n) + "_stride": t.stride()[:3] for n, t in zip(names, tensors)},
+                         mask=mask.data_ptr() if mask is not None else None,
+                         mask_stride=_mask_stride(mask, B, H, Sq, Sk) if mask is not None else None,
+                         dropout_p=float(dropout_p), seed=seed, offset=offset, scale=float(scale),
+                         causal=int(bool(causal)), deterministic=int(bool(deterministic)), dtype=_dtype_code(q))
+        if rc != 0:
+            raise FaError(rc, "fa_backward")
+        return dq, dk, dv
     if not all(t.is_contiguous() for t in tensors):
-        if dropout_p != 0.0:
-            raise ValueError("dropout needs contiguous tensors")
         rc = fa_bwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), dout.data_ptr(), lse.data_ptr(),
                        dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), workspace.data_ptr(), workspace.numel(), B, H, Sq,
                        Sk, D, *(t.stride()[:3] for t in tensors), float(scale), int(bool(causal)),

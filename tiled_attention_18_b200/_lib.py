@@ -70,6 +70,8 @@ SIGNATURES = [
      [ctypes.c_void_p] * 10 + [ctypes.c_longlong, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                ctypes.c_int, ctypes.c_float, ctypes.c_int, ctypes.c_float, ctypes.c_ulonglong,
                                ctypes.c_uint, ctypes.c_int, ctypes.c_int, ctypes.c_void_p]),
+    ("fa_forward", ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p]),
+    ("fa_backward", ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p]),
     ("fa_accumulate", ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_longlong, ctypes.c_int, ctypes.c_void_p]),
     ("fa_merge_partial", ctypes.c_int,
      [ctypes.c_void_p] * 4 + [ctypes.c_longlong, ctypes.c_int, ctypes.c_int, ctypes.c_void_p]),
@@ -205,6 +207,66 @@ def fa_bwd_dropout(q_ptr: int, k_ptr: int, v_ptr: int, o_ptr: int, do_ptr: int, 
                                      int(ws_bytes), B, H, Sq, Sk, D, float(scale), int(causal), float(dropout_p),
                                      int(seed) & (2**64 - 1), int(offset) & 0xffffffff, int(deterministic),
                                      int(dtype), stream))
+
+
+_LLP = ctypes.POINTER(ctypes.c_longlong)
+
+
+class FwdParams(ctypes.Structure):
+    """fa_fwd_params of include/fa.h (same field order and C types)."""
+    _fields_ = [("q", ctypes.c_void_p), ("k", ctypes.c_void_p), ("v", ctypes.c_void_p), ("o", ctypes.c_void_p),
+                ("lse", ctypes.c_void_p), ("B", ctypes.c_int), ("H", ctypes.c_int), ("Sq", ctypes.c_int),
+                ("Sk", ctypes.c_int), ("D", ctypes.c_int), ("q_stride", _LLP), ("k_stride", _LLP),
+                ("v_stride", _LLP), ("o_stride", _LLP), ("mask", ctypes.c_void_p), ("mask_stride", _LLP),
+                ("dropout_p", ctypes.c_float), ("seed", ctypes.c_ulonglong), ("offset", ctypes.c_uint),
+                ("scale", ctypes.c_float), ("causal", ctypes.c_int), ("dtype", ctypes.c_int)]
+
+
+class BwdParams(ctypes.Structure):
+    """fa_bwd_params of include/fa.h (same field order and C types)."""
+    _fields_ = [("q", ctypes.c_void_p), ("k", ctypes.c_void_p), ("v", ctypes.c_void_p), ("o", ctypes.c_void_p),
+                ("dout", ctypes.c_void_p), ("lse", ctypes.c_void_p), ("dq", ctypes.c_void_p),
+                ("dk", ctypes.c_void_p), ("dv", ctypes.c_void_p), ("workspace", ctypes.c_void_p),
+                ("workspace_bytes", ctypes.c_longlong), ("B", ctypes.c_int), ("H", ctypes.c_int),
+                ("Sq", ctypes.c_int), ("Sk", ctypes.c_int), ("D", ctypes.c_int), ("q_stride", _LLP),
+                ("k_stride", _LLP), ("v_stride", _LLP), ("o_stride", _LLP), ("do_stride", _LLP),
+                ("dq_stride", _LLP), ("dk_stride", _LLP), ("dv_stride", _LLP), ("mask", ctypes.c_void_p),
+                ("mask_stride", _LLP), ("dropout_p", ctypes.c_float), ("seed", ctypes.c_ulonglong),
+                ("offset", ctypes.c_uint), ("scale", ctypes.c_float), ("causal", ctypes.c_int),
+                ("deterministic", ctypes.c_int), ("dtype", ctypes.c_int)]
+
+
+def _params(cls, keep: list, **kw):
+    """A params struct; stride triples become C arrays kept alive in ``keep``."""
+    p = cls()
+    for name, val in kw.items():
+        if name.endswith("stride"):
+            if val is not None:
+                arr = (ctypes.c_longlong * 3)(*[int(x) for x in val])
+                keep.append(arr)
+                setattr(p, name, ctypes.cast(arr, _LLP))
+        elif name == "seed":
+            p.seed = int(val) & (2**64 - 1)
+        elif name == "offset":
+            p.offset = int(val) & 0xffffffff
+        else:
+            setattr(p, name, val)
+    return p
+
+
+def fa_forward(stream: int, **kw) -> int:
+    """fa_forward with the fields of fa_fwd_params as keyword arguments (pointers
+    as ints, strides as triples or None)."""
+    keep: list = []
+    p = _params(FwdParams, keep, **kw)
+    return int(load().fa_forward(ctypes.byref(p), stream))
+
+
+def fa_backward(stream: int, **kw) -> int:
+    """fa_backward with the fields of fa_bwd_params as keyword arguments."""
+    keep: list = []
+    p = _params(BwdParams, keep, **kw)
+    return int(load().fa_backward(ctypes.byref(p), stream))
 
 
 def fa_accumulate(acc_ptr: int, x_ptr: int, n: int, dtype: int, stream: int) -> int:

@@ -510,6 +510,32 @@ int fa_bwd_dropout(const void* q, const void* k, const void* v, const void* o, c
                     deterministic, dtype, stream, nullptr, nullptr, &d);
 }
 
+int fa_forward(const fa_fwd_params* p, cudaStream_t stream) {
+    if (!p) return FA_ERR_NULL;
+    if (p->B < 0 || p->H < 0 || p->Sq < 0 || p->Sk < 0) return FA_ERR_SHAPE;
+    fa::DropoutArgs d;
+    std::memset(&d, 0, sizeof(d));
+    if (p->dropout_p != 0.f && !make_dropout(p->dropout_p, p->seed, p->offset, &d)) return FA_ERR_ARG;
+    if (p->B > 0 && p->H > 0 && p->Sq > 0 && p->mask && !p->mask_stride) return FA_ERR_NULL;
+    return forward(p->q, p->k, p->v, p->o, p->lse, p->B, p->H, p->Sq, p->Sk, p->D, p->q_stride, p->k_stride,
+                   p->v_stride, p->o_stride, p->scale, p->causal, p->dtype, stream, Scratch::Allocated,
+                   static_cast<const uint8_t*>(p->mask), p->mask_stride, d.enabled ? &d : nullptr);
+}
+
+int fa_backward(const fa_bwd_params* p, cudaStream_t stream) {
+    if (!p) return FA_ERR_NULL;
+    if (p->B < 0 || p->H < 0 || p->Sq < 0 || p->Sk < 0) return FA_ERR_SHAPE;
+    fa::DropoutArgs d;
+    std::memset(&d, 0, sizeof(d));
+    if (p->dropout_p != 0.f && !make_dropout(p->dropout_p, p->seed, p->offset, &d)) return FA_ERR_ARG;
+    if (p->B > 0 && p->H > 0 && p->Sq > 0 && p->mask && !p->mask_stride) return FA_ERR_NULL;
+    const long long* const strides[8] = {p->q_stride,  p->k_stride,  p->v_stride,  p->o_stride,
+                                         p->do_stride, p->dq_stride, p->dk_stride, p->dv_stride};
+    return backward(p->q, p->k, p->v, p->o, p->dout, p->lse, p->dq, p->dk, p->dv, p->workspace, p->workspace_bytes,
+                    p->B, p->H, p->Sq, p->Sk, p->D, p->scale, p->causal, p->deterministic, p->dtype, stream,
+                    static_cast<const uint8_t*>(p->mask), p->mask_stride, d.enabled ? &d : nullptr, strides);
+}
+
 int fa_merge_partial(float* o_acc, float* lse_acc, const void* o_part, const float* lse_part, long long rows, int D,
                      int dtype, cudaStream_t stream) {
     if (rows < 0 || rows > (1LL << 33)) return FA_ERR_SHAPE;  // 8 rows per block, grid < 2^31

@@ -1361,8 +1361,9 @@ cudaError_t launch_bwd_impl(const BwdLaunchArgs& a, cudaStream_t stream) {
         // D = 128 runs the 64-row-step kernel (its Q/dO maps have 64-row boxes)
         void (*kern)(const BwdParams);
         if constexpr (D == 128)
-            kern = a.drop.enabled ? fa_bwd_kernel_d128<BF16, false, true>
-                                  : (a.mask ? fa_bwd_kernel_d128<BF16, true, false> : fa_bwd_kernel_d128<BF16, false, false>);
+            kern = a.drop.enabled
+                       ? (a.mask ? fa_bwd_kernel_d128<BF16, true, true> : fa_bwd_kernel_d128<BF16, false, true>)
+                       : (a.mask ? fa_bwd_kernel_d128<BF16, true, false> : fa_bwd_kernel_d128<BF16, false, false>);
         else kern = fa_bwd_kernel<D, BF16>;
         const int alloc = (D == 128) ? Bwd2Smem::ALLOC : BwdSmem<64>::ALLOC;
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, alloc);

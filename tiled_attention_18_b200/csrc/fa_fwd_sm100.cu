@@ -1008,6 +1008,12 @@ cudaError_t launch_impl(const LaunchArgs& a, cudaStream_t stream) {
 
 cudaError_t launch_fwd_sm100(const LaunchArgs& a, cudaStream_t stream) {
     if (a.drop.enabled) {
+        if (a.mask) {
+            if (a.D == 128)
+                return a.dtype == 1 ? launch_impl<128, true, true, true>(a, stream)
+                                    : launch_impl<128, false, true, true>(a, stream);
+            return a.dtype == 1 ? launch_impl<64, true, true, true>(a, stream) : launch_impl<64, false, true, true>(a, stream);
+        }
         if (a.D == 128)
             return a.dtype == 1 ? launch_impl<128, true, false, true>(a, stream)
                                 : launch_impl<128, false, false, true>(a, stream);
