@@ -55,7 +55,7 @@ typedef enum {
     FA_OK = 0,
     FA_ERR_NULL = -1,     /* a required pointer is NULL */
     FA_ERR_SHAPE = -2,    /* B, H or S negative, or too large for 32-bit indexing */
-    FA_ERR_HEADDIM = -3,  /* D is not 64, 128 or 256 (64 or 128 for the mask, dropout and backward entries) */
+    FA_ERR_HEADDIM = -3,  /* D is not 64, 128 or 256 (64 or 128 for the backward entries) */
     FA_ERR_DTYPE = -4,    /* dtype is not FA_FP16 or FA_BF16 */
     FA_ERR_ALIGN = -5,    /* q, k, v, o not 16-byte aligned, or lse not 4-byte aligned */
     FA_ERR_ARCH = -6,     /* the current device is not compute capability 10.0 (sm_100) */
@@ -300,8 +300,8 @@ FA_API int fa_bwd_mask(const void* q, const void* k, const void* v, const void* 
  *             weight (the result equals fa_fwd_ex's).
  * seed, offset : the generator's key and the counter's last word; use a new
  *             offset (or seed) for every call that needs fresh decisions.
- * D = 64 or 128 (else FA_ERR_HEADDIM).  Other arguments, ownership and errors
- * as fa_fwd_ex with NULL strides.
+ * D = 64, 128 or 256 (else FA_ERR_HEADDIM).  Other arguments, ownership and
+ * errors as fa_fwd_ex with NULL strides.
  */
 FA_API int fa_fwd_dropout(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Sq,
                           int Sk, int D, float scale, int causal, float dropout_p, unsigned long long seed,
@@ -328,7 +328,8 @@ FA_API int fa_bwd_dropout(const void* q, const void* k, const void* v, const voi
  * The fields mean what the arguments of the same names mean for fa_fwd_ex,
  * fa_fwd_mask and fa_fwd_dropout (fa_bwd_ex, fa_bwd_mask, fa_bwd_dropout):
  * a NULL stride array is contiguous, a NULL mask is no mask, dropout_p = 0 is
- * no dropout.  With a mask or dropout, D = 64 or 128.  The caller owns the
+ * no dropout.  fa_forward takes D = 64, 128 or 256, fa_backward 64 or 128
+ * (with or without a mask and dropout).  The caller owns the
  * struct (read during the call only) and everything it points to.  Errors:
  * FA_ERR_NULL for a NULL params pointer, else those of the separate entries.
  * o and lse given to fa_backward must come from fa_forward with the same

@@ -200,7 +200,7 @@ def test_fa_bwd_empty_problems(lib):
     (dict(ms=(8, 0, 336)), _lib.FA_ERR_STRIDE),
     (dict(mask=A + 4), _lib.FA_ERR_ALIGN),
     (dict(D=80), _lib.FA_ERR_HEADDIM),
-    (dict(D=256), _lib.FA_ERR_HEADDIM),               # the mask is fused into the D = 64/128 kernel only
+    (dict(D=512), _lib.FA_ERR_HEADDIM),               # the mask is fused into the D = 64/128/256 kernels
     (dict(Sq=400, Sk=300, causal=1), _lib.FA_ERR_SHAPE),
 ])
 def test_fa_fwd_mask_invalid_arguments(lib, args, code):
@@ -229,7 +229,7 @@ def test_dropout_entries_reject_bad_arguments(lib):
     args = lambda p, D=128, B=1: (A, A, A, A, A, B, 1, 128, 128, D, 0.1, 0, p, 1, 0, 1, 0)  # noqa: E731
     for p in (-0.1, float("nan"), float("inf"), 1.0, 255.5 / 256):
         assert fa.fa_fwd_dropout(*args(p)) == _lib.FA_ERR_ARG, p
-    assert fa.fa_fwd_dropout(*args(0.2, D=256)) == _lib.FA_ERR_HEADDIM
+    assert fa.fa_fwd_dropout(*args(0.2, D=512)) == _lib.FA_ERR_HEADDIM
     assert fa.fa_fwd_dropout(*args(0.2, B=0)) == _lib.FA_OK  # empty problem, nothing launched
     assert fa.fa_fwd_dropout(*args(0.2, B=-1)) == _lib.FA_ERR_SHAPE
     bargs = lambda p, D=128: (A,) * 10 + (1 << 20, 1, 1, 128, 128, D, 0.1, 0, p, 1, 0, 0, 1, 0)  # noqa: E731
@@ -300,7 +300,7 @@ def test_unified_entries_reject_bad_arguments(lib):
     assert fa.fa_forward(0, **base, dropout_p=-0.1) == _lib.FA_ERR_ARG
     assert fa.fa_forward(0, **base, dropout_p=1.0) == _lib.FA_ERR_ARG
     assert fa.fa_forward(0, **base, mask=A) == _lib.FA_ERR_NULL          # a mask needs its strides
-    assert fa.fa_forward(0, **{**base, "D": 256}, dropout_p=0.1) == _lib.FA_ERR_HEADDIM
+    assert fa.fa_forward(0, **{**base, "D": 512}, dropout_p=0.1) == _lib.FA_ERR_HEADDIM
     assert fa.fa_forward(0, **{**base, "B": 0}, dropout_p=0.1) == _lib.FA_OK
     assert fa.fa_forward(0, **{**base, "B": 2}, q_stride=(7, 64, 64)) == _lib.FA_ERR_STRIDE
     bb = dict(q=A, k=A, v=A, o=A, dout=A, lse=A, dq=A, dk=A, dv=A, workspace=A, workspace_bytes=1 << 30, B=1, H=1,

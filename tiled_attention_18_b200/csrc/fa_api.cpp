@@ -185,7 +185,7 @@ int forward(const void* q, const void* k, const void* v, void* o, float* lse, in
             const uint8_t* mask = nullptr, const long long* mask_stride = nullptr,
             const fa::DropoutArgs* drop = nullptr) {
     if (B < 0 || H < 0 || Sq < 0 || Sk < 0) return FA_ERR_SHAPE;
-    if (D != 64 && D != 128 && !(D == 256 && !mask && !drop)) return FA_ERR_HEADDIM;
+    if (D != 64 && D != 128 && D != 256) return FA_ERR_HEADDIM;
     if (dtype != FA_FP16 && dtype != FA_BF16) return FA_ERR_DTYPE;
     if (!(std::isfinite(scale) && scale > 0.f)) return FA_ERR_SCALE;
     if (causal != 0 && causal != 1) return FA_ERR_ARG;
@@ -309,7 +309,6 @@ int fa_fwd_dropout(const void* q, const void* k, const void* v, void* o, float* 
     fa::DropoutArgs d;
     std::memset(&d, 0, sizeof(d));
     if (!make_dropout(dropout_p, seed, offset, &d)) return FA_ERR_ARG;
-    if (D == 256) return FA_ERR_HEADDIM;
     return forward(q, k, v, o, lse, B, H, Sq, Sk, D, nullptr, nullptr, nullptr, nullptr, scale, causal, dtype, stream,
                    Scratch::Allocated, nullptr, nullptr, &d);
 }

@@ -98,7 +98,41 @@ struct Params {
     int BH, H, Sq, Sk, n_mtiles, n_units, nkv, causal, causal_off;
     float scale_log2;
     unsigned int* sched;
+    const uint8_t* mask;         // explicit boolean mask (MASK kernels): nonzero = attend
+    long long m_sb, m_sh, m_ss;  // its element strides over b, h and the query row
+    uint32_t drop_p8x4, seed_lo, seed_hi, drop_offset;  // dropout (DROP kernels)
+    float keep_scale;            // 1 / (1 - p), or 1
 };
+
+// The mask bytes of keys [kbase, kbase + 64) of one query row as 64 bits (bit c
+// of word c / 32 = key kbase + c may be attended); keys at or past Sk read as
+// 0.  Four 16-byte loads for a whole tile (row and tile start 16-byte
+// aligned), byte loads on the ragged last one.
+__device__ __forceinline__ void mask_bits64(const uint8_t* mrow, int kbase, int Sk, uint32_t (&bits)[2]) {
+    if (kbase + BN <= Sk) {
+        const uint4* src = reinterpret_cast<const uint4*>(mrow + kbase);
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+            uint32_t acc = 0;
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                const uint4 x = __ldg(src + 2 * q + hh);
+                const uint32_t ws[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    // one bit per nonzero byte, gathered into a nibble (byte i -> bit i)
+                    const uint32_t t = __vcmpne4(ws[e], 0u) & 0x01010101u;
+                    acc |= ((t * 0x01020408u) >> 24 & 0xFu) << (16 * hh + 4 * e);
+                }
+            }
+            bits[q] = acc;
+        }
+    } else {
+        bits[0] = bits[1] = 0u;
+        for (int c = 0; c < Sk - kbase; ++c)
+            if (mrow[kbase + c]) bits[c >> 5] |= 1u << (c & 31);
+    }
+}
 
 struct U256 {
     int bh, q0, n;  // head, first query row, key tiles visited
@@ -313,7 +347,7 @@ __device__ void mma(const Params& p, uint8_t* smem, uint32_t tmem, volatile uint
     mbar_drain(bar(L::B_FIN), 0u);
 }
 
-template <bool BF16>
+template <bool BF16, bool MASK, bool DROP>
 __device__ void softmax(const Params& p, uint8_t* smem, uint32_t tmem, int warp_in_group,
                         volatile uint32_t* abort_flag) {
     const uint32_t base = smem_u32(smem);
@@ -336,6 +370,15 @@ __device__ void softmax(const Params& p, uint8_t* smem, uint32_t tmem, int warp_
         const int row = U.q0 + r_in;
         const int key_limit = p.causal ? min(row + p.causal_off, p.Sk - 1) : p.Sk - 1;
         float m_use = -INFINITY, l = 0.f, lr = 0.f;
+        // explicit mask: this row's bits for the next key tile, loaded while the
+        // previous tile's MMAs run (rows past Sq read the last row)
+        const uint8_t* mrow = nullptr;
+        uint32_t mbits[2] = {0u, 0u};
+        if constexpr (MASK) {
+            const int ub = U.bh / p.H, uh = U.bh - ub * p.H;
+            mrow = p.mask + (long long)ub * p.m_sb + (long long)uh * p.m_sh + (long long)min(row, p.Sq - 1) * p.m_ss;
+            mask_bits64(mrow, 0, p.Sk, mbits);
+        }
         for (int j = 0; j < U.n; ++j) {
             const int sb = j & 1;
             if (!__all_sync(0xffffffffu, mbar_wait(bar(L::B_SFULL + sb), s_phase[sb], abort_flag, 90))) return;
@@ -358,6 +401,11 @@ __device__ void softmax(const Params& p, uint8_t* smem, uint32_t tmem, int warp_
 #pragma unroll
                 for (int c = 0; c < BN; ++c)
                     if (c > lim) s[c] = -INFINITY;
+            }
+            if constexpr (MASK) {
+#pragma unroll
+                for (int c = 0; c < BN; ++c)
+                    if (!((mbits[c >> 5] >> (c & 31)) & 1u)) s[c] = -INFINITY;
             }
             float mx = s[0];
 #pragma unroll
@@ -382,6 +430,17 @@ __device__ void softmax(const Params& p, uint8_t* smem, uint32_t tmem, int warp_
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
                 uint32_t pk[16];
+                // dropout: keep masks of the half's 32 keys (two 16-key generator blocks)
+                uint32_t km[8];
+                if constexpr (DROP) {
+                    const uint32_t g0 = (uint32_t)(kbase + 32 * h) >> 4;
+                    const uint4 a = dropout_keep_bytes(g0, (uint32_t)row, (uint32_t)U.bh, p.drop_offset, p.seed_lo,
+                                                       p.seed_hi, p.drop_p8x4);
+                    const uint4 b = dropout_keep_bytes(g0 + 1u, (uint32_t)row, (uint32_t)U.bh, p.drop_offset,
+                                                       p.seed_lo, p.seed_hi, p.drop_p8x4);
+                    km[0] = a.x; km[1] = a.y; km[2] = a.z; km[3] = a.w;
+                    km[4] = b.x; km[5] = b.y; km[6] = b.z; km[7] = b.w;
+                }
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
                     const float e0 = ex2(fmaf(s[32 * h + 2 * i], sl2, neg_m));
@@ -389,6 +448,9 @@ __device__ void softmax(const Params& p, uint8_t* smem, uint32_t tmem, int warp_
                     pk[i] = pk2<BF16>(e0, e1);
                     ls += e0 + e1;
                     if constexpr (Pol<BF16>::NORM_BY_ROUNDED_P) rs = add_bf16_pair(rs, pk[i]);
+                    // the sums keep every weight; P.V sees only the kept ones (keys 2i and
+                    // 2i + 1 are bytes 2i and 2i + 1 of the half's mask: each byte fills a half)
+                    if constexpr (DROP) pk[i] &= __byte_perm(km[i >> 1], 0u, (i & 1) ? 0x3322u : 0x1100u);
                 }
                 // P (16-bit pairs) over the first 32 columns of this S buffer
                 tmem_st16(ts + 16 * h, pk);
@@ -398,10 +460,13 @@ __device__ void softmax(const Params& p, uint8_t* smem, uint32_t tmem, int warp_
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(bar(L::B_PFULL + sb));
+            if constexpr (MASK) {
+                if (j + 1 < U.n) mask_bits64(mrow, kbase + BN, p.Sk, mbits);
+            }
         }
         const float norm = Pol<BF16>::NORM_BY_ROUNDED_P ? lr : l;
         fin_buf[fin_par * BM + r_in] = (l > 0.f)
-            ? make_float2(1.f / norm, (m_use + __log2f(l)) * 0.69314718055994530942f)
+            ? make_float2(p.keep_scale / norm, (m_use + __log2f(l)) * 0.69314718055994530942f)
             : make_float2(0.f, -INFINITY);
         mbar_arrive(bar(L::B_FINAL + fin_par));
         fin_par ^= 1;
@@ -488,7 +553,7 @@ __device__ void correction(const Params& p, uint8_t* smem, uint32_t tmem, int wa
     }
 }
 
-template <bool BF16>
+template <bool BF16, bool MASK, bool DROP>
 __global__ void __launch_bounds__(THREADS, 1) fa_fwd_kernel_d256(const __grid_constant__ Params p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -526,7 +591,7 @@ __global__ void __launch_bounds__(THREADS, 1) fa_fwd_kernel_d256(const __grid_co
     tc_fence_after();
     const uint32_t tmem = misc[0];
     if (wg == 0) {
-        softmax<BF16>(p, smem, tmem, warp & 3, abort_flag);
+        softmax<BF16, MASK, DROP>(p, smem, tmem, warp & 3, abort_flag);
     } else if (wg == 1) {
         correction<BF16>(p, smem, tmem, warp & 3, abort_flag);
     } else {
@@ -542,9 +607,9 @@ __global__ void __launch_bounds__(THREADS, 1) fa_fwd_kernel_d256(const __grid_co
     }
 }
 
-template <bool BF16>
+template <bool BF16, bool MASK, bool DROP>
 cudaError_t launch_impl(const LaunchArgs& a, cudaStream_t stream) {
-    auto kern = fa_fwd_kernel_d256<BF16>;
+    auto kern = fa_fwd_kernel_d256<BF16, MASK, DROP>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC);
     if (e != cudaSuccess) return e;
     Params p;
@@ -567,6 +632,15 @@ cudaError_t launch_impl(const LaunchArgs& a, cudaStream_t stream) {
     p.causal_off = a.Sk - a.Sq;
     p.scale_log2 = a.scale_log2;
     p.sched = a.sched;
+    p.mask = a.mask;
+    p.m_sb = a.mask_stride[0];
+    p.m_sh = a.mask_stride[1];
+    p.m_ss = a.mask_stride[2];
+    p.drop_p8x4 = a.drop.p8 * 0x01010101u;
+    p.seed_lo = a.drop.seed_lo;
+    p.seed_hi = a.drop.seed_hi;
+    p.drop_offset = a.drop.offset;
+    p.keep_scale = a.drop.enabled ? a.drop.keep_scale : 1.f;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)a.grid, 1, 1);
     cfg.blockDim = dim3(THREADS, 1, 1);
@@ -579,8 +653,15 @@ cudaError_t launch_impl(const LaunchArgs& a, cudaStream_t stream) {
 
 int64_t num_units_d256(int64_t BH, int64_t Sq) { return BH * ((Sq + BM - 1) / BM); }
 
+template <bool BF16>
+cudaError_t launch_dtype(const LaunchArgs& a, cudaStream_t stream) {
+    if (a.drop.enabled)
+        return a.mask ? launch_impl<BF16, true, true>(a, stream) : launch_impl<BF16, false, true>(a, stream);
+    return a.mask ? launch_impl<BF16, true, false>(a, stream) : launch_impl<BF16, false, false>(a, stream);
+}
+
 cudaError_t launch_fwd_d256_sm100(const LaunchArgs& a, cudaStream_t stream) {
-    return a.dtype == 1 ? launch_impl<true>(a, stream) : launch_impl<false>(a, stream);
+    return a.dtype == 1 ? launch_dtype<true>(a, stream) : launch_dtype<false>(a, stream);
 }
 
 cudaError_t read_and_clear_status_d256(cudaStream_t stream, int* status, int* site) {
