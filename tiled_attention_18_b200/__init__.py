@@ -1,23 +1,28 @@
-"""B200-native fused attention forward (FlashAttention-2 style) behind a C ABI.
+"""B200-native fused attention (FlashAttention-2 style) behind a C ABI.
 
-``fa_fwd`` and friends (see include/fa.h) are exported by ``libfa.so``, a
-hand-written sm_100a library (TMA, mbarrier pipelines, tcgen05 MMAs into
-TMEM).  This package is the thin Python binding: it marshals torch tensors
-(device memory and streams) into the C call.  No step of the computation runs
-in Python or PyTorch, and there is no fallback path.
+The entries of include/fa.h (forward and backward passes, their mask,
+dropout, strided and combined variants, and the sequence-parallel helpers)
+are exported by ``libfa.so``, a hand-written sm_100a library (TMA, mbarrier
+pipelines, tcgen05 MMAs into TMEM).  This package is the thin Python binding:
+it marshals torch tensors (device memory and streams) into the C calls.  No
+step of the computation runs in Python or PyTorch, and there is no fallback
+path: a missing library raises.  ``sequence_parallel`` orders the library's
+calls and torch.distributed's communication for a sequence split across
+ranks.
 """
 from __future__ import annotations
 
-from ._lib import (FA_BF16, FA_FP16, FaError, fa_accumulate, fa_backward, fa_bwd, fa_forward, fa_bwd_dropout, fa_bwd_ex, fa_bwd_mask, fa_bwd_workspace_size,
-                   fa_check_status, fa_fwd, fa_fwd_dropout, fa_fwd_ex, fa_fwd_mask, fa_fwd_noalloc, fa_merge_finalize, fa_merge_partial, fa_last_timeout_site, fa_num_units, fa_selftest_timeout, fa_status_string,
-                   fa_version, load)
+from ._lib import (FA_BF16, FA_FP16, FaError, fa_accumulate, fa_backward, fa_bwd, fa_bwd_dropout, fa_bwd_ex,
+                   fa_bwd_mask, fa_bwd_workspace_size, fa_check_status, fa_forward, fa_fwd, fa_fwd_dropout, fa_fwd_ex,
+                   fa_fwd_mask, fa_fwd_noalloc, fa_last_timeout_site, fa_merge_finalize, fa_merge_partial,
+                   fa_num_units, fa_selftest_timeout, fa_status_string, fa_version, load)
 
 __all__ = [
-    "FA_BF16", "FA_FP16", "FaError", "fa_accumulate", "fa_backward", "fa_bwd", "fa_forward", "fa_bwd_dropout", "fa_bwd_ex", "fa_bwd_mask", "fa_bwd_workspace_size",
-    "fa_check_status", "fa_fwd", "fa_fwd_dropout", "fa_fwd_ex",
-    "fa_fwd_mask", "fa_merge_finalize", "fa_merge_partial", "flash_attention_backward",
-    "fa_fwd_noalloc", "fa_last_timeout_site",
-    "fa_num_units", "fa_selftest_timeout", "fa_status_string", "fa_version", "flash_attention_forward", "load",
+    "FA_BF16", "FA_FP16", "FaError", "fa_accumulate", "fa_backward", "fa_bwd", "fa_bwd_dropout", "fa_bwd_ex",
+    "fa_bwd_mask", "fa_bwd_workspace_size", "fa_check_status", "fa_forward", "fa_fwd", "fa_fwd_dropout", "fa_fwd_ex",
+    "fa_fwd_mask", "fa_fwd_noalloc", "fa_last_timeout_site", "fa_merge_finalize", "fa_merge_partial",
+    "fa_num_units", "fa_selftest_timeout", "fa_status_string", "fa_version", "flash_attention_backward",
+    "flash_attention_forward", "load",
 ]
 
 
