@@ -51,6 +51,10 @@ thread_local int t_last_site = 0;
 // different streams never do.
 std::mutex g_ws_mu;
 std::map<std::pair<int, cudaStream_t>, unsigned int*> g_ws;
+// Held from a causal call's counter reset to its launch: two host threads
+// launching on one stream must not interleave reset A, reset B, kernel A,
+// kernel B (kernel B would find the counter spent and skip its units).
+std::mutex g_launch_mu;
 
 unsigned int* sched_workspace(int dev, cudaStream_t stream) {
     std::lock_guard<std::mutex> lock(g_ws_mu);
@@ -253,8 +257,10 @@ int forward(const void* q, const void* k, const void* v, void* o, float* lse, in
     a.scale_log2 = (float)((double)scale * 1.4426950408889634074);  // scale * log2(e)
     a.grid = grid;
     a.sched = nullptr;
+    std::unique_lock<std::mutex> launch_lock(g_launch_mu, std::defer_lock);
     if (causal) {
         // units differ in length under the mask: CTAs claim them from a counter
+        launch_lock.lock();
         unsigned int* ctr = nullptr;
         if (scratch == Scratch::Static) {
             if (fa::noalloc_scratch_address(&ctr) != cudaSuccess) {
