@@ -1,8 +1,10 @@
-"""Benchmark of the fused attention forward pass on B200.
+"""Benchmark of the fused attention kernels on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl fa|reference]
-                    [--workload c5|c1|c2|c3|c4|c5a|c5b|sdxl_xattn|bert_large|prefill_cached]
-                    [--no-e2e] [--no-cpu-baseline]
+                    [--workload c5|c1|c2|c3|c4|c5a|c5b|sdxl_xattn|bert_large|prefill_cached|d256_long]
+                    [--pass fwd|bwd|sp] [--mask tril] [--dropout P] [--deterministic]
+                    [--sp-world W] [--sp-mode ring|allgather|ulysses]
+                    [--no-e2e] [--no-cpu-baseline] [--cpu-seconds S]
 
 A step is one pass of the whole forward path over one batch of synthetic
 input.  The default workload is the long-context configuration
@@ -12,8 +14,9 @@ L2, so no L2 flush is needed between steps.
 
 The general-shape workloads (sdxl_xattn: 4096 queries over 77 keys;
 bert_large: B=32, H=16, S=512, D=64 in the BSHD layout; prefill_cached:
-4096 causal queries over 16384 keys) run through fa_fwd_ex; their inputs are
-rotated over enough copies that one rotation touches more than twice the L2.
+4096 causal queries over 16384 keys; d256_long: head dimension 256) run
+through fa_fwd_ex; their inputs are rotated over enough copies that one
+rotation touches more than twice the L2.
 
 Throughput is attention TFLOP/s with the causal case counted at half
 (4*B*H*S^2*D per non-causal run), over the whole job: with N GPUs (one
@@ -21,8 +24,14 @@ process per GPU, torchrun) every rank runs its own independent batch of the
 same shape (weak scaling, no data-path collective) and the value is the
 total work of all ranks over the slowest rank's device time.
 
-``--impl reference`` times the fp64 CPU oracle on bounded row samples of the
-same workload (rank 0 only) and prints the same JSON line with
+Other passes: ``--pass bwd`` times the backward pass (2.5x the forward's
+flops; BSHD workloads through fa_bwd_ex), ``--pass sp`` every rank's
+sequence-parallel schedule run in turn on one GPU.  ``--mask tril`` runs the
+causal case as an explicit lower-triangular mask, ``--dropout P`` adds
+attention dropout (a fresh offset per step).
+
+``--impl reference`` times the fp64 CPU oracle on bounded samples of the
+same workload and pass (rank 0 only) and prints the same JSON line with
 "impl": "reference".
 """
 from __future__ import annotations
