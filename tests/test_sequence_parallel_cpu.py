@@ -201,3 +201,34 @@ def test_ulysses_ranks_equal_full_attention(tmp_path, world, causal):
     for name, ref in refs.items():
         got = np.concatenate([np.load(tmp_path / f"u{name}{r}.npy") for r in range(world)], axis=2)
         assert np.max(np.abs(got - ref)) <= 1e-10, name
+
+
+def test_single_rank_schedules_reduce_to_plain_attention():
+    """World size 1 (no process group): every schedule is attention over the
+    one chunk, forward and backward."""
+    import oracle
+    from tiled_attention_18_b200.sequence_parallel import (ring_attention_backward, ulysses_attention_backward,
+                                                           ulysses_attention_forward)
+    from tiled_attention_18_b200.workloads import make_inputs
+    q, k, v = make_inputs(1, 2, 40, 8, "bf16", seed=21)
+    dout = torch.randn(q.shape, generator=torch.Generator().manual_seed(22)).to(torch.bfloat16)
+    for causal in (False, True):
+        o_ref, lse_ref = oracle.attn_fwd(q, k, v, 0.25, causal, "bf16")
+        ident = lambda x: x.clone()  # noqa: E731  (the one-rank all-to-all)
+        outs = [ring_attention_forward(q, k, v, 0.25, causal, ops=OracleOps(0.25, "bf16"), rank=0, world=1),
+                allgather_attention_forward(q, k, v, 0.25, causal, ops=OracleOps(0.25, "bf16"), rank=0, world=1,
+                                            gather=lambda kv: kv[None]),
+                ulysses_attention_forward(q, k, v, 0.25, causal, ops=OracleOps(0.25, "bf16"), alltoall=ident,
+                                          rank=0, world=1)]
+        for o, lse in outs:
+            assert np.max(np.abs(o.numpy() - o_ref)) <= 1e-12
+            assert np.max(np.abs(lse.numpy() - lse_ref)) <= 1e-12
+        refs = oracle.attn_bwd(q, k, v, dout, 0.25, causal, "bf16")
+        o64, l64 = torch.from_numpy(o_ref), torch.from_numpy(lse_ref)
+        grads = [ring_attention_backward(q, k, v, o64, l64, dout, 0.25, causal, ops=GradOps(0.25), rank=0, world=1,
+                                         exchange=lambda s, payload: (None, payload)),
+                 ulysses_attention_backward(q, k, v, o64, l64, dout, 0.25, causal, ops=GradOps(0.25), alltoall=ident,
+                                            rank=0, world=1)]
+        for g in grads:
+            for a, b in zip(g, refs):
+                assert np.max(np.abs(a.numpy() - b)) <= 1e-10
