@@ -182,3 +182,8 @@ def flash_attention_backward(q, k, v, o, lse, dout, scale: float, causal: bool =
     if rc != 0:
         raise FaError(rc, "fa_bwd")
     return dq, dk, dv
+
+
+from .autograd import attention  # noqa: E402  (the differentiable operation over the two calls above)
+
+__all__.append("attention")
