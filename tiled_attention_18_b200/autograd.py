@@ -12,6 +12,8 @@ from __future__ import annotations
 
 from typing import Optional
 
+import torch
+
 from . import flash_attention_backward, flash_attention_forward
 
 # the two calls, looked up at run time (tests substitute stand-ins)
@@ -19,33 +21,25 @@ _forward = flash_attention_forward
 _backward = flash_attention_backward
 
 
-def _attention_function():
-    import torch
+class _Attention(torch.autograd.Function):
+    @staticmethod
+    def forward(ctx, q, k, v, scale, causal, dropout_p, seed, offset, mask, deterministic):
+        o, lse = _forward(q, k, v, scale, causal, dropout_p=dropout_p, seed=seed, offset=offset, mask=mask)
+        ctx.save_for_backward(q, k, v, o, lse)
+        ctx.mask = mask
+        ctx.args = (scale, causal, dropout_p, seed, offset, deterministic)
+        ctx.mark_non_differentiable(lse)
+        return o, lse
 
-    class _Attention(torch.autograd.Function):
-        @staticmethod
-        def forward(ctx, q, k, v, scale, causal, dropout_p, seed, offset, mask, deterministic):
-            o, lse = _forward(q, k, v, scale, causal, dropout_p=dropout_p, seed=seed, offset=offset, mask=mask)
-            ctx.save_for_backward(q, k, v, o, lse)
-            ctx.mask = mask
-            ctx.args = (scale, causal, dropout_p, seed, offset, deterministic)
-            ctx.mark_non_differentiable(lse)
-            return o, lse
-
-        @staticmethod
-        def backward(ctx, do, _dlse):
-            q, k, v, o, lse = ctx.saved_tensors
-            scale, causal, dropout_p, seed, offset, deterministic = ctx.args
-            # the kernels read dO row by row: give them a dense one
-            do = do.contiguous()
-            dq, dk, dv = _backward(q, k, v, o, lse, do, scale, causal, deterministic=deterministic,
-                                   dropout_p=dropout_p, seed=seed, offset=offset, mask=ctx.mask)
-            return dq, dk, dv, None, None, None, None, None, None, None
-
-    return _Attention
-
-
-_FN = None
+    @staticmethod
+    def backward(ctx, do, _dlse):
+        q, k, v, o, lse = ctx.saved_tensors
+        scale, causal, dropout_p, seed, offset, deterministic = ctx.args
+        # the kernels read dO row by row: give them a dense one
+        do = do.contiguous()
+        dq, dk, dv = _backward(q, k, v, o, lse, do, scale, causal, deterministic=deterministic,
+                               dropout_p=dropout_p, seed=seed, offset=offset, mask=ctx.mask)
+        return dq, dk, dv, None, None, None, None, None, None, None
 
 
 def attention(q, k, v, scale: Optional[float] = None, causal: bool = False, dropout_p: float = 0.0, seed: int = 0,
@@ -58,11 +52,8 @@ def attention(q, k, v, scale: Optional[float] = None, causal: bool = False, drop
     (not differentiable).  Use a new ``offset`` (or ``seed``) for every
     training step that needs fresh dropout decisions.
     """
-    global _FN
-    if _FN is None:
-        _FN = _attention_function()
     if scale is None:
         scale = q.shape[-1] ** -0.5
-    o, lse = _FN.apply(q, k, v, float(scale), bool(causal), float(dropout_p), int(seed), int(offset), mask,
-                       bool(deterministic))
+    o, lse = _Attention.apply(q, k, v, float(scale), bool(causal), float(dropout_p), int(seed), int(offset), mask,
+                              bool(deterministic))
     return (o, lse) if return_lse else o
