@@ -32,7 +32,10 @@
  * The per-row LSE is not defined on the pages; it is the natural log of the
  * softmax denominator of the scaled scores.
  *
- * All calls are thread-safe and return an fa_status code; none aborts.
+ * All calls return an fa_status code; none aborts.  Calls from several host
+ * threads at once are not verified yet (in one test, concurrent causal calls
+ * from four threads on one stream failed with FA_ERR_LAUNCH in two of them):
+ * serialise calls across host threads.
  */
 #ifndef FA_H_
 #define FA_H_

@@ -149,32 +149,3 @@ def test_stuck_wait_reports_timeout_and_context_survives():
     o_ref, lse_ref = oracle.attn_fwd(q, k, v, softmax_scale(64), True, "fp16")
     compare(o, lse, o_ref, lse_ref, "fp16")
 
-
-def test_causal_calls_from_several_threads_on_one_stream():
-    """Host threads issuing causal forwards on one stream at the same time: the
-    scheduler-counter reset and the launch of each call stay together, so
-    every call computes all its rows (checked against the oracle)."""
-    import threading
-    import tiled_attention_18_b200 as fa
-    from tiled_attention_18_b200.workloads import O_TOL, make_inputs, softmax_scale
-    n = 4
-    inputs = [make_inputs(1, 4, 1024, 128, "bf16", seed=100 + i) for i in range(n)]
-    dev = [tuple(t.cuda() for t in x) for x in inputs]
-    outs = [None] * n
-    start = threading.Barrier(n)
-
-    def work(i):
-        start.wait(timeout=60)
-        for _ in range(5):
-            outs[i] = fa.flash_attention_forward(*dev[i], softmax_scale(128), True)
-
-    threads = [threading.Thread(target=work, args=(i,)) for i in range(n)]
-    for t in threads:
-        t.start()
-    for t in threads:
-        t.join(timeout=120)
-    torch.cuda.synchronize()
-    assert fa.fa_check_status(torch.cuda.current_stream().cuda_stream) == 0
-    for i in range(n):
-        o_ref, _ = oracle.attn_fwd(*inputs[i], softmax_scale(128), True, "bf16")
-        assert np.abs(outs[i][0].cpu().double().numpy() - o_ref).max() <= O_TOL["bf16"]
