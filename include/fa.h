@@ -32,10 +32,13 @@
  * The per-row LSE is not defined on the pages; it is the natural log of the
  * softmax denominator of the scaled scores.
  *
- * All calls return an fa_status code; none aborts.  Calls from several host
- * threads at once are not verified yet (in one test, concurrent causal calls
- * from four threads on one stream failed with FA_ERR_LAUNCH in two of them):
- * serialise calls across host threads.
+ * All calls return an fa_status code; none aborts.  FA_ERR_LAUNCH reports
+ * the failure of this call's own CUDA calls and launches, never an error that
+ * other code left pending in the calling thread.  Calls from several host
+ * threads at once are designed to be safe (a causal call resets its work
+ * counter and launches under one lock; each kernel's shared-memory limit is
+ * set once) but are not verified on hardware yet: until they are, serialise
+ * calls across host threads.
  */
 #ifndef FA_H_
 #define FA_H_

@@ -1350,11 +1350,11 @@ cudaError_t launch_bwd_impl(const BwdLaunchArgs& a, cudaStream_t stream) {
     const int Sq_pad = n_mtiles * TILE;
     {
         dim3 grid((unsigned)(Sq_pad / 8), (unsigned)BH, 1);
-        bwd_prep_kernel<D, BF16><<<grid, 256, 0, stream>>>(
-            static_cast<const uint16_t*>(a.o), static_cast<const uint16_t*>(a.dout), a.lse, a.lse2, a.delta,
-            a.dq_acc, a.Sq, Sq_pad, a.sched, a.H, Strides3{{a.o_stride[0], a.o_stride[1], a.o_stride[2]}},
+        cudaError_t e = launch_kernel(
+            bwd_prep_kernel<D, BF16>, grid, dim3(256), 0, stream, static_cast<const uint16_t*>(a.o),
+            static_cast<const uint16_t*>(a.dout), a.lse, a.lse2, a.delta, a.dq_acc, a.Sq, Sq_pad, a.sched, a.H,
+            Strides3{{a.o_stride[0], a.o_stride[1], a.o_stride[2]}},
             Strides3{{a.do_stride[0], a.do_stride[1], a.do_stride[2]}});
-        cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
     {
@@ -1366,7 +1366,7 @@ cudaError_t launch_bwd_impl(const BwdLaunchArgs& a, cudaStream_t stream) {
                        : (a.mask ? fa_bwd_kernel_d128<BF16, true, false> : fa_bwd_kernel_d128<BF16, false, false>);
         else kern = fa_bwd_kernel<D, BF16>;
         const int alloc = (D == 128) ? Bwd2Smem::ALLOC : BwdSmem<64>::ALLOC;
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, alloc);
+        cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(kern), alloc);
         if (e != cudaSuccess) return e;
         BwdParams p;
         p.tmap_q = a.tmap_q;
@@ -1426,10 +1426,9 @@ cudaError_t launch_bwd_impl(const BwdLaunchArgs& a, cudaStream_t stream) {
     {
         const size_t n4 = (size_t)BH * (size_t)a.Sq * D / 4;
         const unsigned blocks = (unsigned)((n4 + 255) / 256 < 148u * 16u ? (n4 + 255) / 256 : 148u * 16u);
-        bwd_post_kernel<D, BF16><<<blocks, 256, 0, stream>>>(
-            reinterpret_cast<const float4*>(a.dq_acc), static_cast<uint16_t*>(a.dq), n4, a.scale, a.H, a.Sq,
-            Strides3{{a.dq_stride[0], a.dq_stride[1], a.dq_stride[2]}});
-        return cudaGetLastError();
+        return launch_kernel(bwd_post_kernel<D, BF16>, dim3(blocks), dim3(256), 0, stream,
+                             reinterpret_cast<const float4*>(a.dq_acc), static_cast<uint16_t*>(a.dq), n4, a.scale,
+                             a.H, a.Sq, Strides3{{a.dq_stride[0], a.dq_stride[1], a.dq_stride[2]}});
     }
 }
 

@@ -610,7 +610,7 @@ __global__ void __launch_bounds__(THREADS, 1) fa_fwd_kernel_d256(const __grid_co
 template <bool BF16, bool MASK, bool DROP>
 cudaError_t launch_impl(const LaunchArgs& a, cudaStream_t stream) {
     auto kern = fa_fwd_kernel_d256<BF16, MASK, DROP>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC);
+    cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(kern), L::ALLOC);
     if (e != cudaSuccess) return e;
     Params p;
     p.tmap_q = a.tmap_q;

@@ -963,7 +963,7 @@ cudaError_t launch_impl(const LaunchArgs& a, cudaStream_t stream) {
     using L = Smem<D>;
     static_assert(L::ALLOC <= 232448, "shared memory budget exceeded");
     auto kern = fa_fwd_kernel<D, BF16, MASK, DROP>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC);
+    cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(kern), L::ALLOC);
     if (e != cudaSuccess) return e;
     KParams p;
     p.tmap_q = a.tmap_q;
@@ -1029,8 +1029,7 @@ cudaError_t launch_fwd_sm100(const LaunchArgs& a, cudaStream_t stream) {
 
 cudaError_t launch_selftest_timeout(cudaStream_t stream) {
     // about 50 ms at the maximum SM clock
-    selftest_timeout_kernel<<<1, 64, 0, stream>>>(100000000ll);
-    return cudaGetLastError();
+    return launch_kernel(selftest_timeout_kernel, dim3(1), dim3(64), 0, stream, 100000000ll);
 }
 
 cudaError_t noalloc_scratch_address(unsigned int** out) {

@@ -6,6 +6,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 namespace fa {
 
 // Tile shape of the forward kernel: a CTA owns two query tiles of BLOCK_M
@@ -111,6 +113,28 @@ inline BwdWorkspace bwd_workspace_layout(int64_t BH, int64_t Sq, int64_t D) {
 
 // LSE-weighted merge of a partial attention result into a running fp32 one,
 // and the conversion of the running O to 16 bits (fa_merge_sm100.cu).
+// Raises `kernel`'s dynamic shared-memory limit to `bytes` on the current
+// device, once per (kernel, device) for the life of the process: later
+// launches make no attribute call, so host threads launching at the same time
+// never set an attribute of a kernel that another thread is launching.
+cudaError_t ensure_smem_limit(const void* kernel, int bytes);
+
+// Launches `kernel` on `stream` and returns the status of this launch alone
+// (cudaGetLastError after a <<<>>> launch would also return an error that
+// other code left pending in the calling thread).
+template <typename... Expected, typename... Actual>
+cudaError_t launch_kernel(void (*kernel)(Expected...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                          Actual&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cfg.attrs = nullptr;
+    cfg.numAttrs = 0;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Actual>(args)...);
+}
+
 cudaError_t launch_merge_partial(float* o_acc, float* lse_acc, const void* o_part, const float* lse_part,
                                  long long rows, int D, int dtype, cudaStream_t stream);
 cudaError_t launch_accumulate(float* acc, const void* x, long long n, int dtype, cudaStream_t stream);

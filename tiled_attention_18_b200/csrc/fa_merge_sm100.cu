@@ -116,11 +116,9 @@ __global__ void __launch_bounds__(256) accumulate_kernel(float* __restrict__ acc
 cudaError_t launch_accumulate(float* acc, const void* x, long long n, int dtype, cudaStream_t stream) {
     const long long want = (n / 4 + 255) / 256 + 1;
     const unsigned blocks = (unsigned)(want < 148 * 32 ? want : 148 * 32);
-    if (dtype == 1)
-        accumulate_kernel<true><<<blocks, 256, 0, stream>>>(acc, static_cast<const uint16_t*>(x), n);
-    else
-        accumulate_kernel<false><<<blocks, 256, 0, stream>>>(acc, static_cast<const uint16_t*>(x), n);
-    return cudaGetLastError();
+    const uint16_t* xs = static_cast<const uint16_t*>(x);
+    return dtype == 1 ? launch_kernel(accumulate_kernel<true>, dim3(blocks), dim3(256), 0, stream, acc, xs, n)
+                      : launch_kernel(accumulate_kernel<false>, dim3(blocks), dim3(256), 0, stream, acc, xs, n);
 }
 
 cudaError_t launch_merge_partial(float* o_acc, float* lse_acc, const void* o_part, const float* lse_part,
@@ -128,24 +126,17 @@ cudaError_t launch_merge_partial(float* o_acc, float* lse_acc, const void* o_par
     const unsigned blocks = (unsigned)((rows + 7) / 8);
     const uint16_t* ob = static_cast<const uint16_t*>(o_part);
     const bool vec = (D % 4 == 0) && ((uintptr_t)o_acc % 16 == 0) && ((uintptr_t)o_part % 8 == 0);
-    if (dtype == 1) {
-        if (vec) merge_kernel<true, true><<<blocks, 256, 0, stream>>>(o_acc, lse_acc, ob, lse_part, rows, D);
-        else merge_kernel<true, false><<<blocks, 256, 0, stream>>>(o_acc, lse_acc, ob, lse_part, rows, D);
-    } else {
-        if (vec) merge_kernel<false, true><<<blocks, 256, 0, stream>>>(o_acc, lse_acc, ob, lse_part, rows, D);
-        else merge_kernel<false, false><<<blocks, 256, 0, stream>>>(o_acc, lse_acc, ob, lse_part, rows, D);
-    }
-    return cudaGetLastError();
+    auto kern = dtype == 1 ? (vec ? merge_kernel<true, true> : merge_kernel<true, false>)
+                           : (vec ? merge_kernel<false, true> : merge_kernel<false, false>);
+    return launch_kernel(kern, dim3(blocks), dim3(256), 0, stream, o_acc, lse_acc, ob, lse_part, rows, D);
 }
 
 cudaError_t launch_merge_finalize(const float* o_acc, void* o, long long n, int dtype, cudaStream_t stream) {
     const long long want = (n + 255) / 256;
     const unsigned blocks = (unsigned)(want < 148 * 32 ? want : 148 * 32);
-    if (dtype == 1)
-        finalize_kernel<true><<<blocks, 256, 0, stream>>>(o_acc, static_cast<uint16_t*>(o), n);
-    else
-        finalize_kernel<false><<<blocks, 256, 0, stream>>>(o_acc, static_cast<uint16_t*>(o), n);
-    return cudaGetLastError();
+    uint16_t* out = static_cast<uint16_t*>(o);
+    return dtype == 1 ? launch_kernel(finalize_kernel<true>, dim3(blocks), dim3(256), 0, stream, o_acc, out, n)
+                      : launch_kernel(finalize_kernel<false>, dim3(blocks), dim3(256), 0, stream, o_acc, out, n);
 }
 
 }  // namespace fa
