@@ -308,3 +308,21 @@ def test_unified_entries_reject_bad_arguments(lib):
     assert fa.fa_backward(0, **bb, dropout_p=float("nan")) == _lib.FA_ERR_ARG
     assert fa.fa_backward(0, **{**bb, "D": 256}) == _lib.FA_ERR_HEADDIM
     assert fa.fa_backward(0, **{**bb, "B": 2, "H": 2}, dq_stride=(64, 0, 64)) == _lib.FA_ERR_STRIDE
+
+
+def test_every_launch_reports_its_own_status():
+    """Kernels launch through cudaLaunchKernelEx and the calls return that
+    launch's status: no <<<>>> launch followed by a thread-global error query,
+    which would also report an error that other code left pending."""
+    import glob
+    import os
+    csrc = os.path.join(os.path.dirname(fa.__file__), "csrc")
+    sources = glob.glob(os.path.join(csrc, "*.cu")) + glob.glob(os.path.join(csrc, "*.cpp"))
+    assert sources
+    for path in sources:
+        text = open(path).read()
+        assert "<<<" not in text, path
+        assert "cudaPeekAtLastError" not in text, path
+        # the shared-memory limit is raised once per kernel and device, not per launch
+        if not path.endswith("fa_api.cpp"):
+            assert "cudaFuncSetAttribute" not in text, path
