@@ -680,7 +680,10 @@ int oracle_attn_fwd_dropout(const uint16_t *q, const uint16_t *k, const uint16_t
                                           0, 0, o, lse);
 }
 
-/* The dropout definition for a list of (bh, i) query rows only. */
+/* The dropout definition for a list of (bh, i) query rows only.  Pinned bit for
+ * bit against the rows of oracle_attn_fwd_dropout (square and Sq != Sk, causal
+ * and not, several thresholds, seeds and offsets): the generator's counter takes
+ * the query row i, never the position r in the list. */
 int oracle_attn_rows_dropout(const uint16_t *q, const uint16_t *k, const uint16_t *v, int64_t B, int64_t H,
                              int64_t Sq, int64_t Sk, int64_t D, float scale, int causal, int dtype, uint32_t p8,
                              uint64_t seed, uint32_t offset, const int64_t *bh_idx, const int64_t *row_idx,

@@ -189,3 +189,27 @@ def test_mask_and_dropout_gradients_match_autograd(causal):
     (o * dout.double()).sum().backward()
     for name, mine, ref in (("dQ", dq, tq.grad), ("dK", dk, tk.grad), ("dV", dv, tv.grad)):
         assert np.allclose(mine, ref.numpy(), rtol=1e-10, atol=1e-12), name
+
+
+@pytest.mark.parametrize("Sq,Sk", [(70, 70), (40, 90), (90, 40)], ids=["square", "sq_lt_sk", "sq_gt_sk"])
+@pytest.mark.parametrize("causal", [False, True], ids=["full", "causal"])
+def test_sampled_rows_equal_full_run(Sq, Sk, causal):
+    """The row-sampled dropout oracle (used by the GPU parity tests and the
+    timed CPU baseline on large shapes) gives, bit for bit, the rows of the full
+    dropout oracle: same keep decisions (the generator's counter takes the
+    query row, not the sample index), same softmax and same scale.  The
+    sample puts rows at positions other than their index, so a row/sample
+    mix-up changes the keep decisions and fails."""
+    from tiled_attention_18_b200.workloads import sample_rows
+    if causal and Sq > Sk:
+        pytest.skip("a causal query needs a key (Sq <= Sk)")
+    B, H, D = 2, 3, 16
+    q, k, v = make_cross_inputs(B, H, Sq, Sk, D, "bf16", seed=23)
+    scale = 0.3
+    for p8, seed, offset in ((26, 7, 0), (128, 0x123456789AB, 5), (255, 3, 2**32 - 1)):
+        o, lse = oracle.attn_fwd_dropout(q, k, v, scale, causal, "bf16", p8, seed, offset)
+        bh, rows = sample_rows(B, H, Sq, n_random=40, edge=3, seed=p8)
+        assert not np.array_equal(rows, np.arange(rows.size) % Sq)
+        orow, lrow = oracle.attn_rows_dropout(q, k, v, scale, causal, "bf16", p8, seed, offset, bh, rows)
+        assert np.array_equal(orow, o.reshape(B * H, Sq, D)[bh, rows])
+        assert np.array_equal(lrow, lse.reshape(B * H, Sq)[bh, rows])
