@@ -34,11 +34,10 @@
  *
  * All calls return an fa_status code; none aborts.  FA_ERR_LAUNCH reports
  * the failure of this call's own CUDA calls and launches, never an error that
- * other code left pending in the calling thread.  Calls from several host
- * threads at once are designed to be safe (a causal call resets its work
- * counter and launches under one lock; each kernel's shared-memory limit is
- * set once) but are not verified on hardware yet: until they are, serialise
- * calls across host threads.
+ * other code left pending in the calling thread; fa_last_cuda_error names the
+ * failed call and its error code.  Calls from several host threads at once
+ * are safe: a causal call resets its work counter and launches under one lock,
+ * and each kernel's shared-memory limit is set once per context.
  */
 #ifndef FA_H_
 #define FA_H_
@@ -73,7 +72,9 @@ typedef enum {
     FA_ERR_STRIDE = -12,  /* fa_fwd_ex, fa_bwd_ex: a stride is negative, zero over an extent > 1,
                              not a multiple of 8 elements (16 bytes), or not below 2^36 elements;
                              the mask entries: a mask stride breaks their rules */
-    FA_ERR_WORKSPACE = -13 /* the fa_bwd entries: workspace NULL, not 256-byte aligned or too small */
+    FA_ERR_WORKSPACE = -13, /* the fa_bwd entries: workspace NULL, not 256-byte aligned or too small */
+    FA_ERR_LIMIT = -14      /* causal forward: more streams of one context have launched causal
+                               forwards than the library's 2048 scheduler-counter slots */
 } fa_status;
 
 /*
@@ -100,12 +101,15 @@ typedef enum {
  *           nearest even.
  * stream  : the CUDA stream to launch on (0 = legacy default stream).
  *
- * Ownership: the caller owns every buffer and the stream.  With causal = 1
- * the library's work scheduler uses a 4-byte counter in device scratch: one
- * per (device, stream), allocated with cudaMalloc by the first causal call on
- * that stream (so that call must not be inside a stream capture) and kept
- * until the process exits; each causal call zeroes it with cudaMemsetAsync on
- * `stream`.  Synchronicity: asynchronous on `stream`; fa_fwd never
+ * Ownership: the caller owns every buffer and the stream; fa_fwd allocates
+ * nothing.  With causal = 1 the library's work scheduler uses a 4-byte
+ * counter: one slot per (context, stream) of a fixed pool of 2048 slots in
+ * libfa.so's own static device memory (64 KiB, part of the loaded module),
+ * handed out by the stream's first causal call; each causal call zeroes its
+ * counter with cudaMemsetAsync on `stream`.  More than 2048 distinct streams
+ * of one context launching causal forwards gives FA_ERR_LIMIT.  The first
+ * call in a context looks up the pool's device address (a host-side query,
+ * no device work).  Synchronicity: asynchronous on `stream`; fa_fwd never
  * synchronises.  Errors: argument checks run before any launch and return a
  * negative fa_status with nothing launched; a launch failure returns
  * FA_ERR_LAUNCH.  A device-side wait that exceeds its bound (about two
@@ -447,6 +451,16 @@ FA_API int fa_check_status(cudaStream_t stream);
  * (wait site) | (CTA index << 8).  0 if none.
  */
 FA_API int fa_last_timeout_site(void);
+
+/*
+ * fa_last_cuda_error -- the CUDA failure behind the calling thread's most
+ * recent FA_ERR_LAUNCH from any entry of this library: returns the cudaError_t
+ * (or, for the tensor-map encoder, the CUresult) code, 0 if no call of this
+ * thread has failed, and sets *site (if site is not NULL) to a static string
+ * naming the call that failed.  Per host thread; a later success does not
+ * clear it.  Diagnostic; the pages have no counterpart.
+ */
+FA_API int fa_last_cuda_error(const char** site);
 
 /*
  * fa_selftest_timeout -- diagnostic for the failure path (no counterpart on

@@ -14,14 +14,14 @@ from __future__ import annotations
 
 from ._lib import (FA_BF16, FA_FP16, FaError, fa_accumulate, fa_backward, fa_bwd, fa_bwd_dropout, fa_bwd_ex,
                    fa_bwd_mask, fa_bwd_workspace_size, fa_check_status, fa_forward, fa_fwd, fa_fwd_dropout, fa_fwd_ex,
-                   fa_fwd_mask, fa_fwd_noalloc, fa_last_timeout_site, fa_merge_finalize, fa_merge_partial,
-                   fa_num_units, fa_selftest_timeout, fa_status_string, fa_version, load)
+                   fa_fwd_mask, fa_fwd_noalloc, fa_last_cuda_error, fa_last_timeout_site, fa_merge_finalize,
+                   fa_merge_partial, fa_num_units, fa_selftest_timeout, fa_status_string, fa_version, load)
 
 __all__ = [
     "FA_BF16", "FA_FP16", "FaError", "fa_accumulate", "fa_backward", "fa_bwd", "fa_bwd_dropout", "fa_bwd_ex",
     "fa_bwd_mask", "fa_bwd_workspace_size", "fa_check_status", "fa_forward", "fa_fwd", "fa_fwd_dropout", "fa_fwd_ex",
-    "fa_fwd_mask", "fa_fwd_noalloc", "fa_last_timeout_site", "fa_merge_finalize", "fa_merge_partial",
-    "fa_num_units", "fa_selftest_timeout", "fa_status_string", "fa_version", "flash_attention_backward",
+    "fa_fwd_mask", "fa_fwd_noalloc", "fa_last_cuda_error", "fa_last_timeout_site", "fa_merge_finalize",
+    "fa_merge_partial", "fa_num_units", "fa_selftest_timeout", "fa_status_string", "fa_version", "flash_attention_backward",
     "flash_attention_forward", "load",
 ]
 

@@ -30,6 +30,7 @@ FA_ERR_ARG = -10
 FA_ERR_PTR = -11
 FA_ERR_STRIDE = -12
 FA_ERR_WORKSPACE = -13
+FA_ERR_LIMIT = -14
 
 _LL3 = ctypes.POINTER(ctypes.c_longlong)
 
@@ -79,6 +80,7 @@ SIGNATURES = [
      [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_longlong, ctypes.c_int, ctypes.c_void_p]),
     ("fa_check_status", ctypes.c_int, [ctypes.c_void_p]),
     ("fa_last_timeout_site", ctypes.c_int, []),
+    ("fa_last_cuda_error", ctypes.c_int, [ctypes.POINTER(ctypes.c_char_p)]),
     ("fa_selftest_timeout", ctypes.c_int, [ctypes.c_void_p]),
     ("fa_status_string", ctypes.c_char_p, [ctypes.c_int]),
     ("fa_version", ctypes.c_int, []),
@@ -92,7 +94,15 @@ _lib = None
 class FaError(RuntimeError):
     def __init__(self, status: int, what: str = "fa_fwd"):
         self.status = status
-        super().__init__(f"{what} failed: {status} ({status_string(status)})")
+        msg = f"{what} failed: {status} ({status_string(status)})"
+        if status == FA_ERR_LAUNCH:
+            # the failing CUDA call of this thread, as the library recorded it
+            try:
+                code, site = fa_last_cuda_error()
+                msg += f"; CUDA error {code} in {site}"
+            except OSError:
+                pass
+        super().__init__(msg)
 
 
 def load() -> ctypes.CDLL:
@@ -290,6 +300,13 @@ def fa_check_status(stream: int = 0) -> int:
 
 def fa_last_timeout_site() -> int:
     return int(load().fa_last_timeout_site())
+
+
+def fa_last_cuda_error():
+    """(code, call name) of the CUDA failure behind this thread's latest FA_ERR_LAUNCH; (0, "") if none."""
+    site = ctypes.c_char_p()
+    code = int(load().fa_last_cuda_error(ctypes.byref(site)))
+    return code, (site.value or b"").decode()
 
 
 def fa_selftest_timeout(stream: int = 0) -> int:

@@ -45,29 +45,78 @@ std::once_flag g_encode_once;
 
 thread_local int t_last_site = 0;
 
-// Scratch of the causal work scheduler: one unit counter per (device, stream),
-// allocated on first use and kept for the life of the process.  Launches on
-// one stream are ordered, so they can share the counter; launches on
-// different streams never do.
+// The CUDA failure behind this thread's most recent FA_ERR_LAUNCH: the
+// cudaError_t (or CUresult) code and the name of the call that returned it.
+thread_local int t_err_code = 0;
+thread_local const char* t_err_site = "";
+
+// Records a failed CUDA call, clears the calling thread's pending error that the
+// failure may have left, and returns FA_ERR_LAUNCH.
+int cuda_fail(int code, const char* site) {
+    t_err_code = code;
+    t_err_site = site;
+    cudaGetLastError();
+    return FA_ERR_LAUNCH;
+}
+
+// Causal work-unit counters: (context id, stream) -> its slot in the library's
+// static counter pool.  Launches on one stream are ordered, so they can share
+// a counter; launches on different streams never do.  Context ids are unique
+// for the life of the process, so a context re-created after cudaDeviceReset
+// starts with fresh slots (the pool's address is looked up again there).
 std::mutex g_ws_mu;
-std::map<std::pair<int, cudaStream_t>, unsigned int*> g_ws;
+std::map<std::pair<unsigned long long, cudaStream_t>, unsigned int*> g_ws;
+std::map<unsigned long long, int> g_ws_used;  // slots handed out per context
 // Held from a causal call's counter reset to its launch: two host threads
 // launching on one stream must not interleave reset A, reset B, kernel A,
 // kernel B (kernel B would find the counter spent and skip its units).
 std::mutex g_launch_mu;
 
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+CtxGetCurrentFn g_ctx_current = nullptr;
+CtxGetIdFn g_ctx_id = nullptr;
+std::once_flag g_ctx_once;
+
 }  // namespace
 
 namespace fa {
 
+cudaError_t current_context_id(unsigned long long* id) {
+    std::call_once(g_ctx_once, [] {
+        void* fn = nullptr;
+        cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            g_ctx_current = reinterpret_cast<CtxGetCurrentFn>(fn);
+        fn = nullptr;
+        q = cudaDriverEntryPointSymbolNotFound;
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            g_ctx_id = reinterpret_cast<CtxGetIdFn>(fn);
+    });
+    if (!g_ctx_current || !g_ctx_id) return cudaErrorNotSupported;
+    CUcontext ctx = nullptr;
+    if (g_ctx_current(&ctx) != CUDA_SUCCESS) return cudaErrorDeviceUninitialized;
+    if (!ctx) {
+        // no context bound to this thread yet: bind the current device's primary one
+        int dev = 0;
+        cudaError_t e = cudaGetDevice(&dev);
+        if (e == cudaSuccess) e = cudaSetDevice(dev);
+        if (e != cudaSuccess) return e;
+        if (g_ctx_current(&ctx) != CUDA_SUCCESS || !ctx) return cudaErrorDeviceUninitialized;
+    }
+    return g_ctx_id(ctx, id) == CUDA_SUCCESS ? cudaSuccess : cudaErrorDeviceUninitialized;
+}
+
 cudaError_t ensure_smem_limit(const void* kernel, int bytes) {
     static std::mutex mu;
-    static std::map<std::pair<const void*, int>, int> done;  // (kernel, device) -> bytes set
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
+    static std::map<std::pair<const void*, unsigned long long>, int> done;  // (kernel, context) -> bytes set
+    unsigned long long ctx = 0;
+    cudaError_t e = current_context_id(&ctx);
     if (e != cudaSuccess) return e;
     std::lock_guard<std::mutex> lock(mu);
-    const auto key = std::make_pair(kernel, dev);
+    const auto key = std::make_pair(kernel, ctx);
     auto it = done.find(key);
     if (it != done.end() && it->second >= bytes) return cudaSuccess;
     e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
@@ -79,30 +128,44 @@ cudaError_t ensure_smem_limit(const void* kernel, int bytes) {
 
 namespace {
 
-unsigned int* sched_workspace(int dev, cudaStream_t stream) {
+// The counter of `stream` in the current context: its slot of the static pool,
+// handed out on the stream's first causal launch.  FA_ERR_LIMIT once every slot
+// of the context is taken.
+int sched_counter(cudaStream_t stream, unsigned int** out) {
+    unsigned long long ctx = 0;
+    cudaError_t e = fa::current_context_id(&ctx);
+    if (e != cudaSuccess) return cuda_fail(e, "cuCtxGetId");
     std::lock_guard<std::mutex> lock(g_ws_mu);
-    const auto key = std::make_pair(dev, stream);
+    const auto key = std::make_pair(ctx, stream);
     auto it = g_ws.find(key);
-    if (it != g_ws.end()) return it->second;
-    void* ptr = nullptr;
-    if (cudaMalloc(&ptr, 256) != cudaSuccess) {
-        cudaGetLastError();
-        return nullptr;
+    if (it != g_ws.end()) {
+        *out = it->second;
+        return FA_OK;
     }
-    g_ws[key] = static_cast<unsigned int*>(ptr);
-    return static_cast<unsigned int*>(ptr);
+    int& used = g_ws_used[ctx];
+    if (used >= fa::SCHED_POOL_SLOTS) return FA_ERR_LIMIT;
+    unsigned int* pool = nullptr;
+    e = fa::sched_pool_address(&pool);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(scheduler pool)");
+    unsigned int* ctr = pool + (size_t)used * fa::SCHED_SLOT_WORDS;
+    ++used;
+    g_ws[key] = ctr;
+    *out = ctr;
+    return FA_OK;
 }
 
 int device_info(DeviceInfo* out) {
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= MAX_DEVICES) return FA_ERR_LAUNCH;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (dev < 0 || dev >= MAX_DEVICES) return cuda_fail(cudaErrorInvalidDevice, "device index");
     std::lock_guard<std::mutex> lock(g_dev_mu);
     DeviceInfo& d = g_dev[dev];
     if (!d.known) {
-        if (cudaDeviceGetAttribute(&d.major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
-            cudaDeviceGetAttribute(&d.minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
-            cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-            return FA_ERR_LAUNCH;
+        e = cudaDeviceGetAttribute(&d.major, cudaDevAttrComputeCapabilityMajor, dev);
+        if (e == cudaSuccess) e = cudaDeviceGetAttribute(&d.minor, cudaDevAttrComputeCapabilityMinor, dev);
+        if (e == cudaSuccess) e = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
         d.known = true;
     }
     *out = d;
@@ -125,10 +188,14 @@ EncodeTiledFn encoder() {
 // chunk of 128 rows of one head, 128-byte swizzle (the swizzle atom the
 // tcgen05 operand descriptors expect).  Rows past S read as zeros and never
 // bleed into the next head, whatever the layout.
+// Returns true on success; on failure records the CUresult for fa_last_cuda_error.
 bool encode_tensor(CUtensorMap* map, const void* ptr, int B, int H, int S, int D, const long long st[3],
                    int dtype, int box_rows = fa::BLOCK_M) {
     EncodeTiledFn enc = encoder();
-    if (!enc) return false;
+    if (!enc) {
+        cuda_fail(cudaErrorNotSupported, "cuTensorMapEncodeTiled entry point");
+        return false;
+    }
     const cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)S, (cuuint64_t)H, (cuuint64_t)B};
     const cuuint64_t strides[3] = {(cuuint64_t)st[2] * 2, (cuuint64_t)st[1] * 2, (cuuint64_t)st[0] * 2};
     const cuuint32_t box[4] = {64, (cuuint32_t)box_rows, 1, 1};
@@ -138,7 +205,11 @@ bool encode_tensor(CUtensorMap* map, const void* ptr, int B, int H, int S, int D
     CUresult r = enc(map, dt, 4, const_cast<void*>(ptr), dims, strides, box, elem, CU_TENSOR_MAP_INTERLEAVE_NONE,
                      CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS;
+    if (r != CUDA_SUCCESS) {
+        cuda_fail((int)r, "cuTensorMapEncodeTiled");
+        return false;
+    }
+    return true;
 }
 
 // Element strides (b, h, s) of one tensor: the caller's, or contiguous BHSD
@@ -245,7 +316,8 @@ int forward(const void* q, const void* k, const void* v, void* o, float* lse, in
     if (rc != FA_OK) return rc;
     if (dev.major != 10 || dev.minor != 0) return FA_ERR_ARCH;
     int cur = 0;
-    cudaGetDevice(&cur);
+    const cudaError_t de = cudaGetDevice(&cur);
+    if (de != cudaSuccess) return cuda_fail(de, "cudaGetDevice");
     const void* ptrs[6] = {q, k, v, o, lse, mask ? (const void*)mask : (const void*)q};
     for (const void* p : ptrs) {
         rc = check_device_pointer(p, cur);
@@ -286,26 +358,19 @@ int forward(const void* q, const void* k, const void* v, void* o, float* lse, in
         launch_lock.lock();
         unsigned int* ctr = nullptr;
         if (scratch == Scratch::Static) {
-            if (fa::noalloc_scratch_address(&ctr) != cudaSuccess) {
-                cudaGetLastError();
-                return FA_ERR_LAUNCH;
-            }
+            const cudaError_t e = fa::noalloc_scratch_address(&ctr);
+            if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(fa_fwd_noalloc scratch)");
         } else {
-            ctr = sched_workspace(cur, stream);
-            if (!ctr) return FA_ERR_LAUNCH;
+            rc = sched_counter(stream, &ctr);
+            if (rc != FA_OK) return rc;
         }
         // the counter keeps the previous call's value: clear it on this stream
-        if (cudaMemsetAsync(ctr, 0, sizeof(unsigned int), stream) != cudaSuccess) {
-            cudaGetLastError();
-            return FA_ERR_LAUNCH;
-        }
+        const cudaError_t e = cudaMemsetAsync(ctr, 0, sizeof(unsigned int), stream);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(scheduler counter)");
         a.sched = ctr;
     }
     const cudaError_t le = (D == 256) ? fa::launch_fwd_d256_sm100(a, stream) : fa::launch_fwd_sm100(a, stream);
-    if (le != cudaSuccess) {
-        cudaGetLastError();
-        return FA_ERR_LAUNCH;
-    }
+    if (le != cudaSuccess) return cuda_fail(le, D == 256 ? "launch(fa_fwd_kernel_d256)" : "launch(fa_fwd_kernel)");
     return FA_OK;
 }
 
@@ -399,10 +464,9 @@ int backward(const void* q, const void* k, const void* v, const void* o, const v
         if (!dk || !dv) return FA_ERR_NULL;
         if (strides && (strides[6] || strides[7])) return FA_ERR_STRIDE;  // zeroed as whole contiguous blocks
         const size_t bytes = (size_t)BH * (size_t)Sk * (size_t)D * 2;
-        if (cudaMemsetAsync(dk, 0, bytes, stream) != cudaSuccess || cudaMemsetAsync(dv, 0, bytes, stream) != cudaSuccess) {
-            cudaGetLastError();
-            return FA_ERR_LAUNCH;
-        }
+        cudaError_t e = cudaMemsetAsync(dk, 0, bytes, stream);
+        if (e == cudaSuccess) e = cudaMemsetAsync(dv, 0, bytes, stream);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(dk, dv)");
         return FA_OK;
     }
     if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv) return FA_ERR_NULL;
@@ -425,7 +489,8 @@ int backward(const void* q, const void* k, const void* v, const void* o, const v
     if (rc != FA_OK) return rc;
     if (dev.major != 10 || dev.minor != 0) return FA_ERR_ARCH;
     int cur = 0;
-    cudaGetDevice(&cur);
+    const cudaError_t de = cudaGetDevice(&cur);
+    if (de != cudaSuccess) return cuda_fail(de, "cudaGetDevice");
     const void* ptrs[11] = {q, k, v, o, dout, lse, dq, dk, dv, workspace, mask ? (const void*)mask : q};
     for (const void* p : ptrs) {
         rc = check_device_pointer(p, cur);
@@ -464,10 +529,8 @@ int backward(const void* q, const void* k, const void* v, const void* o, const v
     a.dq_flags = nullptr;
     if (deterministic) {
         a.dq_flags = reinterpret_cast<int*>(w + ws.flags);
-        if (cudaMemsetAsync(a.dq_flags, 0, (size_t)ws.flags_bytes, stream) != cudaSuccess) {
-            cudaGetLastError();
-            return FA_ERR_LAUNCH;
-        }
+        const cudaError_t e = cudaMemsetAsync(a.dq_flags, 0, (size_t)ws.flags_bytes, stream);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(deterministic turn counters)");
     }
     a.B = B;
     a.H = H;
@@ -479,10 +542,8 @@ int backward(const void* q, const void* k, const void* v, const void* o, const v
     a.scale = scale;
     const int64_t units = BH * ((Sk + 127) / 128);
     a.grid = (int)(units < dev.sms ? units : dev.sms);
-    if (fa::launch_bwd_sm100(a, stream) != cudaSuccess) {
-        cudaGetLastError();
-        return FA_ERR_LAUNCH;
-    }
+    const cudaError_t le = fa::launch_bwd_sm100(a, stream);
+    if (le != cudaSuccess) return cuda_fail(le, "launch(backward kernels)");
     return FA_OK;
 }
 
@@ -566,19 +627,15 @@ int fa_merge_partial(float* o_acc, float* lse_acc, const void* o_part, const flo
     if ((((uintptr_t)o_acc | (uintptr_t)lse_acc | (uintptr_t)lse_part) & 3u) != 0 || ((uintptr_t)o_part & 1u) != 0)
         return FA_ERR_ALIGN;
     int cur = 0;
-    if (cudaGetDevice(&cur) != cudaSuccess) {
-        cudaGetLastError();
-        return FA_ERR_LAUNCH;
-    }
+    const cudaError_t de = cudaGetDevice(&cur);
+    if (de != cudaSuccess) return cuda_fail(de, "cudaGetDevice");
     const void* ptrs[4] = {o_acc, lse_acc, o_part, lse_part};
     for (const void* p : ptrs) {
         const int rc = check_device_pointer(p, cur);
         if (rc != FA_OK) return rc;
     }
-    if (fa::launch_merge_partial(o_acc, lse_acc, o_part, lse_part, rows, D, dtype, stream) != cudaSuccess) {
-        cudaGetLastError();
-        return FA_ERR_LAUNCH;
-    }
+    const cudaError_t le = fa::launch_merge_partial(o_acc, lse_acc, o_part, lse_part, rows, D, dtype, stream);
+    if (le != cudaSuccess) return cuda_fail(le, "launch(fa_merge_partial)");
     return FA_OK;
 }
 
@@ -589,17 +646,13 @@ int fa_merge_finalize(const float* o_acc, void* o, long long n, int dtype, cudaS
     if (!o_acc || !o) return FA_ERR_NULL;
     if (((uintptr_t)o_acc & 3u) != 0 || ((uintptr_t)o & 1u) != 0) return FA_ERR_ALIGN;
     int cur = 0;
-    if (cudaGetDevice(&cur) != cudaSuccess) {
-        cudaGetLastError();
-        return FA_ERR_LAUNCH;
-    }
+    const cudaError_t de = cudaGetDevice(&cur);
+    if (de != cudaSuccess) return cuda_fail(de, "cudaGetDevice");
     int rc = check_device_pointer(o_acc, cur);
     if (rc == FA_OK) rc = check_device_pointer(o, cur);
     if (rc != FA_OK) return rc;
-    if (fa::launch_merge_finalize(o_acc, o, n, dtype, stream) != cudaSuccess) {
-        cudaGetLastError();
-        return FA_ERR_LAUNCH;
-    }
+    const cudaError_t le = fa::launch_merge_finalize(o_acc, o, n, dtype, stream);
+    if (le != cudaSuccess) return cuda_fail(le, "launch(fa_merge_finalize)");
     return FA_OK;
 }
 
@@ -610,29 +663,23 @@ int fa_accumulate(float* acc, const void* x, long long n, int dtype, cudaStream_
     if (!acc || !x) return FA_ERR_NULL;
     if (((uintptr_t)acc & 3u) != 0 || ((uintptr_t)x & 1u) != 0) return FA_ERR_ALIGN;
     int cur = 0;
-    if (cudaGetDevice(&cur) != cudaSuccess) {
-        cudaGetLastError();
-        return FA_ERR_LAUNCH;
-    }
+    const cudaError_t de = cudaGetDevice(&cur);
+    if (de != cudaSuccess) return cuda_fail(de, "cudaGetDevice");
     int rc = check_device_pointer(acc, cur);
     if (rc == FA_OK) rc = check_device_pointer(x, cur);
     if (rc != FA_OK) return rc;
-    if (fa::launch_accumulate(acc, x, n, dtype, stream) != cudaSuccess) {
-        cudaGetLastError();
-        return FA_ERR_LAUNCH;
-    }
+    const cudaError_t le = fa::launch_accumulate(acc, x, n, dtype, stream);
+    if (le != cudaSuccess) return cuda_fail(le, "launch(fa_accumulate)");
     return FA_OK;
 }
 
 int fa_check_status(cudaStream_t stream) {
     // one status word per kernel translation unit; all are read and cleared
     int st[3] = {0, 0, 0}, site[3] = {0, 0, 0};
-    if (fa::read_and_clear_status(stream, &st[0], &site[0]) != cudaSuccess ||
-        fa::read_and_clear_status_bwd(stream, &st[1], &site[1]) != cudaSuccess ||
-        fa::read_and_clear_status_d256(stream, &st[2], &site[2]) != cudaSuccess) {
-        cudaGetLastError();
-        return FA_ERR_LAUNCH;
-    }
+    cudaError_t e = fa::read_and_clear_status(stream, &st[0], &site[0]);
+    if (e == cudaSuccess) e = fa::read_and_clear_status_bwd(stream, &st[1], &site[1]);
+    if (e == cudaSuccess) e = fa::read_and_clear_status_d256(stream, &st[2], &site[2]);
+    if (e != cudaSuccess) return cuda_fail(e, "fa_check_status (stream synchronize / status word copy)");
     for (int i = 0; i < 3; ++i) {
         if (st[i] != fa::DEV_OK) {
             t_last_site = site[i];
@@ -644,15 +691,18 @@ int fa_check_status(cudaStream_t stream) {
 
 int fa_last_timeout_site(void) { return t_last_site; }
 
+int fa_last_cuda_error(const char** site) {
+    if (site) *site = t_err_site;
+    return t_err_code;
+}
+
 int fa_selftest_timeout(cudaStream_t stream) {
     DeviceInfo dev;
     int rc = device_info(&dev);
     if (rc != FA_OK) return rc;
     if (dev.major != 10 || dev.minor != 0) return FA_ERR_ARCH;
-    if (fa::launch_selftest_timeout(stream) != cudaSuccess) {
-        cudaGetLastError();
-        return FA_ERR_LAUNCH;
-    }
+    const cudaError_t le = fa::launch_selftest_timeout(stream);
+    if (le != cudaSuccess) return cuda_fail(le, "launch(selftest_timeout_kernel)");
     return FA_OK;
 }
 
@@ -665,13 +715,14 @@ const char* fa_status_string(int status) {
         case FA_ERR_DTYPE: return "dtype must be FA_FP16 or FA_BF16";
         case FA_ERR_ALIGN: return "q, k, v, o must be 16-byte aligned and lse 4-byte aligned";
         case FA_ERR_ARCH: return "the current device is not sm_100 (B200)";
-        case FA_ERR_LAUNCH: return "CUDA runtime error";
+        case FA_ERR_LAUNCH: return "CUDA runtime error (fa_last_cuda_error names the call)";
         case FA_ERR_TIMEOUT: return "a device-side wait exceeded its bound";
         case FA_ERR_SCALE: return "scale must be finite and > 0";
         case FA_ERR_ARG: return "causal (and deterministic) must be 0 or 1";
         case FA_ERR_PTR: return "pointer is not device memory of the current device";
         case FA_ERR_STRIDE: return "a stride is not positive, a multiple of 8 elements and below 2^36";
         case FA_ERR_WORKSPACE: return "workspace is NULL, not 256-byte aligned or smaller than fa_bwd_workspace_size";
+        case FA_ERR_LIMIT: return "every scheduler-counter slot of this context is taken (too many streams)";
         default: return "unknown status";
     }
 }

@@ -51,6 +51,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <map>
 #include <mutex>
 
 #include "fa_internal.h"
@@ -65,6 +66,11 @@ __device__ int g_status_site = 0;  // (site) | (block << 8) of the first failing
 // loads the library holds it until the process exits).  Word 0 is the causal
 // work-unit counter.  All fa_fwd_noalloc calls share it.
 static __device__ __align__(256) unsigned int g_noalloc_scratch[NOALLOC_SCRATCH_WORDS];
+
+// Work-unit counters of the causal launches of the other forward entries: one
+// 32-byte slot per (context, stream) that has launched a causal forward, handed
+// out by the host layer; part of the module's static data, so no call allocates.
+static __device__ __align__(256) unsigned int g_sched_pool[SCHED_POOL_SLOTS * SCHED_SLOT_WORDS];
 
 namespace {
 
@@ -82,13 +88,6 @@ static_assert(2 * 128 * REG_SOFTMAX + 128 * REG_CORR + 128 * REG_CTRL <= NUM_THR
 static_assert(2 * REG_SOFTMAX + REG_CORR + REG_CTRL <= 512, "register split exceeds a sub-partition");
 
 constexpr uint32_t TMEM_COLS = 512;
-// One weight pair in FMA_EXP2_PERIOD would be computed on the FMA pipe instead
-// of the MUFU (tiles without masking only); 0 disables it.  Measured on B200
-// with S = 16384, D = 128, bf16 (no register spills in any variant):
-// period 0 -> 1034 TFLOP/s, 8 -> 1012, 4 -> 989: the polynomial's extra
-// instructions on the softmax warps cost more than the ex2 they replace.
-constexpr int FMA_EXP2_PERIOD = 0;
-
 // When the softmax moves a row's reference max m (log2 units) to the block max:
 //  - always when the block max exceeds m by more than TAU = 8 (weights stay
 //    <= 2^8, lazy rescale);
@@ -214,30 +213,6 @@ __device__ __forceinline__ void tmem_ld128(uint32_t taddr, float* v) {
         : "memory");
 #pragma unroll
     for (int i = 0; i < 128; ++i) v[i] = __uint_as_float(r[i]);
-}
-
-// 2^x for a pair of x <= 8 on the FMA pipe, used for part of the weights so the
-// MUFU is not the only unit producing them.  Method: Cody-Waite style range
-// reduction x = n + f with n = round(x) taken from the low mantissa bits of
-// x + 1.5*2^23 and f in [-1/2, 1/2]; 2^f by the degree-3 polynomial of least
-// maximum relative error on [-1/2, 1/2] (Remez exchange; coefficients from
-// exp2_poly_fit.py in this directory; max relative error 7.5e-5 evaluated in
-// float32); n is added to the float's exponent field.  x is clamped at -125 so
-// the result stays a normal float (2^-125 where the exact value underflows).
-__device__ __forceinline__ __attribute__((unused)) float2 exp2_fma2(float2 x) {
-    constexpr float SHIFT = 12582912.0f;  // 1.5 * 2^23
-    x.x = fmaxf(x.x, -125.0f);
-    x.y = fmaxf(x.y, -125.0f);
-    const float2 t = __fadd2_rn(x, make_float2(SHIFT, SHIFT));
-    const float2 r = __fadd2_rn(t, make_float2(-SHIFT, -SHIFT));          // round(x), exact
-    const float2 f = __ffma2_rn(r, make_float2(-1.0f, -1.0f), x);         // x - round(x), exact
-    float2 q = __ffma2_rn(make_float2(0.0551716685295105f, 0.0551716685295105f), f,
-                          make_float2(0.2426111251115799f, 0.2426111251115799f));
-    q = __ffma2_rn(q, f, make_float2(0.6932609677314758f, 0.6932609677314758f));
-    q = __ffma2_rn(q, f, make_float2(0.9999280571937561f, 0.9999280571937561f));
-    // bits(t) = bits(1.5 * 2^23) + n; shifting by 23 leaves n << 23 (mod 2^32)
-    return make_float2(__uint_as_float(__float_as_uint(q.x) + (__float_as_uint(t.x) << 23)),
-                       __uint_as_float(__float_as_uint(q.y) + (__float_as_uint(t.y) << 23)));
 }
 
 // acc + the two bf16 halves of a packed pair, each converted exactly (mixed-precision adds)
@@ -682,9 +657,8 @@ __device__ void softmax_role(const KParams& p, uint8_t* smem, uint32_t tmem, int
             float2 lsum0 = make_float2(0.f, 0.f), lsum1 = make_float2(0.f, 0.f);
             float2 rsum0 = make_float2(0.f, 0.f), rsum1 = make_float2(0.f, 0.f);
             // Weights of a quarter row (16 pairs) into packed 16-bit P, stored to
-            // TMEM right away (fewer live registers); in tiles without masking,
-            // one pair in FMA_EXP2_PERIOD uses the FMA-pipe exp2.
-            auto quarter_row = [&](int qr, bool use_fma_exp) {
+            // TMEM right away (fewer live registers).
+            auto quarter_row = [&](int qr) {
                 uint32_t pk[16];
                 // dropout: keep masks of the quarter's 32 keys (two 16-key generator blocks)
                 uint32_t km[8];
@@ -700,14 +674,7 @@ __device__ void softmax_role(const KParams& p, uint8_t* smem, uint32_t tmem, int
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
                     const float2 x = __ffma2_rn(make_float2(s[32 * qr + 2 * i], s[32 * qr + 2 * i + 1]), sl2x2, negm2);
-                    float2 e;
-                    if constexpr (FMA_EXP2_PERIOD > 0) {
-                        constexpr int P = FMA_EXP2_PERIOD > 0 ? FMA_EXP2_PERIOD : 1;
-                        const bool fma_pair = use_fma_exp && (i % P) == P - 1;
-                        e = fma_pair ? exp2_fma2(x) : make_float2(ex2(x.x), ex2(x.y));
-                    } else {
-                        e = make_float2(ex2(x.x), ex2(x.y));
-                    }
+                    const float2 e = make_float2(ex2(x.x), ex2(x.y));
                     pk[i] = pack2<BF16>(e.x, e.y);
                     if (i & 1) lsum1 = __fadd2_rn(lsum1, e); else lsum0 = __fadd2_rn(lsum0, e);
                     if constexpr (Policy<BF16>::NORM_BY_ROUNDED_P) {
@@ -721,13 +688,8 @@ __device__ void softmax_role(const KParams& p, uint8_t* smem, uint32_t tmem, int
                 // P (16-bit, two per column) overwrites the first 64 columns of S
                 tmem_st16(ts + 16 * qr, pk);
             };
-            if (need_mask) {
 #pragma unroll
-                for (int qr = 0; qr < 4; ++qr) quarter_row(qr, false);
-            } else {
-#pragma unroll
-                for (int qr = 0; qr < 4; ++qr) quarter_row(qr, true);
-            }
+            for (int qr = 0; qr < 4; ++qr) quarter_row(qr);
             const float2 ls = __fadd2_rn(lsum0, lsum1);
             l += ls.x + ls.y;
             if constexpr (Policy<BF16>::NORM_BY_ROUNDED_P) {
@@ -1032,24 +994,41 @@ cudaError_t launch_selftest_timeout(cudaStream_t stream) {
     return launch_kernel(selftest_timeout_kernel, dim3(1), dim3(64), 0, stream, 100000000ll);
 }
 
-cudaError_t noalloc_scratch_address(unsigned int** out) {
-    // The array's name in host code is only a stand-in; the device address is
-    // looked up once per device, with that device current.
-    static std::mutex mu;
-    static unsigned int* addr[64] = {};
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
+namespace {
+
+// Device address of a static array in the current context, looked up once per
+// context.  In host code the array's name is only a stand-in, not a device
+// address; cudaGetSymbolAddress gives the address with that context current.
+template <typename T, size_t N>
+cudaError_t symbol_address_per_context(const T (&symbol)[N], std::mutex& mu,
+                                       std::map<unsigned long long, unsigned int*>& cache, unsigned int** out) {
+    unsigned long long ctx = 0;
+    cudaError_t e = current_context_id(&ctx);
     if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
     std::lock_guard<std::mutex> lock(mu);
-    if (!addr[dev]) {
+    auto it = cache.find(ctx);
+    if (it == cache.end()) {
         void* ptr = nullptr;
-        e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+        e = cudaGetSymbolAddress(&ptr, symbol);
         if (e != cudaSuccess) return e;
-        addr[dev] = static_cast<unsigned int*>(ptr);
+        it = cache.emplace(ctx, static_cast<unsigned int*>(ptr)).first;
     }
-    *out = addr[dev];
+    *out = it->second;
     return cudaSuccess;
+}
+
+}  // namespace
+
+cudaError_t noalloc_scratch_address(unsigned int** out) {
+    static std::mutex mu;
+    static std::map<unsigned long long, unsigned int*> cache;
+    return symbol_address_per_context(g_noalloc_scratch, mu, cache, out);
+}
+
+cudaError_t sched_pool_address(unsigned int** out) {
+    static std::mutex mu;
+    static std::map<unsigned long long, unsigned int*> cache;
+    return symbol_address_per_context(g_sched_pool, mu, cache, out);
 }
 
 cudaError_t read_and_clear_status(cudaStream_t stream, int* status, int* site) {

@@ -113,10 +113,11 @@ inline BwdWorkspace bwd_workspace_layout(int64_t BH, int64_t Sq, int64_t D) {
 
 // LSE-weighted merge of a partial attention result into a running fp32 one,
 // and the conversion of the running O to 16 bits (fa_merge_sm100.cu).
-// Raises `kernel`'s dynamic shared-memory limit to `bytes` on the current
-// device, once per (kernel, device) for the life of the process: later
+// Raises `kernel`'s dynamic shared-memory limit to `bytes` in the current
+// context, once per (kernel, context) for the life of the process: later
 // launches make no attribute call, so host threads launching at the same time
-// never set an attribute of a kernel that another thread is launching.
+// never set an attribute of a kernel that another thread is launching.  A
+// context re-created after cudaDeviceReset has a new id and is set again.
 cudaError_t ensure_smem_limit(const void* kernel, int bytes);
 
 // Launches `kernel` on `stream` and returns the status of this launch alone
@@ -166,9 +167,23 @@ cudaError_t read_and_clear_status_d256(cudaStream_t stream, int* status, int* si
 constexpr int NOALLOC_SCRATCH_WORDS = 64;
 constexpr long long NOALLOC_MAX_CLAIMS = 0x7FFFFFFFll;
 
-// Device address of the static scratch array on the current device (looked
-// up once per device).
+// Device address of the static scratch array in the current context (looked
+// up once per context, so a context re-created after cudaDeviceReset gets a
+// fresh lookup).
 cudaError_t noalloc_scratch_address(unsigned int** out);
+
+// Causal work-unit counters of the other forward entries: a static pool of
+// SCHED_POOL_SLOTS counters in the library's own device memory, one slot per
+// (context, stream) that has launched a causal forward, 32 bytes apart.  The
+// pool is part of the loaded module: handing out a slot allocates nothing.
+constexpr int SCHED_POOL_SLOTS = 2048;
+constexpr int SCHED_SLOT_WORDS = 8;
+cudaError_t sched_pool_address(unsigned int** out);
+
+// Unique id of the CUDA context current in the calling thread (the device's
+// primary context unless the caller made another current); binds the
+// current device's primary context to the thread first if none is current.
+cudaError_t current_context_id(unsigned long long* id);
 
 // Launch the diagnostic kernel whose first wait is never satisfied.
 cudaError_t launch_selftest_timeout(cudaStream_t stream);
