@@ -2,14 +2,14 @@
 
 - small and ragged shapes, both head dims, both dtypes, with and without the
   causal mask: every output element against the oracle;
-- the workload configurations: the three smaller ones element by element,
-  the three long-sequence ones (S = 8192, 16384) on sampled rows (every
-  head's first and last rows plus seeded random rows) in the launch
+- the workload configurations, every output element against the full fp64
+  oracle, the long-sequence ones (S = 8192, 16384) in the launch
   configuration the benchmark times;
 - properties that hold at any size: Q = 0 gives the column mean / causal
   prefix mean of V and LSE = log(key count); causal row 0 equals V_0;
 - bitwise determinism across runs, and every output row written.
 """
+import json
 import math
 
 import numpy as np
@@ -18,7 +18,7 @@ import torch
 
 import oracle
 import tiled_attention_18_b200 as fa
-from tiled_attention_18_b200.workloads import WORKLOADS, make_inputs, sample_rows, softmax_scale, workload_inputs
+from tiled_attention_18_b200.workloads import WORKLOADS, make_inputs, softmax_scale, workload_inputs
 
 from gpu_helpers import compare, run_fa
 
@@ -52,25 +52,24 @@ def test_workload_full_compare(name):
     o, lse = run_fa(q, k, v, w.scale, w.causal)
     o_ref, lse_ref = oracle.attn_fwd(q, k, v, w.scale, w.causal, w.dtype)
     r = compare(o, lse, o_ref, lse_ref, w.dtype)
-    print(name, r)
+    print("parity", name, json.dumps(r))
 
 
 @pytest.mark.parametrize("name", ["c4", "c5a", "c5b"])
-def test_workload_sampled_rows(name):
+def test_workload_long_full_compare(name):
+    """The long-sequence workloads (S = 8192 and 16384), every output element
+    against the full fp64 oracle, in the launch configuration the benchmark
+    times (the oracle takes minutes of host time here, all cores)."""
     w = WORKLOADS[name]
     q, k, v = workload_inputs(w)
     o, lse = run_fa(q, k, v, w.scale, w.causal)
-    bh, rows = sample_rows(w.B, w.H, w.S, n_random=1024, edge=2)
-    o_ref, lse_ref = oracle.attn_rows(q, k, v, w.scale, w.causal, w.dtype, bh, rows)
-    og = o.reshape(w.B * w.H, w.S, w.D)[torch.from_numpy(bh), torch.from_numpy(rows)]
-    lg = lse.reshape(w.B * w.H, w.S)[torch.from_numpy(bh), torch.from_numpy(rows)]
-    r = compare(og, lg, o_ref, lse_ref, w.dtype)
-    print(name, r)
-    # every row written (outputs started as NaN)
-    assert torch.isfinite(o).all() and torch.isfinite(lse).all()
+    assert torch.isfinite(o).all() and torch.isfinite(lse).all()  # every row written (outputs started as NaN)
     if w.causal:
         # row 0 attends to key 0 only: O_0 = V_0 exactly
         assert torch.equal(o[:, :, 0], v[:, :, 0])
+    o_ref, lse_ref = oracle.attn_fwd(q, k, v, w.scale, w.causal, w.dtype)
+    r = compare(o, lse, o_ref, lse_ref, w.dtype)
+    print("parity", name, json.dumps(r))
 
 
 @pytest.mark.parametrize("dtype", ["fp16", "bf16"])
@@ -105,6 +104,33 @@ def test_deterministic_and_stream():
     assert fa.fa_check_status(s.cuda_stream) == 0
     for o, lse in outs[1:]:
         assert torch.equal(o, outs[0][0]) and torch.equal(lse, outs[0][1])
+
+
+@pytest.mark.parametrize("D", [128, 256])
+def test_causal_call_on_a_new_stream_allocates_nothing(D):
+    """The causal scheduler's counter comes from a static pool in the library:
+    the first causal fa_fwd on a stream the library has not seen before leaves
+    the device's free memory unchanged, and two streams running at once keep
+    separate counters (both results match a single-stream run bit for bit)."""
+    q, k, v = (t.cuda() for t in make_inputs(1, 4, 1500, D, "bf16", seed=31))
+    scale = softmax_scale(D)
+    o_ref, lse_ref = fa.flash_attention_forward(q, k, v, scale, True)  # kernels loaded
+    streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+    outs = [(torch.empty_like(q), torch.empty((1, 4, 1500), dtype=torch.float32, device="cuda")) for _ in streams]
+    for s in streams:
+        with torch.cuda.stream(s):
+            outs[0][0].zero_()  # each stream's first launch is not the library's
+    torch.cuda.synchronize()
+    free_before, _ = torch.cuda.mem_get_info()
+    for s, (o, lse) in zip(streams, outs):
+        fa.flash_attention_forward(q, k, v, scale, True, out=o, lse=lse, stream=s)
+    torch.cuda.synchronize()
+    free_after, _ = torch.cuda.mem_get_info()
+    assert free_after == free_before, f"device free memory moved by {free_before - free_after} bytes"
+    for s in streams:
+        assert fa.fa_check_status(s.cuda_stream) == 0
+    for o, lse in outs:
+        assert torch.equal(o, o_ref) and torch.equal(lse, lse_ref)
 
 
 def test_scale_is_honoured():
