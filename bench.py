@@ -10,7 +10,9 @@ A step is one pass of the whole forward path over one batch of synthetic
 input.  The default workload is the long-context configuration
 B=1, H=32, S=16384, D=128, bf16, run both without and with the causal mask
 (two fa_fwd launches per step).  Inputs (512 MiB) are larger than the 126 MB
-L2, so no L2 flush is needed between steps.
+L2, so no L2 flush is needed between steps.  Beside the step, the 13B-style
+causal layer (B=1, H=40, S=8192, D=128, Q,K x2) is timed alone with the same
+protocol and reported under "extra_runs" (not part of the step's value).
 
 The general-shape workloads (sdxl_xattn: 4096 queries over 77 keys;
 bert_large: B=32, H=16, S=512, D=64 in the BSHD layout; prefill_cached:
@@ -91,7 +93,7 @@ def peak_tflops():
             p = json.load(f)
         return float(p["bf16_tflops"]), "measured (MEASURED_PEAKS.json bf16_tflops, burst)"
     except Exception:
-        return FALLBACK_BF16_TFLOPS, "fallback (1.59 PFLOP/s pool measurement)"
+        return FALLBACK_BF16_TFLOPS, "fallback (1.59 PFLOP/s, an earlier cuBLAS bf16 measurement on B200)"
 
 
 def kernel_source_hash() -> str:
@@ -209,6 +211,51 @@ def cpu_baseline(name: str, target_s: float = 12.0, dropout: float = 0.0):
                       " algorithmic flops)"}
 
 
+def algorithmic_bytes(w) -> float:
+    """Bytes one forward launch must move: Q, K, V read and O written in 16 bits, the fp32 LSE written."""
+    return float(w.B * w.H * (2 * w.S * w.D * 2 + 2 * w.Skv * w.D * 2 + 4 * w.S))
+
+
+def time_single_run(fa, w, dev, stream, steps: int, warmup: int, rank: int):
+    """Time one forward workload alone (its own inputs, seeded per rank; rotated over
+    device copies when smaller than twice the L2), CUDA events around each launch on
+    the launching stream.  Returns the run's mean launch time and TFLOP/s."""
+    import torch
+    wr = dataclasses.replace(w, seed=rank_seed(w.seed, rank))
+    q, k, v = workload_inputs(wr)
+    set_bytes = sum(t.numel() * t.element_size() for t in (q, k, v))
+    copies = 1 if set_bytes >= 2 * L2_BYTES else min(64, -(-2 * L2_BYTES // set_bytes))
+    ins = [tuple(t.to(dev) for t in (q, k, v)) for _ in range(copies)]
+    o = torch.empty((w.B, w.H, w.S, w.D), dtype=w.torch_dtype, device=dev)
+    lse = torch.empty((w.B, w.H, w.S), dtype=torch.float32, device=dev)
+    dt = fa.FA_BF16 if w.dtype == "bf16" else fa.FA_FP16
+    sid = stream.cuda_stream
+
+    def launch(i):
+        qq, kk, vv = ins[i % copies]
+        st = fa.fa_fwd(qq.data_ptr(), kk.data_ptr(), vv.data_ptr(), o.data_ptr(), lse.data_ptr(), w.B, w.H, w.S,
+                       w.D, w.scale, int(w.causal), dt, sid)
+        if st != 0:
+            raise fa.FaError(st)
+
+    for i in range(warmup):
+        launch(i)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    torch.cuda.synchronize(dev)
+    for i, (a, b) in enumerate(ev):
+        a.record(stream)
+        launch(i)
+        b.record(stream)
+    torch.cuda.synchronize(dev)
+    st = fa.fa_check_status(sid)
+    if st != 0:
+        raise fa.FaError(st, "timed run")
+    mean_ms = float(np.mean([a.elapsed_time(b) for a, b in ev]))
+    return {"run": w.describe(), "launches": steps, "mean_ms": mean_ms,
+            "tflops": w.flops / (mean_ms * 1e-3) / 1e12,
+            "hbm_gbs": algorithmic_bytes(w) / (mean_ms * 1e-3) / 1e9}
+
+
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -216,11 +263,13 @@ def run_reference(args):
     runs = workload_runs(args.workload)
     bwd = args.pass_ == "bwd"
     # the oracle keeps no state between calls: warm-up steps have nothing to warm
-    times = []
+    times, walls = [], []
     for _ in range(args.steps):
         budget = args.cpu_seconds if args.cpu_seconds > 0 else max(2.0, 60.0 / max(args.steps, 1))
+        t0 = time.perf_counter()
         cb = (cpu_baseline_bwd(args.workload, target_s=budget, dropout=args.dropout) if bwd else
               cpu_baseline(args.workload, target_s=budget, dropout=args.dropout))
+        walls.append(time.perf_counter() - t0)
         times.append(cb)
     value = float(np.median([c["value"] for c in times]))
     cb = dict(times[-1])
@@ -231,9 +280,12 @@ def run_reference(args):
     line = {
         "impl": "reference", "metric": BWD_METRIC if bwd else METRIC, "value": value, "unit": UNIT,
         "n_gpus": args.gpus,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_flops / (value * 1e12) * 1e3,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * float(np.mean(walls)),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": label, "note": "fp64 CPU oracle on bounded samples"},
+        "config": {"workload": label,
+                   "note": "fp64 CPU oracle; each step is a bounded sample of the workload (ms_per_step is the"
+                           " measured wall time of one sampled step; value is the sample's TFLOP/s)",
+                   "projected_ms_per_full_step": step_flops / (value * 1e12) * 1e3},
         "cpu_baseline": cb,
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -461,7 +513,7 @@ def hbm_peak():
         with open(PEAKS_PATH) as f:
             return float(json.load(f)["hbm_gbs"]), "measured (MEASURED_PEAKS.json hbm_gbs)"
     except Exception:
-        return FALLBACK_HBM_GBS, "fallback (6.65 TB/s pool measurement)"
+        return FALLBACK_HBM_GBS, "fallback (6.65 TB/s, an earlier copy-bandwidth measurement on B200)"
 
 
 def run_sp(args) -> int:
@@ -622,6 +674,8 @@ def main(argv=None) -> int:
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="do not time the S = 8192 causal layer (c4) beside the default step")
     ap.add_argument("--cpu-seconds", type=float, default=0.0,
                     help="--impl reference: CPU seconds per step (default: about a minute per run)")
     ap.add_argument("--pass", dest="pass_", choices=["fwd", "bwd", "sp"], default="fwd",
@@ -774,13 +828,30 @@ def main(argv=None) -> int:
     step_flops = sum(w.flops for w in runs)
     value = job_throughput(step_flops, args.steps, world, max_ms)
     peak, peak_src = peak_tflops()
-
     # roofline of the kernel: algorithmic flops per launch / mean launch duration
+    hbm, hbm_src = hbm_peak()
     per_run = []
     for i, w in enumerate(runs):
         mean_ms = float(kern_ms[:, i].mean())
-        per_run.append({"run": w.describe(), "mean_ms": mean_ms, "tflops": w.flops / (mean_ms * 1e-3) / 1e12})
+        gbs = algorithmic_bytes(w) / (mean_ms * 1e-3) / 1e9
+        per_run.append({"run": w.describe(), "mean_ms": mean_ms, "tflops": w.flops / (mean_ms * 1e-3) / 1e12,
+                        "frac": w.flops / (mean_ms * 1e-3) / 1e12 / peak,
+                        "hbm_gbs": gbs, "hbm_frac": gbs / hbm})
     achieved = step_flops / (float(kern_ms.sum(axis=1).mean()) * 1e-3) / 1e12
+    step_bytes = sum(algorithmic_bytes(w) for w in runs)
+    hbm_achieved = step_bytes / (float(kern_ms.sum(axis=1).mean()) * 1e-3) / 1e9
+    # fewer work units than SMs: neither the tensor pipe nor HBM can be busy (launch/latency-bound)
+    n_units = sum(fa.fa_num_units(w.B, w.H, w.S) for w in runs if not w.general)
+    bound = "latency" if (not runs[0].general and n_units < torch.cuda.get_device_properties(dev).multi_processor_count
+                          ) else "tensor"
+
+    # the 13B-style layer (S = 8192, causal, Q,K x2) timed beside the default step
+    extra_runs = []
+    if args.workload == "c5" and args.dropout == 0.0 and not tril and not args.no_extra:
+        r = time_single_run(fa, WORKLOADS["c4"], dev, stream, max(args.steps, 10), args.warmup, rank)
+        r["frac"] = r["tflops"] / peak
+        r["hbm_frac"] = r["hbm_gbs"] / hbm
+        extra_runs.append(r)
     # the committed DRAM capture is of the kernels without dropout or an explicit mask
     traffic = traffic_per_launch(args.workload) if (args.dropout == 0.0 and not tril) else None
 
@@ -837,9 +908,12 @@ def main(argv=None) -> int:
                               f"inputs rotated over {max(n_copies)} device copies (> 2x L2 per rotation, no flush)"),
                        "parallelism": f"independent batch per GPU x{world}"},
             "pct_of_peak": 100.0 * value / (peak * world),
-            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": UNIT,
+            "roofline": {"bound": bound, "achieved": achieved, "peak": peak, "unit": UNIT,
                          "frac": achieved / peak, "traffic": traffic, "peak_source": peak_src,
-                         "per_run": per_run},
+                         "per_run": per_run,
+                         "hbm": {"algorithmic_bytes_per_step": step_bytes, "achieved": hbm_achieved, "peak": hbm,
+                                 "unit": "GB/s", "frac": hbm_achieved / hbm, "peak_source": hbm_src}},
+            "extra_runs": extra_runs,
             "clocks": sampler.summary(),
             "e2e": e2e,
             "gpu_launches": len(runs) * args.steps,
