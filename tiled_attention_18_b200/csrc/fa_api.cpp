@@ -172,6 +172,16 @@ int device_info(DeviceInfo* out) {
     return FA_OK;
 }
 
+// cuTensorMapEncodeTiled is a driver call and needs a context current in the
+// calling thread; the runtime calls made before it (attribute and pointer
+// queries) do not bind one in a thread that has made no other CUDA call.
+// Binds the current device's primary context when none is current.
+int bind_context() {
+    unsigned long long ctx = 0;
+    const cudaError_t e = fa::current_context_id(&ctx);
+    return e == cudaSuccess ? FA_OK : cuda_fail(e, "cuCtxGetCurrent / cudaSetDevice (binding a context)");
+}
+
 EncodeTiledFn encoder() {
     std::call_once(g_encode_once, [] {
         void* fn = nullptr;
@@ -315,6 +325,8 @@ int forward(const void* q, const void* k, const void* v, void* o, float* lse, in
     rc = device_info(&dev);
     if (rc != FA_OK) return rc;
     if (dev.major != 10 || dev.minor != 0) return FA_ERR_ARCH;
+    rc = bind_context();
+    if (rc != FA_OK) return rc;
     int cur = 0;
     const cudaError_t de = cudaGetDevice(&cur);
     if (de != cudaSuccess) return cuda_fail(de, "cudaGetDevice");
@@ -488,6 +500,8 @@ int backward(const void* q, const void* k, const void* v, const void* o, const v
     int rc = device_info(&dev);
     if (rc != FA_OK) return rc;
     if (dev.major != 10 || dev.minor != 0) return FA_ERR_ARCH;
+    rc = bind_context();
+    if (rc != FA_OK) return rc;
     int cur = 0;
     const cudaError_t de = cudaGetDevice(&cur);
     if (de != cudaSuccess) return cuda_fail(de, "cudaGetDevice");
