@@ -3,6 +3,7 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl fa|reference]
                     [--workload c5|c1|c2|c3|c4|c5a|c5b|sdxl_xattn|bert_large|prefill_cached|d256_long]
                     [--pass fwd|bwd|sp] [--mask tril] [--dropout P] [--deterministic]
+                    [--block-n 64|128] [--q-tiles 1|2]
                     [--sp-world W] [--sp-mode ring|allgather|ulysses]
                     [--no-e2e] [--no-cpu-baseline] [--cpu-seconds S]
 
@@ -688,6 +689,10 @@ def main(argv=None) -> int:
                          "(the catlass page's mode 1) instead of the in-kernel diagonal skip (mode 2)")
     ap.add_argument("--dropout", type=float, default=0.0,
                     help="attention dropout probability (fa_fwd_dropout / fa_bwd_dropout); 0 = none")
+    ap.add_argument("--block-n", type=int, default=0, choices=[0, 64, 128],
+                    help="forward keys per key tile (0 = automatic, 128); through fa_forward")
+    ap.add_argument("--q-tiles", type=int, default=0, choices=[0, 1, 2],
+                    help="forward 128-row query tiles per work unit (0 = automatic, 2); through fa_forward")
     ap.add_argument("--deterministic", action="store_true",
                     help="with --pass bwd: the deterministic dQ mode (key tiles add in order)")
     args = ap.parse_args(argv)
@@ -781,6 +786,12 @@ def main(argv=None) -> int:
             m = tril[i]
             st = fa.fa_fwd_mask(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), w.B, w.H,
                                 w.S, w.Skv, w.D, m.data_ptr(), (0, 0, m.stride(0)), w.scale, 0, dt, sid)
+        elif args.block_n or args.q_tiles:
+            st = fa.fa_forward(sid, q=q.data_ptr(), k=k.data_ptr(), v=v.data_ptr(), o=o.data_ptr(),
+                               lse=lse.data_ptr(), B=w.B, H=w.H, Sq=w.S, Sk=w.Skv, D=w.D, q_stride=q.stride()[:3],
+                               k_stride=k.stride()[:3], v_stride=v.stride()[:3], o_stride=o.stride()[:3],
+                               scale=w.scale, causal=int(w.causal), dtype=dt, block_n=args.block_n,
+                               q_tiles=args.q_tiles)
         elif w.general:
             st = fa.fa_fwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), w.B, w.H, w.S,
                               w.Skv, w.D, q.stride()[:3], k.stride()[:3], v.stride()[:3], o.stride()[:3], w.scale,
@@ -847,13 +858,15 @@ def main(argv=None) -> int:
 
     # the 13B-style layer (S = 8192, causal, Q,K x2) timed beside the default step
     extra_runs = []
-    if args.workload == "c5" and args.dropout == 0.0 and not tril and not args.no_extra:
+    if (args.workload == "c5" and args.dropout == 0.0 and not tril and not args.no_extra and not args.block_n
+            and not args.q_tiles):
         r = time_single_run(fa, WORKLOADS["c4"], dev, stream, max(args.steps, 10), args.warmup, rank)
         r["frac"] = r["tflops"] / peak
         r["hbm_frac"] = r["hbm_gbs"] / hbm
         extra_runs.append(r)
     # the committed DRAM capture is of the kernels without dropout or an explicit mask
-    traffic = traffic_per_launch(args.workload) if (args.dropout == 0.0 and not tril) else None
+    traffic = (traffic_per_launch(args.workload)
+               if (args.dropout == 0.0 and not tril and not args.block_n and not args.q_tiles) else None)
 
     # end to end through the public call with host buffers
     e2e = None
@@ -900,7 +913,9 @@ def main(argv=None) -> int:
             "scaling": "weak", "vs_baseline": None, "dtype": w0.dtype, "data": "synthetic",
             "config": {"workload": workload_label(args.workload)
                        + (" (causal as an explicit lower-triangular mask, no tile skipping)" if tril else "")
-                       + (f", attention dropout p = {args.dropout:g} (fresh offset per step)" if args.dropout > 0 else ""),
+                       + (f", attention dropout p = {args.dropout:g} (fresh offset per step)" if args.dropout > 0 else "")
+                       + (f", tiling block_n={args.block_n or 128} q_tiles={args.q_tiles or 2}"
+                          if (args.block_n or args.q_tiles) else ""),
                        "B": w0.B, "H": w0.H, "S": w0.S, "D": w0.D,
                        **({"Sk": w0.Skv, "layout": w0.layout} if w0.general else {}),
                        "runs_per_step": len(runs),

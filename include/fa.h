@@ -364,6 +364,15 @@ typedef struct fa_fwd_params {
     float scale;
     int causal;
     int dtype;
+    /* Tiling (0 = automatic: 128-key tiles, two 128-row query tiles per work
+     * unit).  block_n: keys per key tile, 64 or 128; q_tiles: 128-row query
+     * tiles per work unit, 1 or 2.  A manual tiling takes D = 64 or 128 and no
+     * mask or dropout; otherwise FA_ERR_ARG.  The FlashAttention-2 page lets
+     * the caller set the block sizes by hand for particular shapes ("FlashAttention-2
+     * 在昇腾 NPU 上如何做到 3 倍加速？", section 6.1); the catlass page tabulates
+     * block_m x block_n against throughput (section "分块策略不是越大越好"). */
+    int block_n;
+    int q_tiles;
 } fa_fwd_params;
 
 typedef struct fa_bwd_params {

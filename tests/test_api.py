@@ -326,3 +326,17 @@ def test_every_launch_reports_its_own_status():
         # the shared-memory limit is raised once per kernel and device, not per launch
         if not path.endswith("fa_api.cpp"):
             assert "cudaFuncSetAttribute" not in text, path
+
+
+def test_forward_tiling_arguments_are_checked_before_any_device_work():
+    """fa_forward's block_n / q_tiles: 0 (automatic), 64/128 and 1/2; a manual
+    tiling takes D = 64/128 without mask or dropout (FA_ERR_ARG otherwise).
+    All of these are found before a pointer is inspected."""
+    from tiled_attention_18_b200 import _lib
+    base = dict(q=16, k=16, v=16, o=16, lse=16, B=1, H=1, Sq=64, Sk=64, D=128, scale=0.1, causal=0, dtype=1)
+    assert _lib.fa_forward(0, **base, block_n=96) == -10
+    assert _lib.fa_forward(0, **base, q_tiles=3) == -10
+    assert _lib.fa_forward(0, **base, q_tiles=-1) == -10
+    assert _lib.fa_forward(0, **{**base, "D": 256}, block_n=64) == -10
+    assert _lib.fa_forward(0, **base, block_n=64, dropout_p=0.1) == -10
+    assert _lib.fa_forward(0, **base, q_tiles=1, mask=16, mask_stride=(0, 0, 64)) == -10

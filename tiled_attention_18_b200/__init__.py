@@ -46,7 +46,8 @@ def _mask_stride(mask, B, H, Sq, Sk):
 
 
 def flash_attention_forward(q, k, v, scale: float, causal: bool = False, out=None, lse=None, stream=None,
-                            dropout_p: float = 0.0, seed: int = 0, offset: int = 0, mask=None):
+                            dropout_p: float = 0.0, seed: int = 0, offset: int = 0, mask=None, block_n: int = 0,
+                            q_tiles: int = 0):
     """O, LSE for CUDA tensors ``q`` [B, H, Sq, D] and ``k, v`` [B, H, Sk, D] (fp16/bf16).
 
     The tensors may be any strided views whose last dimension is contiguous
@@ -63,7 +64,10 @@ def flash_attention_forward(q, k, v, scale: float, causal: bool = False, out=Non
     flash_attention_backward must be given too).  ``mask`` (a uint8/bool CUDA
     tensor [B|1, H|1, Sq, Sk], nonzero = attend, keys contiguous, row stride a
     multiple of 16 and >= Sk) restricts the keys each query sees.  Mask,
-    dropout, strides and Sq != Sk combine freely (fa_forward).
+    dropout, strides and Sq != Sk combine freely (fa_forward).  ``block_n``
+    (64 or 128 keys per key tile) and ``q_tiles`` (1 or 2 query tiles of 128
+    rows per work unit) set the tiling by hand (0 = automatic; D = 64/128,
+    without mask or dropout).
     """
     import torch
     if q.dim() != 4 or k.dim() != 4 or v.shape != k.shape:
@@ -91,14 +95,14 @@ def flash_attention_forward(q, k, v, scale: float, causal: bool = False, out=Non
         stream = torch.cuda.current_stream(q.device)
     st = int(stream.cuda_stream)
     dt = _dtype_code(q)
-    if dropout_p != 0.0 or mask is not None:
+    if dropout_p != 0.0 or mask is not None or block_n or q_tiles:
         rc = fa_forward(st, q=q.data_ptr(), k=k.data_ptr(), v=v.data_ptr(), o=out.data_ptr(), lse=lse.data_ptr(),
                         B=B, H=H, Sq=Sq, Sk=Sk, D=D, q_stride=q.stride()[:3], k_stride=k.stride()[:3],
                         v_stride=v.stride()[:3], o_stride=out.stride()[:3],
                         mask=mask.data_ptr() if mask is not None else None,
                         mask_stride=_mask_stride(mask, B, H, Sq, Sk) if mask is not None else None,
                         dropout_p=float(dropout_p), seed=seed, offset=offset, scale=float(scale),
-                        causal=int(bool(causal)), dtype=dt)
+                        causal=int(bool(causal)), dtype=dt, block_n=int(block_n), q_tiles=int(q_tiles))
         if rc != 0:
             raise FaError(rc, "fa_forward")
         return out, lse

@@ -229,7 +229,8 @@ class FwdParams(ctypes.Structure):
                 ("Sk", ctypes.c_int), ("D", ctypes.c_int), ("q_stride", _LLP), ("k_stride", _LLP),
                 ("v_stride", _LLP), ("o_stride", _LLP), ("mask", ctypes.c_void_p), ("mask_stride", _LLP),
                 ("dropout_p", ctypes.c_float), ("seed", ctypes.c_ulonglong), ("offset", ctypes.c_uint),
-                ("scale", ctypes.c_float), ("causal", ctypes.c_int), ("dtype", ctypes.c_int)]
+                ("scale", ctypes.c_float), ("causal", ctypes.c_int), ("dtype", ctypes.c_int),
+                ("block_n", ctypes.c_int), ("q_tiles", ctypes.c_int)]
 
 
 class BwdParams(ctypes.Structure):

@@ -291,12 +291,19 @@ int forward(const void* q, const void* k, const void* v, void* o, float* lse, in
             const long long* q_stride, const long long* k_stride, const long long* v_stride,
             const long long* o_stride, float scale, int causal, int dtype, cudaStream_t stream, Scratch scratch,
             const uint8_t* mask = nullptr, const long long* mask_stride = nullptr,
-            const fa::DropoutArgs* drop = nullptr) {
+            const fa::DropoutArgs* drop = nullptr, int block_n = 0, int q_tiles = 0) {
     if (B < 0 || H < 0 || Sq < 0 || Sk < 0) return FA_ERR_SHAPE;
     if (D != 64 && D != 128 && D != 256) return FA_ERR_HEADDIM;
     if (dtype != FA_FP16 && dtype != FA_BF16) return FA_ERR_DTYPE;
     if (!(std::isfinite(scale) && scale > 0.f)) return FA_ERR_SCALE;
     if (causal != 0 && causal != 1) return FA_ERR_ARG;
+    // tiling: 0 = automatic (128-key tiles, two 128-row query tiles per unit);
+    // manual tilings for D = 64/128 without an explicit mask or dropout
+    if ((block_n != 0 && block_n != 64 && block_n != 128) || (q_tiles < 0 || q_tiles > 2)) return FA_ERR_ARG;
+    if (block_n == 0) block_n = fa::BLOCK_N;
+    if (q_tiles == 0) q_tiles = fa::Q_TILES_PER_CTA;
+    const bool manual = block_n != fa::BLOCK_N || q_tiles != fa::Q_TILES_PER_CTA;
+    if (manual && (D == 256 || mask || (drop && drop->enabled))) return FA_ERR_ARG;
     if (B == 0 || H == 0 || Sq == 0) return FA_OK;  // empty problem
     // every query row must see at least one key
     if (Sk == 0 || (causal && Sq > Sk)) return FA_ERR_SHAPE;
@@ -335,7 +342,7 @@ int forward(const void* q, const void* k, const void* v, void* o, float* lse, in
         rc = check_device_pointer(p, cur);
         if (rc != FA_OK) return rc;
     }
-    const int64_t units = (D == 256) ? fa::num_units_d256(BH, Sq) : fa::num_units(BH, Sq);
+    const int64_t units = (D == 256) ? fa::num_units_d256(BH, Sq) : fa::num_units(BH, Sq, q_tiles);
     const int grid = (int)(units < dev.sms ? units : dev.sms);
     // fa_fwd_noalloc's counter is read back as an int: the claims of all CTAs must fit
     if (scratch == Scratch::Static && units + grid > fa::NOALLOC_MAX_CLAIMS) return FA_ERR_SHAPE;
@@ -343,7 +350,7 @@ int forward(const void* q, const void* k, const void* v, void* o, float* lse, in
     fa::LaunchArgs a;
     std::memset(&a, 0, sizeof(a));
     // the D = 256 kernel streams keys and values in 64-row tiles
-    const int kv_box = (D == 256) ? 64 : fa::BLOCK_N;
+    const int kv_box = (D == 256) ? 64 : block_n;
     if (!encode_tensor(&a.tmap_q, q, B, H, Sq, D, qs, dtype) ||
         !encode_tensor(&a.tmap_k, k, B, H, Sk, D, ks, dtype, kv_box) ||
         !encode_tensor(&a.tmap_v, v, B, H, Sk, D, vs, dtype, kv_box))
@@ -364,6 +371,8 @@ int forward(const void* q, const void* k, const void* v, void* o, float* lse, in
     a.scale_log2 = (float)((double)scale * 1.4426950408889634074);  // scale * log2(e)
     a.grid = grid;
     a.sched = nullptr;
+    a.block_n = block_n;
+    a.q_tiles = q_tiles;
     std::unique_lock<std::mutex> launch_lock(g_launch_mu, std::defer_lock);
     if (causal) {
         // units differ in length under the mask: CTAs claim them from a counter
@@ -614,7 +623,8 @@ int fa_forward(const fa_fwd_params* p, cudaStream_t stream) {
     if (p->B > 0 && p->H > 0 && p->Sq > 0 && p->mask && !p->mask_stride) return FA_ERR_NULL;
     return forward(p->q, p->k, p->v, p->o, p->lse, p->B, p->H, p->Sq, p->Sk, p->D, p->q_stride, p->k_stride,
                    p->v_stride, p->o_stride, p->scale, p->causal, p->dtype, stream, Scratch::Allocated,
-                   static_cast<const uint8_t*>(p->mask), p->mask_stride, d.enabled ? &d : nullptr);
+                   static_cast<const uint8_t*>(p->mask), p->mask_stride, d.enabled ? &d : nullptr, p->block_n,
+                   p->q_tiles);
 }
 
 int fa_backward(const fa_bwd_params* p, cudaStream_t stream) {
@@ -732,7 +742,7 @@ const char* fa_status_string(int status) {
         case FA_ERR_LAUNCH: return "CUDA runtime error (fa_last_cuda_error names the call)";
         case FA_ERR_TIMEOUT: return "a device-side wait exceeded its bound";
         case FA_ERR_SCALE: return "scale must be finite and > 0";
-        case FA_ERR_ARG: return "causal (and deterministic) must be 0 or 1";
+        case FA_ERR_ARG: return "causal or deterministic not 0/1, dropout_p out of range, or an unsupported tiling";
         case FA_ERR_PTR: return "pointer is not device memory of the current device";
         case FA_ERR_STRIDE: return "a stride is not positive, a multiple of 8 elements and below 2^36";
         case FA_ERR_WORKSPACE: return "workspace is NULL, not 256-byte aligned or smaller than fa_bwd_workspace_size";

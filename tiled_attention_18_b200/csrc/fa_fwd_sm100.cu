@@ -117,22 +117,26 @@ constexpr uint32_t COL_S1 = 128;
 constexpr uint32_t COL_O0 = 256;
 constexpr uint32_t COL_O1 = 384;
 
-template <int D>
+// Shared-memory layout for head dimension D, key tiles of BN rows and QT query
+// tiles of BLOCK_M rows per work unit.
+template <int D, int BN = BLOCK_N, int QT = Q_TILES_PER_CTA>
 struct Smem {
     static constexpr int CHUNKS = D / 64;                  // 128-byte swizzle atoms along D
-    static constexpr int CHUNK_BYTES = 128 * 128;          // 128 rows x 128 bytes
-    static constexpr int TILE_BYTES = BLOCK_M * D * 2;     // one Q, K or V tile
+    static constexpr int Q_CHUNK_BYTES = BLOCK_M * 128;    // 128 rows x 128 bytes
+    static constexpr int KV_CHUNK_BYTES = BN * 128;        // BN rows x 128 bytes
+    static constexpr int Q_TILE_BYTES = BLOCK_M * D * 2;   // one Q tile
+    static constexpr int KV_TILE_BYTES = BN * D * 2;       // one K or V tile
     // K/V ring: a stage holds V_{s-1} and K_s, the two tiles that are first
     // needed together (O0 += P0 V_{s-1}; S0 = Q0 K_s^T) and last used
     // together (O1 += P1 V_{s-1}; S1 = Q1 K_s^T), so one wait and one release
     // cover both.  A unit streams N + 1 stages (the first without V, the last
-    // without K).
-    static constexpr int STAGE_BYTES = 2 * TILE_BYTES;
-    static constexpr int NSTAGE = (D == 128) ? 2 : 4;
+    // without K).  The ring holds 128 KiB whatever the tile shape.
+    static constexpr int STAGE_BYTES = 2 * KV_TILE_BYTES;
+    static constexpr int NSTAGE = (128 * 1024) / STAGE_BYTES;
     static constexpr int STAGE_K = 0;                      // offset of K_s in a stage
-    static constexpr int STAGE_V = TILE_BYTES;             // offset of V_{s-1}
+    static constexpr int STAGE_V = KV_TILE_BYTES;          // offset of V_{s-1}
     static constexpr int Q_OFF = 0;
-    static constexpr int KV_OFF = Q_OFF + Q_TILES_PER_CTA * TILE_BYTES;
+    static constexpr int KV_OFF = Q_OFF + QT * Q_TILE_BYTES;
     // per-row values handed from the softmax to the correction warpgroup
     static constexpr int ALPHA_OFF = KV_OFF + NSTAGE * STAGE_BYTES;   // float [2][128]
     // float2 [unit parity][tile][row] = (1/l, lse); double-buffered because a
@@ -215,6 +219,19 @@ __device__ __forceinline__ void tmem_ld128(uint32_t taddr, float* v) {
     for (int i = 0; i < 128; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// 32 lanes x 64 consecutive 32-bit columns (a 64-key score row per thread).
+__device__ __forceinline__ void tmem_ld64(uint32_t taddr, float* v) {
+    uint32_t r[64];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x64.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%64];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]), "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]), "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]), "=r"(r[48]), "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]), "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63])
+        : "r"(taddr)
+        : "memory");
+#pragma unroll
+    for (int i = 0; i < 64; ++i) v[i] = __uint_as_float(r[i]);
+}
+
 // acc + the two bf16 halves of a packed pair, each converted exactly (mixed-precision adds)
 __device__ __forceinline__ float2 add_bf16x2(float2 acc, uint32_t pk) {
     float2 r;
@@ -294,7 +311,9 @@ constexpr int CAUSAL_HEAD_GROUP = 8;
 // Work-unit order: with the causal mask, longest units first (query block
 // descending) within head groups, heads innermost; without it, heads
 // outermost so that CTAs running together share one head's K/V in L2.
+template <int BN, int QT>
 __device__ __forceinline__ Unit decode_unit(const KParams& p, int u) {
+    constexpr int ROWS = QT * BLOCK_M;  // query rows per unit
     Unit U;
     int mb;
     if (p.causal) {
@@ -315,14 +334,14 @@ __device__ __forceinline__ Unit decode_unit(const KParams& p, int u) {
     }
 #pragma unroll
     for (int t = 0; t < 2; ++t) {
-        const int q0 = mb * ROWS_PER_UNIT + t * BLOCK_M;
+        const int q0 = mb * ROWS + t * BLOCK_M;
         U.q0[t] = q0;
         int n = 0;
-        if (q0 < p.Sq) {
-            // diagonal bound: key tile j is visited iff its first key j*BLOCK_N is
+        if (t < QT && q0 < p.Sq) {
+            // diagonal bound: key tile j is visited iff its first key j*BN is
             // not after the last key that the tile's last query row sees,
             // q0 + BLOCK_M - 1 + causal_off
-            n = p.causal ? min((q0 + BLOCK_M - 1 + p.causal_off) / BLOCK_N + 1, p.nkv) : p.nkv;
+            n = p.causal ? min((q0 + BLOCK_M - 1 + p.causal_off) / BN + 1, p.nkv) : p.nkv;
         }
         U.n[t] = n;
     }
@@ -334,12 +353,12 @@ __device__ __forceinline__ Unit decode_unit(const KParams& p, int u) {
 
 // Reads the work-unit indices published by the TMA lane, in order.
 // next() returns the unit, -1 when the CTA has no more work, -2 on abort.
-template <int D>
+template <int D, int BN, int QT>
 struct UnitReader {
     int slot = 0;
     uint32_t phase = 0;
     __device__ __forceinline__ int next(uint8_t* smem, volatile uint32_t* abort_flag, int site) {
-        using L = Smem<D>;
+        using L = Smem<D, BN, QT>;
         const uint32_t bar0 = smem_u32(smem) + L::BAR_OFF;
         if (!mbar_wait(bar0 + 8u * (uint32_t)(L::B_UFULL + slot), phase, abort_flag, site)) return -2;
         const int u = reinterpret_cast<volatile int*>(smem + L::UNIT_OFF)[slot];
@@ -349,9 +368,9 @@ struct UnitReader {
     }
 };
 
-template <int D>
+template <int D, int BN, int QT>
 __device__ void producer_role(const KParams& p, uint8_t* smem, volatile uint32_t* abort_flag) {
-    using L = Smem<D>;
+    using L = Smem<D, BN, QT>;
     const uint32_t base = smem_u32(smem);
     const uint32_t bar0 = base + L::BAR_OFF;
     auto bar = [&](int i) { return bar0 + 8u * (uint32_t)i; };
@@ -380,25 +399,25 @@ __device__ void producer_role(const KParams& p, uint8_t* smem, volatile uint32_t
         mbar_arrive(bar(L::B_UFULL + uslot));
         if (++uslot == L::NUNIT) { uslot = 0; uphase ^= 1u; }
         if (u < 0) break;
-        const Unit U = decode_unit(p, u);
+        const Unit U = decode_unit<BN, QT>(p, u);
         const int ub = U.bh / p.H, uh = U.bh - ub * p.H;  // tensor-map coordinates of the head
         if (!mbar_wait(bar(L::B_QEMPTY), qe_phase ^ 1u, abort_flag, 1)) { ok = false; break; }
         qe_phase ^= 1u;
-        const uint32_t qbytes = (U.n[0] > 0 ? L::TILE_BYTES : 0) + (U.n[1] > 0 ? L::TILE_BYTES : 0);
+        const uint32_t qbytes = (U.n[0] > 0 ? L::Q_TILE_BYTES : 0) + (U.n[1] > 0 ? L::Q_TILE_BYTES : 0);
         mbar_expect_tx(bar(L::B_QFULL), qbytes);
         last_q_fill = (int)(qe_phase ^ 1u);  // parity of the q_full phase this fill completes
 #pragma unroll
         for (int t = 0; t < 2; ++t) {
             if (U.n[t] == 0) continue;
-            const uint32_t dst = base + L::Q_OFF + t * L::TILE_BYTES;
+            const uint32_t dst = base + L::Q_OFF + t * L::Q_TILE_BYTES;
 #pragma unroll
             for (int c = 0; c < L::CHUNKS; ++c)
-                tma_load_4d(dst + c * L::CHUNK_BYTES, &p.tmap_q, bar(L::B_QFULL), c * 64, U.q0[t], uh, ub);
+                tma_load_4d(dst + c * L::Q_CHUNK_BYTES, &p.tmap_q, bar(L::B_QFULL), c * 64, U.q0[t], uh, ub);
         }
         // stages 0..N: stage s = (V_{s-1} if s >= 1, K_s if s < N)
         for (int st = 0; st <= U.N; ++st) {
             if (!mbar_wait(bar(L::B_STEMPTY + stage), phase ^ 1u, abort_flag, 2)) { ok = false; break; }
-            const uint32_t bytes = (st >= 1 ? L::TILE_BYTES : 0) + (st < U.N ? L::TILE_BYTES : 0);
+            const uint32_t bytes = (st >= 1 ? L::KV_TILE_BYTES : 0) + (st < U.N ? L::KV_TILE_BYTES : 0);
             mbar_expect_tx(bar(L::B_STFULL + stage), bytes);
             fill_mask |= 1u << stage;
             fill_parity = (fill_parity & ~(1u << stage)) | (phase << stage);
@@ -406,14 +425,14 @@ __device__ void producer_role(const KParams& p, uint8_t* smem, volatile uint32_t
             if (st < U.N) {
 #pragma unroll
                 for (int c = 0; c < L::CHUNKS; ++c)
-                    tma_load_4d(dst + L::STAGE_K + c * L::CHUNK_BYTES, &p.tmap_k, bar(L::B_STFULL + stage), c * 64,
-                                st * BLOCK_N, uh, ub);
+                    tma_load_4d(dst + L::STAGE_K + c * L::KV_CHUNK_BYTES, &p.tmap_k, bar(L::B_STFULL + stage),
+                                c * 64, st * BN, uh, ub);
             }
             if (st >= 1) {
 #pragma unroll
                 for (int c = 0; c < L::CHUNKS; ++c)
-                    tma_load_4d(dst + L::STAGE_V + c * L::CHUNK_BYTES, &p.tmap_v, bar(L::B_STFULL + stage), c * 64,
-                                (st - 1) * BLOCK_N, uh, ub);
+                    tma_load_4d(dst + L::STAGE_V + c * L::KV_CHUNK_BYTES, &p.tmap_v, bar(L::B_STFULL + stage),
+                                c * 64, (st - 1) * BN, uh, ub);
             }
             if (++stage == L::NSTAGE) { stage = 0; phase ^= 1u; }
         }
@@ -426,16 +445,16 @@ __device__ void producer_role(const KParams& p, uint8_t* smem, volatile uint32_t
     }
 }
 
-template <int D, bool BF16>
+template <int D, bool BF16, int BN, int QT>
 __device__ void mma_role(const KParams& p, uint8_t* smem, uint32_t tmem, volatile uint32_t* abort_flag) {
-    using L = Smem<D>;
+    using L = Smem<D, BN, QT>;
     const uint32_t base = smem_u32(smem);
     const uint32_t bar0 = base + L::BAR_OFF;
     auto bar = [&](int i) { return bar0 + 8u * (uint32_t)i; };
-    constexpr uint32_t IDESC_S = make_idesc(BF16, BLOCK_N, false);
+    constexpr uint32_t IDESC_S = make_idesc(BF16, BN, false);
     constexpr uint32_t IDESC_PV = make_idesc(BF16, D, true);
     constexpr int KSTEPS_S = D / 16;        // QK^T: K = D
-    constexpr int KSTEPS_PV = BLOCK_N / 16; // PV: K = BLOCK_N keys
+    constexpr int KSTEPS_PV = BN / 16;      // PV: K = BN keys
 
     // S_t = Q_t K^T : A = Q tile (K-major), B = K tile (K-major), 128-byte swizzle,
     // 8-row groups 1024 bytes apart; K steps of 16 elements advance 32 bytes
@@ -447,14 +466,14 @@ __device__ void mma_role(const KParams& p, uint8_t* smem, uint32_t tmem, volatil
     // K steps of 16 keys advance 2 KiB.
     // Descriptors are built once; a start address (< 256 KiB, 14 bits after >> 4)
     // plus any offset used here stays inside the low half's field.
-    constexpr uint32_t V_LBO = (D == 128) ? (uint32_t)L::CHUNK_BYTES : 1024u;
+    constexpr uint32_t V_LBO = (D == 128) ? (uint32_t)L::KV_CHUNK_BYTES : 1024u;
     const uint64_t dq = sw128_desc(base + L::Q_OFF, 16, 1024);
     const uint64_t dk = sw128_desc(base + L::KV_OFF, 16, 1024);
     const uint64_t dv = sw128_desc(base + L::KV_OFF, V_LBO, 1024);
     const uint32_t dq_lo = (uint32_t)dq, dq_hi = (uint32_t)(dq >> 32);
     const uint32_t dk_lo = (uint32_t)dk, dk_hi = (uint32_t)(dk >> 32);
     const uint32_t dv_lo = (uint32_t)dv, dv_hi = (uint32_t)(dv >> 32);
-    constexpr uint32_t TILE16 = (uint32_t)L::TILE_BYTES >> 4;
+    constexpr uint32_t TILE16 = (uint32_t)L::Q_TILE_BYTES >> 4;
 
     constexpr uint32_t STAGE16 = (uint32_t)L::STAGE_BYTES >> 4;
     auto issue_s = [&](int t, int st) {
@@ -463,8 +482,9 @@ __device__ void mma_role(const KParams& p, uint8_t* smem, uint32_t tmem, volatil
         const uint32_t d_tmem = tmem + (t == 0 ? COL_S0 : COL_S1);
 #pragma unroll
         for (int ks = 0; ks < KSTEPS_S; ++ks) {
-            const uint32_t off = (uint32_t)(((ks & 3) * 32 + (ks >> 2) * L::CHUNK_BYTES) >> 4);
-            tc_mma_ss2(d_tmem, a_lo + off, dq_hi, b_lo + off, dk_hi, IDESC_S, ks > 0 ? 1u : 0u);
+            const uint32_t a_off = (uint32_t)(((ks & 3) * 32 + (ks >> 2) * L::Q_CHUNK_BYTES) >> 4);
+            const uint32_t b_off = (uint32_t)(((ks & 3) * 32 + (ks >> 2) * L::KV_CHUNK_BYTES) >> 4);
+            tc_mma_ss2(d_tmem, a_lo + a_off, dq_hi, b_lo + b_off, dk_hi, IDESC_S, ks > 0 ? 1u : 0u);
         }
     };
     auto issue_pv = [&](int t, int st, bool accumulate) {
@@ -510,11 +530,11 @@ __device__ void mma_role(const KParams& p, uint8_t* smem, uint32_t tmem, volatil
         if (++stage == L::NSTAGE) { stage = 0; phase ^= 1u; }
         return st;
     };
-    UnitReader<D> units;
+    UnitReader<D, BN, QT> units;
     for (;;) {
         const int u = units.next(smem, abort_flag, 32);
         if (u < 0) break;
-        const Unit U = decode_unit(p, u);
+        const Unit U = decode_unit<BN, QT>(p, u);
         const bool tile1_last = U.n[1] == U.N;  // which tile issues the unit's last S
         if (!mbar_wait(bar(L::B_QFULL), qf_phase, abort_flag, 3)) { ok = false; break; }
         qf_phase ^= 1u;
@@ -565,10 +585,11 @@ __device__ void mma_role(const KParams& p, uint8_t* smem, uint32_t tmem, volatil
     mbar_drain(bar(L::B_FIN), 0u);
 }
 
-template <int D, bool BF16, bool MASK, bool DROP>
+template <int D, bool BF16, bool MASK, bool DROP, int BN, int QT>
 __device__ void softmax_role(const KParams& p, uint8_t* smem, uint32_t tmem, int t, int warp_in_group,
                              volatile uint32_t* abort_flag) {
-    using L = Smem<D>;
+    using L = Smem<D, BN, QT>;
+    static_assert(BN == BLOCK_N || (!MASK && !DROP), "the mask and dropout paths take 128-key tiles");
     const uint32_t base = smem_u32(smem);
     const uint32_t bar0 = base + L::BAR_OFF;
     auto bar = [&](int i) { return bar0 + 8u * (uint32_t)i; };
@@ -583,12 +604,12 @@ __device__ void softmax_role(const KParams& p, uint8_t* smem, uint32_t tmem, int
     const float2 sl2x2 = make_float2(sl2, sl2);
 
     uint32_t s_phase = 0;
-    UnitReader<D> units;
+    UnitReader<D, BN, QT> units;
     for (;;) {
         const int u = units.next(smem, abort_flag, 33);
         if (!__all_sync(0xffffffffu, u != -2)) return;
         if (u < 0) break;
-        const Unit U = decode_unit(p, u);
+        const Unit U = decode_unit<BN, QT>(p, u);
         const int n = U.n[t];
         if (n == 0) continue;
         const int row = U.q0[t] + row_in_tile;
@@ -610,15 +631,15 @@ __device__ void softmax_role(const KParams& p, uint8_t* smem, uint32_t tmem, int
             if (!__all_sync(0xffffffffu, mbar_wait(bar(L::B_SFULL + t), s_phase, abort_flag, 16 + t))) return;
             s_phase ^= 1u;
             tc_fence_after();
-            float s[BLOCK_N];
-            tmem_ld128(ts, s);
-            const int kbase = j * BLOCK_N;
+            float s[BN];
+            if constexpr (BN == 128) tmem_ld128(ts, s); else tmem_ld64(ts, s);
+            const int kbase = j * BN;
             const bool need_mask =
-                (kbase + BLOCK_N > p.Sk) || (p.causal && kbase + BLOCK_N - 1 > U.q0[t] + p.causal_off);
+                (kbase + BN > p.Sk) || (p.causal && kbase + BN - 1 > U.q0[t] + p.causal_off);
             if (need_mask) {
                 const int lim = key_limit - kbase;
 #pragma unroll
-                for (int c = 0; c < BLOCK_N; ++c)
+                for (int c = 0; c < BN; ++c)
                     if (c > lim) s[c] = -INFINITY;
             }
             if constexpr (MASK) {
@@ -629,14 +650,14 @@ __device__ void softmax_role(const KParams& p, uint8_t* smem, uint32_t tmem, int
             float mx0 = max3(s[0], s[1], s[2]), mx1 = max3(s[3], s[4], s[5]);
             float mx2 = max3(s[6], s[7], s[8]), mx3 = max3(s[9], s[10], s[11]);
 #pragma unroll
-            for (int c = 12; c < BLOCK_N - 4; c += 8) {
+            for (int c = 12; c < BN - 4; c += 8) {
                 mx0 = max3(mx0, s[c], s[c + 1]);
                 mx1 = max3(mx1, s[c + 2], s[c + 3]);
                 mx2 = max3(mx2, s[c + 4], s[c + 5]);
                 mx3 = max3(mx3, s[c + 6], s[c + 7]);
             }
-            mx0 = max3(mx0, s[BLOCK_N - 4], s[BLOCK_N - 3]);
-            mx1 = max3(mx1, s[BLOCK_N - 2], s[BLOCK_N - 1]);
+            mx0 = max3(mx0, s[BN - 4], s[BN - 3]);
+            mx1 = max3(mx1, s[BN - 2], s[BN - 1]);
             const float m_blk = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
             bool grow = m_blk > m_use + Policy<BF16>::TAU;
             if constexpr (BF16) grow = grow || (m_blk > m_use && ex2(m_blk - m_use) > RESCALE_KAPPA * lr);
@@ -689,7 +710,7 @@ __device__ void softmax_role(const KParams& p, uint8_t* smem, uint32_t tmem, int
                 tmem_st16(ts + 16 * qr, pk);
             };
 #pragma unroll
-            for (int qr = 0; qr < 4; ++qr) quarter_row(qr);
+            for (int qr = 0; qr < BN / 32; ++qr) quarter_row(qr);
             const float2 ls = __fadd2_rn(lsum0, lsum1);
             l += ls.x + ls.y;
             if constexpr (Policy<BF16>::NORM_BY_ROUNDED_P) {
@@ -715,10 +736,10 @@ __device__ void softmax_role(const KParams& p, uint8_t* smem, uint32_t tmem, int
     }
 }
 
-template <int D, bool BF16>
+template <int D, bool BF16, int BN, int QT>
 __device__ void correction_role(const KParams& p, uint8_t* smem, uint32_t tmem, int warp_in_group,
                                 volatile uint32_t* abort_flag) {
-    using L = Smem<D>;
+    using L = Smem<D, BN, QT>;
     const uint32_t base = smem_u32(smem);
     const uint32_t bar0 = base + L::BAR_OFF;
     auto bar = [&](int i) { return bar0 + 8u * (uint32_t)i; };
@@ -804,12 +825,12 @@ __device__ void correction_role(const KParams& p, uint8_t* smem, uint32_t tmem, 
         return true;
     };
 
-    UnitReader<D> units;
+    UnitReader<D, BN, QT> units;
     for (;;) {
         const int u = units.next(smem, abort_flag, 34);
         if (!__all_sync(0xffffffffu, u != -2)) return;
         if (u < 0) break;
-        const Unit U = decode_unit(p, u);
+        const Unit U = decode_unit<BN, QT>(p, u);
         for (int j = 1; j < U.N; ++j) {
             if (j < U.n[0] && !correct(0)) return;
             if (j < U.n[1] && !correct(1)) return;
@@ -819,9 +840,9 @@ __device__ void correction_role(const KParams& p, uint8_t* smem, uint32_t tmem, 
     }
 }
 
-template <int D, bool BF16, bool MASK, bool DROP>
+template <int D, bool BF16, bool MASK, bool DROP, int BN = BLOCK_N, int QT = Q_TILES_PER_CTA>
 __global__ void __launch_bounds__(NUM_THREADS, 1) fa_fwd_kernel(const __grid_constant__ KParams p) {
-    using L = Smem<D>;
+    using L = Smem<D, BN, QT>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t base = smem_u32(smem);
@@ -863,16 +884,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) fa_fwd_kernel(const __grid_con
 
     if (wg < 2) {
         setmaxnreg_inc<REG_SOFTMAX>();
-        softmax_role<D, BF16, MASK, DROP>(p, smem, tmem, wg, warp & 3, abort_flag);
+        softmax_role<D, BF16, MASK, DROP, BN, QT>(p, smem, tmem, wg, warp & 3, abort_flag);
     } else if (wg == 2) {
         setmaxnreg_dec<REG_CORR>();
-        correction_role<D, BF16>(p, smem, tmem, warp & 3, abort_flag);
+        correction_role<D, BF16, BN, QT>(p, smem, tmem, warp & 3, abort_flag);
     } else {
         setmaxnreg_dec<REG_CTRL>();
         if (warp == WARP_TMA) {
-            if (lane == 0) producer_role<D>(p, smem, abort_flag);
+            if (lane == 0) producer_role<D, BN, QT>(p, smem, abort_flag);
         } else if (warp == WARP_MMA) {
-            if (lane == 0) mma_role<D, BF16>(p, smem, tmem, abort_flag);
+            if (lane == 0) mma_role<D, BF16, BN, QT>(p, smem, tmem, abort_flag);
         }
     }
 
@@ -920,11 +941,11 @@ __global__ void __launch_bounds__(64, 1) selftest_timeout_kernel(long long deadl
     }
 }
 
-template <int D, bool BF16, bool MASK, bool DROP = false>
+template <int D, bool BF16, bool MASK, bool DROP = false, int BN = BLOCK_N, int QT = Q_TILES_PER_CTA>
 cudaError_t launch_impl(const LaunchArgs& a, cudaStream_t stream) {
-    using L = Smem<D>;
+    using L = Smem<D, BN, QT>;
     static_assert(L::ALLOC <= 232448, "shared memory budget exceeded");
-    auto kern = fa_fwd_kernel<D, BF16, MASK, DROP>;
+    auto kern = fa_fwd_kernel<D, BF16, MASK, DROP, BN, QT>;
     cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(kern), L::ALLOC);
     if (e != cudaSuccess) return e;
     KParams p;
@@ -940,9 +961,9 @@ cudaError_t launch_impl(const LaunchArgs& a, cudaStream_t stream) {
     p.H = a.H;
     p.Sq = a.Sq;
     p.Sk = a.Sk;
-    p.n_mblk = (a.Sq + ROWS_PER_UNIT - 1) / ROWS_PER_UNIT;
-    p.n_units = (int)num_units(p.BH, a.Sq);
-    p.nkv = (a.Sk + BLOCK_N - 1) / BLOCK_N;
+    p.n_mblk = (a.Sq + QT * BLOCK_M - 1) / (QT * BLOCK_M);
+    p.n_units = p.BH * p.n_mblk;
+    p.nkv = (a.Sk + BN - 1) / BN;
     p.causal = a.causal;
     p.causal_off = a.Sk - a.Sq;
     p.mask = a.mask;
@@ -968,7 +989,23 @@ cudaError_t launch_impl(const LaunchArgs& a, cudaStream_t stream) {
 
 }  // namespace
 
+// Manual tilings (attention without an explicit mask or dropout): key tiles of
+// 64 or 128 rows, one or two 128-row query tiles per work unit.
+template <int D, bool BF16>
+cudaError_t launch_tiled(const LaunchArgs& a, cudaStream_t stream) {
+    if (a.block_n == 64)
+        return a.q_tiles == 1 ? launch_impl<D, BF16, false, false, 64, 1>(a, stream)
+                              : launch_impl<D, BF16, false, false, 64, 2>(a, stream);
+    return a.q_tiles == 1 ? launch_impl<D, BF16, false, false, 128, 1>(a, stream)
+                          : launch_impl<D, BF16, false, false, 128, 2>(a, stream);
+}
+
 cudaError_t launch_fwd_sm100(const LaunchArgs& a, cudaStream_t stream) {
+    if (a.block_n != BLOCK_N || a.q_tiles != Q_TILES_PER_CTA) {
+        if (a.mask || a.drop.enabled) return cudaErrorInvalidValue;  // rejected by the host layer first
+        if (a.D == 128) return a.dtype == 1 ? launch_tiled<128, true>(a, stream) : launch_tiled<128, false>(a, stream);
+        return a.dtype == 1 ? launch_tiled<64, true>(a, stream) : launch_tiled<64, false>(a, stream);
+    }
     if (a.drop.enabled) {
         if (a.mask) {
             if (a.D == 128)

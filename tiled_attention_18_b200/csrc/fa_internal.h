@@ -55,6 +55,8 @@ struct LaunchArgs {
     float scale_log2;       // scale * log2(e)
     int grid;               // persistent CTAs
     unsigned int* sched;    // zeroed device counter for claimed-unit scheduling, or null
+    int block_n;            // keys per key tile: 128 (default) or 64 (D = 64/128 kernel)
+    int q_tiles;            // 128-row query tiles per work unit: 2 (default) or 1
 };
 
 // Backward pass (fa_bwd): tensor maps as for the forward pass (Q, dO over
@@ -147,9 +149,10 @@ cudaError_t launch_bwd_sm100(const BwdLaunchArgs& a, cudaStream_t stream);
 // Status words of the backward kernels (same protocol as read_and_clear_status).
 cudaError_t read_and_clear_status_bwd(cudaStream_t stream, int* status, int* site);
 
-// Number of work units (b, h, 256-row query block).
-inline int64_t num_units(int64_t BH, int64_t S) {
-    return BH * ((S + ROWS_PER_UNIT - 1) / ROWS_PER_UNIT);
+// Number of work units (b, h, query block of q_tiles x 128 rows).
+inline int64_t num_units(int64_t BH, int64_t S, int q_tiles = Q_TILES_PER_CTA) {
+    const int64_t rows = (int64_t)q_tiles * BLOCK_M;
+    return BH * ((S + rows - 1) / rows);
 }
 
 // Launch the persistent forward kernel on `stream`.  Returns a cudaError_t.
