@@ -60,7 +60,7 @@ typedef enum {
     FA_OK = 0,
     FA_ERR_NULL = -1,     /* a required pointer is NULL */
     FA_ERR_SHAPE = -2,    /* B, H or S negative, or too large for 32-bit indexing */
-    FA_ERR_HEADDIM = -3,  /* D is not 64, 128 or 256 (64 or 128 for the backward entries) */
+    FA_ERR_HEADDIM = -3,  /* D is not 64, 128 or 256 */
     FA_ERR_DTYPE = -4,    /* dtype is not FA_FP16 or FA_BF16 */
     FA_ERR_ALIGN = -5,    /* q, k, v, o not 16-byte aligned, or lse not 4-byte aligned */
     FA_ERR_ARCH = -6,     /* the current device is not compute capability 10.0 (sm_100) */
@@ -234,8 +234,13 @@ FA_API long long fa_bwd_workspace_size(int B, int H, int Sq, int D);
  *              256-byte aligned (else FA_ERR_WORKSPACE); contents on entry do
  *              not matter; used only during the call's kernels on `stream`, so
  *              calls that may overlap on the GPU need separate workspaces.
- * B, H, Sq, Sk, D, scale, causal, dtype: as fa_fwd_ex.  B or H 0 is an empty
- *              problem (FA_OK, nothing launched); Sq = 0 zeroes dK and dV.
+ * B, H, Sq, Sk, D, scale, causal, dtype: as fa_fwd_ex (D = 64, 128 or 256).
+ *              B or H 0 is an empty problem (FA_OK, nothing launched); Sq = 0
+ *              zeroes dK and dV.  D = 256 forms each 128-key tile's gradients
+ *              in two passes, one per half of the head dimension, each
+ *              recomputing the full-width scores (the pages name 64, 128 and 256
+ *              as the common head dimensions: "FlashAttention-2 在昇腾 NPU 上
+ *              如何做到 3 倍加速？", section 3.2).
  * deterministic: 0 = dQ is accumulated in fp32 across key tiles with atomic
  *              adds (fastest; its last bits may differ between runs); 1 = the
  *              key tiles of a head add their dQ parts in key-tile order (the
@@ -280,7 +285,7 @@ FA_API int fa_bwd_ex(const void* q, const void* k, const void* v, const void* o,
  * over b, h and the query row, 0 broadcasting over b or h; all multiples of 16,
  * row stride >= Sk; 16-byte aligned).  Masked (query, key) pairs contribute no
  * gradient; rows that saw no key (LSE = -inf) get dQ = 0.  o and lse must come
- * from fa_fwd_mask with the same mask.  D = 64 or 128; other arguments, modes
+ * from fa_fwd_mask with the same mask.  D = 64, 128 or 256; other arguments, modes
  * and errors as fa_bwd.
  */
 FA_API int fa_bwd_mask(const void* q, const void* k, const void* v, const void* o, const void* dout,
@@ -322,7 +327,7 @@ FA_API int fa_fwd_dropout(const void* q, const void* k, const void* v, void* o, 
  * with the same dropout_p, seed and offset the kernel regenerates the same
  * keep decisions, and dV_j = sum_i P_ij z_ij dO_i, dP_ij = z_ij dO_i . v_j,
  * dS_ij = P_ij (dP_ij - dO_i . O_i).  o and lse must come from fa_fwd_dropout
- * with the same arguments.  D = 64 or 128; other arguments, modes and errors
+ * with the same arguments.  D = 64, 128 or 256; other arguments, modes and errors
  * as fa_bwd; dropout_p as fa_fwd_dropout.
  */
 FA_API int fa_bwd_dropout(const void* q, const void* k, const void* v, const void* o, const void* dout,
@@ -338,7 +343,7 @@ FA_API int fa_bwd_dropout(const void* q, const void* k, const void* v, const voi
  * The fields mean what the arguments of the same names mean for fa_fwd_ex,
  * fa_fwd_mask and fa_fwd_dropout (fa_bwd_ex, fa_bwd_mask, fa_bwd_dropout):
  * a NULL stride array is contiguous, a NULL mask is no mask, dropout_p = 0 is
- * no dropout.  fa_forward takes D = 64, 128 or 256, fa_backward 64 or 128
+ * no dropout.  fa_forward and fa_backward take D = 64, 128 or 256
  * (with or without a mask and dropout).  The caller owns the
  * struct (read during the call only) and everything it points to.  Errors:
  * FA_ERR_NULL for a NULL params pointer, else those of the separate entries.

@@ -157,13 +157,17 @@ def test_bwd_workspace_size(lib):
     rows = up(B * H * 384 * 4)
     flags = up(B * H * 5 * 4 * 4)
     assert fa.fa_bwd_workspace_size(B, H, S, D) == acc + 2 * rows + flags + 256
+    # D = 256: twice the dQ accumulator and a turn counter per half of the head dimension
+    acc = up(B * H * S * 256 * 4)
+    flags = up(B * H * 5 * 2 * 4 * 4)
+    assert fa.fa_bwd_workspace_size(B, H, S, 256) == acc + 2 * rows + flags + 256
 
 
 @pytest.mark.parametrize("args,code", [
     (dict(Sq=-1), _lib.FA_ERR_SHAPE),
     (dict(Sk=0), _lib.FA_ERR_SHAPE),
     (dict(Sq=300, Sk=200, causal=1), _lib.FA_ERR_SHAPE),
-    (dict(D=256), _lib.FA_ERR_HEADDIM),
+    (dict(D=512), _lib.FA_ERR_HEADDIM),
     (dict(dtype=3), _lib.FA_ERR_DTYPE),
     (dict(scale=math.nan), _lib.FA_ERR_SCALE),
     (dict(causal=5), _lib.FA_ERR_ARG),
@@ -235,7 +239,7 @@ def test_dropout_entries_reject_bad_arguments(lib):
     bargs = lambda p, D=128: (A,) * 10 + (1 << 20, 1, 1, 128, 128, D, 0.1, 0, p, 1, 0, 0, 1, 0)  # noqa: E731
     for p in (-0.5, float("nan"), 1.0):
         assert fa.fa_bwd_dropout(*bargs(p)) == _lib.FA_ERR_ARG, p
-    assert fa.fa_bwd_dropout(*bargs(0.1, D=256)) == _lib.FA_ERR_HEADDIM
+    assert fa.fa_bwd_dropout(*bargs(0.1, D=512)) == _lib.FA_ERR_HEADDIM
     assert ok  # the shapes above are otherwise valid
 
 
@@ -306,7 +310,7 @@ def test_unified_entries_reject_bad_arguments(lib):
     bb = dict(q=A, k=A, v=A, o=A, dout=A, lse=A, dq=A, dk=A, dv=A, workspace=A, workspace_bytes=1 << 30, B=1, H=1,
               Sq=128, Sk=128, D=128, scale=0.1, causal=0, deterministic=0, dtype=1)
     assert fa.fa_backward(0, **bb, dropout_p=float("nan")) == _lib.FA_ERR_ARG
-    assert fa.fa_backward(0, **{**bb, "D": 256}) == _lib.FA_ERR_HEADDIM
+    assert fa.fa_backward(0, **{**bb, "D": 512}) == _lib.FA_ERR_HEADDIM
     assert fa.fa_backward(0, **{**bb, "B": 2, "H": 2}, dq_stride=(64, 0, 64)) == _lib.FA_ERR_STRIDE
 
 

@@ -445,7 +445,7 @@ int fa_fwd_noalloc(const void* q, const void* k, const void* v, void* o, float* 
 
 long long fa_bwd_workspace_size(int B, int H, int Sq, int D) {
     if (B < 0 || H < 0 || Sq < 0) return FA_ERR_SHAPE;
-    if (D != 64 && D != 128) return FA_ERR_HEADDIM;
+    if (D != 64 && D != 128 && D != 256) return FA_ERR_HEADDIM;
     if (B == 0 || H == 0 || Sq == 0) return 0;
     return (long long)fa::bwd_workspace_layout((int64_t)B * H, Sq, D).total;
 }
@@ -460,7 +460,7 @@ int backward(const void* q, const void* k, const void* v, const void* o, const v
              const long long* mask_stride, const fa::DropoutArgs* drop = nullptr,
              const long long* const* strides = nullptr) {
     if (B < 0 || H < 0 || Sq < 0 || Sk < 0) return FA_ERR_SHAPE;
-    if (D != 64 && D != 128) return FA_ERR_HEADDIM;
+    if (D != 64 && D != 128 && D != 256) return FA_ERR_HEADDIM;
     if (dtype != FA_FP16 && dtype != FA_BF16) return FA_ERR_DTYPE;
     if (!(std::isfinite(scale) && scale > 0.f)) return FA_ERR_SCALE;
     if (causal != 0 && causal != 1) return FA_ERR_ARG;
@@ -521,8 +521,8 @@ int backward(const void* q, const void* k, const void* v, const void* o, const v
     }
     fa::BwdLaunchArgs a;
     std::memset(&a, 0, sizeof(a));
-    // the D = 128 backward kernel steps through 64 query rows at a time
-    const int q_box = (D == 128) ? 64 : fa::BLOCK_M;
+    // the D = 128 and 256 backward kernel steps through 64 query rows at a time
+    const int q_box = (D >= 128) ? 64 : fa::BLOCK_M;
     if (!encode_tensor(&a.tmap_q, q, B, H, Sq, D, st[0], dtype, q_box) ||
         !encode_tensor(&a.tmap_do, dout, B, H, Sq, D, st[4], dtype, q_box) ||
         !encode_tensor(&a.tmap_k, k, B, H, Sk, D, st[1], dtype) ||
@@ -563,7 +563,8 @@ int backward(const void* q, const void* k, const void* v, const void* o, const v
     a.dtype = dtype;
     a.causal = causal;
     a.scale = scale;
-    const int64_t units = BH * ((Sk + 127) / 128);
+    // D = 256: a unit is (head, key tile, half of the head dimension)
+    const int64_t units = BH * ((Sk + 127) / 128) * (D == 256 ? 2 : 1);
     a.grid = (int)(units < dev.sms ? units : dev.sms);
     const cudaError_t le = fa::launch_bwd_sm100(a, stream);
     if (le != cudaSuccess) return cuda_fail(le, "launch(backward kernels)");
@@ -735,7 +736,7 @@ const char* fa_status_string(int status) {
         case FA_OK: return "ok";
         case FA_ERR_NULL: return "a required pointer is NULL";
         case FA_ERR_SHAPE: return "invalid B, H, Sq or Sk (or causal with Sq > Sk)";
-        case FA_ERR_HEADDIM: return "head dimension must be 64, 128 or 256 (64 or 128 for fa_fwd_mask and fa_bwd)";
+        case FA_ERR_HEADDIM: return "head dimension must be 64, 128 or 256";
         case FA_ERR_DTYPE: return "dtype must be FA_FP16 or FA_BF16";
         case FA_ERR_ALIGN: return "q, k, v, o must be 16-byte aligned and lse 4-byte aligned";
         case FA_ERR_ARCH: return "the current device is not sm_100 (B200)";

@@ -23,7 +23,7 @@
 //   2. the fused kernel: one persistent CTA per SM; a work unit is (b, h,
 //      128-key tile).  The CTA keeps K_n, V_n in shared memory and dK, dV in
 //      tensor memory and walks the query rows that see its keys (D = 64,
-//      fa_bwd_kernel: 128-row steps; D = 128, fa_bwd_kernel_d128: 64-row steps
+//      fa_bwd_kernel: 128-row steps; D = 128 and 256, fa_bwd_kernel_wide: 64-row steps
 //      with double-buffered scores, see below):
 //        S^T = K Q_m^T, dP^T = V dO_m^T   (tcgen05.mma, fp32 in TMEM)
 //        P^T, dS^T                          (one key row per thread, packed to
@@ -62,7 +62,7 @@ constexpr uint32_t UNIT_READERS_BWD = 1 + 2 * TILE;  // MMA lane + two warpgroup
 
 // Tensor-memory columns of fa_bwd_kernel (D = 64): S^T/P^T, dP^T/dS^T, the dV
 // and dK accumulators and dQ of one step (the template also fits D = 128 by
-// putting dQ_m in the dP^T columns, but D = 128 runs fa_bwd_kernel_d128).
+// putting dQ_m in the dP^T columns, but D = 128 runs fa_bwd_kernel_wide).
 constexpr uint32_t COL_S = 0;
 constexpr uint32_t COL_DP = 128;
 constexpr uint32_t COL_DV = 256;
@@ -147,6 +147,7 @@ struct BUnit {
     int n;      // key tile
     int m_lo;   // first query tile that sees a key of the tile
     int T;      // query tiles visited
+    int half;   // D = 256: the 128-wide half of the head dimension whose dK, dV, dQ this unit forms
 };
 
 // Units: with the causal mask the number of query tiles falls with the key
@@ -744,7 +745,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) fa_bwd_kernel(const __grid_con
 }
 
 // ------------------------------------------------------------------------
-// D = 128: 64-row query steps with double-buffered S^T / dP^T.
+// D = 128 and 256: 64-row query steps with double-buffered S^T / dP^T.
 //
 // Tensor memory: S0 [0,64) dP0 [64,128) S1 [128,192) dP1 [192,256), dV
 // [256,384), dK [384,512).  While the dS warpgroup turns step g's S^T, dP^T
@@ -756,6 +757,14 @@ __global__ void __launch_bounds__(BWD_THREADS, 1) fa_bwd_kernel(const __grid_con
 // no wait; only its dP^T waits for that buffer's dQ^T read-out, and the S^T
 // MMAs issued before it cover that latency.  Q and dO stream through three 32 KiB stages.  Every role
 // derives buffer, stage and barrier parities from the global step count g.
+//
+// D = 256: dK and dV of a 128-key tile would fill the 512 tensor-memory columns
+// by themselves, so a work unit is (head, key tile, half of D): it computes
+// the full-D scores S^T = K Q^T and dP^T = V dO^T (16 K steps), then dK, dV and
+// dQ for its 128-wide half only, in the same column layout as D = 128; the
+// two halves of a key tile are two units (S^T and dP^T are formed twice: 1.4x
+// the MMA work of one pass).  K and V (64 KiB each) stay in shared memory, so
+// one 64 KiB Q/dO stage is all that fits.
 constexpr int QM = 64;  // query rows per step
 // 16 warps: warpgroup 0 = TMA lane (warp 0) and MMA lane (warp 1); warpgroups 1
 // and 3 = the dS work of query columns [0, 32) and [32, 64) of each step (two
@@ -765,18 +774,25 @@ constexpr int BWD2_THREADS = 512;
 constexpr uint32_t UNIT_READERS_BWD2 = 1 + 3 * TILE;
 // Register split (launch: 128 per thread): control 64, dS 176 each, output 96;
 // per SM sub-partition one warp of each warpgroup: 64 + 176 + 96 + 176 = 512.
-constexpr int REG2_CTRL = 64;
-constexpr int REG2_DS = 176;
-constexpr int REG2_OUT = 96;
-static_assert(REG2_CTRL + 2 * REG2_DS + REG2_OUT <= 4 * 128, "register split exceeds the launch budget");
+// D = 256 moves 8 registers from each dS warp to the output warp (its dQ and
+// dK/dV addresses depend on the unit's half of the head dimension).
+template <int D>
+struct Reg2 {
+    static constexpr int CTRL = 64;
+    static constexpr int DS = (D == 128) ? 176 : 168;
+    static constexpr int OUT = (D == 128) ? 96 : 112;
+    static_assert(CTRL + 2 * DS + OUT <= 4 * 128, "register split exceeds the launch budget");
+};
 
+template <int D>
 struct Bwd2Smem {
-    static constexpr int D = 128;
+    static constexpr int CHUNKS = D / 64;            // 64-column chunks of a row
+    static constexpr int HALVES = D / 128;           // passes over the head dimension per key tile
     static constexpr int KCHUNK = TILE * 128;        // K/V: [128 rows][64 cols] per chunk
     static constexpr int QCHUNK = QM * 128;          // Q/dO: [64 rows][64 cols] per chunk
-    static constexpr int KV_TILE = TILE * D * 2;     // 32 KiB
-    static constexpr int Q_TILE = QM * D * 2;        // 16 KiB
-    static constexpr int NSTAGE = 3;
+    static constexpr int KV_TILE = TILE * D * 2;     // 32 KiB (D = 128), 64 KiB (D = 256)
+    static constexpr int Q_TILE = QM * D * 2;        // 16 KiB, 32 KiB
+    static constexpr int NSTAGE = (D == 128) ? 3 : 1;
     static constexpr int K_OFF = 0;
     static constexpr int V_OFF = KV_TILE;
     static constexpr int STAGE_OFF = 2 * KV_TILE;    // stage: Q_m, dO_m
@@ -814,9 +830,14 @@ constexpr uint32_t COL2_DK = 384;
 __device__ __forceinline__ uint32_t col2_s(uint32_t b) { return 128u * b; }
 __device__ __forceinline__ uint32_t col2_dp(uint32_t b) { return 128u * b + 64u; }
 
-// Units for 64-row steps: m_lo counts steps.
+// Units for 64-row steps: m_lo counts steps; with D = 256 the two halves of a
+// key tile are consecutive units.
+template <int D>
 __device__ __forceinline__ BUnit decode_bwd2_unit(const BwdParams& p, int u) {
     BUnit U;
+    constexpr int HALVES = Bwd2Smem<D>::HALVES;
+    U.half = u % HALVES;
+    u /= HALVES;
     if (p.causal) {
         causal_unit_order(p, u, &U.bh, &U.n);
         const int q_first = U.n * TILE - p.causal_off;
@@ -830,11 +851,12 @@ __device__ __forceinline__ BUnit decode_bwd2_unit(const BwdParams& p, int u) {
     return U;
 }
 
+template <int D>
 struct Bwd2UnitReader {
     int slot = 0;
     uint32_t phase = 0;
     __device__ __forceinline__ int next(uint8_t* smem, volatile uint32_t* abort_flag, int site) {
-        using L = Bwd2Smem;
+        using L = Bwd2Smem<D>;
         const uint32_t bar0 = smem_u32(smem) + L::BAR_OFF;
         if (!mbar_wait(bar0 + 8u * (uint32_t)(L::B_UFULL + slot), phase, abort_flag, site)) return -2;
         const int u = reinterpret_cast<volatile int*>(smem + L::UNIT_OFF)[slot];
@@ -844,8 +866,9 @@ struct Bwd2UnitReader {
     }
 };
 
+template <int D>
 __device__ void bwd2_producer(const BwdParams& p, uint8_t* smem, volatile uint32_t* abort_flag) {
-    using L = Bwd2Smem;
+    using L = Bwd2Smem<D>;
     const uint32_t base = smem_u32(smem);
     const uint32_t bar0 = base + L::BAR_OFF;
     auto bar = [&](int i) { return bar0 + 8u * (uint32_t)i; };
@@ -865,7 +888,7 @@ __device__ void bwd2_producer(const BwdParams& p, uint8_t* smem, volatile uint32
         mbar_arrive(bar(L::B_UFULL + uslot));
         if (++uslot == 2) { uslot = 0; uphase ^= 1u; }
         if (u < 0) break;
-        const BUnit U = decode_bwd2_unit(p, u);
+        const BUnit U = decode_bwd2_unit<D>(p, u);
         const int b = U.bh / p.H, h = U.bh - b * p.H;
         const uint32_t kvp = (uint32_t)nunit & 1u;
         if (!mbar_wait(bar(L::B_KVEMPTY), kvp ^ 1u, abort_flag, 61)) { ok = false; break; }
@@ -873,7 +896,7 @@ __device__ void bwd2_producer(const BwdParams& p, uint8_t* smem, volatile uint32
         kv_fill = (int)kvp;
         ++nunit;
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
+        for (int c = 0; c < L::CHUNKS; ++c) {
             tma_load_4d(base + L::K_OFF + c * L::KCHUNK, &p.tmap_k, bar(L::B_KVFULL), c * 64, U.n * TILE, h, b);
             tma_load_4d(base + L::V_OFF + c * L::KCHUNK, &p.tmap_v, bar(L::B_KVFULL), c * 64, U.n * TILE, h, b);
         }
@@ -887,7 +910,7 @@ __device__ void bwd2_producer(const BwdParams& p, uint8_t* smem, volatile uint32
             fill_parity = (fill_parity & ~(1u << st)) | (sp << st);
             const uint32_t dst = base + L::STAGE_OFF + st * L::STAGE_BYTES;
 #pragma unroll
-            for (int c = 0; c < 2; ++c) {
+            for (int c = 0; c < L::CHUNKS; ++c) {
                 tma_load_4d(dst + c * L::QCHUNK, &p.tmap_q, bar(L::B_QFULL + st), c * 64, m * QM, h, b);
                 tma_load_4d(dst + L::Q_TILE + c * L::QCHUNK, &p.tmap_do, bar(L::B_QFULL + st), c * 64, m * QM, h, b);
             }
@@ -905,9 +928,9 @@ __device__ void bwd2_producer(const BwdParams& p, uint8_t* smem, volatile uint32
     }
 }
 
-template <bool BF16>
+template <int D, bool BF16>
 __device__ void bwd2_mma(const BwdParams& p, uint8_t* smem, uint32_t tmem, volatile uint32_t* abort_flag) {
-    using L = Bwd2Smem;
+    using L = Bwd2Smem<D>;
     const uint32_t base = smem_u32(smem);
     const uint32_t bar0 = base + L::BAR_OFF;
     auto bar = [&](int i) { return bar0 + 8u * (uint32_t)i; };
@@ -934,7 +957,7 @@ __device__ void bwd2_mma(const BwdParams& p, uint8_t* smem, uint32_t tmem, volat
     // S^T or dP^T of one step: A = K or V (128 keys), B = Q or dO (64 queries), K = D
     auto issue_sp = [&](uint32_t d_tmem, uint64_t a, uint32_t b_off16) {
 #pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
+        for (int ks = 0; ks < D / 16; ++ks) {
             const uint32_t in_chunk = (uint32_t)((ks & 3) * 32) >> 4;
             const uint32_t a_off = in_chunk + (uint32_t)(((ks >> 2) * L::KCHUNK) >> 4);
             const uint32_t b_off = in_chunk + (uint32_t)(((ks >> 2) * L::QCHUNK) >> 4);
@@ -946,11 +969,15 @@ __device__ void bwd2_mma(const BwdParams& p, uint8_t* smem, uint32_t tmem, volat
     // packed pairs of queries [32c, 32c + 32) sit in columns 32c .. 32c + 15 of
     // the buffer (each dS warpgroup packs into its own columns), so the K step
     // of queries 16 ks .. 16 ks + 15 reads columns 32 (ks / 2) + 8 (ks % 2).
+    // (D = 256: B is the unit's 128-wide half of dO or Q, chunks 2 half and 2 half + 1)
+    constexpr bool SPLIT = L::HALVES > 1;
+    uint32_t half_q16 = 0, half_k16 = 0;
     auto issue_kv = [&](uint32_t d_tmem, uint32_t a_tmem, uint32_t b_off16, bool accumulate) {
 #pragma unroll
         for (int ks = 0; ks < QM / 16; ++ks)
             tc_mma_ts2(d_tmem, a_tmem + (uint32_t)((ks >> 1) * 32 + (ks & 1) * 8),
-                       lo(b_stage_mn) + b_off16 + (uint32_t)(ks * (2048 >> 4)), hi(b_stage_mn), IDESC_KV,
+                       lo(b_stage_mn) + (SPLIT ? half_q16 : 0u) + b_off16 + (uint32_t)(ks * (2048 >> 4)), hi(b_stage_mn),
+                       IDESC_KV,
                        (accumulate || ks > 0) ? 1u : 0u);
     };
     auto wait_p = [&](uint32_t bar_idx, uint32_t parity, int site) -> bool {
@@ -960,13 +987,17 @@ __device__ void bwd2_mma(const BwdParams& p, uint8_t* smem, uint32_t tmem, volat
     uint32_t g = 0;
     int nunit = 0;
     bool ok = true;
-    Bwd2UnitReader units;
+    Bwd2UnitReader<D> units;
     for (;;) {
         const int u = units.next(smem, abort_flag, 63);
         if (u < 0) break;
-        const BUnit U = decode_bwd2_unit(p, u);
+        const BUnit U = decode_bwd2_unit<D>(p, u);
         const uint32_t kvp = (uint32_t)nunit & 1u;
         ++nunit;
+        if constexpr (SPLIT) {
+            half_q16 = (uint32_t)(U.half * 2 * L::QCHUNK) >> 4;
+            half_k16 = (uint32_t)(U.half * 2 * L::KCHUNK) >> 4;
+        }
         if (!wait_p(L::B_KVFULL, kvp, 64)) { ok = false; break; }
         // step g's S^T and dP^T into buffer g & 1
         auto issue_step = [&](uint32_t gs) -> bool {
@@ -986,7 +1017,10 @@ __device__ void bwd2_mma(const BwdParams& p, uint8_t* smem, uint32_t tmem, volat
         for (int t = 0; t < U.T; ++t, ++g) {
             const uint32_t b = g & 1u;
             const int st = (int)(g % L::NSTAGE);
-            if (t + 1 < U.T && !issue_step(g + 1)) { ok = false; break; }
+            // the next step's scores run while this step's dS is formed; with a single
+            // Q/dO stage (D = 256) the next step's Q and dO can only load once this
+            // step's dK and dV products have released the stage, so they come later
+            if (L::NSTAGE > 1 && t + 1 < U.T && !issue_step(g + 1)) { ok = false; break; }
             if (!wait_p(L::B_PFULL + b, (g >> 1) & 1u, 67)) { ok = false; break; }
             tc_fence_after();
             if (t == 0) {
@@ -1001,11 +1035,12 @@ __device__ void bwd2_mma(const BwdParams& p, uint8_t* smem, uint32_t tmem, volat
 #pragma unroll
             for (int ks = 0; ks < TILE / 16; ++ks) {
                 const uint32_t off = (uint32_t)(ks * (2048 >> 4));
-                tc_mma_ss2(tmem + col2_dp(b), lo(a_kt) + off, hi(a_kt), lo(b_ds) + b * DS16 + off, hi(b_ds), IDESC_DQ,
-                           ks > 0 ? 1u : 0u);
+                tc_mma_ss2(tmem + col2_dp(b), lo(a_kt) + (SPLIT ? half_k16 : 0u) + off, hi(a_kt),
+                           lo(b_ds) + b * DS16 + off, hi(b_ds), IDESC_DQ, ks > 0 ? 1u : 0u);
             }
             tc_commit(bar(L::B_DQFULL + b));
             tc_commit(bar(L::B_DSEMPTY + b));
+            if (L::NSTAGE == 1 && t + 1 < U.T && !issue_step(g + 1)) { ok = false; break; }
         }
         if (!ok) break;
         tc_commit(bar(L::B_DKVFULL));
@@ -1016,10 +1051,10 @@ __device__ void bwd2_mma(const BwdParams& p, uint8_t* smem, uint32_t tmem, volat
     mbar_drain(bar(L::B_FIN), 0u);
 }
 
-template <bool BF16, bool MASK, bool DROP>
+template <int D, bool BF16, bool MASK, bool DROP>
 __device__ void bwd2_ds_role(const BwdParams& p, uint8_t* smem, uint32_t tmem, int warp_in_group, int c,
                              volatile uint32_t* abort_flag) {
-    using L = Bwd2Smem;
+    using L = Bwd2Smem<D>;
     const uint32_t base = smem_u32(smem);
     const uint32_t bar0 = base + L::BAR_OFF;
     auto bar = [&](int i) { return bar0 + 8u * (uint32_t)i; };
@@ -1029,12 +1064,12 @@ __device__ void bwd2_ds_role(const BwdParams& p, uint8_t* smem, uint32_t tmem, i
     const float sl2 = p.scale_log2;
     const int sw = row & 7;
     uint32_t g = 0;
-    Bwd2UnitReader units;
+    Bwd2UnitReader<D> units;
     for (;;) {
         const int u = units.next(smem, abort_flag, 69);
         if (!__all_sync(0xffffffffu, u != -2)) return;
         if (u < 0) break;
-        const BUnit U = decode_bwd2_unit(p, u);
+        const BUnit U = decode_bwd2_unit<D>(p, u);
         const int key = U.n * TILE + row;
         const bool key_ok = key < p.Sk;
         const int q_min = p.causal ? key - p.causal_off : 0;
@@ -1109,10 +1144,10 @@ __device__ void bwd2_ds_role(const BwdParams& p, uint8_t* smem, uint32_t tmem, i
     }
 }
 
-template <bool BF16>
+template <int D, bool BF16>
 __device__ void bwd2_out_role(const BwdParams& p, uint8_t* smem, uint32_t tmem, int warp_in_group,
                               volatile uint32_t* abort_flag) {
-    using L = Bwd2Smem;
+    using L = Bwd2Smem<D>;
     const uint32_t base = smem_u32(smem);
     const uint32_t bar0 = base + L::BAR_OFF;
     auto bar = [&](int i) { return bar0 + 8u * (uint32_t)i; };
@@ -1121,12 +1156,13 @@ __device__ void bwd2_out_role(const BwdParams& p, uint8_t* smem, uint32_t tmem, 
     const uint32_t lane_sel = (uint32_t)(warp_in_group * 32) << 16;
     uint32_t g = 0;
     int nunit = 0;
-    Bwd2UnitReader units;
+    Bwd2UnitReader<D> units;
     for (;;) {
         const int u = units.next(smem, abort_flag, 73);
         if (!__all_sync(0xffffffffu, u != -2)) return;
         if (u < 0) break;
-        const BUnit U = decode_bwd2_unit(p, u);
+        const BUnit U = decode_bwd2_unit<D>(p, u);
+        const int half = (L::HALVES > 1) ? U.half : 0;  // a constant 0 with one pass
         const uint32_t kvp = (uint32_t)nunit & 1u;
         ++nunit;
         for (int t = 0; t < U.T; ++t, ++g) {
@@ -1135,7 +1171,7 @@ __device__ void bwd2_out_role(const BwdParams& p, uint8_t* smem, uint32_t tmem, 
             if (!__all_sync(0xffffffffu, mbar_wait(bar(L::B_DQFULL + b), (g >> 1) & 1u, abort_flag, 74))) return;
             tc_fence_after();
             // dQ[q][d] += dQ^T[d][q]: consecutive threads take consecutive d (coalesced)
-            float* dst = p.dq_acc + ((size_t)U.bh * (size_t)p.Sq + (size_t)m * QM) * 128 + row;
+            float* dst = p.dq_acc + ((size_t)U.bh * (size_t)p.Sq + (size_t)m * QM) * D + (size_t)half * 128 + row;
             const int nq = min(QM, p.Sq - m * QM);
             if (!p.dq_flags) {
                 // read the whole step, free the columns, then add with atomics
@@ -1146,14 +1182,14 @@ __device__ void bwd2_out_role(const BwdParams& p, uint8_t* smem, uint32_t tmem, 
                 mbar_arrive(bar(L::B_DQEMPTY + b));
 #pragma unroll
                 for (int j = 0; j < 32; ++j)
-                    if (j < nq) atomicAdd(dst + (size_t)j * 128, __uint_as_float(r0[j]));
+                    if (j < nq) atomicAdd(dst + (size_t)j * D, __uint_as_float(r0[j]));
 #pragma unroll
                 for (int j = 0; j < 32; ++j)
-                    if (32 + j < nq) atomicAdd(dst + (size_t)(32 + j) * 128, __uint_as_float(r1[j]));
+                    if (32 + j < nq) atomicAdd(dst + (size_t)(32 + j) * D, __uint_as_float(r1[j]));
             } else {
                 // this key tile's turn for the step, then 32 queries at a time:
                 // read-modify-write in batches of 16 (loads in flight together)
-                int* flag = p.dq_flags + ((size_t)U.bh * p.flag_steps + m) * 4 + warp_in_group;
+                int* flag = p.dq_flags + (((size_t)U.bh * p.flag_steps + m) * L::HALVES + half) * 4 + warp_in_group;
                 if (!wait_turn(flag, U.n, abort_flag, 57)) return;
 #pragma unroll 1
                 for (int hh = 0; hh < 2; ++hh) {
@@ -1169,12 +1205,12 @@ __device__ void bwd2_out_role(const BwdParams& p, uint8_t* smem, uint32_t tmem, 
 #pragma unroll
                         for (int j = 0; j < 16; ++j) {
                             const int jq = 32 * hh + 16 * h + j;
-                            v[j] = jq < nq ? __ldcg(dst + (size_t)jq * 128) : 0.f;
+                            v[j] = jq < nq ? __ldcg(dst + (size_t)jq * D) : 0.f;
                         }
 #pragma unroll
                         for (int j = 0; j < 16; ++j) {
                             const int jq = 32 * hh + 16 * h + j;
-                            if (jq < nq) __stcg(dst + (size_t)jq * 128, v[j] + __uint_as_float(r[16 * h + j]));
+                            if (jq < nq) __stcg(dst + (size_t)jq * D, v[j] + __uint_as_float(r[16 * h + j]));
                         }
                     }
                 }
@@ -1187,8 +1223,9 @@ __device__ void bwd2_out_role(const BwdParams& p, uint8_t* smem, uint32_t tmem, 
         const bool valid = key < p.Sk;
         const int ub = U.bh / p.H, uh = U.bh - ub * p.H;
         const long long kr = valid ? key : 0;
-        uint8_t* dv_row = p.dv + ub * p.dv_s[0] + uh * p.dv_s[1] + kr * p.dv_s[2];
-        uint8_t* dk_row = p.dk + ub * p.dk_s[0] + uh * p.dk_s[1] + kr * p.dk_s[2];
+        // this unit's 128 columns of the dK and dV rows (its half of D at D = 256)
+        uint8_t* dv_row = p.dv + ub * p.dv_s[0] + uh * p.dv_s[1] + kr * p.dv_s[2] + half * 256;
+        uint8_t* dk_row = p.dk + ub * p.dk_s[0] + uh * p.dk_s[1] + kr * p.dk_s[2] + half * 256;
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
             uint32_t r[32];
@@ -1216,9 +1253,9 @@ __device__ void bwd2_out_role(const BwdParams& p, uint8_t* smem, uint32_t tmem, 
     }
 }
 
-template <bool BF16, bool MASK, bool DROP>
-__global__ void __launch_bounds__(BWD2_THREADS, 1) fa_bwd_kernel_d128(const __grid_constant__ BwdParams p) {
-    using L = Bwd2Smem;
+template <int D, bool BF16, bool MASK, bool DROP>
+__global__ void __launch_bounds__(BWD2_THREADS, 1) fa_bwd_kernel_wide(const __grid_constant__ BwdParams p) {
+    using L = Bwd2Smem<D>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t base = smem_u32(smem);
@@ -1256,15 +1293,15 @@ __global__ void __launch_bounds__(BWD2_THREADS, 1) fa_bwd_kernel_d128(const __gr
     tc_fence_after();
     const uint32_t tmem = misc[0];
     if (wg == 0) {
-        setmaxnreg_dec<REG2_CTRL>();
-        if (warp == BW_TMA && lane == 0) bwd2_producer(p, smem, abort_flag);
-        if (warp == BW_MMA && lane == 0) bwd2_mma<BF16>(p, smem, tmem, abort_flag);
+        setmaxnreg_dec<Reg2<D>::CTRL>();
+        if (warp == BW_TMA && lane == 0) bwd2_producer<D>(p, smem, abort_flag);
+        if (warp == BW_MMA && lane == 0) bwd2_mma<D, BF16>(p, smem, tmem, abort_flag);
     } else if (wg == 1 || wg == 3) {
-        setmaxnreg_inc<REG2_DS>();
-        bwd2_ds_role<BF16, MASK, DROP>(p, smem, tmem, warp & 3, wg == 1 ? 0 : 1, abort_flag);
+        setmaxnreg_inc<Reg2<D>::DS>();
+        bwd2_ds_role<D, BF16, MASK, DROP>(p, smem, tmem, warp & 3, wg == 1 ? 0 : 1, abort_flag);
     } else {
-        setmaxnreg_dec<REG2_OUT>();
-        bwd2_out_role<BF16>(p, smem, tmem, warp & 3, abort_flag);
+        setmaxnreg_dec<Reg2<D>::OUT>();
+        bwd2_out_role<D, BF16>(p, smem, tmem, warp & 3, abort_flag);
     }
     tc_fence_before();
     __syncthreads();
@@ -1344,7 +1381,8 @@ __global__ void __launch_bounds__(256) bwd_post_kernel(const float4* __restrict_
 template <int D, bool BF16>
 cudaError_t launch_bwd_impl(const BwdLaunchArgs& a, cudaStream_t stream) {
     static_assert(BwdSmem<64>::ALLOC <= 232448, "shared memory budget exceeded");
-    static_assert(Bwd2Smem::ALLOC <= 232448, "shared memory budget exceeded");
+    static_assert(Bwd2Smem<128>::ALLOC <= 232448, "shared memory budget exceeded");
+    static_assert(Bwd2Smem<256>::ALLOC <= 232448, "shared memory budget exceeded");
     const int BH = a.B * a.H;
     const int n_mtiles = (a.Sq + TILE - 1) / TILE;
     const int Sq_pad = n_mtiles * TILE;
@@ -1358,14 +1396,17 @@ cudaError_t launch_bwd_impl(const BwdLaunchArgs& a, cudaStream_t stream) {
         if (e != cudaSuccess) return e;
     }
     {
-        // D = 128 runs the 64-row-step kernel (its Q/dO maps have 64-row boxes)
+        // D = 128 and 256 run the 64-row-step kernel (its Q/dO maps have 64-row boxes)
+        constexpr bool WIDE = D >= 128;
+        constexpr int DW = WIDE ? D : 128;
         void (*kern)(const BwdParams);
-        if constexpr (D == 128)
+        if constexpr (WIDE)
             kern = a.drop.enabled
-                       ? (a.mask ? fa_bwd_kernel_d128<BF16, true, true> : fa_bwd_kernel_d128<BF16, false, true>)
-                       : (a.mask ? fa_bwd_kernel_d128<BF16, true, false> : fa_bwd_kernel_d128<BF16, false, false>);
+                       ? (a.mask ? fa_bwd_kernel_wide<DW, BF16, true, true> : fa_bwd_kernel_wide<DW, BF16, false, true>)
+                       : (a.mask ? fa_bwd_kernel_wide<DW, BF16, true, false>
+                                 : fa_bwd_kernel_wide<DW, BF16, false, false>);
         else kern = fa_bwd_kernel<D, BF16>;
-        const int alloc = (D == 128) ? Bwd2Smem::ALLOC : BwdSmem<64>::ALLOC;
+        const int alloc = WIDE ? Bwd2Smem<DW>::ALLOC : BwdSmem<64>::ALLOC;
         cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(kern), alloc);
         if (e != cudaSuccess) return e;
         BwdParams p;
@@ -1387,9 +1428,9 @@ cudaError_t launch_bwd_impl(const BwdLaunchArgs& a, cudaStream_t stream) {
         p.Sq = a.Sq;
         p.Sk = a.Sk;
         p.Sq_pad = Sq_pad;
-        p.n_mtiles = (D == 128) ? (a.Sq + QM - 1) / QM : n_mtiles;
+        p.n_mtiles = WIDE ? (a.Sq + QM - 1) / QM : n_mtiles;
         p.n_ktiles = (a.Sk + TILE - 1) / TILE;
-        p.n_units = BH * p.n_ktiles;
+        p.n_units = BH * p.n_ktiles * (WIDE ? Bwd2Smem<DW>::HALVES : 1);
         p.causal = a.causal;
         p.causal_off = a.Sk - a.Sq;
         {
@@ -1414,10 +1455,10 @@ cudaError_t launch_bwd_impl(const BwdLaunchArgs& a, cudaStream_t stream) {
         p.seed_hi = a.drop.seed_hi;
         p.drop_offset = a.drop.offset;
         p.keep_scale = a.drop.enabled ? a.drop.keep_scale : 1.f;
-        p.flag_steps = (D == 128) ? (a.Sq + QM - 1) / QM : n_mtiles;
+        p.flag_steps = WIDE ? (a.Sq + QM - 1) / QM : n_mtiles;
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3((unsigned)a.grid, 1, 1);
-        cfg.blockDim = dim3(D == 128 ? BWD2_THREADS : BWD_THREADS, 1, 1);
+        cfg.blockDim = dim3(WIDE ? BWD2_THREADS : BWD_THREADS, 1, 1);
         cfg.dynamicSmemBytes = alloc;
         cfg.stream = stream;
         e = cudaLaunchKernelEx(&cfg, kern, p);
@@ -1435,6 +1476,9 @@ cudaError_t launch_bwd_impl(const BwdLaunchArgs& a, cudaStream_t stream) {
 }  // namespace
 
 cudaError_t launch_bwd_sm100(const BwdLaunchArgs& a, cudaStream_t stream) {
+    if (a.D == 256) {
+        return a.dtype == 1 ? launch_bwd_impl<256, true>(a, stream) : launch_bwd_impl<256, false>(a, stream);
+    }
     if (a.D == 128) {
         return a.dtype == 1 ? launch_bwd_impl<128, true>(a, stream) : launch_bwd_impl<128, false>(a, stream);
     }

@@ -107,7 +107,7 @@ inline BwdWorkspace bwd_workspace_layout(int64_t BH, int64_t Sq, int64_t D) {
     w.lse2 = up(BH * Sq * D * 4);
     w.delta = w.lse2 + up(BH * Sq_pad * 4);
     w.flags = w.delta + up(BH * Sq_pad * 4);
-    w.flags_bytes = BH * ((Sq + 63) / 64) * 4 * 4;  // [BH][64-row steps][4 warps] int
+    w.flags_bytes = BH * ((Sq + 63) / 64) * (D == 256 ? 2 : 1) * 4 * 4;  // [BH][64-row steps][D/128 halves][4 warps] int
     w.sched = w.flags + up(w.flags_bytes);
     w.total = w.sched + 256;
     return w;
