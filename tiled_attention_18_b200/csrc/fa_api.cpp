@@ -536,6 +536,20 @@ int backward(const void* q, const void* k, const void* v, const void* o, const v
         a.dv_stride[i] = st[7][i];
     }
     uint8_t* w = static_cast<uint8_t*>(workspace);
+    // the fp32 dQ accumulator as a 3-D tensor [B*H][Sq][D] for the TMA engine's
+    // bulk reduce-add (D = 128): boxes of 64 rows x 128 values, rows past Sq clipped
+    if (D == 128) {
+        EncodeTiledFn enc = encoder();
+        if (!enc) return cuda_fail(cudaErrorNotSupported, "cuTensorMapEncodeTiled entry point");
+        const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)Sq, (cuuint64_t)BH};
+        const cuuint64_t strides[2] = {(cuuint64_t)D * 4, (cuuint64_t)Sq * D * 4};
+        const cuuint32_t box[3] = {128, 64, 1};
+        const cuuint32_t elem[3] = {1, 1, 1};
+        const CUresult r = enc(&a.tmap_dq, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, w + ws.dq_acc, dims, strides, box, elem,
+                               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                               CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (r != CUDA_SUCCESS) return cuda_fail((int)r, "cuTensorMapEncodeTiled (dQ accumulator)");
+    }
     a.o = o;
     a.dout = dout;
     a.lse = lse;

@@ -120,6 +120,7 @@ struct BwdParams {
     CUtensorMap tmap_k;
     CUtensorMap tmap_v;
     CUtensorMap tmap_do;
+    CUtensorMap tmap_dq;  // fp32 dQ accumulator [BH][Sq][D], box {128, 64, 1} (bulk reduce-add)
     const float* lse2;    // [BH][Sq_pad] LSE * log2(e), +inf on padded rows
     const float* delta;   // [BH][Sq_pad] rowsum(dO * O), 0 on padded rows
     float* dq_acc;        // [BH][Sq][D] fp32, zeroed by the prep kernel
@@ -196,6 +197,21 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_
                  "l"(src), "r"(bytes), "r"(bar)
                  : "memory");
 }
+
+// TMA bulk reduce-add of a shared-memory box into a 3-D fp32 tensor (rows past
+// the tensor's extent are clipped), tracked by this thread's bulk groups.
+__device__ __forceinline__ void tma_reduce_add_3d(const CUtensorMap* map, uint32_t src, int c0, int c1, int c2) {
+    asm volatile(
+        "cp.reduce.async.bulk.tensor.3d.global.shared::cta.add.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+            reinterpret_cast<uint64_t>(map)),
+        "r"(src), "r"(c0), "r"(c1), "r"(c2)
+        : "memory");
+    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// Wait until this thread's bulk groups have read their shared-memory sources
+// (`read`) or completed.
+__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 __device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
     asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
@@ -801,7 +817,13 @@ struct Bwd2Smem {
     static constexpr int DS_BYTES = TILE * QM * 2;                 // 16 KiB
     static constexpr int STATS_OFF = DS_OFF + 2 * DS_BYTES;          // per stage: lse2[64], delta[64]
     static constexpr int STATS_BYTES = 2 * QM * 4;
-    static constexpr int BAR_OFF = STATS_OFF + NSTAGE * STATS_BYTES;
+    // D = 128, atomic mode: a step's dQ (64 queries x 128 fp32, row-major) staged
+    // for one bulk reduce-add by the TMA engine; it does not fit beside D = 256's
+    // K and V, which keep per-element atomics
+    static constexpr bool DQ_BULK = (D == 128);
+    static constexpr int DQS_OFF = STATS_OFF + NSTAGE * STATS_BYTES;  // 128-byte aligned
+    static constexpr int DQS_BYTES = DQ_BULK ? QM * 128 * 4 : 0;
+    static constexpr int BAR_OFF = DQS_OFF + DQS_BYTES;
     enum {
         B_KVFULL = 0,
         B_KVEMPTY,
@@ -817,7 +839,8 @@ struct Bwd2Smem {
         B_DSEMPTY = B_DQEMPTY + 2,  // [2]
         B_QFULL = B_DSEMPTY + 2,    // [NSTAGE]
         B_QEMPTY = B_QFULL + NSTAGE,
-        NBAR = B_QEMPTY + NSTAGE
+        B_DQSYNC = B_QEMPTY + NSTAGE,  // the output warpgroup's own barrier (dQ staging)
+        NBAR = B_DQSYNC + 1
     };
     static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
     static constexpr int UNIT_OFF = MISC_OFF + 16;
@@ -1154,6 +1177,14 @@ __device__ void bwd2_out_role(const BwdParams& p, uint8_t* smem, uint32_t tmem, 
     const int lane = threadIdx.x & 31;
     const int row = warp_in_group * 32 + lane;  // head-dimension index for dQ^T, key row for dK/dV
     const uint32_t lane_sel = (uint32_t)(warp_in_group * 32) << 16;
+    // barrier of the 128 output threads around the dQ staging (bounded waits)
+    uint32_t sync_phase = 0;
+    auto group_sync = [&](int site) -> bool {
+        mbar_arrive(bar(L::B_DQSYNC));
+        const bool ok = mbar_wait(bar(L::B_DQSYNC), sync_phase, abort_flag, site);
+        sync_phase ^= 1u;
+        return ok;
+    };
     uint32_t g = 0;
     int nunit = 0;
     Bwd2UnitReader<D> units;
@@ -1173,7 +1204,29 @@ __device__ void bwd2_out_role(const BwdParams& p, uint8_t* smem, uint32_t tmem, 
             // dQ[q][d] += dQ^T[d][q]: consecutive threads take consecutive d (coalesced)
             float* dst = p.dq_acc + ((size_t)U.bh * (size_t)p.Sq + (size_t)m * QM) * D + (size_t)half * 128 + row;
             const int nq = min(QM, p.Sq - m * QM);
-            if (!p.dq_flags) {
+            if (!p.dq_flags && L::DQ_BULK) {
+                // once the previous step's reduce has read the staging, copy dQ^T
+                // out of TMEM as dQ[q][d] (each lane holds one d over the 64
+                // queries: a warp writes 32 consecutive floats per query), free
+                // the columns, and let one thread hand the box to the TMA engine as
+                // a bulk reduce-add (rows past Sq are clipped)
+                const bool issuer = threadIdx.x == 2 * 128;  // first thread of the output warpgroup
+                if (issuer) bulk_wait_read();
+                if (!__all_sync(0xffffffffu, group_sync(76))) return;
+                float* stg = reinterpret_cast<float*>(smem + L::DQS_OFF) + row;
+#pragma unroll 1
+                for (int hh = 0; hh < 2; ++hh) {
+                    uint32_t r[32];
+                    tmem_ld32u(tmem + lane_sel + col2_dp(b) + 32 * hh, r);
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) stg[(32 * hh + j) * 128] = __uint_as_float(r[j]);
+                }
+                tc_fence_before();
+                mbar_arrive(bar(L::B_DQEMPTY + b));
+                fence_async_smem();
+                if (!__all_sync(0xffffffffu, group_sync(77))) return;
+                if (issuer) tma_reduce_add_3d(&p.tmap_dq, base + L::DQS_OFF, half * 128, m * QM, U.bh);
+            } else if (!p.dq_flags) {
                 // read the whole step, free the columns, then add with atomics
                 uint32_t r0[32], r1[32];
                 tmem_ld32u(tmem + lane_sel + col2_dp(b), r0);
@@ -1267,7 +1320,8 @@ __global__ void __launch_bounds__(BWD2_THREADS, 1) fa_bwd_kernel_wide(const __gr
     if (threadIdx.x == 0) {
         for (int i = 0; i < L::NBAR; ++i) {
             uint32_t count = 1;
-            if ((i >= L::B_DQEMPTY && i < L::B_DQEMPTY + 2) || i == L::B_DKVEMPTY) count = TILE;  // one warpgroup
+            if ((i >= L::B_DQEMPTY && i < L::B_DQEMPTY + 2) || i == L::B_DKVEMPTY || i == L::B_DQSYNC)
+                count = TILE;  // one warpgroup
             if (i >= L::B_PFULL && i < L::B_PFULL + 2) count = 2 * TILE;  // both dS warpgroups
             if (i >= L::B_UEMPTY && i < L::B_UEMPTY + 2) count = UNIT_READERS_BWD2;
             mbar_init(base + L::BAR_OFF + 8 * i, count);
@@ -1302,6 +1356,8 @@ __global__ void __launch_bounds__(BWD2_THREADS, 1) fa_bwd_kernel_wide(const __gr
     } else {
         setmaxnreg_dec<Reg2<D>::OUT>();
         bwd2_out_role<D, BF16>(p, smem, tmem, warp & 3, abort_flag);
+        // the bulk dQ reductions this thread issued finish before the CTA exits
+        if (threadIdx.x == 2 * 128) bulk_wait_all();
     }
     tc_fence_before();
     __syncthreads();
@@ -1414,6 +1470,7 @@ cudaError_t launch_bwd_impl(const BwdLaunchArgs& a, cudaStream_t stream) {
         p.tmap_k = a.tmap_k;
         p.tmap_v = a.tmap_v;
         p.tmap_do = a.tmap_do;
+        p.tmap_dq = a.tmap_dq;
         p.lse2 = a.lse2;
         p.delta = a.delta;
         p.dq_acc = a.dq_acc;

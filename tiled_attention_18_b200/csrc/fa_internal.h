@@ -67,6 +67,7 @@ struct BwdLaunchArgs {
     CUtensorMap tmap_k;
     CUtensorMap tmap_v;
     CUtensorMap tmap_do;
+    CUtensorMap tmap_dq;    // fp32 dQ accumulator [BH][Sq][D], box {128, 64, 1}, for bulk reduce-add
     const void* o;          // [B,H,Sq,D] 16-bit at o_stride
     const void* dout;       // [B,H,Sq,D] 16-bit at do_stride
     // element strides over b, h and the row (d contiguous) of O, dO and the gradients
