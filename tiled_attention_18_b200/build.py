@@ -4,7 +4,8 @@
 
 The library holds the C ABI of include/fa.h (host code in csrc/fa_api.cpp)
 and the sm_100a kernels (csrc/fa_fwd_sm100.cu forward for D = 64/128,
-csrc/fa_fwd_d256_sm100.cu forward for D = 256, csrc/fa_bwd_sm100.cu backward,
+csrc/fa_fwd_d256_sm100.cu forward for D = 256,
+csrc/fa_fwd_short_sm100.cu forward for key sets of at most 128 keys, csrc/fa_bwd_sm100.cu backward,
 with the shared device helpers of csrc/sm100_helpers.cuh).  It links the CUDA runtime
 statically and reaches cuTensorMapEncodeTiled through the runtime's driver
 entry-point query, so it needs no libcuda at link time.
@@ -23,7 +24,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libfa.so")
 SOURCES = [os.path.join(CSRC, "fa_fwd_sm100.cu"), os.path.join(CSRC, "fa_fwd_d256_sm100.cu"),
-           os.path.join(CSRC, "fa_bwd_sm100.cu"), os.path.join(CSRC, "fa_merge_sm100.cu"),
+           os.path.join(CSRC, "fa_fwd_short_sm100.cu"), os.path.join(CSRC, "fa_bwd_sm100.cu"), os.path.join(CSRC, "fa_merge_sm100.cu"),
            os.path.join(CSRC, "fa_api.cpp")]
 HEADERS = [os.path.join(CSRC, "fa_internal.h"), os.path.join(CSRC, "sm100_helpers.cuh"),
            os.path.join(INCLUDE, "fa.h")]

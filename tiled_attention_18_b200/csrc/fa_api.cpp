@@ -300,6 +300,7 @@ int forward(const void* q, const void* k, const void* v, void* o, float* lse, in
     // tiling: 0 = automatic (128-key tiles, two 128-row query tiles per unit);
     // manual tilings for D = 64/128 without an explicit mask or dropout
     if ((block_n != 0 && block_n != 64 && block_n != 128) || (q_tiles < 0 || q_tiles > 2)) return FA_ERR_ARG;
+    const bool auto_tiling = block_n == 0 && q_tiles == 0;
     if (block_n == 0) block_n = fa::BLOCK_N;
     if (q_tiles == 0) q_tiles = fa::Q_TILES_PER_CTA;
     const bool manual = block_n != fa::BLOCK_N || q_tiles != fa::Q_TILES_PER_CTA;
@@ -342,18 +343,24 @@ int forward(const void* q, const void* k, const void* v, void* o, float* lse, in
         rc = check_device_pointer(p, cur);
         if (rc != FA_OK) return rc;
     }
-    const int64_t units = (D == 256) ? fa::num_units_d256(BH, Sq) : fa::num_units(BH, Sq, q_tiles);
+    // every key of a head in one tile: the short-key kernel (query tiles of 128
+    // rows, keys and values loaded once per head), with automatic tiling
+    const bool short_keys = auto_tiling && D != 256 && !mask && !(drop && drop->enabled) && Sk <= fa::SHORT_SK_MAX;
+    const int64_t units = short_keys ? BH * ((Sq + fa::BLOCK_M - 1) / fa::BLOCK_M)
+                          : (D == 256) ? fa::num_units_d256(BH, Sq) : fa::num_units(BH, Sq, q_tiles);
     const int grid = (int)(units < dev.sms ? units : dev.sms);
     // fa_fwd_noalloc's counter is read back as an int: the claims of all CTAs must fit
-    if (scratch == Scratch::Static && units + grid > fa::NOALLOC_MAX_CLAIMS) return FA_ERR_SHAPE;
+    if (scratch == Scratch::Static && !short_keys && units + grid > fa::NOALLOC_MAX_CLAIMS) return FA_ERR_SHAPE;
 
     fa::LaunchArgs a;
     std::memset(&a, 0, sizeof(a));
-    // the D = 256 kernel streams keys and values in 64-row tiles
-    const int kv_box = (D == 256) ? 64 : block_n;
+    // the D = 256 kernel streams keys and values in 64-row tiles; the short-key
+    // kernel loads all Sk keys of a head at once (rounded up to 16 rows)
+    const int kv_box = short_keys ? (Sk + 15) / 16 * 16 : (D == 256) ? 64 : block_n;
     if (!encode_tensor(&a.tmap_q, q, B, H, Sq, D, qs, dtype) ||
         !encode_tensor(&a.tmap_k, k, B, H, Sk, D, ks, dtype, kv_box) ||
-        !encode_tensor(&a.tmap_v, v, B, H, Sk, D, vs, dtype, kv_box))
+        !encode_tensor(&a.tmap_v, v, B, H, Sk, D, vs, dtype, kv_box) ||
+        (short_keys && !encode_tensor(&a.tmap_o, o, B, H, Sq, D, os, dtype)))
         return FA_ERR_LAUNCH;
     a.o = o;
     a.lse = lse;
@@ -374,7 +381,7 @@ int forward(const void* q, const void* k, const void* v, void* o, float* lse, in
     a.block_n = block_n;
     a.q_tiles = q_tiles;
     std::unique_lock<std::mutex> launch_lock(g_launch_mu, std::defer_lock);
-    if (causal) {
+    if (causal && !short_keys) {
         // units differ in length under the mask: CTAs claim them from a counter
         launch_lock.lock();
         unsigned int* ctr = nullptr;
@@ -389,6 +396,11 @@ int forward(const void* q, const void* k, const void* v, void* o, float* lse, in
         const cudaError_t e = cudaMemsetAsync(ctr, 0, sizeof(unsigned int), stream);
         if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(scheduler counter)");
         a.sched = ctr;
+    }
+    if (short_keys) {
+        const cudaError_t le = fa::launch_fwd_short_sm100(a, stream);
+        if (le != cudaSuccess) return cuda_fail(le, "launch(fa_fwd_kernel_short)");
+        return FA_OK;
     }
     const cudaError_t le = (D == 256) ? fa::launch_fwd_d256_sm100(a, stream) : fa::launch_fwd_sm100(a, stream);
     if (le != cudaSuccess) return cuda_fail(le, D == 256 ? "launch(fa_fwd_kernel_d256)" : "launch(fa_fwd_kernel)");
@@ -714,12 +726,13 @@ int fa_accumulate(float* acc, const void* x, long long n, int dtype, cudaStream_
 
 int fa_check_status(cudaStream_t stream) {
     // one status word per kernel translation unit; all are read and cleared
-    int st[3] = {0, 0, 0}, site[3] = {0, 0, 0};
+    int st[4] = {0, 0, 0, 0}, site[4] = {0, 0, 0, 0};
     cudaError_t e = fa::read_and_clear_status(stream, &st[0], &site[0]);
     if (e == cudaSuccess) e = fa::read_and_clear_status_bwd(stream, &st[1], &site[1]);
     if (e == cudaSuccess) e = fa::read_and_clear_status_d256(stream, &st[2], &site[2]);
+    if (e == cudaSuccess) e = fa::read_and_clear_status_short(stream, &st[3], &site[3]);
     if (e != cudaSuccess) return cuda_fail(e, "fa_check_status (stream synchronize / status word copy)");
-    for (int i = 0; i < 3; ++i) {
+    for (int i = 0; i < 4; ++i) {
         if (st[i] != fa::DEV_OK) {
             t_last_site = site[i];
             return FA_ERR_TIMEOUT;

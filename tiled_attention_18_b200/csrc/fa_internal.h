@@ -16,6 +16,9 @@ constexpr int BLOCK_M = 128;
 constexpr int BLOCK_N = 128;
 constexpr int Q_TILES_PER_CTA = 2;
 constexpr int ROWS_PER_UNIT = BLOCK_M * Q_TILES_PER_CTA;
+// Short key sets (at most one key tile per head) take the short-key kernel
+// when the tiling is automatic and there is no explicit mask or dropout.
+constexpr int SHORT_SK_MAX = 128;
 
 // Device-side status codes written to the status word by the kernel.
 constexpr int DEV_OK = 0;
@@ -39,6 +42,7 @@ struct LaunchArgs {
     CUtensorMap tmap_q;     // 4-D maps over [B][H][S][D] (innermost first: D, S, H, B) with
     CUtensorMap tmap_k;     // the tensors' own strides, box {64, 128, 1, 1}, 128-byte swizzle
     CUtensorMap tmap_v;
+    CUtensorMap tmap_o;     // short-key kernel only: the output, box {64, 128, 1, 1}
     void* o;                // [B,H,Sq,D] 16-bit at o_stride
     float* lse;             // [B,H,Sq] fp32, contiguous
     long long o_stride[3];  // element strides of O over b, h, s (d is contiguous)
@@ -164,6 +168,12 @@ cudaError_t launch_fwd_sm100(const LaunchArgs& a, cudaStream_t stream);
 cudaError_t launch_fwd_d256_sm100(const LaunchArgs& a, cudaStream_t stream);
 int64_t num_units_d256(int64_t BH, int64_t Sq);
 cudaError_t read_and_clear_status_d256(cudaStream_t stream, int* status, int* site);
+
+// Launch the short-key forward kernel (Sk <= SHORT_SK_MAX, D = 64/128, no mask
+// or dropout; K/V maps with a box of Sk rounded up to 16 rows, tmap_o set).
+cudaError_t launch_fwd_short_sm100(const LaunchArgs& a, cudaStream_t stream);
+// Status word of the short-key kernel's translation unit.
+cudaError_t read_and_clear_status_short(cudaStream_t stream, int* status, int* site);
 
 // fa_fwd_noalloc: size of its static scratch array (256 bytes; word 0 is the
 // causal unit counter) and the largest number of unit claims the counter
