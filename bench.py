@@ -64,8 +64,11 @@ FALLBACK_BF16_TFLOPS = 1590.0
 FALLBACK_HBM_GBS = 6650.0
 DROPOUT_SEED = 0x5EED5EED5EED
 PEAKS_PATH = os.path.join(ROOT, "MEASURED_PEAKS.json")
-TRAFFIC_PATH = os.path.join(ROOT, "profiles", "fa_fwd_traffic.json")
-KERNEL_SRC = os.path.join(ROOT, "tiled_attention_18_b200", "csrc", "fa_fwd_sm100.cu")
+# committed DRAM captures (one workload each), matched by workload and by the
+# hash of the kernel sources they were taken on
+TRAFFIC_PATHS = [os.path.join(ROOT, "profiles", name) for name in ("fa_fwd_traffic.json", "fa_fwd_short_traffic.json")]
+CSRC = os.path.join(ROOT, "tiled_attention_18_b200", "csrc")
+KERNEL_SRC = os.path.join(CSRC, "fa_fwd_sm100.cu")
 L2_BYTES = 126 * 1024 * 1024
 ALL_WORKLOADS = {**WORKLOADS, **GENERAL_WORKLOADS}
 
@@ -97,26 +100,30 @@ def peak_tflops():
         return FALLBACK_BF16_TFLOPS, "fallback (1.59 PFLOP/s, an earlier cuBLAS bf16 measurement on B200)"
 
 
-def kernel_source_hash() -> str:
-    """Hash of the forward kernel's sources (its file and the shared device helpers)."""
+def kernel_source_hash(kernel_file: str = "fa_fwd_sm100.cu") -> str:
+    """Hash of a forward kernel's sources (its file and the shared device helpers)."""
     import hashlib
     h = hashlib.sha256()
-    for path in (KERNEL_SRC, os.path.join(os.path.dirname(KERNEL_SRC), "sm100_helpers.cuh")):
+    for path in (os.path.join(CSRC, kernel_file), os.path.join(CSRC, "sm100_helpers.cuh")):
         with open(path, "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
 
 
 def traffic_per_launch(workload: str):
-    """DRAM bytes per step from the committed ncu summary, if taken on this kernel source and workload."""
-    try:
-        with open(TRAFFIC_PATH) as f:
-            t = json.load(f)
-        if t.get("kernel_source_sha256_16") != kernel_source_hash() or t.get("workload_key", "c5") != workload:
-            return None
-        return float(t["dram_bytes_per_step"])
-    except Exception:
-        return None
+    """DRAM bytes per step from a committed ncu summary, if taken on this kernel source and workload."""
+    for path in TRAFFIC_PATHS:
+        try:
+            with open(path) as f:
+                t = json.load(f)
+            if t.get("workload_key", "c5") != workload:
+                continue
+            if t.get("kernel_source_sha256_16") != kernel_source_hash(t.get("kernel_file", "fa_fwd_sm100.cu")):
+                return None
+            return float(t["dram_bytes_per_step"])
+        except Exception:
+            continue
+    return None
 
 
 class ClockSampler:
@@ -693,6 +700,11 @@ def main(argv=None) -> int:
                     help="forward keys per key tile (0 = automatic, 128); through fa_forward")
     ap.add_argument("--q-tiles", type=int, default=0, choices=[0, 1, 2],
                     help="forward 128-row query tiles per work unit (0 = automatic, 2); through fa_forward")
+    ap.add_argument("--graph", action="store_true",
+                    help="forward: capture each run's STEPS launches (inputs rotated as usual) in one CUDA graph and "
+                         "time its replay, so that the per-launch host cost (argument checks, tensor maps, "
+                         "cudaLaunchKernelEx) leaves the device timeline; for kernels shorter than that host cost. "
+                         "Per-launch times are the graph's time / STEPS")
     ap.add_argument("--deterministic", action="store_true",
                     help="with --pass bwd: the deterministic dQ mode (key tiles add in order)")
     args = ap.parse_args(argv)
@@ -768,7 +780,7 @@ def main(argv=None) -> int:
                 jj = torch.arange(pad, device=dev)[None, :]
                 tril[i] = ((jj <= ii + (w.Skv - w.S)) & (jj < w.Skv)).to(torch.uint8).contiguous()
 
-    def launch(i, step=0):
+    def launch(i, step=0, sid=sid):
         w = runs[i]
         q, k, v = (view(w, t) for t in dev_in[i][step % n_copies[i]])
         o, lse = dev_out[i]
@@ -811,6 +823,25 @@ def main(argv=None) -> int:
     if st != 0:
         raise fa.FaError(st, "warm-up")
 
+    # --graph: each run's STEPS launches captured in one graph, replayed on the timing stream
+    graphs = None
+    if args.graph:
+        if args.dropout > 0.0:
+            raise SystemExit("--graph takes runs without dropout (the offset changes per step)")
+        cap = torch.cuda.Stream(dev)
+        cap.wait_stream(stream)
+        graphs = []
+        for i in range(len(runs)):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=cap):
+                for s_ in range(args.steps):
+                    launch(i, s_, cap.cuda_stream)
+            graphs.append(g)
+        stream.wait_stream(cap)
+        for g in graphs:
+            g.replay()
+        torch.cuda.synchronize(dev)
+
     # timed region: per-launch events on the launching stream
     ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in runs]
           for _ in range(args.steps)]
@@ -821,11 +852,17 @@ def main(argv=None) -> int:
     barrier()
     torch.cuda.synchronize(dev)
     start.record(stream)
-    for s in range(args.steps):
+    if graphs is not None:
         for i in range(len(runs)):
-            ev[s][i][0].record(stream)
-            launch(i, s)
-            ev[s][i][1].record(stream)
+            ev[0][i][0].record(stream)
+            graphs[i].replay()
+            ev[0][i][1].record(stream)
+    else:
+        for s in range(args.steps):
+            for i in range(len(runs)):
+                ev[s][i][0].record(stream)
+                launch(i, s)
+                ev[s][i][1].record(stream)
     stop.record(stream)
     torch.cuda.synchronize(dev)
     barrier()
@@ -834,7 +871,10 @@ def main(argv=None) -> int:
     if st != 0:
         raise fa.FaError(st, "timed region")
     elapsed_ms = start.elapsed_time(stop)
-    kern_ms = np.array([[a.elapsed_time(b) for (a, b) in row] for row in ev])  # [steps, runs]
+    if graphs is not None:
+        kern_ms = np.array([[a.elapsed_time(b) / args.steps for (a, b) in ev[0]]] * args.steps)
+    else:
+        kern_ms = np.array([[a.elapsed_time(b) for (a, b) in row] for row in ev])  # [steps, runs]
     max_ms = max_over_ranks(elapsed_ms, device=dev)
     step_flops = sum(w.flops for w in runs)
     value = job_throughput(step_flops, args.steps, world, max_ms)
@@ -855,6 +895,11 @@ def main(argv=None) -> int:
     n_units = sum(fa.fa_num_units(w.B, w.H, w.S) for w in runs if not w.general)
     bound = "latency" if (not runs[0].general and n_units < torch.cuda.get_device_properties(dev).multi_processor_count
                           ) else "tensor"
+    # short key sets (Sk <= 128, automatic tiling, no mask or dropout) take the
+    # short-key kernel: one score tile per query tile, bound by moving Q in and O out
+    if (all(w.Skv <= 128 and w.D != 256 for w in runs) and not tril and args.dropout == 0.0
+            and not args.block_n and not args.q_tiles):
+        bound = "hbm"
 
     # the 13B-style layer (S = 8192, causal, Q,K x2) timed beside the default step
     extra_runs = []
@@ -921,13 +966,22 @@ def main(argv=None) -> int:
                        "runs_per_step": len(runs),
                        "l2": ("inputs larger than L2 (no flush)" if max(n_copies) == 1 else
                               f"inputs rotated over {max(n_copies)} device copies (> 2x L2 per rotation, no flush)"),
-                       "parallelism": f"independent batch per GPU x{world}"},
+                       "parallelism": f"independent batch per GPU x{world}",
+                       "timing": ("each run's launches replayed from one CUDA graph (host launch cost off the device "
+                                  "timeline; per-launch time = graph time / steps)"
+                                  if graphs is not None else "each launch through the C ABI, events around each")},
             "pct_of_peak": 100.0 * value / (peak * world),
-            "roofline": {"bound": bound, "achieved": achieved, "peak": peak, "unit": UNIT,
-                         "frac": achieved / peak, "traffic": traffic, "peak_source": peak_src,
-                         "per_run": per_run,
-                         "hbm": {"algorithmic_bytes_per_step": step_bytes, "achieved": hbm_achieved, "peak": hbm,
-                                 "unit": "GB/s", "frac": hbm_achieved / hbm, "peak_source": hbm_src}},
+            "roofline": ({"bound": bound, "achieved": achieved, "peak": peak, "unit": UNIT,
+                          "frac": achieved / peak, "traffic": traffic, "peak_source": peak_src,
+                          "per_run": per_run,
+                          "hbm": {"algorithmic_bytes_per_step": step_bytes, "achieved": hbm_achieved, "peak": hbm,
+                                  "unit": "GB/s", "frac": hbm_achieved / hbm, "peak_source": hbm_src}}
+                         if bound != "hbm" else
+                         {"bound": "hbm", "achieved": hbm_achieved, "peak": hbm, "unit": "GB/s",
+                          "frac": hbm_achieved / hbm, "traffic": traffic, "peak_source": hbm_src,
+                          "algorithmic_bytes_per_step": step_bytes, "per_run": per_run,
+                          "tensor": {"achieved": achieved, "peak": peak, "unit": UNIT, "frac": achieved / peak,
+                                     "peak_source": peak_src}}),
             "extra_runs": extra_runs,
             "clocks": sampler.summary(),
             "e2e": e2e,

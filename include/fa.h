@@ -204,9 +204,12 @@ FA_API int fa_fwd_mask(const void* q, const void* k, const void* v, void* o, flo
  * fa_bwd_workspace_size -- bytes of device workspace fa_bwd needs for B*H
  * heads of Sq query rows of dimension D: an fp32 dQ accumulator
  * [B*H][Sq][D], two fp32 row-statistic arrays [B*H][Sq rounded up to 128],
- * the deterministic mode's turn counters [B*H][Sq/64 rounded up][4] int and a
- * 256-byte scheduler counter, each part 256-byte aligned.  0 for an
- * empty problem, a negative fa_status on invalid sizes.  Host only.
+ * the deterministic mode's turn counters [B*H][Sq/64 rounded up][4] int, a
+ * 256-byte scheduler counter and two fp32 arrays [B*H][128][D] for the
+ * partial sums of dK and dV (used when Sk <= 128 and the (head, key tile)
+ * units are fewer than the SMs: the query range is then split across units),
+ * each part 256-byte aligned.  0 for an empty problem, a negative fa_status
+ * on invalid sizes.  Host only.
  */
 FA_API long long fa_bwd_workspace_size(int B, int H, int Sq, int D);
 

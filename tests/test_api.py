@@ -150,17 +150,19 @@ def test_bwd_workspace_size(lib):
     assert fa.fa_bwd_workspace_size(1, 1, -1, 64) == _lib.FA_ERR_SHAPE
     assert fa.fa_bwd_workspace_size(1, 1, 10, 96) == _lib.FA_ERR_HEADDIM
     # dQ accumulator (fp32) + two padded fp32 row arrays + turn counters + 256-byte
-    # scheduler counter, 256-aligned parts
+    # scheduler counter + dK/dV partial sums, 256-aligned parts
     B, H, S, D = 2, 3, 300, 128
     up = lambda x: -(-x // 256) * 256  # noqa: E731
     acc = up(B * H * S * D * 4)
     rows = up(B * H * 384 * 4)
     flags = up(B * H * 5 * 4 * 4)
-    assert fa.fa_bwd_workspace_size(B, H, S, D) == acc + 2 * rows + flags + 256
+    kv = up(2 * B * H * 128 * D * 4)  # fp32 dK/dV partial sums of a split query range (<= 128 keys)
+    assert fa.fa_bwd_workspace_size(B, H, S, D) == acc + 2 * rows + flags + 256 + kv
     # D = 256: twice the dQ accumulator and a turn counter per half of the head dimension
     acc = up(B * H * S * 256 * 4)
     flags = up(B * H * 5 * 2 * 4 * 4)
-    assert fa.fa_bwd_workspace_size(B, H, S, 256) == acc + 2 * rows + flags + 256
+    kv = up(2 * B * H * 128 * 256 * 4)
+    assert fa.fa_bwd_workspace_size(B, H, S, 256) == acc + 2 * rows + flags + 256 + kv
 
 
 @pytest.mark.parametrize("args,code", [

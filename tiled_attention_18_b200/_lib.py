@@ -109,6 +109,9 @@ def load() -> ctypes.CDLL:
     """Load libfa.so (raises OSError if it is missing: build it with
     ``python -m tiled_attention_18_b200.build``)."""
     global _lib
+    lib = _lib
+    if lib is not None:  # loaded: no lock on the per-call path
+        return lib
     with _lock:
         if _lib is not None:
             return _lib
@@ -137,13 +140,24 @@ def fa_fwd_noalloc(q_ptr: int, k_ptr: int, v_ptr: int, o_ptr: int, lse_ptr: int,
                                      int(causal), int(dtype), stream))
 
 
+_LL3_CACHE = {}
+
+
 def _strides(st):
+    """A (b, h, s) stride triple as a C array (arrays are read-only to the library,
+    so one array per distinct triple is kept and reused)."""
     if st is None:
         return None
-    vals = [int(x) for x in st]
-    if len(vals) != 3:
-        raise ValueError("a stride triple (b, h, s) is expected")
-    return (ctypes.c_longlong * 3)(*vals)
+    key = tuple(st)
+    arr = _LL3_CACHE.get(key)
+    if arr is None:
+        vals = [int(x) for x in key]
+        if len(vals) != 3:
+            raise ValueError("a stride triple (b, h, s) is expected")
+        arr = (ctypes.c_longlong * 3)(*vals)
+        if len(_LL3_CACHE) < 4096:
+            _LL3_CACHE[key] = arr
+    return arr
 
 
 def fa_fwd_ex(q_ptr: int, k_ptr: int, v_ptr: int, o_ptr: int, lse_ptr: int, B: int, H: int, Sq: int, Sk: int,

@@ -569,6 +569,8 @@ int backward(const void* q, const void* k, const void* v, const void* o, const v
     a.dk = dk;
     a.dv = dv;
     a.dq_acc = reinterpret_cast<float*>(w + ws.dq_acc);
+    a.dk_acc = reinterpret_cast<float*>(w + ws.kv_acc);
+    a.dv_acc = a.dk_acc + BH * fa::KV_ACC_ROWS * D;
     a.lse2 = reinterpret_cast<float*>(w + ws.lse2);
     a.delta = reinterpret_cast<float*>(w + ws.delta);
     a.sched = reinterpret_cast<unsigned int*>(w + ws.sched);
@@ -592,6 +594,7 @@ int backward(const void* q, const void* k, const void* v, const void* o, const v
     // D = 256: a unit is (head, key tile, half of the head dimension)
     const int64_t units = BH * ((Sk + 127) / 128) * (D == 256 ? 2 : 1);
     a.grid = (int)(units < dev.sms ? units : dev.sms);
+    a.sms = dev.sms;  // a split query range (short key sets) resizes the grid
     const cudaError_t le = fa::launch_bwd_sm100(a, stream);
     if (le != cudaSuccess) return cuda_fail(le, "launch(backward kernels)");
     return FA_OK;

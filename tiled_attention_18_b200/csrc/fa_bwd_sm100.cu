@@ -127,6 +127,13 @@ struct BwdParams {
     uint8_t* dk;          // [B][H][Sk][D] 16-bit at byte strides dk_s (over b, h, key row)
     uint8_t* dv;          // the same at dv_s
     long long dk_s[3], dv_s[3];
+    // Split query range (key sets of at most KV_ACC_ROWS keys, few units): a
+    // unit takes chunk c of its key tile's query steps, q_chunk steps long, and
+    // adds its dK (scaled) and dV in fp32 to dk_acc / dv_acc [BH][KV_ACC_ROWS][D]
+    // instead of writing them; q_split = 1: off
+    int q_split, q_chunk;
+    float* dk_acc;
+    float* dv_acc;
     int BH, H, Sq, Sk, Sq_pad, n_mtiles, n_ktiles, n_units, causal, causal_off;
     int head_group;       // causal claim order: heads per group (their Q, dO, dQ fit in L2)
     int* dq_flags;        // deterministic mode: [BH][flag_steps][4] key tiles added so far per
@@ -165,8 +172,22 @@ __device__ __forceinline__ void causal_unit_order(const BwdParams& p, int u, int
     *bh = g * p.head_group + (within - *n * gh);
 }
 
+// Split query range: chunk c of the unit's steps [m_lo, n_mtiles).  The host
+// picks q_chunk so that no chunk is empty (one key tile: m_lo = 0).
+__device__ __forceinline__ void split_query_range(const BwdParams& p, int c, BUnit& U) {
+    const int lo = max(U.m_lo, c * p.q_chunk);
+    const int hi = min(U.m_lo + U.T, (c + 1) * p.q_chunk);
+    U.m_lo = lo;
+    U.T = hi - lo;
+}
+
 __device__ __forceinline__ BUnit decode_bwd_unit(const BwdParams& p, int u) {
     BUnit U;
+    int c = 0;
+    if (p.q_split > 1) {
+        c = u % p.q_split;
+        u /= p.q_split;
+    }
     if (p.causal) {
         causal_unit_order(p, u, &U.bh, &U.n);
         // query q sees key j iff j <= q + causal_off: the first query that sees
@@ -179,6 +200,8 @@ __device__ __forceinline__ BUnit decode_bwd_unit(const BwdParams& p, int u) {
         U.m_lo = 0;
     }
     U.T = p.n_mtiles - U.m_lo;
+    U.half = 0;
+    if (p.q_split > 1) split_query_range(p, c, U);
     return U;
 }
 
@@ -216,6 +239,32 @@ __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wa
 __device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
     asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
                  : "memory");
+}
+
+// Split query range: one thread's key row of dV and dK (W columns of fp32 in
+// TMEM from dv_col / dk_col) added to the fp32 accumulator rows, dK scaled.
+// The TMEM loads are warp-collective: every lane loads, valid lanes add.
+template <int W>
+__device__ __noinline__ void kv_partial_add(uint32_t dv_col, uint32_t dk_col, float* dva, float* dka,
+                                               float scale, bool valid) {
+#pragma unroll 1
+    for (int c = 0; c < W / 32; ++c) {
+        uint32_t r[32];
+        tmem_ld32u(dv_col + 32 * c, r);
+        if (valid) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                red_add_v4(dva + 32 * c + 4 * i, __uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]),
+                           __uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3]));
+        }
+        tmem_ld32u(dk_col + 32 * c, r);
+        if (valid) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                red_add_v4(dka + 32 * c + 4 * i, __uint_as_float(r[4 * i]) * scale, __uint_as_float(r[4 * i + 1]) * scale,
+                           __uint_as_float(r[4 * i + 2]) * scale, __uint_as_float(r[4 * i + 3]) * scale);
+        }
+    }
 }
 
 // Deterministic dQ: the key tiles of one head add their dQ contributions to
@@ -675,26 +724,33 @@ __device__ void bwd_out_role(const BwdParams& p, uint8_t* smem, uint32_t tmem, i
         const long long kr = valid ? key : 0;
         uint8_t* dv_row = p.dv + ub * p.dv_s[0] + uh * p.dv_s[1] + kr * p.dv_s[2];
         uint8_t* dk_row = p.dk + ub * p.dk_s[0] + uh * p.dk_s[1] + kr * p.dk_s[2];
+        if (p.q_split > 1) {
+            // this unit's share of the key row's sums, added in fp32 (key < KV_ACC_ROWS)
+            const size_t acc_row = ((size_t)U.bh * KV_ACC_ROWS + (size_t)kr) * D;
+            kv_partial_add<D>(tmem + lane_sel + COL_DV, tmem + lane_sel + C::DK, p.dv_acc + acc_row,
+                              p.dk_acc + acc_row, p.scale, valid);
+        } else {
 #pragma unroll 1
-        for (int c = 0; c < D / 32; ++c) {
-            uint32_t r[32];
-            uint32_t w[16];
-            tmem_ld32u(tmem + lane_sel + COL_DV + 32 * c, r);
+            for (int c = 0; c < D / 32; ++c) {
+                uint32_t r[32];
+                uint32_t w[16];
+                tmem_ld32u(tmem + lane_sel + COL_DV + 32 * c, r);
 #pragma unroll
-            for (int i = 0; i < 16; ++i) w[i] = pack2<BF16>(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
-            if (valid) {
-                uint4* d = reinterpret_cast<uint4*>(dv_row + c * 64);
+                for (int i = 0; i < 16; ++i) w[i] = pack2<BF16>(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
+                if (valid) {
+                    uint4* d = reinterpret_cast<uint4*>(dv_row + c * 64);
 #pragma unroll
-                for (int i = 0; i < 4; ++i) d[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
-            }
-            tmem_ld32u(tmem + lane_sel + C::DK + 32 * c, r);
+                    for (int i = 0; i < 4; ++i) d[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+                }
+                tmem_ld32u(tmem + lane_sel + C::DK + 32 * c, r);
 #pragma unroll
-            for (int i = 0; i < 16; ++i)
-                w[i] = pack2<BF16>(__uint_as_float(r[2 * i]) * p.scale, __uint_as_float(r[2 * i + 1]) * p.scale);
-            if (valid) {
-                uint4* d = reinterpret_cast<uint4*>(dk_row + c * 64);
+                for (int i = 0; i < 16; ++i)
+                    w[i] = pack2<BF16>(__uint_as_float(r[2 * i]) * p.scale, __uint_as_float(r[2 * i + 1]) * p.scale);
+                if (valid) {
+                    uint4* d = reinterpret_cast<uint4*>(dk_row + c * 64);
 #pragma unroll
-                for (int i = 0; i < 4; ++i) d[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+                    for (int i = 0; i < 4; ++i) d[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+                }
             }
         }
         tc_fence_before();
@@ -859,6 +915,11 @@ template <int D>
 __device__ __forceinline__ BUnit decode_bwd2_unit(const BwdParams& p, int u) {
     BUnit U;
     constexpr int HALVES = Bwd2Smem<D>::HALVES;
+    int c = 0;
+    if (p.q_split > 1) {
+        c = u % p.q_split;
+        u /= p.q_split;
+    }
     U.half = u % HALVES;
     u /= HALVES;
     if (p.causal) {
@@ -871,6 +932,7 @@ __device__ __forceinline__ BUnit decode_bwd2_unit(const BwdParams& p, int u) {
         U.m_lo = 0;
     }
     U.T = p.n_mtiles - U.m_lo;  // n_mtiles counts 64-row steps here
+    if (p.q_split > 1) split_query_range(p, c, U);
     return U;
 }
 
@@ -1167,7 +1229,9 @@ __device__ void bwd2_ds_role(const BwdParams& p, uint8_t* smem, uint32_t tmem, i
     }
 }
 
-template <int D, bool BF16>
+// SPLIT: the unit's dK, dV are partial sums over a split query range, added in
+// fp32 (a separate instantiation: the branch alone costs the role registers)
+template <int D, bool BF16, bool SPLIT>
 __device__ void bwd2_out_role(const BwdParams& p, uint8_t* smem, uint32_t tmem, int warp_in_group,
                               volatile uint32_t* abort_flag) {
     using L = Bwd2Smem<D>;
@@ -1279,26 +1343,33 @@ __device__ void bwd2_out_role(const BwdParams& p, uint8_t* smem, uint32_t tmem, 
         // this unit's 128 columns of the dK and dV rows (its half of D at D = 256)
         uint8_t* dv_row = p.dv + ub * p.dv_s[0] + uh * p.dv_s[1] + kr * p.dv_s[2] + half * 256;
         uint8_t* dk_row = p.dk + ub * p.dk_s[0] + uh * p.dk_s[1] + kr * p.dk_s[2] + half * 256;
+        if constexpr (SPLIT) {
+            // this unit's share of the key row's sums (its half of D), added in fp32
+            const size_t acc_row = ((size_t)U.bh * KV_ACC_ROWS + (size_t)kr) * D + (size_t)half * 128;
+            kv_partial_add<128>(tmem + lane_sel + COL2_DV, tmem + lane_sel + COL2_DK, p.dv_acc + acc_row,
+                                p.dk_acc + acc_row, p.scale, valid);
+        } else {
 #pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-            uint32_t r[32];
-            uint32_t w[16];
-            tmem_ld32u(tmem + lane_sel + COL2_DV + 32 * c, r);
+            for (int c = 0; c < 4; ++c) {
+                uint32_t r[32];
+                uint32_t w[16];
+                tmem_ld32u(tmem + lane_sel + COL2_DV + 32 * c, r);
 #pragma unroll
-            for (int i = 0; i < 16; ++i) w[i] = pack2<BF16>(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
-            if (valid) {
-                uint4* d = reinterpret_cast<uint4*>(dv_row + c * 64);
+                for (int i = 0; i < 16; ++i) w[i] = pack2<BF16>(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
+                if (valid) {
+                    uint4* d = reinterpret_cast<uint4*>(dv_row + c * 64);
 #pragma unroll
-                for (int i = 0; i < 4; ++i) d[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
-            }
-            tmem_ld32u(tmem + lane_sel + COL2_DK + 32 * c, r);
+                    for (int i = 0; i < 4; ++i) d[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+                }
+                tmem_ld32u(tmem + lane_sel + COL2_DK + 32 * c, r);
 #pragma unroll
-            for (int i = 0; i < 16; ++i)
-                w[i] = pack2<BF16>(__uint_as_float(r[2 * i]) * p.scale, __uint_as_float(r[2 * i + 1]) * p.scale);
-            if (valid) {
-                uint4* d = reinterpret_cast<uint4*>(dk_row + c * 64);
+                for (int i = 0; i < 16; ++i)
+                    w[i] = pack2<BF16>(__uint_as_float(r[2 * i]) * p.scale, __uint_as_float(r[2 * i + 1]) * p.scale);
+                if (valid) {
+                    uint4* d = reinterpret_cast<uint4*>(dk_row + c * 64);
 #pragma unroll
-                for (int i = 0; i < 4; ++i) d[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+                    for (int i = 0; i < 4; ++i) d[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+                }
             }
         }
         tc_fence_before();
@@ -1306,7 +1377,7 @@ __device__ void bwd2_out_role(const BwdParams& p, uint8_t* smem, uint32_t tmem, 
     }
 }
 
-template <int D, bool BF16, bool MASK, bool DROP>
+template <int D, bool BF16, bool MASK, bool DROP, bool SPLIT = false>
 __global__ void __launch_bounds__(BWD2_THREADS, 1) fa_bwd_kernel_wide(const __grid_constant__ BwdParams p) {
     using L = Bwd2Smem<D>;
     extern __shared__ uint8_t smem_raw[];
@@ -1355,7 +1426,7 @@ __global__ void __launch_bounds__(BWD2_THREADS, 1) fa_bwd_kernel_wide(const __gr
         bwd2_ds_role<D, BF16, MASK, DROP>(p, smem, tmem, warp & 3, wg == 1 ? 0 : 1, abort_flag);
     } else {
         setmaxnreg_dec<Reg2<D>::OUT>();
-        bwd2_out_role<D, BF16>(p, smem, tmem, warp & 3, abort_flag);
+        bwd2_out_role<D, BF16, SPLIT>(p, smem, tmem, warp & 3, abort_flag);
         // the bulk dQ reductions this thread issued finish before the CTA exits
         if (threadIdx.x == 2 * 128) bulk_wait_all();
     }
@@ -1434,6 +1505,29 @@ __global__ void __launch_bounds__(256) bwd_post_kernel(const float4* __restrict_
     }
 }
 
+// Split query range: dK, dV = the fp32 partial sums (dK already scaled),
+// rounded to the 16-bit dtype, written at their element strides over b, h and
+// the key row (4 elements per thread).
+template <int D, bool BF16>
+__global__ void __launch_bounds__(256) bwd_post_kv_kernel(const float4* __restrict__ dk_acc,
+                                                          const float4* __restrict__ dv_acc, uint16_t* __restrict__ dk,
+                                                          uint16_t* __restrict__ dv, size_t n4, int H, int Sk,
+                                                          Strides3 ks, Strides3 vs) {
+    constexpr int G = D / 4;  // 4-element groups per row
+    for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n4; i += (size_t)gridDim.x * blockDim.x) {
+        const size_t rowi = i / G;  // (bh, key)
+        const int d = (int)(i - rowi * G) * 4;
+        const long long bh = (long long)(rowi / (size_t)Sk), key = (long long)(rowi - (size_t)bh * Sk);
+        const size_t src = ((size_t)bh * KV_ACC_ROWS + (size_t)key) * G + (size_t)(d / 4);
+        const float4 a = dk_acc[src], b = dv_acc[src];
+        const long long ub = bh / H, uh = bh % H;
+        *reinterpret_cast<uint2*>(dk + ub * ks.s[0] + uh * ks.s[1] + key * ks.s[2] + d) =
+            make_uint2(pack2<BF16>(a.x, a.y), pack2<BF16>(a.z, a.w));
+        *reinterpret_cast<uint2*>(dv + ub * vs.s[0] + uh * vs.s[1] + key * vs.s[2] + d) =
+            make_uint2(pack2<BF16>(b.x, b.y), pack2<BF16>(b.z, b.w));
+    }
+}
+
 template <int D, bool BF16>
 cudaError_t launch_bwd_impl(const BwdLaunchArgs& a, cudaStream_t stream) {
     static_assert(BwdSmem<64>::ALLOC <= 232448, "shared memory budget exceeded");
@@ -1462,6 +1556,9 @@ cudaError_t launch_bwd_impl(const BwdLaunchArgs& a, cudaStream_t stream) {
                        : (a.mask ? fa_bwd_kernel_wide<DW, BF16, true, false>
                                  : fa_bwd_kernel_wide<DW, BF16, false, false>);
         else kern = fa_bwd_kernel<D, BF16>;
+        // the wide kernel adds split partial sums in its own instantiation, taken
+        // without an explicit mask or dropout
+        const bool can_split = !WIDE || (!a.mask && !a.drop.enabled);
         const int alloc = WIDE ? Bwd2Smem<DW>::ALLOC : BwdSmem<64>::ALLOC;
         cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(kern), alloc);
         if (e != cudaSuccess) return e;
@@ -1513,13 +1610,53 @@ cudaError_t launch_bwd_impl(const BwdLaunchArgs& a, cudaStream_t stream) {
         p.drop_offset = a.drop.offset;
         p.keep_scale = a.drop.enabled ? a.drop.keep_scale : 1.f;
         p.flag_steps = WIDE ? (a.Sq + QM - 1) / QM : n_mtiles;
+        // Split query range: a key set of at most KV_ACC_ROWS keys (one key tile)
+        // whose units leave SMs idle takes chunks of q_chunk steps per unit, about
+        // two units per SM; not in deterministic mode (the fp32 adds of the
+        // partial sums come in any order)
+        p.q_split = 1;
+        p.q_chunk = p.n_mtiles;
+        p.dk_acc = a.dk_acc;
+        p.dv_acc = a.dv_acc;
+        int grid = a.grid;
+        if (can_split && a.dk_acc && a.dv_acc && !a.dq_flags && a.Sk <= KV_ACC_ROWS && a.sms > 0 &&
+            p.n_units < a.sms && p.n_mtiles > 1) {
+            const int want = (2 * a.sms + p.n_units - 1) / p.n_units;  // chunks per key tile
+            p.q_chunk = (p.n_mtiles + want - 1) / want;
+            p.q_split = (p.n_mtiles + p.q_chunk - 1) / p.q_chunk;      // no chunk is empty
+            if (p.q_split > 1) {
+                if constexpr (WIDE) {
+                    kern = fa_bwd_kernel_wide<DW, BF16, false, false, true>;
+                    e = ensure_smem_limit(reinterpret_cast<const void*>(kern), alloc);
+                    if (e != cudaSuccess) return e;
+                }
+                p.n_units *= p.q_split;
+                grid = p.n_units < a.sms ? p.n_units : a.sms;
+                const size_t bytes = (size_t)BH * KV_ACC_ROWS * D * sizeof(float);
+                e = cudaMemsetAsync(a.dk_acc, 0, bytes, stream);
+                if (e == cudaSuccess) e = cudaMemsetAsync(a.dv_acc, 0, bytes, stream);
+                if (e != cudaSuccess) return e;
+            } else {
+                p.q_chunk = p.n_mtiles;
+            }
+        }
         cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3((unsigned)a.grid, 1, 1);
+        cfg.gridDim = dim3((unsigned)grid, 1, 1);
         cfg.blockDim = dim3(WIDE ? BWD2_THREADS : BWD_THREADS, 1, 1);
         cfg.dynamicSmemBytes = alloc;
         cfg.stream = stream;
         e = cudaLaunchKernelEx(&cfg, kern, p);
         if (e != cudaSuccess) return e;
+        if (p.q_split > 1) {
+            const size_t n4 = (size_t)BH * (size_t)a.Sk * D / 4;
+            const unsigned blocks = (unsigned)((n4 + 255) / 256 < 148u * 16u ? (n4 + 255) / 256 : 148u * 16u);
+            e = launch_kernel(bwd_post_kv_kernel<D, BF16>, dim3(blocks), dim3(256), 0, stream,
+                              reinterpret_cast<const float4*>(a.dk_acc), reinterpret_cast<const float4*>(a.dv_acc),
+                              static_cast<uint16_t*>(a.dk), static_cast<uint16_t*>(a.dv), n4, a.H, a.Sk,
+                              Strides3{{a.dk_stride[0], a.dk_stride[1], a.dk_stride[2]}},
+                              Strides3{{a.dv_stride[0], a.dv_stride[1], a.dv_stride[2]}});
+            if (e != cudaSuccess) return e;
+        }
     }
     {
         const size_t n4 = (size_t)BH * (size_t)a.Sq * D / 4;

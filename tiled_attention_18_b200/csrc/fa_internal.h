@@ -19,6 +19,10 @@ constexpr int ROWS_PER_UNIT = BLOCK_M * Q_TILES_PER_CTA;
 // Short key sets (at most one key tile per head) take the short-key kernel
 // when the tiling is automatic and there is no explicit mask or dropout.
 constexpr int SHORT_SK_MAX = 128;
+// The backward's fp32 dK/dV partial sums, used when a key set of at most this
+// many keys gives fewer work units than SMs (the query range is then split
+// across units): [B*H][KV_ACC_ROWS][D] each, in the workspace.
+constexpr int KV_ACC_ROWS = 128;
 
 // Device-side status codes written to the status word by the kernel.
 constexpr int DEV_OK = 0;
@@ -81,6 +85,8 @@ struct BwdLaunchArgs {
     void* dk;               // [B,H,Sk,D] 16-bit
     void* dv;               // [B,H,Sk,D] 16-bit
     float* dq_acc;          // workspace: [B*H][Sq][D] fp32
+    float* dk_acc;          // workspace: [B*H][KV_ACC_ROWS][D] fp32 dK partial sums (split query range)
+    float* dv_acc;          // workspace: the same for dV
     float* lse2;            // workspace: [B*H][Sq_pad] fp32
     float* delta;           // workspace: [B*H][Sq_pad] fp32
     unsigned int* sched;    // workspace: unit counter
@@ -97,12 +103,13 @@ struct BwdLaunchArgs {
     int causal;
     float scale;
     int grid;
+    int sms;                // SMs of the device (the split decision sizes units against it)
 };
 
 // Byte offsets of the backward workspace parts (each 256-byte aligned) and
 // its total size.  Sq_pad = Sq rounded up to a multiple of 128.
 struct BwdWorkspace {
-    int64_t dq_acc, lse2, delta, flags, flags_bytes, sched, total;
+    int64_t dq_acc, lse2, delta, flags, flags_bytes, sched, kv_acc, total;
 };
 inline BwdWorkspace bwd_workspace_layout(int64_t BH, int64_t Sq, int64_t D) {
     auto up = [](int64_t x) { return (x + 255) / 256 * 256; };
@@ -114,7 +121,8 @@ inline BwdWorkspace bwd_workspace_layout(int64_t BH, int64_t Sq, int64_t D) {
     w.flags = w.delta + up(BH * Sq_pad * 4);
     w.flags_bytes = BH * ((Sq + 63) / 64) * (D == 256 ? 2 : 1) * 4 * 4;  // [BH][64-row steps][D/128 halves][4 warps] int
     w.sched = w.flags + up(w.flags_bytes);
-    w.total = w.sched + 256;
+    w.kv_acc = w.sched + 256;
+    w.total = w.kv_acc + up(2 * BH * KV_ACC_ROWS * D * 4);
     return w;
 }
 
