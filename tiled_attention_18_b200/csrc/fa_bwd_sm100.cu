@@ -1439,52 +1439,77 @@ __global__ void __launch_bounds__(BWD2_THREADS, 1) fa_bwd_kernel_wide(const __gr
     }
 }
 
-template <bool BF16>
-__device__ __forceinline__ float load16(const uint16_t* p) {
-    const uint16_t x = *p;
-    if constexpr (BF16) return __bfloat162float(__ushort_as_bfloat16(x));
-    else return __half2float(__ushort_as_half(x));
+
+// Per (bh, query row) of the padded row range: Delta = sum_d dO O in fp32,
+// LSE * log2(e), and the row of the dQ accumulator cleared.  A row is taken by
+// D / 8 lanes, each with one 16-byte load of O and of dO (several rows per
+// warp when D < 256: more loads in flight per warp).  Padded rows get +inf
+// (weight 0) and Delta = 0.  Block (0, 0) also clears the scheduler counter,
+// which the main kernel (next on the stream) reads.
+template <int D>
+struct PrepShape {
+    static constexpr int LANES = D / 8;                      // lanes per row
+    static constexpr int ROWS_PER_WARP = 32 / LANES;
+    static constexpr int ROWS_PER_BLOCK = 8 * ROWS_PER_WARP;  // 256 threads
+};
+
+__device__ __forceinline__ float dot8(uint4 a, uint4 b, bool bf16) {
+    const uint32_t wa[4] = {a.x, a.y, a.z, a.w}, wb[4] = {b.x, b.y, b.z, b.w};
+    float acc = 0.f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        float2 fa, fb;
+        if (bf16) {
+            fa = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wa[i]));
+            fb = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wb[i]));
+        } else {
+            fa = __half22float2(*reinterpret_cast<const __half2*>(&wa[i]));
+            fb = __half22float2(*reinterpret_cast<const __half2*>(&wb[i]));
+        }
+        acc = fmaf(fa.x, fb.x, acc);
+        acc = fmaf(fa.y, fb.y, acc);
+    }
+    return acc;
 }
 
-// One warp per (bh, query row) of the padded row range: Delta = sum_d dO O in
-// fp32, LSE * log2(e), and the row of the dQ accumulator cleared.  Padded rows
-// get +inf (weight 0) and Delta = 0.  Block (0, 0) also clears the scheduler
-// counter, which the main kernel (next on the stream) reads.
 template <int D, bool BF16>
 __global__ void __launch_bounds__(256) bwd_prep_kernel(const uint16_t* __restrict__ o, const uint16_t* __restrict__ dout,
                                                        const float* __restrict__ lse, float* __restrict__ lse2,
                                                        float* __restrict__ delta, float* __restrict__ dq_acc, int Sq,
                                                        int Sq_pad, unsigned int* sched, int H, Strides3 os,
                                                        Strides3 dos) {
-    constexpr int PER_LANE = D / 32;
+    using PS = PrepShape<D>;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int row = blockIdx.x * 8 + warp;
+    const int sub = lane / PS::LANES, part = lane - sub * PS::LANES;  // row within the warp, 8-element part
+    const int row = blockIdx.x * PS::ROWS_PER_BLOCK + warp * PS::ROWS_PER_WARP + sub;
     const size_t bh = blockIdx.y;
     if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0 && sched) *sched = 0u;
-    if (row >= Sq_pad) return;
-    if (row >= Sq) {
-        if (lane == 0) {
+    float acc = 0.f;
+    const bool real = row < Sq;
+    if (real) {
+        const long long ub = (long long)(bh / H), uh = (long long)(bh % H);
+        const long long eo = ub * os.s[0] + uh * os.s[1] + row * os.s[2] + part * 8;
+        const long long ed = ub * dos.s[0] + uh * dos.s[1] + row * dos.s[2] + part * 8;
+        const uint4 ov = *reinterpret_cast<const uint4*>(o + eo);
+        const uint4 dv = *reinterpret_cast<const uint4*>(dout + ed);
+        acc = dot8(ov, dv, BF16);
+        float4* z = reinterpret_cast<float4*>(dq_acc + (bh * (size_t)Sq + (size_t)row) * D + (size_t)part * 8);
+        z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+        z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    // sum over the row's lanes (aligned groups of LANES lanes)
+#pragma unroll
+    for (int s = PS::LANES / 2; s > 0; s >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, s);
+    if (part == 0 && row < Sq_pad) {
+        if (real) {
+            // a row that saw no key (LSE = -inf) gets +inf, i.e. weights 0
+            const float lv = lse[bh * (size_t)Sq + row];
+            lse2[bh * Sq_pad + row] = (lv == -INFINITY) ? __int_as_float(0x7f800000) : lv * 1.4426950408889634f;
+            delta[bh * Sq_pad + row] = acc;
+        } else {
             lse2[bh * Sq_pad + row] = __int_as_float(0x7f800000);  // +inf
             delta[bh * Sq_pad + row] = 0.f;
         }
-        return;
-    }
-    const size_t e0 = (bh * (size_t)Sq + (size_t)row) * D + (size_t)lane * PER_LANE;  // dQ accumulator (contiguous)
-    const long long ub = (long long)(bh / H), uh = (long long)(bh % H);
-    const long long eo = ub * os.s[0] + uh * os.s[1] + row * os.s[2] + lane * PER_LANE;
-    const long long ed = ub * dos.s[0] + uh * dos.s[1] + row * dos.s[2] + lane * PER_LANE;
-    float acc = 0.f;
-#pragma unroll
-    for (int i = 0; i < PER_LANE; ++i) acc = fmaf(load16<BF16>(o + eo + i), load16<BF16>(dout + ed + i), acc);
-#pragma unroll
-    for (int s = 16; s > 0; s >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, s);
-#pragma unroll
-    for (int i = 0; i < PER_LANE; ++i) dq_acc[e0 + i] = 0.f;
-    if (lane == 0) {
-        // a row that saw no key (LSE = -inf) gets +inf, i.e. weights 0
-        const float lv = lse[bh * (size_t)Sq + row];
-        lse2[bh * Sq_pad + row] = (lv == -INFINITY) ? __int_as_float(0x7f800000) : lv * 1.4426950408889634f;
-        delta[bh * Sq_pad + row] = acc;
     }
 }
 
@@ -1537,7 +1562,8 @@ cudaError_t launch_bwd_impl(const BwdLaunchArgs& a, cudaStream_t stream) {
     const int n_mtiles = (a.Sq + TILE - 1) / TILE;
     const int Sq_pad = n_mtiles * TILE;
     {
-        dim3 grid((unsigned)(Sq_pad / 8), (unsigned)BH, 1);
+        dim3 grid((unsigned)((Sq_pad + PrepShape<D>::ROWS_PER_BLOCK - 1) / PrepShape<D>::ROWS_PER_BLOCK),
+                  (unsigned)BH, 1);
         cudaError_t e = launch_kernel(
             bwd_prep_kernel<D, BF16>, grid, dim3(256), 0, stream, static_cast<const uint16_t*>(a.o),
             static_cast<const uint16_t*>(a.dout), a.lse, a.lse2, a.delta, a.dq_acc, a.Sq, Sq_pad, a.sched, a.H,
