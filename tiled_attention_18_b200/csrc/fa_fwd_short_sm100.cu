@@ -15,10 +15,11 @@
 //    head are loaded once per range segment into one of two slots, so the next
 //    head's keys load while the last tiles of the current head finish;
 //  * warp 12 (TMA): Q tiles into a ring of stages, K/V on head changes;
-//  * warp 13 (MMA, issued by lane 0): S_i = Q_i K^T into TMEM slot i mod NS (three
-//    slots for D = 64, two for D = 128), issued up to NS tiles ahead, so a
-//    softmax warpgroup finds its next tile's scores ready; O_i = P_i V into O
-//    slot i mod 2 with P_i read from TMEM;
+//  * warp 13 (issued by lane 0): S_i = Q_i K^T into TMEM slot i mod NS (three
+//    slots for D = 64, two for D = 128) once the P.V of tile i - NS has read
+//    the slot, so a softmax warpgroup finds its next tile's scores ready;
+//  * warp 15 (issued by lane 0): O_i = P_i V into O slot i mod 2 with P_i read
+//    from TMEM (two issuing warps: the waits of one do not hold the other);
 //  * warpgroups 0 and 1 (softmax): warpgroup i mod 2 takes tile i, one query
 //    row per thread: masks keys past Sk (and past the diagonal when causal)
 //    in the 16-key chunks that hold keys, takes the row max, writes P as
@@ -58,6 +59,7 @@ constexpr int THREADS = 512;         // 16 warps
 constexpr int W_TMA = 12;
 constexpr int W_MMA = 13;
 constexpr int W_STORE = 14;
+constexpr int W_PV = 15;
 constexpr int REG_LAUNCH = 128;      // 65536 / 512
 constexpr int REG_SOFTMAX = 184;
 constexpr int REG_EPI = 80;
@@ -99,7 +101,8 @@ struct SLayout {
     // which waits for the epilogue of tile i + 3)
     static constexpr int B_STATS = B_OFULL + 2;
     static constexpr int B_OSTAGED = B_STATS + 8;           // [NQ] epilogue -> store, by stage (128)
-    static constexpr int B_FIN = B_OSTAGED + NQ;            // MMA: all issued MMAs complete
+    static constexpr int B_PDONE = B_OSTAGED + NQ;          // [NS] P.V warp -> S warp: the slot's P read
+    static constexpr int B_FIN = B_PDONE + NS;              // both MMA warps: all their MMAs complete (2 commits)
     static constexpr int NBAR = B_FIN + 1;
     static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;     // tmem base, abort flag
     static constexpr int BYTES = MISC_OFF + 16;
@@ -268,7 +271,8 @@ __device__ void producer_role(const SParams& p, uint8_t* smem, volatile uint32_t
 }
 
 template <int D, bool BF16>
-__device__ void mma_role(const SParams& p, uint8_t* smem, uint32_t tmem, volatile uint32_t* abort_flag) {
+__device__ void mma_role(const SParams& p, uint8_t* smem, uint32_t tmem, bool is_pv_warp,
+                         volatile uint32_t* abort_flag) {
     using L = SLayout<D>;
     const uint32_t base = smem_u32(smem);
     auto bar = [&](int i) { return base + L::BAR_OFF + 8u * (uint32_t)i; };
@@ -349,23 +353,25 @@ __device__ void mma_role(const SParams& p, uint8_t* smem, uint32_t tmem, volatil
         if (pp.mt == 0) ++kv_p;
         return true;
     };
-    // S_j goes into the slot that P_{j-NS} occupied, so it follows the P.V of
-    // tile j - NS (MMAs of one thread run in issue order); when tile j is the
-    // first of K/V index k >= 2 it also follows the last P.V of index k - 2,
-    // whose completion lets the producer refill that K/V slot for index k.
-    // `done` is the last tile whose P.V has been issued, so every tile of a K/V
-    // index below kv_p has had its P.V.  S_{i+1} is always issuable once P.V_i
-    // is (index k - 2 then ends before tile i + 1).
-    auto can_issue = [&](int j, int done) {
-        if (j >= n || j > done + L::NS) return false;
-        return kv_s < 2 || kv_p >= kv_s - 1;
-    };
-
-    int next_s = 0;
-    while (ok && can_issue(next_s, -1)) ok = issue_s(next_s++);
-    for (int i = 0; ok && i < n; ++i) {
-        ok = issue_pv(i);
-        while (ok && can_issue(next_s, i)) ok = issue_s(next_s++);
+    // Two issuing warps: this warp (S_j into slot j mod NS once the P.V of tile
+    // j - NS has completed: that slot held its P) and the P.V warp.  A new
+    // K/V slot's first S waits for the slot's fill, which follows the last P.V
+    // of the index two before (issued by the other warp, whose P and therefore
+    // S came earlier): no wait cycle.
+    if (is_pv_warp) {
+        for (int i = 0; ok && i < n; ++i) {
+            ok = issue_pv(i);
+            if (ok && leader) tc_commit(bar(L::B_PDONE + i % L::NS));
+            __syncwarp();
+        }
+    } else {
+        for (int j = 0; ok && j < n; ++j) {
+            if (j >= L::NS) {
+                ok = warp_wait(bar(L::B_PDONE + j % L::NS), (uint32_t)(j / L::NS - 1) & 1u, abort_flag, 151);
+                if (!ok) break;
+            }
+            ok = issue_s(j);
+        }
     }
     if (leader) tc_commit(bar(L::B_FIN));
     __syncwarp();
@@ -558,8 +564,9 @@ __global__ void __launch_bounds__(THREADS, 1) fa_fwd_kernel_short(const __grid_c
     if (threadIdx.x == 0) {
         for (int i = 0; i < L::NBAR; ++i) {
             uint32_t count = 1;  // TMA transaction or tcgen05.commit arrivals, or the store thread
-            if ((i >= L::B_PFULL && i < L::B_OFULL) || (i >= L::B_STATS && i < L::B_FIN))
+            if ((i >= L::B_PFULL && i < L::B_OFULL) || (i >= L::B_STATS && i < L::B_PDONE))
                 count = BM;      // one arrival per thread of a warpgroup (P, O read out, stats, staged O)
+            if (i == L::B_FIN) count = 2;  // one commit from each MMA warp
             mbar_init(base + L::BAR_OFF + 8 * i, count);
         }
         *abort_flag = 0u;
@@ -593,7 +600,7 @@ __global__ void __launch_bounds__(THREADS, 1) fa_fwd_kernel_short(const __grid_c
     } else {
         setmaxnreg_dec<REG_CTRL>();
         if (warp == W_TMA) producer_role<D>(p, smem, abort_flag);
-        else if (warp == W_MMA) mma_role<D, BF16>(p, smem, tmem, abort_flag);
+        else if (warp == W_MMA || warp == W_PV) mma_role<D, BF16>(p, smem, tmem, warp == W_PV, abort_flag);
         else if (warp == W_STORE) store_role<D>(p, smem, abort_flag);
     }
 
