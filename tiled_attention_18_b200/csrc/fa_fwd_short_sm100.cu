@@ -21,8 +21,10 @@
 //  * warp 15 (issued by lane 0): O_i = P_i V into O slot i mod 2 with P_i read
 //    from TMEM (two issuing warps: the waits of one do not hold the other);
 //  * warpgroups 0 and 1 (softmax): warpgroup i mod 2 takes tile i, one query
-//    row per thread: masks keys past Sk (and past the diagonal when causal)
-//    in the 16-key chunks that hold keys, takes the row max, writes P as
+//    row per thread: reads the row's 16-key chunks that hold keys with one
+//    TMEM wait (the chunk count is a template parameter chosen per launch),
+//    masks keys past Sk (and past the diagonal when causal), takes the row
+//    max, writes P as
 //    packed 16-bit pairs over S, and leaves 1/l and the LSE of its row in the
 //    row's first bytes of the tile's Q stage (Q is dead once S is formed);
 //  * warpgroup 2 (epilogue): scales O by 1/l, converts it and writes it over
@@ -168,29 +170,6 @@ __device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8])
     asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr), "r"(r[0]),
                  "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
                  : "memory");
-}
-
-// 32 lanes x 16 consecutive 32-bit columns, waited for.
-__device__ __forceinline__ void tmem_ld16f(uint32_t taddr, float (&v)[16]) {
-    uint32_t r[16];
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n\t"
-        "tcgen05.wait::ld.sync.aligned;"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-        : "r"(taddr)
-        : "memory");
-#pragma unroll
-    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
-}
-
-// Keys past the row's last visible key (lim = its column in this chunk) drop out.
-__device__ __forceinline__ void mask_chunk(float (&x)[16], int lim) {
-    if (lim < 15) {
-#pragma unroll
-        for (int j = 0; j < 16; ++j)
-            if (j > lim) x[j] = -INFINITY;
-    }
 }
 
 __device__ __forceinline__ void tma_store_4d(const CUtensorMap* map, uint32_t src, int c0, int c1, int c2, int c3) {
@@ -378,16 +357,42 @@ __device__ void mma_role(const SParams& p, uint8_t* smem, uint32_t tmem, bool is
     mbar_drain(bar(L::B_FIN), 0u);
 }
 
-template <int D, bool BF16>
-__device__ void softmax_role(const SParams& p, uint8_t* smem, uint32_t tmem, int b, int warp_in_group,
-                             volatile uint32_t* abort_flag) {
+// NC 16-key chunks of a row (32 lanes x 16 columns each) loaded with one
+// wait; the empty statements after the wait tie each register to it, so no
+// use of a value can be scheduled before the load has completed.
+template <int NC>
+__device__ __forceinline__ void tmem_ld_chunks(uint32_t taddr, uint32_t (&r)[NC * 16]) {
+#pragma unroll
+    for (int c = 0; c < NC; ++c) {
+        uint32_t* x = r + 16 * c;
+        asm volatile(
+            "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+            : "=r"(x[0]), "=r"(x[1]), "=r"(x[2]), "=r"(x[3]), "=r"(x[4]), "=r"(x[5]), "=r"(x[6]), "=r"(x[7]),
+              "=r"(x[8]), "=r"(x[9]), "=r"(x[10]), "=r"(x[11]), "=r"(x[12]), "=r"(x[13]), "=r"(x[14]), "=r"(x[15])
+            : "r"(taddr + 16u * (uint32_t)c));
+    }
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int c = 0; c < NC; ++c) {
+        uint32_t* x = r + 16 * c;
+        asm volatile("" : "+r"(x[0]), "+r"(x[1]), "+r"(x[2]), "+r"(x[3]), "+r"(x[4]), "+r"(x[5]), "+r"(x[6]),
+                     "+r"(x[7]), "+r"(x[8]), "+r"(x[9]), "+r"(x[10]), "+r"(x[11]), "+r"(x[12]), "+r"(x[13]),
+                     "+r"(x[14]), "+r"(x[15]));
+    }
+}
+
+// The softmax of the tiles of warpgroup b for rows whose keys fill NC 16-key
+// chunks (NC = skp / 16, a compile-time count: the row is read from TMEM with
+// one wait and kept in registers for the max and the weights).
+template <int D, bool BF16, int NC>
+__device__ void softmax_tiles(const SParams& p, uint8_t* smem, uint32_t tmem, int b, int warp_in_group,
+                              volatile uint32_t* abort_flag) {
     using L = SLayout<D>;
     const uint32_t base = smem_u32(smem);
     auto bar = [&](int i) { return base + L::BAR_OFF + 8u * (uint32_t)i; };
     const int lane = threadIdx.x & 31;
     const int r = warp_in_group * 32 + lane;  // row in the tile = TMEM lane
     const uint32_t lane_sel = (uint32_t)(warp_in_group * 32) << 16;
-    const int nc = p.skp / 16;  // 16-key chunks holding keys
     const float sl2 = p.scale_log2;
     const float2 sl2x2 = make_float2(sl2, sl2);
     int t0, n;
@@ -402,35 +407,32 @@ __device__ void softmax_role(const SParams& p, uint8_t* smem, uint32_t tmem, int
         if (!__all_sync(0xffffffffu, mbar_wait(bar(L::B_SFULL + slot), (uint32_t)(i / L::NS) & 1u, abort_flag, 145 + b)))
             return;
         tc_fence_after();
-        // Two passes over the 16-key chunks that hold keys, each reading its
-        // chunk from TMEM: the loops stay small, so their code is fetched once
-        // per launch and stays cached (the kernel runs only a few tiles per CTA).
-        float mx = -INFINITY;
-#pragma unroll 1
-        for (int c = 0; c < nc; ++c) {
-            float x[16];
-            tmem_ld16f(ts + 16u * (uint32_t)c, x);
-            mask_chunk(x, key_limit - 16 * c);
-            const float a0 = max3(x[0], x[1], x[2]), a1 = max3(x[3], x[4], x[5]);
-            const float a2 = max3(x[6], x[7], x[8]), a3 = max3(x[9], x[10], x[11]);
-            const float a4 = max3(x[12], x[13], x[14]);
-            mx = max3(mx, max3(a0, a1, a2), max3(a3, a4, x[15]));
+        uint32_t u[NC * 16];
+        tmem_ld_chunks<NC>(ts, u);
+        float x[NC * 16];
+        // keys past the row's last visible key drop out
+#pragma unroll
+        for (int c = 0; c < NC * 16; ++c) x[c] = (c > key_limit) ? -INFINITY : __uint_as_float(u[c]);
+        float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < NC; ++c) {
+            const float* y = x + 16 * c;
+            mx0 = max3(mx0, max3(y[0], y[1], y[2]), max3(y[3], y[4], y[5]));
+            mx1 = max3(mx1, max3(y[6], y[7], y[8]), max3(y[9], y[10], y[11]));
+            mx0 = max3(mx0, y[12], y[13]);
+            mx1 = max3(mx1, y[14], y[15]);
         }
         // every row sees key 0, so the max is finite
-        const float m = mx * sl2;
+        const float m = fmaxf(mx0, mx1) * sl2;
         const float2 negm2 = make_float2(-m, -m);
         float2 lsum0 = make_float2(0.f, 0.f), lsum1 = make_float2(0.f, 0.f);
         float2 rsum0 = make_float2(0.f, 0.f), rsum1 = make_float2(0.f, 0.f);
-        // P of chunk c (8 columns) lands on columns already read: those of chunk c / 2
-#pragma unroll 1
-        for (int c = 0; c < nc; ++c) {
-            float x[16];
-            tmem_ld16f(ts + 16u * (uint32_t)c, x);
-            mask_chunk(x, key_limit - 16 * c);
+#pragma unroll
+        for (int c = 0; c < NC; ++c) {
             uint32_t pk[8];
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
-                const float2 y = __ffma2_rn(make_float2(x[2 * j], x[2 * j + 1]), sl2x2, negm2);
+                const float2 y = __ffma2_rn(make_float2(x[16 * c + 2 * j], x[16 * c + 2 * j + 1]), sl2x2, negm2);
                 const float2 e = make_float2(ex2(y.x), ex2(y.y));
                 pk[j] = pack2<BF16>(e.x, e.y);
                 if (j & 1) lsum1 = __fadd2_rn(lsum1, e); else lsum0 = __fadd2_rn(lsum0, e);
@@ -454,6 +456,21 @@ __device__ void softmax_role(const SParams& p, uint8_t* smem, uint32_t tmem, int
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(bar(L::B_PFULL + slot));
+    }
+}
+
+template <int D, bool BF16>
+__device__ void softmax_role(const SParams& p, uint8_t* smem, uint32_t tmem, int b, int warp_in_group,
+                             volatile uint32_t* abort_flag) {
+    switch (p.skp / 16) {
+        case 1: softmax_tiles<D, BF16, 1>(p, smem, tmem, b, warp_in_group, abort_flag); break;
+        case 2: softmax_tiles<D, BF16, 2>(p, smem, tmem, b, warp_in_group, abort_flag); break;
+        case 3: softmax_tiles<D, BF16, 3>(p, smem, tmem, b, warp_in_group, abort_flag); break;
+        case 4: softmax_tiles<D, BF16, 4>(p, smem, tmem, b, warp_in_group, abort_flag); break;
+        case 5: softmax_tiles<D, BF16, 5>(p, smem, tmem, b, warp_in_group, abort_flag); break;
+        case 6: softmax_tiles<D, BF16, 6>(p, smem, tmem, b, warp_in_group, abort_flag); break;
+        case 7: softmax_tiles<D, BF16, 7>(p, smem, tmem, b, warp_in_group, abort_flag); break;
+        default: softmax_tiles<D, BF16, 8>(p, smem, tmem, b, warp_in_group, abort_flag); break;
     }
 }
 
