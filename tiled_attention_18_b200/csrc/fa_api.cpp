@@ -533,8 +533,8 @@ int backward(const void* q, const void* k, const void* v, const void* o, const v
     }
     fa::BwdLaunchArgs a;
     std::memset(&a, 0, sizeof(a));
-    // the D = 128 and 256 backward kernel steps through 64 query rows at a time
-    const int q_box = (D >= 128) ? 64 : fa::BLOCK_M;
+    // the backward kernel steps through 64 query rows at a time
+    const int q_box = 64;
     if (!encode_tensor(&a.tmap_q, q, B, H, Sq, D, st[0], dtype, q_box) ||
         !encode_tensor(&a.tmap_do, dout, B, H, Sq, D, st[4], dtype, q_box) ||
         !encode_tensor(&a.tmap_k, k, B, H, Sk, D, st[1], dtype) ||
@@ -549,13 +549,13 @@ int backward(const void* q, const void* k, const void* v, const void* o, const v
     }
     uint8_t* w = static_cast<uint8_t*>(workspace);
     // the fp32 dQ accumulator as a 3-D tensor [B*H][Sq][D] for the TMA engine's
-    // bulk reduce-add (D = 128): boxes of 64 rows x 128 values, rows past Sq clipped
-    if (D == 128) {
+    // bulk reduce-add (D = 64, 128): boxes of 64 rows x D values, rows past Sq clipped
+    if (D == 64 || D == 128) {
         EncodeTiledFn enc = encoder();
         if (!enc) return cuda_fail(cudaErrorNotSupported, "cuTensorMapEncodeTiled entry point");
         const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)Sq, (cuuint64_t)BH};
         const cuuint64_t strides[2] = {(cuuint64_t)D * 4, (cuuint64_t)Sq * D * 4};
-        const cuuint32_t box[3] = {128, 64, 1};
+        const cuuint32_t box[3] = {(cuuint32_t)D, 64, 1};
         const cuuint32_t elem[3] = {1, 1, 1};
         const CUresult r = enc(&a.tmap_dq, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, w + ws.dq_acc, dims, strides, box, elem,
                                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,

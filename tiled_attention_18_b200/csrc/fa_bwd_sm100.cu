@@ -20,19 +20,23 @@
 // Three launches on the caller's stream:
 //   1. bwd_prep_kernel: Delta_i, LSE_i * log2(e) (rows padded to a multiple of
 //      128: +inf, so that their weights are 0) and a zeroed fp32 dQ accumulator;
-//   2. the fused kernel: one persistent CTA per SM; a work unit is (b, h,
-//      128-key tile).  The CTA keeps K_n, V_n in shared memory and dK, dV in
-//      tensor memory and walks the query rows that see its keys (D = 64,
-//      fa_bwd_kernel: 128-row steps; D = 128 and 256, fa_bwd_kernel_wide: 64-row steps
-//      with double-buffered scores, see below):
+//   2. fa_bwd_kernel_wide: one persistent CTA per SM; a work unit is (b, h,
+//      128-key tile[, half of D at D = 256][, chunk of the query range]).  The
+//      CTA keeps K_n, V_n in shared memory and dK, dV in tensor memory and
+//      walks the query rows that see its keys in 64-row steps with
+//      double-buffered scores (see below):
 //        S^T = K Q_m^T, dP^T = V dO_m^T   (tcgen05.mma, fp32 in TMEM)
 //        P^T, dS^T                          (one key row per thread, packed to
 //                                            16 bits in TMEM; dS^T also to SMEM)
 //        dV += P^T dO_m, dK += dS^T Q_m     (A operand from TMEM)
-//        dQ_m = dS K                        (A = dS from SMEM, MN-major)
-//      dQ_m is added to the fp32 accumulator with vector reductions; dK, dV
-//      are written once per unit;
-//   3. bwd_post_kernel: dQ = scale * accumulator, rounded to the 16-bit dtype.
+//        dQ_m^T = K^T dS^T                  (into the step's dP^T columns)
+//      dQ_m is added to the fp32 accumulator (a TMA bulk reduce-add, or
+//      per-element atomics, or in key-tile order in deterministic mode); dK,
+//      dV are written once per unit.  D = 64 runs the D = 128 instantiation:
+//      its loads of the second 64-column chunk of Q, K, V and dO read past D
+//      and fill with zeros, which add nothing to the scores or gradients;
+//   3. bwd_post_kernel: dQ = scale * accumulator, rounded to the 16-bit dtype
+//      (and, after a split query range, bwd_post_kv_kernel for dK and dV).
 //
 // Every mbarrier wait is bounded like the forward kernel's (abort flag, status
 // word read by fa_check_status, drained copies, TMEM freed).
@@ -53,63 +57,10 @@ __device__ int g_status_site = 0;
 
 #include "sm100_helpers.cuh"
 
-constexpr int BWD_THREADS = 384;   // 12 warps
 constexpr int BW_TMA = 0;          // warp 0 lane 0: TMA loads and unit claims
 constexpr int BW_MMA = 1;          // warp 1 lane 0: every tcgen05.mma; TMEM owner
 constexpr int TILE = 128;          // keys per unit and query rows per step
 constexpr uint32_t BWD_TMEM_COLS = 512;
-constexpr uint32_t UNIT_READERS_BWD = 1 + 2 * TILE;  // MMA lane + two warpgroups
-
-// Tensor-memory columns of fa_bwd_kernel (D = 64): S^T/P^T, dP^T/dS^T, the dV
-// and dK accumulators and dQ of one step (the template also fits D = 128 by
-// putting dQ_m in the dP^T columns, but D = 128 runs fa_bwd_kernel_wide).
-constexpr uint32_t COL_S = 0;
-constexpr uint32_t COL_DP = 128;
-constexpr uint32_t COL_DV = 256;
-template <int D>
-struct Cols {
-    static constexpr uint32_t DK = COL_DV + D;
-    static constexpr uint32_t DQ = (D == 128) ? COL_DP : COL_DV + 2 * D;
-    static_assert(DQ + D <= BWD_TMEM_COLS || DQ == COL_DP, "tensor memory budget");
-};
-
-template <int D>
-struct BwdSmem {
-    static constexpr int CHUNKS = D / 64;           // 128-byte column chunks of a tile
-    static constexpr int CHUNK_BYTES = TILE * 128;  // 128 rows x 64 elements x 2 bytes
-    static constexpr int TILE_BYTES = TILE * D * 2;
-    static constexpr int NSTAGE = 2;
-    static constexpr int K_OFF = 0;
-    static constexpr int V_OFF = TILE_BYTES;
-    static constexpr int STAGE_OFF = 2 * TILE_BYTES;        // stage: Q_m, dO_m
-    static constexpr int STAGE_BYTES = 2 * TILE_BYTES;
-    static constexpr int DS_OFF = STAGE_OFF + NSTAGE * STAGE_BYTES;  // dS^T [128 keys][128 queries]
-    static constexpr int DS_BYTES = TILE * TILE * 2;
-    static constexpr int STATS_OFF = DS_OFF + DS_BYTES;      // per stage: lse2[128], delta[128]
-    static constexpr int STATS_BYTES = 2 * TILE * 4;
-    static constexpr int BAR_OFF = STATS_OFF + NSTAGE * STATS_BYTES;
-    enum {
-        B_KVFULL = 0,
-        B_KVEMPTY,
-        B_SFULL,
-        B_PFULL,
-        B_DSEMPTY,
-        B_DQFULL,
-        B_DQEMPTY,
-        B_DKVFULL,
-        B_DKVEMPTY,
-        B_FIN,
-        B_UFULL,               // [2]
-        B_UEMPTY = B_UFULL + 2,  // [2]
-        B_QFULL = B_UEMPTY + 2,  // [NSTAGE]
-        B_QEMPTY = B_QFULL + NSTAGE,
-        NBAR = B_QEMPTY + NSTAGE
-    };
-    static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;  // [0] TMEM base, [1] abort flag
-    static constexpr int UNIT_OFF = MISC_OFF + 16;       // unit ring, int[2]
-    static constexpr int BYTES = UNIT_OFF + 8;
-    static constexpr int ALLOC = BYTES + 1024;           // slack for 1 KiB alignment
-};
 
 struct Strides3 {
     long long s[3];  // element strides over b, h and the row
@@ -135,6 +86,7 @@ struct BwdParams {
     float* dk_acc;
     float* dv_acc;
     int BH, H, Sq, Sk, Sq_pad, n_mtiles, n_ktiles, n_units, causal, causal_off;
+    int dh;               // head dimension of the tensors (64: run by the D = 128 kernel on zero-padded operands)
     int head_group;       // causal claim order: heads per group (their Q, dO, dQ fit in L2)
     int* dq_flags;        // deterministic mode: [BH][flag_steps][4] key tiles added so far per
                           // (head, query step, warp); null: dQ is added with atomics
@@ -181,30 +133,6 @@ __device__ __forceinline__ void split_query_range(const BwdParams& p, int c, BUn
     U.T = hi - lo;
 }
 
-__device__ __forceinline__ BUnit decode_bwd_unit(const BwdParams& p, int u) {
-    BUnit U;
-    int c = 0;
-    if (p.q_split > 1) {
-        c = u % p.q_split;
-        u /= p.q_split;
-    }
-    if (p.causal) {
-        causal_unit_order(p, u, &U.bh, &U.n);
-        // query q sees key j iff j <= q + causal_off: the first query that sees
-        // key n*128 is n*128 - causal_off
-        const int q_first = U.n * TILE - p.causal_off;
-        U.m_lo = q_first > 0 ? q_first / TILE : 0;
-    } else {
-        U.bh = u / p.n_ktiles;
-        U.n = u - U.bh * p.n_ktiles;
-        U.m_lo = 0;
-    }
-    U.T = p.n_mtiles - U.m_lo;
-    U.half = 0;
-    if (p.q_split > 1) split_query_range(p, c, U);
-    return U;
-}
-
 __host__ __device__ constexpr uint32_t make_idesc_bwd(bool bf16, int N, bool a_mn_major, bool b_mn_major) {
     return (1u << 4)                                   // D format: f32
            | ((bf16 ? 1u : 0u) << 7)                   // A format
@@ -244,11 +172,10 @@ __device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float 
 // Split query range: one thread's key row of dV and dK (W columns of fp32 in
 // TMEM from dv_col / dk_col) added to the fp32 accumulator rows, dK scaled.
 // The TMEM loads are warp-collective: every lane loads, valid lanes add.
-template <int W>
 __device__ __noinline__ void kv_partial_add(uint32_t dv_col, uint32_t dk_col, float* dva, float* dka,
-                                               float scale, bool valid) {
+                                            float scale, bool valid, int width) {
 #pragma unroll 1
-    for (int c = 0; c < W / 32; ++c) {
+    for (int c = 0; c < width / 32; ++c) {
         uint32_t r[32];
         tmem_ld32u(dv_col + 32 * c, r);
         if (valid) {
@@ -372,452 +299,9 @@ __device__ __forceinline__ void fence_async_smem() {
 
 // Reads the work-unit indices published by the TMA lane (same protocol as the
 // forward kernel's ring): -1 when the CTA has no more work, -2 on abort.
-template <int D>
-struct BwdUnitReader {
-    int slot = 0;
-    uint32_t phase = 0;
-    __device__ __forceinline__ int next(uint8_t* smem, volatile uint32_t* abort_flag, int site) {
-        using L = BwdSmem<D>;
-        const uint32_t bar0 = smem_u32(smem) + L::BAR_OFF;
-        if (!mbar_wait(bar0 + 8u * (uint32_t)(L::B_UFULL + slot), phase, abort_flag, site)) return -2;
-        const int u = reinterpret_cast<volatile int*>(smem + L::UNIT_OFF)[slot];
-        mbar_arrive(bar0 + 8u * (uint32_t)(L::B_UEMPTY + slot));
-        if (++slot == 2) { slot = 0; phase ^= 1u; }
-        return u;
-    }
-};
-
-template <int D>
-__device__ void bwd_producer(const BwdParams& p, uint8_t* smem, volatile uint32_t* abort_flag) {
-    using L = BwdSmem<D>;
-    const uint32_t base = smem_u32(smem);
-    const uint32_t bar0 = base + L::BAR_OFF;
-    auto bar = [&](int i) { return bar0 + 8u * (uint32_t)i; };
-    volatile int* ring = reinterpret_cast<volatile int*>(smem + L::UNIT_OFF);
-    int uslot = 0;
-    uint32_t uphase = 0, kv_phase = 0, phase = 0;
-    int stage = 0;
-    bool ok = true;
-    int kv_fill = -1;             // parity of the last K/V fill, -1 if none
-    uint32_t fill_mask = 0, fill_parity = 0;
-    for (int k = 0;; ++k) {
-        int u = p.sched ? (int)atomicAdd(p.sched, 1u) : (int)blockIdx.x + k * (int)gridDim.x;
-        if (u >= p.n_units) u = -1;
-        if (!mbar_wait(bar(L::B_UEMPTY + uslot), uphase ^ 1u, abort_flag, 40)) { ok = false; break; }
-        ring[uslot] = u;
-        mbar_arrive(bar(L::B_UFULL + uslot));
-        if (++uslot == 2) { uslot = 0; uphase ^= 1u; }
-        if (u < 0) break;
-        const BUnit U = decode_bwd_unit(p, u);
-        const int b = U.bh / p.H, h = U.bh - b * p.H;
-        if (!mbar_wait(bar(L::B_KVEMPTY), kv_phase ^ 1u, abort_flag, 41)) { ok = false; break; }
-        mbar_expect_tx(bar(L::B_KVFULL), 2 * L::TILE_BYTES);
-        kv_fill = (int)kv_phase;
-        kv_phase ^= 1u;
-#pragma unroll
-        for (int c = 0; c < L::CHUNKS; ++c) {
-            tma_load_4d(base + L::K_OFF + c * L::CHUNK_BYTES, &p.tmap_k, bar(L::B_KVFULL), c * 64, U.n * TILE, h, b);
-            tma_load_4d(base + L::V_OFF + c * L::CHUNK_BYTES, &p.tmap_v, bar(L::B_KVFULL), c * 64, U.n * TILE, h, b);
-        }
-        for (int t = 0; t < U.T; ++t) {
-            const int m = U.m_lo + t;
-            if (!mbar_wait(bar(L::B_QEMPTY + stage), phase ^ 1u, abort_flag, 42)) { ok = false; break; }
-            mbar_expect_tx(bar(L::B_QFULL + stage), 2 * L::TILE_BYTES + L::STATS_BYTES);
-            fill_mask |= 1u << stage;
-            fill_parity = (fill_parity & ~(1u << stage)) | (phase << stage);
-            const uint32_t dst = base + L::STAGE_OFF + stage * L::STAGE_BYTES;
-#pragma unroll
-            for (int c = 0; c < L::CHUNKS; ++c) {
-                tma_load_4d(dst + c * L::CHUNK_BYTES, &p.tmap_q, bar(L::B_QFULL + stage), c * 64, m * TILE, h, b);
-                tma_load_4d(dst + L::TILE_BYTES + c * L::CHUNK_BYTES, &p.tmap_do, bar(L::B_QFULL + stage), c * 64,
-                            m * TILE, h, b);
-            }
-            const size_t srow = (size_t)U.bh * (size_t)p.Sq_pad + (size_t)m * TILE;
-            const uint32_t sdst = base + L::STATS_OFF + stage * L::STATS_BYTES;
-            bulk_load(sdst, p.lse2 + srow, TILE * 4, bar(L::B_QFULL + stage));
-            bulk_load(sdst + TILE * 4, p.delta + srow, TILE * 4, bar(L::B_QFULL + stage));
-            if (++stage == L::NSTAGE) { stage = 0; phase ^= 1u; }
-        }
-        if (!ok) break;
-    }
-    if (!ok) {
-        for (int i = 0; i < L::NSTAGE; ++i)
-            if (fill_mask & (1u << i)) mbar_drain(bar(L::B_QFULL + i), (fill_parity >> i) & 1u);
-        if (kv_fill >= 0) mbar_drain(bar(L::B_KVFULL), (uint32_t)kv_fill);
-    }
-}
-
-template <int D, bool BF16>
-__device__ void bwd_mma(const BwdParams& p, uint8_t* smem, uint32_t tmem, volatile uint32_t* abort_flag) {
-    using L = BwdSmem<D>;
-    using C = Cols<D>;
-    const uint32_t base = smem_u32(smem);
-    const uint32_t bar0 = base + L::BAR_OFF;
-    auto bar = [&](int i) { return bar0 + 8u * (uint32_t)i; };
-    constexpr uint32_t IDESC_S = make_idesc_bwd(BF16, TILE, false, false);  // S^T, dP^T: N = 128 queries
-    constexpr uint32_t IDESC_KV = make_idesc_bwd(BF16, D, false, true);     // dV, dK: A in TMEM, B MN-major
-    constexpr uint32_t IDESC_DQ = make_idesc_bwd(BF16, D, true, true);      // dQ: A = dS MN-major, B = K MN-major
-    constexpr uint32_t MN_LBO = (D == 128) ? (uint32_t)L::CHUNK_BYTES : 1024u;
-
-    // K-major operands (K, V, Q, dO as [rows][D], 128-byte swizzle): a K step of
-    // 16 elements advances 32 bytes inside a swizzle atom and 16 KiB across
-    // 64-column chunks.  MN-major operands (Q, dO, K as [rows][D] read along D;
-    // dS^T as [keys][queries] read along the queries): 64-element chunks 16 KiB
-    // apart (leading byte offset), 8-row groups 1024 bytes apart; a K step of 16
-    // rows advances 2 KiB.
-    const uint64_t dk_k = sw128_desc(base + L::K_OFF, 16, 1024);
-    const uint64_t dv_k = sw128_desc(base + L::V_OFF, 16, 1024);
-    const uint64_t dstage_k = sw128_desc(base + L::STAGE_OFF, 16, 1024);
-    const uint64_t dstage_mn = sw128_desc(base + L::STAGE_OFF, MN_LBO, 1024);
-    const uint64_t dk_mn = sw128_desc(base + L::K_OFF, MN_LBO, 1024);
-    const uint64_t ds_mn = sw128_desc(base + L::DS_OFF, (uint32_t)L::CHUNK_BYTES, 1024);
-    constexpr uint32_t STAGE16 = (uint32_t)L::STAGE_BYTES >> 4;
-    constexpr uint32_t TILE16 = (uint32_t)L::TILE_BYTES >> 4;
-
-    // D(tmem) = A(smem, K-major over D) B(smem, K-major over D)^T
-    auto issue_kmajor = [&](uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t b_off16) {
-#pragma unroll
-        for (int ks = 0; ks < D / 16; ++ks) {
-            const uint32_t off = (uint32_t)(((ks & 3) * 32 + (ks >> 2) * L::CHUNK_BYTES) >> 4);
-            tc_mma_ss2(d_tmem, (uint32_t)a + off, (uint32_t)(a >> 32), (uint32_t)b + b_off16 + off,
-                       (uint32_t)(b >> 32), IDESC_S, ks > 0 ? 1u : 0u);
-        }
-    };
-    // D(tmem) (+)= A(tmem, 16-bit pairs) B(smem, MN-major), K = 128 rows
-    auto issue_ts = [&](uint32_t d_tmem, uint32_t a_tmem, uint64_t b, uint32_t b_off16, bool accumulate) {
-#pragma unroll
-        for (int ks = 0; ks < TILE / 16; ++ks)
-            tc_mma_ts2(d_tmem, a_tmem + (uint32_t)(ks * 8), (uint32_t)b + b_off16 + (uint32_t)(ks * (2048 >> 4)),
-                       (uint32_t)(b >> 32), IDESC_KV, (accumulate || ks > 0) ? 1u : 0u);
-    };
-
-    uint32_t kv_phase = 0, phase = 0, p_phase = 0, dqe_phase = 0, dkve_phase = 0;
-    int stage = 0;
-    BwdUnitReader<D> units;
-    for (;;) {
-        const int u = units.next(smem, abort_flag, 43);
-        if (u < 0) break;
-        const BUnit U = decode_bwd_unit(p, u);
-        if (!mbar_wait(bar(L::B_KVFULL), kv_phase, abort_flag, 44)) break;
-        kv_phase ^= 1u;
-        bool ok = true;
-        for (int t = 0; t < U.T; ++t) {
-            const int st = stage;
-            if (!mbar_wait(bar(L::B_QFULL + st), phase, abort_flag, 45)) { ok = false; break; }
-            if (++stage == L::NSTAGE) { stage = 0; phase ^= 1u; }
-            const uint32_t q_off16 = (uint32_t)st * STAGE16;
-            const uint32_t do_off16 = q_off16 + TILE16;
-            // S^T = K Q_m^T
-            issue_kmajor(tmem + COL_S, dk_k, dstage_k, q_off16);
-            // dP^T = V dO_m^T (at D = 128 these columns hold the previous dQ: wait for its read-out)
-            if (C::DQ == COL_DP) {
-                if (!mbar_wait(bar(L::B_DQEMPTY), dqe_phase ^ 1u, abort_flag, 46)) { ok = false; break; }
-                dqe_phase ^= 1u;
-                tc_fence_after();
-            }
-            issue_kmajor(tmem + COL_DP, dv_k, dstage_k, do_off16);
-            tc_commit(bar(L::B_SFULL));
-            // P^T and dS^T from the dS warpgroup
-            if (!mbar_wait(bar(L::B_PFULL), p_phase, abort_flag, 47)) { ok = false; break; }
-            p_phase ^= 1u;
-            tc_fence_after();
-            if (t == 0) {
-                // the previous unit's dK and dV have been read out
-                if (!mbar_wait(bar(L::B_DKVEMPTY), dkve_phase ^ 1u, abort_flag, 48)) { ok = false; break; }
-                dkve_phase ^= 1u;
-                tc_fence_after();
-            }
-            issue_ts(tmem + COL_DV, tmem + COL_S, dstage_mn, do_off16, t > 0);  // dV += P^T dO_m
-            issue_ts(tmem + C::DK, tmem + COL_DP, dstage_mn, q_off16, t > 0);  // dK += dS^T Q_m
-            tc_commit(bar(L::B_QEMPTY + st));
-            if (C::DQ != COL_DP) {
-                if (!mbar_wait(bar(L::B_DQEMPTY), dqe_phase ^ 1u, abort_flag, 46)) { ok = false; break; }
-                dqe_phase ^= 1u;
-                tc_fence_after();
-            }
-            // dQ_m = dS K: A = dS (queries x keys) read MN-major from dS^T, B = K read MN-major
-#pragma unroll
-            for (int ks = 0; ks < TILE / 16; ++ks) {
-                const uint32_t off = (uint32_t)(ks * (2048 >> 4));
-                tc_mma_ss2(tmem + C::DQ, (uint32_t)ds_mn + off, (uint32_t)(ds_mn >> 32), (uint32_t)dk_mn + off,
-                           (uint32_t)(dk_mn >> 32), IDESC_DQ, ks > 0 ? 1u : 0u);
-            }
-            tc_commit(bar(L::B_DQFULL));
-            tc_commit(bar(L::B_DSEMPTY));
-        }
-        if (!ok) break;
-        tc_commit(bar(L::B_DKVFULL));
-        tc_commit(bar(L::B_KVEMPTY));
-    }
-    // all MMAs issued by this thread have completed once B_FIN fires
-    tc_commit(bar(L::B_FIN));
-    mbar_drain(bar(L::B_FIN), 0u);
-}
-
-// P^T and dS^T: one key row per thread (TMEM lane), 32 queries at a time.
-template <int D, bool BF16>
-__device__ void bwd_ds_role(const BwdParams& p, uint8_t* smem, uint32_t tmem, int warp_in_group,
-                            volatile uint32_t* abort_flag) {
-    using L = BwdSmem<D>;
-    const uint32_t base = smem_u32(smem);
-    const uint32_t bar0 = base + L::BAR_OFF;
-    auto bar = [&](int i) { return bar0 + 8u * (uint32_t)i; };
-    const int lane = threadIdx.x & 31;
-    const int row = warp_in_group * 32 + lane;  // key row within the tile
-    const uint32_t lane_sel = (uint32_t)(warp_in_group * 32) << 16;
-    const float sl2 = p.scale_log2;
-    uint32_t s_phase = 0, dse_phase = 0, phase = 0;
-    int stage = 0;
-    // this thread's row of the dS^T tile: 128-byte rows, 8-row groups 1 KiB apart,
-    // 16-byte granules XOR-swizzled by the row index (the TMA/UMMA 128-byte swizzle)
-    uint8_t* ds_row = smem + L::DS_OFF + (row >> 3) * 1024 + (row & 7) * 128;
-    const int sw = row & 7;
-    BwdUnitReader<D> units;
-    for (;;) {
-        const int u = units.next(smem, abort_flag, 49);
-        if (!__all_sync(0xffffffffu, u != -2)) return;
-        if (u < 0) break;
-        const BUnit U = decode_bwd_unit(p, u);
-        const int key = U.n * TILE + row;
-        const bool key_ok = key < p.Sk;
-        const int q_min = p.causal ? key - p.causal_off : 0;  // first query that sees this key
-        const uint8_t* mhead =
-            p.mask ? p.mask + (long long)(U.bh / p.H) * p.m_sb + (long long)(U.bh % p.H) * p.m_sh : nullptr;
-        for (int t = 0; t < U.T; ++t) {
-            const int m = U.m_lo + t;
-            const int st = stage;
-            const uint32_t st_phase = phase;
-            if (++stage == L::NSTAGE) { stage = 0; phase ^= 1u; }
-            if (!__all_sync(0xffffffffu, mbar_wait(bar(L::B_SFULL), s_phase, abort_flag, 50))) return;
-            s_phase ^= 1u;
-            // the stage's row statistics came with its TMA fill: observe that fill
-            // here too (the phase cannot move on before this warpgroup arrives on
-            // B_PFULL, since the stage is released only after the P.V / dS.Q MMAs)
-            if (!__all_sync(0xffffffffu, mbar_wait(bar(L::B_QFULL + st), st_phase, abort_flag, 55))) return;
-            // the previous dQ MMA has read the dS^T tile
-            if (!__all_sync(0xffffffffu, mbar_wait(bar(L::B_DSEMPTY), dse_phase ^ 1u, abort_flag, 51))) return;
-            dse_phase ^= 1u;
-            tc_fence_after();
-            const float* lse2s = reinterpret_cast<const float*>(smem + L::STATS_OFF + st * L::STATS_BYTES);
-            const float* dls = lse2s + TILE;
-            const bool need_mask = !key_ok || (m * TILE < q_min) || p.mask != nullptr;
-#pragma unroll 1
-            for (int c = 0; c < 4; ++c) {
-                // explicit mask: this key's bits over the chunk's 32 queries
-                const uint32_t mbits = p.mask ? mask_col_bits(mhead, p.m_ss, p.Sq, p.Sk, m * TILE + 32 * c,
-                                                              U.n * TILE + warp_in_group * 32)
-                                              : 0xffffffffu;
-                // dropout: this key's keep bits over the chunk's 32 queries
-                const uint32_t zbits =
-                    p.drop ? dropout_col_bits(p, U.bh, m * TILE + 32 * c, U.n * TILE + warp_in_group * 32)
-                           : 0xffffffffu;
-                uint32_t sr[32], dr[32];
-                tmem_ld32u(tmem + lane_sel + COL_S + 32 * c, sr);
-                tmem_ld32u(tmem + lane_sel + COL_DP + 32 * c, dr);
-                uint32_t pk[16], dk[16];
-#pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const int j = 32 * c + 2 * i;
-                    const float2 l2 = *reinterpret_cast<const float2*>(lse2s + j);
-                    const float2 dl = *reinterpret_cast<const float2*>(dls + j);
-                    float p0 = ex2(fmaf(__uint_as_float(sr[2 * i]), sl2, -l2.x));
-                    float p1 = ex2(fmaf(__uint_as_float(sr[2 * i + 1]), sl2, -l2.y));
-                    if (need_mask) {
-                        const int q = m * TILE + j;
-                        if (!key_ok || q < q_min || !((mbits >> (2 * i)) & 1u)) p0 = 0.f;
-                        if (!key_ok || q + 1 < q_min || !((mbits >> (2 * i + 1)) & 1u)) p1 = 0.f;
-                    }
-                    // dropout factors: 1 / (1 - p) for a kept weight, 0 for a dropped one
-                    float z0 = 1.f, z1 = 1.f;
-                    if (p.drop) {
-                        z0 = ((zbits >> (2 * i)) & 1u) ? p.keep_scale : 0.f;
-                        z1 = ((zbits >> (2 * i + 1)) & 1u) ? p.keep_scale : 0.f;
-                    }
-                    const float d0 = p0 * (__uint_as_float(dr[2 * i]) * z0 - dl.x);
-                    const float d1 = p1 * (__uint_as_float(dr[2 * i + 1]) * z1 - dl.y);
-                    pk[i] = pack2<BF16>(p0 * z0, p1 * z1);
-                    dk[i] = pack2<BF16>(d0, d1);
-                }
-                tmem_st16(tmem + lane_sel + COL_S + 16 * c, pk);
-                tmem_st16(tmem + lane_sel + COL_DP + 16 * c, dk);
-                // queries 32c .. 32c+31 of this key row: chunk c/2, granules (c%2)*4 .. +3
-                uint8_t* chunk = ds_row + (c >> 1) * L::CHUNK_BYTES;
-#pragma unroll
-                for (int g = 0; g < 4; ++g) {
-                    const int gr = ((c & 1) * 4 + g) ^ sw;
-                    *reinterpret_cast<uint4*>(chunk + gr * 16) =
-                        make_uint4(dk[4 * g], dk[4 * g + 1], dk[4 * g + 2], dk[4 * g + 3]);
-                }
-            }
-            tmem_wait_st();
-            fence_async_smem();
-            tc_fence_before();
-            mbar_arrive(bar(L::B_PFULL));
-        }
-    }
-}
-
-// dQ_m read-out (one query row per thread) into the fp32 accumulator, and the
-// unit's dK, dV (one key row per thread) to global memory.
-template <int D, bool BF16>
-__device__ void bwd_out_role(const BwdParams& p, uint8_t* smem, uint32_t tmem, int warp_in_group,
-                             volatile uint32_t* abort_flag) {
-    using L = BwdSmem<D>;
-    using C = Cols<D>;
-    const uint32_t base = smem_u32(smem);
-    const uint32_t bar0 = base + L::BAR_OFF;
-    auto bar = [&](int i) { return bar0 + 8u * (uint32_t)i; };
-    const int lane = threadIdx.x & 31;
-    const int row = warp_in_group * 32 + lane;
-    const uint32_t lane_sel = (uint32_t)(warp_in_group * 32) << 16;
-    uint32_t dq_phase = 0, dkv_phase = 0;
-    BwdUnitReader<D> units;
-    for (;;) {
-        const int u = units.next(smem, abort_flag, 52);
-        if (!__all_sync(0xffffffffu, u != -2)) return;
-        if (u < 0) break;
-        const BUnit U = decode_bwd_unit(p, u);
-        for (int t = 0; t < U.T; ++t) {
-            const int m = U.m_lo + t;
-            if (!__all_sync(0xffffffffu, mbar_wait(bar(L::B_DQFULL), dq_phase, abort_flag, 53))) return;
-            dq_phase ^= 1u;
-            tc_fence_after();
-            const int q = m * TILE + row;
-            const bool valid = q < p.Sq;
-            float* dst = p.dq_acc + ((size_t)U.bh * (size_t)p.Sq + (size_t)(valid ? q : 0)) * D;
-            int* flag = p.dq_flags ? p.dq_flags + ((size_t)U.bh * p.flag_steps + m) * 4 + warp_in_group : nullptr;
-            if (flag && !wait_turn(flag, U.n, abort_flag, 56)) return;
-#pragma unroll 1
-            for (int c = 0; c < D / 32; ++c) {
-                uint32_t r[32];
-                tmem_ld32u(tmem + lane_sel + C::DQ + 32 * c, r);
-                if (valid) {
-                    if (flag) {
-#pragma unroll
-                        for (int i = 0; i < 8; ++i) {
-                            float4* a4 = reinterpret_cast<float4*>(dst + 32 * c + 4 * i);
-                            float4 v = __ldcg(a4);
-                            v.x += __uint_as_float(r[4 * i]);
-                            v.y += __uint_as_float(r[4 * i + 1]);
-                            v.z += __uint_as_float(r[4 * i + 2]);
-                            v.w += __uint_as_float(r[4 * i + 3]);
-                            __stcg(a4, v);
-                        }
-                    } else {
-#pragma unroll
-                        for (int i = 0; i < 8; ++i)
-                            red_add_v4(dst + 32 * c + 4 * i, __uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]),
-                                       __uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3]));
-                    }
-                }
-            }
-            if (flag) pass_turn(flag, U.n + 1);
-            tc_fence_before();
-            mbar_arrive(bar(L::B_DQEMPTY));
-        }
-        if (!__all_sync(0xffffffffu, mbar_wait(bar(L::B_DKVFULL), dkv_phase, abort_flag, 54))) return;
-        dkv_phase ^= 1u;
-        tc_fence_after();
-        const int key = U.n * TILE + row;
-        const bool valid = key < p.Sk;
-        const int ub = U.bh / p.H, uh = U.bh - ub * p.H;
-        const long long kr = valid ? key : 0;
-        uint8_t* dv_row = p.dv + ub * p.dv_s[0] + uh * p.dv_s[1] + kr * p.dv_s[2];
-        uint8_t* dk_row = p.dk + ub * p.dk_s[0] + uh * p.dk_s[1] + kr * p.dk_s[2];
-        if (p.q_split > 1) {
-            // this unit's share of the key row's sums, added in fp32 (key < KV_ACC_ROWS)
-            const size_t acc_row = ((size_t)U.bh * KV_ACC_ROWS + (size_t)kr) * D;
-            kv_partial_add<D>(tmem + lane_sel + COL_DV, tmem + lane_sel + C::DK, p.dv_acc + acc_row,
-                              p.dk_acc + acc_row, p.scale, valid);
-        } else {
-#pragma unroll 1
-            for (int c = 0; c < D / 32; ++c) {
-                uint32_t r[32];
-                uint32_t w[16];
-                tmem_ld32u(tmem + lane_sel + COL_DV + 32 * c, r);
-#pragma unroll
-                for (int i = 0; i < 16; ++i) w[i] = pack2<BF16>(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
-                if (valid) {
-                    uint4* d = reinterpret_cast<uint4*>(dv_row + c * 64);
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) d[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
-                }
-                tmem_ld32u(tmem + lane_sel + C::DK + 32 * c, r);
-#pragma unroll
-                for (int i = 0; i < 16; ++i)
-                    w[i] = pack2<BF16>(__uint_as_float(r[2 * i]) * p.scale, __uint_as_float(r[2 * i + 1]) * p.scale);
-                if (valid) {
-                    uint4* d = reinterpret_cast<uint4*>(dk_row + c * 64);
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) d[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
-                }
-            }
-        }
-        tc_fence_before();
-        mbar_arrive(bar(L::B_DKVEMPTY));
-    }
-}
-
-template <int D, bool BF16>
-__global__ void __launch_bounds__(BWD_THREADS, 1) fa_bwd_kernel(const __grid_constant__ BwdParams p) {
-    using L = BwdSmem<D>;
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    const uint32_t base = smem_u32(smem);
-    const int warp = threadIdx.x >> 5;
-    const int lane = threadIdx.x & 31;
-    const int wg = warp >> 2;
-    uint32_t* misc = reinterpret_cast<uint32_t*>(smem + L::MISC_OFF);
-    volatile uint32_t* abort_flag = misc + 1;
-
-    if (threadIdx.x == 0) {
-        for (int i = 0; i < L::NBAR; ++i) {
-            uint32_t count = 1;  // TMA transaction or tcgen05.commit arrivals
-            if (i == L::B_PFULL || i == L::B_DQEMPTY || i == L::B_DKVEMPTY) count = TILE;  // one warpgroup
-            if (i >= L::B_UEMPTY && i < L::B_UEMPTY + 2) count = UNIT_READERS_BWD;
-            mbar_init(base + L::BAR_OFF + 8 * i, count);
-        }
-        *abort_flag = 0u;
-        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-    }
-    if (warp == BW_TMA && lane == 0) {
-        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&p.tmap_q)) : "memory");
-        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&p.tmap_k)) : "memory");
-        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&p.tmap_v)) : "memory");
-        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&p.tmap_do)) : "memory");
-    }
-    if (warp == BW_MMA) {
-        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(misc)),
-                     "r"(BWD_TMEM_COLS)
-                     : "memory");
-        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = misc[0];
-
-    if (wg == 0) {
-        if (warp == BW_TMA && lane == 0) bwd_producer<D>(p, smem, abort_flag);
-        if (warp == BW_MMA && lane == 0) bwd_mma<D, BF16>(p, smem, tmem, abort_flag);
-    } else if (wg == 1) {
-        bwd_ds_role<D, BF16>(p, smem, tmem, warp & 3, abort_flag);
-    } else {
-        bwd_out_role<D, BF16>(p, smem, tmem, warp & 3, abort_flag);
-    }
-
-    tc_fence_before();
-    __syncthreads();
-    if (warp == BW_MMA) {
-        tc_fence_after();
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(BWD_TMEM_COLS)
-                     : "memory");
-    }
-}
-
 // ------------------------------------------------------------------------
-// D = 128 and 256: 64-row query steps with double-buffered S^T / dP^T.
+// 64-row query steps with double-buffered S^T / dP^T (D = 64 on the D = 128
+// instantiation with zero-padded operands, D = 128, D = 256).
 //
 // Tensor memory: S0 [0,64) dP0 [64,128) S1 [128,192) dP1 [192,256), dV
 // [256,384), dK [384,512).  While the dS warpgroup turns step g's S^T, dP^T
@@ -1231,7 +715,7 @@ __device__ void bwd2_ds_role(const BwdParams& p, uint8_t* smem, uint32_t tmem, i
 
 // SPLIT: the unit's dK, dV are partial sums over a split query range, added in
 // fp32 (a separate instantiation: the branch alone costs the role registers)
-template <int D, bool BF16, bool SPLIT>
+template <int D, bool BF16, bool SPLIT, int DH>
 __device__ void bwd2_out_role(const BwdParams& p, uint8_t* smem, uint32_t tmem, int warp_in_group,
                               volatile uint32_t* abort_flag) {
     using L = Bwd2Smem<D>;
@@ -1266,7 +750,9 @@ __device__ void bwd2_out_role(const BwdParams& p, uint8_t* smem, uint32_t tmem, 
             if (!__all_sync(0xffffffffu, mbar_wait(bar(L::B_DQFULL + b), (g >> 1) & 1u, abort_flag, 74))) return;
             tc_fence_after();
             // dQ[q][d] += dQ^T[d][q]: consecutive threads take consecutive d (coalesced)
-            float* dst = p.dq_acc + ((size_t)U.bh * (size_t)p.Sq + (size_t)m * QM) * D + (size_t)half * 128 + row;
+            constexpr int dh = DH;
+            const bool d_ok = DH >= 128 || row < DH;  // lanes past a 64-wide head dimension hold zeros
+            float* dst = p.dq_acc + ((size_t)U.bh * (size_t)p.Sq + (size_t)m * QM) * dh + (size_t)half * 128 + row;
             const int nq = min(QM, p.Sq - m * QM);
             if (!p.dq_flags && L::DQ_BULK) {
                 // once the previous step's reduce has read the staging, copy dQ^T
@@ -1277,13 +763,17 @@ __device__ void bwd2_out_role(const BwdParams& p, uint8_t* smem, uint32_t tmem, 
                 const bool issuer = threadIdx.x == 2 * 128;  // first thread of the output warpgroup
                 if (issuer) bulk_wait_read();
                 if (!__all_sync(0xffffffffu, group_sync(76))) return;
+                // staging rows of min(dh, 128) values: the box of the dQ accumulator's map
+                constexpr int sstride = dh < 128 ? dh : 128;
                 float* stg = reinterpret_cast<float*>(smem + L::DQS_OFF) + row;
 #pragma unroll 1
                 for (int hh = 0; hh < 2; ++hh) {
                     uint32_t r[32];
                     tmem_ld32u(tmem + lane_sel + col2_dp(b) + 32 * hh, r);
+                    if (d_ok) {
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) stg[(32 * hh + j) * 128] = __uint_as_float(r[j]);
+                        for (int j = 0; j < 32; ++j) stg[(32 * hh + j) * sstride] = __uint_as_float(r[j]);
+                    }
                 }
                 tc_fence_before();
                 mbar_arrive(bar(L::B_DQEMPTY + b));
@@ -1299,10 +789,10 @@ __device__ void bwd2_out_role(const BwdParams& p, uint8_t* smem, uint32_t tmem, 
                 mbar_arrive(bar(L::B_DQEMPTY + b));
 #pragma unroll
                 for (int j = 0; j < 32; ++j)
-                    if (j < nq) atomicAdd(dst + (size_t)j * D, __uint_as_float(r0[j]));
+                    if (d_ok && j < nq) atomicAdd(dst + (size_t)j * dh, __uint_as_float(r0[j]));
 #pragma unroll
                 for (int j = 0; j < 32; ++j)
-                    if (32 + j < nq) atomicAdd(dst + (size_t)(32 + j) * D, __uint_as_float(r1[j]));
+                    if (d_ok && 32 + j < nq) atomicAdd(dst + (size_t)(32 + j) * dh, __uint_as_float(r1[j]));
             } else {
                 // this key tile's turn for the step, then 32 queries at a time:
                 // read-modify-write in batches of 16 (loads in flight together)
@@ -1322,12 +812,12 @@ __device__ void bwd2_out_role(const BwdParams& p, uint8_t* smem, uint32_t tmem, 
 #pragma unroll
                         for (int j = 0; j < 16; ++j) {
                             const int jq = 32 * hh + 16 * h + j;
-                            v[j] = jq < nq ? __ldcg(dst + (size_t)jq * D) : 0.f;
+                            v[j] = (d_ok && jq < nq) ? __ldcg(dst + (size_t)jq * dh) : 0.f;
                         }
 #pragma unroll
                         for (int j = 0; j < 16; ++j) {
                             const int jq = 32 * hh + 16 * h + j;
-                            if (jq < nq) __stcg(dst + (size_t)jq * D, v[j] + __uint_as_float(r[16 * h + j]));
+                            if (d_ok && jq < nq) __stcg(dst + (size_t)jq * dh, v[j] + __uint_as_float(r[16 * h + j]));
                         }
                     }
                 }
@@ -1343,14 +833,15 @@ __device__ void bwd2_out_role(const BwdParams& p, uint8_t* smem, uint32_t tmem, 
         // this unit's 128 columns of the dK and dV rows (its half of D at D = 256)
         uint8_t* dv_row = p.dv + ub * p.dv_s[0] + uh * p.dv_s[1] + kr * p.dv_s[2] + half * 256;
         uint8_t* dk_row = p.dk + ub * p.dk_s[0] + uh * p.dk_s[1] + kr * p.dk_s[2] + half * 256;
+        constexpr int ncol = DH < 128 ? DH : 128;  // this unit's columns of the rows
         if constexpr (SPLIT) {
             // this unit's share of the key row's sums (its half of D), added in fp32
-            const size_t acc_row = ((size_t)U.bh * KV_ACC_ROWS + (size_t)kr) * D + (size_t)half * 128;
-            kv_partial_add<128>(tmem + lane_sel + COL2_DV, tmem + lane_sel + COL2_DK, p.dv_acc + acc_row,
-                                p.dk_acc + acc_row, p.scale, valid);
+            const size_t acc_row = ((size_t)U.bh * KV_ACC_ROWS + (size_t)kr) * DH + (size_t)half * 128;
+            kv_partial_add(tmem + lane_sel + COL2_DV, tmem + lane_sel + COL2_DK, p.dv_acc + acc_row,
+                           p.dk_acc + acc_row, p.scale, valid, ncol);
         } else {
 #pragma unroll 1
-            for (int c = 0; c < 4; ++c) {
+            for (int c = 0; c < ncol / 32; ++c) {
                 uint32_t r[32];
                 uint32_t w[16];
                 tmem_ld32u(tmem + lane_sel + COL2_DV + 32 * c, r);
@@ -1377,7 +868,8 @@ __device__ void bwd2_out_role(const BwdParams& p, uint8_t* smem, uint32_t tmem, 
     }
 }
 
-template <int D, bool BF16, bool MASK, bool DROP, bool SPLIT = false>
+// DH: the tensors' head dimension (64: this D = 128 kernel on zero-padded operands)
+template <int D, bool BF16, bool MASK, bool DROP, bool SPLIT = false, int DH = D>
 __global__ void __launch_bounds__(BWD2_THREADS, 1) fa_bwd_kernel_wide(const __grid_constant__ BwdParams p) {
     using L = Bwd2Smem<D>;
     extern __shared__ uint8_t smem_raw[];
@@ -1426,7 +918,7 @@ __global__ void __launch_bounds__(BWD2_THREADS, 1) fa_bwd_kernel_wide(const __gr
         bwd2_ds_role<D, BF16, MASK, DROP>(p, smem, tmem, warp & 3, wg == 1 ? 0 : 1, abort_flag);
     } else {
         setmaxnreg_dec<Reg2<D>::OUT>();
-        bwd2_out_role<D, BF16, SPLIT>(p, smem, tmem, warp & 3, abort_flag);
+        bwd2_out_role<D, BF16, SPLIT, DH>(p, smem, tmem, warp & 3, abort_flag);
         // the bulk dQ reductions this thread issued finish before the CTA exits
         if (threadIdx.x == 2 * 128) bulk_wait_all();
     }
@@ -1555,7 +1047,6 @@ __global__ void __launch_bounds__(256) bwd_post_kv_kernel(const float4* __restri
 
 template <int D, bool BF16>
 cudaError_t launch_bwd_impl(const BwdLaunchArgs& a, cudaStream_t stream) {
-    static_assert(BwdSmem<64>::ALLOC <= 232448, "shared memory budget exceeded");
     static_assert(Bwd2Smem<128>::ALLOC <= 232448, "shared memory budget exceeded");
     static_assert(Bwd2Smem<256>::ALLOC <= 232448, "shared memory budget exceeded");
     const int BH = a.B * a.H;
@@ -1572,20 +1063,21 @@ cudaError_t launch_bwd_impl(const BwdLaunchArgs& a, cudaStream_t stream) {
         if (e != cudaSuccess) return e;
     }
     {
-        // D = 128 and 256 run the 64-row-step kernel (its Q/dO maps have 64-row boxes)
-        constexpr bool WIDE = D >= 128;
-        constexpr int DW = WIDE ? D : 128;
-        void (*kern)(const BwdParams);
-        if constexpr (WIDE)
-            kern = a.drop.enabled
-                       ? (a.mask ? fa_bwd_kernel_wide<DW, BF16, true, true> : fa_bwd_kernel_wide<DW, BF16, false, true>)
-                       : (a.mask ? fa_bwd_kernel_wide<DW, BF16, true, false>
-                                 : fa_bwd_kernel_wide<DW, BF16, false, false>);
-        else kern = fa_bwd_kernel<D, BF16>;
-        // the wide kernel adds split partial sums in its own instantiation, taken
+        // every head dimension runs the 64-row-step kernel (its Q/dO maps have
+        // 64-row boxes); D = 64 runs its D = 128 instantiation, whose loads of
+        // the second 64-column chunk read past D and fill with zeros, so the
+        // padding adds nothing to the scores, dK, dV or dQ
+        constexpr int DW = D >= 128 ? D : 128;
+        void (*kern)(const BwdParams) =
+            a.drop.enabled
+                ? (a.mask ? fa_bwd_kernel_wide<DW, BF16, true, true, false, D>
+                          : fa_bwd_kernel_wide<DW, BF16, false, true, false, D>)
+                : (a.mask ? fa_bwd_kernel_wide<DW, BF16, true, false, false, D>
+                          : fa_bwd_kernel_wide<DW, BF16, false, false, false, D>);
+        // split partial sums are added by their own instantiation, taken
         // without an explicit mask or dropout
-        const bool can_split = !WIDE || (!a.mask && !a.drop.enabled);
-        const int alloc = WIDE ? Bwd2Smem<DW>::ALLOC : BwdSmem<64>::ALLOC;
+        const bool can_split = !a.mask && !a.drop.enabled;
+        const int alloc = Bwd2Smem<DW>::ALLOC;
         cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(kern), alloc);
         if (e != cudaSuccess) return e;
         BwdParams p;
@@ -1608,11 +1100,12 @@ cudaError_t launch_bwd_impl(const BwdLaunchArgs& a, cudaStream_t stream) {
         p.Sq = a.Sq;
         p.Sk = a.Sk;
         p.Sq_pad = Sq_pad;
-        p.n_mtiles = WIDE ? (a.Sq + QM - 1) / QM : n_mtiles;
+        p.n_mtiles = (a.Sq + QM - 1) / QM;  // 64-row steps
         p.n_ktiles = (a.Sk + TILE - 1) / TILE;
-        p.n_units = BH * p.n_ktiles * (WIDE ? Bwd2Smem<DW>::HALVES : 1);
+        p.n_units = BH * p.n_ktiles * Bwd2Smem<DW>::HALVES;
         p.causal = a.causal;
         p.causal_off = a.Sk - a.Sq;
+        p.dh = D;
         {
             // heads whose Q, dO (16-bit) and dQ accumulator (fp32) take <= 48 MiB
             const long long per_head = (long long)a.Sq * D * 8;
@@ -1635,7 +1128,7 @@ cudaError_t launch_bwd_impl(const BwdLaunchArgs& a, cudaStream_t stream) {
         p.seed_hi = a.drop.seed_hi;
         p.drop_offset = a.drop.offset;
         p.keep_scale = a.drop.enabled ? a.drop.keep_scale : 1.f;
-        p.flag_steps = WIDE ? (a.Sq + QM - 1) / QM : n_mtiles;
+        p.flag_steps = (a.Sq + QM - 1) / QM;
         // Split query range: a key set of at most KV_ACC_ROWS keys (one key tile)
         // whose units leave SMs idle takes chunks of q_chunk steps per unit, about
         // two units per SM; not in deterministic mode (the fp32 adds of the
@@ -1651,11 +1144,9 @@ cudaError_t launch_bwd_impl(const BwdLaunchArgs& a, cudaStream_t stream) {
             p.q_chunk = (p.n_mtiles + want - 1) / want;
             p.q_split = (p.n_mtiles + p.q_chunk - 1) / p.q_chunk;      // no chunk is empty
             if (p.q_split > 1) {
-                if constexpr (WIDE) {
-                    kern = fa_bwd_kernel_wide<DW, BF16, false, false, true>;
-                    e = ensure_smem_limit(reinterpret_cast<const void*>(kern), alloc);
-                    if (e != cudaSuccess) return e;
-                }
+                kern = fa_bwd_kernel_wide<DW, BF16, false, false, true, D>;
+                e = ensure_smem_limit(reinterpret_cast<const void*>(kern), alloc);
+                if (e != cudaSuccess) return e;
                 p.n_units *= p.q_split;
                 grid = p.n_units < a.sms ? p.n_units : a.sms;
                 const size_t bytes = (size_t)BH * KV_ACC_ROWS * D * sizeof(float);
@@ -1668,7 +1159,7 @@ cudaError_t launch_bwd_impl(const BwdLaunchArgs& a, cudaStream_t stream) {
         }
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3((unsigned)grid, 1, 1);
-        cfg.blockDim = dim3(WIDE ? BWD2_THREADS : BWD_THREADS, 1, 1);
+        cfg.blockDim = dim3(BWD2_THREADS, 1, 1);
         cfg.dynamicSmemBytes = alloc;
         cfg.stream = stream;
         e = cudaLaunchKernelEx(&cfg, kern, p);
