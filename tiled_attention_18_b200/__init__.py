@@ -26,13 +26,28 @@ __all__ = [
 ]
 
 
+_DTYPE_CODES = None
+
+
 def _dtype_code(t) -> int:
+    global _DTYPE_CODES
+    if _DTYPE_CODES is None:
+        import torch
+        _DTYPE_CODES = {torch.float16: FA_FP16, torch.bfloat16: FA_BF16}
+    code = _DTYPE_CODES.get(t.dtype)
+    if code is None:
+        raise TypeError(f"unsupported dtype {t.dtype}; expected float16 or bfloat16")
+    return code
+
+
+def _current_stream_handle(device) -> int:
+    """The raw handle of torch's current stream on ``device`` (a plain int, without
+    building a torch Stream object on every call when torch exposes it)."""
     import torch
-    if t.dtype == torch.float16:
-        return FA_FP16
-    if t.dtype == torch.bfloat16:
-        return FA_BF16
-    raise TypeError(f"unsupported dtype {t.dtype}; expected float16 or bfloat16")
+    raw = getattr(torch._C, "_cuda_getCurrentRawStream", None)
+    if raw is not None:
+        return int(raw(device.index if device.index is not None else torch.cuda.current_device()))
+    return int(torch.cuda.current_stream(device).cuda_stream)
 
 
 def _mask_stride(mask, B, H, Sq, Sk):
@@ -91,9 +106,7 @@ def flash_attention_forward(q, k, v, scale: float, causal: bool = False, out=Non
         raise ValueError("out must be like q, contiguous in its last dimension")
     if lse.shape != (B, H, Sq) or lse.dtype != torch.float32 or not lse.is_contiguous():
         raise ValueError("lse must be a contiguous float32 [B, H, Sq] tensor")
-    if stream is None:
-        stream = torch.cuda.current_stream(q.device)
-    st = int(stream.cuda_stream)
+    st = _current_stream_handle(q.device) if stream is None else int(stream.cuda_stream)
     dt = _dtype_code(q)
     if dropout_p != 0.0 or mask is not None or block_n or q_tiles:
         rc = fa_forward(st, q=q.data_ptr(), k=k.data_ptr(), v=v.data_ptr(), o=out.data_ptr(), lse=lse.data_ptr(),
@@ -148,12 +161,11 @@ def flash_attention_backward(q, k, v, o, lse, dout, scale: float, causal: bool =
         raise FaError(nbytes, "fa_bwd_workspace_size")
     if workspace is None:
         workspace = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=q.device)
-    if stream is None:
-        stream = torch.cuda.current_stream(q.device)
+    sid = _current_stream_handle(q.device) if stream is None else int(stream.cuda_stream)
     tensors = (q, k, v, o, dout, dq, dk, dv)
     if dropout_p != 0.0 or mask is not None:
         names = ("q", "k", "v", "o", "dout", "dq", "dk", "dv")
-        rc = fa_backward(int(stream.cuda_stream), **{n: t.data_ptr() for n, t in zip(names, tensors)},
+        rc = fa_backward(sid, **{n: t.data_ptr() for n, t in zip(names, tensors)},
                          lse=lse.data_ptr(), workspace=workspace.data_ptr(), workspace_bytes=workspace.numel(),
                          B=B, H=H, Sq=Sq, Sk=Sk, D=D,
                          **{("do" if n == "dout" else n) + "_stride": t.stride()[:3] for n, t in zip(names, tensors)},
@@ -168,7 +180,7 @@ def flash_attention_backward(q, k, v, o, lse, dout, scale: float, causal: bool =
         rc = fa_bwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), dout.data_ptr(), lse.data_ptr(),
                        dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), workspace.data_ptr(), workspace.numel(), B, H, Sq,
                        Sk, D, *(t.stride()[:3] for t in tensors), float(scale), int(bool(causal)),
-                       int(bool(deterministic)), _dtype_code(q), int(stream.cuda_stream))
+                       int(bool(deterministic)), _dtype_code(q), sid)
         if rc != 0:
             raise FaError(rc, "fa_bwd_ex")
         return dq, dk, dv
@@ -176,13 +188,13 @@ def flash_attention_backward(q, k, v, o, lse, dout, scale: float, causal: bool =
         rc = fa_bwd_dropout(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), dout.data_ptr(), lse.data_ptr(),
                             dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), workspace.data_ptr(), workspace.numel(), B, H,
                             Sq, Sk, D, float(scale), int(bool(causal)), float(dropout_p), int(seed), int(offset),
-                            int(bool(deterministic)), _dtype_code(q), int(stream.cuda_stream))
+                            int(bool(deterministic)), _dtype_code(q), sid)
         if rc != 0:
             raise FaError(rc, "fa_bwd_dropout")
         return dq, dk, dv
     rc = fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), dout.data_ptr(), lse.data_ptr(),
                 dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), workspace.data_ptr(), workspace.numel(), B, H, Sq, Sk, D,
-                float(scale), int(bool(causal)), int(bool(deterministic)), _dtype_code(q), int(stream.cuda_stream))
+                float(scale), int(bool(causal)), int(bool(deterministic)), _dtype_code(q), sid)
     if rc != 0:
         raise FaError(rc, "fa_bwd")
     return dq, dk, dv
