@@ -5,7 +5,7 @@
                     [--pass fwd|bwd|sp] [--mask tril] [--dropout P] [--deterministic]
                     [--block-n 64|128] [--q-tiles 1|2]
                     [--sp-world W] [--sp-mode ring|allgather|ulysses]
-                    [--no-e2e] [--no-cpu-baseline] [--cpu-seconds S]
+                    [--no-e2e] [--e2e-chunks C] [--no-cpu-baseline] [--cpu-seconds S]
 
 A step is one pass of the whole forward path over one batch of synthetic
 input.  The default workload is the long-context configuration
@@ -32,6 +32,13 @@ flops; BSHD workloads through fa_bwd_ex), ``--pass sp`` every rank's
 sequence-parallel schedule run in turn on one GPU.  ``--mask tril`` runs the
 causal case as an explicit lower-triangular mask, ``--dropout P`` adds
 attention dropout (a fresh offset per step).
+
+The end-to-end figure ("e2e") times steps through the same public calls with
+pinned host buffers: each step uploads its inputs and downloads O and LSE.
+The forward pass splits each step into chunks of whole batches (or heads of
+a single batch) and pipelines them over three streams, so that the copies
+in both directions overlap the kernels; the downloaded results are checked
+bit for bit against one launch over all heads.
 
 ``--impl reference`` times the fp64 CPU oracle on bounded samples of the
 same workload and pass (rank 0 only) and prints the same JSON line with
@@ -463,13 +470,67 @@ def run_bwd(args) -> int:
         h2d = sum(hb[n].numel() * hb[n].element_size() for hb in host for n in names_in)
         d2h = sum(hb[n].numel() * hb[n].element_size() for hb in host for n in names_out)
 
-        def e2e_step():
-            for i, (hb, b) in enumerate(zip(host, bufs)):
-                for n in names_in:
-                    b[n].copy_(hb[n], non_blocking=True)
+        # chunks of whole batches (or heads of a single BHSD batch) pipelined
+        # over three streams, as in the forward pass; dropout keeps one chunk
+        # (its keep decisions are drawn per absolute head index)
+        def chunk_plan(w):
+            if args.dropout > 0.0 or args.e2e_chunks <= 1:
+                return 0, [(0, w.B)]
+            if w.B > 1:
+                n, ax, total = min(args.e2e_chunks, w.B), 0, w.B
+            elif w.layout == "bhsd":
+                n, ax, total = min(args.e2e_chunks, w.H), 1, w.H
+            else:
+                return 0, [(0, w.B)]
+            edges = [total * c // n for c in range(n + 1)]
+            return ax, [(edges[c], edges[c + 1] - edges[c]) for c in range(n)]
+
+        plans = [chunk_plan(w) for w in runs]
+        up_s, dn_s = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        ev_up = [[torch.cuda.Event() for _ in p[1]] for p in plans]
+        ev_k = [[torch.cuda.Event() for _ in p[1]] for p in plans]
+        n_chunk_max = max(len(p[1]) for p in plans)
+
+        def launch_chunk(i, ax, a, n):
+            w, b = runs[i], bufs[i]
+            if len(plans[i][1]) == 1:
                 launch(i)
-                for n in names_out:
-                    hb[n].copy_(b[n], non_blocking=True)
+                return
+            names = ("q", "k", "v", "o", "dout", "dq", "dk", "dv")
+            t = {nm: b[nm].narrow(ax, a, n) for nm in names + ("lse",)}
+            st = fa.fa_bwd_ex(*(t[nm].data_ptr() for nm in names[:5]), t["lse"].data_ptr(),
+                              *(t[nm].data_ptr() for nm in names[5:]), b["ws"].data_ptr(), b["nbytes"],
+                              t["q"].shape[0], t["q"].shape[1], w.S, w.Skv, w.D,
+                              *(t[nm].stride()[:3] for nm in names), w.scale, int(w.causal), int(args.deterministic),
+                              b["dt"], sid)
+            if st != 0:
+                raise fa.FaError(st, "fa_bwd_ex")
+
+        def e2e_step():
+            start_ev = torch.cuda.Event()
+            start_ev.record(stream)
+            up_s.wait_event(start_ev)
+            dn_s.wait_event(start_ev)
+            for c in range(n_chunk_max):
+                for i, (hb, b) in enumerate(zip(host, bufs)):
+                    ax, rng = plans[i]
+                    if c >= len(rng):
+                        continue
+                    a, n = rng[c]
+                    with torch.cuda.stream(up_s):
+                        for nm in names_in:
+                            b[nm].narrow(ax, a, n).copy_(hb[nm].narrow(ax, a, n), non_blocking=True)
+                    ev_up[i][c].record(up_s)
+                    stream.wait_event(ev_up[i][c])
+                    launch_chunk(i, ax, a, n)
+                    ev_k[i][c].record(stream)
+                    dn_s.wait_event(ev_k[i][c])
+                    with torch.cuda.stream(dn_s):
+                        for nm in names_out:
+                            hb[nm].narrow(ax, a, n).copy_(b[nm].narrow(ax, a, n), non_blocking=True)
+            done_ev = torch.cuda.Event()
+            done_ev.record(dn_s)
+            stream.wait_event(done_ev)
 
         for _ in range(2):
             e2e_step()
@@ -482,7 +543,20 @@ def run_bwd(args) -> int:
         torch.cuda.synchronize(dev)
         e2e = {"value": job_throughput(step_flops, args.e2e_steps, world,
                                        max_over_ranks(e0.elapsed_time(e1), device=dev)),
-               "unit": UNIT, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+               "unit": UNIT, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+               "overlap": (f"{n_chunk_max} chunks per step; uploads, launches and downloads on three streams"
+                           if n_chunk_max > 1 else "none")}
+        # the chunked gradients against one launch over all heads (fp32 sums
+        # of dQ, and of split dK/dV, may add in another order)
+        for i in range(len(runs)):
+            launch(i)
+        torch.cuda.synchronize(dev)
+        for i, (hb, b) in enumerate(zip(host, bufs)):
+            for nm in names_out:
+                ref = b[nm].float().cpu()
+                err = float((hb[nm].float() - ref).abs().max())
+                if not err <= 0.02 * float(ref.abs().max()) + 1e-6:
+                    raise SystemExit(f"end-to-end {nm} of run {i} differs from a whole launch by {err}")
     cb = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cb = cpu_baseline_bwd(args.workload, dropout=args.dropout)
@@ -680,6 +754,9 @@ def main(argv=None) -> int:
     ap.add_argument("--impl", choices=["fa", "reference"], default="fa")
     ap.add_argument("--workload", default="c5", choices=["c5"] + list(ALL_WORKLOADS))
     ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--e2e-chunks", type=int, default=8,
+                    help="chunks (batches, or heads of a single batch) per end-to-end step, pipelined over "
+                         "three streams (upload, launches, download)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extra", action="store_true",
@@ -922,15 +999,73 @@ def main(argv=None) -> int:
                   if i == 0 or host_in[i] is not host_in[0])
         d2h = sum(o.numel() * o.element_size() + l.numel() * l.element_size() for (o, l) in host_out)
 
-        def e2e_step():
-            for i, w in enumerate(runs):
-                if i == 0 or host_in[i] is not host_in[0]:
-                    for hsrc, dsrc in zip(host_in[i], dev_in[i][0]):
-                        dsrc.copy_(hsrc, non_blocking=True)
+        # The heads are independent problems: each step uploads its inputs in
+        # chunks (whole batches, or heads of a single batch: contiguous ranges
+        # of every storage tensor) on one stream, runs each chunk's launches on
+        # the timing stream once its upload has landed, and downloads each
+        # chunk's O and LSE on a third stream once its launches are done, so
+        # the copies in both directions overlap the kernels.  A step starts
+        # after the previous step's last download: nothing is shared across
+        # steps.
+        plain = args.dropout == 0.0 and not tril and not args.block_n and not args.q_tiles
+        n_chunks = max(1, args.e2e_chunks) if plain else 1
+
+        def chunk_plan(w):
+            if w.B > 1:
+                n, ax_s, ax_l, total = min(n_chunks, w.B), 0, 0, w.B
+            else:
+                n, ax_s, ax_l, total = min(n_chunks, w.H), (1 if w.layout == "bhsd" else 2), 1, w.H
+            edges = [total * c // n for c in range(n + 1)]
+            return ax_s, ax_l, [(edges[c], edges[c + 1] - edges[c]) for c in range(n)]
+
+        plans = [chunk_plan(w) for w in runs]
+        n_steps_chunk = max(len(p[2]) for p in plans)
+        up_s, dn_s = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        ev_up = [[torch.cuda.Event() for _ in p[2]] for p in plans]
+        ev_k = [[torch.cuda.Event() for _ in p[2]] for p in plans]
+
+        def launch_chunk(i, ax_s, ax_l, a, n):
+            w = runs[i]
+            if len(plans[i][2]) == 1:
                 launch(i)
-                dev_out_o, dev_out_l = dev_out[i]
-                host_out[i][0].copy_(dev_out_o, non_blocking=True)
-                host_out[i][1].copy_(dev_out_l, non_blocking=True)
+                return
+            q, k, v = (view(w, t.narrow(ax_s, a, n)) for t in dev_in[i][0])
+            o = view(w, dev_out[i][0].narrow(ax_s, a, n))
+            lse = dev_out[i][1].narrow(ax_l, a, n)
+            dt = fa.FA_BF16 if w.dtype == "bf16" else fa.FA_FP16
+            st = fa.fa_fwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), q.shape[0],
+                              q.shape[1], w.S, w.Skv, w.D, q.stride()[:3], k.stride()[:3], v.stride()[:3],
+                              o.stride()[:3], w.scale, int(w.causal), dt, sid)
+            if st != 0:
+                raise fa.FaError(st)
+
+        def e2e_step():
+            start = torch.cuda.Event()
+            start.record(stream)
+            up_s.wait_event(start)
+            dn_s.wait_event(start)
+            for c in range(n_steps_chunk):
+                for i in range(len(runs)):
+                    ax_s, ax_l, rng = plans[i]
+                    if c >= len(rng):
+                        continue
+                    a, n = rng[c]
+                    owner = 0 if (i > 0 and host_in[i] is host_in[0]) else i
+                    if owner == i:
+                        with torch.cuda.stream(up_s):
+                            for hsrc, dsrc in zip(host_in[i], dev_in[i][0]):
+                                dsrc.narrow(ax_s, a, n).copy_(hsrc.narrow(ax_s, a, n), non_blocking=True)
+                        ev_up[i][c].record(up_s)
+                    stream.wait_event(ev_up[owner][c])
+                    launch_chunk(i, ax_s, ax_l, a, n)
+                    ev_k[i][c].record(stream)
+                    dn_s.wait_event(ev_k[i][c])
+                    with torch.cuda.stream(dn_s):
+                        host_out[i][0].narrow(ax_s, a, n).copy_(dev_out[i][0].narrow(ax_s, a, n), non_blocking=True)
+                        host_out[i][1].narrow(ax_l, a, n).copy_(dev_out[i][1].narrow(ax_l, a, n), non_blocking=True)
+            done = torch.cuda.Event()
+            done.record(dn_s)
+            stream.wait_event(done)
 
         for _ in range(2):
             e2e_step()
@@ -944,7 +1079,17 @@ def main(argv=None) -> int:
         torch.cuda.synchronize(dev)
         barrier()
         e2e_val = job_throughput(step_flops, args.e2e_steps, world, max_over_ranks(e0.elapsed_time(e1), device=dev))
-        e2e = {"value": e2e_val, "unit": UNIT, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+        e2e = {"value": e2e_val, "unit": UNIT, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+               "overlap": (f"{n_steps_chunk} chunks per step; uploads, launches and downloads on three streams"
+                           if n_steps_chunk > 1 else "none")}
+        # the chunked launches compute each head exactly as one launch over all
+        # heads does: the downloaded results equal a whole launch's bit for bit
+        for i in range(len(runs)):
+            launch(i)
+        torch.cuda.synchronize(dev)
+        for i in range(len(runs)):
+            if not (torch.equal(host_out[i][0], dev_out[i][0].cpu()) and torch.equal(host_out[i][1], dev_out[i][1].cpu())):
+                raise SystemExit(f"end-to-end results of run {i} differ from a whole launch")
 
     cb = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
