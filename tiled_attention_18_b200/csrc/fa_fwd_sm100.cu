@@ -117,9 +117,9 @@ constexpr uint32_t COL_S1 = 128;
 constexpr uint32_t COL_O0 = 256;
 constexpr uint32_t COL_O1 = 384;
 
-// Shared-memory layout for head dimension D, key tiles of BN rows and QT query
-// tiles of BLOCK_M rows per work unit.
-template <int D, int BN = BLOCK_N, int QT = Q_TILES_PER_CTA>
+// Shared-memory layout for head dimension D, key tiles of BN rows, QT query
+// tiles of BLOCK_M rows per work unit and NQB_ Q buffers.
+template <int D, int BN = BLOCK_N, int QT = Q_TILES_PER_CTA, int NQB_ = 1>
 struct Smem {
     static constexpr int CHUNKS = D / 64;                  // 128-byte swizzle atoms along D
     static constexpr int Q_CHUNK_BYTES = BLOCK_M * 128;    // 128 rows x 128 bytes
@@ -135,8 +135,14 @@ struct Smem {
     static constexpr int NSTAGE = (128 * 1024) / STAGE_BYTES;
     static constexpr int STAGE_K = 0;                      // offset of K_s in a stage
     static constexpr int STAGE_V = KV_TILE_BYTES;          // offset of V_{s-1}
+    // Q buffers: with two (D = 64 only: at D = 128 the K/V ring needs the
+    // bytes) the next unit's Q loads while this unit's last key tiles run, and
+    // the next unit's first S is issued before this unit's last P.V
+    static constexpr int NQB = NQB_;
+    static_assert(NQB == 1 || (NQB == 2 && D == 64), "two Q buffers fit at D = 64 only");
+    static constexpr int QBUF_BYTES = QT * Q_TILE_BYTES;
     static constexpr int Q_OFF = 0;
-    static constexpr int KV_OFF = Q_OFF + QT * Q_TILE_BYTES;
+    static constexpr int KV_OFF = Q_OFF + NQB * QBUF_BYTES;
     // per-row values handed from the softmax to the correction warpgroup
     static constexpr int ALPHA_OFF = KV_OFF + NSTAGE * STAGE_BYTES;   // float [2][128]
     // float2 [unit parity][tile][row] = (1/l, lse); double-buffered because a
@@ -146,9 +152,9 @@ struct Smem {
     static constexpr int FIN_OFF = ALPHA_OFF + 2 * BLOCK_M * 4;
     static constexpr int BAR_OFF = FIN_OFF + 2 * 2 * BLOCK_M * 8;
     // barrier indices
-    static constexpr int B_QFULL = 0;
-    static constexpr int B_QEMPTY = 1;
-    static constexpr int B_STFULL = 2;                     // [NSTAGE] TMA -> MMA
+    static constexpr int B_QFULL = 0;                      // [NQB] TMA -> MMA
+    static constexpr int B_QEMPTY = NQB;                   // [NQB] MMA -> TMA: the unit's last S issued
+    static constexpr int B_STFULL = 2 * NQB;               // [NSTAGE] TMA -> MMA
     static constexpr int B_STEMPTY = B_STFULL + NSTAGE;    // [NSTAGE] MMA -> TMA
     static constexpr int B_SFULL = B_STEMPTY + NSTAGE;     // [2] MMA -> softmax: S_t ready
     // [2] softmax + correction -> MMA: P_t written and O_t ready for it (rescaled,
@@ -320,12 +326,12 @@ __device__ __forceinline__ Unit decode_unit(const KParams& p, int u) {
 
 // Reads the work-unit indices published by the TMA lane, in order.
 // next() returns the unit, -1 when the CTA has no more work, -2 on abort.
-template <int D, int BN, int QT>
+template <int D, int BN, int QT, int NQB>
 struct UnitReader {
     int slot = 0;
     uint32_t phase = 0;
     __device__ __forceinline__ int next(uint8_t* smem, volatile uint32_t* abort_flag, int site) {
-        using L = Smem<D, BN, QT>;
+        using L = Smem<D, BN, QT, NQB>;
         const uint32_t bar0 = smem_u32(smem) + L::BAR_OFF;
         if (!mbar_wait(bar0 + 8u * (uint32_t)(L::B_UFULL + slot), phase, abort_flag, site)) return -2;
         const int u = reinterpret_cast<volatile int*>(smem + L::UNIT_OFF)[slot];
@@ -335,18 +341,19 @@ struct UnitReader {
     }
 };
 
-template <int D, int BN, int QT>
+template <int D, int BN, int QT, int NQB>
 __device__ void producer_role(const KParams& p, uint8_t* smem, volatile uint32_t* abort_flag) {
-    using L = Smem<D, BN, QT>;
+    using L = Smem<D, BN, QT, NQB>;
     const uint32_t base = smem_u32(smem);
     const uint32_t bar0 = base + L::BAR_OFF;
     auto bar = [&](int i) { return bar0 + 8u * (uint32_t)i; };
     int stage = 0;
     uint32_t phase = 0;
-    uint32_t qe_phase = 0;
+    int qk = 0;                  // Q fills issued
+    uint32_t q_fill_mask = 0;    // Q buffers with a fill issued
+    uint32_t q_fill_parity = 0;  // parity of each Q buffer's last fill
     uint32_t fill_mask = 0;    // stages with a fill issued
     uint32_t fill_parity = 0;  // parity of each stage's last fill
-    int last_q_fill = -1;
     bool ok = true;
     volatile int* ring = reinterpret_cast<volatile int*>(smem + L::UNIT_OFF);
     int uslot = 0;
@@ -368,18 +375,22 @@ __device__ void producer_role(const KParams& p, uint8_t* smem, volatile uint32_t
         if (u < 0) break;
         const Unit U = decode_unit<BN, QT>(p, u);
         const int ub = U.bh / p.H, uh = U.bh - ub * p.H;  // tensor-map coordinates of the head
-        if (!mbar_wait(bar(L::B_QEMPTY), qe_phase ^ 1u, abort_flag, 1)) { ok = false; break; }
-        qe_phase ^= 1u;
+        // Q buffer of this unit: fill number qk of the CTA goes to buffer qk mod NQB
+        const int qb = qk % L::NQB;
+        const uint32_t qph = (uint32_t)(qk / L::NQB) & 1u;
+        ++qk;
+        if (!mbar_wait(bar(L::B_QEMPTY + qb), qph ^ 1u, abort_flag, 1)) { ok = false; break; }
         const uint32_t qbytes = (U.n[0] > 0 ? L::Q_TILE_BYTES : 0) + (U.n[1] > 0 ? L::Q_TILE_BYTES : 0);
-        mbar_expect_tx(bar(L::B_QFULL), qbytes);
-        last_q_fill = (int)(qe_phase ^ 1u);  // parity of the q_full phase this fill completes
+        mbar_expect_tx(bar(L::B_QFULL + qb), qbytes);
+        q_fill_mask |= 1u << qb;
+        q_fill_parity = (q_fill_parity & ~(1u << qb)) | (qph << qb);
 #pragma unroll
         for (int t = 0; t < 2; ++t) {
             if (U.n[t] == 0) continue;
-            const uint32_t dst = base + L::Q_OFF + t * L::Q_TILE_BYTES;
+            const uint32_t dst = base + L::Q_OFF + qb * L::QBUF_BYTES + t * L::Q_TILE_BYTES;
 #pragma unroll
             for (int c = 0; c < L::CHUNKS; ++c)
-                tma_load_4d(dst + c * L::Q_CHUNK_BYTES, &p.tmap_q, bar(L::B_QFULL), c * 64, U.q0[t], uh, ub);
+                tma_load_4d(dst + c * L::Q_CHUNK_BYTES, &p.tmap_q, bar(L::B_QFULL + qb), c * 64, U.q0[t], uh, ub);
         }
         // stages 0..N: stage s = (V_{s-1} if s >= 1, K_s if s < N)
         for (int st = 0; st <= U.N; ++st) {
@@ -408,13 +419,14 @@ __device__ void producer_role(const KParams& p, uint8_t* smem, volatile uint32_t
         // drain the copies this thread issued before leaving
         for (int i = 0; i < L::NSTAGE; ++i)
             if (fill_mask & (1u << i)) mbar_drain(bar(L::B_STFULL + i), (fill_parity >> i) & 1u);
-        if (last_q_fill >= 0) mbar_drain(bar(L::B_QFULL), (uint32_t)last_q_fill);
+        for (int i = 0; i < L::NQB; ++i)
+            if (q_fill_mask & (1u << i)) mbar_drain(bar(L::B_QFULL + i), (q_fill_parity >> i) & 1u);
     }
 }
 
-template <int D, bool BF16, int BN, int QT>
+template <int D, bool BF16, int BN, int QT, int NQB>
 __device__ void mma_role(const KParams& p, uint8_t* smem, uint32_t tmem, volatile uint32_t* abort_flag) {
-    using L = Smem<D, BN, QT>;
+    using L = Smem<D, BN, QT, NQB>;
     const uint32_t base = smem_u32(smem);
     const uint32_t bar0 = base + L::BAR_OFF;
     auto bar = [&](int i) { return bar0 + 8u * (uint32_t)i; };
@@ -443,8 +455,9 @@ __device__ void mma_role(const KParams& p, uint8_t* smem, uint32_t tmem, volatil
     constexpr uint32_t TILE16 = (uint32_t)L::Q_TILE_BYTES >> 4;
 
     constexpr uint32_t STAGE16 = (uint32_t)L::STAGE_BYTES >> 4;
+    uint32_t qbuf16 = 0;  // this unit's Q buffer offset (16-byte units)
     auto issue_s = [&](int t, int st) {
-        const uint32_t a_lo = dq_lo + (uint32_t)t * TILE16;
+        const uint32_t a_lo = dq_lo + qbuf16 + (uint32_t)t * TILE16;
         const uint32_t b_lo = dk_lo + (uint32_t)st * STAGE16 + ((uint32_t)L::STAGE_K >> 4);
         const uint32_t d_tmem = tmem + (t == 0 ? COL_S0 : COL_S1);
 #pragma unroll
@@ -467,7 +480,7 @@ __device__ void mma_role(const KParams& p, uint8_t* smem, uint32_t tmem, volatil
 
     int stage = 0;
     uint32_t phase = 0;
-    uint32_t qf_phase = 0;
+    int qk = 0;  // units whose Q was used
     uint32_t p_phase[2] = {0u, 0u};
     bool ok = true;
 
@@ -497,20 +510,31 @@ __device__ void mma_role(const KParams& p, uint8_t* smem, uint32_t tmem, volatil
         if (++stage == L::NSTAGE) { stage = 0; phase ^= 1u; }
         return st;
     };
-    UnitReader<D, BN, QT> units;
-    for (;;) {
-        const int u = units.next(smem, abort_flag, 32);
-        if (u < 0) break;
-        const Unit U = decode_unit<BN, QT>(p, u);
-        const bool tile1_last = U.n[1] == U.N;  // which tile issues the unit's last S
-        if (!mbar_wait(bar(L::B_QFULL), qf_phase, abort_flag, 3)) { ok = false; break; }
-        qf_phase ^= 1u;
-        // prologue: stage 0 (K_0), S0 = Q0 K_0^T
-        int cur = wait_stage(4);
-        if (cur < 0) { ok = false; break; }
-        issue_s(0, cur);
+    // A unit's prologue: its Q, stage 0 (K_0), S0 = Q0 K_0^T.
+    auto start_unit = [&](const Unit& Un, int& cur_out, int& qb_out) -> bool {
+        const int qbn = qk % L::NQB;
+        if (!mbar_wait(bar(L::B_QFULL + qbn), (uint32_t)(qk / L::NQB) & 1u, abort_flag, 3)) return false;
+        ++qk;
+        qbuf16 = (uint32_t)(qbn * L::QBUF_BYTES) >> 4;
+        const int c0 = wait_stage(4);
+        if (c0 < 0) return false;
+        issue_s(0, c0);
         tc_commit(bar(L::B_SFULL + 0));
-        if (U.N == 1 && !tile1_last) tc_commit(bar(L::B_QEMPTY));
+        if (Un.N == 1 && Un.n[1] != Un.N) tc_commit(bar(L::B_QEMPTY + qbn));
+        cur_out = c0;
+        qb_out = qbn;
+        return true;
+    };
+    UnitReader<D, BN, QT, NQB> units;
+    int u = units.next(smem, abort_flag, 32);
+    Unit U{};
+    int cur = -1, qb = 0;
+    if (u >= 0) {
+        U = decode_unit<BN, QT>(p, u);
+        if (!start_unit(U, cur, qb)) ok = false;
+    }
+    while (ok && u >= 0) {
+        const bool tile1_last = U.n[1] == U.N;  // which tile issues the unit's last S
         for (int j = 0; j < U.N; ++j) {
             // ---- tile 1 on stage j: O1 += P1 V_{j-1}, S1 = Q1 K_j^T
             if (j >= 1 && j - 1 < U.n[1]) {
@@ -522,7 +546,7 @@ __device__ void mma_role(const KParams& p, uint8_t* smem, uint32_t tmem, volatil
                 tc_commit(bar(L::B_SFULL + 1));
             }
             tc_commit(bar(L::B_STEMPTY + cur));  // V_{j-1} and K_j: last readers issued
-            if (j == U.N - 1 && tile1_last) tc_commit(bar(L::B_QEMPTY));
+            if (j == U.N - 1 && tile1_last) tc_commit(bar(L::B_QEMPTY + qb));
             // ---- tile 0 on stage j+1: O0 += P0 V_j, S0 = Q0 K_{j+1}^T
             const int nxt = wait_stage(6);
             if (nxt < 0) { ok = false; break; }
@@ -534,28 +558,50 @@ __device__ void mma_role(const KParams& p, uint8_t* smem, uint32_t tmem, volatil
             if (j + 1 < U.n[0]) {
                 issue_s(0, nxt);
                 tc_commit(bar(L::B_SFULL + 0));
-                if (j + 1 == U.N - 1 && !tile1_last) tc_commit(bar(L::B_QEMPTY));
+                if (j + 1 == U.N - 1 && !tile1_last) tc_commit(bar(L::B_QEMPTY + qb));
             }
             cur = nxt;
         }
         if (!ok) break;
-        // stage N holds V_{N-1}: O1 += P1 V_{N-1}, then release it
-        if (U.n[1] > 0) {
-            if (!wait_pv_inputs(1, 12)) { ok = false; break; }
-            issue_pv(1, cur, U.N - 1 > 0);
-            tc_commit(bar(L::B_OFULL + 1));
+        // stage N holds V_{N-1}: O1 += P1 V_{N-1}, then release it.  With two Q
+        // buffers the next unit's first S goes first, so that its tile 0 starts
+        // while this unit's tile 1 finishes (as between key tiles of a unit).
+        auto finish_unit = [&]() -> bool {
+            if (U.n[1] > 0) {
+                if (!wait_pv_inputs(1, 12)) return false;
+                issue_pv(1, cur, U.N - 1 > 0);
+                tc_commit(bar(L::B_OFULL + 1));
+            }
+            tc_commit(bar(L::B_STEMPTY + cur));
+            return true;
+        };
+        if constexpr (L::NQB == 1) {
+            if (!finish_unit()) { ok = false; break; }
         }
-        tc_commit(bar(L::B_STEMPTY + cur));
+        const int u2 = units.next(smem, abort_flag, 32);
+        Unit U2{};
+        int cur2 = -1, qb2 = 0;
+        if (u2 >= 0) {
+            U2 = decode_unit<BN, QT>(p, u2);
+            if (!start_unit(U2, cur2, qb2)) { ok = false; break; }
+        }
+        if constexpr (L::NQB == 2) {
+            if (!finish_unit()) { ok = false; break; }
+        }
+        u = u2;
+        U = U2;
+        cur = cur2;
+        qb = qb2;
     }
     // all MMAs issued by this thread have completed once B_FIN fires
     tc_commit(bar(L::B_FIN));
     mbar_drain(bar(L::B_FIN), 0u);
 }
 
-template <int D, bool BF16, bool MASK, bool DROP, int BN, int QT>
+template <int D, bool BF16, bool MASK, bool DROP, int BN, int QT, int NQB>
 __device__ void softmax_role(const KParams& p, uint8_t* smem, uint32_t tmem, int t, int warp_in_group,
                              volatile uint32_t* abort_flag) {
-    using L = Smem<D, BN, QT>;
+    using L = Smem<D, BN, QT, NQB>;
     static_assert(BN == BLOCK_N || (!MASK && !DROP), "the mask and dropout paths take 128-key tiles");
     const uint32_t base = smem_u32(smem);
     const uint32_t bar0 = base + L::BAR_OFF;
@@ -571,7 +617,7 @@ __device__ void softmax_role(const KParams& p, uint8_t* smem, uint32_t tmem, int
     const float2 sl2x2 = make_float2(sl2, sl2);
 
     uint32_t s_phase = 0;
-    UnitReader<D, BN, QT> units;
+    UnitReader<D, BN, QT, NQB> units;
     for (;;) {
         const int u = units.next(smem, abort_flag, 33);
         if (!__all_sync(0xffffffffu, u != -2)) return;
@@ -703,10 +749,10 @@ __device__ void softmax_role(const KParams& p, uint8_t* smem, uint32_t tmem, int
     }
 }
 
-template <int D, bool BF16, int BN, int QT>
+template <int D, bool BF16, int BN, int QT, int NQB>
 __device__ void correction_role(const KParams& p, uint8_t* smem, uint32_t tmem, int warp_in_group,
                                 volatile uint32_t* abort_flag) {
-    using L = Smem<D, BN, QT>;
+    using L = Smem<D, BN, QT, NQB>;
     const uint32_t base = smem_u32(smem);
     const uint32_t bar0 = base + L::BAR_OFF;
     auto bar = [&](int i) { return bar0 + 8u * (uint32_t)i; };
@@ -792,7 +838,7 @@ __device__ void correction_role(const KParams& p, uint8_t* smem, uint32_t tmem, 
         return true;
     };
 
-    UnitReader<D, BN, QT> units;
+    UnitReader<D, BN, QT, NQB> units;
     for (;;) {
         const int u = units.next(smem, abort_flag, 34);
         if (!__all_sync(0xffffffffu, u != -2)) return;
@@ -807,9 +853,9 @@ __device__ void correction_role(const KParams& p, uint8_t* smem, uint32_t tmem, 
     }
 }
 
-template <int D, bool BF16, bool MASK, bool DROP, int BN = BLOCK_N, int QT = Q_TILES_PER_CTA>
+template <int D, bool BF16, bool MASK, bool DROP, int BN = BLOCK_N, int QT = Q_TILES_PER_CTA, int NQB = 1>
 __global__ void __launch_bounds__(NUM_THREADS, 1) fa_fwd_kernel(const __grid_constant__ KParams p) {
-    using L = Smem<D, BN, QT>;
+    using L = Smem<D, BN, QT, NQB>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t base = smem_u32(smem);
@@ -851,16 +897,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) fa_fwd_kernel(const __grid_con
 
     if (wg < 2) {
         setmaxnreg_inc<REG_SOFTMAX>();
-        softmax_role<D, BF16, MASK, DROP, BN, QT>(p, smem, tmem, wg, warp & 3, abort_flag);
+        softmax_role<D, BF16, MASK, DROP, BN, QT, NQB>(p, smem, tmem, wg, warp & 3, abort_flag);
     } else if (wg == 2) {
         setmaxnreg_dec<REG_CORR>();
-        correction_role<D, BF16, BN, QT>(p, smem, tmem, warp & 3, abort_flag);
+        correction_role<D, BF16, BN, QT, NQB>(p, smem, tmem, warp & 3, abort_flag);
     } else {
         setmaxnreg_dec<REG_CTRL>();
         if (warp == WARP_TMA) {
-            if (lane == 0) producer_role<D, BN, QT>(p, smem, abort_flag);
+            if (lane == 0) producer_role<D, BN, QT, NQB>(p, smem, abort_flag);
         } else if (warp == WARP_MMA) {
-            if (lane == 0) mma_role<D, BF16, BN, QT>(p, smem, tmem, abort_flag);
+            if (lane == 0) mma_role<D, BF16, BN, QT, NQB>(p, smem, tmem, abort_flag);
         }
     }
 
@@ -908,11 +954,11 @@ __global__ void __launch_bounds__(64, 1) selftest_timeout_kernel(long long deadl
     }
 }
 
-template <int D, bool BF16, bool MASK, bool DROP = false, int BN = BLOCK_N, int QT = Q_TILES_PER_CTA>
+template <int D, bool BF16, bool MASK, bool DROP = false, int BN = BLOCK_N, int QT = Q_TILES_PER_CTA, int NQB = 1>
 cudaError_t launch_impl(const LaunchArgs& a, cudaStream_t stream) {
-    using L = Smem<D, BN, QT>;
+    using L = Smem<D, BN, QT, NQB>;
     static_assert(L::ALLOC <= 232448, "shared memory budget exceeded");
-    auto kern = fa_fwd_kernel<D, BF16, MASK, DROP, BN, QT>;
+    auto kern = fa_fwd_kernel<D, BF16, MASK, DROP, BN, QT, NQB>;
     cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(kern), L::ALLOC);
     if (e != cudaSuccess) return e;
     KParams p;
@@ -990,6 +1036,12 @@ cudaError_t launch_fwd_sm100(const LaunchArgs& a, cudaStream_t stream) {
         return a.dtype == 1 ? launch_impl<128, true, false>(a, stream) : launch_impl<128, false, false>(a, stream);
     }
     if (a.mask) return a.dtype == 1 ? launch_impl<64, true, true>(a, stream) : launch_impl<64, false, true>(a, stream);
+    // two Q buffers when a CTA runs two or more units (more shared memory per
+    // CTA; for one unit per CTA they cannot help)
+    const int n_units = a.B * a.H * ((a.Sq + Q_TILES_PER_CTA * BLOCK_M - 1) / (Q_TILES_PER_CTA * BLOCK_M));
+    if (n_units >= 2 * a.grid)
+        return a.dtype == 1 ? launch_impl<64, true, false, false, BLOCK_N, Q_TILES_PER_CTA, 2>(a, stream)
+                            : launch_impl<64, false, false, false, BLOCK_N, Q_TILES_PER_CTA, 2>(a, stream);
     return a.dtype == 1 ? launch_impl<64, true, false>(a, stream) : launch_impl<64, false, false>(a, stream);
 }
 
