@@ -909,6 +909,7 @@ __global__ void __launch_bounds__(BWD2_THREADS, 1) fa_bwd_kernel_wide(const __gr
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = misc[0];
+    grid_dependency_sync();  // the previous kernel in the stream has completed
     if (wg == 0) {
         setmaxnreg_dec<Reg2<D>::CTRL>();
         if (warp == BW_TMA && lane == 0) bwd2_producer<D>(p, smem, abort_flag);
@@ -970,6 +971,7 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const uint16_t* __restric
                                                        float* __restrict__ delta, float* __restrict__ dq_acc, int Sq,
                                                        int Sq_pad, unsigned int* sched, int H, Strides3 os,
                                                        Strides3 dos) {
+    grid_dependency_sync();
     using PS = PrepShape<D>;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int sub = lane / PS::LANES, part = lane - sub * PS::LANES;  // row within the warp, 8-element part
@@ -1010,6 +1012,7 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const uint16_t* __restric
 template <int D, bool BF16>
 __global__ void __launch_bounds__(256) bwd_post_kernel(const float4* __restrict__ acc, uint16_t* __restrict__ dq,
                                                        size_t n4, float scale, int H, int Sq, Strides3 qs) {
+    grid_dependency_sync();
     constexpr int G = D / 4;  // 4-element groups per row
     for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n4; i += (size_t)gridDim.x * blockDim.x) {
         const float4 a = acc[i];
@@ -1030,6 +1033,7 @@ __global__ void __launch_bounds__(256) bwd_post_kv_kernel(const float4* __restri
                                                           const float4* __restrict__ dv_acc, uint16_t* __restrict__ dk,
                                                           uint16_t* __restrict__ dv, size_t n4, int H, int Sk,
                                                           Strides3 ks, Strides3 vs) {
+    grid_dependency_sync();
     constexpr int G = D / 4;  // 4-element groups per row
     for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n4; i += (size_t)gridDim.x * blockDim.x) {
         const size_t rowi = i / G;  // (bh, key)
@@ -1162,6 +1166,8 @@ cudaError_t launch_bwd_impl(const BwdLaunchArgs& a, cudaStream_t stream) {
         cfg.blockDim = dim3(BWD2_THREADS, 1, 1);
         cfg.dynamicSmemBytes = alloc;
         cfg.stream = stream;
+        cudaLaunchAttribute attr[1];
+        set_programmatic_launch(cfg, attr);
         e = cudaLaunchKernelEx(&cfg, kern, p);
         if (e != cudaSuccess) return e;
         if (p.q_split > 1) {

@@ -590,6 +590,7 @@ __global__ void __launch_bounds__(THREADS, 1) fa_fwd_kernel_d256(const __grid_co
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = misc[0];
+    grid_dependency_sync();  // the previous kernel in the stream has completed
     if (wg == 0) {
         softmax<BF16, MASK, DROP>(p, smem, tmem, warp & 3, abort_flag);
     } else if (wg == 1) {
@@ -646,6 +647,8 @@ cudaError_t launch_impl(const LaunchArgs& a, cudaStream_t stream) {
     cfg.blockDim = dim3(THREADS, 1, 1);
     cfg.dynamicSmemBytes = L::ALLOC;
     cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    set_programmatic_launch(cfg, attr);
     return cudaLaunchKernelEx(&cfg, kern, p);
 }
 

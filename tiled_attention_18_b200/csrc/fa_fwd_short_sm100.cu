@@ -607,6 +607,7 @@ __global__ void __launch_bounds__(THREADS, 1) fa_fwd_kernel_short(const __grid_c
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = misc[0];
+    grid_dependency_sync();  // the previous kernel in the stream has completed
 
     if (wg < 2) {
         setmaxnreg_inc<REG_SOFTMAX>();
@@ -659,6 +660,8 @@ cudaError_t launch_short(const LaunchArgs& a, cudaStream_t stream) {
     cfg.blockDim = dim3(THREADS, 1, 1);
     cfg.dynamicSmemBytes = L::ALLOC;
     cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    set_programmatic_launch(cfg, attr);
     return cudaLaunchKernelEx(&cfg, kern, p);
 }
 

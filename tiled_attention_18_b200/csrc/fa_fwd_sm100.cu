@@ -894,6 +894,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) fa_fwd_kernel(const __grid_con
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = misc[0];
+    grid_dependency_sync();  // the previous kernel in the stream has completed
 
     if (wg < 2) {
         setmaxnreg_inc<REG_SOFTMAX>();
@@ -924,6 +925,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) fa_fwd_kernel(const __grid_con
 // the status word.  Thread 32 waits on another barrier and leaves on the abort
 // flag; TMEM held by the CTA is released before the kernel ends.
 __global__ void __launch_bounds__(64, 1) selftest_timeout_kernel(long long deadline_cycles) {
+    grid_dependency_sync();
     __shared__ __align__(8) uint64_t bars[2];
     __shared__ uint32_t tm;
     __shared__ uint32_t abort_s;
@@ -995,8 +997,8 @@ cudaError_t launch_impl(const LaunchArgs& a, cudaStream_t stream) {
     cfg.blockDim = dim3(NUM_THREADS, 1, 1);
     cfg.dynamicSmemBytes = L::ALLOC;
     cfg.stream = stream;
-    cfg.attrs = nullptr;
-    cfg.numAttrs = 0;
+    cudaLaunchAttribute attr[1];
+    set_programmatic_launch(cfg, attr);
     return cudaLaunchKernelEx(&cfg, kern, p);
 }
 

@@ -135,9 +135,34 @@ inline BwdWorkspace bwd_workspace_layout(int64_t BH, int64_t Sq, int64_t D) {
 // context re-created after cudaDeviceReset has a new id and is set again.
 cudaError_t ensure_smem_limit(const void* kernel, int bytes);
 
-// Launches `kernel` on `stream` and returns the status of this launch alone
-// (cudaGetLastError after a <<<>>> launch would also return an error that
-// other code left pending in the calling thread).
+// Programmatic dependent launch.  Every kernel of this library is launched
+// with programmatic stream serialization: it may start while the kernel before
+// it in the stream is still running (its CTAs take SMs as that kernel's CTAs
+// leave them), does its set-up (barriers, tensor memory, descriptor
+// prefetches), and then waits in grid_dependency_sync() until that kernel has
+// completed and its memory writes are visible, before touching global memory.
+// Each kernel also lets its own successor start early.  A kernel launched
+// without the attribute, or after work that is not a kernel, passes the wait
+// at once.
+inline void set_programmatic_launch(cudaLaunchConfig_t& cfg, cudaLaunchAttribute (&attr)[1]) {
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+}
+
+#ifdef __CUDACC__
+// Called by every thread of a CTA before its first global-memory access.
+__device__ __forceinline__ void grid_dependency_sync() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+#endif
+
+// Launches `kernel` on `stream` (as a programmatic dependent launch: the
+// kernel must call grid_dependency_sync() first) and returns the status of
+// this launch alone (cudaGetLastError after a <<<>>> launch would also return
+// an error that other code left pending in the calling thread).
 template <typename... Expected, typename... Actual>
 cudaError_t launch_kernel(void (*kernel)(Expected...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
                           Actual&&... args) {
@@ -146,8 +171,8 @@ cudaError_t launch_kernel(void (*kernel)(Expected...), dim3 grid, dim3 block, si
     cfg.blockDim = block;
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
-    cfg.attrs = nullptr;
-    cfg.numAttrs = 0;
+    cudaLaunchAttribute attr[1];
+    set_programmatic_launch(cfg, attr);
     return cudaLaunchKernelEx(&cfg, kernel, std::forward<Actual>(args)...);
 }
 

@@ -49,6 +49,7 @@ template <bool BF16, bool VEC>
 __global__ void __launch_bounds__(256) merge_kernel(float* __restrict__ o_acc, float* __restrict__ lse_acc,
                                                     const uint16_t* __restrict__ o_part,
                                                     const float* __restrict__ lse_part, long long rows, int D) {
+    grid_dependency_sync();
     const long long row = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     if (row >= rows) return;
@@ -85,6 +86,7 @@ __global__ void __launch_bounds__(256) merge_kernel(float* __restrict__ o_acc, f
 template <bool BF16>
 __global__ void __launch_bounds__(256) finalize_kernel(const float* __restrict__ o_acc, uint16_t* __restrict__ o,
                                                        long long n) {
+    grid_dependency_sync();
     for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x)
         o[i] = from_f32<BF16>(o_acc[i]);
 }
@@ -94,6 +96,7 @@ __global__ void __launch_bounds__(256) finalize_kernel(const float* __restrict__
 template <bool BF16>
 __global__ void __launch_bounds__(256) accumulate_kernel(float* __restrict__ acc, const uint16_t* __restrict__ x,
                                                          long long n) {
+    grid_dependency_sync();
     const long long step = (long long)gridDim.x * blockDim.x;
     long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     if ((n & 3) == 0 && ((uintptr_t)acc & 15) == 0 && ((uintptr_t)x & 7) == 0) {
