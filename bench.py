@@ -108,10 +108,12 @@ def peak_tflops():
 
 
 def kernel_source_hash(kernel_file: str = "fa_fwd_sm100.cu") -> str:
-    """Hash of a forward kernel's sources (its file and the shared device helpers)."""
+    """Hash of a forward kernel's sources (its file, the shared device helpers
+    and the internal header with the launch helpers)."""
     import hashlib
     h = hashlib.sha256()
-    for path in (os.path.join(CSRC, kernel_file), os.path.join(CSRC, "sm100_helpers.cuh")):
+    for path in (os.path.join(CSRC, kernel_file), os.path.join(CSRC, "sm100_helpers.cuh"),
+                 os.path.join(CSRC, "fa_internal.h")):
         with open(path, "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
