@@ -81,10 +81,15 @@ struct BwdParams {
     // Split query range (key sets of at most KV_ACC_ROWS keys, few units): a
     // unit takes chunk c of its key tile's query steps, q_chunk steps long, and
     // adds its dK (scaled) and dV in fp32 to dk_acc / dv_acc [BH][KV_ACC_ROWS][D]
-    // instead of writing them; q_split = 1: off
+    // instead of writing them; q_split = 1: off.  With one key tile per head a
+    // step's dQ rows are complete in the unit that forms them: the split
+    // instantiation of the D = 128 kernel (which has the dQ staging tile)
+    // writes them to dq (16-bit, byte strides dq_s) directly.
     int q_split, q_chunk;
     float* dk_acc;
     float* dv_acc;
+    uint8_t* dq;
+    long long dq_s[3];
     int BH, H, Sq, Sk, Sq_pad, n_mtiles, n_ktiles, n_units, causal, causal_off;
     int dh;               // head dimension of the tensors (64: run by the D = 128 kernel on zero-padded operands)
     int head_group;       // causal claim order: heads per group (their Q, dO, dQ fit in L2)
@@ -754,7 +759,42 @@ __device__ void bwd2_out_role(const BwdParams& p, uint8_t* smem, uint32_t tmem, 
             const bool d_ok = DH >= 128 || row < DH;  // lanes past a 64-wide head dimension hold zeros
             float* dst = p.dq_acc + ((size_t)U.bh * (size_t)p.Sq + (size_t)m * QM) * dh + (size_t)half * 128 + row;
             const int nq = min(QM, p.Sq - m * QM);
-            if (!p.dq_flags && L::DQ_BULK) {
+            if constexpr (SPLIT && L::DQ_BULK) {
+                // one key tile per head: copy dQ^T out of TMEM as dQ[q][d] into the
+                // staging tile (once every thread has read the previous step's),
+                // free the columns, then write the rows scaled and rounded to dQ,
+                // four values per thread and access (rows past Sq skipped)
+                if (!__all_sync(0xffffffffu, group_sync(76))) return;
+                constexpr int sstride = dh < 128 ? dh : 128;
+                float* stg = reinterpret_cast<float*>(smem + L::DQS_OFF) + row;
+#pragma unroll 1
+                for (int hh = 0; hh < 2; ++hh) {
+                    uint32_t r[32];
+                    tmem_ld32u(tmem + lane_sel + col2_dp(b) + 32 * hh, r);
+                    if (d_ok) {
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) stg[(32 * hh + j) * sstride] = __uint_as_float(r[j]);
+                    }
+                }
+                tc_fence_before();
+                mbar_arrive(bar(L::B_DQEMPTY + b));
+                if (!__all_sync(0xffffffffu, group_sync(77))) return;
+                // thread `row` takes chunk j = row mod CPR of rows row / CPR + k * QSTEP
+                constexpr int CPR = sstride / 4;  // 4-value chunks per staged row
+                constexpr int QSTEP = 128 / CPR;
+                const int j = row % CPR;
+                const int ub = U.bh / p.H, uh = U.bh - ub * p.H;
+                const long long rs = p.dq_s[2];
+                uint8_t* dp = p.dq + ub * p.dq_s[0] + uh * p.dq_s[1] + ((long long)m * QM + row / CPR) * rs +
+                              half * 256 + j * 8;
+                const float4* sp = reinterpret_cast<const float4*>(smem + L::DQS_OFF) + row;
+#pragma unroll 1
+                for (int q = row / CPR; q < nq; q += QSTEP, dp += QSTEP * rs, sp += 128) {
+                    const float4 v = *sp;
+                    *reinterpret_cast<uint2*>(dp) = make_uint2(pack2<BF16>(v.x * p.scale, v.y * p.scale),
+                                                               pack2<BF16>(v.z * p.scale, v.w * p.scale));
+                }
+            } else if (!p.dq_flags && L::DQ_BULK) {
                 // once the previous step's reduce has read the staging, copy dQ^T
                 // out of TMEM as dQ[q][d] (each lane holds one d over the 64
                 // queries: a warp writes 32 consecutive floats per query), free
@@ -934,11 +974,13 @@ __global__ void __launch_bounds__(BWD2_THREADS, 1) fa_bwd_kernel_wide(const __gr
 
 
 // Per (bh, query row) of the padded row range: Delta = sum_d dO O in fp32,
-// LSE * log2(e), and the row of the dQ accumulator cleared.  A row is taken by
-// D / 8 lanes, each with one 16-byte load of O and of dO (several rows per
-// warp when D < 256: more loads in flight per warp).  Padded rows get +inf
-// (weight 0) and Delta = 0.  Block (0, 0) also clears the scheduler counter,
-// which the main kernel (next on the stream) reads.
+// LSE * log2(e), and the row of the dQ accumulator cleared (unless dq_acc is
+// null: the split mode writes dQ directly).  A row is taken by D / 8 lanes,
+// each with one 16-byte load of O and of dO (several rows per warp when
+// D < 256: more loads in flight per warp).  Padded rows get +inf (weight 0)
+// and Delta = 0.  Block (0, 0) also clears the scheduler counter, which the
+// main kernel (next on the stream) reads, and all blocks together clear
+// kv_n4 float4s at kv_zero (the split mode's dK/dV partial sums), if given.
 template <int D>
 struct PrepShape {
     static constexpr int LANES = D / 8;                      // lanes per row
@@ -970,8 +1012,13 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const uint16_t* __restric
                                                        const float* __restrict__ lse, float* __restrict__ lse2,
                                                        float* __restrict__ delta, float* __restrict__ dq_acc, int Sq,
                                                        int Sq_pad, unsigned int* sched, int H, Strides3 os,
-                                                       Strides3 dos) {
+                                                       Strides3 dos, float4* __restrict__ kv_zero, size_t kv_n4) {
     grid_dependency_sync();
+    if (kv_zero) {
+        // the split mode's fp32 dK/dV partial sums, spread over all blocks
+        const size_t blk = (size_t)blockIdx.y * gridDim.x + blockIdx.x, nthr = (size_t)gridDim.x * gridDim.y * 256;
+        for (size_t i = blk * 256 + threadIdx.x; i < kv_n4; i += nthr) kv_zero[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
     using PS = PrepShape<D>;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int sub = lane / PS::LANES, part = lane - sub * PS::LANES;  // row within the warp, 8-element part
@@ -987,9 +1034,11 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const uint16_t* __restric
         const uint4 ov = *reinterpret_cast<const uint4*>(o + eo);
         const uint4 dv = *reinterpret_cast<const uint4*>(dout + ed);
         acc = dot8(ov, dv, BF16);
-        float4* z = reinterpret_cast<float4*>(dq_acc + (bh * (size_t)Sq + (size_t)row) * D + (size_t)part * 8);
-        z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
-        z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (dq_acc) {  // null when the main kernel writes dQ directly
+            float4* z = reinterpret_cast<float4*>(dq_acc + (bh * (size_t)Sq + (size_t)row) * D + (size_t)part * 8);
+            z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+            z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
     }
     // sum over the row's lanes (aligned groups of LANES lanes)
 #pragma unroll
@@ -1056,31 +1105,53 @@ cudaError_t launch_bwd_impl(const BwdLaunchArgs& a, cudaStream_t stream) {
     const int BH = a.B * a.H;
     const int n_mtiles = (a.Sq + TILE - 1) / TILE;
     const int Sq_pad = n_mtiles * TILE;
+    constexpr int DW = D >= 128 ? D : 128;
+    // Split query range: a key set of at most KV_ACC_ROWS keys (one key tile)
+    // whose units leave SMs idle takes chunks of q_chunk steps per unit, about
+    // two units per SM; not in deterministic mode (the fp32 adds of the
+    // partial sums come in any order), nor with an explicit mask or dropout
+    // (the split instantiation has neither)
+    const int n_steps = (a.Sq + QM - 1) / QM;  // 64-row steps
+    const int n_units1 = BH * ((a.Sk + TILE - 1) / TILE) * Bwd2Smem<DW>::HALVES;
+    int q_chunk = n_steps, q_split = 1;
+    if (!a.mask && !a.drop.enabled && a.dk_acc && a.dv_acc && !a.dq_flags && a.Sk <= KV_ACC_ROWS && a.sms > 0 &&
+        n_units1 < a.sms && n_steps > 1) {
+        const int want = (2 * a.sms + n_units1 - 1) / n_units1;  // chunks per key tile
+        q_chunk = (n_steps + want - 1) / want;
+        q_split = (n_steps + q_chunk - 1) / q_chunk;  // no chunk is empty
+        if (q_split == 1) q_chunk = n_steps;
+    }
+    const bool split = q_split > 1;
+    // the split D = 64/128 kernel writes dQ itself (through its dQ staging
+    // tile): no accumulator to clear and no dQ post kernel
+    const bool dq_direct = split && Bwd2Smem<DW>::DQ_BULK;
     {
         dim3 grid((unsigned)((Sq_pad + PrepShape<D>::ROWS_PER_BLOCK - 1) / PrepShape<D>::ROWS_PER_BLOCK),
                   (unsigned)BH, 1);
+        // split: the dK/dV partial sums (contiguous) cleared too
         cudaError_t e = launch_kernel(
             bwd_prep_kernel<D, BF16>, grid, dim3(256), 0, stream, static_cast<const uint16_t*>(a.o),
-            static_cast<const uint16_t*>(a.dout), a.lse, a.lse2, a.delta, a.dq_acc, a.Sq, Sq_pad, a.sched, a.H,
-            Strides3{{a.o_stride[0], a.o_stride[1], a.o_stride[2]}},
-            Strides3{{a.do_stride[0], a.do_stride[1], a.do_stride[2]}});
+            static_cast<const uint16_t*>(a.dout), a.lse, a.lse2, a.delta, dq_direct ? nullptr : a.dq_acc, a.Sq, Sq_pad,
+            a.sched, a.H, Strides3{{a.o_stride[0], a.o_stride[1], a.o_stride[2]}},
+            Strides3{{a.do_stride[0], a.do_stride[1], a.do_stride[2]}},
+            split ? reinterpret_cast<float4*>(a.dk_acc) : nullptr,
+            split ? (size_t)2 * BH * KV_ACC_ROWS * D / 4 : (size_t)0);
         if (e != cudaSuccess) return e;
     }
     {
         // every head dimension runs the 64-row-step kernel (its Q/dO maps have
         // 64-row boxes); D = 64 runs its D = 128 instantiation, whose loads of
         // the second 64-column chunk read past D and fill with zeros, so the
-        // padding adds nothing to the scores, dK, dV or dQ
-        constexpr int DW = D >= 128 ? D : 128;
+        // padding adds nothing to the scores, dK, dV or dQ.  The split mode
+        // has its own instantiation (partial sums added; dQ written directly
+        // at D = 64/128).
         void (*kern)(const BwdParams) =
-            a.drop.enabled
+            split ? fa_bwd_kernel_wide<DW, BF16, false, false, true, D>
+            : a.drop.enabled
                 ? (a.mask ? fa_bwd_kernel_wide<DW, BF16, true, true, false, D>
                           : fa_bwd_kernel_wide<DW, BF16, false, true, false, D>)
                 : (a.mask ? fa_bwd_kernel_wide<DW, BF16, true, false, false, D>
                           : fa_bwd_kernel_wide<DW, BF16, false, false, false, D>);
-        // split partial sums are added by their own instantiation, taken
-        // without an explicit mask or dropout
-        const bool can_split = !a.mask && !a.drop.enabled;
         const int alloc = Bwd2Smem<DW>::ALLOC;
         cudaError_t e = ensure_smem_limit(reinterpret_cast<const void*>(kern), alloc);
         if (e != cudaSuccess) return e;
@@ -1095,16 +1166,18 @@ cudaError_t launch_bwd_impl(const BwdLaunchArgs& a, cudaStream_t stream) {
         p.dq_acc = a.dq_acc;
         p.dk = static_cast<uint8_t*>(a.dk);
         p.dv = static_cast<uint8_t*>(a.dv);
+        p.dq = static_cast<uint8_t*>(a.dq);
         for (int i = 0; i < 3; ++i) {
             p.dk_s[i] = a.dk_stride[i] * 2;
             p.dv_s[i] = a.dv_stride[i] * 2;
+            p.dq_s[i] = a.dq_stride[i] * 2;
         }
         p.BH = BH;
         p.H = a.H;
         p.Sq = a.Sq;
         p.Sk = a.Sk;
         p.Sq_pad = Sq_pad;
-        p.n_mtiles = (a.Sq + QM - 1) / QM;  // 64-row steps
+        p.n_mtiles = n_steps;
         p.n_ktiles = (a.Sk + TILE - 1) / TILE;
         p.n_units = BH * p.n_ktiles * Bwd2Smem<DW>::HALVES;
         p.causal = a.causal;
@@ -1133,34 +1206,12 @@ cudaError_t launch_bwd_impl(const BwdLaunchArgs& a, cudaStream_t stream) {
         p.drop_offset = a.drop.offset;
         p.keep_scale = a.drop.enabled ? a.drop.keep_scale : 1.f;
         p.flag_steps = (a.Sq + QM - 1) / QM;
-        // Split query range: a key set of at most KV_ACC_ROWS keys (one key tile)
-        // whose units leave SMs idle takes chunks of q_chunk steps per unit, about
-        // two units per SM; not in deterministic mode (the fp32 adds of the
-        // partial sums come in any order)
-        p.q_split = 1;
-        p.q_chunk = p.n_mtiles;
+        p.q_split = q_split;
+        p.q_chunk = q_chunk;
         p.dk_acc = a.dk_acc;
         p.dv_acc = a.dv_acc;
-        int grid = a.grid;
-        if (can_split && a.dk_acc && a.dv_acc && !a.dq_flags && a.Sk <= KV_ACC_ROWS && a.sms > 0 &&
-            p.n_units < a.sms && p.n_mtiles > 1) {
-            const int want = (2 * a.sms + p.n_units - 1) / p.n_units;  // chunks per key tile
-            p.q_chunk = (p.n_mtiles + want - 1) / want;
-            p.q_split = (p.n_mtiles + p.q_chunk - 1) / p.q_chunk;      // no chunk is empty
-            if (p.q_split > 1) {
-                kern = fa_bwd_kernel_wide<DW, BF16, false, false, true, D>;
-                e = ensure_smem_limit(reinterpret_cast<const void*>(kern), alloc);
-                if (e != cudaSuccess) return e;
-                p.n_units *= p.q_split;
-                grid = p.n_units < a.sms ? p.n_units : a.sms;
-                const size_t bytes = (size_t)BH * KV_ACC_ROWS * D * sizeof(float);
-                e = cudaMemsetAsync(a.dk_acc, 0, bytes, stream);
-                if (e == cudaSuccess) e = cudaMemsetAsync(a.dv_acc, 0, bytes, stream);
-                if (e != cudaSuccess) return e;
-            } else {
-                p.q_chunk = p.n_mtiles;
-            }
-        }
+        p.n_units *= q_split;
+        const int grid = split ? (p.n_units < a.sms ? p.n_units : a.sms) : a.grid;
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3((unsigned)grid, 1, 1);
         cfg.blockDim = dim3(BWD2_THREADS, 1, 1);
@@ -1170,7 +1221,7 @@ cudaError_t launch_bwd_impl(const BwdLaunchArgs& a, cudaStream_t stream) {
         set_programmatic_launch(cfg, attr);
         e = cudaLaunchKernelEx(&cfg, kern, p);
         if (e != cudaSuccess) return e;
-        if (p.q_split > 1) {
+        if (split) {
             const size_t n4 = (size_t)BH * (size_t)a.Sk * D / 4;
             const unsigned blocks = (unsigned)((n4 + 255) / 256 < 148u * 16u ? (n4 + 255) / 256 : 148u * 16u);
             e = launch_kernel(bwd_post_kv_kernel<D, BF16>, dim3(blocks), dim3(256), 0, stream,
@@ -1178,7 +1229,7 @@ cudaError_t launch_bwd_impl(const BwdLaunchArgs& a, cudaStream_t stream) {
                               static_cast<uint16_t*>(a.dk), static_cast<uint16_t*>(a.dv), n4, a.H, a.Sk,
                               Strides3{{a.dk_stride[0], a.dk_stride[1], a.dk_stride[2]}},
                               Strides3{{a.dv_stride[0], a.dv_stride[1], a.dv_stride[2]}});
-            if (e != cudaSuccess) return e;
+            if (e != cudaSuccess || dq_direct) return e;  // dQ was written by the main kernel
         }
     }
     {
