@@ -33,3 +33,26 @@ def test_reference_arm_json_line(extra):
         assert line["metric"].startswith("attention bwd")
     if "--dropout" in extra:
         assert "dropout" in line["config"]["workload"]
+
+
+def test_peak_follows_the_sampled_clocks(monkeypatch, tmp_path):
+    """The roofline denominator is the burst bf16 figure at full clock and the
+    sustained one when the timed region ran power-capped; both kinds are read
+    from the peaks file when it has them, else from the fallback figures."""
+    sys.path.insert(0, ROOT)
+    import bench
+    full = {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"]}
+    capped = {"sm_mhz": 1728.5, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"]}
+    slow_no_reason = {"sm_mhz": 1500.0, "sm_max_mhz": 1965.0, "reasons": []}
+    monkeypatch.setattr(bench, "PEAKS_PATH", str(tmp_path / "absent.json"))
+    assert bench.peak_tflops(None)[0] == bench.FALLBACK_BF16_TFLOPS
+    assert bench.peak_tflops(full)[0] == bench.FALLBACK_BF16_TFLOPS
+    assert bench.peak_tflops(slow_no_reason)[0] == bench.FALLBACK_BF16_TFLOPS
+    peak, src, burst = bench.peak_tflops(capped)
+    assert peak == bench.FALLBACK_BF16_TFLOPS_SUSTAINED and burst == bench.FALLBACK_BF16_TFLOPS
+    assert "sustained" in src
+    path = tmp_path / "peaks.json"
+    path.write_text(json.dumps({"bf16_tflops": 1637.9, "bf16_tflops_sustained": 1420.0, "hbm_gbs": 7000.0}))
+    monkeypatch.setattr(bench, "PEAKS_PATH", str(path))
+    assert bench.peak_tflops(full)[:1] == (1637.9,)
+    assert bench.peak_tflops(capped)[0] == 1420.0 and bench.peak_tflops(capped)[2] == 1637.9
