@@ -32,9 +32,10 @@
 //        dQ_m^T = K^T dS^T                  (into the step's dP^T columns)
 //      dQ_m is added to the fp32 accumulator (a TMA bulk reduce-add, or
 //      per-element atomics, or in key-tile order in deterministic mode); dK,
-//      dV are written once per unit.  D = 64 runs the D = 128 instantiation:
-//      its loads of the second 64-column chunk of Q, K, V and dO read past D
-//      and fill with zeros, which add nothing to the scores or gradients;
+//      dV are written once per unit.  D = 64 runs the D = 128 instantiation
+//      on the first 64-column chunk of Q, K, V and dO: the scores reduce over
+//      it alone, and the lanes of dQ^T and the columns of dK, dV past 64 that
+//      the other chunk feeds are never written out;
 //   3. bwd_post_kernel: dQ = scale * accumulator, rounded to the 16-bit dtype
 //      (and, after a split query range, bwd_post_kv_kernel for dK and dV).
 //
@@ -91,7 +92,7 @@ struct BwdParams {
     uint8_t* dq;
     long long dq_s[3];
     int BH, H, Sq, Sk, Sq_pad, n_mtiles, n_ktiles, n_units, causal, causal_off;
-    int dh;               // head dimension of the tensors (64: run by the D = 128 kernel on zero-padded operands)
+    int dh;               // head dimension of the tensors (64: run by the D = 128 kernel on its first column chunk)
     int head_group;       // causal claim order: heads per group (their Q, dO, dQ fit in L2)
     int* dq_flags;        // deterministic mode: [BH][flag_steps][4] key tiles added so far per
                           // (head, query step, warp); null: dQ is added with atomics
@@ -306,7 +307,7 @@ __device__ __forceinline__ void fence_async_smem() {
 // forward kernel's ring): -1 when the CTA has no more work, -2 on abort.
 // ------------------------------------------------------------------------
 // 64-row query steps with double-buffered S^T / dP^T (D = 64 on the D = 128
-// instantiation with zero-padded operands, D = 128, D = 256).
+// instantiation with its second column chunk unused, D = 128, D = 256).
 //
 // Tensor memory: S0 [0,64) dP0 [64,128) S1 [128,192) dP1 [192,256), dV
 // [256,384), dK [384,512).  While the dS warpgroup turns step g's S^T, dP^T
@@ -440,9 +441,15 @@ struct Bwd2UnitReader {
     }
 };
 
-template <int D>
+// DH < D (the D = 128 kernel on D = 64 tensors): only the first DH / 64
+// column chunks of K, V, Q and dO are loaded.  The scores reduce over those
+// chunks only; the products that read the other chunks (dQ^T's rows, dK's and
+// dV's columns past DH) are never written out, so those chunks may hold any
+// data.
+template <int D, int DH>
 __device__ void bwd2_producer(const BwdParams& p, uint8_t* smem, volatile uint32_t* abort_flag) {
     using L = Bwd2Smem<D>;
+    constexpr int CH = (DH < D) ? DH / 64 : L::CHUNKS;  // column chunks loaded
     const uint32_t base = smem_u32(smem);
     const uint32_t bar0 = base + L::BAR_OFF;
     auto bar = [&](int i) { return bar0 + 8u * (uint32_t)i; };
@@ -466,11 +473,11 @@ __device__ void bwd2_producer(const BwdParams& p, uint8_t* smem, volatile uint32
         const int b = U.bh / p.H, h = U.bh - b * p.H;
         const uint32_t kvp = (uint32_t)nunit & 1u;
         if (!mbar_wait(bar(L::B_KVEMPTY), kvp ^ 1u, abort_flag, 61)) { ok = false; break; }
-        mbar_expect_tx(bar(L::B_KVFULL), 2 * L::KV_TILE);
+        mbar_expect_tx(bar(L::B_KVFULL), 2 * CH * L::KCHUNK);
         kv_fill = (int)kvp;
         ++nunit;
 #pragma unroll
-        for (int c = 0; c < L::CHUNKS; ++c) {
+        for (int c = 0; c < CH; ++c) {
             tma_load_4d(base + L::K_OFF + c * L::KCHUNK, &p.tmap_k, bar(L::B_KVFULL), c * 64, U.n * TILE, h, b);
             tma_load_4d(base + L::V_OFF + c * L::KCHUNK, &p.tmap_v, bar(L::B_KVFULL), c * 64, U.n * TILE, h, b);
         }
@@ -479,12 +486,12 @@ __device__ void bwd2_producer(const BwdParams& p, uint8_t* smem, volatile uint32
             const int st = (int)(g % L::NSTAGE);
             const uint32_t sp = (g / L::NSTAGE) & 1u;
             if (!mbar_wait(bar(L::B_QEMPTY + st), sp ^ 1u, abort_flag, 62)) { ok = false; break; }
-            mbar_expect_tx(bar(L::B_QFULL + st), 2 * L::Q_TILE + L::STATS_BYTES);
+            mbar_expect_tx(bar(L::B_QFULL + st), 2 * CH * L::QCHUNK + L::STATS_BYTES);
             fill_mask |= 1u << st;
             fill_parity = (fill_parity & ~(1u << st)) | (sp << st);
             const uint32_t dst = base + L::STAGE_OFF + st * L::STAGE_BYTES;
 #pragma unroll
-            for (int c = 0; c < L::CHUNKS; ++c) {
+            for (int c = 0; c < CH; ++c) {
                 tma_load_4d(dst + c * L::QCHUNK, &p.tmap_q, bar(L::B_QFULL + st), c * 64, m * QM, h, b);
                 tma_load_4d(dst + L::Q_TILE + c * L::QCHUNK, &p.tmap_do, bar(L::B_QFULL + st), c * 64, m * QM, h, b);
             }
@@ -502,7 +509,7 @@ __device__ void bwd2_producer(const BwdParams& p, uint8_t* smem, volatile uint32
     }
 }
 
-template <int D, bool BF16>
+template <int D, bool BF16, int DH>
 __device__ void bwd2_mma(const BwdParams& p, uint8_t* smem, uint32_t tmem, volatile uint32_t* abort_flag) {
     using L = Bwd2Smem<D>;
     const uint32_t base = smem_u32(smem);
@@ -528,10 +535,11 @@ __device__ void bwd2_mma(const BwdParams& p, uint8_t* smem, uint32_t tmem, volat
     auto lo = [](uint64_t d) { return (uint32_t)d; };
     auto hi = [](uint64_t d) { return (uint32_t)(d >> 32); };
 
-    // S^T or dP^T of one step: A = K or V (128 keys), B = Q or dO (64 queries), K = D
+    // S^T or dP^T of one step: A = K or V (128 keys), B = Q or dO (64 queries),
+    // K = the tensors' head dimension (the loaded chunks)
     auto issue_sp = [&](uint32_t d_tmem, uint64_t a, uint32_t b_off16) {
 #pragma unroll
-        for (int ks = 0; ks < D / 16; ++ks) {
+        for (int ks = 0; ks < (DH < D ? DH : D) / 16; ++ks) {
             const uint32_t in_chunk = (uint32_t)((ks & 3) * 32) >> 4;
             const uint32_t a_off = in_chunk + (uint32_t)(((ks >> 2) * L::KCHUNK) >> 4);
             const uint32_t b_off = in_chunk + (uint32_t)(((ks >> 2) * L::QCHUNK) >> 4);
@@ -908,7 +916,7 @@ __device__ void bwd2_out_role(const BwdParams& p, uint8_t* smem, uint32_t tmem, 
     }
 }
 
-// DH: the tensors' head dimension (64: this D = 128 kernel on zero-padded operands)
+// DH: the tensors' head dimension (64: this D = 128 kernel on its first column chunk)
 template <int D, bool BF16, bool MASK, bool DROP, bool SPLIT = false, int DH = D>
 __global__ void __launch_bounds__(BWD2_THREADS, 1) fa_bwd_kernel_wide(const __grid_constant__ BwdParams p) {
     using L = Bwd2Smem<D>;
@@ -952,8 +960,8 @@ __global__ void __launch_bounds__(BWD2_THREADS, 1) fa_bwd_kernel_wide(const __gr
     grid_dependency_sync();  // the previous kernel in the stream has completed
     if (wg == 0) {
         setmaxnreg_dec<Reg2<D>::CTRL>();
-        if (warp == BW_TMA && lane == 0) bwd2_producer<D>(p, smem, abort_flag);
-        if (warp == BW_MMA && lane == 0) bwd2_mma<D, BF16>(p, smem, tmem, abort_flag);
+        if (warp == BW_TMA && lane == 0) bwd2_producer<D, DH>(p, smem, abort_flag);
+        if (warp == BW_MMA && lane == 0) bwd2_mma<D, BF16, DH>(p, smem, tmem, abort_flag);
     } else if (wg == 1 || wg == 3) {
         setmaxnreg_inc<Reg2<D>::DS>();
         bwd2_ds_role<D, BF16, MASK, DROP>(p, smem, tmem, warp & 3, wg == 1 ? 0 : 1, abort_flag);
@@ -1140,9 +1148,9 @@ cudaError_t launch_bwd_impl(const BwdLaunchArgs& a, cudaStream_t stream) {
     }
     {
         // every head dimension runs the 64-row-step kernel (its Q/dO maps have
-        // 64-row boxes); D = 64 runs its D = 128 instantiation, whose loads of
-        // the second 64-column chunk read past D and fill with zeros, so the
-        // padding adds nothing to the scores, dK, dV or dQ.  The split mode
+        // 64-row boxes); D = 64 runs its D = 128 instantiation on the first
+        // 64-column chunk of every operand (the scores reduce over it alone;
+        // what the unused chunk would feed is never written out).  The split mode
         // has its own instantiation (partial sums added; dQ written directly
         // at D = 64/128).
         void (*kern)(const BwdParams) =
