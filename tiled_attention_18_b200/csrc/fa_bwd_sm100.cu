@@ -529,6 +529,12 @@ __device__ void bwd2_mma(const BwdParams& p, uint8_t* smem, uint32_t tmem, volat
     const uint64_t b_stage_mn = sw128_desc(base + L::STAGE_OFF, (uint32_t)L::QCHUNK, 1024);
     const uint64_t a_kt = sw128_desc(base + L::K_OFF, (uint32_t)L::KCHUNK, 1024);
     const uint64_t b_ds = sw128_desc(base + L::DS_OFF, 1024, 1024);
+    const uint64_t a_ds = sw128_desc(base + L::DS_OFF, 16, 1024);  // dS^T as a K-major A (K = 64 queries)
+    // DH < D (D = 64 tensors): dQ^T is issued before dV and dK, and dK takes
+    // dS^T from shared memory, so dQ^T's read-out (which the step after next's
+    // dP^T waits for) starts one product pair earlier.  At the full head
+    // dimension the extra shared-memory operand of dK costs more than it saves.
+    constexpr bool DQ_FIRST = DH < D;
     constexpr uint32_t STAGE16 = (uint32_t)L::STAGE_BYTES >> 4;
     constexpr uint32_t QTILE16 = (uint32_t)L::Q_TILE >> 4;
     constexpr uint32_t DS16 = (uint32_t)L::DS_BYTES >> 4;
@@ -610,17 +616,32 @@ __device__ void bwd2_mma(const BwdParams& p, uint8_t* smem, uint32_t tmem, volat
                 tc_fence_after();
             }
             const uint32_t q16 = (uint32_t)st * STAGE16;
-            issue_kv(tmem + COL2_DV, tmem + col2_s(b), q16 + QTILE16, t > 0);  // dV += P^T dO_m
-            issue_kv(tmem + COL2_DK, tmem + col2_dp(b), q16, t > 0);          // dK += dS^T Q_m
-            tc_commit(bar(L::B_QEMPTY + st));
             // dQ^T = K^T dS^T into this step's dP columns
+            auto issue_dq = [&]() {
 #pragma unroll
-            for (int ks = 0; ks < TILE / 16; ++ks) {
-                const uint32_t off = (uint32_t)(ks * (2048 >> 4));
-                tc_mma_ss2(tmem + col2_dp(b), lo(a_kt) + (SPLIT ? half_k16 : 0u) + off, hi(a_kt),
-                           lo(b_ds) + b * DS16 + off, hi(b_ds), IDESC_DQ, ks > 0 ? 1u : 0u);
+                for (int ks = 0; ks < TILE / 16; ++ks) {
+                    const uint32_t off = (uint32_t)(ks * (2048 >> 4));
+                    tc_mma_ss2(tmem + col2_dp(b), lo(a_kt) + (SPLIT ? half_k16 : 0u) + off, hi(a_kt),
+                               lo(b_ds) + b * DS16 + off, hi(b_ds), IDESC_DQ, ks > 0 ? 1u : 0u);
+                }
+                tc_commit(bar(L::B_DQFULL + b));
+            };
+            if constexpr (DQ_FIRST) {
+                issue_dq();
+                issue_kv(tmem + COL2_DV, tmem + col2_s(b), q16 + QTILE16, t > 0);  // dV += P^T dO_m
+                // dK += dS^T Q_m, A = dS^T from shared memory (16 queries = 32 bytes per K step)
+#pragma unroll
+                for (int ks = 0; ks < QM / 16; ++ks)
+                    tc_mma_ss2(tmem + COL2_DK, lo(a_ds) + b * DS16 + (uint32_t)((ks * 32) >> 4), hi(a_ds),
+                               lo(b_stage_mn) + (SPLIT ? half_q16 : 0u) + q16 + (uint32_t)(ks * (2048 >> 4)),
+                               hi(b_stage_mn), IDESC_KV, (t > 0 || ks > 0) ? 1u : 0u);
+                tc_commit(bar(L::B_QEMPTY + st));
+            } else {
+                issue_kv(tmem + COL2_DV, tmem + col2_s(b), q16 + QTILE16, t > 0);  // dV += P^T dO_m
+                issue_kv(tmem + COL2_DK, tmem + col2_dp(b), q16, t > 0);          // dK += dS^T Q_m
+                tc_commit(bar(L::B_QEMPTY + st));
+                issue_dq();
             }
-            tc_commit(bar(L::B_DQFULL + b));
             tc_commit(bar(L::B_DSEMPTY + b));
             if (L::NSTAGE == 1 && t + 1 < U.T && !issue_step(g + 1)) { ok = false; break; }
         }
@@ -633,7 +654,8 @@ __device__ void bwd2_mma(const BwdParams& p, uint8_t* smem, uint32_t tmem, volat
     mbar_drain(bar(L::B_FIN), 0u);
 }
 
-template <int D, bool BF16, bool MASK, bool DROP>
+// DH < D: dK reads dS^T from shared memory, so it is not stored to TMEM.
+template <int D, bool BF16, bool MASK, bool DROP, int DH>
 __device__ void bwd2_ds_role(const BwdParams& p, uint8_t* smem, uint32_t tmem, int warp_in_group, int c,
                              volatile uint32_t* abort_flag) {
     using L = Bwd2Smem<D>;
@@ -710,7 +732,7 @@ __device__ void bwd2_ds_role(const BwdParams& p, uint8_t* smem, uint32_t tmem, i
                 // packed into the first 16 of this warpgroup's own 32 columns: the other
                 // dS warpgroup may still be reading its raw scores from the rest
                 tmem_st16(tmem + lane_sel + col2_s(b) + 32 * c, pk);
-                tmem_st16(tmem + lane_sel + col2_dp(b) + 32 * c, dk);
+                if constexpr (!(DH < D)) tmem_st16(tmem + lane_sel + col2_dp(b) + 32 * c, dk);
 #pragma unroll
                 for (int gi = 0; gi < 4; ++gi) {
                     const int gr = (c * 4 + gi) ^ sw;
@@ -964,7 +986,7 @@ __global__ void __launch_bounds__(BWD2_THREADS, 1) fa_bwd_kernel_wide(const __gr
         if (warp == BW_MMA && lane == 0) bwd2_mma<D, BF16, DH>(p, smem, tmem, abort_flag);
     } else if (wg == 1 || wg == 3) {
         setmaxnreg_inc<Reg2<D>::DS>();
-        bwd2_ds_role<D, BF16, MASK, DROP>(p, smem, tmem, warp & 3, wg == 1 ? 0 : 1, abort_flag);
+        bwd2_ds_role<D, BF16, MASK, DROP, DH>(p, smem, tmem, warp & 3, wg == 1 ? 0 : 1, abort_flag);
     } else {
         setmaxnreg_dec<Reg2<D>::OUT>();
         bwd2_out_role<D, BF16, SPLIT, DH>(p, smem, tmem, warp & 3, abort_flag);
