@@ -30,6 +30,7 @@
 //                                            16 bits in TMEM; dS^T also to SMEM)
 //        dV += P^T dO_m, dK += dS^T Q_m     (A operand from TMEM)
 //        dQ_m^T = K^T dS^T                  (into the step's dP^T columns)
+//      (D = 64: dQ_m^T first, and dK takes dS^T from SMEM, not TMEM)
 //      dQ_m is added to the fp32 accumulator (a TMA bulk reduce-add, or
 //      per-element atomics, or in key-tile order in deterministic mode); dK,
 //      dV are written once per unit.  D = 64 runs the D = 128 instantiation
