@@ -38,6 +38,13 @@
  * failed call and its error code.  Calls from several host threads at once
  * are safe: a causal call resets its work counter and launches under one lock,
  * and each kernel's shared-memory limit is set once per context.
+ *
+ * Every kernel is launched with programmatic stream serialization: it may
+ * begin (barrier set-up, tensor memory, descriptor prefetch) while the kernel
+ * before it in the stream is still running, and it waits for that kernel to
+ * complete, with its writes visible, before it reads or writes any tensor.
+ * Work of other code in the stream (kernels, copies, memsets, event waits)
+ * orders with these calls exactly as with ordinary launches.
  */
 #ifndef FA_H_
 #define FA_H_
