@@ -81,6 +81,17 @@ L2_BYTES = 126 * 1024 * 1024
 ALL_WORKLOADS = {**WORKLOADS, **GENERAL_WORKLOADS}
 
 
+def e2e_chunks(B: int, H: int, n_chunks: int):
+    """Split of one end-to-end step into chunks that are contiguous ranges of
+    every tensor: whole batches when B > 1, else heads of the single batch.
+    Returns ("b" or "h", [(first, count), ...]) covering the axis in order
+    with counts differing by at most one."""
+    axis, total = ("b", B) if B > 1 else ("h", H)
+    n = max(1, min(n_chunks, total))
+    edges = [total * c // n for c in range(n + 1)]
+    return axis, [(edges[c], edges[c + 1] - edges[c]) for c in range(n)]
+
+
 def workload_runs(name: str):
     """The fa_fwd runs of one step: (Workload, ...)."""
     if name == "c5":
@@ -498,16 +509,13 @@ def run_bwd(args) -> int:
         # over three streams, as in the forward pass; dropout keeps one chunk
         # (its keep decisions are drawn per absolute head index)
         def chunk_plan(w):
-            if args.dropout > 0.0 or args.e2e_chunks <= 1:
+            # the tensors here are [B, H, S, D] views, so the head axis is 1 in
+            # either storage layout; a head range of a BSHD batch is not one
+            # block of memory, so BSHD with B = 1 keeps one chunk
+            if args.dropout > 0.0 or (w.B == 1 and w.layout != "bhsd"):
                 return 0, [(0, w.B)]
-            if w.B > 1:
-                n, ax, total = min(args.e2e_chunks, w.B), 0, w.B
-            elif w.layout == "bhsd":
-                n, ax, total = min(args.e2e_chunks, w.H), 1, w.H
-            else:
-                return 0, [(0, w.B)]
-            edges = [total * c // n for c in range(n + 1)]
-            return ax, [(edges[c], edges[c + 1] - edges[c]) for c in range(n)]
+            axis, rng = e2e_chunks(w.B, w.H, args.e2e_chunks)
+            return (0 if axis == "b" else 1), rng
 
         plans = [chunk_plan(w) for w in runs]
         up_s, dn_s = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
@@ -1039,12 +1047,11 @@ def main(argv=None) -> int:
         n_chunks = max(1, args.e2e_chunks) if plain else 1
 
         def chunk_plan(w):
-            if w.B > 1:
-                n, ax_s, ax_l, total = min(n_chunks, w.B), 0, 0, w.B
-            else:
-                n, ax_s, ax_l, total = min(n_chunks, w.H), (1 if w.layout == "bhsd" else 2), 1, w.H
-            edges = [total * c // n for c in range(n + 1)]
-            return ax_s, ax_l, [(edges[c], edges[c + 1] - edges[c]) for c in range(n)]
+            # storage tensors: the head axis is 1 in BHSD, 2 in BSHD; LSE is [B, H, S]
+            axis, rng = e2e_chunks(w.B, w.H, n_chunks)
+            if axis == "b":
+                return 0, 0, rng
+            return (1 if w.layout == "bhsd" else 2), 1, rng
 
         plans = [chunk_plan(w) for w in runs]
         n_steps_chunk = max(len(p[2]) for p in plans)

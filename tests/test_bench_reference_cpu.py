@@ -56,3 +56,22 @@ def test_peak_follows_the_sampled_clocks(monkeypatch, tmp_path):
     monkeypatch.setattr(bench, "PEAKS_PATH", str(path))
     assert bench.peak_tflops(full)[:1] == (1637.9,)
     assert bench.peak_tflops(capped)[0] == 1420.0 and bench.peak_tflops(capped)[2] == 1637.9
+
+
+@pytest.mark.parametrize("B,H,n", [(1, 32, 8), (32, 16, 8), (2, 10, 8), (1, 3, 8), (4, 40, 1), (1, 1, 16), (3, 7, 2)])
+def test_e2e_chunks_cover_the_axis(B, H, n):
+    """The end-to-end step's chunks: whole batches when B > 1, else heads;
+    contiguous, in order, covering the axis once, sizes within one."""
+    sys.path.insert(0, ROOT)
+    import bench
+    axis, rng = bench.e2e_chunks(B, H, n)
+    total = B if B > 1 else H
+    assert axis == ("b" if B > 1 else "h")
+    assert len(rng) == max(1, min(n, total))
+    pos = 0
+    for first, count in rng:
+        assert first == pos and count >= 1
+        pos += count
+    assert pos == total
+    sizes = [c for _, c in rng]
+    assert max(sizes) - min(sizes) <= 1
