@@ -594,6 +594,22 @@ __global__ void __launch_bounds__(THREADS, 1) fa_fwd_kernel_short(const __grid_c
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&p.tmap_q)) : "memory");
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&p.tmap_k)) : "memory");
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&p.tmap_v)) : "memory");
+        // the first tile's Q and its head's K and V into L2 while the previous
+        // kernel in the stream may still run: a prefetch only warms L2, the
+        // point of coherence, so the loads after the dependency wait still see
+        // that kernel's writes
+        int t0, n;
+        tile_range(p, t0, n);
+        if (n > 0) {
+            TilePos pos;
+            pos.init(p, t0);
+#pragma unroll
+            for (int c = 0; c < L::CHUNKS; ++c) {
+                l2_prefetch_4d(&p.tmap_q, c * 64, pos.mt * BM, pos.uh, pos.ub);
+                l2_prefetch_4d(&p.tmap_k, c * 64, 0, pos.uh, pos.ub);
+                l2_prefetch_4d(&p.tmap_v, c * 64, 0, pos.uh, pos.ub);
+            }
+        }
     }
     if (warp == W_STORE && lane == 0)
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&p.tmap_o)) : "memory");

@@ -233,6 +233,17 @@ __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
 // Shared-memory matrix descriptor for a 128-byte-swizzled operand (sm_100 format:
 // start>>4 in [0,14), leading byte offset>>4 in [16,30), stride byte offset>>4
 // in [32,46), version 1 at bit 46, layout type 2 (128-byte swizzle) in [61,64)).
+// Prefetch of one box of a 4-D tensor map into L2 (no shared memory, no
+// barrier).  Used before a kernel's grid dependency wait: it only warms L2,
+// the point of coherence, so later loads still see the previous kernel's
+// writes.
+__device__ __forceinline__ void l2_prefetch_4d(const CUtensorMap* map, int c0, int c1, int c2, int c3) {
+    asm volatile("cp.async.bulk.prefetch.tensor.4d.L2.global.tile [%0, {%1, %2, %3, %4}];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+                 : "memory");
+}
+
 __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
     uint64_t d = 0;
     d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
