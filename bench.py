@@ -35,10 +35,11 @@ attention dropout (a fresh offset per step).
 
 The end-to-end figure ("e2e") times steps through the same public calls with
 pinned host buffers: each step uploads its inputs and downloads O and LSE.
-The forward pass splits each step into chunks of whole batches (or heads of
-a single batch) and pipelines them over three streams, so that the copies
-in both directions overlap the kernels; the downloaded results are checked
-bit for bit against one launch over all heads.
+Each step is split into chunks of whole batches (or heads of a single
+batch) pipelined over three streams, so that the copies in both directions
+overlap the kernels, and consecutive steps overlap on two sets of device
+buffers; the downloaded forward results are checked bit for bit against one
+launch over all heads.
 
 ``--impl reference`` times the fp64 CPU oracle on bounded samples of the
 same workload and pass (rank 0 only) and prints the same JSON line with
@@ -506,8 +507,9 @@ def run_bwd(args) -> int:
         d2h = sum(hb[n].numel() * hb[n].element_size() for hb in host for n in names_out)
 
         # chunks of whole batches (or heads of a single BHSD batch) pipelined
-        # over three streams, as in the forward pass; dropout keeps one chunk
-        # (its keep decisions are drawn per absolute head index)
+        # over three streams, consecutive steps on two sets of device buffers,
+        # as in the forward pass; dropout keeps one chunk (its keep decisions
+        # are drawn per absolute head index) and no step overlap
         def chunk_plan(w):
             # the tensors here are [B, H, S, D] views, so the head axis is 1 in
             # either storage layout; a head range of a BSHD batch is not one
@@ -522,9 +524,18 @@ def run_bwd(args) -> int:
         ev_up = [[torch.cuda.Event() for _ in p[1]] for p in plans]
         ev_k = [[torch.cuda.Event() for _ in p[1]] for p in plans]
         n_chunk_max = max(len(p[1]) for p in plans)
+        overlap_steps = n_chunk_max > 1
+        # the second set: the step's inputs and gradients (the workspace is
+        # used by one launch at a time on the timing stream, so one suffices)
+        buf_sets = [bufs]
+        if overlap_steps:
+            buf_sets.append([dict(b, **{nm: torch.empty_like(b[nm]) for nm in names_in + names_out}) for b in bufs])
+        ev_kend = [torch.cuda.Event(), torch.cuda.Event()]
+        ev_dnend = [torch.cuda.Event(), torch.cuda.Event()]
+        step_count = [0]
 
-        def launch_chunk(i, ax, a, n):
-            w, b = runs[i], bufs[i]
+        def launch_chunk(i, ax, a, n, ps):
+            w, b = runs[i], buf_sets[ps][i]
             if len(plans[i][1]) == 1:
                 launch(i)
                 return
@@ -539,12 +550,19 @@ def run_bwd(args) -> int:
                 raise fa.FaError(st, "fa_bwd_ex")
 
         def e2e_step():
-            start_ev = torch.cuda.Event()
-            start_ev.record(stream)
-            up_s.wait_event(start_ev)
-            dn_s.wait_event(start_ev)
+            ps = step_count[0] % 2 if overlap_steps else 0
+            step_count[0] += 1
+            if not overlap_steps:
+                start_ev = torch.cuda.Event()
+                start_ev.record(stream)
+                up_s.wait_event(start_ev)
+                dn_s.wait_event(start_ev)
+            else:
+                up_s.wait_event(ev_kend[ps])      # this set's inputs read by its previous step
+                stream.wait_event(ev_dnend[ps])   # this set's gradients downloaded by its previous step
             for c in range(n_chunk_max):
-                for i, (hb, b) in enumerate(zip(host, bufs)):
+                for i, hb in enumerate(host):
+                    b = buf_sets[ps][i]
                     ax, rng = plans[i]
                     if c >= len(rng):
                         continue
@@ -554,30 +572,42 @@ def run_bwd(args) -> int:
                             b[nm].narrow(ax, a, n).copy_(hb[nm].narrow(ax, a, n), non_blocking=True)
                     ev_up[i][c].record(up_s)
                     stream.wait_event(ev_up[i][c])
-                    launch_chunk(i, ax, a, n)
+                    launch_chunk(i, ax, a, n, ps)
                     ev_k[i][c].record(stream)
                     dn_s.wait_event(ev_k[i][c])
                     with torch.cuda.stream(dn_s):
                         for nm in names_out:
                             hb[nm].narrow(ax, a, n).copy_(b[nm].narrow(ax, a, n), non_blocking=True)
-            done_ev = torch.cuda.Event()
-            done_ev.record(dn_s)
-            stream.wait_event(done_ev)
+            ev_kend[ps].record(stream)
+            ev_dnend[ps].record(dn_s)
+            if not overlap_steps:
+                stream.wait_event(ev_dnend[ps])
+
+        def join():
+            for s_ in (up_s, dn_s):
+                ev = torch.cuda.Event()
+                ev.record(s_)
+                stream.wait_event(ev)
 
         for _ in range(2):
             e2e_step()
+        join()
         torch.cuda.synchronize(dev)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
+        up_s.wait_event(e0)
+        dn_s.wait_event(e0)
         for _ in range(args.e2e_steps):
             e2e_step()
+        join()
         e1.record(stream)
         torch.cuda.synchronize(dev)
         e2e = {"value": job_throughput(step_flops, args.e2e_steps, world,
                                        max_over_ranks(e0.elapsed_time(e1), device=dev)),
                "unit": UNIT, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-               "overlap": (f"{n_chunk_max} chunks per step; uploads, launches and downloads on three streams"
-                           if n_chunk_max > 1 else "none")}
+               "overlap": (f"{n_chunk_max} chunks per step; uploads, launches and downloads on three streams; "
+                           "consecutive steps overlap on two sets of device buffers"
+                           if overlap_steps else "none")}
         # the chunked gradients against one launch over all heads (fp32 sums
         # of dQ, and of split dK/dV, may add in another order)
         for i in range(len(runs)):
@@ -1040,9 +1070,11 @@ def main(argv=None) -> int:
         # of every storage tensor) on one stream, runs each chunk's launches on
         # the timing stream once its upload has landed, and downloads each
         # chunk's O and LSE on a third stream once its launches are done, so
-        # the copies in both directions overlap the kernels.  A step starts
-        # after the previous step's last download: nothing is shared across
-        # steps.
+        # the copies in both directions overlap the kernels.  Consecutive steps
+        # overlap too, as requests do in a serving loop: they alternate between
+        # two sets of device buffers, and a step's upload into a set waits only
+        # for the launches that read that set two steps before, its launches
+        # only for that step's downloads of the set's outputs.
         plain = args.dropout == 0.0 and not tril and not args.block_n and not args.q_tiles
         n_chunks = max(1, args.e2e_chunks) if plain else 1
 
@@ -1058,15 +1090,28 @@ def main(argv=None) -> int:
         up_s, dn_s = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
         ev_up = [[torch.cuda.Event() for _ in p[2]] for p in plans]
         ev_k = [[torch.cuda.Event() for _ in p[2]] for p in plans]
+        # the second set of device buffers (inputs shared between runs stay shared)
+        overlap_steps = n_steps_chunk > 1
+        sets_in, sets_out = [[t[0] for t in dev_in]], [list(dev_out)]
+        if overlap_steps:
+            second_in = []
+            for i in range(len(runs)):
+                shared = i > 0 and host_in[i] is host_in[0]
+                second_in.append(second_in[0] if shared else tuple(torch.empty_like(t) for t in dev_in[i][0]))
+            sets_in.append(second_in)
+            sets_out.append([(torch.empty_like(o), torch.empty_like(l)) for (o, l) in dev_out])
+        ev_kend = [torch.cuda.Event(), torch.cuda.Event()]  # a set's last launch of its latest step
+        ev_dnend = [torch.cuda.Event(), torch.cuda.Event()]  # a set's last download of its latest step
+        step_count = [0]
 
-        def launch_chunk(i, ax_s, ax_l, a, n):
+        def launch_chunk(i, ax_s, ax_l, a, n, ps):
             w = runs[i]
             if len(plans[i][2]) == 1:
                 launch(i)
                 return
-            q, k, v = (view(w, t.narrow(ax_s, a, n)) for t in dev_in[i][0])
-            o = view(w, dev_out[i][0].narrow(ax_s, a, n))
-            lse = dev_out[i][1].narrow(ax_l, a, n)
+            q, k, v = (view(w, t.narrow(ax_s, a, n)) for t in sets_in[ps][i])
+            o = view(w, sets_out[ps][i][0].narrow(ax_s, a, n))
+            lse = sets_out[ps][i][1].narrow(ax_l, a, n)
             dt = fa.FA_BF16 if w.dtype == "bf16" else fa.FA_FP16
             st = fa.fa_fwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), q.shape[0],
                               q.shape[1], w.S, w.Skv, w.D, q.stride()[:3], k.stride()[:3], v.stride()[:3],
@@ -1075,10 +1120,16 @@ def main(argv=None) -> int:
                 raise fa.FaError(st)
 
         def e2e_step():
-            start = torch.cuda.Event()
-            start.record(stream)
-            up_s.wait_event(start)
-            dn_s.wait_event(start)
+            ps = step_count[0] % 2 if overlap_steps else 0
+            step_count[0] += 1
+            if not overlap_steps:
+                start = torch.cuda.Event()
+                start.record(stream)
+                up_s.wait_event(start)
+                dn_s.wait_event(start)
+            else:
+                up_s.wait_event(ev_kend[ps])      # this set's inputs read by its previous step
+                stream.wait_event(ev_dnend[ps])   # this set's outputs downloaded by its previous step
             for c in range(n_steps_chunk):
                 for i in range(len(runs)):
                     ax_s, ax_l, rng = plans[i]
@@ -1088,35 +1139,50 @@ def main(argv=None) -> int:
                     owner = 0 if (i > 0 and host_in[i] is host_in[0]) else i
                     if owner == i:
                         with torch.cuda.stream(up_s):
-                            for hsrc, dsrc in zip(host_in[i], dev_in[i][0]):
+                            for hsrc, dsrc in zip(host_in[i], sets_in[ps][i]):
                                 dsrc.narrow(ax_s, a, n).copy_(hsrc.narrow(ax_s, a, n), non_blocking=True)
                         ev_up[i][c].record(up_s)
                     stream.wait_event(ev_up[owner][c])
-                    launch_chunk(i, ax_s, ax_l, a, n)
+                    launch_chunk(i, ax_s, ax_l, a, n, ps)
                     ev_k[i][c].record(stream)
                     dn_s.wait_event(ev_k[i][c])
                     with torch.cuda.stream(dn_s):
-                        host_out[i][0].narrow(ax_s, a, n).copy_(dev_out[i][0].narrow(ax_s, a, n), non_blocking=True)
-                        host_out[i][1].narrow(ax_l, a, n).copy_(dev_out[i][1].narrow(ax_l, a, n), non_blocking=True)
-            done = torch.cuda.Event()
-            done.record(dn_s)
-            stream.wait_event(done)
+                        o_src, l_src = sets_out[ps][i]
+                        host_out[i][0].narrow(ax_s, a, n).copy_(o_src.narrow(ax_s, a, n), non_blocking=True)
+                        host_out[i][1].narrow(ax_l, a, n).copy_(l_src.narrow(ax_l, a, n), non_blocking=True)
+            ev_kend[ps].record(stream)
+            ev_dnend[ps].record(dn_s)
+            if not overlap_steps:
+                stream.wait_event(ev_dnend[ps])
+
+        def join():
+            # the timing stream waits for everything the steps put on the copy streams
+            for s_ in (up_s, dn_s):
+                ev = torch.cuda.Event()
+                ev.record(s_)
+                stream.wait_event(ev)
 
         for _ in range(2):
             e2e_step()
+        join()
         torch.cuda.synchronize(dev)
         barrier()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
+        # the copy streams start no earlier than the timed region
+        up_s.wait_event(e0)
+        dn_s.wait_event(e0)
         for _ in range(args.e2e_steps):
             e2e_step()
+        join()
         e1.record(stream)
         torch.cuda.synchronize(dev)
         barrier()
         e2e_val = job_throughput(step_flops, args.e2e_steps, world, max_over_ranks(e0.elapsed_time(e1), device=dev))
         e2e = {"value": e2e_val, "unit": UNIT, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-               "overlap": (f"{n_steps_chunk} chunks per step; uploads, launches and downloads on three streams"
-                           if n_steps_chunk > 1 else "none")}
+               "overlap": (f"{n_steps_chunk} chunks per step; uploads, launches and downloads on three streams; "
+                           "consecutive steps overlap on two sets of device buffers"
+                           if overlap_steps else "none")}
         # the chunked launches compute each head exactly as one launch over all
         # heads does: the downloaded results equal a whole launch's bit for bit
         for i in range(len(runs)):
