@@ -819,7 +819,7 @@ def main(argv=None) -> int:
     ap.add_argument("--impl", choices=["fa", "reference"], default="fa")
     ap.add_argument("--workload", default="c5", choices=["c5"] + list(ALL_WORKLOADS))
     ap.add_argument("--e2e-steps", type=int, default=10)
-    ap.add_argument("--e2e-chunks", type=int, default=8,
+    ap.add_argument("--e2e-chunks", type=int, default=4,
                     help="chunks (batches, or heads of a single batch) per end-to-end step, pipelined over "
                          "three streams (upload, launches, download)")
     ap.add_argument("--no-e2e", action="store_true")
