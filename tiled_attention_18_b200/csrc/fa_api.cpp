@@ -392,9 +392,17 @@ int forward(const void* q, const void* k, const void* v, void* o, float* lse, in
             rc = sched_counter(stream, &ctr);
             if (rc != FA_OK) return rc;
         }
-        // the counter keeps the previous call's value: clear it on this stream
-        const cudaError_t e = cudaMemsetAsync(ctr, 0, sizeof(unsigned int), stream);
-        if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(scheduler counter)");
+        if (scratch == Scratch::Static) {
+            // the shared no-allocation counter keeps the previous call's value:
+            // clear it on this stream
+            const cudaError_t e = cudaMemsetAsync(ctr, 0, sizeof(unsigned int), stream);
+            if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(scheduler counter)");
+        } else {
+            // a stream's own slot starts zeroed (static memory) and every launch
+            // leaves it zeroed: no memset, so the launch can overlap the tail of
+            // the kernel before it in the stream
+            a.sched_reset = 1;
+        }
         a.sched = ctr;
     }
     if (short_keys) {

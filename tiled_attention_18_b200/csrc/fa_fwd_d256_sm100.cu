@@ -98,6 +98,7 @@ struct Params {
     int BH, H, Sq, Sk, n_mtiles, n_units, nkv, causal, causal_off;
     float scale_log2;
     unsigned int* sched;
+    int sched_reset;  // the last CTA to finish zeroes sched[0] and sched[1] for the next launch
     const uint8_t* mask;         // explicit boolean mask (MASK kernels): nonzero = attend
     long long m_sb, m_sh, m_ss;  // its element strides over b, h and the query row
     uint32_t drop_p8x4, seed_lo, seed_hi, drop_offset;  // dropout (DROP kernels)
@@ -606,6 +607,15 @@ __global__ void __launch_bounds__(THREADS, 1) fa_fwd_kernel_d256(const __grid_co
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS_D256)
                      : "memory");
     }
+    if (p.sched_reset && threadIdx.x == 0) {
+        // as in the D = 64/128 kernel: the last CTA clears the counter and the count
+        __threadfence();
+        if (atomicAdd(p.sched + 1, 1u) == gridDim.x - 1u) {
+            __threadfence();
+            atomicExch(p.sched, 0u);
+            atomicExch(p.sched + 1, 0u);
+        }
+    }
 }
 
 template <bool BF16, bool MASK, bool DROP>
@@ -633,6 +643,7 @@ cudaError_t launch_impl(const LaunchArgs& a, cudaStream_t stream) {
     p.causal_off = a.Sk - a.Sq;
     p.scale_log2 = a.scale_log2;
     p.sched = a.sched;
+    p.sched_reset = a.sched_reset;
     p.mask = a.mask;
     p.m_sb = a.mask_stride[0];
     p.m_sh = a.mask_stride[1];

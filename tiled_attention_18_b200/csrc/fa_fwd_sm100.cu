@@ -197,6 +197,9 @@ struct KParams {
     long long m_sb, m_sh, m_ss;  // its element strides over b, h and the query row (keys contiguous)
     float scale_log2;
     unsigned int* sched;  // zeroed unit counter (claim order), or null for the static order
+    // sched[1] counts the CTAs that have finished; the last one zeroes both
+    // words for the next launch on the same stream (no memset between launches)
+    int sched_reset;
     // dropout (DROP kernels): threshold in every byte, generator key, counter word 3, 1 / (1 - p)
     uint32_t drop_p8x4, seed_lo, seed_hi, drop_offset;
     float keep_scale;
@@ -918,6 +921,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) fa_fwd_kernel(const __grid_con
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(TMEM_COLS)
                      : "memory");
     }
+    if (p.sched_reset && threadIdx.x == 0) {
+        // this CTA's claims are done (its producer has left); the last CTA to
+        // get here clears the counter and the count for the stream's next launch
+        __threadfence();
+        if (atomicAdd(p.sched + 1, 1u) == gridDim.x - 1u) {
+            __threadfence();
+            atomicExch(p.sched, 0u);
+            atomicExch(p.sched + 1, 0u);
+        }
+    }
 }
 
 // Diagnostic kernel for the failure path: thread 0 waits on an mbarrier that
@@ -987,6 +1000,7 @@ cudaError_t launch_impl(const LaunchArgs& a, cudaStream_t stream) {
     p.m_ss = a.mask_stride[2];
     p.scale_log2 = a.scale_log2;
     p.sched = a.sched;
+    p.sched_reset = a.sched_reset;
     p.drop_p8x4 = a.drop.p8 * 0x01010101u;
     p.seed_lo = a.drop.seed_lo;
     p.seed_hi = a.drop.seed_hi;

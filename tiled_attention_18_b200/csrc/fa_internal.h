@@ -63,6 +63,7 @@ struct LaunchArgs {
     float scale_log2;       // scale * log2(e)
     int grid;               // persistent CTAs
     unsigned int* sched;    // zeroed device counter for claimed-unit scheduling, or null
+    int sched_reset;        // the launch zeroes sched[0] and sched[1] again as its last CTA ends
     int block_n;            // keys per key tile: 128 (default) or 64 (D = 64/128 kernel)
     int q_tiles;            // 128-row query tiles per work unit: 2 (default) or 1
 };
