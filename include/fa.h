@@ -36,8 +36,11 @@
  * the failure of this call's own CUDA calls and launches, never an error that
  * other code left pending in the calling thread; fa_last_cuda_error names the
  * failed call and its error code.  Calls from several host threads at once
- * are safe: a causal call resets its work counter and launches under one lock,
- * and each kernel's shared-memory limit is set once per context.
+ * are safe: a causal call takes its stream's work counter and launches under
+ * one lock (the counter is cleared by the last CTA of each launch, so no
+ * memset precedes a causal launch except in fa_fwd_noalloc, whose counter all
+ * streams share), and each kernel's shared-memory limit is set once per
+ * context.
  *
  * Every kernel is launched with programmatic stream serialization: it may
  * begin (barrier set-up, tensor memory, descriptor prefetch) while the kernel
