@@ -112,11 +112,12 @@ typedef enum {
  * stream  : the CUDA stream to launch on (0 = legacy default stream).
  *
  * Ownership: the caller owns every buffer and the stream; fa_fwd allocates
- * nothing.  With causal = 1 the library's work scheduler uses a 4-byte
- * counter: one slot per (context, stream) of a fixed pool of 2048 slots in
- * libfa.so's own static device memory (64 KiB, part of the loaded module),
- * handed out by the stream's first causal call; each causal call zeroes its
- * counter with cudaMemsetAsync on `stream`.  More than 2048 distinct streams
+ * nothing.  With causal = 1 the library's work scheduler uses a counter
+ * (claimed units and finished CTAs): one slot per (context, stream) of a
+ * fixed pool of 2048 slots in libfa.so's own static device memory (64 KiB,
+ * part of the loaded module), handed out by the stream's first causal call;
+ * the slot starts zeroed and the last CTA of every causal launch zeroes it
+ * again, so no memset precedes the launch.  More than 2048 distinct streams
  * of one context launching causal forwards gives FA_ERR_LIMIT.  The first
  * call in a context looks up the pool's device address (a host-side query,
  * no device work).  Synchronicity: asynchronous on `stream`; fa_fwd never
