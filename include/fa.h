@@ -215,7 +215,8 @@ FA_API int fa_fwd_mask(const void* q, const void* k, const void* v, void* o, flo
  * fa_bwd_workspace_size -- bytes of device workspace fa_bwd needs for B*H
  * heads of Sq query rows of dimension D: an fp32 dQ accumulator
  * [B*H][Sq][D], two fp32 row-statistic arrays [B*H][Sq rounded up to 128],
- * the deterministic mode's turn counters [B*H][Sq/64 rounded up][4] int, a
+ * the deterministic mode's turn counters [B*H][Sq/64 rounded up][1, or 2 at
+ * D = 256][4] int, a
  * 256-byte scheduler counter and two fp32 arrays [B*H][128][D] for the
  * partial sums of dK and dV (used when Sk <= 128 and the (head, key tile)
  * units are fewer than the SMs: the query range is then split across units),
@@ -267,8 +268,12 @@ FA_API long long fa_bwd_workspace_size(int B, int H, int Sq, int D);
  * Numerics: S, P, dP, dS, Delta and all accumulation in fp32; P and dS are
  * rounded to dtype before their products; the outputs are rounded to nearest
  * even.
- * Three kernels run on `stream` (row statistics, the fused backward, dQ
- * conversion); nothing is allocated; asynchronous.  Errors as fa_fwd.
+ * Kernels alone run on `stream`, with no memset or copy between them: row
+ * statistics (which also clears the workspace parts the call needs zeroed:
+ * the dQ accumulator, the turn counters, the dK/dV partial sums), the fused
+ * backward, then the dQ conversion, or with a split query range the dK/dV
+ * conversion (plus the dQ conversion at D = 256); Sq = 0 runs two memsets of
+ * dK and dV instead.  Nothing is allocated; asynchronous.  Errors as fa_fwd.
  */
 FA_API int fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
                   void* dq, void* dk, void* dv, void* workspace, long long workspace_bytes, int B, int H, int Sq,

@@ -587,9 +587,7 @@ int backward(const void* q, const void* k, const void* v, const void* o, const v
     if (drop) a.drop = *drop;
     a.dq_flags = nullptr;
     if (deterministic) {
-        a.dq_flags = reinterpret_cast<int*>(w + ws.flags);
-        const cudaError_t e = cudaMemsetAsync(a.dq_flags, 0, (size_t)ws.flags_bytes, stream);
-        if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(deterministic turn counters)");
+        a.dq_flags = reinterpret_cast<int*>(w + ws.flags);  // cleared by the backward's first kernel
     }
     a.B = B;
     a.H = H;

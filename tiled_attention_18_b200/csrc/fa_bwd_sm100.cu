@@ -1043,13 +1043,17 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const uint16_t* __restric
                                                        const float* __restrict__ lse, float* __restrict__ lse2,
                                                        float* __restrict__ delta, float* __restrict__ dq_acc, int Sq,
                                                        int Sq_pad, unsigned int* sched, int H, Strides3 os,
-                                                       Strides3 dos, float4* __restrict__ kv_zero, size_t kv_n4) {
+                                                       Strides3 dos, float4* __restrict__ kv_zero, size_t kv_n4,
+                                                       int* __restrict__ flags_zero, size_t n_flags) {
     grid_dependency_sync();
-    if (kv_zero) {
-        // the split mode's fp32 dK/dV partial sums, spread over all blocks
-        const size_t blk = (size_t)blockIdx.y * gridDim.x + blockIdx.x, nthr = (size_t)gridDim.x * gridDim.y * 256;
+    // buffers cleared here rather than by a memset between the kernels, spread
+    // over all blocks: the split mode's fp32 dK/dV partial sums, and the
+    // deterministic mode's turn counters
+    const size_t blk = (size_t)blockIdx.y * gridDim.x + blockIdx.x, nthr = (size_t)gridDim.x * gridDim.y * 256;
+    if (kv_zero)
         for (size_t i = blk * 256 + threadIdx.x; i < kv_n4; i += nthr) kv_zero[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-    }
+    if (flags_zero)
+        for (size_t i = blk * 256 + threadIdx.x; i < n_flags; i += nthr) flags_zero[i] = 0;
     using PS = PrepShape<D>;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int sub = lane / PS::LANES, part = lane - sub * PS::LANES;  // row within the warp, 8-element part
@@ -1159,14 +1163,16 @@ cudaError_t launch_bwd_impl(const BwdLaunchArgs& a, cudaStream_t stream) {
     {
         dim3 grid((unsigned)((Sq_pad + PrepShape<D>::ROWS_PER_BLOCK - 1) / PrepShape<D>::ROWS_PER_BLOCK),
                   (unsigned)BH, 1);
-        // split: the dK/dV partial sums (contiguous) cleared too
+        // split: the dK/dV partial sums (contiguous) cleared too; deterministic:
+        // the turn counters, [BH][64-row steps][passes over D][4 warps]
         cudaError_t e = launch_kernel(
             bwd_prep_kernel<D, BF16>, grid, dim3(256), 0, stream, static_cast<const uint16_t*>(a.o),
             static_cast<const uint16_t*>(a.dout), a.lse, a.lse2, a.delta, dq_direct ? nullptr : a.dq_acc, a.Sq, Sq_pad,
             a.sched, a.H, Strides3{{a.o_stride[0], a.o_stride[1], a.o_stride[2]}},
             Strides3{{a.do_stride[0], a.do_stride[1], a.do_stride[2]}},
             split ? reinterpret_cast<float4*>(a.dk_acc) : nullptr,
-            split ? (size_t)2 * BH * KV_ACC_ROWS * D / 4 : (size_t)0);
+            split ? (size_t)2 * BH * KV_ACC_ROWS * D / 4 : (size_t)0, a.dq_flags,
+            a.dq_flags ? (size_t)BH * (size_t)n_steps * Bwd2Smem<DW>::HALVES * 4 : (size_t)0);
         if (e != cudaSuccess) return e;
     }
     {
